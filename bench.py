@@ -1,0 +1,414 @@
+#!/usr/bin/env python
+"""Benchmark of the routed MoE expert-FFN layer forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step is one moe_forward (router -> top-k -> histogram/permutation ->
+activation quantisation -> gate|up projection + SwiGLU -> down projection ->
+combine) over one batch of the prefill workload: T=4096 tokens, hidden 2048,
+128 experts, top-8, intermediate 768, NVFP4 weights and activations (W4A4,
+static activation scales), Zipf(1.1)-skewed routing.  Inputs are seeded and
+synthetic and resident in HBM; L2 is flushed (a 256 MiB write) between timed
+steps, outside the timed events.  Time is taken with CUDA events on the
+launching stream, max over ranks.  With N > 1 every rank runs an independent
+replica (the layer needs no collective: tokens are independent given the
+weights), so scaling is weak and `value` is the tokens of all ranks divided
+by the slowest rank's time.
+
+Rank 0 prints one JSON line.  Besides the contract keys it carries:
+  stages       per-stage device time (ms) from the library's stage events
+  roofline     the dominant stage against the measured peak
+  e2e          the same metric with the input copied from pinned host memory
+               and the output copied back inside the timed region
+  decode       the decode workload's expert-weight streaming rate (GB/s)
+  cpu_baseline the CPU oracle on a bounded token sample (rank 0, N = 1)
+  clocks       nvidia-smi samples taken during the timed region
+`--impl reference` times the CPU oracle instead (the only other arm).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer tokens/s at T=4096 prefill; decode weight GB/s (% of HBM peak)"
+FP4_PER_BF16 = 4.0      # nominal dense FP4 : BF16 tensor rate on B200 (9 : 2.25 PFLOP/s)
+FP8_PER_BF16 = 2.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="prefill")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------ clocks --
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.2)
+        self.proc.terminate()
+        self.proc.wait()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        load = [s for s in sm if s > 0.5 * max(sm)] or sm
+        return {"sm_mhz": float(np.median(load)), "sm_max_mhz": float(max(smax)), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------- layers -----
+def build_layer(ops, synth, torch, w, static: bool):
+    """Weights drawn on the GPU (CUDA Philox), quantised and prepared by the library."""
+    fmt = ops.FMT_BY_NAME[w.fmt]
+    ws = ops.new_workspace(4096)
+    banks = []
+    chunks13, chunks2 = [], []
+    for e in range(w.E):
+        chunks13.append(synth.cuda_normal((1, 2 * w.I, w.H), w.w_std, synth.TID_W13 + e))
+        chunks2.append(synth.cuda_normal((1, w.H, w.I), w.w_std, synth.TID_W2 + e))
+    w13 = torch.cat(chunks13)
+    w2 = torch.cat(chunks2)
+    del chunks13, chunks2
+    bank = ops.quantize_bank(fmt, w13, w2, ws)
+    del w13, w2
+    if static and fmt != ops.FMT_MXFP4:
+        a13, a2 = synth.static_act_scales()
+        bank.a13_gs = torch.tensor([a13], dtype=torch.float32, device="cuda")
+        bank.a2_gs = torch.tensor([a2], dtype=torch.float32, device="cuda")
+    prepared = ops.moe_prepare_weights(bank)
+    torch.cuda.synchronize()
+    x = synth.cuda_normal((w.T, w.H), 1.0, synth.TID_X, dtype=torch.bfloat16)
+    wr = synth.cuda_normal((w.E, w.H), w.wr_std, synth.TID_WR, dtype=torch.bfloat16)
+    bias = synth.cuda_router_bias(w)
+    return prepared, x, wr, bias
+
+
+def algorithmic(w, bank_fmt: str, offsets: np.ndarray):
+    """FLOPs and bytes of one forward by definition (routed slots only;
+    weights of experts with at least one slot; x, out, Wr)."""
+    T, H, E, k, I = w.T, w.H, w.E, w.k, w.I
+    S = T * k
+    flops_up = 2.0 * S * H * 2 * I
+    flops_down = 2.0 * S * I * H
+    counts = np.diff(offsets)
+    active = int((counts > 0).sum())
+    if bank_fmt == "fp8":
+        per13, per2 = 2 * I * H, H * I
+    else:
+        bs = 16 if bank_fmt == "nvfp4" else 32
+        per13 = 2 * I * H // 2 + 2 * I * H // bs
+        per2 = H * I // 2 + H * I // bs
+    wbytes_up = active * per13
+    wbytes_down = active * per2
+    io = T * H * 2 * 2 + E * H * 2
+    return dict(flops_up=flops_up, flops_down=flops_down, wbytes_up=wbytes_up, wbytes_down=wbytes_down,
+                io_bytes=io, active_experts=active, max_over_mean=float(counts.max() / max(counts.mean(), 1e-9)),
+                zero_experts=int((counts == 0).sum()))
+
+
+def time_forward(ops, torch, layer, w, act, steps, warmup, flush, stage=True, host_io=False):
+    prepared, x, wr, bias = layer
+    dev = x.device
+    ws = ops.new_workspace(ops.workspace_size(w.T, w.k, prepared, None, act))
+    out = torch.empty_like(x)
+    if host_io:
+        x_host = x.cpu().pin_memory()
+        out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    n_ev = 2 * len(ops.STAGES)
+    stream = torch.cuda.current_stream()
+
+    def one(i, evs=None, rec=None):
+        if evs is not None:
+            ops.moe_set_stage_events(evs)
+        if rec is not None:
+            rec[0].record(stream)
+        if host_io:
+            x.copy_(x_host, non_blocking=True)
+        ops.moe_forward(x, wr, bias, w.k, prepared, None, act, ws, out=out)
+        if host_io:
+            out_host.copy_(out, non_blocking=True)
+        if rec is not None:
+            rec[1].record(stream)
+        if evs is not None:
+            ops.moe_set_stage_events(None)
+
+    for i in range(warmup):
+        one(i)
+    torch.cuda.synchronize()
+    if ops.moe_get_device_status(ws) != 0:
+        raise RuntimeError("device status reported a fault during warm-up")
+    stage_evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(steps)] if stage else None
+    step_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    launches0 = ops.moe_kernel_launch_count()
+    torch.cuda.synchronize()
+    for i in range(steps):
+        flush.zero_()
+        one(i, stage_evs[i] if stage else None, step_evs[i])
+    torch.cuda.synchronize()
+    launches = ops.moe_kernel_launch_count() - launches0
+    per_step = [a.elapsed_time(b) for a, b in step_evs]
+    stages = {}
+    if stage:
+        for si, name in enumerate(ops.STAGES):
+            vals = []
+            for evs in stage_evs:
+                try:
+                    vals.append(evs[2 * si].elapsed_time(evs[2 * si + 1]))
+                except RuntimeError:
+                    pass
+            if vals:
+                stages[name] = float(np.mean(vals))
+    # routing histogram of the last step (for the algorithmic byte count)
+    idx, _ = ops.moe_route(x, wr, bias, w.k, ops.new_workspace(ops.workspace_size(w.T, w.k, prepared, None, act)))
+    off, _, _ = ops.moe_permute(idx, w.E, ops.new_workspace(1 << 24))
+    return dict(ms=per_step, stages=stages, launches=launches, offsets=off.cpu().numpy(),
+                status=ops.moe_get_device_status(ws))
+
+
+# ------------------------------------------------------------ CPU oracle ----
+def cpu_oracle_sample(w, target_s: float, static: bool, max_tokens: int | None = None):
+    """The oracle as it stands, on a bounded token sample of the workload."""
+    import oracle
+    from quantized_expert_ffn_top_b200 import synth
+    fmt = {"nvfp4": 1, "mxfp4": 2, "fp8": 3}[w.fmt]
+    t0 = time.time()
+    W = oracle.quantize_expert_weights(fmt, synth.all_w13(w), synth.all_w2(w))
+    x = synth.x_bits(w)
+    wr = synth.router_bits(w)
+    b = synth.router_bias(w)
+    a13, a2 = synth.static_act_scales() if static else (0.0, 0.0)
+    setup_s = time.time() - t0
+    threads = oracle.default_threads()
+    n = 4
+    tok_s = None
+    used = 0
+    spent = 0.0
+    while True:
+        toks = np.arange(n, dtype=np.int32) * (w.T // max(n, 1))
+        t1 = time.time()
+        oracle.moe_forward(x, wr, b, w.k, W, act=1, a13_static=a13, a2_static=a2, tokens=toks, nthreads=threads)
+        dt = time.time() - t1
+        spent += dt
+        used = n
+        tok_s = n / dt
+        if dt * 2 > target_s or spent > target_s or (max_tokens and n >= max_tokens):
+            break
+        n = int(min(max(n * 2, n * target_s / max(dt, 1e-3) * 0.5), max_tokens or 1 << 30))
+    return {"value": tok_s, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{used} evenly spaced tokens of the {w.name} workload (T={w.T}), fp64 oracle, "
+                      f"{threads} OpenMP threads; weights drawn and quantised on the host in {setup_s:.0f} s"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from quantized_expert_ffn_top_b200 import synth
+    import oracle
+    w = synth.workload(args.workload)
+    fmt = {"nvfp4": 1, "mxfp4": 2, "fp8": 3}[w.fmt]
+    W = oracle.quantize_expert_weights(fmt, synth.all_w13(w), synth.all_w2(w))
+    x = synth.x_bits(w)
+    wr = synth.router_bits(w)
+    b = synth.router_bias(w)
+    a13, a2 = synth.static_act_scales()
+    threads = oracle.default_threads()
+    n = 8
+    rng = np.random.default_rng(0)
+
+    def step():
+        toks = rng.choice(w.T, size=n, replace=False).astype(np.int32)
+        oracle.moe_forward(x, wr, b, w.k, W, act=1, a13_static=a13, a2_static=a2, tokens=toks, nthreads=threads)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.time()
+    for _ in range(args.steps):
+        step()
+    dt = time.time() - t0
+    v = n * args.steps / dt
+    line = {"metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": workload_name(w), "sample_tokens_per_step": n},
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                             "sample": f"{n} random tokens per step of the {w.name} workload"},
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def workload_name(w) -> str:
+    s = (f"{w.name}: T={w.T} H={w.H} E={w.E} top-{w.k} I={w.I} {w.fmt.upper()} weights, "
+         f"{'W4A4' if w.fmt != 'fp8' else 'W8A8'} activations, {w.router} router")
+    if w.shared_I:
+        s += f", shared expert I={w.shared_I}"
+    return s
+
+
+# ------------------------------------------------------------------ main ----
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    import torch
+    import torch.distributed as dist
+    from quantized_expert_ffn_top_b200 import ops, synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    ops.lib()
+    pk, pk_kind = peaks()
+    w = synth.workload(args.workload)
+    act = ops.ACT_MATCH
+    layer = build_layer(ops, synth, torch, w, static=True)
+    l2 = torch.cuda.get_device_properties(local).L2_cache_size
+    flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device="cuda")
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    clock = ClockSampler(local)
+    barrier()
+    clock.start()
+    res = time_forward(ops, torch, layer, w, act, args.steps, args.warmup, flush)
+    barrier()
+    clocks = clock.stop()
+    ms = float(np.mean(res["ms"]))
+    total_s = float(np.sum(res["ms"])) / 1e3
+    if world > 1:
+        t = torch.tensor([total_s], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_s = float(t.item())
+    value = world * w.T * args.steps / total_s
+
+    # end to end: pinned host input -> device -> forward -> host output
+    barrier()
+    res_e2e = time_forward(ops, torch, layer, w, act, args.steps, 2, flush, stage=False, host_io=True)
+    e2e_s = float(np.sum(res_e2e["ms"])) / 1e3
+    if world > 1:
+        t = torch.tensor([e2e_s], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_s = float(t.item())
+    e2e = {"value": world * w.T * args.steps / e2e_s, "unit": "tokens/s",
+           "h2d_bytes_per_step": w.T * w.H * 2, "d2h_bytes_per_step": w.T * w.H * 2}
+
+    alg = algorithmic(w, w.fmt, res["offsets"])
+    stages = res["stages"]
+    # dominant stage and its roofline
+    dom = max(stages, key=stages.get) if stages else "ffn_up"
+    peak_tensor = pk["bf16_tflops"] * (FP4_PER_BF16 if w.fmt != "fp8" else FP8_PER_BF16)
+    if dom in ("ffn_up", "ffn_down"):
+        flops = alg["flops_up"] if dom == "ffn_up" else alg["flops_down"]
+        achieved = flops / (stages[dom] * 1e-3) / 1e12
+        roof = {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": peak_tensor, "unit": "TFLOP/s",
+                "frac": achieved / peak_tensor, "traffic": None,
+                "peak_source": f"{pk_kind} bf16 x {FP4_PER_BF16 if w.fmt != 'fp8' else FP8_PER_BF16:g} nominal ratio"}
+    else:
+        roof = {"kernel": dom, "bound": "hbm", "achieved": None, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": None, "traffic": None, "peak_source": pk_kind}
+
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "nvfp4" if w.fmt == "nvfp4" else w.fmt, "data": "synthetic",
+            "config": {"workload": workload_name(w), "global_batch": world * w.T, "parallelism": f"replicas x{world}",
+                       "act_scales": "static", "l2": "flushed between steps (write of 2x L2 bytes)",
+                       "routing": {"active_experts": alg["active_experts"], "max_over_mean": alg["max_over_mean"],
+                                   "zero_experts": alg["zero_experts"]}},
+            "stages_ms": stages, "roofline": roof, "e2e": e2e, "gpu_launches": int(res["launches"]),
+            "clocks": clocks, "device_status": res["status"]}
+
+    if not args.no_decode:
+        wd = synth.workload("decode")
+        dl = build_layer(ops, synth, torch, wd, static=False)
+        rd = time_forward(ops, torch, dl, wd, act, max(args.steps, 20), args.warmup, flush)
+        ad = algorithmic(wd, wd.fmt, rd["offsets"])
+        ffn_ms = rd["stages"].get("ffn_up", 0.0) + rd["stages"].get("ffn_down", 0.0)
+        gbs = (ad["wbytes_up"] + ad["wbytes_down"]) / (ffn_ms * 1e-3) / 1e9 if ffn_ms else None
+        line["decode"] = {"workload": workload_name(wd), "act_scales": "dynamic", "ms_per_step": float(np.mean(rd["ms"])),
+                          "tokens_per_s": wd.T / (float(np.mean(rd["ms"])) * 1e-3),
+                          "expert_weight_bytes": ad["wbytes_up"] + ad["wbytes_down"],
+                          "active_experts": ad["active_experts"], "ffn_ms": ffn_ms, "weight_gbs": gbs,
+                          "hbm_frac": gbs / pk["hbm_gbs"] if gbs else None, "stages_ms": rd["stages"]}
+        del dl
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_oracle_sample(w, args.cpu_seconds, static=True)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,267 @@
+/*
+ * moe_b200.h -- C ABI of the B200 (sm_100a) routed MoE expert FFN layer.
+ *
+ * The layer is the forward pass of a routed Mixture-of-Experts block as the
+ * FreeToken engine serves it (FreeToken upstream README, "About": MoE serving
+ * over MXFP4 / NVFP4 / FP8 / BF16 checkpoints):
+ *
+ *   logits = x Wr^T (+ b)                                    moe_route
+ *   idx, w = top-k of softmax(logits), renormalised          moe_route(_logits)
+ *   counts, offsets, stable permutation of the T*k slots     moe_permute
+ *   y_p    = SwiGLU expert FFN of x[perm_token[p]] over the
+ *            quantised weights of the slot's expert          moe_grouped_ffn
+ *   out_t  = sum_j w[t,j] y_{inv_perm[t*k+j]} (+ shared_t)    moe_combine
+ *   all of the above, enqueued as one call                   moe_forward
+ *
+ * Conventions shared by every entry point
+ *  - Pointers marked (device) are CUDA device pointers; (host) are host
+ *    pointers.  The caller owns every buffer.  No call allocates device
+ *    memory: scratch space comes from the caller's workspace `ws` of
+ *    `ws_bytes` bytes, sized by moe_workspace_size().
+ *  - bf16 tensors are passed as uint16_t bit patterns; all tensors are
+ *    row-major and contiguous.
+ *  - Calls are asynchronous on `stream` (never the legacy default stream
+ *    implicitly), perform no host synchronisation (except
+ *    moe_get_device_status) and are safe to capture in a CUDA graph once the
+ *    weights are prepared.
+ *  - Argument errors are detected on the host before anything is enqueued and
+ *    return MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED; outputs are then left
+ *    untouched.  An unknown format is MOE_ERR_UNSUPPORTED, never a silent
+ *    success with uninitialised output (the failure mode the
+ *    atomicmilkshake/FreeToken fork README describes under "What else
+ *    changed" for a kernel switch without a default).
+ *  - Faults found on the device (an expert index out of range, a NaN or
+ *    all -inf logit row, a bounded wait that ran out) set a status word inside
+ *    `ws`; the affected outputs are written with zeros, never left
+ *    uninitialised.  moe_get_device_status() reads and clears the word.
+ *  - A launch failure returns MOE_ERR_CUDA.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* moe_stream_t; /* identical to cudaStream_t */
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,
+  MOE_ERR_UNSUPPORTED = 2,
+  MOE_ERR_WORKSPACE = 3,
+  MOE_ERR_CUDA = 4,
+  MOE_ERR_DEVICE_FAULT = 5,
+  MOE_ERR_TIMEOUT = 6
+} moe_status;
+
+/* Expert weight formats.
+ *  NVFP4: e2m1 elements packed two per byte (element 2i in the low nibble),
+ *         one e4m3 scale per 16 elements along K, one fp32 global scale per
+ *         tensor part.
+ *  MXFP4: e2m1 elements as above, one e8m0 scale per 32 elements along K
+ *         (OCP Microscaling Formats v1.0).
+ *  FP8:   e4m3 elements, one fp32 per-tensor scale per part: the per-tensor
+ *         W8A8 scheme of FreeToken commit 58f4b9ec0e, where a fused
+ *         projection keeps one scale per part and the parts' row ranges come
+ *         from the load-time weight_scale run-lengths. */
+typedef enum { MOE_FMT_NVFP4 = 1, MOE_FMT_MXFP4 = 2, MOE_FMT_FP8 = 3 } moe_fmt;
+
+/* Activation precision.
+ *  BF16:  activations stay in bf16/fp32 (weight-only quantisation).
+ *  MATCH: activations are quantised to the weights' format before each
+ *         projection (W4A4 for NVFP4/MXFP4, W8A8 for FP8), the scheme of the
+ *         fused FP8 projection path (FreeToken commit 58f4b9ec0e) and of the
+ *         W4A8 decode kernel the atomicmilkshake fork names ("Known limits").
+ *         x and h are quantised with the same rules as the weights; a tensor
+ *         scale is static when given (a13_gs / a2_gs) and otherwise derived
+ *         from the tensor's amax (NVFP4: amax/2688, FP8: amax/448). */
+typedef enum { MOE_ACT_BF16 = 0, MOE_ACT_MATCH = 1 } moe_act;
+
+/* Layout of a moe_weights bundle. CANONICAL is the layout documented below.
+ * PREPARED is the device layout moe_prepare_weights() writes once at load
+ * time (gate/up rows interleaved, scales blocked for the tensor cores);
+ * only moe_prepare_weights() produces it. */
+typedef enum { MOE_LAYOUT_CANONICAL = 0, MOE_LAYOUT_PREPARED = 1 } moe_layout;
+
+/* One expert bank: E experts of one format, all tensors (device), read only.
+ * Merged gate|up projection ("merged projections", atomicmilkshake fork
+ * README, "What else changed") followed by the down projection
+ * ("ffn_down_exps", same README, "Known limits").  CANONICAL layout:
+ *   w13    [E][2I][H/2]  (FP8: [E][2I][H])   rows 0..I-1 gate, I..2I-1 up
+ *   w13_sf [E][2I][H/16] e4m3 (NVFP4) | [E][2I][H/32] e8m0 (MXFP4) | NULL (FP8)
+ *   w13_gs [E][2] fp32   gate and up part scales (NVFP4, FP8); NULL for MXFP4
+ *   w2     [E][H][I/2]   (FP8: [E][H][I])
+ *   w2_sf  [E][H][I/16] | [E][H][I/32] | NULL
+ *   w2_gs  [E] fp32      (NVFP4, FP8); NULL for MXFP4
+ *   a13_gs, a2_gs: one fp32 each, the static activation scale of x and of h
+ *          in MATCH mode (NVFP4 global scale / FP8 per-tensor scale); NULL
+ *          selects the dynamic amax-derived scale.  Unused for MXFP4.
+ * The pointed-to memory must stay valid while calls that use it run. */
+typedef struct {
+  int32_t fmt, E, H, I, layout;
+  const uint8_t* w13;
+  const uint8_t* w13_sf;
+  const float* w13_gs;
+  const uint8_t* w2;
+  const uint8_t* w2_sf;
+  const float* w2_gs;
+  const float* a13_gs;
+  const float* a2_gs;
+} moe_weights;
+
+/* Human-readable name of a status code (static string). */
+const char* moe_status_string(moe_status s);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+int32_t moe_version(void);
+
+/* Bytes of workspace every entry point of this header needs for a layer of
+ * T tokens, top-k, the given routed bank and optional shared expert bank
+ * (NULL), activation mode `act`.  One workspace of this size serves every
+ * call below for that layer; returns 0 on invalid arguments. */
+size_t moe_workspace_size(int64_t T, int32_t k, const moe_weights* routed, const moe_weights* shared,
+                          int32_t act);
+
+/* Bytes moe_prepare_weights() writes for a CANONICAL bank. */
+size_t moe_prepared_weights_size(const moe_weights* canonical);
+
+/* One-time, load-time repack of a CANONICAL bank into the device layout the
+ * kernels read (the role the FTW "fast weight format" plays in the FreeToken
+ * upstream README, "About"): gate/up rows interleaved (row 2i = gate i,
+ * row 2i+1 = up i) and scale factors blocked per 128 rows x 4 scale columns.
+ * Writes into `dst` (device, dst_bytes >= moe_prepared_weights_size()),
+ * fills *prepared (host) with pointers into dst and into the canonical
+ * bank's scalar arrays (w13_gs, w2_gs, a13_gs, a2_gs are shared, not copied).
+ * Requires H % 64 == 0 and I % 64 == 0 (MXFP4: % 128).  Enqueued on `stream`. */
+moe_status moe_prepare_weights(const moe_weights* canonical, void* dst, size_t dst_bytes,
+                               moe_weights* prepared, moe_stream_t stream);
+
+/* Quantise `rows` x `K` values into a CANONICAL-layout tensor of format
+ * `fmt`, with the same rules the layer applies to activations:
+ *   NVFP4: sc = e4m3(bmax/(6 g)), r = 1/(dec(sc) g), q = e2m1(x r)  (16-blocks)
+ *   MXFP4: c = clamp(floor(log2 bmax) - 2 + 127, 0, 254), q = e2m1(x 2^(127-c))
+ *   FP8:   q = e4m3(x * (1/s))
+ * in fp32, round-to-nearest-even, saturating.  x (device) is fp32
+ * (x_dtype 0) or bf16 bits (x_dtype 1).  scale_in (device, one fp32) is the
+ * NVFP4 global scale g / FP8 scale s; NULL derives it from the amax of all
+ * rows*K values (NVFP4 amax/2688, FP8 amax/448, 1 when the amax is 0).
+ * scale_out (device, nullable) receives the scale used.  codes (device):
+ * [rows][K/2] (FP8: [rows][K]); sf (device): [rows][K/16 | K/32], NULL for
+ * FP8.  K % 16 (NVFP4) / 32 (MXFP4) == 0.  Used to quantise checkpoints on the
+ * device, and the same device code quantises activations inside the layer. */
+moe_status moe_quantize(int32_t fmt, const void* x, int32_t x_dtype, int64_t rows, int64_t K,
+                        const float* scale_in, uint8_t* codes, uint8_t* sf, float* scale_out, void* ws,
+                        size_t ws_bytes, moe_stream_t stream);
+
+/* Router.  logits[t,e] = sum_h x[t,h] Wr[e,h] (+ bias[e]) in fp32;
+ * idx[t, 0..k-1] = the k largest logits in descending order, ties to the
+ * lower expert index; w[t,j] = exp(L_j - L_0) / sum_i exp(L_i - L_0) over the
+ * selected k (softmax over E renormalised over the top k).
+ *  x [T][H] bf16 (device), wr [E][H] bf16 (device), bias [E] fp32 (device,
+ *  nullable), logits [T][E] fp32 (device, nullable output), topk_idx [T][k]
+ *  int32 (device out), topk_w [T][k] fp32 (device out).
+ * 1 <= k <= E <= 1024; T >= 0 (T == 0 enqueues nothing).  A row with a NaN
+ * logit or no finite logit sets the device status word. */
+moe_status moe_route(const uint16_t* x, int64_t T, int32_t H, const uint16_t* wr, const float* bias, int32_t E,
+                     int32_t k, float* logits, int32_t* topk_idx, float* topk_w, void* ws, size_t ws_bytes,
+                     moe_stream_t stream);
+
+/* Top-k and renormalisation alone, from fp32 logits [T][E] (device). */
+moe_status moe_route_logits(const float* logits, int64_t T, int32_t E, int32_t k, int32_t* topk_idx,
+                            float* topk_w, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Token-to-expert histogram and stable permutation of the S = T*k slots
+ * (slot i = t*k + j, expert topk_idx[i]):
+ *   offsets[e]    exclusive prefix sum of the counts, offsets[E] = S   [E+1]
+ *   perm_token[p] token of the slot at expert-major position p         [S]
+ *   inv_perm[i]   position of slot i                                    [S]
+ * Positions within one expert follow the flat slot index (stable).  The
+ * expert segments are the "slot pool" rows the atomicmilkshake fork README
+ * ("Known limits") indexes per expert.  All pointers device.  Built without
+ * global atomics: per-chunk counts, a scan, then a rank pass.  An index
+ * outside [0, E) sets the device status word (the slot is dropped). */
+moe_status moe_permute(const int32_t* topk_idx, int64_t T, int32_t k, int32_t E, int32_t* offsets,
+                       int32_t* perm_token, int32_t* inv_perm, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Grouped SwiGLU expert FFN over the permuted slots: for expert e and every
+ * position p in [offsets[e], offsets[e+1]) with token t = perm_token[p]:
+ *   [g | u] = act(x_t) W13_e^T,  h = g / (1 + exp(-g)) * u,
+ *   y_perm[p] = act(h) W2_e^T                      (bf16 [S][H], device out)
+ * act() is the identity (BF16) or the quantiser of the weights' format
+ * (MATCH, see moe_act; the tensor amax of h is taken over all S slots).
+ * x [T][H] bf16, perm_token [S], offsets [E+1] (device); w must be
+ * PREPARED.  Small batches stream each active expert's weights once through
+ * a vectorised GEMV (the decode split of the atomicmilkshake fork README,
+ * "Quant types": MMVQ for decode, MMQ for prefill); large batches run a
+ * tcgen05 block-scaled grouped GEMM.  The choice is a host heuristic on the
+ * arguments (T*k versus E), never a device read-back. */
+moe_status moe_grouped_ffn(const uint16_t* x, int64_t T, int32_t k, const int32_t* perm_token,
+                           const int32_t* offsets, const moe_weights* w, int32_t act, uint16_t* y_perm, void* ws,
+                           size_t ws_bytes, moe_stream_t stream);
+
+/* Weighted un-permute: out[t] = sum_{j<k} w[t,j] y_perm[inv_perm[t*k+j]]
+ * (+ shared_y[t]) accumulated in fp32 in order j = 0..k-1, rounded once to
+ * bf16.  y_perm [T*k][H], shared_y [T][H] (nullable), out [T][H] bf16;
+ * inv_perm [T*k], topk_w [T][k]; all device. */
+moe_status moe_combine(const uint16_t* y_perm, const int32_t* inv_perm, const float* topk_w, int64_t T, int32_t k,
+                       int32_t H, const uint16_t* shared_y, uint16_t* out, void* ws, size_t ws_bytes,
+                       moe_stream_t stream);
+
+/* The whole layer in one call: route -> permute -> grouped FFN -> (shared
+ * expert, a dense SwiGLU FFN of the same format on every token with weight
+ * 1.0, the always-on expert the Domir6/FreeToken fork README lists under
+ * "Changes in this fork") -> combine.  x [T][H] bf16, wr [E][H] bf16,
+ * bias [E] (nullable), out [T][H] bf16 (device).  routed and shared
+ * (nullable, E == 1) must be PREPARED and of one format; the shared expert
+ * reads the same quantised x as the routed experts.  Intermediates live in
+ * `ws`. */
+moe_status moe_forward(const uint16_t* x, int64_t T, const uint16_t* wr, const float* bias, int32_t k,
+                       const moe_weights* routed, const moe_weights* shared, int32_t act, uint16_t* out, void* ws,
+                       size_t ws_bytes, moe_stream_t stream);
+
+/* Synchronises `stream`, copies the device status word of `ws` into
+ * *host_status (a moe_status value: MOE_OK, MOE_ERR_DEVICE_FAULT or
+ * MOE_ERR_TIMEOUT) and clears it.  Returns MOE_ERR_CUDA if the
+ * synchronisation itself fails. */
+moe_status moe_get_device_status(void* ws, moe_stream_t stream, int32_t* host_status);
+
+/* Process-wide switches for A/B measurement (the pattern of the
+ * FREETOKEN_FP8_ROWWISE_MM variable in FreeToken commit 58f4b9ec0e).
+ *   MOE_OPT_FFN_PATH: 0 = heuristic (default), 1 = force the GEMV path,
+ *                     2 = force the tensor-core GEMM path (returns
+ *                     MOE_ERR_UNSUPPORTED where the shapes do not allow it).
+ * Not thread-safe; set before enqueuing. */
+typedef enum { MOE_OPT_FFN_PATH = 1 } moe_option;
+moe_status moe_set_option(int32_t option, int32_t value);
+
+/* Measurement hooks.
+ * moe_set_stage_events: when `events` is non-NULL it must hold
+ * 2 * MOE_STAGE_COUNT cudaEvent_t handles; moe_forward and moe_grouped_ffn
+ * then record events[2*s] before and events[2*s+1] after stage s on their
+ * stream, so a caller can time each stage with cudaEventElapsedTime.  Stages
+ * a call does not run are not recorded.  NULL turns the hook off.  Not
+ * thread-safe; the handles must outlive the calls that record them.
+ * moe_kernel_launch_count: number of kernels this library has launched in
+ * the process so far (host-side count of kernel launches). */
+typedef enum {
+  MOE_STAGE_ROUTE = 0,      /* router logits + top-k */
+  MOE_STAGE_PERMUTE = 1,    /* histogram, scan, permutation */
+  MOE_STAGE_ACT_QUANT = 2,  /* activation amax / quantisation of x */
+  MOE_STAGE_FFN_UP = 3,     /* gate|up projection + SwiGLU */
+  MOE_STAGE_FFN_DOWN = 4,   /* down projection */
+  MOE_STAGE_SHARED = 5,     /* shared expert (both projections) */
+  MOE_STAGE_COMBINE = 6,    /* weighted un-permute */
+  MOE_STAGE_COUNT = 7
+} moe_stage;
+moe_status moe_set_stage_events(void* const* events, int32_t n_events);
+uint64_t moe_kernel_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

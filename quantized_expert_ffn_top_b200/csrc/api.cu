@@ -1,0 +1,524 @@
+// C ABI of the B200 MoE layer (declared in include/moe_b200.h): argument
+// checks on the host, workspace carving, path choice, and the launch
+// sequence.  Every step of the layer runs in the kernels of this library.
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "kernels.cuh"
+
+namespace moe {
+namespace {
+
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Sequential carving of the workspace (base == nullptr only measures).
+struct Carver {
+  char* base;
+  size_t off;
+  explicit Carver(void* b) : base(static_cast<char*>(b)), off(0) {}
+  template <typename T>
+  T* take(size_t count) {
+    off = align_up(off, kAlign);
+    T* p = base ? reinterpret_cast<T*>(base + off) : nullptr;
+    off += count * sizeof(T);
+    return p;
+  }
+};
+
+struct Scalars {
+  int32_t* status;
+  float* x_amax;
+  float* h_amax;
+  float* sh_h_amax;
+};
+
+Scalars carve_head(Carver& c) {
+  Scalars s;
+  s.status = c.take<int32_t>(1);
+  float* f = c.take<float>(8);
+  s.x_amax = f;
+  s.h_amax = f ? f + 1 : nullptr;
+  s.sh_h_amax = f ? f + 2 : nullptr;
+  return s;
+}
+
+int g_ffn_path = 0;  // MOE_OPT_FFN_PATH
+
+// Measurement hook (moe_set_stage_events).
+cudaEvent_t g_stage_events[2 * MOE_STAGE_COUNT];
+bool g_stage_on = false;
+
+void stage_mark(int stage, bool end, cudaStream_t s) {
+  if (g_stage_on) cudaEventRecord(g_stage_events[2 * stage + (end ? 1 : 0)], s);
+}
+
+int num_sms() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cached[dev] == 0) {
+    int v = 0;
+    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    cached[dev] = v > 0 ? v : 148;
+  }
+  return cached[dev];
+}
+
+moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+#define MOE_TRY(expr)                          \
+  do {                                         \
+    cudaError_t _e = (expr);                   \
+    if (_e != cudaSuccess) return MOE_ERR_CUDA; \
+  } while (0)
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int block_size(int fmt) { return fmt == MOE_FMT_NVFP4 ? 16 : (fmt == MOE_FMT_MXFP4 ? 32 : 0); }
+
+// Shape and pointer checks of a weight bank.
+moe_status check_weights(const moe_weights* w, bool need_prepared) {
+  if (!w) return MOE_ERR_INVALID_ARG;
+  if (w->fmt != MOE_FMT_NVFP4 && w->fmt != MOE_FMT_MXFP4 && w->fmt != MOE_FMT_FP8) return MOE_ERR_UNSUPPORTED;
+  if (w->E < 1 || w->E > 1024 || w->H <= 0 || w->I <= 0) return MOE_ERR_INVALID_ARG;
+  if (w->H % 128 != 0 || w->I % 128 != 0) return MOE_ERR_UNSUPPORTED;
+  if (w->layout != MOE_LAYOUT_CANONICAL && w->layout != MOE_LAYOUT_PREPARED) return MOE_ERR_INVALID_ARG;
+  if (need_prepared && w->layout != MOE_LAYOUT_PREPARED) return MOE_ERR_UNSUPPORTED;
+  if (!w->w13 || !w->w2) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(w->w13) || !aligned16(w->w2) || !aligned16(w->w13_sf) || !aligned16(w->w2_sf))
+    return MOE_ERR_INVALID_ARG;
+  if (w->fmt != MOE_FMT_FP8 && (!w->w13_sf || !w->w2_sf)) return MOE_ERR_INVALID_ARG;
+  if (w->fmt != MOE_FMT_MXFP4 && (!w->w13_gs || !w->w2_gs)) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+// ---------------------------------------------------------------- layouts --
+struct RouteWs {
+  Scalars head;
+  float* logits;
+};
+RouteWs carve_route(Carver& c, int64_t T, int E) {
+  RouteWs r;
+  r.head = carve_head(c);
+  r.logits = c.take<float>((size_t)T * E);
+  return r;
+}
+
+struct PermWs {
+  Scalars head;
+  PermuteScratch scratch;
+};
+PermWs carve_perm(Carver& c, int64_t S, int E) {
+  PermWs p;
+  p.head = carve_head(c);
+  p.scratch.nchunks = (int)((S + permute_chunk_slots() - 1) / permute_chunk_slots());
+  p.scratch.chunk_counts = c.take<int32_t>((size_t)(p.scratch.nchunks > 0 ? p.scratch.nchunks : 1) * E);
+  return p;
+}
+
+struct FfnScratch {
+  float* h;  // [S][I]
+};
+FfnScratch carve_ffn(Carver& c, int64_t S, const moe_weights* w) {
+  FfnScratch f;
+  f.h = c.take<float>((size_t)S * w->I);
+  return f;
+}
+
+struct ForwardWs {
+  Scalars head;
+  float* logits;
+  int32_t* idx;
+  float* w;
+  int32_t* offsets;
+  int32_t* perm;
+  int32_t* inv;
+  PermuteScratch pscratch;
+  uint16_t* y_perm;
+  FfnScratch ffn;
+  int32_t* sh_offsets;
+  int32_t* sh_perm;
+  uint16_t* sh_y;
+  FfnScratch sh_ffn;
+};
+ForwardWs carve_forward(Carver& c, int64_t T, int k, const moe_weights* routed, const moe_weights* shared) {
+  ForwardWs f;
+  const int E = routed->E;
+  const int64_t S = T * k;
+  f.head = carve_head(c);
+  f.logits = c.take<float>((size_t)T * E);
+  f.idx = c.take<int32_t>((size_t)S);
+  f.w = c.take<float>((size_t)S);
+  f.offsets = c.take<int32_t>((size_t)E + 1);
+  f.perm = c.take<int32_t>((size_t)S);
+  f.inv = c.take<int32_t>((size_t)S);
+  f.pscratch.nchunks = (int)((S + permute_chunk_slots() - 1) / permute_chunk_slots());
+  f.pscratch.chunk_counts = c.take<int32_t>((size_t)(f.pscratch.nchunks > 0 ? f.pscratch.nchunks : 1) * E);
+  f.y_perm = c.take<uint16_t>((size_t)S * routed->H);
+  f.ffn = carve_ffn(c, S, routed);
+  if (shared) {
+    f.sh_offsets = c.take<int32_t>(2);
+    f.sh_perm = c.take<int32_t>((size_t)T);
+    f.sh_y = c.take<uint16_t>((size_t)T * routed->H);
+    f.sh_ffn = carve_ffn(c, T, shared);
+  } else {
+    f.sh_offsets = f.sh_perm = nullptr;
+    f.sh_y = nullptr;
+    f.sh_ffn.h = nullptr;
+  }
+  return f;
+}
+
+// --------------------------------------------------------------- helpers --
+__global__ void identity_routing_kernel(int64_t T, int32_t* offsets, int32_t* perm) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < T) perm[i] = (int32_t)i;
+  if (i == 0) {
+    offsets[0] = 0;
+    offsets[1] = (int32_t)T;
+  }
+}
+
+bool use_gemm_path(const moe_weights* w, int64_t S, int act) {
+  (void)w;
+  (void)S;
+  (void)act;
+  return false;
+}
+
+// Grouped FFN on already-validated arguments.  x_amax must hold amax(x) when
+// the x scale is dynamic (MATCH, NVFP4/FP8, no a13_gs).
+moe_status run_grouped_ffn(const uint16_t* x, int64_t T, int64_t S, const int32_t* perm, const int32_t* offsets,
+                           const moe_weights* w, int act, uint16_t* y_perm, const FfnScratch& scratch,
+                           float* x_amax, float* h_amax, int32_t* status, cudaStream_t s,
+                           bool shared_stage = false) {
+  if (S == 0) return MOE_OK;
+  if (g_ffn_path == 2) return MOE_ERR_UNSUPPORTED;
+  const bool mark = !shared_stage;
+  GemvArgs a;
+  a.fmt = w->fmt;
+  a.act = act;
+  a.E = w->E;
+  a.H = w->H;
+  a.I = w->I;
+  a.w13 = w->w13;
+  a.w13_sf = w->w13_sf;
+  a.w13_gs = w->w13_gs;
+  a.w2 = w->w2;
+  a.w2_sf = w->w2_sf;
+  a.w2_gs = w->w2_gs;
+  a.x_scale = w->a13_gs;
+  a.h_scale = w->a2_gs;
+  a.x = x;
+  a.T = T;
+  a.S = S;
+  a.perm_token = perm;
+  a.offsets = offsets;
+  a.x_amax = x_amax;
+  a.h_amax = (act == MOE_ACT_MATCH && w->fmt != MOE_FMT_MXFP4 && !w->a2_gs) ? h_amax : nullptr;
+  a.h = scratch.h;
+  a.y_perm = y_perm;
+  a.status = status;
+  if (mark) stage_mark(MOE_STAGE_FFN_UP, false, s);
+  MOE_TRY(launch_gemv_up(a, s));
+  if (mark) stage_mark(MOE_STAGE_FFN_UP, true, s);
+  if (mark) stage_mark(MOE_STAGE_FFN_DOWN, false, s);
+  MOE_TRY(launch_gemv_down(a, s));
+  if (mark) stage_mark(MOE_STAGE_FFN_DOWN, true, s);
+  return MOE_OK;
+}
+
+bool dynamic_x_scale(const moe_weights* w, int act) {
+  return act == MOE_ACT_MATCH && w->fmt != MOE_FMT_MXFP4 && !w->a13_gs;
+}
+
+}  // namespace
+
+static uint64_t g_launches = 0;
+static std::mutex g_launch_mu;
+void count_launches(int n) {
+  std::lock_guard<std::mutex> lk(g_launch_mu);
+  g_launches += (uint64_t)n;
+}
+uint64_t launches_so_far() {
+  std::lock_guard<std::mutex> lk(g_launch_mu);
+  return g_launches;
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+const char* moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG: invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED: unsupported format, layout or shape";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE: workspace too small";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA: CUDA launch or runtime error";
+    case MOE_ERR_DEVICE_FAULT: return "MOE_ERR_DEVICE_FAULT: invalid data found on the device";
+    case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT: a bounded device wait ran out";
+  }
+  return "unknown moe_status";
+}
+
+int32_t moe_version(void) { return 100; }
+
+moe_status moe_set_option(int32_t option, int32_t value) {
+  if (option == MOE_OPT_FFN_PATH) {
+    if (value < 0 || value > 2) return MOE_ERR_INVALID_ARG;
+    g_ffn_path = value;
+    return MOE_OK;
+  }
+  return MOE_ERR_INVALID_ARG;
+}
+
+size_t moe_workspace_size(int64_t T, int32_t k, const moe_weights* routed, const moe_weights* shared, int32_t act) {
+  if (T < 0 || k < 1 || check_weights(routed, false) != MOE_OK) return 0;
+  if (shared && (check_weights(shared, false) != MOE_OK || shared->E != 1)) return 0;
+  if (act != MOE_ACT_BF16 && act != MOE_ACT_MATCH) return 0;
+  Carver c(nullptr);
+  carve_forward(c, T, k, routed, shared);
+  size_t need = c.off;
+  Carver c2(nullptr);
+  carve_head(c2);
+  carve_ffn(c2, T * k, routed);
+  need = need > c2.off ? need : c2.off;
+  return align_up(need, kAlign);
+}
+
+size_t moe_prepared_weights_size(const moe_weights* w) {
+  if (check_weights(w, false) != MOE_OK) return 0;
+  const int64_t E = w->E, H = w->H, I = w->I;
+  const int bs = block_size(w->fmt);
+  const int64_t rb13 = w->fmt == MOE_FMT_FP8 ? H : H / 2, rb2 = w->fmt == MOE_FMT_FP8 ? I : I / 2;
+  Carver c(nullptr);
+  c.take<uint8_t>((size_t)(E * 2 * I * rb13));
+  c.take<uint8_t>((size_t)(E * H * rb2));
+  if (bs) {
+    c.take<uint8_t>((size_t)(E * 2 * I * (H / bs)));
+    c.take<uint8_t>((size_t)(E * H * (I / bs)));
+  }
+  return align_up(c.off, kAlign);
+}
+
+moe_status moe_prepare_weights(const moe_weights* w, void* dst, size_t dst_bytes, moe_weights* prepared,
+                               moe_stream_t stream) {
+  moe_status st = check_weights(w, false);
+  if (st != MOE_OK) return st;
+  if (w->layout != MOE_LAYOUT_CANONICAL || !dst || !prepared) return MOE_ERR_INVALID_ARG;
+  if (dst_bytes < moe_prepared_weights_size(w)) return MOE_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t E = w->E, H = w->H, I = w->I;
+  const int bs = block_size(w->fmt);
+  const int64_t rb13 = w->fmt == MOE_FMT_FP8 ? H : H / 2, rb2 = w->fmt == MOE_FMT_FP8 ? I : I / 2;
+  Carver c(dst);
+  uint8_t* w13 = c.take<uint8_t>((size_t)(E * 2 * I * rb13));
+  uint8_t* w2 = c.take<uint8_t>((size_t)(E * H * rb2));
+  uint8_t* sf13 = nullptr;
+  uint8_t* sf2 = nullptr;
+  if (bs) {
+    sf13 = c.take<uint8_t>((size_t)(E * 2 * I * (H / bs)));
+    sf2 = c.take<uint8_t>((size_t)(E * H * (I / bs)));
+  }
+  MOE_TRY(launch_prepare_rows(w->fmt, w->w13, w13, E, 2 * I, rb13, true, s));
+  MOE_TRY(launch_prepare_rows(w->fmt, w->w2, w2, E, H, rb2, false, s));
+  if (bs) {
+    MOE_TRY(launch_prepare_sf(w->w13_sf, sf13, E, 2 * I, H / bs, H / bs, true, s));
+    MOE_TRY(launch_prepare_sf(w->w2_sf, sf2, E, H, I / bs, I / bs, false, s));
+  }
+  *prepared = *w;
+  prepared->layout = MOE_LAYOUT_PREPARED;
+  prepared->w13 = w13;
+  prepared->w2 = w2;
+  prepared->w13_sf = sf13;
+  prepared->w2_sf = sf2;
+  return MOE_OK;
+}
+
+moe_status moe_quantize(int32_t fmt, const void* x, int32_t x_dtype, int64_t rows, int64_t K, const float* scale_in,
+                        uint8_t* codes, uint8_t* sf, float* scale_out, void* ws, size_t ws_bytes,
+                        moe_stream_t stream) {
+  if (fmt != MOE_FMT_NVFP4 && fmt != MOE_FMT_MXFP4 && fmt != MOE_FMT_FP8) return MOE_ERR_UNSUPPORTED;
+  if (rows < 0 || K <= 0 || (x_dtype != 0 && x_dtype != 1)) return MOE_ERR_INVALID_ARG;
+  const int bs = fmt == MOE_FMT_MXFP4 ? 32 : 16;
+  if (K % bs != 0) return MOE_ERR_UNSUPPORTED;
+  if (rows > 0 && (!x || !codes || (fmt != MOE_FMT_FP8 && !sf))) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(codes)) return MOE_ERR_INVALID_ARG;
+  Carver c(ws);
+  Scalars head = carve_head(c);
+  if (!ws || ws_bytes < c.off) return MOE_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (rows == 0) return MOE_OK;
+  if (fmt != MOE_FMT_MXFP4 && !scale_in) MOE_TRY(launch_amax(x, x_dtype, rows * K, head.x_amax, num_sms(), s));
+  return cuda_status(launch_quantize(fmt, x, x_dtype, rows, K, scale_in, head.x_amax, codes, sf, scale_out,
+                                     num_sms(), s));
+}
+
+moe_status moe_route(const uint16_t* x, int64_t T, int32_t H, const uint16_t* wr, const float* bias, int32_t E,
+                     int32_t k, float* logits, int32_t* topk_idx, float* topk_w, void* ws, size_t ws_bytes,
+                     moe_stream_t stream) {
+  if (T < 0 || H <= 0 || H % 8 != 0 || E < 1 || E > 1024 || k < 1 || k > E) return MOE_ERR_INVALID_ARG;
+  if (T > 0 && (!x || !wr || !topk_idx || !topk_w)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(wr)) return MOE_ERR_INVALID_ARG;
+  Carver c(ws);
+  RouteWs r = carve_route(c, logits ? 0 : T, E);
+  if (!ws || ws_bytes < c.off) return MOE_ERR_WORKSPACE;
+  if (T == 0) return MOE_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  float* L = logits ? logits : r.logits;
+  MOE_TRY(launch_router_logits(x, T, H, wr, bias, E, L, s));
+  return cuda_status(launch_topk(L, T, E, k, topk_idx, topk_w, r.head.status, s));
+}
+
+moe_status moe_route_logits(const float* logits, int64_t T, int32_t E, int32_t k, int32_t* topk_idx, float* topk_w,
+                            void* ws, size_t ws_bytes, moe_stream_t stream) {
+  if (T < 0 || E < 1 || E > 1024 || k < 1 || k > E) return MOE_ERR_INVALID_ARG;
+  if (T > 0 && (!logits || !topk_idx || !topk_w)) return MOE_ERR_INVALID_ARG;
+  Carver c(ws);
+  Scalars head = carve_head(c);
+  if (!ws || ws_bytes < c.off) return MOE_ERR_WORKSPACE;
+  return cuda_status(launch_topk(logits, T, E, k, topk_idx, topk_w, head.status,
+                                 reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_permute(const int32_t* topk_idx, int64_t T, int32_t k, int32_t E, int32_t* offsets,
+                       int32_t* perm_token, int32_t* inv_perm, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  if (T < 0 || k < 1 || E < 1 || E > 1024 || T * (int64_t)k > INT32_MAX) return MOE_ERR_INVALID_ARG;
+  if (!offsets || (T > 0 && (!topk_idx || !perm_token || !inv_perm))) return MOE_ERR_INVALID_ARG;
+  Carver c(ws);
+  PermWs p = carve_perm(c, T * k, E);
+  if (!ws || ws_bytes < c.off) return MOE_ERR_WORKSPACE;
+  return cuda_status(launch_permute(topk_idx, T * k, k, E, offsets, perm_token, inv_perm, p.scratch, p.head.status,
+                                    reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_grouped_ffn(const uint16_t* x, int64_t T, int32_t k, const int32_t* perm_token, const int32_t* offsets,
+                           const moe_weights* w, int32_t act, uint16_t* y_perm, void* ws, size_t ws_bytes,
+                           moe_stream_t stream) {
+  moe_status st = check_weights(w, true);
+  if (st != MOE_OK) return st;
+  if (T < 0 || k < 1 || (act != MOE_ACT_BF16 && act != MOE_ACT_MATCH)) return MOE_ERR_INVALID_ARG;
+  if (T > 0 && (!x || !perm_token || !offsets || !y_perm)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(y_perm)) return MOE_ERR_INVALID_ARG;
+  const int64_t S = T * k;
+  Carver c(ws);
+  Scalars head = carve_head(c);
+  FfnScratch f = carve_ffn(c, S, w);
+  if (!ws || ws_bytes < c.off) return MOE_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (S == 0) return MOE_OK;
+  if (dynamic_x_scale(w, act)) {
+    stage_mark(MOE_STAGE_ACT_QUANT, false, s);
+    MOE_TRY(launch_amax(x, 1, T * w->H, head.x_amax, num_sms(), s));
+    stage_mark(MOE_STAGE_ACT_QUANT, true, s);
+  }
+  return run_grouped_ffn(x, T, S, perm_token, offsets, w, act, y_perm, f, head.x_amax, head.h_amax, head.status, s);
+}
+
+moe_status moe_combine(const uint16_t* y_perm, const int32_t* inv_perm, const float* topk_w, int64_t T, int32_t k,
+                       int32_t H, const uint16_t* shared_y, uint16_t* out, void* ws, size_t ws_bytes,
+                       moe_stream_t stream) {
+  if (T < 0 || k < 1 || H <= 0 || H % 8 != 0) return MOE_ERR_INVALID_ARG;
+  if (T > 0 && (!y_perm || !inv_perm || !topk_w || !out)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(y_perm) || !aligned16(out) || !aligned16(shared_y)) return MOE_ERR_INVALID_ARG;
+  Carver c(ws);
+  Scalars head = carve_head(c);
+  if (!ws || ws_bytes < c.off) return MOE_ERR_WORKSPACE;
+  return cuda_status(launch_combine(y_perm, inv_perm, topk_w, T, k, H, shared_y, out, head.status,
+                                    reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_forward(const uint16_t* x, int64_t T, const uint16_t* wr, const float* bias, int32_t k,
+                       const moe_weights* routed, const moe_weights* shared, int32_t act, uint16_t* out, void* ws,
+                       size_t ws_bytes, moe_stream_t stream) {
+  moe_status st = check_weights(routed, true);
+  if (st != MOE_OK) return st;
+  if (shared) {
+    st = check_weights(shared, true);
+    if (st != MOE_OK) return st;
+    if (shared->E != 1 || shared->H != routed->H || shared->fmt != routed->fmt) return MOE_ERR_INVALID_ARG;
+  }
+  const int E = routed->E, H = routed->H;
+  if (T < 0 || k < 1 || k > E || (act != MOE_ACT_BF16 && act != MOE_ACT_MATCH)) return MOE_ERR_INVALID_ARG;
+  if (T * (int64_t)k > INT32_MAX) return MOE_ERR_INVALID_ARG;
+  if (T > 0 && (!x || !wr || !out)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(wr) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+  Carver c(ws);
+  ForwardWs f = carve_forward(c, T, k, routed, shared);
+  if (!ws || ws_bytes < c.off) return MOE_ERR_WORKSPACE;
+  if (T == 0) return MOE_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t S = T * k;
+  // 1. router
+  stage_mark(MOE_STAGE_ROUTE, false, s);
+  MOE_TRY(launch_router_logits(x, T, H, wr, bias, E, f.logits, s));
+  MOE_TRY(launch_topk(f.logits, T, E, k, f.idx, f.w, f.head.status, s));
+  stage_mark(MOE_STAGE_ROUTE, true, s);
+  // 2. histogram + permutation
+  stage_mark(MOE_STAGE_PERMUTE, false, s);
+  MOE_TRY(launch_permute(f.idx, S, k, E, f.offsets, f.perm, f.inv, f.pscratch, f.head.status, s));
+  stage_mark(MOE_STAGE_PERMUTE, true, s);
+  // 3. dynamic activation scale of x (shared by routed and shared experts)
+  if (dynamic_x_scale(routed, act)) {
+    stage_mark(MOE_STAGE_ACT_QUANT, false, s);
+    MOE_TRY(launch_amax(x, 1, T * H, f.head.x_amax, num_sms(), s));
+    stage_mark(MOE_STAGE_ACT_QUANT, true, s);
+  }
+  // 4. routed experts
+  st = run_grouped_ffn(x, T, S, f.perm, f.offsets, routed, act, f.y_perm, f.ffn, f.head.x_amax, f.head.h_amax,
+                       f.head.status, s);
+  if (st != MOE_OK) return st;
+  // 5. shared expert: every token, identity order; it reads routed's x scale
+  if (shared) {
+    stage_mark(MOE_STAGE_SHARED, false, s);
+    identity_routing_kernel<<<(unsigned)((T + 255) / 256), 256, 0, s>>>(T, f.sh_offsets, f.sh_perm);
+    count_launches(1);
+    MOE_TRY(cudaGetLastError());
+    moe_weights sh = *shared;
+    sh.a13_gs = routed->a13_gs;
+    st = run_grouped_ffn(x, T, T, f.sh_perm, f.sh_offsets, &sh, act, f.sh_y, f.sh_ffn, f.head.x_amax,
+                         f.head.sh_h_amax, f.head.status, s, true);
+    if (st != MOE_OK) return st;
+    stage_mark(MOE_STAGE_SHARED, true, s);
+  }
+  // 6. combine
+  stage_mark(MOE_STAGE_COMBINE, false, s);
+  st = cuda_status(launch_combine(f.y_perm, f.inv, f.w, T, k, H, f.sh_y, out, f.head.status, s));
+  stage_mark(MOE_STAGE_COMBINE, true, s);
+  return st;
+}
+
+moe_status moe_set_stage_events(void* const* events, int32_t n_events) {
+  if (!events) {
+    g_stage_on = false;
+    return MOE_OK;
+  }
+  if (n_events < 2 * MOE_STAGE_COUNT) return MOE_ERR_INVALID_ARG;
+  for (int i = 0; i < 2 * MOE_STAGE_COUNT; ++i) {
+    if (!events[i]) return MOE_ERR_INVALID_ARG;
+    g_stage_events[i] = reinterpret_cast<cudaEvent_t>(events[i]);
+  }
+  g_stage_on = true;
+  return MOE_OK;
+}
+
+uint64_t moe_kernel_launch_count(void) { return launches_so_far(); }
+
+moe_status moe_get_device_status(void* ws, moe_stream_t stream, int32_t* host_status) {
+  if (!ws || !host_status) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int32_t v = 0;
+  if (cudaMemcpyAsync(&v, ws, sizeof(int32_t), cudaMemcpyDeviceToHost, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaMemsetAsync(ws, 0, sizeof(int32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+  *host_status = v;
+  return MOE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,60 @@
+// Weighted un-permute combine: out[t] = sum_{j<k} w[t,j] * y_perm[inv_perm[t*k+j]]
+// (+ shared_y[t]), accumulated in fp32 in the order j = 0..k-1 and rounded
+// once to bf16.  The always-on shared expert enters with weight 1.0 (the
+// shared expert of the Domir6/FreeToken fork README, "Changes in this fork").
+// One block per token; each thread owns 8 consecutive columns (16-byte loads).
+#include "kernels.cuh"
+
+namespace moe {
+
+__global__ void __launch_bounds__(128) combine_kernel(const uint16_t* __restrict__ y_perm,
+                                                      const int32_t* __restrict__ inv_perm,
+                                                      const float* __restrict__ w, int64_t T, int k, int H,
+                                                      const uint16_t* __restrict__ shared_y,
+                                                      uint16_t* __restrict__ out, int32_t* status) {
+  const int64_t t = blockIdx.x;
+  const int64_t S = T * k;
+  for (int c = threadIdx.x * 8; c < H; c += blockDim.x * 8) {
+    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    for (int j = 0; j < k; ++j) {
+      const int32_t p = __ldg(inv_perm + t * k + j);
+      if (p < 0 || p >= S) {
+        if (c == threadIdx.x * 8 && p >= S) raise_status(status, MOE_ERR_DEVICE_FAULT);
+        continue;
+      }
+      const float wj = __ldg(w + t * k + j);
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(y_perm + (int64_t)p * H + c));
+      const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        acc[2 * i] = fmaf(wj, __uint_as_float(vv[i] << 16), acc[2 * i]);
+        acc[2 * i + 1] = fmaf(wj, __uint_as_float(vv[i] & 0xFFFF0000u), acc[2 * i + 1]);
+      }
+    }
+    if (shared_y) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(shared_y + t * H + c));
+      const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        acc[2 * i] += __uint_as_float(vv[i] << 16);
+        acc[2 * i + 1] += __uint_as_float(vv[i] & 0xFFFF0000u);
+      }
+    }
+    uint4 o;
+    uint32_t* po = &o.x;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      po[i] = (uint32_t)f32_to_bf16_rn(acc[2 * i]) | ((uint32_t)f32_to_bf16_rn(acc[2 * i + 1]) << 16);
+    *reinterpret_cast<uint4*>(out + t * H + c) = o;
+  }
+}
+
+cudaError_t launch_combine(const uint16_t* y_perm, const int32_t* inv_perm, const float* w, int64_t T, int k, int H,
+                           const uint16_t* shared_y, uint16_t* out, int32_t* status, cudaStream_t s) {
+  if (T == 0) return cudaSuccess;
+  combine_kernel<<<(unsigned)T, 128, 0, s>>>(y_perm, inv_perm, w, T, k, H, shared_y, out, status);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,81 @@
+// Kernel launchers of the B200 MoE layer (internal; the C ABI is in api.cu).
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+
+// Host-side count of kernel launches (moe_kernel_launch_count).
+void count_launches(int n);
+
+__device__ __forceinline__ float load_f32(const float* p) { return __ldg(p); }
+__device__ __forceinline__ float load_f32(const uint16_t* p) { return bf16_to_f32(__ldg(p)); }
+
+// Blocked scale-factor layout of PREPARED banks and of the GEMM path's
+// quantised activations: per 128 rows and per group of 4 consecutive scale
+// columns, one 512-byte block in which row r's 4 scales sit at byte
+// (r % 32) * 16 + ((r % 128) / 32) * 4 -- the order in which the tensor core
+// scale-factor copy (tcgen05.cp 32x128b, replicated to the four lane
+// quarters) lays 128 rows x 4 scales into tensor memory.
+__host__ __device__ __forceinline__ int64_t sf_blocked_offset(int64_t row, int64_t col, int64_t ncols) {
+  const int64_t groups = ncols / 4;  // scale columns are padded to a multiple of 4
+  return ((row / 128) * groups + col / 4) * 512 + (row % 32) * 16 + ((row % 128) / 32) * 4 + (col % 4);
+}
+
+// quant.cu
+cudaError_t launch_amax(const void* x, int x_dtype, int64_t n, float* out, int num_sms, cudaStream_t s);
+cudaError_t launch_quantize(int fmt, const void* x, int x_dtype, int64_t rows, int64_t K, const float* scale_in,
+                            const float* amax, uint8_t* codes, uint8_t* sf, float* scale_out, int num_sms,
+                            cudaStream_t s);
+
+// route.cu
+cudaError_t launch_router_logits(const uint16_t* x, int64_t T, int H, const uint16_t* wr, const float* bias, int E,
+                                 float* logits, cudaStream_t s);
+cudaError_t launch_topk(const float* logits, int64_t T, int E, int k, int32_t* idx, float* w, int32_t* status,
+                        cudaStream_t s);
+
+// permute.cu
+struct PermuteScratch {
+  int32_t* chunk_counts;   // [nchunks][E]
+  int nchunks;
+};
+int permute_chunk_slots();
+cudaError_t launch_permute(const int32_t* idx, int64_t S, int k, int E, int32_t* offsets, int32_t* perm_token,
+                           int32_t* inv_perm, PermuteScratch scratch, int32_t* status, cudaStream_t s);
+
+// gemv.cu -- small-batch expert FFN (one pass over each active expert).
+struct GemvArgs {
+  int fmt, act, E, H, I;
+  const uint8_t* w13;      // prepared
+  const uint8_t* w13_sf;
+  const float* w13_gs;
+  const uint8_t* w2;
+  const uint8_t* w2_sf;
+  const float* w2_gs;
+  const float* x_scale;    // MATCH: static scale (device) or nullptr
+  const float* h_scale;
+  const uint16_t* x;       // [T][H]
+  int64_t T;
+  int64_t S;               // slots: offsets must satisfy 0 <= offsets[e] <= offsets[e+1] <= S
+  const int32_t* perm_token;
+  const int32_t* offsets;
+  float* x_amax;           // workspace scalars (dynamic scales)
+  float* h_amax;
+  float* h;                // [S][I] fp32
+  uint16_t* y_perm;        // [S][H]
+  int32_t* status;
+};
+cudaError_t launch_gemv_up(const GemvArgs& a, cudaStream_t s);
+cudaError_t launch_gemv_down(const GemvArgs& a, cudaStream_t s);
+
+// combine.cu
+cudaError_t launch_combine(const uint16_t* y_perm, const int32_t* inv_perm, const float* w, int64_t T, int k, int H,
+                           const uint16_t* shared_y, uint16_t* out, int32_t* status, cudaStream_t s);
+
+// prepare.cu
+cudaError_t launch_prepare_rows(int fmt, const uint8_t* src, uint8_t* dst, int64_t E, int64_t R, int64_t row_bytes,
+                                bool interleave, cudaStream_t s);
+cudaError_t launch_prepare_sf(const uint8_t* src, uint8_t* dst, int64_t E, int64_t R, int64_t ncols,
+                              int64_t ncols_padded, bool interleave, cudaStream_t s);
+
+}  // namespace moe

@@ -1,0 +1,175 @@
+// Token-to-expert histogram, offsets and stable permutation of the T*k slots,
+// without global atomics.
+//
+// The permuted order is the expert-major "slot pool" of the
+// atomicmilkshake/FreeToken fork README ("Known limits"): every expert's slots
+// form one contiguous segment, so the grouped FFN reads each expert's weights
+// for a dense block of rows.  Slots keep their flat order i = t*k + j inside a
+// segment (stable), which makes the permutation unique and bit-comparable.
+//
+// Three passes over chunks of kChunk slots (8 warps x 256):
+//   1. per chunk and expert, the count (warp-private counters fed by
+//      __match_any_sync, one writer lane per expert and step);
+//   2. one block: per expert the exclusive prefix over chunks, the totals, and
+//      the exclusive prefix over experts -> offsets;
+//   3. per chunk again: each warp's base = chunk base + earlier warps'
+//      counts, and each slot's rank among equal experts earlier in its warp
+//      step -> perm_token[p] = t, inv_perm[i] = p.
+#include "kernels.cuh"
+
+namespace moe {
+
+constexpr int kPermWarps = 8;
+constexpr int kSlotsPerWarp = 256;
+constexpr int kChunk = kPermWarps * kSlotsPerWarp;
+
+int permute_chunk_slots() { return kChunk; }
+
+// Reads the expert of slot i, or -1 past the end / for an invalid index.
+__device__ __forceinline__ int slot_expert(const int32_t* idx, int64_t S, int64_t i, int E, int32_t* status) {
+  if (i >= S) return -1;
+  const int e = __ldg(idx + i);
+  if (e < 0 || e >= E) {
+    raise_status(status, MOE_ERR_DEVICE_FAULT);
+    return -1;
+  }
+  return e;
+}
+
+// Counts of each warp's 256-slot range into cnt[warp][e] (smem).
+__device__ __forceinline__ void warp_counts(const int32_t* idx, int64_t S, int64_t base, int E, int32_t* cnt,
+                                            int32_t* status) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int32_t* my = cnt + warp * E;
+  for (int st = 0; st < kSlotsPerWarp / 32; ++st) {
+    const int64_t i = base + (int64_t)warp * kSlotsPerWarp + st * 32 + lane;
+    const int e = slot_expert(idx, S, i, E, status);
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    const int leader = __ffs(peers) - 1;
+    if (e >= 0 && lane == leader) my[e] += __popc(peers);
+    __syncwarp();
+  }
+}
+
+__global__ void __launch_bounds__(kPermWarps * 32) perm_count_kernel(const int32_t* __restrict__ idx, int64_t S,
+                                                                     int E, int32_t* __restrict__ chunk_counts,
+                                                                     int32_t* status) {
+  extern __shared__ int32_t cnt[];  // [kPermWarps][E]
+  for (int i = threadIdx.x; i < kPermWarps * E; i += blockDim.x) cnt[i] = 0;
+  __syncthreads();
+  const int64_t base = (int64_t)blockIdx.x * kChunk;
+  warp_counts(idx, S, base, E, cnt, status);
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int32_t s = 0;
+#pragma unroll
+    for (int w = 0; w < kPermWarps; ++w) s += cnt[w * E + e];
+    chunk_counts[(int64_t)blockIdx.x * E + e] = s;
+  }
+}
+
+// One block of 1024 threads.  Turns chunk_counts[c][e] into the absolute base
+// position of chunk c's first slot of expert e, and writes offsets[0..E].
+__global__ void __launch_bounds__(1024) perm_scan_kernel(int32_t* __restrict__ chunk_counts, int nchunks, int E,
+                                                         int32_t* __restrict__ offsets) {
+  __shared__ int32_t tot[1024];
+  __shared__ int32_t warp_tot[32];
+  const int e = threadIdx.x;
+  int32_t run = 0;
+  if (e < E) {
+    for (int c = 0; c < nchunks; ++c) {
+      const int32_t v = chunk_counts[(int64_t)c * E + e];
+      chunk_counts[(int64_t)c * E + e] = run;
+      run += v;
+    }
+  }
+  // exclusive scan of the totals over experts
+  const int lane = e & 31, warp = e >> 5;
+  int32_t incl = run;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int32_t n = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += n;
+  }
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int32_t v = warp_tot[lane];
+    int32_t vi = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t n = __shfl_up_sync(0xffffffffu, vi, o);
+      if (lane >= o) vi += n;
+    }
+    warp_tot[lane] = vi - v;
+  }
+  __syncthreads();
+  const int32_t excl = incl - run + warp_tot[warp];
+  tot[e] = excl;
+  if (e < E) offsets[e] = excl;
+  if (e == E - 1) offsets[E] = excl + run;
+  __syncthreads();
+  if (e < E)
+    for (int c = 0; c < nchunks; ++c) chunk_counts[(int64_t)c * E + e] += tot[e];
+}
+
+__global__ void __launch_bounds__(kPermWarps * 32) perm_scatter_kernel(const int32_t* __restrict__ idx, int64_t S,
+                                                                       int k, int E,
+                                                                       const int32_t* __restrict__ chunk_base,
+                                                                       int32_t* __restrict__ perm_token,
+                                                                       int32_t* __restrict__ inv_perm) {
+  extern __shared__ int32_t cnt[];  // [kPermWarps][E]
+  for (int i = threadIdx.x; i < kPermWarps * E; i += blockDim.x) cnt[i] = 0;
+  __syncthreads();
+  const int64_t base = (int64_t)blockIdx.x * kChunk;
+  warp_counts(idx, S, base, E, cnt, nullptr);
+  __syncthreads();
+  // exclusive prefix over warps per expert, offset by the chunk's base
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int32_t run = chunk_base[(int64_t)blockIdx.x * E + e];
+#pragma unroll
+    for (int w = 0; w < kPermWarps; ++w) {
+      const int32_t v = cnt[w * E + e];
+      cnt[w * E + e] = run;
+      run += v;
+    }
+  }
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int32_t* my = cnt + warp * E;
+  for (int st = 0; st < kSlotsPerWarp / 32; ++st) {
+    const int64_t i = base + (int64_t)warp * kSlotsPerWarp + st * 32 + lane;
+    const int e = slot_expert(idx, S, i, E, nullptr);
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    const int leader = __ffs(peers) - 1;
+    if (e >= 0) {
+      const int rank = __popc(peers & ((1u << lane) - 1u));
+      const int32_t p = my[e] + rank;
+      perm_token[p] = (int32_t)(i / k);
+      inv_perm[i] = p;
+    } else if (i < S) {
+      inv_perm[i] = -1;
+    }
+    __syncwarp();
+    if (e >= 0 && lane == leader) my[e] += __popc(peers);
+    __syncwarp();
+  }
+}
+
+cudaError_t launch_permute(const int32_t* idx, int64_t S, int k, int E, int32_t* offsets, int32_t* perm_token,
+                           int32_t* inv_perm, PermuteScratch scratch, int32_t* status, cudaStream_t s) {
+  const int nchunks = (int)((S + kChunk - 1) / kChunk);
+  if (nchunks == 0) {
+    // no slots: offsets are all zero
+    return cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (E + 1), s);
+  }
+  const size_t smem = sizeof(int32_t) * kPermWarps * E;
+  perm_count_kernel<<<nchunks, kPermWarps * 32, smem, s>>>(idx, S, E, scratch.chunk_counts, status);
+  perm_scan_kernel<<<1, 1024, 0, s>>>(scratch.chunk_counts, nchunks, E, offsets);
+  perm_scatter_kernel<<<nchunks, kPermWarps * 32, smem, s>>>(idx, S, k, E, scratch.chunk_counts, perm_token,
+                                                              inv_perm);
+  count_launches(3);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,207 @@
+// Router: logits = x Wr^T (+ b) and top-k with renormalisation.
+//
+// The routed MoE layer picks k experts per token from a learned router (the
+// MoE models the FreeToken upstream README lists under "About"; the router is
+// also what the Domir6/FreeToken fork's "router lookahead" measures, "Changes
+// in this fork").  Selection is on the logits -- softmax is monotone -- with
+// ties to the lower expert index; the k weights are the softmax over all E
+// experts renormalised over the selected k, i.e. exp(L_j - L_0) / sum.
+#include <math.h>
+
+#include "kernels.cuh"
+
+namespace moe {
+
+// ------------------------------------------------------------ logits ------
+// Small T (decode): one warp per (expert, group of up to 8 tokens); lanes
+// stride over H with 16-byte loads of the Wr row and of each token row.
+constexpr int kSmallTGroup = 8;
+
+__global__ void __launch_bounds__(128) router_logits_small_kernel(const uint16_t* __restrict__ x, int64_t T, int H,
+                                                                  const uint16_t* __restrict__ wr,
+                                                                  const float* __restrict__ bias, int E,
+                                                                  float* __restrict__ logits) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int e = blockIdx.x * 4 + warp;
+  const int64_t t0 = (int64_t)blockIdx.y * kSmallTGroup;
+  if (e >= E) return;
+  const int nt = (int)((T - t0) < kSmallTGroup ? (T - t0) : kSmallTGroup);
+  float acc[kSmallTGroup];
+#pragma unroll
+  for (int i = 0; i < kSmallTGroup; ++i) acc[i] = 0.0f;
+  const uint16_t* wrow = wr + (int64_t)e * H;
+  for (int h = lane * 8; h < H; h += 32 * 8) {
+    const uint4 wv = __ldg(reinterpret_cast<const uint4*>(wrow + h));
+    const uint32_t wa[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+    for (int i = 0; i < kSmallTGroup; ++i) {
+      if (i < nt) {
+        const uint4 xv = __ldg(reinterpret_cast<const uint4*>(x + (t0 + i) * H + h));
+        const uint32_t xa[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          acc[i] = fmaf(__uint_as_float(xa[q] << 16), __uint_as_float(wa[q] << 16), acc[i]);
+          acc[i] = fmaf(__uint_as_float(xa[q] & 0xFFFF0000u), __uint_as_float(wa[q] & 0xFFFF0000u), acc[i]);
+        }
+      }
+    }
+  }
+  const float b = bias ? __ldg(bias + e) : 0.0f;
+#pragma unroll
+  for (int i = 0; i < kSmallTGroup; ++i) {
+    float v = warp_sum(acc[i]);
+    if (lane == 0 && i < nt) logits[(t0 + i) * E + e] = v + b;
+  }
+}
+
+// Larger T: 64 tokens x 64 experts per block, K in chunks of 32 staged in
+// shared memory, 4 x 4 outputs per thread on the CUDA cores.
+__global__ void __launch_bounds__(256) router_logits_tiled_kernel(const uint16_t* __restrict__ x, int64_t T, int H,
+                                                                  const uint16_t* __restrict__ wr,
+                                                                  const float* __restrict__ bias, int E,
+                                                                  float* __restrict__ logits) {
+  __shared__ float xs[32][65];
+  __shared__ float ws[32][65];
+  const int tid = threadIdx.x;
+  const int64_t t0 = (int64_t)blockIdx.x * 64;
+  const int e0 = blockIdx.y * 64;
+  const int tr = tid / 16, tc = tid % 16;  // 16 x 16 threads, 4 x 4 each
+  float acc[4][4] = {};
+  for (int h0 = 0; h0 < H; h0 += 32) {
+    // 64 rows x 32 columns of x and of Wr: 2048 values each, 8 per thread
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int idx = tid + i * 256;
+      const int r = idx / 32, c = idx % 32;
+      const int64_t t = t0 + r;
+      const int e = e0 + r;
+      const bool hin = h0 + c < H;
+      xs[c][r] = (t < T && hin) ? bf16_to_f32(__ldg(x + t * H + h0 + c)) : 0.0f;
+      ws[c][r] = (e < E && hin) ? bf16_to_f32(__ldg(wr + (int64_t)e * H + h0 + c)) : 0.0f;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int c = 0; c < 32; ++c) {
+      float a[4], b[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        a[i] = xs[c][tr * 4 + i];
+        b[i] = ws[c][tc * 4 + i];
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int64_t t = t0 + tr * 4 + i;
+    if (t >= T) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int e = e0 + tc * 4 + j;
+      if (e < E) logits[t * E + e] = acc[i][j] + (bias ? __ldg(bias + e) : 0.0f);
+    }
+  }
+}
+
+cudaError_t launch_router_logits(const uint16_t* x, int64_t T, int H, const uint16_t* wr, const float* bias, int E,
+                                 float* logits, cudaStream_t s) {
+  if (T == 0) return cudaSuccess;
+  if (T <= 64 && H % 8 == 0) {
+    dim3 grid((E + 3) / 4, (unsigned)((T + kSmallTGroup - 1) / kSmallTGroup));
+    router_logits_small_kernel<<<grid, 128, 0, s>>>(x, T, H, wr, bias, E, logits);
+  } else {
+    dim3 grid((unsigned)((T + 63) / 64), (E + 63) / 64);
+    router_logits_tiled_kernel<<<grid, 256, 0, s>>>(x, T, H, wr, bias, E, logits);
+  }
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+// -------------------------------------------------------------- top-k -----
+// One warp per token; lane l holds logits l, l+32, ... in registers.  Each
+// round picks the largest not-yet-taken logit (ties -> lower index) with a
+// warp arg-max; lane 0 writes the index and exp(L - L_0); a final pass divides
+// by the sum.  A NaN, or a row without a finite logit, raises the status word
+// and writes indices 0..k-1 with zero weights.
+template <int J>
+__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, int64_t T, int E, int k,
+                                                   int32_t* __restrict__ idx, float* __restrict__ w,
+                                                   int32_t* status) {
+  const int lane = threadIdx.x & 31;
+  const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= T) return;
+  const float* L = logits + t * E;
+  float v[J];
+  bool bad = false;
+#pragma unroll
+  for (int j = 0; j < J; ++j) {
+    const int e = lane + 32 * j;
+    v[j] = e < E ? __ldg(L + e) : -INFINITY;
+    if (e < E && isnan(v[j])) bad = true;
+  }
+  uint32_t taken = 0u;
+#pragma unroll
+  for (int j = 0; j < J; ++j)
+    if (lane + 32 * j >= E) taken |= 1u << j;
+  float top = 0.0f, sum = 0.0f;
+  bad = __any_sync(0xffffffffu, bad);
+  for (int r = 0; r < k; ++r) {
+    float bv = -INFINITY;
+    int be = 0x7fffffff;
+#pragma unroll
+    for (int j = 0; j < J; ++j) {
+      const int e = lane + 32 * j;
+      if (!(taken & (1u << j)) && (v[j] > bv || (v[j] == bv && e < be))) {
+        bv = v[j];
+        be = e;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+      if (ov > bv || (ov == bv && oe < be)) {
+        bv = ov;
+        be = oe;
+      }
+    }
+    if (be != 0x7fffffff && (be & 31) == lane) taken |= 1u << (be >> 5);
+    if (r == 0) {
+      top = bv;
+      if (!(top > -INFINITY)) bad = true;
+    }
+    const float ex = expf(bv - top);
+    sum += ex;
+    if (lane == 0) {
+      idx[t * k + r] = bad ? r : be;
+      w[t * k + r] = bad ? 0.0f : ex;
+    }
+  }
+  __syncwarp();
+  if (bad) {
+    if (lane == 0) raise_status(status, MOE_ERR_DEVICE_FAULT);
+    return;
+  }
+  for (int r = lane; r < k; r += 32) w[t * k + r] = __fdiv_rn(w[t * k + r], sum);
+}
+
+cudaError_t launch_topk(const float* logits, int64_t T, int E, int k, int32_t* idx, float* w, int32_t* status,
+                        cudaStream_t s) {
+  if (T == 0) return cudaSuccess;
+  const unsigned grid = (unsigned)((T + 7) / 8);
+  const int J = (E + 31) / 32;
+  if (J <= 1) topk_kernel<1><<<grid, 256, 0, s>>>(logits, T, E, k, idx, w, status);
+  else if (J <= 2) topk_kernel<2><<<grid, 256, 0, s>>>(logits, T, E, k, idx, w, status);
+  else if (J <= 4) topk_kernel<4><<<grid, 256, 0, s>>>(logits, T, E, k, idx, w, status);
+  else if (J <= 8) topk_kernel<8><<<grid, 256, 0, s>>>(logits, T, E, k, idx, w, status);
+  else if (J <= 16) topk_kernel<16><<<grid, 256, 0, s>>>(logits, T, E, k, idx, w, status);
+  else topk_kernel<32><<<grid, 256, 0, s>>>(logits, T, E, k, idx, w, status);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,339 @@
+"""Thin ctypes binding of ``libmoe_b200.so`` (C ABI in include/moe_b200.h).
+
+Argument marshalling only: every function passes raw device pointers, sizes
+and torch's current CUDA stream to the library entry point of the same name
+and raises ``MoeError`` on a non-OK status.  There is no CPU fallback: if the
+library is missing or no CUDA device is present, the call fails.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass, field, replace
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmoe_b200.so")
+
+MOE_OK = 0
+FMT_NVFP4, FMT_MXFP4, FMT_FP8 = 1, 2, 3
+ACT_BF16, ACT_MATCH = 0, 1
+LAYOUT_CANONICAL, LAYOUT_PREPARED = 0, 1
+OPT_FFN_PATH = 1
+FMT_BY_NAME = {"nvfp4": FMT_NVFP4, "mxfp4": FMT_MXFP4, "fp8": FMT_FP8}
+
+EXPORTED = (
+    "moe_status_string", "moe_version", "moe_set_option", "moe_workspace_size", "moe_prepared_weights_size",
+    "moe_prepare_weights", "moe_quantize", "moe_route", "moe_route_logits", "moe_permute", "moe_grouped_ffn",
+    "moe_combine", "moe_forward", "moe_get_device_status", "moe_set_stage_events", "moe_kernel_launch_count",
+)
+STAGES = ("route", "permute", "act_quant", "ffn_up", "ffn_down", "shared", "combine")
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {status_string(status)}")
+        self.status = status
+
+
+class MoeWeightsC(ctypes.Structure):
+    _fields_ = [
+        ("fmt", ctypes.c_int32), ("E", ctypes.c_int32), ("H", ctypes.c_int32), ("I", ctypes.c_int32),
+        ("layout", ctypes.c_int32),
+        ("w13", ctypes.c_void_p), ("w13_sf", ctypes.c_void_p), ("w13_gs", ctypes.c_void_p),
+        ("w2", ctypes.c_void_p), ("w2_sf", ctypes.c_void_p), ("w2_gs", ctypes.c_void_p),
+        ("a13_gs", ctypes.c_void_p), ("a2_gs", ctypes.c_void_p),
+    ]
+
+
+_lib = None
+
+
+def lib():
+    """Load the library (raises if it was not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m quantized_expert_ffn_top_b200.build` "
+                               "(the layer has no CPU fallback)")
+        L = ctypes.CDLL(LIB_PATH)
+        _declare(L)
+        _lib = L
+    return _lib
+
+
+def _declare(L):
+    P, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+    W = ctypes.POINTER(MoeWeightsC)
+    sig = {
+        "moe_status_string": ([ctypes.c_int], ctypes.c_char_p),
+        "moe_version": ([], i32),
+        "moe_set_option": ([i32, i32], ctypes.c_int),
+        "moe_workspace_size": ([i64, i32, W, W, i32], sz),
+        "moe_prepared_weights_size": ([W], sz),
+        "moe_prepare_weights": ([W, P, sz, W, P], ctypes.c_int),
+        "moe_quantize": ([i32, P, i32, i64, i64, P, P, P, P, P, sz, P], ctypes.c_int),
+        "moe_route": ([P, i64, i32, P, P, i32, i32, P, P, P, P, sz, P], ctypes.c_int),
+        "moe_route_logits": ([P, i64, i32, i32, P, P, P, sz, P], ctypes.c_int),
+        "moe_permute": ([P, i64, i32, i32, P, P, P, P, sz, P], ctypes.c_int),
+        "moe_grouped_ffn": ([P, i64, i32, P, P, W, i32, P, P, sz, P], ctypes.c_int),
+        "moe_combine": ([P, P, P, i64, i32, i32, P, P, P, sz, P], ctypes.c_int),
+        "moe_forward": ([P, i64, P, P, i32, W, W, i32, P, P, sz, P], ctypes.c_int),
+        "moe_get_device_status": ([P, P, ctypes.POINTER(ctypes.c_int32)], ctypes.c_int),
+        "moe_set_stage_events": ([ctypes.POINTER(ctypes.c_void_p), i32], ctypes.c_int),
+        "moe_kernel_launch_count": ([], ctypes.c_uint64),
+    }
+    for name, (args, res) in sig.items():
+        f = getattr(L, name)
+        f.argtypes = args
+        f.restype = res
+
+
+def status_string(st: int) -> str:
+    return lib().moe_status_string(int(st)).decode()
+
+
+def _check(st: int, where: str):
+    if st != MOE_OK:
+        raise MoeError(st, where)
+
+
+def _p(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("device tensor expected")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+# ------------------------------------------------------------ weight bank --
+@dataclass
+class WeightBank:
+    """Device tensors of one expert bank (see moe_weights in the header)."""
+    fmt: int
+    E: int
+    H: int
+    I: int
+    w13: torch.Tensor
+    w13_sf: torch.Tensor | None
+    w13_gs: torch.Tensor | None
+    w2: torch.Tensor
+    w2_sf: torch.Tensor | None
+    w2_gs: torch.Tensor | None
+    a13_gs: torch.Tensor | None = None
+    a2_gs: torch.Tensor | None = None
+    layout: int = LAYOUT_CANONICAL
+    keep: list = field(default_factory=list)   # owners of memory the pointers reference
+
+    def struct(self) -> MoeWeightsC:
+        v = lambda t: None if t is None else t.data_ptr()
+        return MoeWeightsC(self.fmt, self.E, self.H, self.I, self.layout, v(self.w13), v(self.w13_sf),
+                           v(self.w13_gs), v(self.w2), v(self.w2_sf), v(self.w2_gs), v(self.a13_gs), v(self.a2_gs))
+
+    def nbytes(self) -> int:
+        return sum(t.numel() * t.element_size() for t in (self.w13, self.w13_sf, self.w2, self.w2_sf) if t is not None)
+
+
+def _ref(b: WeightBank | None):
+    return None if b is None else ctypes.byref(b.struct())
+
+
+def workspace_size(T: int, k: int, routed: WeightBank, shared: WeightBank | None = None, act: int = ACT_MATCH) -> int:
+    r = routed.struct()
+    s = shared.struct() if shared is not None else None
+    n = lib().moe_workspace_size(int(T), int(k), ctypes.byref(r), ctypes.byref(s) if s is not None else None,
+                                 int(act))
+    if n == 0:
+        raise MoeError(1, "moe_workspace_size")
+    return int(n)
+
+
+def new_workspace(nbytes: int, device=None) -> torch.Tensor:
+    """A zeroed workspace (the status word must start at zero)."""
+    return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device or "cuda")
+
+
+def moe_prepare_weights(bank: WeightBank, stream=None) -> WeightBank:
+    c = bank.struct()
+    n = lib().moe_prepared_weights_size(ctypes.byref(c))
+    if n == 0:
+        raise MoeError(2, "moe_prepared_weights_size")
+    dst = torch.empty(int(n), dtype=torch.uint8, device=bank.w13.device)
+    out = MoeWeightsC()
+    _check(lib().moe_prepare_weights(ctypes.byref(c), _p(dst), n, ctypes.byref(out), _stream(stream)),
+           "moe_prepare_weights")
+
+    def view(ptr, numel):
+        if not ptr:
+            return None
+        off = ptr - dst.data_ptr()
+        return dst[off:off + numel]
+
+    rb13 = bank.H if bank.fmt == FMT_FP8 else bank.H // 2
+    rb2 = bank.I if bank.fmt == FMT_FP8 else bank.I // 2
+    bs = {FMT_NVFP4: 16, FMT_MXFP4: 32}.get(bank.fmt, 0)
+    return replace(bank, layout=LAYOUT_PREPARED,
+                   w13=view(out.w13, bank.E * 2 * bank.I * rb13),
+                   w2=view(out.w2, bank.E * bank.H * rb2),
+                   w13_sf=view(out.w13_sf, bank.E * 2 * bank.I * bank.H // bs) if bs else None,
+                   w2_sf=view(out.w2_sf, bank.E * bank.H * bank.I // bs) if bs else None,
+                   keep=[dst, bank])
+
+
+# ------------------------------------------------------------ entry points --
+def moe_quantize(fmt: int, x: torch.Tensor, scale_in: torch.Tensor | None = None, ws: torch.Tensor | None = None,
+                 stream=None):
+    """x: [rows][K] fp32 or bf16 (device).  Returns (codes, sf, scale_used)."""
+    rows, K = x.shape
+    dt = {torch.float32: 0, torch.bfloat16: 1}[x.dtype]
+    cb = K if fmt == FMT_FP8 else K // 2
+    codes = torch.empty((rows, cb), dtype=torch.uint8, device=x.device)
+    bs = {FMT_NVFP4: 16, FMT_MXFP4: 32}.get(fmt, 0)
+    sf = torch.empty((rows, K // bs), dtype=torch.uint8, device=x.device) if bs else None
+    scale_out = torch.ones(1, dtype=torch.float32, device=x.device)
+    ws = ws if ws is not None else new_workspace(4096, x.device)
+    _check(lib().moe_quantize(fmt, _p(x.contiguous()), dt, rows, K, _p(scale_in), _p(codes), _p(sf), _p(scale_out),
+                              _p(ws), ws.numel(), _stream(stream)), "moe_quantize")
+    return codes, sf, scale_out
+
+
+def moe_route(x: torch.Tensor, wr: torch.Tensor, bias: torch.Tensor | None, k: int, ws: torch.Tensor,
+              logits: torch.Tensor | None = None, stream=None):
+    """x [T][H] bf16, wr [E][H] bf16 -> (topk_idx int32 [T][k], topk_w fp32 [T][k])."""
+    T, H = x.shape
+    E = wr.shape[0]
+    idx = torch.empty((T, k), dtype=torch.int32, device=x.device)
+    w = torch.empty((T, k), dtype=torch.float32, device=x.device)
+    _check(lib().moe_route(_p(x), T, H, _p(wr), _p(bias), E, k, _p(logits), _p(idx), _p(w), _p(ws), ws.numel(),
+                           _stream(stream)), "moe_route")
+    return idx, w
+
+
+def moe_route_logits(logits: torch.Tensor, k: int, ws: torch.Tensor, stream=None):
+    T, E = logits.shape
+    idx = torch.empty((T, k), dtype=torch.int32, device=logits.device)
+    w = torch.empty((T, k), dtype=torch.float32, device=logits.device)
+    _check(lib().moe_route_logits(_p(logits), T, E, k, _p(idx), _p(w), _p(ws), ws.numel(), _stream(stream)),
+           "moe_route_logits")
+    return idx, w
+
+
+def moe_permute(topk_idx: torch.Tensor, E: int, ws: torch.Tensor, stream=None):
+    T, k = topk_idx.shape
+    S = T * k
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=topk_idx.device)
+    perm = torch.empty(S, dtype=torch.int32, device=topk_idx.device)
+    inv = torch.empty(S, dtype=torch.int32, device=topk_idx.device)
+    _check(lib().moe_permute(_p(topk_idx), T, k, E, _p(offsets), _p(perm), _p(inv), _p(ws), ws.numel(),
+                             _stream(stream)), "moe_permute")
+    return offsets, perm, inv
+
+
+def moe_grouped_ffn(x: torch.Tensor, k: int, perm_token: torch.Tensor, offsets: torch.Tensor, w: WeightBank,
+                    act: int, ws: torch.Tensor, y_perm: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    T, H = x.shape
+    y = y_perm if y_perm is not None else torch.empty((T * k, H), dtype=torch.bfloat16, device=x.device)
+    ws_ = w.struct()
+    _check(lib().moe_grouped_ffn(_p(x), T, k, _p(perm_token), _p(offsets), ctypes.byref(ws_), act, _p(y), _p(ws),
+                                 ws.numel(), _stream(stream)), "moe_grouped_ffn")
+    return y
+
+
+def moe_combine(y_perm: torch.Tensor, inv_perm: torch.Tensor, topk_w: torch.Tensor, ws: torch.Tensor,
+                shared_y: torch.Tensor | None = None, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    T, k = topk_w.shape
+    H = y_perm.shape[1]
+    o = out if out is not None else torch.empty((T, H), dtype=torch.bfloat16, device=y_perm.device)
+    _check(lib().moe_combine(_p(y_perm), _p(inv_perm), _p(topk_w), T, k, H, _p(shared_y), _p(o), _p(ws),
+                             ws.numel(), _stream(stream)), "moe_combine")
+    return o
+
+
+def moe_forward(x: torch.Tensor, wr: torch.Tensor, bias: torch.Tensor | None, k: int, routed: WeightBank,
+                shared: WeightBank | None, act: int, ws: torch.Tensor, out: torch.Tensor | None = None,
+                stream=None) -> torch.Tensor:
+    T, H = x.shape
+    o = out if out is not None else torch.empty((T, H), dtype=torch.bfloat16, device=x.device)
+    r = routed.struct()
+    s = shared.struct() if shared is not None else None
+    _check(lib().moe_forward(_p(x), T, _p(wr), _p(bias), k, ctypes.byref(r),
+                             ctypes.byref(s) if s is not None else None, act, _p(o), _p(ws), ws.numel(),
+                             _stream(stream)), "moe_forward")
+    return o
+
+
+def moe_get_device_status(ws: torch.Tensor, stream=None) -> int:
+    v = ctypes.c_int32(0)
+    _check(lib().moe_get_device_status(_p(ws), _stream(stream), ctypes.byref(v)), "moe_get_device_status")
+    return int(v.value)
+
+
+def moe_set_option(option: int, value: int):
+    _check(lib().moe_set_option(int(option), int(value)), "moe_set_option")
+
+
+# ----------------------------------------------------- device-side banks --
+def quantize_bank(fmt: int, w13: torch.Tensor, w2: torch.Tensor, ws: torch.Tensor | None = None) -> WeightBank:
+    """fp32 expert weights on the device -> CANONICAL bank, quantised by the
+    library (one amax-derived scale per part for NVFP4 / FP8).
+    w13 [E][2I][H] (gate rows first), w2 [E][H][I]."""
+    E, twoI, H = w13.shape
+    I = twoI // 2
+    dev = w13.device
+    bs = {FMT_NVFP4: 16, FMT_MXFP4: 32}.get(fmt, 0)
+    cb13 = H if fmt == FMT_FP8 else H // 2
+    cb2 = I if fmt == FMT_FP8 else I // 2
+    c13 = torch.empty((E, twoI, cb13), dtype=torch.uint8, device=dev)
+    c2 = torch.empty((E, H, cb2), dtype=torch.uint8, device=dev)
+    s13 = torch.empty((E, twoI, H // bs), dtype=torch.uint8, device=dev) if bs else None
+    s2 = torch.empty((E, H, I // bs), dtype=torch.uint8, device=dev) if bs else None
+    g13 = torch.ones((E, 2), dtype=torch.float32, device=dev) if fmt != FMT_MXFP4 else None
+    g2 = torch.ones(E, dtype=torch.float32, device=dev) if fmt != FMT_MXFP4 else None
+    ws = ws if ws is not None else new_workspace(4096, dev)
+    L = lib()
+    st = _stream()
+    for e in range(E):
+        parts = [(w13[e, :I], c13[e, :I], None if s13 is None else s13[e, :I], None if g13 is None else g13[e, 0:1]),
+                 (w13[e, I:], c13[e, I:], None if s13 is None else s13[e, I:], None if g13 is None else g13[e, 1:2]),
+                 (w2[e], c2[e], None if s2 is None else s2[e], None if g2 is None else g2[e:e + 1])]
+        for src, codes, sf, gs in parts:
+            rows, K = src.shape
+            _check(L.moe_quantize(fmt, _p(src), 0, rows, K, None, _p(codes), _p(sf), _p(gs), _p(ws), ws.numel(),
+                                  st), "moe_quantize")
+    return WeightBank(fmt, E, H, I, c13, s13, g13, c2, s2, g2)
+
+
+def bank_from_host(fmt: int, E: int, H: int, I: int, w13, w13_sf, w13_gs, w2, w2_sf, w2_gs, a13_gs=None,
+                   a2_gs=None, device="cuda") -> WeightBank:
+    """A CANONICAL bank from host arrays (numpy or torch); scalars as floats."""
+    def dev(a, dtype):
+        if a is None:
+            return None
+        t = torch.as_tensor(a)
+        return t.to(device=device, dtype=dtype).contiguous()
+
+    def scal(v):
+        return None if v is None else torch.tensor([float(v)], dtype=torch.float32, device=device)
+
+    return WeightBank(fmt, E, H, I, dev(w13, torch.uint8), dev(w13_sf, torch.uint8), dev(w13_gs, torch.float32),
+                      dev(w2, torch.uint8), dev(w2_sf, torch.uint8), dev(w2_gs, torch.float32), scal(a13_gs),
+                      scal(a2_gs))
+
+
+def moe_set_stage_events(events):
+    """events: list of 2 * len(STAGES) torch.cuda.Event(enable_timing=True), or None."""
+    if events is None:
+        _check(lib().moe_set_stage_events(None, 0), "moe_set_stage_events")
+        return
+    arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    _check(lib().moe_set_stage_events(arr, len(events)), "moe_set_stage_events")
+
+
+def moe_kernel_launch_count() -> int:
+    return int(lib().moe_kernel_launch_count())

@@ -1,0 +1,84 @@
+"""The C-ABI library without a GPU: it loads, exports every function the
+headers declare, and rejects bad arguments on the host before touching the
+device.  (No compute call runs here.)"""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+from quantized_expert_ffn_top_b200 import build, ops
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return ops.lib()
+
+
+def _declared():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(h).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        for m in re.finditer(r"\b(moe_[a-z0-9_]+)\s*\(", src):
+            names.add(m.group(1))
+    return names
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = _declared()
+    assert {"moe_route", "moe_permute", "moe_grouped_ffn", "moe_combine", "moe_forward"} <= names
+    for n in names:
+        assert hasattr(L, n), n
+    assert names == set(ops.EXPORTED)
+
+
+def test_status_strings_and_version(L):
+    for s in range(7):
+        assert ops.status_string(s).startswith("MOE_")
+    assert L.moe_version() >= 100
+
+
+def _bank(fmt=1, E=8, H=128, I=256, layout=0, ptr=256):
+    return ops.MoeWeightsC(fmt, E, H, I, layout, ptr, ptr, ptr, ptr, ptr, ptr, None, None)
+
+
+def test_workspace_and_prepared_sizes(L):
+    b = _bank()
+    n = L.moe_workspace_size(8, 2, ctypes.byref(b), None, 1)
+    assert n > 0 and n % 256 == 0
+    assert L.moe_workspace_size(4096, 8, ctypes.byref(_bank(E=128, H=2048, I=768)), None, 1) > n
+    assert L.moe_workspace_size(8, 2, ctypes.byref(_bank(fmt=7)), None, 1) == 0
+    assert L.moe_workspace_size(8, 2, ctypes.byref(_bank(H=100)), None, 1) == 0
+    p = L.moe_prepared_weights_size(ctypes.byref(b))
+    # w13 8*512*64 + w2 8*128*128 + sf13 8*512*8 + sf2 8*128*16 bytes, 256-aligned pieces
+    assert p >= 8 * 512 * 64 + 8 * 128 * 128 + 8 * 512 * 8 + 8 * 128 * 16
+
+
+def test_host_side_argument_errors(L):
+    P = ctypes.c_void_p
+    one = P(256)
+    # k > E
+    assert L.moe_route(one, 4, 128, one, None, 8, 9, None, one, one, one, 1 << 20, None) == ops.MoeError(1, "").status
+    assert L.moe_route_logits(one, 4, 8, 0, one, one, one, 1 << 20, None) == 1
+    # workspace too small
+    assert L.moe_route_logits(one, 4, 8, 2, one, one, one, 16, None) == 3
+    # unknown format / canonical bank where a prepared one is required
+    b = _bank(fmt=9)
+    assert L.moe_grouped_ffn(one, 4, 2, one, one, ctypes.byref(b), 1, one, one, 1 << 20, None) == 2
+    c = _bank(layout=0)
+    assert L.moe_forward(one, 4, one, None, 2, ctypes.byref(c), None, 1, one, one, 1 << 30, None) == 2
+    # shape not a multiple of 128
+    d = _bank(H=96, layout=1)
+    assert L.moe_forward(one, 4, one, None, 2, ctypes.byref(d), None, 1, one, one, 1 << 30, None) == 2
+    # quantize: K not a multiple of the block, unknown format
+    assert L.moe_quantize(1, one, 0, 2, 24, None, one, one, None, one, 1 << 20, None) == 2
+    assert L.moe_quantize(4, one, 0, 2, 32, None, one, one, None, one, 1 << 20, None) == 2
+    # permute: E out of range
+    assert L.moe_permute(one, 4, 2, 2000, one, one, one, one, 1 << 20, None) == 1
+    assert L.moe_set_option(1, 5) == 1 and L.moe_set_option(99, 0) == 1
+    assert L.moe_set_option(1, 0) == 0

@@ -1,0 +1,258 @@
+"""CUDA path against the oracle, through the C ABI, on seeded inputs.
+
+Integer and byte results (quantised codes and scales, routing indices,
+offsets and permutations) must match bit for bit; floating-point outputs must
+be within the layer's max-abs-relative bound of 2e-2 of the fp64 oracle.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from quantized_expert_ffn_top_b200 import ops, synth
+from tests.gpu_helpers import (TOL, ambiguous_tokens, bits_to_dev_bf16, dev_to_f64, device_bank, max_abs_rel,
+                               oracle_bank, routed_inputs)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    assert torch.cuda.is_available(), "the GPU tests need a CUDA device"
+    ops.lib()
+    ops.moe_set_option(ops.OPT_FFN_PATH, 0)
+    yield
+    ops.moe_set_option(ops.OPT_FFN_PATH, 0)
+
+
+def ws(nbytes=1 << 24):
+    return ops.new_workspace(nbytes)
+
+
+# ----------------------------------------------------------- quantisers ----
+def _all_finite_bf16_as_f32(limit=None):
+    bits = np.arange(1 << 16, dtype=np.uint32)
+    f = (bits << 16).view(np.float32)
+    f = f[np.isfinite(f)]
+    if limit is not None:
+        f = f[np.abs(f) < limit]
+    return f
+
+
+def test_e4m3_conversion_matches_oracle_on_every_bf16():
+    f = _all_finite_bf16_as_f32()
+    n = (f.size // 16) * 16
+    x = torch.from_numpy(f[:n].reshape(-1, 16)).cuda()
+    codes, _, _ = ops.moe_quantize(ops.FMT_FP8, x, scale_in=torch.ones(1, device="cuda"))
+    got = codes.cpu().numpy().reshape(-1)
+    ref = np.array([oracle.e4m3_encode(float(v)) for v in f[:n]], np.uint8)
+    bad = np.nonzero(got != ref)[0]
+    assert bad.size == 0, f"{bad.size} mismatches, first: {f[bad[:5]]} got {got[bad[:5]]} ref {ref[bad[:5]]}"
+
+
+def test_e2m1_conversion_matches_oracle_on_every_bf16_below_8():
+    # blocks of 32 led by 4.0 have MXFP4 scale 2^0, so every element goes
+    # through e2m1 rounding with multiplier 1
+    f = _all_finite_bf16_as_f32(limit=8.0)
+    per = 31
+    nb = f.size // per
+    blocks = np.zeros((nb, 32), np.float32)
+    blocks[:, 0] = 4.0
+    blocks[:, 1:] = f[:nb * per].reshape(nb, per)
+    x = torch.from_numpy(blocks).cuda()
+    codes, sf, _ = ops.moe_quantize(ops.FMT_MXFP4, x)
+    assert np.all(sf.cpu().numpy() == 127)
+    c = codes.cpu().numpy()
+    nib = np.empty((nb, 32), np.uint8)
+    nib[:, 0::2] = c & 15
+    nib[:, 1::2] = c >> 4
+    ref = np.array([oracle.e2m1_encode(float(v)) for v in blocks[:, 1:].reshape(-1)], np.uint8).reshape(nb, per)
+    bad = np.nonzero(nib[:, 1:] != ref)
+    assert bad[0].size == 0, f"{bad[0].size} mismatches: {blocks[:, 1:][bad][:5]} got {nib[:, 1:][bad][:5]}"
+
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "mxfp4", "fp8"])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("static", [False, True])
+def test_quantize_matches_oracle(fmt, dtype, static):
+    rng = np.random.default_rng(11)
+    rows, K = 96, 512
+    xf = (rng.standard_normal((rows, K)) * rng.uniform(1e-3, 30, (rows, 1))).astype(np.float32)
+    xf[7, 64:96] = 0.0
+    xf[9, :] = 0.0
+    if dtype == "bf16":
+        bits = synth.to_bf16_bits(xf)
+        xf = (bits.astype(np.uint32) << 16).view(np.float32)
+        xd = bits_to_dev_bf16(bits)
+    else:
+        xd = torch.from_numpy(xf).cuda()
+    f = {"nvfp4": 1, "mxfp4": 2, "fp8": 3}[fmt]
+    scale = 0.0123 if static else None
+    sd = torch.tensor([scale], dtype=torch.float32, device="cuda") if static else None
+    codes, sf, s_used = ops.moe_quantize(f, xd, scale_in=sd)
+    if f == 1:
+        g = scale if static else oracle.nvfp4_global_scale(oracle.amax(xf))
+        rc, rs = oracle.quant_nvfp4(xf, g)
+    elif f == 2:
+        g = 1.0
+        rc, rs = oracle.quant_mxfp4(xf)
+    else:
+        g = scale if static else oracle.fp8_scale(oracle.amax(xf))
+        rc, rs = oracle.quant_fp8(xf, g), None
+    assert np.array_equal(codes.cpu().numpy(), rc)
+    if rs is not None:
+        assert np.array_equal(sf.cpu().numpy(), rs)
+    if f != 2:
+        assert float(s_used.item()) == np.float32(g)
+
+
+# --------------------------------------------------------------- routing ----
+@pytest.mark.parametrize("T,E,k", [(1, 8, 2), (37, 128, 8), (300, 256, 8), (5, 1024, 16), (9, 7, 7), (64, 40, 1)])
+def test_route_logits_bit_exact(T, E, k):
+    L = synth.random_logits(T, E, kind="uniform" if E != 40 else "normal")
+    L[0, :] = L[0, 0]  # a row of equal logits
+    idx, w = ops.moe_route_logits(torch.from_numpy(L).cuda(), k, ws())
+    ridx, rw, st = oracle.topk(L.astype(np.float64), k)
+    assert st == 0
+    assert np.array_equal(idx.cpu().numpy(), ridx)
+    assert np.allclose(w.cpu().numpy(), rw, rtol=2e-6, atol=1e-7)
+
+
+def test_route_logits_flags_invalid_rows():
+    L = np.zeros((4, 16), np.float32)
+    L[1, 3] = np.nan
+    L[2, :] = -np.inf
+    L[3, 5] = -np.inf
+    W = ws()
+    idx, w = ops.moe_route_logits(torch.from_numpy(L).cuda(), 4, W)
+    assert ops.moe_get_device_status(W) == ops.MoeError(5, "").status
+    assert ops.moe_get_device_status(W) == 0  # cleared
+    wn = w.cpu().numpy()
+    assert np.all(wn[1] == 0) and np.all(wn[2] == 0)
+    assert np.allclose(wn[3], 0.25)
+
+
+@pytest.mark.parametrize("name", ["tiny", "decode", "prefill"])
+def test_route_matches_oracle(name):
+    w = synth.workload(name)
+    x, wr, b = routed_inputs(w)
+    logits = torch.empty((w.T, w.E), dtype=torch.float32, device="cuda")
+    idx, wt = ops.moe_route(bits_to_dev_bf16(x), bits_to_dev_bf16(wr),
+                            None if b is None else torch.from_numpy(b).cuda(), w.k, ws(), logits=logits)
+    RL = oracle.router_logits(x, wr, b)
+    gl = logits.cpu().numpy().astype(np.float64)
+    assert max_abs_rel(gl, RL) < 1e-5
+    ridx, rw, _ = oracle.topk(RL, w.k)
+    amb = ambiguous_tokens(RL, w.k, 1e-4)
+    assert amb.mean() < 0.05
+    gi = idx.cpu().numpy()
+    assert np.array_equal(gi[~amb], ridx[~amb])
+    assert np.allclose(wt.cpu().numpy()[~amb], rw[~amb], rtol=1e-4, atol=1e-6)
+    # ambiguous tokens: still k distinct experts, ordered by the GPU's logits
+    for t in np.nonzero(amb)[0]:
+        assert len(set(gi[t])) == w.k
+        assert np.all(np.diff(gl[t, gi[t]]) <= 0)
+
+
+# ----------------------------------------------------------- permutation ----
+@pytest.mark.parametrize("T,k,E,skew", [(8, 2, 8, 0.0), (4, 8, 128, 0.0), (4096, 8, 128, 1.1), (16384, 8, 256, 1.1),
+                                        (777, 1, 1, 0.0), (50, 16, 1024, 0.3), (3000, 5, 37, 2.0)])
+def test_permute_bit_exact(T, k, E, skew):
+    if k > E:
+        pytest.skip("k > E")
+    idx = synth.random_topk_idx(T, k, E, skew=skew) if E > 1 else np.zeros((T, k), np.int32)
+    off, perm, inv = ops.moe_permute(torch.from_numpy(idx).cuda(), E, ws(1 << 26))
+    roff, rperm, rinv, st = oracle.permute(idx, E)
+    assert st == 0
+    assert np.array_equal(off.cpu().numpy(), roff)
+    assert np.array_equal(perm.cpu().numpy(), rperm)
+    assert np.array_equal(inv.cpu().numpy(), rinv)
+
+
+def test_permute_empty_and_bad_index():
+    W = ws()
+    off, _, _ = ops.moe_permute(torch.zeros((0, 4), dtype=torch.int32, device="cuda"), 6, W)
+    assert not off.cpu().numpy().any()
+    idx = np.array([[0, 1], [2, 9]], np.int32)
+    off, perm, inv = ops.moe_permute(torch.from_numpy(idx).cuda(), 4, W)
+    assert ops.moe_get_device_status(W) == 5
+    assert inv.cpu().numpy()[3] == -1
+    assert off.cpu().numpy()[-1] == 3
+
+
+# ------------------------------------------------------------ grouped FFN ----
+FFN_CASES = [
+    ("tiny", {}, 0), ("tiny", {}, 1), ("tiny", {}, 2),
+    ("decode", {}, 0), ("decode", {}, 1),
+    ("tiny", dict(fmt="mxfp4", H=256, I=256, E=4, k=2, T=6), 0),
+    ("tiny", dict(fmt="mxfp4", H=256, I=256, E=4, k=2, T=6), 1),
+    ("tiny", dict(fmt="fp8", H=256, I=128, E=8, k=2, T=10), 0),
+    ("tiny", dict(fmt="fp8", H=256, I=128, E=8, k=2, T=10), 1),
+    ("tiny", dict(T=40, E=4, k=2, H=128, I=128), 1),       # > 8 tokens per expert
+]
+
+
+@pytest.mark.parametrize("name,over,mode", FFN_CASES)
+def test_grouped_ffn_matches_oracle(name, over, mode):
+    """mode 0 = BF16 activations, 1 = MATCH dynamic scales, 2 = MATCH static."""
+    w = synth.workload(name, **over)
+    W, _ = oracle_bank(w)
+    a13, a2 = synth.static_act_scales() if mode == 2 else (None, None)
+    bank = device_bank(W, a13, a2)
+    idx = synth.random_topk_idx(w.T, w.k, w.E, skew=0.5)
+    off, perm, inv, _ = oracle.permute(idx, w.E)
+    x = synth.x_bits(w)
+    act = 0 if mode == 0 else 1
+    y = ops.moe_grouped_ffn(bits_to_dev_bf16(x), w.k, torch.from_numpy(perm).cuda(), torch.from_numpy(off).cuda(),
+                            bank, act, ws(ops.workspace_size(w.T, w.k, bank, None, act)))
+    ry, _ = oracle.grouped_ffn(x, perm, off, W, act, a13 or 0.0, a2 or 0.0)
+    err = max_abs_rel(dev_to_f64(y), ry)
+    assert err < TOL, err
+
+
+def test_combine_matches_oracle():
+    T, k, H = 33, 4, 256
+    rng = np.random.default_rng(12)
+    S = T * k
+    y = synth.to_bf16_bits(rng.standard_normal((S, H)).astype(np.float32))
+    sh = synth.to_bf16_bits(rng.standard_normal((T, H)).astype(np.float32))
+    inv = rng.permutation(S).astype(np.int32)
+    w = rng.dirichlet(np.ones(k), size=T).astype(np.float32)
+    W = ws()
+    out = ops.moe_combine(bits_to_dev_bf16(y), torch.from_numpy(inv).cuda(), torch.from_numpy(w).cuda(), W,
+                          shared_y=bits_to_dev_bf16(sh))
+    yf = (y.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    shf = (sh.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    ref = oracle.combine(yf, inv, w.astype(np.float64), k, shf)
+    got = dev_to_f64(out)
+    # one bf16 rounding of the fp32 sum
+    assert np.all(np.abs(got - ref) <= np.abs(ref) * 2 ** -8 + 1e-6)
+    assert ops.moe_get_device_status(W) == 0
+
+
+# --------------------------------------------------------------- forward ----
+FWD_CASES = [
+    ("tiny", {}, 1, False), ("tiny", {}, 0, False), ("tiny", {}, 1, True),
+    ("decode", {}, 1, False), ("decode", {}, 0, False), ("decode", {}, 1, True),
+    ("fp8_shared", dict(T=24, H=256, E=16, k=4, I=128, shared_I=128), 1, False),
+    ("tiny", dict(fmt="mxfp4", T=12, H=256, E=8, k=2, I=256), 1, False),
+]
+
+
+@pytest.mark.parametrize("name,over,act,static", FWD_CASES)
+def test_forward_matches_oracle(name, over, act, static):
+    w = synth.workload(name, **over)
+    W, Ws = oracle_bank(w)
+    a13, a2 = synth.static_act_scales() if static else (None, None)
+    bank = device_bank(W, a13, a2)
+    sbank = device_bank(Ws, None, a2) if Ws is not None else None
+    x, wr, b = routed_inputs(w)
+    W_ = ws(ops.workspace_size(w.T, w.k, bank, sbank, act))
+    out = ops.moe_forward(bits_to_dev_bf16(x), bits_to_dev_bf16(wr), None if b is None else torch.from_numpy(b).cuda(),
+                          w.k, bank, sbank, act, W_)
+    assert ops.moe_get_device_status(W_) == 0
+    r = oracle.moe_forward(x, wr, b, w.k, W, Ws, act=act, a13_static=a13 or 0.0, a2_static=a2 or 0.0,
+                           sh_a2_static=a2 or 0.0)
+    keep = ~ambiguous_tokens(r["logits"], w.k, 1e-4, boundary_only=True)
+    err = max_abs_rel(dev_to_f64(out)[keep], r["out"][keep])
+    assert err < TOL, err
