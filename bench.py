@@ -307,6 +307,23 @@ def workload_name(w) -> str:
     return s
 
 
+# ------------------------------------------------------------- replicas ----
+def max_over_ranks(value: float, device="cuda") -> float:
+    """The slowest rank's time (no-op without an initialised process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_rank: int, steps: int, world: int, slowest_s: float) -> float:
+    """Whole-job tokens/s: every replica's tokens over the slowest replica's time."""
+    return world * tokens_per_rank * steps / slowest_s
+
+
 # ------------------------------------------------------------------ main ----
 def main():
     args = parse()
@@ -344,22 +361,15 @@ def main():
     barrier()
     clocks = clock.stop()
     ms = float(np.mean(res["ms"]))
-    total_s = float(np.sum(res["ms"])) / 1e3
-    if world > 1:
-        t = torch.tensor([total_s], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_s = float(t.item())
-    value = world * w.T * args.steps / total_s
+    total_s = max_over_ranks(float(np.sum(res["ms"])) / 1e3)
+    ms = total_s * 1e3 / args.steps
+    value = job_throughput(w.T, args.steps, world, total_s)
 
     # end to end: pinned host input -> device -> forward -> host output
     barrier()
     res_e2e = time_forward(ops, torch, layer, w, act, args.steps, 2, flush, stage=False, host_io=True)
-    e2e_s = float(np.sum(res_e2e["ms"])) / 1e3
-    if world > 1:
-        t = torch.tensor([e2e_s], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_s = float(t.item())
-    e2e = {"value": world * w.T * args.steps / e2e_s, "unit": "tokens/s",
+    e2e_s = max_over_ranks(float(np.sum(res_e2e["ms"])) / 1e3)
+    e2e = {"value": job_throughput(w.T, args.steps, world, e2e_s), "unit": "tokens/s",
            "h2d_bytes_per_step": w.T * w.H * 2, "d2h_bytes_per_step": w.T * w.H * 2}
 
     alg = algorithmic(w, w.fmt, res["offsets"])

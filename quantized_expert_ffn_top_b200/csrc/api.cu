@@ -5,6 +5,7 @@
 #include <cstring>
 #include <mutex>
 
+#include "gemm_tc.cuh"
 #include "kernels.cuh"
 
 namespace moe {
@@ -119,12 +120,39 @@ PermWs carve_perm(Carver& c, int64_t S, int E) {
   return p;
 }
 
+constexpr int kGemmBN = 128;  // token tile of the tensor-core path
+
+int64_t padded_rows(int64_t S, int E) { return (int64_t)align_up((size_t)(S + (int64_t)E * 127), 128) + 256; }
+int64_t max_tiles(int64_t S, int E) { return S / kGemmBN + E + 1; }
+
+// Scratch of the grouped FFN: GEMV path (h fp32 per compact slot) and tensor
+// core path (padded, blocked quantised activations and the tile plan).
 struct FfnScratch {
-  float* h;  // [S][I]
+  float* h;          // GEMV: [S][I] fp32
+  int32_t* poff;     // GEMM: [E+1] padded offsets
+  TileEntry* tiles;  //       [max_tiles]
+  int32_t* ntiles;
+  uint8_t* xq;       //       [P][H/2 | H] codes of x in padded rows
+  uint8_t* xsf;      //       [P * H/bs] blocked scales
+  uint8_t* hq;       //       [P][I/2 | I]
+  uint8_t* hsf;
+  float* h32;        //       [P][I] fp32 h (dynamic h scale / FP8)
+  int64_t P;
 };
 FfnScratch carve_ffn(Carver& c, int64_t S, const moe_weights* w) {
   FfnScratch f;
+  const int bs = w->fmt == MOE_FMT_NVFP4 ? 16 : (w->fmt == MOE_FMT_MXFP4 ? 32 : 0);
+  const int64_t rbh = w->fmt == MOE_FMT_FP8 ? w->H : w->H / 2, rbi = w->fmt == MOE_FMT_FP8 ? w->I : w->I / 2;
+  f.P = padded_rows(S, w->E);
   f.h = c.take<float>((size_t)S * w->I);
+  f.poff = c.take<int32_t>((size_t)w->E + 1);
+  f.tiles = c.take<TileEntry>((size_t)max_tiles(S, w->E));
+  f.ntiles = c.take<int32_t>(1);
+  f.xq = c.take<uint8_t>((size_t)(f.P * rbh));
+  f.xsf = bs ? c.take<uint8_t>((size_t)(f.P * (w->H / bs))) : nullptr;
+  f.hq = c.take<uint8_t>((size_t)(f.P * rbi));
+  f.hsf = bs ? c.take<uint8_t>((size_t)(f.P * (w->I / bs))) : nullptr;
+  f.h32 = c.take<float>((size_t)(f.P * w->I));
   return f;
 }
 
@@ -182,11 +210,106 @@ __global__ void identity_routing_kernel(int64_t T, int32_t* offsets, int32_t* pe
   }
 }
 
+bool gemm_shapes_ok(const moe_weights* w, int act) {
+  if (act != MOE_ACT_MATCH || !tensor_maps_available()) return false;
+  const int kb = w->fmt == MOE_FMT_FP8 ? 128 : 256;
+  return w->H % kb == 0 && w->I % kb == 0 && w->I % 64 == 0;
+}
+
+// Tensor cores once the average expert has enough rows to fill a tile; the
+// weight-streaming GEMV below that.  Arguments only, no device read-back.
 bool use_gemm_path(const moe_weights* w, int64_t S, int act) {
-  (void)w;
-  (void)S;
-  (void)act;
-  return false;
+  if (g_ffn_path == 1) return false;
+  if (!gemm_shapes_ok(w, act)) return false;
+  if (g_ffn_path == 2) return true;
+  return S >= 8 * (int64_t)w->E;
+}
+
+moe_status run_gemm_ffn(const uint16_t* x, int64_t T, int64_t S, const int32_t* perm, const int32_t* offsets,
+                        const moe_weights* w, uint16_t* y_perm, const FfnScratch& f, float* x_amax, float* h_amax,
+                        int32_t* status, cudaStream_t s, bool mark) {
+  const int E = w->E, H = w->H, I = w->I, fmt = w->fmt;
+  const int sms = num_sms();
+  MOE_TRY(launch_plan(offsets, E, S, kGemmBN, f.poff, f.tiles, f.ntiles, (int)max_tiles(S, E), status, s));
+  if (mark) stage_mark(MOE_STAGE_ACT_QUANT, false, s);
+  QuantPaddedArgs qa;
+  qa.E = E;
+  qa.K = H;
+  qa.S = S;
+  qa.T = T;
+  qa.P = f.P;
+  qa.offsets = offsets;
+  qa.poff = f.poff;
+  qa.perm_token = perm;
+  qa.x = x;
+  qa.h32 = nullptr;
+  qa.scale = w->a13_gs;
+  qa.amax = x_amax;
+  qa.codes = f.xq;
+  qa.sf = f.xsf;
+  qa.status = status;
+  MOE_TRY(launch_quant_padded(qa, true, fmt, sms, s));
+  if (mark) stage_mark(MOE_STAGE_ACT_QUANT, true, s);
+  // gate|up projection + SwiGLU: quantise h in the epilogue when its scale
+  // needs no global reduction (MXFP4, or a static NVFP4 scale)
+  const bool fused_h = fmt == MOE_FMT_MXFP4 || (fmt == MOE_FMT_NVFP4 && w->a2_gs);
+  GemmArgs g;
+  memset(&g, 0, sizeof(g));
+  g.fmt = fmt;
+  g.E = E;
+  g.K = H;
+  g.R = 2 * I;
+  g.w_sf = w->w13_sf;
+  g.b_sf = f.xsf;
+  g.w_gs = w->w13_gs;
+  g.act_scale = w->a13_gs;
+  g.act_amax = x_amax;
+  g.tiles = f.tiles;
+  g.num_tiles = f.ntiles;
+  g.I = I;
+  g.hq = f.hq;
+  g.hsf = f.hsf;
+  g.h_scale = w->a2_gs;
+  g.h32 = f.h32;
+  g.h_amax = fused_h ? nullptr : h_amax;
+  g.status = status;
+  if (mark) stage_mark(MOE_STAGE_FFN_UP, false, s);
+  if (!fused_h) MOE_TRY(cudaMemsetAsync(h_amax, 0, sizeof(float), s));
+  MOE_TRY(launch_grouped_gemm(g, fused_h ? kEpiUpQuant : kEpiUpF32, kGemmBN, w->w13, (int64_t)E * 2 * I,
+                              f.xq, f.P, sms, s));
+  if (!fused_h) {
+    QuantPaddedArgs qh = qa;
+    qh.K = I;
+    qh.h32 = f.h32;
+    qh.scale = w->a2_gs;
+    qh.amax = h_amax;
+    qh.codes = f.hq;
+    qh.sf = f.hsf;
+    MOE_TRY(launch_quant_padded(qh, false, fmt, sms, s));
+  }
+  if (mark) stage_mark(MOE_STAGE_FFN_UP, true, s);
+  // down projection -> y_perm
+  GemmArgs d;
+  memset(&d, 0, sizeof(d));
+  d.fmt = fmt;
+  d.E = E;
+  d.K = I;
+  d.R = H;
+  d.w_sf = w->w2_sf;
+  d.b_sf = f.hsf;
+  d.w_gs = w->w2_gs;
+  d.act_scale = w->a2_gs;
+  d.act_amax = h_amax;
+  d.tiles = f.tiles;
+  d.num_tiles = f.ntiles;
+  d.I = I;
+  d.y = y_perm;
+  d.ldy = H;
+  d.status = status;
+  if (mark) stage_mark(MOE_STAGE_FFN_DOWN, false, s);
+  MOE_TRY(launch_grouped_gemm(d, kEpiDown, kGemmBN, w->w2, (int64_t)E * H, f.hq, f.P, sms, s));
+  if (mark) stage_mark(MOE_STAGE_FFN_DOWN, true, s);
+  return MOE_OK;
 }
 
 // Grouped FFN on already-validated arguments.  x_amax must hold amax(x) when
@@ -196,8 +319,10 @@ moe_status run_grouped_ffn(const uint16_t* x, int64_t T, int64_t S, const int32_
                            float* x_amax, float* h_amax, int32_t* status, cudaStream_t s,
                            bool shared_stage = false) {
   if (S == 0) return MOE_OK;
-  if (g_ffn_path == 2) return MOE_ERR_UNSUPPORTED;
   const bool mark = !shared_stage;
+  if (use_gemm_path(w, S, act))
+    return run_gemm_ffn(x, T, S, perm, offsets, w, y_perm, scratch, x_amax, h_amax, status, s, mark);
+  if (g_ffn_path == 2) return MOE_ERR_UNSUPPORTED;
   GemvArgs a;
   a.fmt = w->fmt;
   a.act = act;

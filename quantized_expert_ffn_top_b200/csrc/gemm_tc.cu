@@ -1,0 +1,591 @@
+// Tensor-core grouped expert GEMM for large batches (sm_100a tcgen05).
+//
+// The prefill half of the prefill/decode split the atomicmilkshake/FreeToken
+// fork README describes ("Quant types": MMQ for prefill), rebuilt for B200:
+// block-scaled tcgen05.mma (kind::mxf4nvf4 for NVFP4 / MXFP4, kind::f8f6f4
+// for FP8 W8A8 -- the per-tensor FP8 projection of FreeToken commit
+// 58f4b9ec0e) with accumulators in tensor memory, operands staged by TMA.
+//
+// Orientation ("swap AB"): the MMA's M side is 128 weight rows of one expert
+// and its N side is a tile of that expert's tokens (the permuted slots).
+// Weight rows always fill M = 128, while a ragged expert segment only pads N
+// to a multiple of 16, so skewed routing wastes little work.
+//
+// Per CTA (persistent, one per SM), 2 + kEpiWarps warps:
+//   warp 0   one thread issues TMA tile loads of A (weights) and B (quantised
+//            activations) and bulk copies of their scale blocks into a ring of
+//            shared-memory stages;
+//   warp 1   allocates tensor memory; one thread copies each stage's scales
+//            into tensor memory (tcgen05.cp) and issues the MMAs;
+//   others   epilogue: read the accumulator from tensor memory (tcgen05.ld),
+//            apply the tensor scales and write the result: SwiGLU and the
+//            quantised h for the gate|up projection, bf16 y for the down
+//            projection.
+// Accumulators are double buffered in tensor memory so the epilogue of one
+// tile overlaps the MMAs of the next.  Every wait is bounded: on timeout the
+// kernel raises MOE_ERR_TIMEOUT, drains, frees its tensor memory and exits.
+//
+// Layouts (all prepared by the library):
+//  * weights: PREPARED rows (W13: row 2i gate i, row 2i+1 up i), K-major;
+//    scales blocked per 128 rows x 4 scale columns (sf_blocked_offset);
+//  * activations: expert segments start on a multiple of 128 rows
+//    ("padded" rows), K-major codes, scales blocked the same way.
+#include <cuda.h>
+
+#include "kernels.cuh"
+#include "gemm_tc.cuh"
+#include "tc_ptx.cuh"
+
+namespace moe {
+namespace {
+
+template <int FMT>
+struct FmtTraits {
+  static constexpr int kBK = FMT == MOE_FMT_FP8 ? 128 : 256;      // K elements per stage (128 bytes per row)
+  static constexpr int kMmaK = FMT == MOE_FMT_FP8 ? 32 : 64;
+  static constexpr int kSteps = kBK / kMmaK;                        // MMAs per stage
+  static constexpr int kBs = FMT == MOE_FMT_NVFP4 ? 16 : (FMT == MOE_FMT_MXFP4 ? 32 : 0);
+  static constexpr int kGroups = kBs ? kBK / (4 * kBs) : 0;         // 4-column scale groups per stage
+};
+
+template <int FMT, int EPI, int BN>
+struct Cfg {
+  using F = FmtTraits<FMT>;
+  static constexpr int kA = 128 * 128;
+  static constexpr int kB = BN * 128;
+  static constexpr int kSFA = F::kGroups * 512;
+  static constexpr int kSFB = F::kGroups * 512 * (BN / 128);
+  static constexpr int kStage = ((kA + kB + kSFA + kSFB) + 1023) / 1024 * 1024;
+  static constexpr int kStages = (200 * 1024) / kStage < 8 ? (200 * 1024) / kStage : 8;
+  static constexpr int kAccStages = BN == 256 ? 1 : 2;
+  static constexpr int kEpiWarps = 8;
+  static constexpr int kThreads = (2 + kEpiWarps) * 32;
+  static constexpr uint32_t kSfaCol = kAccStages * BN;
+  static constexpr uint32_t kSfbCol = kSfaCol + F::kGroups * 4;
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kTx = kA + kB + kSFA + kSFB;
+  static constexpr int kSmem = kStages * kStage + 1024 /*align*/ + 1024 /*barriers etc.*/;
+  static_assert(kSfbCol + F::kGroups * 4 * (BN / 128) <= kTmemCols, "tensor memory overflow");
+};
+
+__device__ __forceinline__ float act_scale_of(int fmt, const float* st, const float* amax) {
+  if (fmt == MOE_FMT_MXFP4) return 1.0f;
+  if (st) return __ldg(st);
+  if (!amax) return 1.0f;
+  return fmt == MOE_FMT_NVFP4 ? nvfp4_tensor_scale(*amax) : fp8_tensor_scale(*amax);
+}
+
+template <int FMT, int EPI, int BN>
+__global__ void __launch_bounds__(Cfg<FMT, EPI, BN>::kThreads, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                        const GemmArgs g) {
+  using C = Cfg<FMT, EPI, BN>;
+  using F = FmtTraits<FMT>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* ctrl = smem + C::kStages * C::kStage;
+  uint64_t* full = reinterpret_cast<uint64_t*>(ctrl);
+  uint64_t* empty = full + C::kStages;
+  uint64_t* tfull = empty + C::kStages;
+  uint64_t* tempty = tfull + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* xmax = reinterpret_cast<float*>(tmem_slot + 4);  // [kEpiWarps][16] MXFP4 block max exchange
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      tc::mbar_init(&full[s], 1);
+      tc::mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      tc::mbar_init(&tfull[a], 1);
+      tc::mbar_init(&tempty[a], C::kEpiWarps);
+    }
+    *abort = 0;
+    tc::fence_mbar_init();
+    tc::prefetch_tmap(&tmap_a);
+    tc::prefetch_tmap(&tmap_b);
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(tmem_slot, C::kTmemCols);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  const int MT = g.R / 128;
+  const int ntiles = __ldg(g.num_tiles) * MT;
+  const int nkb = g.K / F::kBK;
+  const int ncols_w = F::kBs ? g.K / F::kBs : 0;  // scale columns per row (multiple of 4)
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int t = blockIdx.x; t < ntiles && !*abort; t += gridDim.x) {
+        const TileEntry te = g.tiles[t / MT];
+        const int mt = t % MT;
+        const uint8_t* sfa = F::kBs ? g.w_sf + (size_t)te.e * g.R * ncols_w + (size_t)mt * (ncols_w / 4) * 512 : nullptr;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!tc::mbar_wait(&empty[stage], phase ^ 1u, abort)) {
+            raise_status(g.status, MOE_ERR_TIMEOUT);
+            *abort = 1;
+            break;
+          }
+          uint8_t* st = smem + stage * C::kStage;
+          tc::mbar_expect_tx(&full[stage], C::kTx);
+          tc::tma_load_2d(st, &tmap_a, &full[stage], kb * 128, te.e * g.R + mt * 128);
+          tc::tma_load_2d(st + C::kA, &tmap_b, &full[stage], kb * 128, te.row0);
+          if (F::kBs) {
+            tc::bulk_load(st + C::kA + C::kB, sfa + (size_t)kb * F::kGroups * 512, C::kSFA, &full[stage]);
+            for (int nb = 0; nb < BN / 128; ++nb) {
+              const uint8_t* sfb =
+                  g.b_sf + ((size_t)(te.row0 / 128 + nb) * (ncols_w / 4) + (size_t)kb * F::kGroups) * 512;
+              tc::bulk_load(st + C::kA + C::kB + C::kSFA + nb * F::kGroups * 512, sfb, F::kGroups * 512,
+                            &full[stage]);
+            }
+          }
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      for (int t = blockIdx.x; t < ntiles && !*abort; t += gridDim.x) {
+        const TileEntry te = g.tiles[t / MT];
+        if (!tc::mbar_wait(&tempty[acc], acc_phase ^ 1u, abort)) {
+          raise_status(g.status, MOE_ERR_TIMEOUT);
+          *abort = 1;
+          break;
+        }
+        tc::fence_after_sync();
+        const uint32_t n_mma = (uint32_t)min(BN, (te.nvalid + 15) & ~15);
+        const uint32_t d = tmem + acc * BN;
+        bool ok = true;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!tc::mbar_wait(&full[stage], phase, abort)) {
+            raise_status(g.status, MOE_ERR_TIMEOUT);
+            *abort = 1;
+            ok = false;
+            break;
+          }
+          tc::fence_after_sync();
+          uint8_t* st = smem + stage * C::kStage;
+          const uint32_t sa = tc::smem_u32(st), sb = tc::smem_u32(st + C::kA);
+          if (F::kBs) {
+            const uint32_t ssfa = tc::smem_u32(st + C::kA + C::kB);
+            const uint32_t ssfb = ssfa + C::kSFA;
+            for (int grp = 0; grp < F::kGroups; ++grp) {
+              tc::sf_copy(tmem + C::kSfaCol + 4 * grp, tc::desc_sf(ssfa + grp * 512));
+              for (int nb = 0; nb < BN / 128; ++nb)
+                tc::sf_copy(tmem + C::kSfbCol + grp * 4 * (BN / 128) + nb * 4,
+                            tc::desc_sf(ssfb + (nb * F::kGroups + grp) * 512));
+            }
+          }
+#pragma unroll
+          for (int kk = 0; kk < F::kSteps; ++kk) {
+            const uint64_t da = tc::desc_sw128(sa) + (uint64_t)(kk * 2);  // +32 bytes per MMA along K
+            const uint64_t db = tc::desc_sw128(sb) + (uint64_t)(kk * 2);
+            const uint32_t accum = (kb > 0 || kk > 0) ? 1u : 0u;
+            if (FMT == MOE_FMT_NVFP4) {
+              tc::mma_nvf4(d, da, db, tc::idesc_mxf4(n_mma, false, 0, 0), tmem + C::kSfaCol + 4 * kk,
+                           tmem + C::kSfbCol + kk * 4 * (BN / 128), accum);
+            } else if (FMT == MOE_FMT_MXFP4) {
+              const uint32_t id = (uint32_t)(kk & 1) * 2;  // two MMAs share one group of four e8m0 scales
+              tc::mma_mxf4(d, da, db, tc::idesc_mxf4(n_mma, true, id, id), tmem + C::kSfaCol + 4 * (kk >> 1),
+                           tmem + C::kSfbCol + (kk >> 1) * 4 * (BN / 128), accum);
+            } else {
+              tc::mma_f8(d, da, db, tc::idesc_f8(n_mma), accum);
+            }
+          }
+          tc::mma_commit(&empty[stage]);
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc::mma_commit(&tfull[acc]);
+        if (++acc == C::kAccStages) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int ew = warp - 2;
+    const int q = warp & 3;                      // tensor-memory lane quarter of this warp
+    const int half = ew / 4;                     // which half of the tile's columns
+    const float gact = act_scale_of(FMT, g.act_scale, g.act_amax);
+    const float g2 = (EPI == kEpiUpQuant && FMT == MOE_FMT_NVFP4) ? act_scale_of(FMT, g.h_scale, nullptr) : 1.0f;
+    float hmax = 0.0f;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+      if (!tc::mbar_wait(&tfull[acc], acc_phase, abort)) {
+        if (lane == 0) raise_status(g.status, MOE_ERR_TIMEOUT);
+        *abort = 1;
+        break;
+      }
+      tc::fence_after_sync();
+      const TileEntry te = g.tiles[t / MT];
+      const int mt = t % MT;
+      const int ncol = min(BN, (te.nvalid + 15) & ~15);
+      const int c_lo = half * (BN / 2), c_hi = min(ncol, (half + 1) * (BN / 2));
+      const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+      if (EPI == kEpiDown) {
+        const int o = mt * 128 + q * 32 + lane;
+        const float sc = (FMT == MOE_FMT_MXFP4) ? 1.0f : __ldg(g.w_gs + te.e) * gact;
+        for (int c0 = c_lo; c0 < c_hi; c0 += 16) {
+          float v[16];
+          tc::tmem_ld16(tbase + c0, v);
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const int tok = c0 + c;
+            if (tok < te.nvalid) g.y[(size_t)(te.p0 + tok) * g.ldy + o] = f32_to_bf16_rn(v[c] * sc);
+          }
+        }
+      } else {
+        const int part = lane & 1;
+        const float sc = (FMT == MOE_FMT_MXFP4) ? 1.0f : __ldg(g.w_gs + te.e * 2 + part) * gact;
+        const int f_base = mt * 64 + q * 16;       // this warp's 16 features
+        const int f = f_base + (lane >> 1);
+        for (int c0 = c_lo; c0 < c_hi; c0 += 16) {
+          float v[16];
+          tc::tmem_ld16(tbase + c0, v);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float a = v[2 * i] * sc, b = v[2 * i + 1] * sc;
+            const float recv = __shfl_xor_sync(0xffffffffu, part ? a : b, 1);
+            const float gg = part ? recv : a;
+            const float uu = part ? b : recv;
+            const float h = gg / (1.0f + __expf(-gg)) * uu;
+            const int tok = c0 + 2 * i + part;
+            const bool valid = tok < te.nvalid;
+            if (EPI == kEpiUpF32) {
+              if (valid) {
+                g.h32[(size_t)(te.row0 + tok) * g.I + f] = h;
+                hmax = fmaxf(hmax, fabsf(h));
+              }
+            } else {
+              // quantise h: one 16-feature block per warp and token (NVFP4),
+              // two warps per 32-feature block (MXFP4)
+              float bmax = fabsf(h);
+#pragma unroll
+              for (int o = 2; o < 32; o <<= 1) bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, o));
+              uint32_t code = 0, scode = 0;
+              if (FMT == MOE_FMT_NVFP4) {
+                float r;
+                nvfp4_block_scale(bmax, g2, scode, r);
+                code = r != 0.0f ? (e2m1x2_encode(__fmul_rn(h, r), 0.0f) & 0xFu) : 0u;
+              } else {
+                // exchange the 16-feature maxima with the partner warp (q ^ 1)
+                const int bar = 1 + ew / 2;
+                if (lane < 2) xmax[ew * 16 + 2 * i + lane] = bmax;
+                asm volatile("bar.sync %0, 64;" ::"r"(bar) : "memory");
+                const float other = xmax[(ew ^ 1) * 16 + 2 * i + part];
+                asm volatile("bar.sync %0, 64;" ::"r"(bar) : "memory");
+                float inv;
+                mxfp4_block_scale(fmaxf(bmax, other), scode, inv);
+                code = e2m1x2_encode(__fmul_rn(h, inv), 0.0f) & 0xFu;
+              }
+              // pack: byte j of the warp's 8 holds features 2j (lo) and 2j+1 (hi)
+              const uint32_t hi = __shfl_down_sync(0xffffffffu, code, 2);
+              const uint32_t byte = code | (hi << 4);
+              uint32_t w0 = 0, w1 = 0;
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                w0 |= (__shfl_sync(0xffffffffu, byte, 4 * j + part) & 0xFFu) << (8 * j);
+                w1 |= (__shfl_sync(0xffffffffu, byte, 16 + 4 * j + part) & 0xFFu) << (8 * j);
+              }
+              if (lane < 2 && valid) {
+                const size_t row = (size_t)(te.row0 + tok);
+                *reinterpret_cast<uint2*>(g.hq + row * (g.I / 2) + f_base / 2) = make_uint2(w0, w1);
+                if (FMT == MOE_FMT_NVFP4)
+                  g.hsf[sf_blocked_offset((int64_t)row, f_base / 16, g.I / 16)] = (uint8_t)scode;
+                else if ((q & 1) == 0)
+                  g.hsf[sf_blocked_offset((int64_t)row, f_base / 32, g.I / 32)] = (uint8_t)scode;
+              }
+            }
+          }
+        }
+      }
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&tempty[acc]);
+      if (++acc == C::kAccStages) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+    if (EPI == kEpiUpF32 && g.h_amax) {
+      hmax = warp_max(hmax);
+      if (lane == 0) atomic_max_nonneg(g.h_amax, hmax);
+    }
+  }
+
+  __syncwarp();
+  __syncthreads();
+  if (*abort) {
+    // let copies and MMAs already in flight land before the memory goes away
+    const long long t0 = clock64();
+    while (clock64() - t0 < 2000000LL) {
+    }
+  }
+  tc::fence_after_sync();
+  if (warp == 1) tc::tmem_dealloc(tmem, C::kTmemCols);
+}
+
+// ------------------------------------------------------------- tensor maps --
+using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                 const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiled encode_fn() {
+  static EncodeTiled fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiled>(p);
+  }
+  return fn;
+}
+
+// Rows of `row_bytes` bytes, box = 128 bytes x box_rows rows, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t row_bytes, int box_rows) {
+  EncodeTiled fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+  cuuint32_t box[2] = {128u, (cuuint32_t)box_rows};
+  cuuint32_t es[2] = {1u, 1u};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int FMT, int EPI, int BN>
+cudaError_t launch_cfg(const GemmArgs& g, const void* a_base, int64_t a_rows, const void* b_base, int64_t b_rows,
+                       int num_sms, cudaStream_t s) {
+  using C = Cfg<FMT, EPI, BN>;
+  CUtensorMap ma, mb;
+  const int64_t rb = FMT == MOE_FMT_FP8 ? g.K : g.K / 2;
+  if (!make_map(&ma, a_base, a_rows, rb, 128) || !make_map(&mb, b_base, b_rows, rb, BN))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<FMT, EPI, BN>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+  if (e != cudaSuccess) return e;
+  grouped_gemm_kernel<FMT, EPI, BN><<<num_sms, C::kThreads, C::kSmem, s>>>(ma, mb, g);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+template <int FMT, int EPI>
+cudaError_t launch_bn(const GemmArgs& g, int bn, const void* a, int64_t ar, const void* b, int64_t br, int sms,
+                      cudaStream_t s) {
+  if (bn == 256) return launch_cfg<FMT, EPI, 256>(g, a, ar, b, br, sms, s);
+  return launch_cfg<FMT, EPI, 128>(g, a, ar, b, br, sms, s);
+}
+
+template <int FMT>
+cudaError_t launch_epi(const GemmArgs& g, int epi, int bn, const void* a, int64_t ar, const void* b, int64_t br,
+                       int sms, cudaStream_t s) {
+  if (epi == kEpiDown) return launch_bn<FMT, kEpiDown>(g, bn, a, ar, b, br, sms, s);
+  if (epi == kEpiUpF32) return launch_bn<FMT, kEpiUpF32>(g, bn, a, ar, b, br, sms, s);
+  if (FMT == MOE_FMT_FP8) return cudaErrorInvalidValue;
+  return launch_bn<FMT, kEpiUpQuant>(g, bn, a, ar, b, br, sms, s);
+}
+
+}  // namespace
+
+cudaError_t launch_grouped_gemm(const GemmArgs& g, int epi, int bn, const void* a_base, int64_t a_rows,
+                                const void* b_base, int64_t b_rows, int num_sms, cudaStream_t s) {
+  switch (g.fmt) {
+    case MOE_FMT_NVFP4: return launch_epi<MOE_FMT_NVFP4>(g, epi, bn, a_base, a_rows, b_base, b_rows, num_sms, s);
+    case MOE_FMT_MXFP4: return launch_epi<MOE_FMT_MXFP4>(g, epi, bn, a_base, a_rows, b_base, b_rows, num_sms, s);
+    case MOE_FMT_FP8: return launch_epi<MOE_FMT_FP8>(g, epi, bn, a_base, a_rows, b_base, b_rows, num_sms, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+bool tensor_maps_available() { return encode_fn() != nullptr; }
+
+// ---------------------------------------------------------------- planning --
+// One block: padded offsets (every expert segment starts on a multiple of 128
+// rows) and the tile list (expert, first padded row, valid rows, first slot).
+__global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ offsets, int E, int64_t S, int bn,
+                                                    int32_t* __restrict__ poff, TileEntry* __restrict__ tiles,
+                                                    int32_t* __restrict__ num_tiles, int max_tiles,
+                                                    int32_t* status) {
+  __shared__ int32_t s_pad[1024], s_til[1024];
+  __shared__ int bad;
+  const int e = threadIdx.x;
+  if (e == 0) bad = (offsets[0] != 0 || offsets[E] != S) ? 1 : 0;
+  __syncthreads();
+  int32_t n = 0, pad = 0, til = 0, o0 = 0;
+  if (e < E) {
+    o0 = offsets[e];
+    n = offsets[e + 1] - o0;
+    if (n < 0) {
+      bad = 1;
+      n = 0;
+    }
+    pad = (n + 127) / 128 * 128;
+    til = (n + bn - 1) / bn;
+  }
+  s_pad[e] = pad;
+  s_til[e] = til;
+  __syncthreads();
+  // inclusive Hillis-Steele scans (E <= 1024)
+  for (int d = 1; d < 1024; d <<= 1) {
+    const int32_t a = e >= d ? s_pad[e - d] : 0, b = e >= d ? s_til[e - d] : 0;
+    __syncthreads();
+    s_pad[e] += a;
+    s_til[e] += b;
+    __syncthreads();
+  }
+  const int32_t pbase = s_pad[e] - pad, tbase = s_til[e] - til;
+  if (e < E) {
+    poff[e] = pbase;
+    for (int j = 0; j < til && tbase + j < max_tiles; ++j) {
+      TileEntry te;
+      te.e = e;
+      te.row0 = pbase + j * bn;
+      te.nvalid = min(bn, n - j * bn);
+      te.p0 = o0 + j * bn;
+      tiles[tbase + j] = te;
+    }
+  }
+  __syncthreads();
+  if (e == E - 1) {
+    poff[E] = s_pad[e];
+    *num_tiles = bad ? 0 : min(s_til[e], max_tiles);
+    if (bad) raise_status(status, MOE_ERR_DEVICE_FAULT);
+  }
+}
+
+cudaError_t launch_plan(const int32_t* offsets, int E, int64_t S, int bn, int32_t* poff, TileEntry* tiles,
+                        int32_t* num_tiles, int max_tiles, int32_t* status, cudaStream_t s) {
+  plan_kernel<<<1, 1024, 0, s>>>(offsets, E, S, bn, poff, tiles, num_tiles, max_tiles, status);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------- padded quantisation --
+// Quantises activation rows into the padded, blocked layout the GEMM reads.
+// Source row of slot p: x[perm_token[p]] (bf16, SRC_X) or h32[padded row]
+// (fp32); destination: padded row poff[e] + (p - offsets[e]).
+template <int FMT, bool SRC_X>
+__global__ void __launch_bounds__(256) quant_padded_kernel(QuantPaddedArgs a) {
+  constexpr int bs = FMT == MOE_FMT_MXFP4 ? 32 : 16;
+  const int nb = a.K / bs;
+  const int64_t total = a.S * nb;
+  const float scale = act_scale_of(FMT, a.scale, a.amax);
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t it = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; it < total; it += stride) {
+    const int p = (int)(it / nb), b = (int)(it % nb);
+    const int e = segment_of(a.offsets, a.E, p);
+    const int64_t row = (int64_t)__ldg(a.poff + e) + (p - __ldg(a.offsets + e));
+    if (row < 0 || row >= a.P || p < __ldg(a.offsets + e)) {
+      if (b == 0) raise_status(a.status, MOE_ERR_DEVICE_FAULT);
+      continue;
+    }
+    float v[bs];
+    float bmax = 0.0f;
+    if (SRC_X) {
+      const int t = __ldg(a.perm_token + p);
+      if (t < 0 || t >= a.T) {
+        if (b == 0) raise_status(a.status, MOE_ERR_DEVICE_FAULT);
+#pragma unroll
+        for (int i = 0; i < bs; ++i) v[i] = 0.0f;
+      } else {
+        const uint16_t* src = a.x + (int64_t)t * a.K + b * bs;
+#pragma unroll
+        for (int i = 0; i < bs; i += 8) {
+          const uint4 w = __ldg(reinterpret_cast<const uint4*>(src + i));
+          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            v[i + 2 * j] = __uint_as_float(ww[j] << 16);
+            v[i + 2 * j + 1] = __uint_as_float(ww[j] & 0xFFFF0000u);
+          }
+        }
+      }
+    } else {
+      const float* src = a.h32 + row * a.K + b * bs;
+#pragma unroll
+      for (int i = 0; i < bs; i += 4) {
+        const float4 w = *reinterpret_cast<const float4*>(src + i);
+        v[i] = w.x;
+        v[i + 1] = w.y;
+        v[i + 2] = w.z;
+        v[i + 3] = w.w;
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < bs; ++i) bmax = fmaxf(bmax, fabsf(v[i]));
+    if constexpr (FMT == MOE_FMT_NVFP4) {
+      uint32_t sc;
+      float r;
+      nvfp4_block_scale(bmax, scale, sc, r);
+      *reinterpret_cast<uint2*>(a.codes + row * (a.K / 2) + b * 8) = nvfp4_encode16(v, r);
+      a.sf[sf_blocked_offset(row, b, nb)] = (uint8_t)sc;
+    } else if constexpr (FMT == MOE_FMT_MXFP4) {
+      uint32_t c;
+      float inv;
+      mxfp4_block_scale(bmax, c, inv);
+      uint4 w;
+      w.x = e2m1_encode8(v, inv);
+      w.y = e2m1_encode8(v + 8, inv);
+      w.z = e2m1_encode8(v + 16, inv);
+      w.w = e2m1_encode8(v + 24, inv);
+      *reinterpret_cast<uint4*>(a.codes + row * (a.K / 2) + b * 16) = w;
+      a.sf[sf_blocked_offset(row, b, nb)] = (uint8_t)c;
+    } else {
+      const float inv = __frcp_rn(scale);
+      uint4 w;
+      uint32_t* pw = &w.x;
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        pw[i] = e4m3x2_encode(__fmul_rn(v[4 * i], inv), __fmul_rn(v[4 * i + 1], inv)) |
+                (e4m3x2_encode(__fmul_rn(v[4 * i + 2], inv), __fmul_rn(v[4 * i + 3], inv)) << 16);
+      *reinterpret_cast<uint4*>(a.codes + row * a.K + b * 16) = w;
+    }
+  }
+}
+
+cudaError_t launch_quant_padded(const QuantPaddedArgs& a, bool src_x, int fmt, int num_sms, cudaStream_t s) {
+  const int bs = fmt == MOE_FMT_MXFP4 ? 32 : 16;
+  const int64_t total = a.S * (a.K / bs);
+  if (total == 0) return cudaSuccess;
+  const int64_t blocks = (total + 255) / 256;
+  const int grid = (int)(blocks < (int64_t)num_sms * 16 ? blocks : (int64_t)num_sms * 16);
+#define MOE_QP(F)                                                              \
+  if (src_x) quant_padded_kernel<F, true><<<grid, 256, 0, s>>>(a);           \
+  else quant_padded_kernel<F, false><<<grid, 256, 0, s>>>(a);
+  switch (fmt) {
+    case MOE_FMT_NVFP4: MOE_QP(MOE_FMT_NVFP4) break;
+    case MOE_FMT_MXFP4: MOE_QP(MOE_FMT_MXFP4) break;
+    case MOE_FMT_FP8: MOE_QP(MOE_FMT_FP8) break;
+    default: return cudaErrorInvalidValue;
+  }
+#undef MOE_QP
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

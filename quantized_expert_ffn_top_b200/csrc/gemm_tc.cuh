@@ -1,0 +1,62 @@
+// Internal interface of the tensor-core grouped GEMM path (gemm_tc.cu).
+#pragma once
+
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace moe {
+
+// One token tile of one expert: the padded row of its first token, the
+// number of valid tokens (<= tile width) and the compact slot of its first
+// token (offsets[e] + j * tile width).
+struct TileEntry {
+  int32_t e, row0, nvalid, p0;
+};
+
+enum { kEpiUpQuant = 0, kEpiUpF32 = 1, kEpiDown = 2 };
+
+struct GemmArgs {
+  int fmt, E, K, R;            // reduction length, weight rows per expert
+  const uint8_t* w_sf;         // PREPARED blocked weight scales (NULL for FP8)
+  const uint8_t* b_sf;         // blocked activation scales over padded rows
+  const float* w_gs;           // [E][2] gate/up part scales, or [E] down scales
+  const float* act_scale;      // static activation scale of the B operand, or NULL
+  const float* act_amax;       // amax of the B operand's source (dynamic scale)
+  const TileEntry* tiles;
+  const int32_t* num_tiles;
+  int I;                       // up: h row length
+  uint8_t* hq;                 // up (quantised): h codes [padded rows][I/2]
+  uint8_t* hsf;                //                 h scales, blocked
+  const float* h_scale;        //                 static h scale (NVFP4)
+  float* h32;                  // up (fp32): h [padded rows][I]
+  float* h_amax;               //            amax of h
+  uint16_t* y;                 // down: y_perm [S][ldy] bf16
+  int ldy;
+  int32_t* status;
+};
+
+struct QuantPaddedArgs {
+  int E, K;
+  int64_t S, T;
+  int64_t P;                   // padded rows allocated (writes stay below)
+  const int32_t* offsets;      // [E+1] compact
+  const int32_t* poff;         // [E+1] padded
+  const int32_t* perm_token;   // x source: token of each slot
+  const uint16_t* x;           // [T][K] bf16
+  const float* h32;            // or fp32 rows at padded positions
+  const float* scale;          // static tensor scale or NULL
+  const float* amax;           // dynamic: amax buffer
+  uint8_t* codes;              // [padded rows][K/2 | K]
+  uint8_t* sf;                 // blocked
+  int32_t* status;
+};
+
+cudaError_t launch_plan(const int32_t* offsets, int E, int64_t S, int bn, int32_t* poff, TileEntry* tiles,
+                        int32_t* num_tiles, int max_tiles, int32_t* status, cudaStream_t s);
+cudaError_t launch_quant_padded(const QuantPaddedArgs& a, bool src_x, int fmt, int num_sms, cudaStream_t s);
+cudaError_t launch_grouped_gemm(const GemmArgs& g, int epi, int bn, const void* a_base, int64_t a_rows,
+                                const void* b_base, int64_t b_rows, int num_sms, cudaStream_t s);
+bool tensor_maps_available();
+
+}  // namespace moe

@@ -331,6 +331,9 @@ def moe_set_stage_events(events):
     if events is None:
         _check(lib().moe_set_stage_events(None, 0), "moe_set_stage_events")
         return
+    for e in events:
+        if not e.cuda_event:     # torch creates the CUDA event on first record
+            e.record()
     arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
     _check(lib().moe_set_stage_events(arr, len(events)), "moe_set_stage_events")
 

@@ -1,0 +1,128 @@
+"""Tensor-core grouped GEMM path against the oracle (and against the GEMV
+path), through the C ABI: ragged and skewed expert segments, every format,
+static and dynamic activation scales, and the full-size workloads on sampled
+tokens in the configuration the benchmark times."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from quantized_expert_ffn_top_b200 import ops, synth
+from tests.gpu_helpers import (TOL, ambiguous_tokens, bits_to_dev_bf16, dev_to_f64, device_bank, max_abs_rel,
+                               oracle_bank, routed_inputs)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _path():
+    assert torch.cuda.is_available()
+    ops.moe_set_option(ops.OPT_FFN_PATH, 0)
+    yield
+    ops.moe_set_option(ops.OPT_FFN_PATH, 0)
+
+
+GEMM_CASES = [
+    # name, overrides, static scales, routing skew
+    ("nvfp4-static", dict(fmt="nvfp4", T=200, H=512, E=8, k=2, I=256), True, 1.2),
+    ("nvfp4-dynamic", dict(fmt="nvfp4", T=200, H=512, E=8, k=2, I=256), False, 1.2),
+    ("mxfp4", dict(fmt="mxfp4", T=160, H=512, E=6, k=2, I=256), False, 0.8),
+    ("fp8", dict(fmt="fp8", T=150, H=256, E=10, k=3, I=256), False, 1.0),
+    ("nvfp4-big-expert", dict(fmt="nvfp4", T=400, H=256, E=4, k=1, I=512), True, 3.0),
+    ("nvfp4-some-empty", dict(fmt="nvfp4", T=64, H=256, E=32, k=2, I=256), True, 2.5),
+]
+
+
+def _run(over, static, skew, path):
+    w = synth.workload("tiny", **over)
+    W, _ = oracle_bank(w)
+    a13, a2 = synth.static_act_scales() if static else (None, None)
+    bank = device_bank(W, a13, a2)
+    idx = synth.random_topk_idx(w.T, w.k, w.E, skew=skew)
+    off, perm, inv, _ = oracle.permute(idx, w.E)
+    x = synth.x_bits(w)
+    ws = ops.new_workspace(ops.workspace_size(w.T, w.k, bank, None, 1))
+    ops.moe_set_option(ops.OPT_FFN_PATH, path)
+    y = ops.moe_grouped_ffn(bits_to_dev_bf16(x), w.k, torch.from_numpy(perm).cuda(), torch.from_numpy(off).cuda(),
+                            bank, 1, ws)
+    torch.cuda.synchronize()
+    st = ops.moe_get_device_status(ws)
+    return w, W, x, perm, off, a13, a2, dev_to_f64(y), st
+
+
+@pytest.mark.parametrize("name,over,static,skew", GEMM_CASES)
+def test_gemm_path_matches_oracle(name, over, static, skew):
+    w, W, x, perm, off, a13, a2, y, st = _run(over, static, skew, 2)
+    assert st == 0
+    ry, _ = oracle.grouped_ffn(x, perm, off, W, 1, a13 or 0.0, a2 or 0.0)
+    err = max_abs_rel(y, ry)
+    assert err < TOL, err
+    # per expert too: a wrong tile or a dropped segment shows up here
+    for e in range(w.E):
+        a, b = off[e], off[e + 1]
+        if b > a:
+            assert max_abs_rel(y[a:b], ry[a:b]) < 5 * TOL, e
+
+
+@pytest.mark.parametrize("name,over,static,skew", GEMM_CASES[:4])
+def test_gemm_and_gemv_paths_agree(name, over, static, skew):
+    *_, yg, st1 = _run(over, static, skew, 2)
+    *_, yv, st2 = _run(over, static, skew, 1)
+    assert st1 == 0 and st2 == 0
+    assert max_abs_rel(yg, yv) < TOL
+
+
+@pytest.fixture(scope="module")
+def prefill_layer():
+    w = synth.workload("prefill")
+    W, _ = oracle_bank(w)
+    return w, W
+
+
+def test_prefill_forward_full_size_sampled(prefill_layer):
+    """T=4096 prefill through moe_forward in the benchmark's configuration
+    (tensor-core path, static activation scales), 48 sampled tokens."""
+    w, W = prefill_layer
+    a13, a2 = synth.static_act_scales()
+    bank = device_bank(W, a13, a2)
+    x, wr, b = routed_inputs(w)
+    ws = ops.new_workspace(ops.workspace_size(w.T, w.k, bank, None, 1))
+    out = ops.moe_forward(bits_to_dev_bf16(x), bits_to_dev_bf16(wr), torch.from_numpy(b).cuda(), w.k, bank, None, 1,
+                          ws)
+    assert ops.moe_get_device_status(ws) == 0
+    toks = np.linspace(0, w.T - 1, 48).astype(np.int32)
+    r = oracle.moe_forward(x, wr, b, w.k, W, act=1, a13_static=a13, a2_static=a2, tokens=toks)
+    keep = ~ambiguous_tokens(r["logits"], w.k, 1e-4, boundary_only=True)
+    got = dev_to_f64(out)[toks]
+    err = max_abs_rel(got[keep], r["out"][keep])
+    assert err < TOL, err
+
+
+def test_decode_forward_full_size(prefill_layer):
+    """The decode workload shares the prefill layer's weights (T=4)."""
+    _, W = prefill_layer
+    w = synth.workload("decode")
+    bank = device_bank(W)
+    x, wr, b = routed_inputs(w)
+    ws = ops.new_workspace(ops.workspace_size(w.T, w.k, bank, None, 1))
+    out = ops.moe_forward(bits_to_dev_bf16(x), bits_to_dev_bf16(wr), None, w.k, bank, None, 1, ws)
+    assert ops.moe_get_device_status(ws) == 0
+    r = oracle.moe_forward(x, wr, b, w.k, W, act=1)
+    assert max_abs_rel(dev_to_f64(out), r["out"]) < TOL
+
+
+def test_fp8_shared_forward_full_size():
+    """T=512, E=256 routed top-8 + one shared expert, FP8 W8A8 with dynamic
+    per-tensor activation scales (all tokens: the h scale couples them)."""
+    w = synth.workload("fp8_shared")
+    W, Ws = oracle_bank(w)
+    bank = device_bank(W)
+    sbank = device_bank(Ws)
+    x, wr, b = routed_inputs(w)
+    ws = ops.new_workspace(ops.workspace_size(w.T, w.k, bank, sbank, 1))
+    out = ops.moe_forward(bits_to_dev_bf16(x), bits_to_dev_bf16(wr), None, w.k, bank, sbank, 1, ws)
+    assert ops.moe_get_device_status(ws) == 0
+    r = oracle.moe_forward(x, wr, b, w.k, W, Ws, act=1)
+    keep = ~ambiguous_tokens(r["logits"], w.k, 1e-4, boundary_only=True)
+    err = max_abs_rel(dev_to_f64(out)[keep], r["out"][keep])
+    assert err < TOL, err
