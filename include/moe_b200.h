@@ -238,6 +238,29 @@ moe_status moe_get_device_status(void* ws, moe_stream_t stream, int32_t* host_st
 typedef enum { MOE_OPT_FFN_PATH = 1 } moe_option;
 moe_status moe_set_option(int32_t option, int32_t value);
 
+/* moe_permute for callers that cannot allocate device memory (no workspace
+ * argument).  This entry point is an engineering addition: the pages have no
+ * counterpart to it.  It computes exactly what moe_permute computes.  Callers
+ * that cannot provide a workspace -- a runtime that has handed all free device
+ * memory to its own caches, code running during CUDA stream capture, where
+ * cudaMalloc is not allowed, or a host program with no device allocator -- get
+ * the permutation's scratch (per-chunk expert counts) from a fixed
+ * 256 KiB array that every GPU loading this library holds until the process
+ * exits.
+ *  Limit: ceil(T*k / 2048) * E <= 65536 (e.g. T*k <= 1,048,576 slots for
+ *  E = 128, 524,288 for E = 256); larger sizes return MOE_ERR_WORKSPACE and
+ *  enqueue nothing.
+ *  dev_status (device, nullable, one int32 the caller zeroes): raised to
+ *  MOE_ERR_DEVICE_FAULT for an expert index outside [0, E).
+ *  The first call on a device looks up the array's device address (once per
+ *  device), so make that first call before any stream capture.  The array's
+ *  contents are rewritten by every call, so nothing needs clearing, but calls
+ *  that overlap on the GPU share the array and race: serialise them.  No
+ *  device memory is allocated or freed. */
+moe_status moe_permute_fixed_scratch(const int32_t* topk_idx, int64_t T, int32_t k, int32_t E, int32_t* offsets,
+                                     int32_t* perm_token, int32_t* inv_perm, int32_t* dev_status,
+                                     moe_stream_t stream);
+
 /* Measurement hooks.
  * moe_set_stage_events: when `events` is non-NULL it must hold
  * 2 * MOE_STAGE_COUNT cudaEvent_t handles; moe_forward and moe_grouped_ffn

@@ -15,6 +15,8 @@
 //   3. per chunk again: each warp's base = chunk base + earlier warps'
 //      counts, and each slot's rank among equal experts earlier in its warp
 //      step -> perm_token[p] = t, inv_perm[i] = p.
+#include <mutex>
+
 #include "kernels.cuh"
 
 namespace moe {
@@ -173,3 +175,65 @@ cudaError_t launch_permute(const int32_t* idx, int64_t S, int k, int E, int32_t*
 }
 
 }  // namespace moe
+
+// ---------------------------------------------------------------------------
+// moe_permute without a workspace.
+//
+// Some callers cannot hand this library a workspace: a serving runtime that
+// has already given all free device memory to its expert cache and KV pool,
+// code that runs while a stream is being captured (cudaMalloc is not allowed
+// there), or a host program with no device allocator of its own.  For them,
+// the permutation's only scratch (the per-chunk expert counts) lives in the
+// fixed array below, which every GPU that loads this library holds until the
+// process exits.  The counts are fully rewritten by each call, so nothing has
+// to be cleared first; calls that overlap on the GPU share the array and race.
+// ---------------------------------------------------------------------------
+namespace moe {
+namespace {
+
+constexpr int kFixedScratchInts = 65536;  // 256 KiB: nchunks * E <= 65536
+static __device__ __align__(256) int32_t g_fixed_perm_scratch[kFixedScratchInts];
+
+constexpr int kMaxDevices = 64;
+int32_t* g_fixed_scratch_ptr[kMaxDevices] = {nullptr};
+std::mutex g_fixed_scratch_mu;
+
+// Device address of the array on the current device, looked up once per device.
+cudaError_t fixed_scratch_ptr(int32_t** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(g_fixed_scratch_mu);
+  if (!g_fixed_scratch_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_fixed_perm_scratch);
+    if (e != cudaSuccess) return e;
+    g_fixed_scratch_ptr[dev] = static_cast<int32_t*>(p);
+  }
+  *out = g_fixed_scratch_ptr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+}  // namespace moe
+
+extern "C" moe_status moe_permute_fixed_scratch(const int32_t* topk_idx, int64_t T, int32_t k, int32_t E,
+                                                int32_t* offsets, int32_t* perm_token, int32_t* inv_perm,
+                                                int32_t* dev_status, moe_stream_t stream) {
+  using namespace moe;
+  if (T < 0 || k < 1 || E < 1 || E > 1024 || T * (int64_t)k > INT32_MAX) return MOE_ERR_INVALID_ARG;
+  if (!offsets || (T > 0 && (!topk_idx || !perm_token || !inv_perm))) return MOE_ERR_INVALID_ARG;
+  const int64_t S = T * k;
+  const int64_t nchunks = (S + kChunk - 1) / kChunk;
+  if (nchunks * (int64_t)E > kFixedScratchInts) return MOE_ERR_WORKSPACE;  // beyond the fixed capacity
+  int32_t* scratch = nullptr;
+  if (fixed_scratch_ptr(&scratch) != cudaSuccess) return MOE_ERR_CUDA;
+  PermuteScratch ps;
+  ps.chunk_counts = scratch;
+  ps.nchunks = (int)nchunks;
+  return launch_permute(topk_idx, S, k, E, offsets, perm_token, inv_perm, ps, dev_status,
+                        reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? MOE_OK
+             : MOE_ERR_CUDA;
+}

@@ -27,6 +27,7 @@ EXPORTED = (
     "moe_status_string", "moe_version", "moe_set_option", "moe_workspace_size", "moe_prepared_weights_size",
     "moe_prepare_weights", "moe_quantize", "moe_route", "moe_route_logits", "moe_permute", "moe_grouped_ffn",
     "moe_combine", "moe_forward", "moe_get_device_status", "moe_set_stage_events", "moe_kernel_launch_count",
+    "moe_permute_fixed_scratch",
 )
 STAGES = ("route", "permute", "act_quant", "ffn_up", "ffn_down", "shared", "combine")
 
@@ -83,6 +84,7 @@ def _declare(L):
         "moe_get_device_status": ([P, P, ctypes.POINTER(ctypes.c_int32)], ctypes.c_int),
         "moe_set_stage_events": ([ctypes.POINTER(ctypes.c_void_p), i32], ctypes.c_int),
         "moe_kernel_launch_count": ([], ctypes.c_uint64),
+        "moe_permute_fixed_scratch": ([P, i64, i32, i32, P, P, P, P, P], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -183,7 +185,7 @@ def moe_prepare_weights(bank: WeightBank, stream=None) -> WeightBank:
                    w2=view(out.w2, bank.E * bank.H * rb2),
                    w13_sf=view(out.w13_sf, bank.E * 2 * bank.I * bank.H // bs) if bs else None,
                    w2_sf=view(out.w2_sf, bank.E * bank.H * bank.I // bs) if bs else None,
-                   keep=[dst, bank])
+                   keep=[dst])
 
 
 # ------------------------------------------------------------ entry points --
