@@ -139,6 +139,8 @@ def build_layer(ops, synth, torch, w, static: bool):
         bank.a2_gs = torch.tensor([a2], dtype=torch.float32, device="cuda")
     prepared = ops.moe_prepare_weights(bank)
     torch.cuda.synchronize()
+    del bank
+    torch.cuda.empty_cache()
     x = synth.cuda_normal((w.T, w.H), 1.0, synth.TID_X, dtype=torch.bfloat16)
     wr = synth.cuda_normal((w.E, w.H), w.wr_std, synth.TID_WR, dtype=torch.bfloat16)
     bias = synth.cuda_router_bias(w)
@@ -169,61 +171,77 @@ def algorithmic(w, bank_fmt: str, offsets: np.ndarray):
 
 
 def time_forward(ops, torch, layer, w, act, steps, warmup, flush, stage=True, host_io=False):
+    """Times `steps` forwards.  Device-resident runs replay a CUDA graph of
+    moe_forward (one graph launch per step, L2 flushed before each, CUDA
+    events around each replay); the per-stage split comes from a second graph
+    that records the library's stage events.  host_io runs time the eager
+    user call with the host<->device copies inside the events."""
     prepared, x, wr, bias = layer
-    dev = x.device
     ws = ops.new_workspace(ops.workspace_size(w.T, w.k, prepared, None, act))
     out = torch.empty_like(x)
+    stream = torch.cuda.current_stream()
+
+    def fwd():
+        ops.moe_forward(x, wr, bias, w.k, prepared, None, act, ws, out=out)
+
+    l0 = ops.moe_kernel_launch_count()
+    for _ in range(max(warmup, 1)):
+        fwd()
+    torch.cuda.synchronize()
+    per_step_launches = (ops.moe_kernel_launch_count() - l0) // max(warmup, 1)
+    if ops.moe_get_device_status(ws) != 0:
+        raise RuntimeError("device status reported a fault during warm-up")
+    step_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    stages = {}
     if host_io:
         x_host = x.cpu().pin_memory()
         out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    n_ev = 2 * len(ops.STAGES)
-    stream = torch.cuda.current_stream()
-
-    def one(i, evs=None, rec=None):
-        if evs is not None:
-            ops.moe_set_stage_events(evs)
-        if rec is not None:
-            rec[0].record(stream)
-        if host_io:
+        torch.cuda.synchronize()
+        for i in range(steps):
+            flush.zero_()
+            step_evs[i][0].record(stream)
             x.copy_(x_host, non_blocking=True)
-        ops.moe_forward(x, wr, bias, w.k, prepared, None, act, ws, out=out)
-        if host_io:
+            fwd()
             out_host.copy_(out, non_blocking=True)
-        if rec is not None:
-            rec[1].record(stream)
-        if evs is not None:
-            ops.moe_set_stage_events(None)
-
-    for i in range(warmup):
-        one(i)
-    torch.cuda.synchronize()
-    if ops.moe_get_device_status(ws) != 0:
-        raise RuntimeError("device status reported a fault during warm-up")
-    stage_evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(steps)] if stage else None
-    step_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
-    launches0 = ops.moe_kernel_launch_count()
-    torch.cuda.synchronize()
-    for i in range(steps):
-        flush.zero_()
-        one(i, stage_evs[i] if stage else None, step_evs[i])
-    torch.cuda.synchronize()
-    launches = ops.moe_kernel_launch_count() - launches0
+            step_evs[i][1].record(stream)
+        torch.cuda.synchronize()
+    else:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            fwd()
+        torch.cuda.synchronize()
+        for i in range(steps):
+            flush.zero_()
+            step_evs[i][0].record(stream)
+            graph.replay()
+            step_evs[i][1].record(stream)
+        torch.cuda.synchronize()
+        if stage:
+            evs = [torch.cuda.Event(enable_timing=True) for _ in range(2 * len(ops.STAGES))]
+            ops.moe_set_stage_events(evs)
+            g2 = torch.cuda.CUDAGraph()
+            try:
+                with torch.cuda.graph(g2):
+                    fwd()
+            finally:
+                ops.moe_set_stage_events(None)
+            acc = {n: [] for n in ops.STAGES}
+            for i in range(steps):
+                flush.zero_()
+                g2.replay()
+                torch.cuda.synchronize()
+                for si, name in enumerate(ops.STAGES):
+                    try:
+                        acc[name].append(evs[2 * si].elapsed_time(evs[2 * si + 1]))
+                    except RuntimeError:
+                        pass
+            stages = {n: float(np.mean(v)) for n, v in acc.items() if v}
+            del g2
+        del graph
     per_step = [a.elapsed_time(b) for a, b in step_evs]
-    stages = {}
-    if stage:
-        for si, name in enumerate(ops.STAGES):
-            vals = []
-            for evs in stage_evs:
-                try:
-                    vals.append(evs[2 * si].elapsed_time(evs[2 * si + 1]))
-                except RuntimeError:
-                    pass
-            if vals:
-                stages[name] = float(np.mean(vals))
-    # routing histogram of the last step (for the algorithmic byte count)
     idx, _ = ops.moe_route(x, wr, bias, w.k, ops.new_workspace(ops.workspace_size(w.T, w.k, prepared, None, act)))
     off, _, _ = ops.moe_permute(idx, w.E, ops.new_workspace(1 << 24))
-    return dict(ms=per_step, stages=stages, launches=launches, offsets=off.cpu().numpy(),
+    return dict(ms=per_step, stages=stages, launches=per_step_launches * steps, offsets=off.cpu().numpy(),
                 status=ops.moe_get_device_status(ws))
 
 

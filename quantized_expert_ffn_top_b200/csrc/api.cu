@@ -52,8 +52,10 @@ int g_ffn_path = 0;  // MOE_OPT_FFN_PATH
 cudaEvent_t g_stage_events[2 * MOE_STAGE_COUNT];
 bool g_stage_on = false;
 
+// External records, so that events captured into a CUDA graph stay readable
+// by the caller after each replay.
 void stage_mark(int stage, bool end, cudaStream_t s) {
-  if (g_stage_on) cudaEventRecord(g_stage_events[2 * stage + (end ? 1 : 0)], s);
+  if (g_stage_on) cudaEventRecordWithFlags(g_stage_events[2 * stage + (end ? 1 : 0)], s, cudaEventRecordExternal);
 }
 
 int num_sms() {
@@ -97,14 +99,20 @@ moe_status check_weights(const moe_weights* w, bool need_prepared) {
 }
 
 // ---------------------------------------------------------------- layouts --
+// Router scratch: logits (when the caller passes none) and the token tiles
+// of the tensor-core router GEMM.
 struct RouteWs {
   Scalars head;
   float* logits;
+  TileEntry* tiles;
+  int32_t* ntiles;
 };
-RouteWs carve_route(Carver& c, int64_t T, int E) {
+RouteWs carve_route(Carver& c, int64_t T, int E, bool need_logits) {
   RouteWs r;
   r.head = carve_head(c);
-  r.logits = c.take<float>((size_t)T * E);
+  r.logits = c.take<float>(need_logits ? (size_t)T * E : 0);
+  r.tiles = c.take<TileEntry>((size_t)(T / 128 + 1));
+  r.ntiles = c.take<int32_t>(1);
   return r;
 }
 
@@ -159,6 +167,8 @@ FfnScratch carve_ffn(Carver& c, int64_t S, const moe_weights* w) {
 struct ForwardWs {
   Scalars head;
   float* logits;
+  TileEntry* rtiles;
+  int32_t* rntiles;
   int32_t* idx;
   float* w;
   int32_t* offsets;
@@ -178,6 +188,8 @@ ForwardWs carve_forward(Carver& c, int64_t T, int k, const moe_weights* routed, 
   const int64_t S = T * k;
   f.head = carve_head(c);
   f.logits = c.take<float>((size_t)T * E);
+  f.rtiles = c.take<TileEntry>((size_t)(T / 128 + 1));
+  f.rntiles = c.take<int32_t>(1);
   f.idx = c.take<int32_t>((size_t)S);
   f.w = c.take<float>((size_t)S);
   f.offsets = c.take<int32_t>((size_t)E + 1);
@@ -208,6 +220,15 @@ __global__ void identity_routing_kernel(int64_t T, int32_t* offsets, int32_t* pe
     offsets[0] = 0;
     offsets[1] = (int32_t)T;
   }
+}
+
+// Router logits: tcgen05 bf16 GEMM when the shapes allow it and the batch is
+// large enough to matter, CUDA cores otherwise.
+cudaError_t run_router(const uint16_t* x, int64_t T, int H, const uint16_t* wr, const float* bias, int E,
+                       float* logits, TileEntry* tiles, int32_t* ntiles, int32_t* status, cudaStream_t s) {
+  if (T >= 128 && E % 128 == 0 && H % 64 == 0 && tensor_maps_available())
+    return launch_router_gemm(x, T, H, wr, bias, E, logits, tiles, ntiles, status, num_sms(), s);
+  return launch_router_logits(x, T, H, wr, bias, E, logits, s);
 }
 
 bool gemm_shapes_ok(const moe_weights* w, int act) {
@@ -492,12 +513,12 @@ moe_status moe_route(const uint16_t* x, int64_t T, int32_t H, const uint16_t* wr
   if (T > 0 && (!x || !wr || !topk_idx || !topk_w)) return MOE_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(wr)) return MOE_ERR_INVALID_ARG;
   Carver c(ws);
-  RouteWs r = carve_route(c, logits ? 0 : T, E);
+  RouteWs r = carve_route(c, T, E, logits == nullptr);
   if (!ws || ws_bytes < c.off) return MOE_ERR_WORKSPACE;
   if (T == 0) return MOE_OK;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   float* L = logits ? logits : r.logits;
-  MOE_TRY(launch_router_logits(x, T, H, wr, bias, E, L, s));
+  MOE_TRY(run_router(x, T, H, wr, bias, E, L, r.tiles, r.ntiles, r.head.status, s));
   return cuda_status(launch_topk(L, T, E, k, topk_idx, topk_w, r.head.status, s));
 }
 
@@ -582,7 +603,7 @@ moe_status moe_forward(const uint16_t* x, int64_t T, const uint16_t* wr, const f
   const int64_t S = T * k;
   // 1. router
   stage_mark(MOE_STAGE_ROUTE, false, s);
-  MOE_TRY(launch_router_logits(x, T, H, wr, bias, E, f.logits, s));
+  MOE_TRY(run_router(x, T, H, wr, bias, E, f.logits, f.rtiles, f.rntiles, f.head.status, s));
   MOE_TRY(launch_topk(f.logits, T, E, k, f.idx, f.w, f.head.status, s));
   stage_mark(MOE_STAGE_ROUTE, true, s);
   // 2. histogram + permutation

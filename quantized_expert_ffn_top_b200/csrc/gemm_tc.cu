@@ -41,8 +41,9 @@ namespace {
 
 template <int FMT>
 struct FmtTraits {
-  static constexpr int kBK = FMT == MOE_FMT_FP8 ? 128 : 256;      // K elements per stage (128 bytes per row)
-  static constexpr int kMmaK = FMT == MOE_FMT_FP8 ? 32 : 64;
+  // K elements per stage (128 bytes per row) and per MMA
+  static constexpr int kBK = FMT == kFmtBF16 ? 64 : (FMT == MOE_FMT_FP8 ? 128 : 256);
+  static constexpr int kMmaK = FMT == kFmtBF16 ? 16 : (FMT == MOE_FMT_FP8 ? 32 : 64);
   static constexpr int kSteps = kBK / kMmaK;                        // MMAs per stage
   static constexpr int kBs = FMT == MOE_FMT_NVFP4 ? 16 : (FMT == MOE_FMT_MXFP4 ? 32 : 0);
   static constexpr int kGroups = kBs ? kBK / (4 * kBs) : 0;         // 4-column scale groups per stage
@@ -64,7 +65,9 @@ struct Cfg {
   static constexpr uint32_t kSfbCol = kSfaCol + F::kGroups * 4;
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kTx = kA + kB + kSFA + kSFB;
-  static constexpr int kSmem = kStages * kStage + 1024 /*align*/ + 1024 /*barriers etc.*/;
+  static constexpr int kEpiTile = 16 * 32 * 4;  // per warp pair: 16 tokens x 32 rows, fp32
+  static constexpr int kSmem = kStages * kStage + 1024 /*align*/ + 1024 /*barriers etc.*/ +
+                               (kEpiWarps / 2) * kEpiTile;
   static_assert(kSfbCol + F::kGroups * 4 * (BN / 128) <= kTmemCols, "tensor memory overflow");
 };
 
@@ -90,7 +93,7 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN>::kThreads, 1)
   uint64_t* tempty = tfull + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* xmax = reinterpret_cast<float*>(tmem_slot + 4);  // [kEpiWarps][16] MXFP4 block max exchange
+  float* epi_tiles = reinterpret_cast<float*>(ctrl + 1024);  // [kEpiWarps / 2][16 tokens][32]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -205,8 +208,10 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN>::kThreads, 1)
               const uint32_t id = (uint32_t)(kk & 1) * 2;  // two MMAs share one group of four e8m0 scales
               tc::mma_mxf4(d, da, db, tc::idesc_mxf4(n_mma, true, id, id), tmem + C::kSfaCol + 4 * (kk >> 1),
                            tmem + C::kSfbCol + (kk >> 1) * 4 * (BN / 128), accum);
-            } else {
+            } else if (FMT == MOE_FMT_FP8) {
               tc::mma_f8(d, da, db, tc::idesc_f8(n_mma), accum);
+            } else {
+              tc::mma_bf16(d, da, db, tc::idesc_bf16(n_mma), accum);
             }
           }
           tc::mma_commit(&empty[stage]);
@@ -245,7 +250,19 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN>::kThreads, 1)
       const int ncol = min(BN, (te.nvalid + 15) & ~15);
       const int c_lo = half * (BN / 2), c_hi = min(ncol, (half + 1) * (BN / 2));
       const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
-      if (EPI == kEpiDown) {
+      if (EPI == kEpiLogits) {
+        const int o = mt * 128 + q * 32 + lane;  // expert
+        const float b = g.bias ? __ldg(g.bias + o) : 0.0f;
+        for (int c0 = c_lo; c0 < c_hi; c0 += 16) {
+          float v[16];
+          tc::tmem_ld16(tbase + c0, v);
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const int tok = c0 + c;
+            if (tok < te.nvalid) g.logits[(size_t)(te.p0 + tok) * g.ldy + o] = v[c] + b;
+          }
+        }
+      } else if (EPI == kEpiDown) {
         const int o = mt * 128 + q * 32 + lane;
         const float sc = (FMT == MOE_FMT_MXFP4) ? 1.0f : __ldg(g.w_gs + te.e) * gact;
         for (int c0 = c_lo; c0 < c_hi; c0 += 16) {
@@ -258,10 +275,18 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN>::kThreads, 1)
           }
         }
       } else {
+        // gate|up rows interleave (even lane gate, odd lane up): one shuffle
+        // pairs them, SwiGLU runs on every lane, and the h values go through
+        // a shared-memory tile so that each lane then owns 8 consecutive
+        // features of one token (half a NVFP4 block, a quarter of an MXFP4
+        // block) for the block maximum, the codes and 16-byte stores.
         const int part = lane & 1;
         const float sc = (FMT == MOE_FMT_MXFP4) ? 1.0f : __ldg(g.w_gs + te.e * 2 + part) * gact;
-        const int f_base = mt * 64 + q * 16;       // this warp's 16 features
-        const int f = f_base + (lane >> 1);
+        const int pp = q & 1;                                  // position in the warp pair
+        float* tile = epi_tiles + (ew >> 1) * (16 * 32);       // [16 tokens][32 features] of the pair
+        const int fl = lane >> 1;                              // feature within the warp's 16
+        const int f_pair = mt * 64 + (q >> 1) * 32;            // first feature of the pair
+        const int bar = 1 + (ew >> 1);
         for (int c0 = c_lo; c0 < c_hi; c0 += 16) {
           float v[16];
           tc::tmem_ld16(tbase + c0, v);
@@ -271,55 +296,53 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN>::kThreads, 1)
             const float recv = __shfl_xor_sync(0xffffffffu, part ? a : b, 1);
             const float gg = part ? recv : a;
             const float uu = part ? b : recv;
-            const float h = gg / (1.0f + __expf(-gg)) * uu;
-            const int tok = c0 + 2 * i + part;
-            const bool valid = tok < te.nvalid;
-            if (EPI == kEpiUpF32) {
-              if (valid) {
-                g.h32[(size_t)(te.row0 + tok) * g.I + f] = h;
-                hmax = fmaxf(hmax, fabsf(h));
-              }
+            const float h = __fdividef(gg, 1.0f + __expf(-gg)) * uu;
+            tile[(2 * i + part) * 32 + pp * 16 + fl] = h;
+          }
+          asm volatile("bar.sync %0, 64;" ::"r"(bar) : "memory");
+          // each of the pair's 64 threads: token tl, features [8 * qq, 8 * qq + 8)
+          const int tid = pp * 32 + lane;
+          const int tl = tid >> 2, qq = tid & 3;
+          const float4 lo = *reinterpret_cast<const float4*>(tile + tl * 32 + 8 * qq);
+          const float4 hi = *reinterpret_cast<const float4*>(tile + tl * 32 + 8 * qq + 4);
+          float hv[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+          const int tok = c0 + tl;
+          const bool valid = tok < te.nvalid;
+          const size_t row = (size_t)(te.row0 + tok);
+          if (EPI == kEpiUpF32) {
+            if (valid) {
+              float4* dst = reinterpret_cast<float4*>(g.h32 + row * g.I + f_pair + 8 * qq);
+              dst[0] = lo;
+              dst[1] = hi;
+#pragma unroll
+              for (int j = 0; j < 8; ++j) hmax = fmaxf(hmax, fabsf(hv[j]));
+            }
+          } else {
+            float bmax = 0.0f;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) bmax = fmaxf(bmax, fabsf(hv[j]));
+            uint32_t word = 0, scode = 0;
+            if (FMT == MOE_FMT_NVFP4) {
+              bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 1));   // 16-feature block
+              float r;
+              nvfp4_block_scale(bmax, g2, scode, r);
+              word = r != 0.0f ? e2m1_encode8(hv, r) : 0u;
             } else {
-              // quantise h: one 16-feature block per warp and token (NVFP4),
-              // two warps per 32-feature block (MXFP4)
-              float bmax = fabsf(h);
-#pragma unroll
-              for (int o = 2; o < 32; o <<= 1) bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, o));
-              uint32_t code = 0, scode = 0;
-              if (FMT == MOE_FMT_NVFP4) {
-                float r;
-                nvfp4_block_scale(bmax, g2, scode, r);
-                code = r != 0.0f ? (e2m1x2_encode(__fmul_rn(h, r), 0.0f) & 0xFu) : 0u;
-              } else {
-                // exchange the 16-feature maxima with the partner warp (q ^ 1)
-                const int bar = 1 + ew / 2;
-                if (lane < 2) xmax[ew * 16 + 2 * i + lane] = bmax;
-                asm volatile("bar.sync %0, 64;" ::"r"(bar) : "memory");
-                const float other = xmax[(ew ^ 1) * 16 + 2 * i + part];
-                asm volatile("bar.sync %0, 64;" ::"r"(bar) : "memory");
-                float inv;
-                mxfp4_block_scale(fmaxf(bmax, other), scode, inv);
-                code = e2m1x2_encode(__fmul_rn(h, inv), 0.0f) & 0xFu;
-              }
-              // pack: byte j of the warp's 8 holds features 2j (lo) and 2j+1 (hi)
-              const uint32_t hi = __shfl_down_sync(0xffffffffu, code, 2);
-              const uint32_t byte = code | (hi << 4);
-              uint32_t w0 = 0, w1 = 0;
-#pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                w0 |= (__shfl_sync(0xffffffffu, byte, 4 * j + part) & 0xFFu) << (8 * j);
-                w1 |= (__shfl_sync(0xffffffffu, byte, 16 + 4 * j + part) & 0xFFu) << (8 * j);
-              }
-              if (lane < 2 && valid) {
-                const size_t row = (size_t)(te.row0 + tok);
-                *reinterpret_cast<uint2*>(g.hq + row * (g.I / 2) + f_base / 2) = make_uint2(w0, w1);
-                if (FMT == MOE_FMT_NVFP4)
-                  g.hsf[sf_blocked_offset((int64_t)row, f_base / 16, g.I / 16)] = (uint8_t)scode;
-                else if ((q & 1) == 0)
-                  g.hsf[sf_blocked_offset((int64_t)row, f_base / 32, g.I / 32)] = (uint8_t)scode;
-              }
+              bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 1));   // 32-feature block
+              bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 2));
+              float inv;
+              mxfp4_block_scale(bmax, scode, inv);
+              word = e2m1_encode8(hv, inv);
+            }
+            if (valid) {
+              *reinterpret_cast<uint32_t*>(g.hq + row * (g.I / 2) + f_pair / 2 + 4 * qq) = word;
+              if (FMT == MOE_FMT_NVFP4 && (qq & 1) == 0)
+                g.hsf[sf_blocked_offset((int64_t)row, (f_pair + 8 * qq) / 16, g.I / 16)] = (uint8_t)scode;
+              if (FMT == MOE_FMT_MXFP4 && qq == 0)
+                g.hsf[sf_blocked_offset((int64_t)row, f_pair / 32, g.I / 32)] = (uint8_t)scode;
             }
           }
+          asm volatile("bar.sync %0, 64;" ::"r"(bar) : "memory");
         }
       }
       tc::fence_before_sync();
@@ -383,7 +406,7 @@ cudaError_t launch_cfg(const GemmArgs& g, const void* a_base, int64_t a_rows, co
                        int num_sms, cudaStream_t s) {
   using C = Cfg<FMT, EPI, BN>;
   CUtensorMap ma, mb;
-  const int64_t rb = FMT == MOE_FMT_FP8 ? g.K : g.K / 2;
+  const int64_t rb = FMT == kFmtBF16 ? 2 * (int64_t)g.K : (FMT == MOE_FMT_FP8 ? g.K : g.K / 2);
   if (!make_map(&ma, a_base, a_rows, rb, 128) || !make_map(&mb, b_base, b_rows, rb, BN))
     return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<FMT, EPI, BN>,
@@ -423,6 +446,48 @@ cudaError_t launch_grouped_gemm(const GemmArgs& g, int epi, int bn, const void* 
 }
 
 bool tensor_maps_available() { return encode_fn() != nullptr; }
+
+__global__ void dense_plan_kernel(int64_t T, int bn, TileEntry* __restrict__ tiles, int32_t* __restrict__ num_tiles) {
+  const int n = (int)((T + bn - 1) / bn);
+  for (int j = blockIdx.x * blockDim.x + threadIdx.x; j < n; j += gridDim.x * blockDim.x) {
+    TileEntry te;
+    te.e = 0;
+    te.row0 = j * bn;
+    te.nvalid = (int)min((int64_t)bn, T - (int64_t)j * bn);
+    te.p0 = j * bn;
+    tiles[j] = te;
+  }
+  if (blockIdx.x == 0 && threadIdx.x == 0) *num_tiles = n;
+}
+
+cudaError_t launch_dense_plan(int64_t T, int bn, TileEntry* tiles, int32_t* num_tiles, cudaStream_t s) {
+  dense_plan_kernel<<<1, 256, 0, s>>>(T, bn, tiles, num_tiles);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_router_gemm(const uint16_t* x, int64_t T, int H, const uint16_t* wr, const float* bias, int E,
+                               float* logits, TileEntry* tiles, int32_t* num_tiles, int32_t* status, int num_sms,
+                               cudaStream_t s) {
+  constexpr int kBN = 128;
+  cudaError_t e = launch_dense_plan(T, kBN, tiles, num_tiles, s);
+  if (e != cudaSuccess) return e;
+  GemmArgs g;
+  memset(&g, 0, sizeof(g));
+  g.fmt = kFmtBF16;
+  g.E = 1;
+  g.K = H;
+  g.R = E;
+  g.tiles = tiles;
+  g.num_tiles = num_tiles;
+  g.logits = logits;
+  g.bias = bias;
+  g.ldy = E;
+  g.status = status;
+  const int64_t ntiles = (T + kBN - 1) / kBN * (E / 128);
+  const int grid = (int)(ntiles < num_sms ? ntiles : num_sms);
+  return launch_cfg<kFmtBF16, kEpiLogits, kBN>(g, wr, E, x, T, grid, s);
+}
 
 // ---------------------------------------------------------------- planning --
 // One block: padded offsets (every expert segment starts on a multiple of 128
@@ -487,32 +552,38 @@ cudaError_t launch_plan(const int32_t* offsets, int E, int64_t S, int bn, int32_
 
 // ---------------------------------------------------- padded quantisation --
 // Quantises activation rows into the padded, blocked layout the GEMM reads.
-// Source row of slot p: x[perm_token[p]] (bf16, SRC_X) or h32[padded row]
-// (fp32); destination: padded row poff[e] + (p - offsets[e]).
+// One warp per slot p: its source row is x[perm_token[p]] (bf16, SRC_X) or
+// h32[padded row] (fp32), its destination the padded row poff[e] + (p -
+// offsets[e]); lane l quantises scale blocks l, l + 32, ... of the row.
 template <int FMT, bool SRC_X>
 __global__ void __launch_bounds__(256) quant_padded_kernel(QuantPaddedArgs a) {
   constexpr int bs = FMT == MOE_FMT_MXFP4 ? 32 : 16;
   const int nb = a.K / bs;
-  const int64_t total = a.S * nb;
+  const int lane = threadIdx.x & 31;
   const float scale = act_scale_of(FMT, a.scale, a.amax);
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t it = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; it < total; it += stride) {
-    const int p = (int)(it / nb), b = (int)(it % nb);
-    const int e = segment_of(a.offsets, a.E, p);
-    const int64_t row = (int64_t)__ldg(a.poff + e) + (p - __ldg(a.offsets + e));
-    if (row < 0 || row >= a.P || p < __ldg(a.offsets + e)) {
-      if (b == 0) raise_status(a.status, MOE_ERR_DEVICE_FAULT);
+  const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t p = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); p < a.S; p += warps) {
+    int64_t row = -1;
+    int t = -1;
+    if (lane == 0) {
+      const int e = segment_of(a.offsets, a.E, (int)p);
+      const int32_t o = __ldg(a.offsets + e);
+      row = (int64_t)__ldg(a.poff + e) + (p - o);
+      if (row < 0 || row >= a.P || p < o) row = -1;
+      if (SRC_X) {
+        t = __ldg(a.perm_token + p);
+        if (t < 0 || t >= a.T) row = -1;
+      }
+    }
+    row = __shfl_sync(0xffffffffu, row, 0);
+    t = __shfl_sync(0xffffffffu, t, 0);
+    if (row < 0) {
+      if (lane == 0) raise_status(a.status, MOE_ERR_DEVICE_FAULT);
       continue;
     }
-    float v[bs];
-    float bmax = 0.0f;
-    if (SRC_X) {
-      const int t = __ldg(a.perm_token + p);
-      if (t < 0 || t >= a.T) {
-        if (b == 0) raise_status(a.status, MOE_ERR_DEVICE_FAULT);
-#pragma unroll
-        for (int i = 0; i < bs; ++i) v[i] = 0.0f;
-      } else {
+    for (int b = lane; b < nb; b += 32) {
+      float v[bs];
+      if (SRC_X) {
         const uint16_t* src = a.x + (int64_t)t * a.K + b * bs;
 #pragma unroll
         for (int i = 0; i < bs; i += 8) {
@@ -524,56 +595,55 @@ __global__ void __launch_bounds__(256) quant_padded_kernel(QuantPaddedArgs a) {
             v[i + 2 * j + 1] = __uint_as_float(ww[j] & 0xFFFF0000u);
           }
         }
+      } else {
+        const float* src = a.h32 + row * a.K + b * bs;
+#pragma unroll
+        for (int i = 0; i < bs; i += 4) {
+          const float4 w = *reinterpret_cast<const float4*>(src + i);
+          v[i] = w.x;
+          v[i + 1] = w.y;
+          v[i + 2] = w.z;
+          v[i + 3] = w.w;
+        }
       }
-    } else {
-      const float* src = a.h32 + row * a.K + b * bs;
+      float bmax = 0.0f;
 #pragma unroll
-      for (int i = 0; i < bs; i += 4) {
-        const float4 w = *reinterpret_cast<const float4*>(src + i);
-        v[i] = w.x;
-        v[i + 1] = w.y;
-        v[i + 2] = w.z;
-        v[i + 3] = w.w;
+      for (int i = 0; i < bs; ++i) bmax = fmaxf(bmax, fabsf(v[i]));
+      if constexpr (FMT == MOE_FMT_NVFP4) {
+        uint32_t sc;
+        float r;
+        nvfp4_block_scale(bmax, scale, sc, r);
+        *reinterpret_cast<uint2*>(a.codes + row * (a.K / 2) + b * 8) = nvfp4_encode16(v, r);
+        a.sf[sf_blocked_offset(row, b, nb)] = (uint8_t)sc;
+      } else if constexpr (FMT == MOE_FMT_MXFP4) {
+        uint32_t c;
+        float inv;
+        mxfp4_block_scale(bmax, c, inv);
+        uint4 w;
+        w.x = e2m1_encode8(v, inv);
+        w.y = e2m1_encode8(v + 8, inv);
+        w.z = e2m1_encode8(v + 16, inv);
+        w.w = e2m1_encode8(v + 24, inv);
+        *reinterpret_cast<uint4*>(a.codes + row * (a.K / 2) + b * 16) = w;
+        a.sf[sf_blocked_offset(row, b, nb)] = (uint8_t)c;
+      } else {
+        const float inv = __frcp_rn(scale);
+        uint4 w;
+        uint32_t* pw = &w.x;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          pw[i] = e4m3x2_encode(__fmul_rn(v[4 * i], inv), __fmul_rn(v[4 * i + 1], inv)) |
+                  (e4m3x2_encode(__fmul_rn(v[4 * i + 2], inv), __fmul_rn(v[4 * i + 3], inv)) << 16);
+        *reinterpret_cast<uint4*>(a.codes + row * a.K + b * 16) = w;
       }
-    }
-#pragma unroll
-    for (int i = 0; i < bs; ++i) bmax = fmaxf(bmax, fabsf(v[i]));
-    if constexpr (FMT == MOE_FMT_NVFP4) {
-      uint32_t sc;
-      float r;
-      nvfp4_block_scale(bmax, scale, sc, r);
-      *reinterpret_cast<uint2*>(a.codes + row * (a.K / 2) + b * 8) = nvfp4_encode16(v, r);
-      a.sf[sf_blocked_offset(row, b, nb)] = (uint8_t)sc;
-    } else if constexpr (FMT == MOE_FMT_MXFP4) {
-      uint32_t c;
-      float inv;
-      mxfp4_block_scale(bmax, c, inv);
-      uint4 w;
-      w.x = e2m1_encode8(v, inv);
-      w.y = e2m1_encode8(v + 8, inv);
-      w.z = e2m1_encode8(v + 16, inv);
-      w.w = e2m1_encode8(v + 24, inv);
-      *reinterpret_cast<uint4*>(a.codes + row * (a.K / 2) + b * 16) = w;
-      a.sf[sf_blocked_offset(row, b, nb)] = (uint8_t)c;
-    } else {
-      const float inv = __frcp_rn(scale);
-      uint4 w;
-      uint32_t* pw = &w.x;
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-        pw[i] = e4m3x2_encode(__fmul_rn(v[4 * i], inv), __fmul_rn(v[4 * i + 1], inv)) |
-                (e4m3x2_encode(__fmul_rn(v[4 * i + 2], inv), __fmul_rn(v[4 * i + 3], inv)) << 16);
-      *reinterpret_cast<uint4*>(a.codes + row * a.K + b * 16) = w;
     }
   }
 }
 
 cudaError_t launch_quant_padded(const QuantPaddedArgs& a, bool src_x, int fmt, int num_sms, cudaStream_t s) {
-  const int bs = fmt == MOE_FMT_MXFP4 ? 32 : 16;
-  const int64_t total = a.S * (a.K / bs);
-  if (total == 0) return cudaSuccess;
-  const int64_t blocks = (total + 255) / 256;
-  const int grid = (int)(blocks < (int64_t)num_sms * 16 ? blocks : (int64_t)num_sms * 16);
+  if (a.S == 0) return cudaSuccess;
+  const int64_t blocks = (a.S + 7) / 8;
+  const int grid = (int)(blocks < (int64_t)num_sms * 8 ? blocks : (int64_t)num_sms * 8);
 #define MOE_QP(F)                                                              \
   if (src_x) quant_padded_kernel<F, true><<<grid, 256, 0, s>>>(a);           \
   else quant_padded_kernel<F, false><<<grid, 256, 0, s>>>(a);

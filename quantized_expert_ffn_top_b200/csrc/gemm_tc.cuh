@@ -14,7 +14,10 @@ struct TileEntry {
   int32_t e, row0, nvalid, p0;
 };
 
-enum { kEpiUpQuant = 0, kEpiUpF32 = 1, kEpiDown = 2 };
+enum { kEpiUpQuant = 0, kEpiUpF32 = 1, kEpiDown = 2, kEpiLogits = 3 };
+
+// Operand type of the router GEMM (bf16 x and Wr) next to the moe_fmt values.
+constexpr int kFmtBF16 = 4;
 
 struct GemmArgs {
   int fmt, E, K, R;            // reduction length, weight rows per expert
@@ -33,6 +36,8 @@ struct GemmArgs {
   float* h_amax;               //            amax of h
   uint16_t* y;                 // down: y_perm [S][ldy] bf16
   int ldy;
+  float* logits;               // router: logits [T][ldy] fp32 (+ bias)
+  const float* bias;
   int32_t* status;
 };
 
@@ -58,5 +63,10 @@ cudaError_t launch_quant_padded(const QuantPaddedArgs& a, bool src_x, int fmt, i
 cudaError_t launch_grouped_gemm(const GemmArgs& g, int epi, int bn, const void* a_base, int64_t a_rows,
                                 const void* b_base, int64_t b_rows, int num_sms, cudaStream_t s);
 bool tensor_maps_available();
+cudaError_t launch_dense_plan(int64_t T, int bn, TileEntry* tiles, int32_t* num_tiles, cudaStream_t s);
+// Router logits on the tensor cores: logits[T][E] = x Wr^T (+ bias); E % 128 == 0, H % 64 == 0.
+cudaError_t launch_router_gemm(const uint16_t* x, int64_t T, int H, const uint16_t* wr, const float* bias, int E,
+                               float* logits, TileEntry* tiles, int32_t* num_tiles, int32_t* status, int num_sms,
+                               cudaStream_t s);
 
 }  // namespace moe

@@ -123,6 +123,15 @@ __device__ __forceinline__ void mma_f8(uint32_t d, uint64_t a, uint64_t b, uint3
       : "memory");
 }
 
+// bf16 x bf16 (kind::f16), fp32 accumulate.
+__device__ __forceinline__ void mma_bf16(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // 32 lanes x 16 columns of 32-bit accumulators (lane = thread of the warp).
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
   uint32_t r[16];
@@ -169,6 +178,10 @@ __host__ __device__ constexpr uint32_t idesc_mxf4(uint32_t n, bool e8m0, uint32_
 //  e4m3 x e4m3: accumulator format F32 at bit 4, formats 0 (E4M3).
 __host__ __device__ constexpr uint32_t idesc_f8(uint32_t n) {
   return (1u << 4) | ((n >> 3) << 17) | ((128u >> 4) << 24);
+}
+//  bf16 x bf16: accumulator F32, A and B format BF16 (1).
+__host__ __device__ constexpr uint32_t idesc_bf16(uint32_t n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((n >> 3) << 17) | ((128u >> 4) << 24);
 }
 
 }  // namespace tc

@@ -132,9 +132,11 @@ def test_route_logits_flags_invalid_rows():
     assert np.allclose(wn[3], 0.25)
 
 
-@pytest.mark.parametrize("name", ["tiny", "decode", "prefill"])
-def test_route_matches_oracle(name):
-    w = synth.workload(name)
+@pytest.mark.parametrize("name,over", [("tiny", {}), ("decode", {}), ("prefill", {}), ("large", dict(T=300)),
+                                       ("fp8_shared", dict(T=130))])
+def test_route_matches_oracle(name, over):
+    """Small batches use the CUDA-core router, larger ones the tcgen05 bf16 GEMM."""
+    w = synth.workload(name, **over)
     x, wr, b = routed_inputs(w)
     logits = torch.empty((w.T, w.E), dtype=torch.float32, device="cuda")
     idx, wt = ops.moe_route(bits_to_dev_bf16(x), bits_to_dev_bf16(wr),
