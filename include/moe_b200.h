@@ -235,7 +235,10 @@ moe_status moe_get_device_status(void* ws, moe_stream_t stream, int32_t* host_st
  *                     2 = force the tensor-core GEMM path (returns
  *                     MOE_ERR_UNSUPPORTED where the shapes do not allow it).
  * Not thread-safe; set before enqueuing. */
-typedef enum { MOE_OPT_FFN_PATH = 1 } moe_option;
+/*   MOE_OPT_GEMM_TILE_N: token-tile width of the tensor-core path, 256
+ *                     (default; N = 256 MMAs, one accumulator drained to
+ *                     registers) or 128 (two accumulators). */
+typedef enum { MOE_OPT_FFN_PATH = 1, MOE_OPT_GEMM_TILE_N = 2 } moe_option;
 moe_status moe_set_option(int32_t option, int32_t value);
 
 /* moe_permute for callers that cannot allocate device memory (no workspace

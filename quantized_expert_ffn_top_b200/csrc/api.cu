@@ -128,10 +128,10 @@ PermWs carve_perm(Carver& c, int64_t S, int E) {
   return p;
 }
 
-constexpr int kGemmBN = 128;  // token tile of the tensor-core path
+int g_gemm_bn = 256;  // token tile of the tensor-core path (MOE_OPT_GEMM_TILE_N)
 
 int64_t padded_rows(int64_t S, int E) { return (int64_t)align_up((size_t)(S + (int64_t)E * 127), 128) + 256; }
-int64_t max_tiles(int64_t S, int E) { return S / kGemmBN + E + 1; }
+int64_t max_tiles(int64_t S, int E) { return S / 128 + E + 1; }
 
 // Scratch of the grouped FFN: GEMV path (h fp32 per compact slot) and tensor
 // core path (padded, blocked quantised activations and the tile plan).
@@ -251,7 +251,7 @@ moe_status run_gemm_ffn(const uint16_t* x, int64_t T, int64_t S, const int32_t* 
                         int32_t* status, cudaStream_t s, bool mark) {
   const int E = w->E, H = w->H, I = w->I, fmt = w->fmt;
   const int sms = num_sms();
-  MOE_TRY(launch_plan(offsets, E, S, kGemmBN, f.poff, f.tiles, f.ntiles, (int)max_tiles(S, E), status, s));
+  MOE_TRY(launch_plan(offsets, E, S, g_gemm_bn, f.poff, f.tiles, f.ntiles, (int)max_tiles(S, E), status, s));
   if (mark) stage_mark(MOE_STAGE_ACT_QUANT, false, s);
   QuantPaddedArgs qa;
   qa.E = E;
@@ -296,7 +296,7 @@ moe_status run_gemm_ffn(const uint16_t* x, int64_t T, int64_t S, const int32_t* 
   g.status = status;
   if (mark) stage_mark(MOE_STAGE_FFN_UP, false, s);
   if (!fused_h) MOE_TRY(cudaMemsetAsync(h_amax, 0, sizeof(float), s));
-  MOE_TRY(launch_grouped_gemm(g, fused_h ? kEpiUpQuant : kEpiUpF32, kGemmBN, w->w13, (int64_t)E * 2 * I,
+  MOE_TRY(launch_grouped_gemm(g, fused_h ? kEpiUpQuant : kEpiUpF32, g_gemm_bn, w->w13, (int64_t)E * 2 * I,
                               f.xq, f.P, sms, s));
   if (!fused_h) {
     QuantPaddedArgs qh = qa;
@@ -328,7 +328,7 @@ moe_status run_gemm_ffn(const uint16_t* x, int64_t T, int64_t S, const int32_t* 
   d.ldy = H;
   d.status = status;
   if (mark) stage_mark(MOE_STAGE_FFN_DOWN, false, s);
-  MOE_TRY(launch_grouped_gemm(d, kEpiDown, kGemmBN, w->w2, (int64_t)E * H, f.hq, f.P, sms, s));
+  MOE_TRY(launch_grouped_gemm(d, kEpiDown, g_gemm_bn, w->w2, (int64_t)E * H, f.hq, f.P, sms, s));
   if (mark) stage_mark(MOE_STAGE_FFN_DOWN, true, s);
   return MOE_OK;
 }
@@ -419,6 +419,11 @@ moe_status moe_set_option(int32_t option, int32_t value) {
   if (option == MOE_OPT_FFN_PATH) {
     if (value < 0 || value > 2) return MOE_ERR_INVALID_ARG;
     g_ffn_path = value;
+    return MOE_OK;
+  }
+  if (option == MOE_OPT_GEMM_TILE_N) {
+    if (value != 128 && value != 256) return MOE_ERR_INVALID_ARG;
+    g_gemm_bn = value;
     return MOE_OK;
   }
   return MOE_ERR_INVALID_ARG;

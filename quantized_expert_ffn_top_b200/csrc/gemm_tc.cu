@@ -59,7 +59,9 @@ struct Cfg {
   static constexpr int kStage = ((kA + kB + kSFA + kSFB) + 1023) / 1024 * 1024;
   static constexpr int kStages = (200 * 1024) / kStage < 8 ? (200 * 1024) / kStage : 8;
   static constexpr int kAccStages = BN == 256 ? 1 : 2;
-  static constexpr int kEpiWarps = 8;
+  // 64 accumulator columns per epilogue warp: 2 (BN 128) or 4 (BN 256) warps
+  // per tensor-memory lane quarter
+  static constexpr int kEpiWarps = BN == 256 ? 16 : 8;
   static constexpr int kThreads = (2 + kEpiWarps) * 32;
   static constexpr uint32_t kSfaCol = kAccStages * BN;
   static constexpr uint32_t kSfbCol = kSfaCol + F::kGroups * 4;
@@ -78,9 +80,19 @@ __device__ __forceinline__ float act_scale_of(int fmt, const float* st, const fl
   return fmt == MOE_FMT_NVFP4 ? nvfp4_tensor_scale(*amax) : fp8_tensor_scale(*amax);
 }
 
+// Token-operand maps with box heights 16, 32, 64, 128, 256 rows: a tile
+// loads only the rows it covers, rounded up to one of these.
+struct TokenMaps {
+  CUtensorMap m[5];
+};
+
+__device__ __forceinline__ int token_box_index(int rows) {
+  return rows <= 16 ? 0 : (rows <= 32 ? 1 : (rows <= 64 ? 2 : (rows <= 128 ? 3 : 4)));
+}
+
 template <int FMT, int EPI, int BN>
 __global__ void __launch_bounds__(Cfg<FMT, EPI, BN>::kThreads, 1)
-    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ TokenMaps tmaps_b,
                         const GemmArgs g) {
   using C = Cfg<FMT, EPI, BN>;
   using F = FmtTraits<FMT>;
@@ -108,7 +120,8 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN>::kThreads, 1)
     *abort = 0;
     tc::fence_mbar_init();
     tc::prefetch_tmap(&tmap_a);
-    tc::prefetch_tmap(&tmap_b);
+#pragma unroll
+    for (int i = 0; i < 5; ++i) tc::prefetch_tmap(&tmaps_b.m[i]);
   }
   if (warp == 1) {
     tc::tmem_alloc(tmem_slot, C::kTmemCols);
@@ -123,116 +136,134 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN>::kThreads, 1)
   const int nkb = g.K / F::kBK;
   const int ncols_w = F::kBs ? g.K / F::kBs : 0;  // scale columns per row (multiple of 4)
 
+  // The producer and MMA warps run their loops with the whole warp, so the
+  // loop state stays warp-uniform, and one elected lane issues the copies
+  // and tensor-core instructions (a divergent single-thread loop issues them
+  // at about half the rate).
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      for (int t = blockIdx.x; t < ntiles && !*abort; t += gridDim.x) {
-        const TileEntry te = g.tiles[t / MT];
-        const int mt = t % MT;
-        const uint8_t* sfa = F::kBs ? g.w_sf + (size_t)te.e * g.R * ncols_w + (size_t)mt * (ncols_w / 4) * 512 : nullptr;
-        for (int kb = 0; kb < nkb; ++kb) {
-          if (!tc::mbar_wait(&empty[stage], phase ^ 1u, abort)) {
-            raise_status(g.status, MOE_ERR_TIMEOUT);
-            *abort = 1;
-            break;
-          }
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int t = blockIdx.x; t < ntiles && !*abort; t += gridDim.x) {
+      const TileEntry te = g.tiles[t / MT];
+      const int mt = t % MT;
+      const uint8_t* sfa = F::kBs ? g.w_sf + (size_t)te.e * g.R * ncols_w + (size_t)mt * (ncols_w / 4) * 512 : nullptr;
+      for (int kb = 0; kb < nkb; ++kb) {
+        if (!tc::mbar_wait(&empty[stage], phase ^ 1u, abort)) {
+          if (lane == 0) raise_status(g.status, MOE_ERR_TIMEOUT);
+          *abort = 1;
+          break;
+        }
+        if (tc::elect_one()) {
           uint8_t* st = smem + stage * C::kStage;
-          tc::mbar_expect_tx(&full[stage], C::kTx);
+          const int bi = token_box_index(min(te.nvalid, BN));
+          const uint32_t brows = 16u << bi;
+          const int nblk = (min(te.nvalid, BN) + 127) / 128;   // 128-row scale blocks in use
+          tc::mbar_expect_tx(&full[stage], C::kA + brows * 128u + C::kSFA + nblk * F::kGroups * 512);
           tc::tma_load_2d(st, &tmap_a, &full[stage], kb * 128, te.e * g.R + mt * 128);
-          tc::tma_load_2d(st + C::kA, &tmap_b, &full[stage], kb * 128, te.row0);
+          tc::tma_load_2d(st + C::kA, &tmaps_b.m[bi], &full[stage], kb * 128, te.row0);
           if (F::kBs) {
             tc::bulk_load(st + C::kA + C::kB, sfa + (size_t)kb * F::kGroups * 512, C::kSFA, &full[stage]);
-            for (int nb = 0; nb < BN / 128; ++nb) {
+            for (int nb = 0; nb < nblk; ++nb) {
               const uint8_t* sfb =
                   g.b_sf + ((size_t)(te.row0 / 128 + nb) * (ncols_w / 4) + (size_t)kb * F::kGroups) * 512;
               tc::bulk_load(st + C::kA + C::kB + C::kSFA + nb * F::kGroups * 512, sfb, F::kGroups * 512,
                             &full[stage]);
             }
           }
-          if (++stage == C::kStages) {
-            stage = 0;
-            phase ^= 1u;
-          }
+        }
+        __syncwarp();
+        if (++stage == C::kStages) {
+          stage = 0;
+          phase ^= 1u;
         }
       }
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      int acc = 0;
-      uint32_t acc_phase = 0;
-      for (int t = blockIdx.x; t < ntiles && !*abort; t += gridDim.x) {
-        const TileEntry te = g.tiles[t / MT];
-        if (!tc::mbar_wait(&tempty[acc], acc_phase ^ 1u, abort)) {
-          raise_status(g.status, MOE_ERR_TIMEOUT);
+    int stage = 0;
+    uint32_t phase = 0;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = blockIdx.x; t < ntiles && !*abort; t += gridDim.x) {
+      const TileEntry te = g.tiles[t / MT];
+      if (!tc::mbar_wait(&tempty[acc], acc_phase ^ 1u, abort)) {
+        if (lane == 0) raise_status(g.status, MOE_ERR_TIMEOUT);
+        *abort = 1;
+        break;
+      }
+      tc::fence_after_sync();
+      const uint32_t n_mma = (uint32_t)min(BN, (te.nvalid + 15) & ~15);
+      const uint32_t d = tmem + acc * BN;
+      uint32_t idesc_nv = tc::idesc_mxf4(n_mma, false, 0, 0), idesc_f8 = tc::idesc_f8(n_mma),
+               idesc_bf = tc::idesc_bf16(n_mma);
+      bool ok = true;
+      for (int kb = 0; kb < nkb; ++kb) {
+        if (!tc::mbar_wait(&full[stage], phase, abort)) {
+          if (lane == 0) raise_status(g.status, MOE_ERR_TIMEOUT);
           *abort = 1;
+          ok = false;
           break;
         }
         tc::fence_after_sync();
-        const uint32_t n_mma = (uint32_t)min(BN, (te.nvalid + 15) & ~15);
-        const uint32_t d = tmem + acc * BN;
-        bool ok = true;
-        for (int kb = 0; kb < nkb; ++kb) {
-          if (!tc::mbar_wait(&full[stage], phase, abort)) {
-            raise_status(g.status, MOE_ERR_TIMEOUT);
-            *abort = 1;
-            ok = false;
-            break;
-          }
-          tc::fence_after_sync();
+        if (tc::elect_one()) {
           uint8_t* st = smem + stage * C::kStage;
           const uint32_t sa = tc::smem_u32(st), sb = tc::smem_u32(st + C::kA);
           if (F::kBs) {
-            const uint32_t ssfa = tc::smem_u32(st + C::kA + C::kB);
-            const uint32_t ssfb = ssfa + C::kSFA;
+            const uint64_t dsfa = tc::desc_sf(tc::smem_u32(st + C::kA + C::kB));
+            const uint64_t dsfb = dsfa + (uint64_t)(C::kSFA >> 4);
+#pragma unroll
             for (int grp = 0; grp < F::kGroups; ++grp) {
-              tc::sf_copy(tmem + C::kSfaCol + 4 * grp, tc::desc_sf(ssfa + grp * 512));
+              tc::sf_copy(tmem + C::kSfaCol + 4 * grp, dsfa + (uint64_t)(grp * 32));
+#pragma unroll
               for (int nb = 0; nb < BN / 128; ++nb)
-                tc::sf_copy(tmem + C::kSfbCol + grp * 4 * (BN / 128) + nb * 4,
-                            tc::desc_sf(ssfb + (nb * F::kGroups + grp) * 512));
+                if (nb == 0 || n_mma > 128u)   // second block only for tiles wider than 128 tokens
+                  tc::sf_copy(tmem + C::kSfbCol + grp * 4 * (BN / 128) + nb * 4,
+                              dsfb + (uint64_t)((nb * F::kGroups + grp) * 32));
             }
           }
+          const uint64_t da0 = tc::desc_sw128(sa), db0 = tc::desc_sw128(sb);
 #pragma unroll
           for (int kk = 0; kk < F::kSteps; ++kk) {
-            const uint64_t da = tc::desc_sw128(sa) + (uint64_t)(kk * 2);  // +32 bytes per MMA along K
-            const uint64_t db = tc::desc_sw128(sb) + (uint64_t)(kk * 2);
+            const uint64_t da = da0 + (uint64_t)(kk * 2);  // +32 bytes per MMA along K
+            const uint64_t db = db0 + (uint64_t)(kk * 2);
             const uint32_t accum = (kb > 0 || kk > 0) ? 1u : 0u;
             if (FMT == MOE_FMT_NVFP4) {
-              tc::mma_nvf4(d, da, db, tc::idesc_mxf4(n_mma, false, 0, 0), tmem + C::kSfaCol + 4 * kk,
-                           tmem + C::kSfbCol + kk * 4 * (BN / 128), accum);
+              tc::mma_nvf4(d, da, db, idesc_nv, tmem + C::kSfaCol + 4 * kk, tmem + C::kSfbCol + kk * 4 * (BN / 128),
+                           accum);
             } else if (FMT == MOE_FMT_MXFP4) {
               const uint32_t id = (uint32_t)(kk & 1) * 2;  // two MMAs share one group of four e8m0 scales
               tc::mma_mxf4(d, da, db, tc::idesc_mxf4(n_mma, true, id, id), tmem + C::kSfaCol + 4 * (kk >> 1),
                            tmem + C::kSfbCol + (kk >> 1) * 4 * (BN / 128), accum);
             } else if (FMT == MOE_FMT_FP8) {
-              tc::mma_f8(d, da, db, tc::idesc_f8(n_mma), accum);
+              tc::mma_f8(d, da, db, idesc_f8, accum);
             } else {
-              tc::mma_bf16(d, da, db, tc::idesc_bf16(n_mma), accum);
+              tc::mma_bf16(d, da, db, idesc_bf, accum);
             }
           }
           tc::mma_commit(&empty[stage]);
-          if (++stage == C::kStages) {
-            stage = 0;
-            phase ^= 1u;
-          }
         }
-        if (!ok) break;
-        tc::mma_commit(&tfull[acc]);
-        if (++acc == C::kAccStages) {
-          acc = 0;
-          acc_phase ^= 1u;
+        __syncwarp();
+        if (++stage == C::kStages) {
+          stage = 0;
+          phase ^= 1u;
         }
+      }
+      if (!ok) break;
+      if (tc::elect_one()) tc::mma_commit(&tfull[acc]);
+      __syncwarp();
+      if (++acc == C::kAccStages) {
+        acc = 0;
+        acc_phase ^= 1u;
       }
     }
   } else {
     // ------------------------------------------------------------ epilogue
+    // Each warp drains its 64 accumulator columns into registers, hands the
+    // tensor memory back to the MMA warp at once, then converts and stores.
     const int ew = warp - 2;
     const int q = warp & 3;                      // tensor-memory lane quarter of this warp
-    const int half = ew / 4;                     // which half of the tile's columns
+    const int cw = ew / 4;                       // which 64-column slice of the tile
     const float gact = act_scale_of(FMT, g.act_scale, g.act_amax);
     const float g2 = (EPI == kEpiUpQuant && FMT == MOE_FMT_NVFP4) ? act_scale_of(FMT, g.h_scale, nullptr) : 1.0f;
     float hmax = 0.0f;
@@ -248,48 +279,63 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN>::kThreads, 1)
       const TileEntry te = g.tiles[t / MT];
       const int mt = t % MT;
       const int ncol = min(BN, (te.nvalid + 15) & ~15);
-      const int c_lo = half * (BN / 2), c_hi = min(ncol, (half + 1) * (BN / 2));
-      const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
-      if (EPI == kEpiLogits) {
-        const int o = mt * 128 + q * 32 + lane;  // expert
-        const float b = g.bias ? __ldg(g.bias + o) : 0.0f;
-        for (int c0 = c_lo; c0 < c_hi; c0 += 16) {
-          float v[16];
-          tc::tmem_ld16(tbase + c0, v);
+      const int c_lo = cw * 64;
+      const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN) + (uint32_t)c_lo;
+      uint32_t r0[16], r1[16], r2[16], r3[16];
+      if (c_lo < ncol) {
+        tc::tmem_ld16_async(tbase, r0);
+        tc::tmem_ld16_async(tbase + 16, r1);
+        tc::tmem_ld16_async(tbase + 32, r2);
+        tc::tmem_ld16_async(tbase + 48, r3);
+        tc::tmem_wait16(r0);
+        tc::tmem_wait16(r1);
+        tc::tmem_wait16(r2);
+        tc::tmem_wait16(r3);
+      }
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&tempty[acc]);
+      if (++acc == C::kAccStages) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+      if (c_lo >= ncol) continue;  // both warps of a pair (same slice) skip together
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {
+        const uint32_t* rr = ch == 0 ? r0 : (ch == 1 ? r1 : (ch == 2 ? r2 : r3));
+        float v[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(rr[j]);
+        const int c0 = c_lo + ch * 16;
+        if (EPI == kEpiLogits) {
+          const int o = mt * 128 + q * 32 + lane;  // expert
+          const float b = g.bias ? __ldg(g.bias + o) : 0.0f;
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
             const int tok = c0 + c;
             if (tok < te.nvalid) g.logits[(size_t)(te.p0 + tok) * g.ldy + o] = v[c] + b;
           }
-        }
-      } else if (EPI == kEpiDown) {
-        const int o = mt * 128 + q * 32 + lane;
-        const float sc = (FMT == MOE_FMT_MXFP4) ? 1.0f : __ldg(g.w_gs + te.e) * gact;
-        for (int c0 = c_lo; c0 < c_hi; c0 += 16) {
-          float v[16];
-          tc::tmem_ld16(tbase + c0, v);
+        } else if (EPI == kEpiDown) {
+          const int o = mt * 128 + q * 32 + lane;
+          const float sc = (FMT == MOE_FMT_MXFP4) ? 1.0f : __ldg(g.w_gs + te.e) * gact;
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
             const int tok = c0 + c;
             if (tok < te.nvalid) g.y[(size_t)(te.p0 + tok) * g.ldy + o] = f32_to_bf16_rn(v[c] * sc);
           }
-        }
-      } else {
-        // gate|up rows interleave (even lane gate, odd lane up): one shuffle
-        // pairs them, SwiGLU runs on every lane, and the h values go through
-        // a shared-memory tile so that each lane then owns 8 consecutive
-        // features of one token (half a NVFP4 block, a quarter of an MXFP4
-        // block) for the block maximum, the codes and 16-byte stores.
-        const int part = lane & 1;
-        const float sc = (FMT == MOE_FMT_MXFP4) ? 1.0f : __ldg(g.w_gs + te.e * 2 + part) * gact;
-        const int pp = q & 1;                                  // position in the warp pair
-        float* tile = epi_tiles + (ew >> 1) * (16 * 32);       // [16 tokens][32 features] of the pair
-        const int fl = lane >> 1;                              // feature within the warp's 16
-        const int f_pair = mt * 64 + (q >> 1) * 32;            // first feature of the pair
-        const int bar = 1 + (ew >> 1);
-        for (int c0 = c_lo; c0 < c_hi; c0 += 16) {
-          float v[16];
-          tc::tmem_ld16(tbase + c0, v);
+        } else {
+          // gate|up rows interleave (even lane gate, odd lane up): one shuffle
+          // pairs them, SwiGLU runs on every lane, and the h values go through
+          // a shared-memory tile so that each lane then owns 8 consecutive
+          // features of one token (half a NVFP4 block, a quarter of an MXFP4
+          // block) for the block maximum, the codes and wide stores.
+          const int part = lane & 1;
+          const float sc = (FMT == MOE_FMT_MXFP4) ? 1.0f : __ldg(g.w_gs + te.e * 2 + part) * gact;
+          const int pp = q & 1;                                  // position in the warp pair
+          float* tile = epi_tiles + (ew >> 1) * (16 * 32);       // [16 tokens][32 features] of the pair
+          const int fl = lane >> 1;                              // feature within the warp's 16
+          const int f_pair = mt * 64 + (q >> 1) * 32;            // first feature of the pair
+          const int bar = 1 + (ew >> 1);
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             const float a = v[2 * i] * sc, b = v[2 * i + 1] * sc;
@@ -345,13 +391,6 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN>::kThreads, 1)
           asm volatile("bar.sync %0, 64;" ::"r"(bar) : "memory");
         }
       }
-      tc::fence_before_sync();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&tempty[acc]);
-      if (++acc == C::kAccStages) {
-        acc = 0;
-        acc_phase ^= 1u;
-      }
     }
     if (EPI == kEpiUpF32 && g.h_amax) {
       hmax = warp_max(hmax);
@@ -405,10 +444,12 @@ template <int FMT, int EPI, int BN>
 cudaError_t launch_cfg(const GemmArgs& g, const void* a_base, int64_t a_rows, const void* b_base, int64_t b_rows,
                        int num_sms, cudaStream_t s) {
   using C = Cfg<FMT, EPI, BN>;
-  CUtensorMap ma, mb;
+  CUtensorMap ma;
+  TokenMaps mb;
   const int64_t rb = FMT == kFmtBF16 ? 2 * (int64_t)g.K : (FMT == MOE_FMT_FP8 ? g.K : g.K / 2);
-  if (!make_map(&ma, a_base, a_rows, rb, 128) || !make_map(&mb, b_base, b_rows, rb, BN))
-    return cudaErrorInvalidValue;
+  if (!make_map(&ma, a_base, a_rows, rb, 128)) return cudaErrorInvalidValue;
+  for (int i = 0; i < 5; ++i)
+    if (!make_map(&mb.m[i], b_base, b_rows, rb, (16 << i) < BN ? (16 << i) : BN)) return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<FMT, EPI, BN>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return e;

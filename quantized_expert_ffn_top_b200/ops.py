@@ -21,6 +21,7 @@ FMT_NVFP4, FMT_MXFP4, FMT_FP8 = 1, 2, 3
 ACT_BF16, ACT_MATCH = 0, 1
 LAYOUT_CANONICAL, LAYOUT_PREPARED = 0, 1
 OPT_FFN_PATH = 1
+OPT_GEMM_TILE_N = 2
 FMT_BY_NAME = {"nvfp4": FMT_NVFP4, "mxfp4": FMT_MXFP4, "fp8": FMT_FP8}
 
 EXPORTED = (
