@@ -131,7 +131,8 @@ PermWs carve_perm(Carver& c, int64_t S, int E) {
 int g_gemm_bn = 256;  // token tile of the tensor-core path (MOE_OPT_GEMM_TILE_N)
 
 int64_t padded_rows(int64_t S, int E) { return (int64_t)align_up((size_t)(S + (int64_t)E * 127), 128) + 256; }
-int64_t max_tiles(int64_t S, int E) { return S / 128 + E + 1; }
+// Tile list bound for the smallest token group (8 slots, the GEMV's MMA n).
+int64_t max_tiles(int64_t S, int E) { return S / 8 + E + 1; }
 
 // Scratch of the grouped FFN: GEMV path (h fp32 per compact slot) and tensor
 // core path (padded, blocked quantised activations and the tile plan).
@@ -367,12 +368,17 @@ moe_status run_grouped_ffn(const uint16_t* x, int64_t T, int64_t S, const int32_
   a.h_amax = (act == MOE_ACT_MATCH && w->fmt != MOE_FMT_MXFP4 && !w->a2_gs) ? h_amax : nullptr;
   a.h = scratch.h;
   a.y_perm = y_perm;
+  a.tiles = scratch.tiles;
+  a.num_tiles = scratch.ntiles;
   a.status = status;
+  const int sms = num_sms();
+  MOE_TRY(launch_plan(offsets, w->E, S, kGemvTokens, scratch.poff, scratch.tiles, scratch.ntiles,
+                      (int)max_tiles(S, w->E), status, s));
   if (mark) stage_mark(MOE_STAGE_FFN_UP, false, s);
-  MOE_TRY(launch_gemv_up(a, s));
+  MOE_TRY(launch_gemv_up(a, sms, s));
   if (mark) stage_mark(MOE_STAGE_FFN_UP, true, s);
   if (mark) stage_mark(MOE_STAGE_FFN_DOWN, false, s);
-  MOE_TRY(launch_gemv_down(a, s));
+  MOE_TRY(launch_gemv_down(a, sms, s));
   if (mark) stage_mark(MOE_STAGE_FFN_DOWN, true, s);
   return MOE_OK;
 }

@@ -63,10 +63,13 @@ struct GemvArgs {
   float* h_amax;
   float* h;                // [S][I] fp32
   uint16_t* y_perm;        // [S][H]
+  const struct TileEntry* tiles;  // token groups of at most 8 slots per expert
+  const int32_t* num_tiles;
   int32_t* status;
 };
-cudaError_t launch_gemv_up(const GemvArgs& a, cudaStream_t s);
-cudaError_t launch_gemv_down(const GemvArgs& a, cudaStream_t s);
+constexpr int kGemvTokens = 8;  // token columns of one GEMV work item (the MMA n)
+cudaError_t launch_gemv_up(const GemvArgs& a, int num_sms, cudaStream_t s);
+cudaError_t launch_gemv_down(const GemvArgs& a, int num_sms, cudaStream_t s);
 
 // combine.cu
 cudaError_t launch_combine(const uint16_t* y_perm, const int32_t* inv_perm, const float* w, int64_t T, int k, int H,

@@ -158,8 +158,102 @@ __global__ void __launch_bounds__(kPermWarps * 32) perm_scatter_kernel(const int
   }
 }
 
+// Small batches (decode): the same three passes inside one block of 32
+// warps, each warp owning a contiguous range of ceil(S/32) slots; the
+// per-warp expert counters live in shared memory.  One launch instead of three.
+constexpr int kSmallWarps = 32;
+constexpr int64_t kSmallMaxS = 8192;
+
+__global__ void __launch_bounds__(kSmallWarps * 32) perm_small_kernel(const int32_t* __restrict__ idx, int64_t S,
+                                                                     int k, int E, int32_t* __restrict__ offsets,
+                                                                     int32_t* __restrict__ perm_token,
+                                                                     int32_t* __restrict__ inv_perm,
+                                                                     int32_t* status) {
+  extern __shared__ int32_t cnt[];  // [kSmallWarps][E], then [E] totals
+  int32_t* tot = cnt + kSmallWarps * E;
+  __shared__ int32_t warp_tot[32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t per = ((S + kSmallWarps - 1) / kSmallWarps + 31) / 32 * 32;  // slots per warp, multiple of 32
+  for (int i = threadIdx.x; i < kSmallWarps * E; i += blockDim.x) cnt[i] = 0;
+  __syncthreads();
+  int32_t* my = cnt + warp * E;
+  const int64_t lo = warp * per, hi = min(S, lo + per);
+  for (int64_t base = lo; base < hi; base += 32) {
+    const int64_t i = base + lane;
+    const int e = (i < hi) ? slot_expert(idx, S, i, E, status) : -1;
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    if (e >= 0 && lane == __ffs(peers) - 1) my[e] += __popc(peers);
+    __syncwarp();
+  }
+  __syncthreads();
+  // per expert: exclusive prefix over warps, total
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int32_t run = 0;
+    for (int w = 0; w < kSmallWarps; ++w) {
+      const int32_t v = cnt[w * E + e];
+      cnt[w * E + e] = run;
+      run += v;
+    }
+    tot[e] = run;
+  }
+  __syncthreads();
+  // exclusive scan of the totals over experts (E <= 1024 = blockDim)
+  const int e = threadIdx.x;
+  const int32_t v = e < E ? tot[e] : 0;
+  int32_t incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int32_t n = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += n;
+  }
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int32_t wv = warp_tot[lane];
+    int32_t wi = wv;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t n = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += n;
+    }
+    warp_tot[lane] = wi - wv;
+  }
+  __syncthreads();
+  const int32_t excl = incl - v + warp_tot[warp];
+  __syncthreads();
+  if (e < E) {
+    tot[e] = excl;
+    offsets[e] = excl;
+  }
+  if (e == E - 1) offsets[E] = excl + v;
+  __syncthreads();
+  for (int i = threadIdx.x; i < kSmallWarps * E; i += blockDim.x) cnt[i] += tot[i % E];
+  __syncthreads();
+  for (int64_t base = lo; base < hi; base += 32) {
+    const int64_t i = base + lane;
+    const int ee = (i < hi) ? slot_expert(idx, S, i, E, nullptr) : -1;
+    const unsigned peers = __match_any_sync(0xffffffffu, ee);
+    if (ee >= 0) {
+      const int32_t p = my[ee] + __popc(peers & ((1u << lane) - 1u));
+      perm_token[p] = (int32_t)(i / k);
+      inv_perm[i] = p;
+    } else if (i < hi) {
+      inv_perm[i] = -1;
+    }
+    __syncwarp();
+    if (ee >= 0 && lane == __ffs(peers) - 1) my[ee] += __popc(peers);
+    __syncwarp();
+  }
+}
+
 cudaError_t launch_permute(const int32_t* idx, int64_t S, int k, int E, int32_t* offsets, int32_t* perm_token,
                            int32_t* inv_perm, PermuteScratch scratch, int32_t* status, cudaStream_t s) {
+  const size_t small_smem = sizeof(int32_t) * (size_t)(kSmallWarps + 1) * E;
+  if (S > 0 && S <= kSmallMaxS && small_smem <= 48 * 1024) {
+    perm_small_kernel<<<1, kSmallWarps * 32, small_smem, s>>>(idx, S, k, E, offsets, perm_token, inv_perm, status);
+    count_launches(1);
+    return cudaGetLastError();
+  }
   const int nchunks = (int)((S + kChunk - 1) / kChunk);
   if (nchunks == 0) {
     // no slots: offsets are all zero

@@ -158,7 +158,9 @@ def test_route_matches_oracle(name, over):
 
 # ----------------------------------------------------------- permutation ----
 @pytest.mark.parametrize("T,k,E,skew", [(8, 2, 8, 0.0), (4, 8, 128, 0.0), (4096, 8, 128, 1.1), (16384, 8, 256, 1.1),
-                                        (777, 1, 1, 0.0), (50, 16, 1024, 0.3), (3000, 5, 37, 2.0)])
+                                        (777, 1, 1, 0.0), (50, 16, 1024, 0.3), (3000, 5, 37, 2.0),
+                                        # one-block path up to 8192 slots, then the three-pass path
+                                        (1000, 8, 256, 1.1), (1024, 8, 256, 0.0), (1025, 8, 256, 0.0)])
 def test_permute_bit_exact(T, k, E, skew):
     if k > E:
         pytest.skip("k > E")
@@ -191,6 +193,10 @@ FFN_CASES = [
     ("tiny", dict(fmt="fp8", H=256, I=128, E=8, k=2, T=10), 0),
     ("tiny", dict(fmt="fp8", H=256, I=128, E=8, k=2, T=10), 1),
     ("tiny", dict(T=40, E=4, k=2, H=128, I=128), 1),       # > 8 tokens per expert
+    # K = 128 mod 256: the streamed FP4 rows end on half a 128-byte chunk
+    ("tiny", dict(fmt="mxfp4", H=384, I=384, E=6, k=2, T=20), 1),
+    ("tiny", dict(H=384, I=640, E=5, k=3, T=33), 1),
+    ("tiny", dict(fmt="fp8", H=384, I=640, E=5, k=3, T=33), 1),
 ]
 
 
