@@ -194,11 +194,14 @@ moe_status moe_permute(const int32_t* topk_idx, int64_t T, int32_t k, int32_t E,
  * act() is the identity (BF16) or the quantiser of the weights' format
  * (MATCH, see moe_act; the tensor amax of h is taken over all S slots).
  * x [T][H] bf16, perm_token [S], offsets [E+1] (device); w must be
- * PREPARED.  Small batches stream each active expert's weights once through
- * a vectorised GEMV (the decode split of the atomicmilkshake fork README,
- * "Quant types": MMVQ for decode, MMQ for prefill); large batches run a
- * tcgen05 block-scaled grouped GEMM.  The choice is a host heuristic on the
- * arguments (T*k versus E), never a device read-back. */
+ * PREPARED.  With quantised activations (MATCH) and H, I multiples of 256
+ * (FP4) or 128 (FP8) the FFN runs as a tcgen05 block-scaled grouped GEMM at
+ * every batch size -- 64-token tiles while T*k < 8E (decode: each active
+ * expert's weights stream once), 256-token tiles beyond (prefill).  BF16
+ * activations and other shapes take a TMA-fed mma.sync GEMV that streams
+ * each active expert's weights once (the decode split of the atomicmilkshake
+ * fork README, "Quant types": MMVQ for decode, MMQ for prefill).  The choice
+ * is a host decision on the arguments, never a device read-back. */
 moe_status moe_grouped_ffn(const uint16_t* x, int64_t T, int32_t k, const int32_t* perm_token,
                            const int32_t* offsets, const moe_weights* w, int32_t act, uint16_t* y_perm, void* ws,
                            size_t ws_bytes, moe_stream_t stream);
@@ -206,7 +209,7 @@ moe_status moe_grouped_ffn(const uint16_t* x, int64_t T, int32_t k, const int32_
 /* Weighted un-permute: out[t] = sum_{j<k} w[t,j] y_perm[inv_perm[t*k+j]]
  * (+ shared_y[t]) accumulated in fp32 in order j = 0..k-1, rounded once to
  * bf16.  y_perm [T*k][H], shared_y [T][H] (nullable), out [T][H] bf16;
- * inv_perm [T*k], topk_w [T][k]; all device. */
+ * inv_perm [T*k], topk_w [T][k]; all device; 1 <= k <= 1024. */
 moe_status moe_combine(const uint16_t* y_perm, const int32_t* inv_perm, const float* topk_w, int64_t T, int32_t k,
                        int32_t H, const uint16_t* shared_y, uint16_t* out, void* ws, size_t ws_bytes,
                        moe_stream_t stream);
@@ -235,9 +238,9 @@ moe_status moe_get_device_status(void* ws, moe_stream_t stream, int32_t* host_st
  *                     2 = force the tensor-core GEMM path (returns
  *                     MOE_ERR_UNSUPPORTED where the shapes do not allow it).
  * Not thread-safe; set before enqueuing. */
-/*   MOE_OPT_GEMM_TILE_N: token-tile width of the tensor-core path, 256
- *                     (default; N = 256 MMAs, one accumulator drained to
- *                     registers) or 128 (two accumulators). */
+/*   MOE_OPT_GEMM_TILE_N: token-tile width of the tensor-core path: 0 (default:
+ *                     64 while T*k < 8E, else 256), 64 (four accumulators),
+ *                     128 (two) or 256 (one, drained to registers). */
 typedef enum { MOE_OPT_FFN_PATH = 1, MOE_OPT_GEMM_TILE_N = 2 } moe_option;
 moe_status moe_set_option(int32_t option, int32_t value);
 

@@ -128,7 +128,7 @@ PermWs carve_perm(Carver& c, int64_t S, int E) {
   return p;
 }
 
-int g_gemm_bn = 256;  // token tile of the tensor-core path (MOE_OPT_GEMM_TILE_N)
+int g_gemm_bn = 0;  // token tile of the tensor-core path (MOE_OPT_GEMM_TILE_N); 0 = by batch size
 
 int64_t padded_rows(int64_t S, int E) { return (int64_t)align_up((size_t)(S + (int64_t)E * 127), 128) + 256; }
 // Tile list bound for the smallest token group (8 slots, the GEMV's MMA n).
@@ -238,13 +238,20 @@ bool gemm_shapes_ok(const moe_weights* w, int act) {
   return w->H % kb == 0 && w->I % kb == 0 && w->I % 64 == 0;
 }
 
-// Tensor cores once the average expert has enough rows to fill a tile; the
-// weight-streaming GEMV below that.  Arguments only, no device read-back.
+// Tensor cores whenever the activations are quantised and the shapes allow
+// it; the weight-streaming GEMV for BF16 activations and other shapes.
 bool use_gemm_path(const moe_weights* w, int64_t S, int act) {
+  (void)S;
   if (g_ffn_path == 1) return false;
-  if (!gemm_shapes_ok(w, act)) return false;
-  if (g_ffn_path == 2) return true;
-  return S >= 8 * (int64_t)w->E;
+  return gemm_shapes_ok(w, act);
+}
+
+// Token tile: 64 wide while the average expert holds fewer than 8 slots
+// (decode: deep weight streaming, small B stages), 256 wide beyond.
+// Arguments only, no device read-back.
+int gemm_tile_n(int64_t S, int E) {
+  if (g_gemm_bn) return g_gemm_bn;
+  return S < 8 * (int64_t)E ? 64 : 256;
 }
 
 moe_status run_gemm_ffn(const uint16_t* x, int64_t T, int64_t S, const int32_t* perm, const int32_t* offsets,
@@ -252,7 +259,8 @@ moe_status run_gemm_ffn(const uint16_t* x, int64_t T, int64_t S, const int32_t* 
                         int32_t* status, cudaStream_t s, bool mark) {
   const int E = w->E, H = w->H, I = w->I, fmt = w->fmt;
   const int sms = num_sms();
-  MOE_TRY(launch_plan(offsets, E, S, g_gemm_bn, f.poff, f.tiles, f.ntiles, (int)max_tiles(S, E), status, s));
+  const int bn = gemm_tile_n(S, E);
+  MOE_TRY(launch_plan(offsets, E, S, bn, f.poff, f.tiles, f.ntiles, (int)max_tiles(S, E), status, s));
   if (mark) stage_mark(MOE_STAGE_ACT_QUANT, false, s);
   QuantPaddedArgs qa;
   qa.E = E;
@@ -297,7 +305,7 @@ moe_status run_gemm_ffn(const uint16_t* x, int64_t T, int64_t S, const int32_t* 
   g.status = status;
   if (mark) stage_mark(MOE_STAGE_FFN_UP, false, s);
   if (!fused_h) MOE_TRY(cudaMemsetAsync(h_amax, 0, sizeof(float), s));
-  MOE_TRY(launch_grouped_gemm(g, fused_h ? kEpiUpQuant : kEpiUpF32, g_gemm_bn, w->w13, (int64_t)E * 2 * I,
+  MOE_TRY(launch_grouped_gemm(g, fused_h ? kEpiUpQuant : kEpiUpF32, bn, w->w13, (int64_t)E * 2 * I,
                               f.xq, f.P, sms, s));
   if (!fused_h) {
     QuantPaddedArgs qh = qa;
@@ -329,7 +337,7 @@ moe_status run_gemm_ffn(const uint16_t* x, int64_t T, int64_t S, const int32_t* 
   d.ldy = H;
   d.status = status;
   if (mark) stage_mark(MOE_STAGE_FFN_DOWN, false, s);
-  MOE_TRY(launch_grouped_gemm(d, kEpiDown, g_gemm_bn, w->w2, (int64_t)E * H, f.hq, f.P, sms, s));
+  MOE_TRY(launch_grouped_gemm(d, kEpiDown, bn, w->w2, (int64_t)E * H, f.hq, f.P, sms, s));
   if (mark) stage_mark(MOE_STAGE_FFN_DOWN, true, s);
   return MOE_OK;
 }
@@ -428,7 +436,7 @@ moe_status moe_set_option(int32_t option, int32_t value) {
     return MOE_OK;
   }
   if (option == MOE_OPT_GEMM_TILE_N) {
-    if (value != 128 && value != 256) return MOE_ERR_INVALID_ARG;
+    if (value != 0 && value != 64 && value != 128 && value != 256) return MOE_ERR_INVALID_ARG;
     g_gemm_bn = value;
     return MOE_OK;
   }
@@ -581,7 +589,7 @@ moe_status moe_grouped_ffn(const uint16_t* x, int64_t T, int32_t k, const int32_
 moe_status moe_combine(const uint16_t* y_perm, const int32_t* inv_perm, const float* topk_w, int64_t T, int32_t k,
                        int32_t H, const uint16_t* shared_y, uint16_t* out, void* ws, size_t ws_bytes,
                        moe_stream_t stream) {
-  if (T < 0 || k < 1 || H <= 0 || H % 8 != 0) return MOE_ERR_INVALID_ARG;
+  if (T < 0 || k < 1 || k > 1024 || H <= 0 || H % 8 != 0) return MOE_ERR_INVALID_ARG;
   if (T > 0 && (!y_perm || !inv_perm || !topk_w || !out)) return MOE_ERR_INVALID_ARG;
   if (!aligned16(y_perm) || !aligned16(out) || !aligned16(shared_y)) return MOE_ERR_INVALID_ARG;
   Carver c(ws);

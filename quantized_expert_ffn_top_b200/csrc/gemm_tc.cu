@@ -51,27 +51,42 @@ struct FmtTraits {
 
 template <int FMT, int EPI, int BN>
 struct Cfg {
+  static_assert(BN == 64 || BN == 128 || BN == 256, "token tile width");
   using F = FmtTraits<FMT>;
+  // Scale blocks cover 128 token rows: a 64-wide tile sits in the lower or
+  // upper half of one block (see sfb_col_offset).
+  static constexpr int kSfbBlocks = BN >= 128 ? BN / 128 : 1;
   static constexpr int kA = 128 * 128;
   static constexpr int kB = BN * 128;
   static constexpr int kSFA = F::kGroups * 512;
-  static constexpr int kSFB = F::kGroups * 512 * (BN / 128);
+  static constexpr int kSFB = F::kGroups * 512 * kSfbBlocks;
   static constexpr int kStage = ((kA + kB + kSFA + kSFB) + 1023) / 1024 * 1024;
   static constexpr int kStages = (200 * 1024) / kStage < 8 ? (200 * 1024) / kStage : 8;
-  static constexpr int kAccStages = BN == 256 ? 1 : 2;
-  // 64 accumulator columns per epilogue warp: 2 (BN 128) or 4 (BN 256) warps
-  // per tensor-memory lane quarter
-  static constexpr int kEpiWarps = BN == 256 ? 16 : 8;
+  static constexpr int kAccStages = BN == 256 ? 1 : (BN == 128 ? 2 : 4);
+  // 64 accumulator columns per epilogue warp: 1 (BN 64), 2 (BN 128) or 4
+  // (BN 256) warps per tensor-memory lane quarter
+  static constexpr int kEpiWarps = 4 * (BN / 64);
   static constexpr int kThreads = (2 + kEpiWarps) * 32;
   static constexpr uint32_t kSfaCol = kAccStages * BN;
   static constexpr uint32_t kSfbCol = kSfaCol + F::kGroups * 4;
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr uint32_t kTx = kA + kB + kSFA + kSFB;
   static constexpr int kEpiTile = 16 * 32 * 4;  // per warp pair: 16 tokens x 32 rows, fp32
   static constexpr int kSmem = kStages * kStage + 1024 /*align*/ + 1024 /*barriers etc.*/ +
                                (kEpiWarps / 2) * kEpiTile;
-  static_assert(kSfbCol + F::kGroups * 4 * (BN / 128) <= kTmemCols, "tensor memory overflow");
+  static_assert(kSfbCol + F::kGroups * 4 * kSfbBlocks <= kTmemCols, "tensor memory overflow");
+  // barriers (full, empty, tfull, tempty), the tensor-memory address and the
+  // abort flag share the 1 KB control block
+  static_assert((2 * kStages + 2 * kAccStages) * 8 + 8 <= 1024, "control block overflow");
 };
+
+// Tensor-memory column offset of a tile's first token inside its 128-row
+// scale block: scales of token row r sit in column (r % 128) / 32 of the
+// block's copy, so a 64-wide tile starting half way into the block reads its
+// B scales two columns further on.
+template <int BN>
+__device__ __forceinline__ uint32_t sfb_col_offset(int row0) {
+  return BN >= 128 ? 0u : (uint32_t)((row0 & 127) >> 5);
+}
 
 __device__ __forceinline__ float act_scale_of(int fmt, const float* st, const float* amax) {
   if (fmt == MOE_FMT_MXFP4) return 1.0f;
@@ -102,8 +117,8 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN>::kThreads, 1)
   uint64_t* full = reinterpret_cast<uint64_t*>(ctrl);
   uint64_t* empty = full + C::kStages;
   uint64_t* tfull = empty + C::kStages;
-  uint64_t* tempty = tfull + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  uint64_t* tempty = tfull + C::kAccStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + C::kAccStages);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* epi_tiles = reinterpret_cast<float*>(ctrl + 1024);  // [kEpiWarps / 2][16 tokens][32]
 
@@ -113,7 +128,7 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN>::kThreads, 1)
       tc::mbar_init(&full[s], 1);
       tc::mbar_init(&empty[s], 1);
     }
-    for (int a = 0; a < 2; ++a) {
+    for (int a = 0; a < C::kAccStages; ++a) {
       tc::mbar_init(&tfull[a], 1);
       tc::mbar_init(&tempty[a], C::kEpiWarps);
     }
@@ -195,6 +210,7 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN>::kThreads, 1)
       tc::fence_after_sync();
       const uint32_t n_mma = (uint32_t)min(BN, (te.nvalid + 15) & ~15);
       const uint32_t d = tmem + acc * BN;
+      const uint32_t sfb0 = tmem + C::kSfbCol + sfb_col_offset<BN>(te.row0);
       uint32_t idesc_nv = tc::idesc_mxf4(n_mma, false, 0, 0), idesc_f8 = tc::idesc_f8(n_mma),
                idesc_bf = tc::idesc_bf16(n_mma);
       bool ok = true;
@@ -216,9 +232,9 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN>::kThreads, 1)
             for (int grp = 0; grp < F::kGroups; ++grp) {
               tc::sf_copy(tmem + C::kSfaCol + 4 * grp, dsfa + (uint64_t)(grp * 32));
 #pragma unroll
-              for (int nb = 0; nb < BN / 128; ++nb)
+              for (int nb = 0; nb < C::kSfbBlocks; ++nb)
                 if (nb == 0 || n_mma > 128u)   // second block only for tiles wider than 128 tokens
-                  tc::sf_copy(tmem + C::kSfbCol + grp * 4 * (BN / 128) + nb * 4,
+                  tc::sf_copy(tmem + C::kSfbCol + grp * 4 * C::kSfbBlocks + nb * 4,
                               dsfb + (uint64_t)((nb * F::kGroups + grp) * 32));
             }
           }
@@ -229,12 +245,11 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN>::kThreads, 1)
             const uint64_t db = db0 + (uint64_t)(kk * 2);
             const uint32_t accum = (kb > 0 || kk > 0) ? 1u : 0u;
             if (FMT == MOE_FMT_NVFP4) {
-              tc::mma_nvf4(d, da, db, idesc_nv, tmem + C::kSfaCol + 4 * kk, tmem + C::kSfbCol + kk * 4 * (BN / 128),
-                           accum);
+              tc::mma_nvf4(d, da, db, idesc_nv, tmem + C::kSfaCol + 4 * kk, sfb0 + kk * 4 * C::kSfbBlocks, accum);
             } else if (FMT == MOE_FMT_MXFP4) {
               const uint32_t id = (uint32_t)(kk & 1) * 2;  // two MMAs share one group of four e8m0 scales
               tc::mma_mxf4(d, da, db, tc::idesc_mxf4(n_mma, true, id, id), tmem + C::kSfaCol + 4 * (kk >> 1),
-                           tmem + C::kSfbCol + (kk >> 1) * 4 * (BN / 128), accum);
+                           sfb0 + (kk >> 1) * 4 * C::kSfbBlocks, accum);
             } else if (FMT == MOE_FMT_FP8) {
               tc::mma_f8(d, da, db, idesc_f8, accum);
             } else {
@@ -462,6 +477,7 @@ template <int FMT, int EPI>
 cudaError_t launch_bn(const GemmArgs& g, int bn, const void* a, int64_t ar, const void* b, int64_t br, int sms,
                       cudaStream_t s) {
   if (bn == 256) return launch_cfg<FMT, EPI, 256>(g, a, ar, b, br, sms, s);
+  if (bn == 64) return launch_cfg<FMT, EPI, 64>(g, a, ar, b, br, sms, s);
   return launch_cfg<FMT, EPI, 128>(g, a, ar, b, br, sms, s);
 }
 

@@ -13,44 +13,55 @@
 namespace moe {
 
 // ------------------------------------------------------------ logits ------
-// Small T (decode): one warp per (expert, group of up to 8 tokens); lanes
-// stride over H with 16-byte loads of the Wr row and of each token row.
+// Small T (decode): one block of 8 warps per (expert, group of up to 8
+// tokens).  Each thread takes 8 consecutive columns of every 2048-column
+// stretch of H with 16-byte loads of the Wr row and the token rows, so the
+// block issues all its loads at once; warp sums, then the 8 warps' partial
+// sums are added in shared memory.
 constexpr int kSmallTGroup = 8;
+constexpr int kSmallThreads = 256;
 
-__global__ void __launch_bounds__(128) router_logits_small_kernel(const uint16_t* __restrict__ x, int64_t T, int H,
-                                                                  const uint16_t* __restrict__ wr,
-                                                                  const float* __restrict__ bias, int E,
-                                                                  float* __restrict__ logits) {
+__global__ void __launch_bounds__(kSmallThreads) router_logits_small_kernel(const uint16_t* __restrict__ x, int64_t T,
+                                                                           int H, const uint16_t* __restrict__ wr,
+                                                                           const float* __restrict__ bias, int E,
+                                                                           float* __restrict__ logits) {
+  __shared__ float part[kSmallThreads / 32][kSmallTGroup];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int e = blockIdx.x * 4 + warp;
+  const int e = blockIdx.x;
   const int64_t t0 = (int64_t)blockIdx.y * kSmallTGroup;
-  if (e >= E) return;
   const int nt = (int)((T - t0) < kSmallTGroup ? (T - t0) : kSmallTGroup);
   float acc[kSmallTGroup];
 #pragma unroll
   for (int i = 0; i < kSmallTGroup; ++i) acc[i] = 0.0f;
   const uint16_t* wrow = wr + (int64_t)e * H;
-  for (int h = lane * 8; h < H; h += 32 * 8) {
+  for (int h = threadIdx.x * 8; h < H; h += kSmallThreads * 8) {
     const uint4 wv = __ldg(reinterpret_cast<const uint4*>(wrow + h));
+    uint4 xv[kSmallTGroup];
+#pragma unroll
+    for (int i = 0; i < kSmallTGroup; ++i)
+      xv[i] = i < nt ? __ldg(reinterpret_cast<const uint4*>(x + (t0 + i) * H + h)) : make_uint4(0, 0, 0, 0);
     const uint32_t wa[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
     for (int i = 0; i < kSmallTGroup; ++i) {
-      if (i < nt) {
-        const uint4 xv = __ldg(reinterpret_cast<const uint4*>(x + (t0 + i) * H + h));
-        const uint32_t xa[4] = {xv.x, xv.y, xv.z, xv.w};
+      const uint32_t xa[4] = {xv[i].x, xv[i].y, xv[i].z, xv[i].w};
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          acc[i] = fmaf(__uint_as_float(xa[q] << 16), __uint_as_float(wa[q] << 16), acc[i]);
-          acc[i] = fmaf(__uint_as_float(xa[q] & 0xFFFF0000u), __uint_as_float(wa[q] & 0xFFFF0000u), acc[i]);
-        }
+      for (int q = 0; q < 4; ++q) {
+        acc[i] = fmaf(__uint_as_float(xa[q] << 16), __uint_as_float(wa[q] << 16), acc[i]);
+        acc[i] = fmaf(__uint_as_float(xa[q] & 0xFFFF0000u), __uint_as_float(wa[q] & 0xFFFF0000u), acc[i]);
       }
     }
   }
-  const float b = bias ? __ldg(bias + e) : 0.0f;
 #pragma unroll
   for (int i = 0; i < kSmallTGroup; ++i) {
-    float v = warp_sum(acc[i]);
-    if (lane == 0 && i < nt) logits[(t0 + i) * E + e] = v + b;
+    const float v = warp_sum(acc[i]);
+    if (lane == 0) part[warp][i] = v;
+  }
+  __syncthreads();
+  if (threadIdx.x < nt) {
+    float v = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kSmallThreads / 32; ++w) v += part[w][threadIdx.x];
+    logits[(t0 + threadIdx.x) * E + e] = v + (bias ? __ldg(bias + e) : 0.0f);
   }
 }
 
@@ -111,8 +122,8 @@ cudaError_t launch_router_logits(const uint16_t* x, int64_t T, int H, const uint
                                  float* logits, cudaStream_t s) {
   if (T == 0) return cudaSuccess;
   if (T <= 64 && H % 8 == 0) {
-    dim3 grid((E + 3) / 4, (unsigned)((T + kSmallTGroup - 1) / kSmallTGroup));
-    router_logits_small_kernel<<<grid, 128, 0, s>>>(x, T, H, wr, bias, E, logits);
+    dim3 grid((unsigned)E, (unsigned)((T + kSmallTGroup - 1) / kSmallTGroup));
+    router_logits_small_kernel<<<grid, kSmallThreads, 0, s>>>(x, T, H, wr, bias, E, logits);
   } else {
     dim3 grid((unsigned)((T + 63) / 64), (E + 63) / 64);
     router_logits_tiled_kernel<<<grid, 256, 0, s>>>(x, T, H, wr, bias, E, logits);

@@ -82,3 +82,9 @@ def test_host_side_argument_errors(L):
     assert L.moe_permute(one, 4, 2, 2000, one, one, one, one, 1 << 20, None) == 1
     assert L.moe_set_option(1, 5) == 1 and L.moe_set_option(99, 0) == 1
     assert L.moe_set_option(1, 0) == 0
+    # token tile: 0 (by batch size), 64, 128 or 256
+    assert L.moe_set_option(2, 32) == 1 and L.moe_set_option(2, 96) == 1
+    for v in (64, 128, 256, 0):
+        assert L.moe_set_option(2, v) == 0
+    # combine: k beyond the 1024 the kernel stages
+    assert L.moe_combine(one, one, one, 1, 1025, 8, None, one, one, 1 << 20, None) == 1
