@@ -20,7 +20,8 @@ Rank 0 prints one JSON line.  Besides the contract keys it carries:
   roofline     the dominant stage against the measured peak
   e2e          the same metric with the input copied from pinned host memory
                and the output copied back inside the timed region
-  decode       the decode workload's expert-weight streaming rate (GB/s)
+  decode       the decode workload (T=4, static activation scales): step time
+               and the expert-weight streaming rate of moe_grouped_ffn (GB/s)
   cpu_baseline the CPU oracle on a bounded token sample (rank 0, N = 1)
   clocks       nvidia-smi samples taken during the timed region
 `--impl reference` times the CPU oracle instead (the only other arm).
@@ -56,6 +57,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
+    ap.add_argument("--profile-range", action="store_true",
+                    help="bracket the timed prefill replays with cudaProfilerStart/Stop (for ncu --profile-from-start off)")
     return ap.parse_args()
 
 
@@ -170,6 +173,35 @@ def algorithmic(w, bank_fmt: str, offsets: np.ndarray):
                 zero_experts=int((counts == 0).sum()))
 
 
+PROFILE_RANGE = False
+
+# Sources the grouped GEMM is built from; a stored ncu traffic figure counts
+# only while they are unchanged.
+GEMM_SOURCES = ("gemm_tc.cu", "gemm_tc.cuh", "tc_ptx.cuh", "common.cuh", "kernels.cuh")
+
+
+def gemm_sources_sha256() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in GEMM_SOURCES:
+        with open(os.path.join(ROOT, "quantized_expert_ffn_top_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def measured_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch (read + write) from profiles/traffic.json, or
+    None when none was captured for this kernel and workload or the sources
+    changed since."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p)).get(f"{workload}/{kernel}")
+    if not d or d.get("sources_sha256") != gemm_sources_sha256():
+        return None
+    return d["dram_bytes_per_launch"]
+
+
 def time_forward(ops, torch, layer, w, act, steps, warmup, flush, stage=True, host_io=False):
     """Times `steps` forwards.  Device-resident runs replay a CUDA graph of
     moe_forward (one graph launch per step, L2 flushed before each, CUDA
@@ -210,12 +242,16 @@ def time_forward(ops, torch, layer, w, act, steps, warmup, flush, stage=True, ho
         with torch.cuda.graph(graph):
             fwd()
         torch.cuda.synchronize()
+        if PROFILE_RANGE:
+            torch.cuda.profiler.start()
         for i in range(steps):
             flush.zero_()
             step_evs[i][0].record(stream)
             graph.replay()
             step_evs[i][1].record(stream)
         torch.cuda.synchronize()
+        if PROFILE_RANGE:
+            torch.cuda.profiler.stop()
         if stage:
             evs = [torch.cuda.Event(enable_timing=True) for _ in range(2 * len(ops.STAGES))]
             ops.moe_set_stage_events(evs)
@@ -243,6 +279,40 @@ def time_forward(ops, torch, layer, w, act, steps, warmup, flush, stage=True, ho
     off, _, _ = ops.moe_permute(idx, w.E, ops.new_workspace(1 << 24))
     return dict(ms=per_step, stages=stages, launches=per_step_launches * steps, offsets=off.cpu().numpy(),
                 status=ops.moe_get_device_status(ws))
+
+
+def time_grouped_ffn(ops, torch, layer, w, act, steps, warmup, flush):
+    """Device time of the grouped expert FFN alone (moe_grouped_ffn: tile
+    plan, activation quantisation, gate|up + SwiGLU, down) on the layer's
+    routed slots, one CUDA-graph replay per step, L2 flushed before each."""
+    prepared, x, wr, bias = layer
+    ws = ops.new_workspace(ops.workspace_size(w.T, w.k, prepared, None, act))
+    idx, _ = ops.moe_route(x, wr, bias, w.k, ws)
+    off, perm, _ = ops.moe_permute(idx, w.E, ops.new_workspace(1 << 24))
+    y = torch.empty((w.T * w.k, w.H), dtype=torch.bfloat16, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def ffn():
+        ops.moe_grouped_ffn(x, w.k, perm, off, prepared, act, ws, y_perm=y)
+
+    for _ in range(max(warmup, 1)):
+        ffn()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        ffn()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for i in range(steps):
+        flush.zero_()
+        evs[i][0].record(stream)
+        graph.replay()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    del graph
+    if ops.moe_get_device_status(ws) != 0:
+        raise RuntimeError("device status reported a fault in the grouped FFN")
+    return [a.elapsed_time(b) for a, b in evs], off.cpu().numpy()
 
 
 # ------------------------------------------------------------ CPU oracle ----
@@ -345,6 +415,8 @@ def job_throughput(tokens_per_rank: int, steps: int, world: int, slowest_s: floa
 # ------------------------------------------------------------------ main ----
 def main():
     args = parse()
+    global PROFILE_RANGE
+    PROFILE_RANGE = args.profile_range
     if args.impl == "reference":
         run_reference(args)
         return
@@ -399,7 +471,7 @@ def main():
         flops = alg["flops_up"] if dom == "ffn_up" else alg["flops_down"]
         achieved = flops / (stages[dom] * 1e-3) / 1e12
         roof = {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": peak_tensor, "unit": "TFLOP/s",
-                "frac": achieved / peak_tensor, "traffic": None,
+                "frac": achieved / peak_tensor, "traffic": measured_traffic(dom, w.name),
                 "peak_source": f"{pk_kind} bf16 x {FP4_PER_BF16 if w.fmt != 'fp8' else FP8_PER_BF16:g} nominal ratio"}
     else:
         roof = {"kernel": dom, "bound": "hbm", "achieved": None, "peak": pk["hbm_gbs"], "unit": "GB/s",
@@ -417,15 +489,19 @@ def main():
 
     if not args.no_decode:
         wd = synth.workload("decode")
-        dl = build_layer(ops, synth, torch, wd, static=False)
+        dl = build_layer(ops, synth, torch, wd, static=True)
         rd = time_forward(ops, torch, dl, wd, act, max(args.steps, 20), args.warmup, flush)
-        ad = algorithmic(wd, wd.fmt, rd["offsets"])
-        ffn_ms = rd["stages"].get("ffn_up", 0.0) + rd["stages"].get("ffn_down", 0.0)
+        ffn_runs, d_off = time_grouped_ffn(ops, torch, dl, wd, act, max(args.steps, 20), args.warmup, flush)
+        ad = algorithmic(wd, wd.fmt, d_off)
+        ffn_ms = float(np.mean(ffn_runs))
         gbs = (ad["wbytes_up"] + ad["wbytes_down"]) / (ffn_ms * 1e-3) / 1e9 if ffn_ms else None
-        line["decode"] = {"workload": workload_name(wd), "act_scales": "dynamic", "ms_per_step": float(np.mean(rd["ms"])),
+        line["decode"] = {"workload": workload_name(wd), "act_scales": "static", "ms_per_step": float(np.mean(rd["ms"])),
                           "tokens_per_s": wd.T / (float(np.mean(rd["ms"])) * 1e-3),
                           "expert_weight_bytes": ad["wbytes_up"] + ad["wbytes_down"],
-                          "active_experts": ad["active_experts"], "ffn_ms": ffn_ms, "weight_gbs": gbs,
+                          "active_experts": ad["active_experts"], "ffn_ms": ffn_ms,
+                          "ffn_timing": "moe_grouped_ffn alone, graph replay, L2 flushed", "weight_gbs": gbs,
+                          "traffic": (lambda u, d: u + d if u is not None and d is not None else None)(
+                              measured_traffic("ffn_up", "decode"), measured_traffic("ffn_down", "decode")),
                           "hbm_frac": gbs / pk["hbm_gbs"] if gbs else None, "stages_ms": rd["stages"]}
         del dl
 

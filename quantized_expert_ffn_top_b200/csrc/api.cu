@@ -255,8 +255,8 @@ int gemm_tile_n(int64_t S, int E) {
 }
 
 moe_status run_gemm_ffn(const uint16_t* x, int64_t T, int64_t S, const int32_t* perm, const int32_t* offsets,
-                        const moe_weights* w, uint16_t* y_perm, const FfnScratch& f, float* x_amax, float* h_amax,
-                        int32_t* status, cudaStream_t s, bool mark) {
+                        const int32_t* inv, int k, const moe_weights* w, uint16_t* y_perm, const FfnScratch& f,
+                        float* x_amax, float* h_amax, int32_t* status, cudaStream_t s, bool mark) {
   const int E = w->E, H = w->H, I = w->I, fmt = w->fmt;
   const int sms = num_sms();
   const int bn = gemm_tile_n(S, E);
@@ -271,6 +271,8 @@ moe_status run_gemm_ffn(const uint16_t* x, int64_t T, int64_t S, const int32_t* 
   qa.offsets = offsets;
   qa.poff = f.poff;
   qa.perm_token = perm;
+  qa.inv_perm = inv;
+  qa.k = k;
   qa.x = x;
   qa.h32 = nullptr;
   qa.scale = w->a13_gs;
@@ -344,14 +346,16 @@ moe_status run_gemm_ffn(const uint16_t* x, int64_t T, int64_t S, const int32_t* 
 
 // Grouped FFN on already-validated arguments.  x_amax must hold amax(x) when
 // the x scale is dynamic (MATCH, NVFP4/FP8, no a13_gs).
+// inv (optional, with k = S / T) lets the tensor-core path quantise each
+// token once for all its slots.
 moe_status run_grouped_ffn(const uint16_t* x, int64_t T, int64_t S, const int32_t* perm, const int32_t* offsets,
                            const moe_weights* w, int act, uint16_t* y_perm, const FfnScratch& scratch,
                            float* x_amax, float* h_amax, int32_t* status, cudaStream_t s,
-                           bool shared_stage = false) {
+                           bool shared_stage = false, const int32_t* inv = nullptr, int k = 0) {
   if (S == 0) return MOE_OK;
   const bool mark = !shared_stage;
   if (use_gemm_path(w, S, act))
-    return run_gemm_ffn(x, T, S, perm, offsets, w, y_perm, scratch, x_amax, h_amax, status, s, mark);
+    return run_gemm_ffn(x, T, S, perm, offsets, inv, k, w, y_perm, scratch, x_amax, h_amax, status, s, mark);
   if (g_ffn_path == 2) return MOE_ERR_UNSUPPORTED;
   GemvArgs a;
   a.fmt = w->fmt;
@@ -637,7 +641,7 @@ moe_status moe_forward(const uint16_t* x, int64_t T, const uint16_t* wr, const f
   }
   // 4. routed experts
   st = run_grouped_ffn(x, T, S, f.perm, f.offsets, routed, act, f.y_perm, f.ffn, f.head.x_amax, f.head.h_amax,
-                       f.head.status, s);
+                       f.head.status, s, false, f.inv, k);
   if (st != MOE_OK) return st;
   // 5. shared expert: every token, identity order; it reads routed's x scale
   if (shared) {

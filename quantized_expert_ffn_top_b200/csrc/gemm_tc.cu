@@ -297,15 +297,17 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN>::kThreads, 1)
       const int c_lo = cw * 64;
       const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN) + (uint32_t)c_lo;
       uint32_t r0[16], r1[16], r2[16], r3[16];
-      if (c_lo < ncol) {
+      // 16-column chunks of this warp's slice that hold valid tokens
+      const int nch = c_lo < ncol ? min(4, (ncol - c_lo + 15) >> 4) : 0;
+      if (nch > 0) {
         tc::tmem_ld16_async(tbase, r0);
-        tc::tmem_ld16_async(tbase + 16, r1);
-        tc::tmem_ld16_async(tbase + 32, r2);
-        tc::tmem_ld16_async(tbase + 48, r3);
+        if (nch > 1) tc::tmem_ld16_async(tbase + 16, r1);
+        if (nch > 2) tc::tmem_ld16_async(tbase + 32, r2);
+        if (nch > 3) tc::tmem_ld16_async(tbase + 48, r3);
         tc::tmem_wait16(r0);
-        tc::tmem_wait16(r1);
-        tc::tmem_wait16(r2);
-        tc::tmem_wait16(r3);
+        if (nch > 1) tc::tmem_wait16(r1);
+        if (nch > 2) tc::tmem_wait16(r2);
+        if (nch > 3) tc::tmem_wait16(r3);
       }
       tc::fence_before_sync();
       __syncwarp();
@@ -317,6 +319,7 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN>::kThreads, 1)
       if (c_lo >= ncol) continue;  // both warps of a pair (same slice) skip together
 #pragma unroll
       for (int ch = 0; ch < 4; ++ch) {
+        if (ch >= nch) break;  // both warps of a pair see the same ncol
         const uint32_t* rr = ch == 0 ? r0 : (ch == 1 ? r1 : (ch == 2 ? r2 : r3));
         float v[16];
 #pragma unroll
@@ -697,8 +700,129 @@ __global__ void __launch_bounds__(256) quant_padded_kernel(QuantPaddedArgs a) {
   }
 }
 
+// x rows by token: with a per-tensor (or per-block) activation scale a
+// token's quantised row is the same in each of its k slots, so one warp
+// quantises token t once -- lane l owns 64 consecutive elements of each
+// 2048-element stretch -- and writes the codes and scales to the padded rows
+// of the slots inv_perm[t * k + j].
+template <int FMT>
+__global__ void __launch_bounds__(256) quant_tokens_kernel(QuantPaddedArgs a) {
+  constexpr int bs = FMT == MOE_FMT_MXFP4 ? 32 : 16;
+  constexpr int kPer = 64;
+  constexpr int kWords = FMT == MOE_FMT_FP8 ? 16 : 8;  // 32-bit code words per lane
+  const int nb = a.K / bs;
+  const int lane = threadIdx.x & 31;
+  const float scale = act_scale_of(FMT, a.scale, a.amax);
+  const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < a.T; t += warps) {
+    for (int c0 = 0; c0 < a.K; c0 += 32 * kPer) {
+      const int c = c0 + lane * kPer;
+      const bool active = c < a.K;
+      uint32_t w[kWords];
+      uint32_t sfw = 0;
+      if (active) {
+        float v[kPer];
+        const uint16_t* src = a.x + t * a.K + c;
+#pragma unroll
+        for (int i = 0; i < kPer; i += 8) {
+          const uint4 u = __ldg(reinterpret_cast<const uint4*>(src + i));
+          const uint32_t uu[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            v[i + 2 * j] = __uint_as_float(uu[j] << 16);
+            v[i + 2 * j + 1] = __uint_as_float(uu[j] & 0xFFFF0000u);
+          }
+        }
+        if constexpr (FMT == MOE_FMT_NVFP4) {
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            float bmax = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) bmax = fmaxf(bmax, fabsf(v[16 * b + i]));
+            uint32_t sc;
+            float r;
+            nvfp4_block_scale(bmax, scale, sc, r);
+            const uint2 cw = nvfp4_encode16(v + 16 * b, r);
+            w[2 * b] = cw.x;
+            w[2 * b + 1] = cw.y;
+            sfw |= sc << (8 * b);
+          }
+        } else if constexpr (FMT == MOE_FMT_MXFP4) {
+#pragma unroll
+          for (int b = 0; b < 2; ++b) {
+            float bmax = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) bmax = fmaxf(bmax, fabsf(v[32 * b + i]));
+            uint32_t sc;
+            float inv;
+            mxfp4_block_scale(bmax, sc, inv);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) w[4 * b + q] = e2m1_encode8(v + 32 * b + 8 * q, inv);
+            sfw |= sc << (8 * b);
+          }
+        } else {
+          const float inv = __frcp_rn(scale);
+#pragma unroll
+          for (int i = 0; i < kWords; ++i)
+            w[i] = e4m3x2_encode(__fmul_rn(v[4 * i], inv), __fmul_rn(v[4 * i + 1], inv)) |
+                   (e4m3x2_encode(__fmul_rn(v[4 * i + 2], inv), __fmul_rn(v[4 * i + 3], inv)) << 16);
+        }
+      }
+      for (int j0 = 0; j0 < a.k; j0 += 32) {
+        // lane j resolves the padded row of slot j0 + j (-1: dropped slot, -2: bad)
+        int64_t myrow = -1;
+        if (j0 + lane < a.k) {
+          const int32_t p = __ldg(a.inv_perm + t * a.k + j0 + lane);
+          if (p >= a.S) {
+            myrow = -2;
+          } else if (p >= 0) {
+            const int e = segment_of(a.offsets, a.E, p);
+            const int32_t o = __ldg(a.offsets + e);
+            const int64_t row = (int64_t)__ldg(a.poff + e) + (p - o);
+            myrow = (row >= 0 && row < a.P && p >= o) ? row : -2;
+          }
+        }
+        const int nj = min(32, a.k - j0);
+        for (int jj = 0; jj < nj; ++jj) {
+          const int64_t row = __shfl_sync(0xffffffffu, myrow, jj);
+          if (row < 0) {
+            if (row == -2 && lane == 0 && c0 == 0) raise_status(a.status, MOE_ERR_DEVICE_FAULT);
+            continue;
+          }
+          if (!active) continue;
+          if constexpr (FMT == MOE_FMT_FP8) {
+            uint4* dst = reinterpret_cast<uint4*>(a.codes + row * a.K + c);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) dst[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(a.codes + row * (a.K / 2) + c / 2);
+            dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+            dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+            if constexpr (FMT == MOE_FMT_NVFP4)
+              *reinterpret_cast<uint32_t*>(a.sf + sf_blocked_offset(row, c / bs, nb)) = sfw;
+            else
+              *reinterpret_cast<uint16_t*>(a.sf + sf_blocked_offset(row, c / bs, nb)) = (uint16_t)sfw;
+          }
+        }
+      }
+    }
+  }
+}
+
 cudaError_t launch_quant_padded(const QuantPaddedArgs& a, bool src_x, int fmt, int num_sms, cudaStream_t s) {
   if (a.S == 0) return cudaSuccess;
+  if (src_x && a.inv_perm && a.K % 64 == 0) {
+    const int64_t blocks = (a.T + 7) / 8;
+    const int grid = (int)(blocks < (int64_t)num_sms * 8 ? blocks : (int64_t)num_sms * 8);
+    switch (fmt) {
+      case MOE_FMT_NVFP4: quant_tokens_kernel<MOE_FMT_NVFP4><<<grid, 256, 0, s>>>(a); break;
+      case MOE_FMT_MXFP4: quant_tokens_kernel<MOE_FMT_MXFP4><<<grid, 256, 0, s>>>(a); break;
+      case MOE_FMT_FP8: quant_tokens_kernel<MOE_FMT_FP8><<<grid, 256, 0, s>>>(a); break;
+      default: return cudaErrorInvalidValue;
+    }
+    count_launches(1);
+    return cudaGetLastError();
+  }
   const int64_t blocks = (a.S + 7) / 8;
   const int grid = (int)(blocks < (int64_t)num_sms * 8 ? blocks : (int64_t)num_sms * 8);
 #define MOE_QP(F)                                                              \

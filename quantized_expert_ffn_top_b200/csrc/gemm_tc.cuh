@@ -48,6 +48,8 @@ struct QuantPaddedArgs {
   const int32_t* offsets;      // [E+1] compact
   const int32_t* poff;         // [E+1] padded
   const int32_t* perm_token;   // x source: token of each slot
+  const int32_t* inv_perm;     // x source, optional: slot of each (token, j); then each
+  int k;                       //   token is quantised once and written to its k slots
   const uint16_t* x;           // [T][K] bf16
   const float* h32;            // or fp32 rows at padded positions
   const float* scale;          // static tensor scale or NULL

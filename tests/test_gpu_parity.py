@@ -244,6 +244,9 @@ FWD_CASES = [
     ("decode", {}, 1, False), ("decode", {}, 0, False), ("decode", {}, 1, True),
     ("fp8_shared", dict(T=24, H=256, E=16, k=4, I=128, shared_I=128), 1, False),
     ("tiny", dict(fmt="mxfp4", T=12, H=256, E=8, k=2, I=256), 1, False),
+    # H = 2048 + 256: the per-token x quantiser's second stretch is ragged
+    ("tiny", dict(T=40, H=2304, E=8, k=3, I=256), 1, False),
+    ("tiny", dict(fmt="fp8", T=40, H=2176, E=8, k=3, I=256), 1, False),
 ]
 
 
