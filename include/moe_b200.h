@@ -197,7 +197,7 @@ moe_status moe_permute(const int32_t* topk_idx, int64_t T, int32_t k, int32_t E,
  * PREPARED.  With quantised activations (MATCH) and H, I multiples of 256
  * (FP4) or 128 (FP8) the FFN runs as a tcgen05 block-scaled grouped GEMM at
  * every batch size -- 64-token tiles while T*k < 8E (decode: each active
- * expert's weights stream once), 256-token tiles beyond (prefill).  BF16
+ * expert's weights stream once), 192- or 256-token tiles beyond (prefill).  BF16
  * activations and other shapes take a TMA-fed mma.sync GEMV that streams
  * each active expert's weights once (the decode split of the atomicmilkshake
  * fork README, "Quant types": MMVQ for decode, MMQ for prefill).  The choice
@@ -239,9 +239,14 @@ moe_status moe_get_device_status(void* ws, moe_stream_t stream, int32_t* host_st
  *                     MOE_ERR_UNSUPPORTED where the shapes do not allow it).
  * Not thread-safe; set before enqueuing. */
 /*   MOE_OPT_GEMM_TILE_N: token-tile width of the tensor-core path: 0 (default:
- *                     64 while T*k < 8E, else 256), 64 (four accumulators),
- *                     128 (two) or 256 (one, drained to registers). */
-typedef enum { MOE_OPT_FFN_PATH = 1, MOE_OPT_GEMM_TILE_N = 2 } moe_option;
+ *                     64 while T*k < 8E, 192 while T*k <= 384E, else 256),
+ *                     64 (four accumulators), 128 or 192 (two) or 256 (one,
+ *                     drained to registers).
+ *   MOE_OPT_GEMM_PAIR: 1 runs 256-token tiles on CTA pairs (tcgen05
+ *                     cta_group::2, 256 weight rows per tile) when the weight
+ *                     rows per expert divide by 256; 0 (default) keeps one
+ *                     CTA per 128-row tile. */
+typedef enum { MOE_OPT_FFN_PATH = 1, MOE_OPT_GEMM_TILE_N = 2, MOE_OPT_GEMM_PAIR = 3 } moe_option;
 moe_status moe_set_option(int32_t option, int32_t value);
 
 /* moe_permute for callers that cannot allocate device memory (no workspace

@@ -247,11 +247,14 @@ bool use_gemm_path(const moe_weights* w, int64_t S, int act) {
 }
 
 // Token tile: 64 wide while the average expert holds fewer than 8 slots
-// (decode: deep weight streaming, small B stages), 256 wide beyond.
-// Arguments only, no device read-back.
+// (decode: deep weight streaming, small B stages); 192 wide up to 384 slots
+// per expert on average (two accumulator buffers, so one tile's epilogue
+// overlaps the next tile's MMAs); 256 wide beyond, where full tiles
+// dominate.  Arguments only, no device read-back.
 int gemm_tile_n(int64_t S, int E) {
   if (g_gemm_bn) return g_gemm_bn;
-  return S < 8 * (int64_t)E ? 64 : 256;
+  if (S < 8 * (int64_t)E) return 64;
+  return S <= 384 * (int64_t)E ? 192 : 256;
 }
 
 moe_status run_gemm_ffn(const uint16_t* x, int64_t T, int64_t S, const int32_t* perm, const int32_t* offsets,
@@ -440,8 +443,13 @@ moe_status moe_set_option(int32_t option, int32_t value) {
     return MOE_OK;
   }
   if (option == MOE_OPT_GEMM_TILE_N) {
-    if (value != 0 && value != 64 && value != 128 && value != 256) return MOE_ERR_INVALID_ARG;
+    if (value != 0 && value != 64 && value != 128 && value != 192 && value != 256) return MOE_ERR_INVALID_ARG;
     g_gemm_bn = value;
+    return MOE_OK;
+  }
+  if (option == MOE_OPT_GEMM_PAIR) {
+    if (value != 0 && value != 1) return MOE_ERR_INVALID_ARG;
+    set_gemm_pairs(value != 0);
     return MOE_OK;
   }
   return MOE_ERR_INVALID_ARG;

@@ -49,24 +49,31 @@ struct FmtTraits {
   static constexpr int kGroups = kBs ? kBK / (4 * kBs) : 0;         // 4-column scale groups per stage
 };
 
-template <int FMT, int EPI, int BN>
+// PAIR: a tile is 256 weight rows x BN tokens computed by a cluster of two
+// CTAs (cta_group::2): each CTA stages its 128 weight rows, half of the token
+// rows and all BN tokens' scales, and owns its 128 rows of the accumulator.
+template <int FMT, int EPI, int BN, bool PAIR = false>
 struct Cfg {
-  static_assert(BN == 64 || BN == 128 || BN == 256, "token tile width");
+  static_assert(BN == 64 || BN == 128 || BN == 192 || BN == 256, "token tile width");
+  static_assert(!PAIR || BN == 256, "CTA pairs run 256-token tiles");
   using F = FmtTraits<FMT>;
-  // Scale blocks cover 128 token rows: a 64-wide tile sits in the lower or
-  // upper half of one block (see sfb_col_offset).
-  static constexpr int kSfbBlocks = BN >= 128 ? BN / 128 : 1;
+  // Scale blocks cover 128 token rows; a tile starts on a multiple of 64
+  // rows, so a 192-wide tile may start half way into its first block and
+  // spans two (see sfb_col_offset).
+  static constexpr int kSfbBlocks = (BN + 127) / 128;
   static constexpr int kA = 128 * 128;
-  static constexpr int kB = BN * 128;
+  static constexpr int kB = (PAIR ? BN / 2 : BN) * 128;
   static constexpr int kSFA = F::kGroups * 512;
   static constexpr int kSFB = F::kGroups * 512 * kSfbBlocks;
   static constexpr int kStage = ((kA + kB + kSFA + kSFB) + 1023) / 1024 * 1024;
   static constexpr int kStages = (200 * 1024) / kStage < 8 ? (200 * 1024) / kStage : 8;
-  static constexpr int kAccStages = BN == 256 ? 1 : (BN == 128 ? 2 : 4);
-  // 64 accumulator columns per epilogue warp: 1 (BN 64), 2 (BN 128) or 4
-  // (BN 256) warps per tensor-memory lane quarter
+  static constexpr int kAccStages = BN == 256 ? 1 : (BN >= 128 ? 2 : 4);
+  // 64 accumulator columns per epilogue warp: BN / 64 warps per
+  // tensor-memory lane quarter
   static constexpr int kEpiWarps = 4 * (BN / 64);
   static constexpr int kThreads = (2 + kEpiWarps) * 32;
+  // arrivals that free an accumulator buffer: every epilogue warp of the tile
+  static constexpr uint32_t kTemptyCount = kEpiWarps * (PAIR ? 2 : 1);
   static constexpr uint32_t kSfaCol = kAccStages * BN;
   static constexpr uint32_t kSfbCol = kSfaCol + F::kGroups * 4;
   static constexpr uint32_t kTmemCols = 512;
@@ -81,11 +88,12 @@ struct Cfg {
 
 // Tensor-memory column offset of a tile's first token inside its 128-row
 // scale block: scales of token row r sit in column (r % 128) / 32 of the
-// block's copy, so a 64-wide tile starting half way into the block reads its
-// B scales two columns further on.
+// block's copy and consecutive blocks' copies are adjacent, so a tile
+// starting half way into a block (64- and 192-wide tiles) reads its B scales
+// two columns further on.
 template <int BN>
 __device__ __forceinline__ uint32_t sfb_col_offset(int row0) {
-  return BN >= 128 ? 0u : (uint32_t)((row0 & 127) >> 5);
+  return (BN == 64 || BN == 192) ? (uint32_t)((row0 & 127) >> 5) : 0u;
 }
 
 __device__ __forceinline__ float act_scale_of(int fmt, const float* st, const float* amax) {
@@ -105,11 +113,12 @@ __device__ __forceinline__ int token_box_index(int rows) {
   return rows <= 16 ? 0 : (rows <= 32 ? 1 : (rows <= 64 ? 2 : (rows <= 128 ? 3 : 4)));
 }
 
-template <int FMT, int EPI, int BN>
-__global__ void __launch_bounds__(Cfg<FMT, EPI, BN>::kThreads, 1)
+template <int FMT, int EPI, int BN, bool PAIR>
+__global__ void __launch_bounds__(Cfg<FMT, EPI, BN, PAIR>::kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ TokenMaps tmaps_b,
+                        const __grid_constant__ CUtensorMap tmap_sfa, const __grid_constant__ CUtensorMap tmap_sfb,
                         const GemmArgs g) {
-  using C = Cfg<FMT, EPI, BN>;
+  using C = Cfg<FMT, EPI, BN, PAIR>;
   using F = FmtTraits<FMT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -130,24 +139,39 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN>::kThreads, 1)
     }
     for (int a = 0; a < C::kAccStages; ++a) {
       tc::mbar_init(&tfull[a], 1);
-      tc::mbar_init(&tempty[a], C::kEpiWarps);
+      tc::mbar_init(&tempty[a], C::kTemptyCount);
     }
     *abort = 0;
     tc::fence_mbar_init();
     tc::prefetch_tmap(&tmap_a);
 #pragma unroll
     for (int i = 0; i < 5; ++i) tc::prefetch_tmap(&tmaps_b.m[i]);
+    if (PAIR && F::kBs) {
+      tc::prefetch_tmap(&tmap_sfa);
+      tc::prefetch_tmap(&tmap_sfb);
+    }
   }
   if (warp == 1) {
-    tc::tmem_alloc(tmem_slot, C::kTmemCols);
-    tc::tmem_relinquish();
+    if constexpr (PAIR) {
+      tc::tmem_alloc_pair(tmem_slot, C::kTmemCols);
+      tc::tmem_relinquish_pair();
+    } else {
+      tc::tmem_alloc(tmem_slot, C::kTmemCols);
+      tc::tmem_relinquish();
+    }
   }
   tc::fence_before_sync();
   __syncthreads();
+  // the peer's barriers must be initialised before either CTA signals them
+  if constexpr (PAIR) tc::cluster_sync();
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
-  const int MT = g.R / 128;
+  const uint32_t rank = PAIR ? tc::cluster_rank() : 0u;
+  // tiles: (token tile, weight-row block of 128 rows, or 256 for a pair)
+  const int MT = g.R / (PAIR ? 256 : 128);
   const int ntiles = __ldg(g.num_tiles) * MT;
+  const int t_first = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int t_step = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
   const int nkb = g.K / F::kBK;
   const int ncols_w = F::kBs ? g.K / F::kBs : 0;  // scale columns per row (multiple of 4)
 
@@ -159,9 +183,9 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN>::kThreads, 1)
     // ------------------------------------------------------------ producer
     int stage = 0;
     uint32_t phase = 0;
-    for (int t = blockIdx.x; t < ntiles && !*abort; t += gridDim.x) {
+    for (int t = t_first; t < ntiles && !*abort; t += t_step) {
       const TileEntry te = g.tiles[t / MT];
-      const int mt = t % MT;
+      const int mt = PAIR ? (t % MT) * 2 + (int)rank : t % MT;   // this CTA's 128-row weight block
       const uint8_t* sfa = F::kBs ? g.w_sf + (size_t)te.e * g.R * ncols_w + (size_t)mt * (ncols_w / 4) * 512 : nullptr;
       for (int kb = 0; kb < nkb; ++kb) {
         if (!tc::mbar_wait(&empty[stage], phase ^ 1u, abort)) {
@@ -169,11 +193,32 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN>::kThreads, 1)
           *abort = 1;
           break;
         }
-        if (tc::elect_one()) {
+        if (PAIR && tc::elect_one()) {
+          // Both CTAs load their halves; the bytes complete on the leader's
+          // barrier, which the leader alone arms with the pair's total.
+          uint8_t* st = smem + stage * C::kStage;
+          const int nh = min(BN, (te.nvalid + 31) & ~31) >> 1;      // token rows per CTA
+          const int bi = token_box_index(nh);
+          const uint32_t brows = min(16u << bi, (uint32_t)BN);   // the map's box height
+          const int nblk = (min(te.nvalid, BN) + 127) / 128;
+          const uint32_t cbar = tc::cluster_addr(&full[stage], 0);
+          if (rank == 0)
+            tc::mbar_expect_tx(&full[stage], 2u * (C::kA + brows * 128u + C::kSFA + nblk * F::kGroups * 512));
+          tc::tma_load_2d_pair(st, &tmap_a, cbar, kb * 128, te.e * g.R + mt * 128);
+          tc::tma_load_2d_pair(st + C::kA, &tmaps_b.m[bi], cbar, kb * 128, te.row0 + (int)rank * nh);
+          if (F::kBs) {
+            // scale maps: one 512-byte block per row
+            const int wblk = (te.e * (g.R / 128) + mt) * (ncols_w / 4) + kb * F::kGroups;
+            tc::tma_load_2d_pair(st + C::kA + C::kB, &tmap_sfa, cbar, 0, wblk);
+            for (int nb = 0; nb < nblk; ++nb)
+              tc::tma_load_2d_pair(st + C::kA + C::kB + C::kSFA + nb * F::kGroups * 512, &tmap_sfb, cbar, 0,
+                                   (te.row0 / 128 + nb) * (ncols_w / 4) + kb * F::kGroups);
+          }
+        } else if (!PAIR && tc::elect_one()) {
           uint8_t* st = smem + stage * C::kStage;
           const int bi = token_box_index(min(te.nvalid, BN));
-          const uint32_t brows = 16u << bi;
-          const int nblk = (min(te.nvalid, BN) + 127) / 128;   // 128-row scale blocks in use
+          const uint32_t brows = min(16u << bi, (uint32_t)BN);   // the map's box height
+          const int nblk = ((te.row0 & 127) + min(te.nvalid, BN) + 127) / 128;   // 128-row scale blocks in use
           tc::mbar_expect_tx(&full[stage], C::kA + brows * 128u + C::kSFA + nblk * F::kGroups * 512);
           tc::tma_load_2d(st, &tmap_a, &full[stage], kb * 128, te.e * g.R + mt * 128);
           tc::tma_load_2d(st + C::kA, &tmaps_b.m[bi], &full[stage], kb * 128, te.row0);
@@ -200,7 +245,8 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN>::kThreads, 1)
     uint32_t phase = 0;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int t = blockIdx.x; t < ntiles && !*abort; t += gridDim.x) {
+    // a pair's MMAs are issued by its leader (rank 0) alone
+    for (int t = t_first; (!PAIR || rank == 0) && t < ntiles && !*abort; t += t_step) {
       const TileEntry te = g.tiles[t / MT];
       if (!tc::mbar_wait(&tempty[acc], acc_phase ^ 1u, abort)) {
         if (lane == 0) raise_status(g.status, MOE_ERR_TIMEOUT);
@@ -208,10 +254,12 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN>::kThreads, 1)
         break;
       }
       tc::fence_after_sync();
-      const uint32_t n_mma = (uint32_t)min(BN, (te.nvalid + 15) & ~15);
+      // N: valid tokens rounded up to 16 (to 32 for a pair: each CTA holds N/2)
+      const uint32_t n_mma = (uint32_t)min(BN, PAIR ? (te.nvalid + 31) & ~31 : (te.nvalid + 15) & ~15);
       const uint32_t d = tmem + acc * BN;
       const uint32_t sfb0 = tmem + C::kSfbCol + sfb_col_offset<BN>(te.row0);
-      uint32_t idesc_nv = tc::idesc_mxf4(n_mma, false, 0, 0), idesc_f8 = tc::idesc_f8(n_mma),
+      constexpr uint32_t kM = PAIR ? 256u : 128u;
+      uint32_t idesc_nv = tc::idesc_mxf4(n_mma, false, 0, 0, kM), idesc_f8 = tc::idesc_f8(n_mma, kM),
                idesc_bf = tc::idesc_bf16(n_mma);
       bool ok = true;
       for (int kb = 0; kb < nkb; ++kb) {
@@ -230,12 +278,16 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN>::kThreads, 1)
             const uint64_t dsfb = dsfa + (uint64_t)(C::kSFA >> 4);
 #pragma unroll
             for (int grp = 0; grp < F::kGroups; ++grp) {
-              tc::sf_copy(tmem + C::kSfaCol + 4 * grp, dsfa + (uint64_t)(grp * 32));
+              if constexpr (PAIR) tc::sf_copy_pair(tmem + C::kSfaCol + 4 * grp, dsfa + (uint64_t)(grp * 32));
+              else tc::sf_copy(tmem + C::kSfaCol + 4 * grp, dsfa + (uint64_t)(grp * 32));
 #pragma unroll
               for (int nb = 0; nb < C::kSfbBlocks; ++nb)
-                if (nb == 0 || n_mma > 128u)   // second block only for tiles wider than 128 tokens
-                  tc::sf_copy(tmem + C::kSfbCol + grp * 4 * C::kSfbBlocks + nb * 4,
-                              dsfb + (uint64_t)((nb * F::kGroups + grp) * 32));
+                if (nb == 0 || (uint32_t)(te.row0 & 127) + n_mma > 128u) {  // second block only when the tile reaches it
+                  const uint32_t ta = tmem + C::kSfbCol + grp * 4 * C::kSfbBlocks + nb * 4;
+                  const uint64_t sd = dsfb + (uint64_t)((nb * F::kGroups + grp) * 32);
+                  if constexpr (PAIR) tc::sf_copy_pair(ta, sd);
+                  else tc::sf_copy(ta, sd);
+                }
             }
           }
           const uint64_t da0 = tc::desc_sw128(sa), db0 = tc::desc_sw128(sb);
@@ -245,18 +297,24 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN>::kThreads, 1)
             const uint64_t db = db0 + (uint64_t)(kk * 2);
             const uint32_t accum = (kb > 0 || kk > 0) ? 1u : 0u;
             if (FMT == MOE_FMT_NVFP4) {
-              tc::mma_nvf4(d, da, db, idesc_nv, tmem + C::kSfaCol + 4 * kk, sfb0 + kk * 4 * C::kSfbBlocks, accum);
+              const uint32_t sa_t = tmem + C::kSfaCol + 4 * kk, sb_t = sfb0 + kk * 4 * C::kSfbBlocks;
+              if constexpr (PAIR) tc::mma_nvf4_pair(d, da, db, idesc_nv, sa_t, sb_t, accum);
+              else tc::mma_nvf4(d, da, db, idesc_nv, sa_t, sb_t, accum);
             } else if (FMT == MOE_FMT_MXFP4) {
               const uint32_t id = (uint32_t)(kk & 1) * 2;  // two MMAs share one group of four e8m0 scales
-              tc::mma_mxf4(d, da, db, tc::idesc_mxf4(n_mma, true, id, id), tmem + C::kSfaCol + 4 * (kk >> 1),
-                           sfb0 + (kk >> 1) * 4 * C::kSfbBlocks, accum);
+              const uint32_t sa_t = tmem + C::kSfaCol + 4 * (kk >> 1), sb_t = sfb0 + (kk >> 1) * 4 * C::kSfbBlocks;
+              if constexpr (PAIR) tc::mma_mxf4_pair(d, da, db, tc::idesc_mxf4(n_mma, true, id, id, kM), sa_t, sb_t, accum);
+              else tc::mma_mxf4(d, da, db, tc::idesc_mxf4(n_mma, true, id, id), sa_t, sb_t, accum);
             } else if (FMT == MOE_FMT_FP8) {
-              tc::mma_f8(d, da, db, idesc_f8, accum);
+              if constexpr (PAIR) tc::mma_f8_pair(d, da, db, idesc_f8, accum);
+              else tc::mma_f8(d, da, db, idesc_f8, accum);
             } else {
               tc::mma_bf16(d, da, db, idesc_bf, accum);
             }
           }
-          tc::mma_commit(&empty[stage]);
+          // frees the stage in both CTAs of a pair
+          if constexpr (PAIR) tc::mma_commit_pair(&empty[stage], 0x3);
+          else tc::mma_commit(&empty[stage]);
         }
         __syncwarp();
         if (++stage == C::kStages) {
@@ -265,7 +323,10 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN>::kThreads, 1)
         }
       }
       if (!ok) break;
-      if (tc::elect_one()) tc::mma_commit(&tfull[acc]);
+      if (tc::elect_one()) {
+        if constexpr (PAIR) tc::mma_commit_pair(&tfull[acc], 0x3);
+        else tc::mma_commit(&tfull[acc]);
+      }
       __syncwarp();
       if (++acc == C::kAccStages) {
         acc = 0;
@@ -284,7 +345,7 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN>::kThreads, 1)
     float hmax = 0.0f;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+    for (int t = t_first; t < ntiles; t += t_step) {
       if (!tc::mbar_wait(&tfull[acc], acc_phase, abort)) {
         if (lane == 0) raise_status(g.status, MOE_ERR_TIMEOUT);
         *abort = 1;
@@ -292,7 +353,7 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN>::kThreads, 1)
       }
       tc::fence_after_sync();
       const TileEntry te = g.tiles[t / MT];
-      const int mt = t % MT;
+      const int mt = PAIR ? (t % MT) * 2 + (int)rank : t % MT;   // this CTA's 128 weight rows
       const int ncol = min(BN, (te.nvalid + 15) & ~15);
       const int c_lo = cw * 64;
       const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN) + (uint32_t)c_lo;
@@ -311,7 +372,10 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN>::kThreads, 1)
       }
       tc::fence_before_sync();
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&tempty[acc]);
+      if (lane == 0) {
+        if constexpr (PAIR) tc::mbar_arrive_cluster(tc::cluster_addr(&tempty[acc], 0));   // the leader's MMA waits
+        else tc::mbar_arrive(&tempty[acc]);
+      }
       if (++acc == C::kAccStages) {
         acc = 0;
         acc_phase ^= 1u;
@@ -424,8 +488,14 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN>::kThreads, 1)
     while (clock64() - t0 < 2000000LL) {
     }
   }
+  // Neither CTA of a pair leaves while the other may still signal its
+  // barriers or (leader's MMAs) read its shared memory.
+  if constexpr (PAIR) tc::cluster_sync();
   tc::fence_after_sync();
-  if (warp == 1) tc::tmem_dealloc(tmem, C::kTmemCols);
+  if (warp == 1) {
+    if constexpr (PAIR) tc::tmem_dealloc_pair(tmem, C::kTmemCols);
+    else tc::tmem_dealloc(tmem, C::kTmemCols);
+  }
 }
 
 // ------------------------------------------------------------- tensor maps --
@@ -458,20 +528,77 @@ bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t row_bytes,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int FMT, int EPI, int BN>
+// Scale-factor blocks as rows of a 2D map (128 x 32-bit = one 512-byte block
+// per row), so a stage's groups arrive with one tensor copy.
+bool make_sf_map(CUtensorMap* m, const void* base, int64_t nblocks, int box_blocks) {
+  EncodeTiled fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {128u, (cuuint64_t)nblocks};
+  cuuint64_t strides[1] = {512u};
+  cuuint32_t box[2] = {128u, (cuuint32_t)box_blocks};
+  cuuint32_t es[2] = {1u, 1u};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool g_gemm_pairs = false;  // CTA pairs for 256-token tiles (MOE_OPT_GEMM_PAIR)
+
+template <int FMT, int EPI, int BN, bool PAIR>
 cudaError_t launch_cfg(const GemmArgs& g, const void* a_base, int64_t a_rows, const void* b_base, int64_t b_rows,
                        int num_sms, cudaStream_t s) {
-  using C = Cfg<FMT, EPI, BN>;
-  CUtensorMap ma;
+  using C = Cfg<FMT, EPI, BN, PAIR>;
+  using F = FmtTraits<FMT>;
+  CUtensorMap ma, msfa, msfb;
   TokenMaps mb;
+  memset(&msfa, 0, sizeof(msfa));
+  memset(&msfb, 0, sizeof(msfb));
   const int64_t rb = FMT == kFmtBF16 ? 2 * (int64_t)g.K : (FMT == MOE_FMT_FP8 ? g.K : g.K / 2);
   if (!make_map(&ma, a_base, a_rows, rb, 128)) return cudaErrorInvalidValue;
   for (int i = 0; i < 5; ++i)
     if (!make_map(&mb.m[i], b_base, b_rows, rb, (16 << i) < BN ? (16 << i) : BN)) return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<FMT, EPI, BN>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+  if (PAIR && F::kBs) {
+    const int64_t groups = g.K / F::kBs / 4;  // 512-byte blocks per 128 rows
+    if (!make_sf_map(&msfa, g.w_sf, a_rows / 128 * groups, F::kGroups)) return cudaErrorInvalidValue;
+    if (!make_sf_map(&msfb, g.b_sf, b_rows / 128 * groups, F::kGroups)) return cudaErrorInvalidValue;
+  }
+  auto kern = grouped_gemm_kernel<FMT, EPI, BN, PAIR>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return e;
-  grouped_gemm_kernel<FMT, EPI, BN><<<num_sms, C::kThreads, C::kSmem, s>>>(ma, mb, g);
+  if constexpr (PAIR) {
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.blockDim = dim3(C::kThreads);
+    cfg.dynamicSmemBytes = C::kSmem;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    // persistent: as many pairs as can be resident at once
+    static int max_pairs[16];
+    int dev = 0;
+    e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 16) return cudaErrorInvalidDevice;
+    if (max_pairs[dev] == 0) {
+      cfg.gridDim = dim3((unsigned)(num_sms & ~1));
+      int n = 0;
+      e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+      if (e != cudaSuccess) return e;
+      if (n < 1) return cudaErrorInvalidConfiguration;
+      max_pairs[dev] = n;
+    }
+    const int pairs = max_pairs[dev] < num_sms / 2 ? max_pairs[dev] : num_sms / 2;
+    cfg.gridDim = dim3((unsigned)(2 * pairs));
+    e = cudaLaunchKernelEx(&cfg, kern, ma, mb, msfa, msfb, g);
+    if (e != cudaSuccess) return e;
+  } else {
+    kern<<<num_sms, C::kThreads, C::kSmem, s>>>(ma, mb, msfa, msfb, g);
+  }
   count_launches(1);
   return cudaGetLastError();
 }
@@ -479,9 +606,12 @@ cudaError_t launch_cfg(const GemmArgs& g, const void* a_base, int64_t a_rows, co
 template <int FMT, int EPI>
 cudaError_t launch_bn(const GemmArgs& g, int bn, const void* a, int64_t ar, const void* b, int64_t br, int sms,
                       cudaStream_t s) {
-  if (bn == 256) return launch_cfg<FMT, EPI, 256>(g, a, ar, b, br, sms, s);
-  if (bn == 64) return launch_cfg<FMT, EPI, 64>(g, a, ar, b, br, sms, s);
-  return launch_cfg<FMT, EPI, 128>(g, a, ar, b, br, sms, s);
+  if (bn == 256 && g_gemm_pairs && g.R % 256 == 0 && sms >= 2)
+    return launch_cfg<FMT, EPI, 256, true>(g, a, ar, b, br, sms, s);
+  if (bn == 256) return launch_cfg<FMT, EPI, 256, false>(g, a, ar, b, br, sms, s);
+  if (bn == 192) return launch_cfg<FMT, EPI, 192, false>(g, a, ar, b, br, sms, s);
+  if (bn == 64) return launch_cfg<FMT, EPI, 64, false>(g, a, ar, b, br, sms, s);
+  return launch_cfg<FMT, EPI, 128, false>(g, a, ar, b, br, sms, s);
 }
 
 template <int FMT>
@@ -506,6 +636,8 @@ cudaError_t launch_grouped_gemm(const GemmArgs& g, int epi, int bn, const void* 
 }
 
 bool tensor_maps_available() { return encode_fn() != nullptr; }
+
+void set_gemm_pairs(bool on) { g_gemm_pairs = on; }
 
 __global__ void dense_plan_kernel(int64_t T, int bn, TileEntry* __restrict__ tiles, int32_t* __restrict__ num_tiles) {
   const int n = (int)((T + bn - 1) / bn);
@@ -546,7 +678,7 @@ cudaError_t launch_router_gemm(const uint16_t* x, int64_t T, int H, const uint16
   g.status = status;
   const int64_t ntiles = (T + kBN - 1) / kBN * (E / 128);
   const int grid = (int)(ntiles < num_sms ? ntiles : num_sms);
-  return launch_cfg<kFmtBF16, kEpiLogits, kBN>(g, wr, E, x, T, grid, s);
+  return launch_cfg<kFmtBF16, kEpiLogits, kBN, false>(g, wr, E, x, T, grid, s);
 }
 
 // ---------------------------------------------------------------- planning --

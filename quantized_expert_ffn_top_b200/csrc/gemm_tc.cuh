@@ -65,6 +65,8 @@ cudaError_t launch_quant_padded(const QuantPaddedArgs& a, bool src_x, int fmt, i
 cudaError_t launch_grouped_gemm(const GemmArgs& g, int epi, int bn, const void* a_base, int64_t a_rows,
                                 const void* b_base, int64_t b_rows, int num_sms, cudaStream_t s);
 bool tensor_maps_available();
+// CTA pairs (cta_group::2) for 256-token tiles whose weight rows divide by 256.
+void set_gemm_pairs(bool on);
 cudaError_t launch_dense_plan(int64_t T, int bn, TileEntry* tiles, int32_t* num_tiles, cudaStream_t s);
 // Router logits on the tensor cores: logits[T][E] = x Wr^T (+ bias); E % 128 == 0, H % 64 == 0.
 cudaError_t launch_router_gemm(const uint16_t* x, int64_t T, int H, const uint16_t* wr, const float* bias, int E,

@@ -56,6 +56,29 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, volatile
   return true;
 }
 
+// ----------------------------------------------------- CTA pairs (clusters) --
+// A tile of two CTAs (cluster of 2, cta_group::2): rank 0 issues the MMAs,
+// each CTA stages its half of the operands and owns its half of the result.
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// Address of the same shared-memory object in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t cluster_addr(const void* p, uint32_t rank) {
+  uint32_t d;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(d) : "r"(smem_u32(p)), "r"(rank));
+  return d;
+}
+// Arrive on an mbarrier given by its cluster address (this CTA's or the peer's).
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cbar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cbar) : "memory");
+}
+// All threads of both CTAs (memory ordered at cluster scope).
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ TMA --
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(m) : "memory");
@@ -66,6 +89,15 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* m, uin
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
       "[%4];" ::"r"(smem_u32(dst)),
       "l"(m), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+// The same load into this CTA's shared memory, completing on an mbarrier
+// given by its cluster address, which may be the pair leader's (cta_group::2).
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* m, uint32_t cbar, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+      "[%4];" ::"r"(smem_u32(dst)),
+      "l"(m), "r"(x), "r"(y), "r"(cbar)
       : "memory");
 }
 // Contiguous copy (16-byte aligned addresses, size a multiple of 16).
@@ -88,6 +120,18 @@ __device__ __forceinline__ void tmem_relinquish() {
 __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
   asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
 }
+// Pair forms: both CTAs' warps with the same warp index call them.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
 __device__ __forceinline__ void fence_before_sync() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void fence_after_sync() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
@@ -97,10 +141,25 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
                : "memory");
 }
 
+// Pair form: arrive on the barrier at this address in every CTA of `mask`
+// once all tcgen05 operations of the pair this thread issued completed.
+__device__ __forceinline__ void mma_commit_pair(uint64_t* bar, uint16_t mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"(mask)
+      : "memory");
+}
+
 // Scale factors: 32 rows x 128 bits from shared memory, replicated into the
 // four 32-lane quarters of tensor memory.
 __device__ __forceinline__ void sf_copy(uint32_t taddr, uint64_t sdesc) {
   asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// Pair form: each CTA's shared memory to its own tensor memory.
+__device__ __forceinline__ void sf_copy_pair(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
 // D[tmem] (+)= A[smem] x B[smem]^T, block-scaled e2m1 with e4m3 scales per 16.
@@ -126,6 +185,33 @@ __device__ __forceinline__ void mma_f8(uint32_t d, uint64_t a, uint64_t b, uint3
   asm volatile(
       "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Pair forms (issued by the pair leader): A is M = 256 rows, 128 in each
+// CTA's shared memory at the same offset; B's N columns are split in halves
+// the same way; each CTA's tensor memory receives its 128 rows of D.
+__device__ __forceinline__ void mma_nvf4_pair(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t sfa,
+                                              uint32_t sfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+__device__ __forceinline__ void mma_mxf4_pair(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t sfa,
+                                              uint32_t sfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+__device__ __forceinline__ void mma_f8_pair(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
       "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
       : "memory");
 }
@@ -197,13 +283,15 @@ __device__ __forceinline__ uint64_t desc_sf(uint32_t saddr) {
 //  block-scaled e2m1 x e2m1: formats at bits 7 and 10 (E2M1 = 1), scale
 //  format at bit 23 (0 = e4m3, 1 = e8m0), N/8 at bit 17, M/16 at bit 24,
 //  scale-factor byte ids at bits 29 (A) and 4 (B).
-__host__ __device__ constexpr uint32_t idesc_mxf4(uint32_t n, bool e8m0, uint32_t sfa_id, uint32_t sfb_id) {
-  return (sfb_id << 4) | (1u << 7) | (1u << 10) | ((n >> 3) << 17) | ((e8m0 ? 1u : 0u) << 23) | ((128u >> 4) << 24) |
+//  m = 256 for the CTA-pair forms.
+__host__ __device__ constexpr uint32_t idesc_mxf4(uint32_t n, bool e8m0, uint32_t sfa_id, uint32_t sfb_id,
+                                                  uint32_t m = 128) {
+  return (sfb_id << 4) | (1u << 7) | (1u << 10) | ((n >> 3) << 17) | ((e8m0 ? 1u : 0u) << 23) | ((m >> 4) << 24) |
          (sfa_id << 29);
 }
 //  e4m3 x e4m3: accumulator format F32 at bit 4, formats 0 (E4M3).
-__host__ __device__ constexpr uint32_t idesc_f8(uint32_t n) {
-  return (1u << 4) | ((n >> 3) << 17) | ((128u >> 4) << 24);
+__host__ __device__ constexpr uint32_t idesc_f8(uint32_t n, uint32_t m = 128) {
+  return (1u << 4) | ((n >> 3) << 17) | ((m >> 4) << 24);
 }
 //  bf16 x bf16: accumulator F32, A and B format BF16 (1).
 __host__ __device__ constexpr uint32_t idesc_bf16(uint32_t n) {

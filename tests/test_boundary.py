@@ -86,5 +86,8 @@ def test_host_side_argument_errors(L):
     assert L.moe_set_option(2, 32) == 1 and L.moe_set_option(2, 96) == 1
     for v in (64, 128, 256, 0):
         assert L.moe_set_option(2, v) == 0
+    # CTA pairs on or off
+    assert L.moe_set_option(3, 2) == 1
+    assert L.moe_set_option(3, 0) == 0 and L.moe_set_option(3, 1) == 0
     # combine: k beyond the 1024 the kernel stages
     assert L.moe_combine(one, one, one, 1, 1025, 8, None, one, one, 1 << 20, None) == 1
