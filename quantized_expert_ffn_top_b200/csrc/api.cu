@@ -340,6 +340,7 @@ moe_status run_gemm_ffn(const uint16_t* x, int64_t T, int64_t S, const int32_t* 
   d.I = I;
   d.y = y_perm;
   d.ldy = H;
+  d.y_rows = S;
   d.status = status;
   if (mark) stage_mark(MOE_STAGE_FFN_DOWN, false, s);
   MOE_TRY(launch_grouped_gemm(d, kEpiDown, bn, w->w2, (int64_t)E * H, f.hq, f.P, sms, s));

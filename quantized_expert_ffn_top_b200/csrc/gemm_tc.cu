@@ -117,7 +117,7 @@ template <int FMT, int EPI, int BN, bool PAIR>
 __global__ void __launch_bounds__(Cfg<FMT, EPI, BN, PAIR>::kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ TokenMaps tmaps_b,
                         const __grid_constant__ CUtensorMap tmap_sfa, const __grid_constant__ CUtensorMap tmap_sfb,
-                        const GemmArgs g) {
+                        const __grid_constant__ CUtensorMap tmap_y, const GemmArgs g) {
   using C = Cfg<FMT, EPI, BN, PAIR>;
   using F = FmtTraits<FMT>;
   extern __shared__ uint8_t smem_raw[];
@@ -398,12 +398,30 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN, PAIR>::kThreads, 1)
             if (tok < te.nvalid) g.logits[(size_t)(te.p0 + tok) * g.ldy + o] = v[c] + b;
           }
         } else if (EPI == kEpiDown) {
-          const int o = mt * 128 + q * 32 + lane;
           const float sc = (FMT == MOE_FMT_MXFP4) ? 1.0f : __ldg(g.w_gs + te.e) * gact;
+          if (c0 + 16 <= te.nvalid) {
+            // a full chunk: stage [16 tokens][32 outputs] as bf16 in this
+            // warp's 1 KB and write it with one tensor store
+            uint16_t* stg = reinterpret_cast<uint16_t*>(epi_tiles) + ew * 512;
+            if (lane == 0) tc::bulk_wait_read();   // the previous store has read the buffer
+            __syncwarp();
 #pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const int tok = c0 + c;
-            if (tok < te.nvalid) g.y[(size_t)(te.p0 + tok) * g.ldy + o] = f32_to_bf16_rn(v[c] * sc);
+            for (int c = 0; c < 16; ++c) stg[c * 32 + lane] = f32_to_bf16_rn(v[c] * sc);
+            tc::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tc::tma_store_2d(&tmap_y, stg, mt * 128 + q * 32, te.p0 + c0);
+              tc::bulk_commit();
+            }
+          } else {
+            // the tile's last, partial chunk: the rows past nvalid belong to
+            // the next expert's slots
+            const int o = mt * 128 + q * 32 + lane;
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+              const int tok = c0 + c;
+              if (tok < te.nvalid) g.y[(size_t)(te.p0 + tok) * g.ldy + o] = f32_to_bf16_rn(v[c] * sc);
+            }
           }
         } else {
           // gate|up rows interleave (even lane gate, odd lane up): one shuffle
@@ -474,6 +492,7 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN, PAIR>::kThreads, 1)
         }
       }
     }
+    if (EPI == kEpiDown && lane == 0) tc::bulk_wait_all();   // stores done before the CTA exits
     if (EPI == kEpiUpF32 && g.h_amax) {
       hmax = warp_max(hmax);
       if (lane == 0) atomic_max_nonneg(g.h_amax, hmax);
@@ -542,6 +561,19 @@ bool make_sf_map(CUtensorMap* m, const void* base, int64_t nblocks, int box_bloc
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// y_perm rows for the down projection's tensor stores: box 32 outputs x 16 slots.
+bool make_y_map(CUtensorMap* m, void* base, int64_t rows, int64_t ld) {
+  EncodeTiled fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)ld, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
+  cuuint32_t box[2] = {32u, 16u};
+  cuuint32_t es[2] = {1u, 1u};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, base, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
 bool g_gemm_pairs = false;  // CTA pairs for 256-token tiles (MOE_OPT_GEMM_PAIR)
 
 template <int FMT, int EPI, int BN, bool PAIR>
@@ -549,10 +581,12 @@ cudaError_t launch_cfg(const GemmArgs& g, const void* a_base, int64_t a_rows, co
                        int num_sms, cudaStream_t s) {
   using C = Cfg<FMT, EPI, BN, PAIR>;
   using F = FmtTraits<FMT>;
-  CUtensorMap ma, msfa, msfb;
+  CUtensorMap ma, msfa, msfb, my;
   TokenMaps mb;
   memset(&msfa, 0, sizeof(msfa));
   memset(&msfb, 0, sizeof(msfb));
+  memset(&my, 0, sizeof(my));
+  if (EPI == kEpiDown && (g.y_rows < 1 || !make_y_map(&my, g.y, g.y_rows, g.ldy))) return cudaErrorInvalidValue;
   const int64_t rb = FMT == kFmtBF16 ? 2 * (int64_t)g.K : (FMT == MOE_FMT_FP8 ? g.K : g.K / 2);
   if (!make_map(&ma, a_base, a_rows, rb, 128)) return cudaErrorInvalidValue;
   for (int i = 0; i < 5; ++i)
@@ -594,10 +628,10 @@ cudaError_t launch_cfg(const GemmArgs& g, const void* a_base, int64_t a_rows, co
     }
     const int pairs = max_pairs[dev] < num_sms / 2 ? max_pairs[dev] : num_sms / 2;
     cfg.gridDim = dim3((unsigned)(2 * pairs));
-    e = cudaLaunchKernelEx(&cfg, kern, ma, mb, msfa, msfb, g);
+    e = cudaLaunchKernelEx(&cfg, kern, ma, mb, msfa, msfb, my, g);
     if (e != cudaSuccess) return e;
   } else {
-    kern<<<num_sms, C::kThreads, C::kSmem, s>>>(ma, mb, msfa, msfb, g);
+    kern<<<num_sms, C::kThreads, C::kSmem, s>>>(ma, mb, msfa, msfb, my, g);
   }
   count_launches(1);
   return cudaGetLastError();

@@ -34,8 +34,9 @@ struct GemmArgs {
   const float* h_scale;        //                 static h scale (NVFP4)
   float* h32;                  // up (fp32): h [padded rows][I]
   float* h_amax;               //            amax of h
-  uint16_t* y;                 // down: y_perm [S][ldy] bf16
+  uint16_t* y;                 // down: y_perm [y_rows][ldy] bf16
   int ldy;
+  int64_t y_rows;
   float* logits;               // router: logits [T][ldy] fp32 (+ bias)
   const float* bias;
   int32_t* status;
