@@ -96,12 +96,25 @@ __device__ __forceinline__ float fp8_tensor_scale(float amax) {
 
 // NVFP4 block: scale code sc = e4m3(bmax / (6 g)) and the element multiplier
 // r = 1 / (dec(sc) g); r = 0 marks an all-zero block.
-__device__ __forceinline__ void nvfp4_block_scale(float bmax, float g, uint32_t& sc, float& r) {
-  const float six_g = __fmul_rn(6.0f, g);
-  const float s = __fdiv_rn(bmax, six_g);
-  sc = e4m3_encode(s);
+__device__ __forceinline__ uint32_t nvfp4_scale_code(float bmax, float g) {
+  return e4m3_encode(__fdiv_rn(bmax, __fmul_rn(6.0f, g)));
+}
+__device__ __forceinline__ float nvfp4_multiplier(uint32_t sc, float g) {
   const float dec = e4m3_decode(sc);
-  r = dec != 0.0f ? __frcp_rn(__fmul_rn(dec, g)) : 0.0f;
+  return dec != 0.0f ? __frcp_rn(__fmul_rn(dec, g)) : 0.0f;
+}
+__device__ __forceinline__ void nvfp4_block_scale(float bmax, float g, uint32_t& sc, float& r) {
+  sc = nvfp4_scale_code(bmax, g);
+  r = nvfp4_multiplier(sc, g);
+}
+
+// SiLU(x) = x / (1 + e^-x) = (x/2)(1 + tanh(x/2)), with the hardware tanh
+// approximation (relative error about 2^-11, far below one e2m1 step).
+__device__ __forceinline__ float silu_fast(float x) {
+  const float hx = 0.5f * x;
+  float t;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(hx));
+  return fmaf(hx, t, hx);
 }
 
 // MXFP4 block (OCP MX v1.0 conversion): c = clamp(floor(log2 bmax) - 2 + 127,

@@ -66,7 +66,14 @@ struct Cfg {
   static constexpr int kSFA = F::kGroups * 512;
   static constexpr int kSFB = F::kGroups * 512 * kSfbBlocks;
   static constexpr int kStage = ((kA + kB + kSFA + kSFB) + 1023) / 1024 * 1024;
-  static constexpr int kStages = (200 * 1024) / kStage < 8 ? (200 * 1024) / kStage : 8;
+  // epilogue shared memory: one [32 tokens][36] fp32 tile per warp pair (SwiGLU
+  // transpose; 1 KB of it per warp stages the down projection's stores) and
+  // the NVFP4 h multiplier table
+  static constexpr int kEpiTile = 32 * 36 * 4;
+  static constexpr int kEpiBytes = (4 * (BN / 64) / 2) * kEpiTile + 512;
+  static constexpr int kStages = (220 * 1024 - kEpiBytes - 2048) / kStage < 8
+                                     ? (220 * 1024 - kEpiBytes - 2048) / kStage
+                                     : 8;
   static constexpr int kAccStages = BN == 256 ? 1 : (BN >= 128 ? 2 : 4);
   // 64 accumulator columns per epilogue warp: BN / 64 warps per
   // tensor-memory lane quarter
@@ -77,9 +84,8 @@ struct Cfg {
   static constexpr uint32_t kSfaCol = kAccStages * BN;
   static constexpr uint32_t kSfbCol = kSfaCol + F::kGroups * 4;
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr int kEpiTile = 16 * 32 * 4;  // per warp pair: 16 tokens x 32 rows, fp32
-  static constexpr int kSmem = kStages * kStage + 1024 /*align*/ + 1024 /*barriers etc.*/ +
-                               (kEpiWarps / 2) * kEpiTile;
+  static constexpr int kSmem = kStages * kStage + 1024 /*align*/ + 1024 /*barriers etc.*/ + kEpiBytes;
+  static_assert(kSmem <= 227 * 1024, "shared memory");
   static_assert(kSfbCol + F::kGroups * 4 * kSfbBlocks <= kTmemCols, "tensor memory overflow");
   // barriers (full, empty, tfull, tempty), the tensor-memory address and the
   // abort flag share the 1 KB control block
@@ -129,7 +135,8 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN, PAIR>::kThreads, 1)
   uint64_t* tempty = tfull + C::kAccStages;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + C::kAccStages);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* epi_tiles = reinterpret_cast<float*>(ctrl + 1024);  // [kEpiWarps / 2][16 tokens][32]
+  float* epi_tiles = reinterpret_cast<float*>(ctrl + 1024);  // [kEpiWarps / 2][32 tokens][36]
+  float* r_tab = epi_tiles + (C::kEpiWarps / 2) * (C::kEpiTile / 4);  // NVFP4 h: multiplier per scale code
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -342,6 +349,11 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN, PAIR>::kThreads, 1)
     const int cw = ew / 4;                       // which 64-column slice of the tile
     const float gact = act_scale_of(FMT, g.act_scale, g.act_amax);
     const float g2 = (EPI == kEpiUpQuant && FMT == MOE_FMT_NVFP4) ? act_scale_of(FMT, g.h_scale, nullptr) : 1.0f;
+    if constexpr (EPI == kEpiUpQuant && FMT == MOE_FMT_NVFP4) {
+      // r = 1 / (dec(sc) g) for every non-negative e4m3 code (0 for a zero scale)
+      for (int c = ew * 32 + lane; c < 128; c += C::kEpiWarps * 32) r_tab[c] = nvfp4_multiplier((uint32_t)c, g2);
+      asm volatile("bar.sync 15, %0;" ::"r"(C::kEpiWarps * 32) : "memory");
+    }
     float hmax = 0.0f;
     int acc = 0;
     uint32_t acc_phase = 0;
@@ -425,67 +437,78 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN, PAIR>::kThreads, 1)
           }
         } else {
           // gate|up rows interleave (even lane gate, odd lane up): one shuffle
-          // pairs them, SwiGLU runs on every lane, and the h values go through
-          // a shared-memory tile so that each lane then owns 8 consecutive
-          // features of one token (half a NVFP4 block, a quarter of an MXFP4
-          // block) for the block maximum, the codes and wide stores.
+          // pairs them and SwiGLU runs on every lane.  Two chunks (32 tokens)
+          // pass through the warp pair's shared-memory tile so that each of
+          // the pair's 64 threads then owns 16 consecutive features of one
+          // token -- one NVFP4 block, half an MXFP4 block -- for the block
+          // maximum, the scale, the codes and 8-byte stores.
+          if (ch & 1) continue;  // taken together with the even chunk
           const int part = lane & 1;
           const float sc = (FMT == MOE_FMT_MXFP4) ? 1.0f : __ldg(g.w_gs + te.e * 2 + part) * gact;
-          const int pp = q & 1;                                  // position in the warp pair
-          float* tile = epi_tiles + (ew >> 1) * (16 * 32);       // [16 tokens][32 features] of the pair
-          const int fl = lane >> 1;                              // feature within the warp's 16
-          const int f_pair = mt * 64 + (q >> 1) * 32;            // first feature of the pair
+          const int pp = q & 1;                                       // position in the warp pair
+          float* tile = epi_tiles + (ew >> 1) * (C::kEpiTile / 4);    // [32 tokens][36] of the pair
+          const int fl = lane >> 1;                                   // feature within the warp's 16
+          const int f_pair = mt * 64 + (q >> 1) * 32;                 // first feature of the pair
           const int bar = 1 + (ew >> 1);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float a = v[2 * i] * sc, b = v[2 * i + 1] * sc;
-            const float recv = __shfl_xor_sync(0xffffffffu, part ? a : b, 1);
-            const float gg = part ? recv : a;
-            const float uu = part ? b : recv;
-            const float h = __fdividef(gg, 1.0f + __expf(-gg)) * uu;
-            tile[(2 * i + part) * 32 + pp * 16 + fl] = h;
+          for (int hf = 0; hf < 2; ++hf) {
+            if (hf == 1 && ch + 1 >= nch) break;  // tokens past the tile: their rows are never stored
+            const uint32_t* rh = hf == 0 ? rr : (ch == 0 ? r1 : r3);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float a = __uint_as_float(rh[2 * i]) * sc, b = __uint_as_float(rh[2 * i + 1]) * sc;
+              const float recv = __shfl_xor_sync(0xffffffffu, part ? a : b, 1);
+              const float gg = part ? recv : a;
+              const float uu = part ? b : recv;
+              tile[(hf * 16 + 2 * i + part) * 36 + pp * 16 + fl] = silu_fast(gg) * uu;
+            }
           }
           asm volatile("bar.sync %0, 64;" ::"r"(bar) : "memory");
-          // each of the pair's 64 threads: token tl, features [8 * qq, 8 * qq + 8)
           const int tid = pp * 32 + lane;
-          const int tl = tid >> 2, qq = tid & 3;
-          const float4 lo = *reinterpret_cast<const float4*>(tile + tl * 32 + 8 * qq);
-          const float4 hi = *reinterpret_cast<const float4*>(tile + tl * 32 + 8 * qq + 4);
-          float hv[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+          const int tl = tid >> 1, hh = tid & 1;
+          const float4* src = reinterpret_cast<const float4*>(tile + tl * 36 + 16 * hh);
+          float hv[16];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float4 f = src[j];
+            hv[4 * j] = f.x;
+            hv[4 * j + 1] = f.y;
+            hv[4 * j + 2] = f.z;
+            hv[4 * j + 3] = f.w;
+          }
           const int tok = c0 + tl;
           const bool valid = tok < te.nvalid;
           const size_t row = (size_t)(te.row0 + tok);
+          const int f0 = f_pair + 16 * hh;  // this thread's 16 features
           if (EPI == kEpiUpF32) {
             if (valid) {
-              float4* dst = reinterpret_cast<float4*>(g.h32 + row * g.I + f_pair + 8 * qq);
-              dst[0] = lo;
-              dst[1] = hi;
+              float4* dst = reinterpret_cast<float4*>(g.h32 + row * g.I + f0);
 #pragma unroll
-              for (int j = 0; j < 8; ++j) hmax = fmaxf(hmax, fabsf(hv[j]));
+              for (int j = 0; j < 4; ++j) dst[j] = src[j];
+#pragma unroll
+              for (int j = 0; j < 16; ++j) hmax = fmaxf(hmax, fabsf(hv[j]));
             }
           } else {
             float bmax = 0.0f;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) bmax = fmaxf(bmax, fabsf(hv[j]));
-            uint32_t word = 0, scode = 0;
+            for (int j = 0; j < 16; ++j) bmax = fmaxf(bmax, fabsf(hv[j]));
+            uint2 codes;
+            uint32_t scode;
             if (FMT == MOE_FMT_NVFP4) {
-              bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 1));   // 16-feature block
-              float r;
-              nvfp4_block_scale(bmax, g2, scode, r);
-              word = r != 0.0f ? e2m1_encode8(hv, r) : 0u;
+              scode = nvfp4_scale_code(bmax, g2);
+              codes = nvfp4_encode16(hv, r_tab[scode]);
             } else {
-              bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 1));   // 32-feature block
-              bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 2));
+              bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 1));  // the 32-feature block
               float inv;
               mxfp4_block_scale(bmax, scode, inv);
-              word = e2m1_encode8(hv, inv);
+              codes = make_uint2(e2m1_encode8(hv, inv), e2m1_encode8(hv + 8, inv));
             }
             if (valid) {
-              *reinterpret_cast<uint32_t*>(g.hq + row * (g.I / 2) + f_pair / 2 + 4 * qq) = word;
-              if (FMT == MOE_FMT_NVFP4 && (qq & 1) == 0)
-                g.hsf[sf_blocked_offset((int64_t)row, (f_pair + 8 * qq) / 16, g.I / 16)] = (uint8_t)scode;
-              if (FMT == MOE_FMT_MXFP4 && qq == 0)
-                g.hsf[sf_blocked_offset((int64_t)row, f_pair / 32, g.I / 32)] = (uint8_t)scode;
+              *reinterpret_cast<uint2*>(g.hq + row * (g.I / 2) + f0 / 2) = codes;
+              if (FMT == MOE_FMT_NVFP4)
+                g.hsf[sf_blocked_offset((int64_t)row, f0 / 16, g.I / 16)] = (uint8_t)scode;
+              if (FMT == MOE_FMT_MXFP4 && hh == 0)
+                g.hsf[sf_blocked_offset((int64_t)row, f0 / 32, g.I / 32)] = (uint8_t)scode;
             }
           }
           asm volatile("bar.sync %0, 64;" ::"r"(bar) : "memory");
