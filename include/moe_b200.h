@@ -181,9 +181,10 @@ moe_status moe_route_logits(const float* logits, int64_t T, int32_t E, int32_t k
  *   inv_perm[i]   position of slot i                                    [S]
  * Positions within one expert follow the flat slot index (stable).  The
  * expert segments are the "slot pool" rows the atomicmilkshake fork README
- * ("Known limits") indexes per expert.  All pointers device.  Built without
- * global atomics: per-chunk counts, a scan, then a rank pass.  An index
- * outside [0, E) sets the device status word (the slot is dropped). */
+ * ("Known limits") indexes per expert.  All pointers device.  Counts and
+ * positions need no atomic updates (per-chunk counts, a scan, then a rank
+ * pass), so the result is deterministic.  An index outside [0, E) sets the
+ * device status word (the slot is dropped). */
 moe_status moe_permute(const int32_t* topk_idx, int64_t T, int32_t k, int32_t E, int32_t* offsets,
                        int32_t* perm_token, int32_t* inv_perm, void* ws, size_t ws_bytes, moe_stream_t stream);
 

@@ -99,20 +99,23 @@ moe_status check_weights(const moe_weights* w, bool need_prepared) {
 }
 
 // ---------------------------------------------------------------- layouts --
-// Router scratch: logits (when the caller passes none) and the token tiles
-// of the tensor-core router GEMM.
+// Partial logits of the tensor-core router GEMM split along H: at most as
+// many as 256 SMs can take (the split used at run time is never larger).
+int router_parts_max(int64_t T, int E) {
+  const int64_t items = (T + kRouterBN - 1) / kRouterBN * (E >= 128 ? E / 128 : 1);
+  int64_t ks = items > 0 ? 256 / items : 1;
+  return (int)(ks < 1 ? 1 : (ks > kRouterMaxSplit ? kRouterMaxSplit : ks));
+}
+
+// Router scratch: the (partial) logits.
 struct RouteWs {
   Scalars head;
-  float* logits;
-  TileEntry* tiles;
-  int32_t* ntiles;
+  float* parts;  // [nparts][T][E]
 };
-RouteWs carve_route(Carver& c, int64_t T, int E, bool need_logits) {
+RouteWs carve_route(Carver& c, int64_t T, int E) {
   RouteWs r;
   r.head = carve_head(c);
-  r.logits = c.take<float>(need_logits ? (size_t)T * E : 0);
-  r.tiles = c.take<TileEntry>((size_t)(T / 128 + 1));
-  r.ntiles = c.take<int32_t>(1);
+  r.parts = c.take<float>((size_t)T * E * router_parts_max(T, E));
   return r;
 }
 
@@ -125,6 +128,7 @@ PermWs carve_perm(Carver& c, int64_t S, int E) {
   p.head = carve_head(c);
   p.scratch.nchunks = (int)((S + permute_chunk_slots() - 1) / permute_chunk_slots());
   p.scratch.chunk_counts = c.take<int32_t>((size_t)(p.scratch.nchunks > 0 ? p.scratch.nchunks : 1) * E);
+  p.scratch.ticket = c.take<int32_t>(1);
   return p;
 }
 
@@ -168,8 +172,6 @@ FfnScratch carve_ffn(Carver& c, int64_t S, const moe_weights* w) {
 struct ForwardWs {
   Scalars head;
   float* logits;
-  TileEntry* rtiles;
-  int32_t* rntiles;
   int32_t* idx;
   float* w;
   int32_t* offsets;
@@ -188,9 +190,7 @@ ForwardWs carve_forward(Carver& c, int64_t T, int k, const moe_weights* routed, 
   const int E = routed->E;
   const int64_t S = T * k;
   f.head = carve_head(c);
-  f.logits = c.take<float>((size_t)T * E);
-  f.rtiles = c.take<TileEntry>((size_t)(T / 128 + 1));
-  f.rntiles = c.take<int32_t>(1);
+  f.logits = c.take<float>((size_t)T * E * router_parts_max(T, E));
   f.idx = c.take<int32_t>((size_t)S);
   f.w = c.take<float>((size_t)S);
   f.offsets = c.take<int32_t>((size_t)E + 1);
@@ -198,6 +198,7 @@ ForwardWs carve_forward(Carver& c, int64_t T, int k, const moe_weights* routed, 
   f.inv = c.take<int32_t>((size_t)S);
   f.pscratch.nchunks = (int)((S + permute_chunk_slots() - 1) / permute_chunk_slots());
   f.pscratch.chunk_counts = c.take<int32_t>((size_t)(f.pscratch.nchunks > 0 ? f.pscratch.nchunks : 1) * E);
+  f.pscratch.ticket = c.take<int32_t>(1);
   f.y_perm = c.take<uint16_t>((size_t)S * routed->H);
   f.ffn = carve_ffn(c, S, routed);
   if (shared) {
@@ -223,13 +224,21 @@ __global__ void identity_routing_kernel(int64_t T, int32_t* offsets, int32_t* pe
   }
 }
 
-// Router logits: tcgen05 bf16 GEMM when the shapes allow it and the batch is
-// large enough to matter, CUDA cores otherwise.
+// Router logits into `parts`: *nparts partial sums T*E apart that the top-k
+// kernel adds.  tcgen05 bf16 GEMM (split along H to fill the SMs) when the
+// shapes allow it and the batch is large enough to matter, CUDA cores
+// otherwise.
 cudaError_t run_router(const uint16_t* x, int64_t T, int H, const uint16_t* wr, const float* bias, int E,
-                       float* logits, TileEntry* tiles, int32_t* ntiles, int32_t* status, cudaStream_t s) {
-  if (T >= 128 && E % 128 == 0 && H % 64 == 0 && tensor_maps_available())
-    return launch_router_gemm(x, T, H, wr, bias, E, logits, tiles, ntiles, status, num_sms(), s);
-  return launch_router_logits(x, T, H, wr, bias, E, logits, s);
+                       float* parts, int* nparts, int32_t* status, cudaStream_t s) {
+  if (T >= 128 && E % 128 == 0 && H % 64 == 0 && tensor_maps_available()) {
+    int ks = router_ksplit(T, E, H, num_sms());
+    const int cap = router_parts_max(T, E);
+    ks = ks > cap ? cap : ks;
+    *nparts = ks;
+    return launch_router_gemm(x, T, H, wr, bias, E, parts, T * (int64_t)E, ks, status, num_sms(), s);
+  }
+  *nparts = 1;
+  return launch_router_logits(x, T, H, wr, bias, E, parts, s);
 }
 
 bool gemm_shapes_ok(const moe_weights* w, int act) {
@@ -258,12 +267,14 @@ int gemm_tile_n(int64_t S, int E) {
 }
 
 moe_status run_gemm_ffn(const uint16_t* x, int64_t T, int64_t S, const int32_t* perm, const int32_t* offsets,
-                        const int32_t* inv, int k, const moe_weights* w, uint16_t* y_perm, const FfnScratch& f,
-                        float* x_amax, float* h_amax, int32_t* status, cudaStream_t s, bool mark) {
+                        const int32_t* inv, int k, const int32_t* slot_expert, const moe_weights* w,
+                        uint16_t* y_perm, const FfnScratch& f,
+                        float* x_amax, float* h_amax, int32_t* status, cudaStream_t s, bool mark, bool planned) {
   const int E = w->E, H = w->H, I = w->I, fmt = w->fmt;
   const int sms = num_sms();
   const int bn = gemm_tile_n(S, E);
-  MOE_TRY(launch_plan(offsets, E, S, bn, f.poff, f.tiles, f.ntiles, (int)max_tiles(S, E), status, s));
+  if (!planned)
+    MOE_TRY(launch_plan(offsets, E, S, bn, f.poff, f.tiles, f.ntiles, (int)max_tiles(S, E), status, s));
   if (mark) stage_mark(MOE_STAGE_ACT_QUANT, false, s);
   QuantPaddedArgs qa;
   qa.E = E;
@@ -276,6 +287,7 @@ moe_status run_gemm_ffn(const uint16_t* x, int64_t T, int64_t S, const int32_t* 
   qa.perm_token = perm;
   qa.inv_perm = inv;
   qa.k = k;
+  qa.slot_expert = slot_expert;
   qa.x = x;
   qa.h32 = nullptr;
   qa.scale = w->a13_gs;
@@ -355,11 +367,13 @@ moe_status run_gemm_ffn(const uint16_t* x, int64_t T, int64_t S, const int32_t* 
 moe_status run_grouped_ffn(const uint16_t* x, int64_t T, int64_t S, const int32_t* perm, const int32_t* offsets,
                            const moe_weights* w, int act, uint16_t* y_perm, const FfnScratch& scratch,
                            float* x_amax, float* h_amax, int32_t* status, cudaStream_t s,
-                           bool shared_stage = false, const int32_t* inv = nullptr, int k = 0) {
+                           bool shared_stage = false, const int32_t* inv = nullptr, int k = 0,
+                           const int32_t* slot_expert = nullptr, bool planned = false) {
   if (S == 0) return MOE_OK;
   const bool mark = !shared_stage;
   if (use_gemm_path(w, S, act))
-    return run_gemm_ffn(x, T, S, perm, offsets, inv, k, w, y_perm, scratch, x_amax, h_amax, status, s, mark);
+    return run_gemm_ffn(x, T, S, perm, offsets, inv, k, slot_expert, w, y_perm, scratch, x_amax, h_amax, status, s,
+                        mark, planned);
   if (g_ffn_path == 2) return MOE_ERR_UNSUPPORTED;
   GemvArgs a;
   a.fmt = w->fmt;
@@ -388,8 +402,9 @@ moe_status run_grouped_ffn(const uint16_t* x, int64_t T, int64_t S, const int32_
   a.num_tiles = scratch.ntiles;
   a.status = status;
   const int sms = num_sms();
-  MOE_TRY(launch_plan(offsets, w->E, S, kGemvTokens, scratch.poff, scratch.tiles, scratch.ntiles,
-                      (int)max_tiles(S, w->E), status, s));
+  if (!planned)
+    MOE_TRY(launch_plan(offsets, w->E, S, kGemvTokens, scratch.poff, scratch.tiles, scratch.ntiles,
+                        (int)max_tiles(S, w->E), status, s));
   if (mark) stage_mark(MOE_STAGE_FFN_UP, false, s);
   MOE_TRY(launch_gemv_up(a, sms, s));
   if (mark) stage_mark(MOE_STAGE_FFN_UP, true, s);
@@ -545,13 +560,14 @@ moe_status moe_route(const uint16_t* x, int64_t T, int32_t H, const uint16_t* wr
   if (T > 0 && (!x || !wr || !topk_idx || !topk_w)) return MOE_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(wr)) return MOE_ERR_INVALID_ARG;
   Carver c(ws);
-  RouteWs r = carve_route(c, T, E, logits == nullptr);
+  RouteWs r = carve_route(c, T, E);
   if (!ws || ws_bytes < c.off) return MOE_ERR_WORKSPACE;
   if (T == 0) return MOE_OK;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  float* L = logits ? logits : r.logits;
-  MOE_TRY(run_router(x, T, H, wr, bias, E, L, r.tiles, r.ntiles, r.head.status, s));
-  return cuda_status(launch_topk(L, T, E, k, topk_idx, topk_w, r.head.status, s));
+  int nparts = 1;
+  MOE_TRY(run_router(x, T, H, wr, bias, E, r.parts, &nparts, r.head.status, s));
+  return cuda_status(
+      launch_topk(r.parts, nparts, T * (int64_t)E, logits, T, E, k, topk_idx, topk_w, r.head.status, s));
 }
 
 moe_status moe_route_logits(const float* logits, int64_t T, int32_t E, int32_t k, int32_t* topk_idx, float* topk_w,
@@ -561,7 +577,7 @@ moe_status moe_route_logits(const float* logits, int64_t T, int32_t E, int32_t k
   Carver c(ws);
   Scalars head = carve_head(c);
   if (!ws || ws_bytes < c.off) return MOE_ERR_WORKSPACE;
-  return cuda_status(launch_topk(logits, T, E, k, topk_idx, topk_w, head.status,
+  return cuda_status(launch_topk(logits, 1, 0, nullptr, T, E, k, topk_idx, topk_w, head.status,
                                  reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -573,7 +589,7 @@ moe_status moe_permute(const int32_t* topk_idx, int64_t T, int32_t k, int32_t E,
   PermWs p = carve_perm(c, T * k, E);
   if (!ws || ws_bytes < c.off) return MOE_ERR_WORKSPACE;
   return cuda_status(launch_permute(topk_idx, T * k, k, E, offsets, perm_token, inv_perm, p.scratch, p.head.status,
-                                    reinterpret_cast<cudaStream_t>(stream)));
+                                    reinterpret_cast<cudaStream_t>(stream), nullptr, nullptr));
 }
 
 moe_status moe_grouped_ffn(const uint16_t* x, int64_t T, int32_t k, const int32_t* perm_token, const int32_t* offsets,
@@ -635,12 +651,21 @@ moe_status moe_forward(const uint16_t* x, int64_t T, const uint16_t* wr, const f
   const int64_t S = T * k;
   // 1. router
   stage_mark(MOE_STAGE_ROUTE, false, s);
-  MOE_TRY(run_router(x, T, H, wr, bias, E, f.logits, f.rtiles, f.rntiles, f.head.status, s));
-  MOE_TRY(launch_topk(f.logits, T, E, k, f.idx, f.w, f.head.status, s));
+  int nparts = 1;
+  MOE_TRY(run_router(x, T, H, wr, bias, E, f.logits, &nparts, f.head.status, s));
+  MOE_TRY(launch_topk(f.logits, nparts, T * (int64_t)E, nullptr, T, E, k, f.idx, f.w, f.head.status, s));
   stage_mark(MOE_STAGE_ROUTE, true, s);
   // 2. histogram + permutation
   stage_mark(MOE_STAGE_PERMUTE, false, s);
-  MOE_TRY(launch_permute(f.idx, S, k, E, f.offsets, f.perm, f.inv, f.pscratch, f.head.status, s));
+  // the permutation also writes the routed FFN's tile plan when it runs in one block
+  PlanOut plan;
+  plan.bn = use_gemm_path(routed, S, act) ? gemm_tile_n(S, E) : kGemvTokens;
+  plan.poff = f.ffn.poff;
+  plan.tiles = f.ffn.tiles;
+  plan.ntiles = f.ffn.ntiles;
+  plan.max_tiles = (int)max_tiles(S, E);
+  bool planned = false;
+  MOE_TRY(launch_permute(f.idx, S, k, E, f.offsets, f.perm, f.inv, f.pscratch, f.head.status, s, &plan, &planned));
   stage_mark(MOE_STAGE_PERMUTE, true, s);
   // 3. dynamic activation scale of x (shared by routed and shared experts)
   if (dynamic_x_scale(routed, act)) {
@@ -650,7 +675,7 @@ moe_status moe_forward(const uint16_t* x, int64_t T, const uint16_t* wr, const f
   }
   // 4. routed experts
   st = run_grouped_ffn(x, T, S, f.perm, f.offsets, routed, act, f.y_perm, f.ffn, f.head.x_amax, f.head.h_amax,
-                       f.head.status, s, false, f.inv, k);
+                       f.head.status, s, false, f.inv, k, f.idx, planned);
   if (st != MOE_OK) return st;
   // 5. shared expert: every token, identity order; it reads routed's x scale
   if (shared) {

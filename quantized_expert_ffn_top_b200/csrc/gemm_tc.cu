@@ -176,7 +176,25 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN, PAIR>::kThreads, 1)
   const uint32_t rank = PAIR ? tc::cluster_rank() : 0u;
   // tiles: (token tile, weight-row block of 128 rows, or 256 for a pair)
   const int MT = g.R / (PAIR ? 256 : 128);
-  const int ntiles = __ldg(g.num_tiles) * MT;
+  // The router GEMM may split K over ksplit CTAs per tile (partial logits
+  // that the top-k kernel adds); work item t -> tile t / ksplit, split t % ksplit.
+  const int ksplit = EPI == kEpiLogits ? g.ksplit : 1;
+  // dense_rows > 0: the token tiles are the plain row blocks [i*BN, i*BN + BN)
+  // of dense_rows rows (no tile list)
+  auto tile_at = [&](int i) -> TileEntry {
+    TileEntry te;
+    if (g.dense_rows > 0) {
+      te.e = 0;
+      te.row0 = i * BN;
+      te.nvalid = (int)min((int64_t)BN, g.dense_rows - (int64_t)i * BN);
+      te.p0 = i * BN;
+    } else {
+      te = g.tiles[i];
+    }
+    return te;
+  };
+  const int ntok = g.dense_rows > 0 ? (int)((g.dense_rows + BN - 1) / BN) : __ldg(g.num_tiles);
+  const int ntiles = ntok * MT * ksplit;
   const int t_first = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
   const int t_step = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
   const int nkb = g.K / F::kBK;
@@ -191,10 +209,12 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN, PAIR>::kThreads, 1)
     int stage = 0;
     uint32_t phase = 0;
     for (int t = t_first; t < ntiles && !*abort; t += t_step) {
-      const TileEntry te = g.tiles[t / MT];
-      const int mt = PAIR ? (t % MT) * 2 + (int)rank : t % MT;   // this CTA's 128-row weight block
+      const int tt = t / ksplit, split = t % ksplit;
+      const int kb0 = split * nkb / ksplit, kb1 = (split + 1) * nkb / ksplit;
+      const TileEntry te = tile_at(tt / MT);
+      const int mt = PAIR ? (tt % MT) * 2 + (int)rank : tt % MT;   // this CTA's 128-row weight block
       const uint8_t* sfa = F::kBs ? g.w_sf + (size_t)te.e * g.R * ncols_w + (size_t)mt * (ncols_w / 4) * 512 : nullptr;
-      for (int kb = 0; kb < nkb; ++kb) {
+      for (int kb = kb0; kb < kb1; ++kb) {
         if (!tc::mbar_wait(&empty[stage], phase ^ 1u, abort)) {
           if (lane == 0) raise_status(g.status, MOE_ERR_TIMEOUT);
           *abort = 1;
@@ -254,7 +274,9 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN, PAIR>::kThreads, 1)
     uint32_t acc_phase = 0;
     // a pair's MMAs are issued by its leader (rank 0) alone
     for (int t = t_first; (!PAIR || rank == 0) && t < ntiles && !*abort; t += t_step) {
-      const TileEntry te = g.tiles[t / MT];
+      const int tt = t / ksplit, split = t % ksplit;
+      const int kb0 = split * nkb / ksplit, kb1 = (split + 1) * nkb / ksplit;
+      const TileEntry te = tile_at(tt / MT);
       if (!tc::mbar_wait(&tempty[acc], acc_phase ^ 1u, abort)) {
         if (lane == 0) raise_status(g.status, MOE_ERR_TIMEOUT);
         *abort = 1;
@@ -269,7 +291,7 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN, PAIR>::kThreads, 1)
       uint32_t idesc_nv = tc::idesc_mxf4(n_mma, false, 0, 0, kM), idesc_f8 = tc::idesc_f8(n_mma, kM),
                idesc_bf = tc::idesc_bf16(n_mma);
       bool ok = true;
-      for (int kb = 0; kb < nkb; ++kb) {
+      for (int kb = kb0; kb < kb1; ++kb) {
         if (!tc::mbar_wait(&full[stage], phase, abort)) {
           if (lane == 0) raise_status(g.status, MOE_ERR_TIMEOUT);
           *abort = 1;
@@ -302,7 +324,7 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN, PAIR>::kThreads, 1)
           for (int kk = 0; kk < F::kSteps; ++kk) {
             const uint64_t da = da0 + (uint64_t)(kk * 2);  // +32 bytes per MMA along K
             const uint64_t db = db0 + (uint64_t)(kk * 2);
-            const uint32_t accum = (kb > 0 || kk > 0) ? 1u : 0u;
+            const uint32_t accum = (kb > kb0 || kk > 0) ? 1u : 0u;
             if (FMT == MOE_FMT_NVFP4) {
               const uint32_t sa_t = tmem + C::kSfaCol + 4 * kk, sb_t = sfb0 + kk * 4 * C::kSfbBlocks;
               if constexpr (PAIR) tc::mma_nvf4_pair(d, da, db, idesc_nv, sa_t, sb_t, accum);
@@ -364,8 +386,9 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN, PAIR>::kThreads, 1)
         break;
       }
       tc::fence_after_sync();
-      const TileEntry te = g.tiles[t / MT];
-      const int mt = PAIR ? (t % MT) * 2 + (int)rank : t % MT;   // this CTA's 128 weight rows
+      const int tt = t / ksplit, split = t % ksplit;
+      const TileEntry te = tile_at(tt / MT);
+      const int mt = PAIR ? (tt % MT) * 2 + (int)rank : tt % MT;   // this CTA's 128 weight rows
       const int ncol = min(BN, (te.nvalid + 15) & ~15);
       const int c_lo = cw * 64;
       const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN) + (uint32_t)c_lo;
@@ -403,11 +426,12 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN, PAIR>::kThreads, 1)
         const int c0 = c_lo + ch * 16;
         if (EPI == kEpiLogits) {
           const int o = mt * 128 + q * 32 + lane;  // expert
-          const float b = g.bias ? __ldg(g.bias + o) : 0.0f;
+          const float b = (g.bias && split == 0) ? __ldg(g.bias + o) : 0.0f;   // the bias joins split 0
+          float* out = g.logits + (size_t)split * g.split_stride;
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
             const int tok = c0 + c;
-            if (tok < te.nvalid) g.logits[(size_t)(te.p0 + tok) * g.ldy + o] = v[c] + b;
+            if (tok < te.nvalid) out[(size_t)(te.p0 + tok) * g.ldy + o] = v[c] + b;
           }
         } else if (EPI == kEpiDown) {
           const float sc = (FMT == MOE_FMT_MXFP4) ? 1.0f : __ldg(g.w_gs + te.e) * gact;
@@ -696,46 +720,34 @@ bool tensor_maps_available() { return encode_fn() != nullptr; }
 
 void set_gemm_pairs(bool on) { g_gemm_pairs = on; }
 
-__global__ void dense_plan_kernel(int64_t T, int bn, TileEntry* __restrict__ tiles, int32_t* __restrict__ num_tiles) {
-  const int n = (int)((T + bn - 1) / bn);
-  for (int j = blockIdx.x * blockDim.x + threadIdx.x; j < n; j += gridDim.x * blockDim.x) {
-    TileEntry te;
-    te.e = 0;
-    te.row0 = j * bn;
-    te.nvalid = (int)min((int64_t)bn, T - (int64_t)j * bn);
-    te.p0 = j * bn;
-    tiles[j] = te;
-  }
-  if (blockIdx.x == 0 && threadIdx.x == 0) *num_tiles = n;
-}
 
-cudaError_t launch_dense_plan(int64_t T, int bn, TileEntry* tiles, int32_t* num_tiles, cudaStream_t s) {
-  dense_plan_kernel<<<1, 256, 0, s>>>(T, bn, tiles, num_tiles);
-  count_launches(1);
-  return cudaGetLastError();
+int router_ksplit(int64_t T, int E, int H, int num_sms) {
+  const int64_t items = (T + kRouterBN - 1) / kRouterBN * (E / 128);
+  int ks = items > 0 ? (int)(num_sms / items) : 1;
+  ks = ks < 1 ? 1 : (ks > kRouterMaxSplit ? kRouterMaxSplit : ks);
+  while (ks > 1 && (H / 64) / ks < 4) --ks;  // at least four 64-wide K blocks per split
+  return ks;
 }
 
 cudaError_t launch_router_gemm(const uint16_t* x, int64_t T, int H, const uint16_t* wr, const float* bias, int E,
-                               float* logits, TileEntry* tiles, int32_t* num_tiles, int32_t* status, int num_sms,
+                               float* logits_parts, int64_t part_stride, int ksplit, int32_t* status, int num_sms,
                                cudaStream_t s) {
-  constexpr int kBN = 128;
-  cudaError_t e = launch_dense_plan(T, kBN, tiles, num_tiles, s);
-  if (e != cudaSuccess) return e;
   GemmArgs g;
   memset(&g, 0, sizeof(g));
   g.fmt = kFmtBF16;
   g.E = 1;
   g.K = H;
   g.R = E;
-  g.tiles = tiles;
-  g.num_tiles = num_tiles;
-  g.logits = logits;
+  g.dense_rows = T;
+  g.logits = logits_parts;
   g.bias = bias;
+  g.ksplit = ksplit;
+  g.split_stride = part_stride;
   g.ldy = E;
   g.status = status;
-  const int64_t ntiles = (T + kBN - 1) / kBN * (E / 128);
-  const int grid = (int)(ntiles < num_sms ? ntiles : num_sms);
-  return launch_cfg<kFmtBF16, kEpiLogits, kBN, false>(g, wr, E, x, T, grid, s);
+  const int64_t items = (T + kRouterBN - 1) / kRouterBN * (E / 128) * ksplit;
+  const int grid = (int)(items < num_sms ? items : num_sms);
+  return launch_cfg<kFmtBF16, kEpiLogits, kRouterBN, false>(g, wr, E, x, T, grid, s);
 }
 
 // ---------------------------------------------------------------- planning --
@@ -899,39 +911,74 @@ __global__ void __launch_bounds__(256) quant_tokens_kernel(QuantPaddedArgs a) {
   constexpr int bs = FMT == MOE_FMT_MXFP4 ? 32 : 16;
   constexpr int kPer = 64;
   constexpr int kWords = FMT == MOE_FMT_FP8 ? 16 : 8;  // 32-bit code words per lane
+  constexpr int kLaneBytes = kWords * 4;
+  constexpr int kVec = kLaneBytes / 16;
+  __shared__ uint4 tbuf[8][32 * kVec];  // per warp: the stretch's codes, for the reorder
   const int nb = a.K / bs;
   const int lane = threadIdx.x & 31;
   const float scale = act_scale_of(FMT, a.scale, a.amax);
   const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  // NVFP4: the multiplier r = 1 / (dec(sc) g) of every non-negative scale code
+  __shared__ float r_tab[128];
+  if (FMT == MOE_FMT_NVFP4) {
+    for (int i = threadIdx.x; i < 128; i += blockDim.x) r_tab[i] = nvfp4_multiplier((uint32_t)i, scale);
+    __syncthreads();
+  }
+  // padded row of the slot of (token t, pick j): -1 for a dropped slot, -2 if
+  // the permutation is inconsistent
+  auto resolve = [&](int64_t t, int j) -> int64_t {
+    if (j >= a.k) return -1;
+    const int32_t p = __ldg(a.inv_perm + t * a.k + j);
+    if (p >= a.S) return -2;
+    if (p < 0) return -1;
+    int e;
+    if (a.slot_expert) {
+      e = __ldg(a.slot_expert + t * a.k + j);
+      if (e < 0 || e >= a.E) return -2;
+    } else {
+      e = segment_of(a.offsets, a.E, p);
+    }
+    const int32_t o = __ldg(a.offsets + e), o1 = __ldg(a.offsets + e + 1);
+    const int64_t row = (int64_t)__ldg(a.poff + e) + (p - o);
+    return (row >= 0 && row < a.P && p >= o && p < o1) ? row : -2;
+  };
   for (int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < a.T; t += warps) {
+    const int64_t row_first = resolve(t, lane);  // issued before the x loads
     for (int c0 = 0; c0 < a.K; c0 += 32 * kPer) {
       const int c = c0 + lane * kPer;
       const bool active = c < a.K;
       uint32_t w[kWords];
       uint32_t sfw = 0;
       if (active) {
-        float v[kPer];
-        const uint16_t* src = a.x + t * a.K + c;
+        // the lane's 64 bf16 values stay packed (32 registers); each scale
+        // block is unpacked when it is quantised
+        uint32_t raw[kPer / 2];
+        const uint4* src = reinterpret_cast<const uint4*>(a.x + t * a.K + c);
 #pragma unroll
-        for (int i = 0; i < kPer; i += 8) {
-          const uint4 u = __ldg(reinterpret_cast<const uint4*>(src + i));
-          const uint32_t uu[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            v[i + 2 * j] = __uint_as_float(uu[j] << 16);
-            v[i + 2 * j + 1] = __uint_as_float(uu[j] & 0xFFFF0000u);
-          }
+        for (int i = 0; i < kPer / 8; ++i) {
+          const uint4 u = __ldg(src + i);
+          raw[4 * i] = u.x;
+          raw[4 * i + 1] = u.y;
+          raw[4 * i + 2] = u.z;
+          raw[4 * i + 3] = u.w;
         }
+        auto unpack = [&](float* v, int first, int n) {
+#pragma unroll
+          for (int i = 0; i < n / 2; ++i) {
+            v[2 * i] = __uint_as_float(raw[first / 2 + i] << 16);
+            v[2 * i + 1] = __uint_as_float(raw[first / 2 + i] & 0xFFFF0000u);
+          }
+        };
         if constexpr (FMT == MOE_FMT_NVFP4) {
 #pragma unroll
           for (int b = 0; b < 4; ++b) {
+            float v[16];
+            unpack(v, 16 * b, 16);
             float bmax = 0.0f;
 #pragma unroll
-            for (int i = 0; i < 16; ++i) bmax = fmaxf(bmax, fabsf(v[16 * b + i]));
-            uint32_t sc;
-            float r;
-            nvfp4_block_scale(bmax, scale, sc, r);
-            const uint2 cw = nvfp4_encode16(v + 16 * b, r);
+            for (int i = 0; i < 16; ++i) bmax = fmaxf(bmax, fabsf(v[i]));
+            const uint32_t sc = nvfp4_scale_code(bmax, scale);
+            const uint2 cw = nvfp4_encode16(v, r_tab[sc]);
             w[2 * b] = cw.x;
             w[2 * b + 1] = cw.y;
             sfw |= sc << (8 * b);
@@ -939,38 +986,48 @@ __global__ void __launch_bounds__(256) quant_tokens_kernel(QuantPaddedArgs a) {
         } else if constexpr (FMT == MOE_FMT_MXFP4) {
 #pragma unroll
           for (int b = 0; b < 2; ++b) {
+            float v[32];
+            unpack(v, 32 * b, 32);
             float bmax = 0.0f;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) bmax = fmaxf(bmax, fabsf(v[32 * b + i]));
+            for (int i = 0; i < 32; ++i) bmax = fmaxf(bmax, fabsf(v[i]));
             uint32_t sc;
             float inv;
             mxfp4_block_scale(bmax, sc, inv);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) w[4 * b + q] = e2m1_encode8(v + 32 * b + 8 * q, inv);
+            for (int q = 0; q < 4; ++q) w[4 * b + q] = e2m1_encode8(v + 8 * q, inv);
             sfw |= sc << (8 * b);
           }
         } else {
           const float inv = __frcp_rn(scale);
 #pragma unroll
-          for (int i = 0; i < kWords; ++i)
-            w[i] = e4m3x2_encode(__fmul_rn(v[4 * i], inv), __fmul_rn(v[4 * i + 1], inv)) |
-                   (e4m3x2_encode(__fmul_rn(v[4 * i + 2], inv), __fmul_rn(v[4 * i + 3], inv)) << 16);
-        }
-      }
-      for (int j0 = 0; j0 < a.k; j0 += 32) {
-        // lane j resolves the padded row of slot j0 + j (-1: dropped slot, -2: bad)
-        int64_t myrow = -1;
-        if (j0 + lane < a.k) {
-          const int32_t p = __ldg(a.inv_perm + t * a.k + j0 + lane);
-          if (p >= a.S) {
-            myrow = -2;
-          } else if (p >= 0) {
-            const int e = segment_of(a.offsets, a.E, p);
-            const int32_t o = __ldg(a.offsets + e);
-            const int64_t row = (int64_t)__ldg(a.poff + e) + (p - o);
-            myrow = (row >= 0 && row < a.P && p >= o) ? row : -2;
+          for (int i = 0; i < kWords; ++i) {
+            float v[4];
+            unpack(v, 4 * i, 4);
+            w[i] = e4m3x2_encode(__fmul_rn(v[0], inv), __fmul_rn(v[1], inv)) |
+                   (e4m3x2_encode(__fmul_rn(v[2], inv), __fmul_rn(v[3], inv)) << 16);
           }
         }
+      }
+      // Codes in store order: lane l's 16-byte pieces v are bytes 512 v + 16 l
+      // of the stretch, so every store instruction covers 512 contiguous bytes.
+      uint4* tb = tbuf[threadIdx.x >> 5];
+      if (active) {
+#pragma unroll
+        for (int v = 0; v < kVec; ++v) tb[lane * kVec + v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+      }
+      __syncwarp();
+      const int seg = min(a.K - c0, 32 * kPer) * kLaneBytes / kPer;  // code bytes in this stretch
+      uint4 wc[kVec];
+#pragma unroll
+      for (int v = 0; v < kVec; ++v) {
+        const int off = 512 * v + 16 * lane;
+        wc[v] = off < seg ? tb[off / 16] : make_uint4(0, 0, 0, 0);
+      }
+      __syncwarp();
+      for (int j0 = 0; j0 < a.k; j0 += 32) {
+        // lane j resolves the padded row of slot j0 + j (-1: dropped slot, -2: bad)
+        const int64_t myrow = (j0 == 0) ? row_first : resolve(t, j0 + lane);
         const int nj = min(32, a.k - j0);
         for (int jj = 0; jj < nj; ++jj) {
           const int64_t row = __shfl_sync(0xffffffffu, myrow, jj);
@@ -978,20 +1035,16 @@ __global__ void __launch_bounds__(256) quant_tokens_kernel(QuantPaddedArgs a) {
             if (row == -2 && lane == 0 && c0 == 0) raise_status(a.status, MOE_ERR_DEVICE_FAULT);
             continue;
           }
-          if (!active) continue;
-          if constexpr (FMT == MOE_FMT_FP8) {
-            uint4* dst = reinterpret_cast<uint4*>(a.codes + row * a.K + c);
+          uint4* dst = reinterpret_cast<uint4*>(a.codes + row * ((int64_t)a.K * kLaneBytes / kPer) +
+                                                (int64_t)c0 * kLaneBytes / kPer);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) dst[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
-          } else {
-            uint4* dst = reinterpret_cast<uint4*>(a.codes + row * (a.K / 2) + c / 2);
-            dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-            dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-            if constexpr (FMT == MOE_FMT_NVFP4)
-              *reinterpret_cast<uint32_t*>(a.sf + sf_blocked_offset(row, c / bs, nb)) = sfw;
-            else
-              *reinterpret_cast<uint16_t*>(a.sf + sf_blocked_offset(row, c / bs, nb)) = (uint16_t)sfw;
-          }
+          for (int v = 0; v < kVec; ++v)
+            if (512 * v + 16 * lane < seg) dst[(512 * v) / 16 + lane] = wc[v];
+          if (!active) continue;
+          if constexpr (FMT == MOE_FMT_NVFP4)
+            *reinterpret_cast<uint32_t*>(a.sf + sf_blocked_offset(row, c / bs, nb)) = sfw;
+          else if constexpr (FMT == MOE_FMT_MXFP4)
+            *reinterpret_cast<uint16_t*>(a.sf + sf_blocked_offset(row, c / bs, nb)) = (uint16_t)sfw;
         }
       }
     }

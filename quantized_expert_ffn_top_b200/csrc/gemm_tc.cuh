@@ -39,6 +39,9 @@ struct GemmArgs {
   int64_t y_rows;
   float* logits;               // router: logits [T][ldy] fp32 (+ bias)
   const float* bias;
+  int ksplit;                  // router: K split over this many partial outputs,
+  int64_t split_stride;        //         split s at logits + s * split_stride
+  int64_t dense_rows;          // > 0: token tiles are plain row blocks (no tile list)
   int32_t* status;
 };
 
@@ -51,6 +54,7 @@ struct QuantPaddedArgs {
   const int32_t* perm_token;   // x source: token of each slot
   const int32_t* inv_perm;     // x source, optional: slot of each (token, j); then each
   int k;                       //   token is quantised once and written to its k slots
+  const int32_t* slot_expert;  //   optional with it: expert of each (token, j) (top-k indices)
   const uint16_t* x;           // [T][K] bf16
   const float* h32;            // or fp32 rows at padded positions
   const float* scale;          // static tensor scale or NULL
@@ -68,10 +72,13 @@ cudaError_t launch_grouped_gemm(const GemmArgs& g, int epi, int bn, const void* 
 bool tensor_maps_available();
 // CTA pairs (cta_group::2) for 256-token tiles whose weight rows divide by 256.
 void set_gemm_pairs(bool on);
-cudaError_t launch_dense_plan(int64_t T, int bn, TileEntry* tiles, int32_t* num_tiles, cudaStream_t s);
-// Router logits on the tensor cores: logits[T][E] = x Wr^T (+ bias); E % 128 == 0, H % 64 == 0.
+// Router logits on the tensor cores, K split over ksplit partial outputs
+// (logits_parts + s * part_stride, the bias in part 0; the top-k kernel adds
+// them): E % 128 == 0, H % 64 == 0.  64-token tiles.
+constexpr int kRouterBN = 64;
+constexpr int kRouterMaxSplit = 4;
+int router_ksplit(int64_t T, int E, int H, int num_sms);
 cudaError_t launch_router_gemm(const uint16_t* x, int64_t T, int H, const uint16_t* wr, const float* bias, int E,
-                               float* logits, TileEntry* tiles, int32_t* num_tiles, int32_t* status, int num_sms,
+                               float* logits_parts, int64_t part_stride, int ksplit, int32_t* status, int num_sms,
                                cudaStream_t s);
-
 }  // namespace moe

@@ -31,17 +31,31 @@ cudaError_t launch_quantize(int fmt, const void* x, int x_dtype, int64_t rows, i
 // route.cu
 cudaError_t launch_router_logits(const uint16_t* x, int64_t T, int H, const uint16_t* wr, const float* bias, int E,
                                  float* logits, cudaStream_t s);
-cudaError_t launch_topk(const float* logits, int64_t T, int E, int k, int32_t* idx, float* w, int32_t* status,
-                        cudaStream_t s);
+// logits: nparts partial sums part_stride apart (1 = plain logits); logits_out
+// (nullable) receives their sum.
+cudaError_t launch_topk(const float* logits, int nparts, int64_t part_stride, float* logits_out, int64_t T, int E,
+                        int k, int32_t* idx, float* w, int32_t* status, cudaStream_t s);
 
 // permute.cu
 struct PermuteScratch {
   int32_t* chunk_counts;   // [nchunks][E]
+  int32_t* ticket;         // one int: blocks done counting
   int nchunks;
 };
 int permute_chunk_slots();
+// Tile plan the permutation may write on the way (bn = 0: none).
+struct PlanOut {
+  int bn;
+  int32_t* poff;                  // [E+1] padded offsets
+  struct TileEntry* tiles;        // [max_tiles]
+  int32_t* ntiles;
+  int max_tiles;
+};
+// *planned (nullable) tells whether `plan` was written; if not, the caller
+// runs the plan kernel itself.
 cudaError_t launch_permute(const int32_t* idx, int64_t S, int k, int E, int32_t* offsets, int32_t* perm_token,
-                           int32_t* inv_perm, PermuteScratch scratch, int32_t* status, cudaStream_t s);
+                           int32_t* inv_perm, PermuteScratch scratch, int32_t* status, cudaStream_t s,
+                           const PlanOut* plan, bool* planned);
 
 // gemv.cu -- small-batch expert FFN (one pass over each active expert).
 struct GemvArgs {

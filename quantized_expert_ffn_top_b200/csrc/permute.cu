@@ -1,5 +1,6 @@
 // Token-to-expert histogram, offsets and stable permutation of the T*k slots,
-// without global atomics.
+// with no atomic updates of the counts or positions (the result is
+// deterministic).
 //
 // The permuted order is the expert-major "slot pool" of the
 // atomicmilkshake/FreeToken fork README ("Known limits"): every expert's slots
@@ -7,16 +8,22 @@
 // for a dense block of rows.  Slots keep their flat order i = t*k + j inside a
 // segment (stable), which makes the permutation unique and bit-comparable.
 //
-// Three passes over chunks of kChunk slots (8 warps x 256):
+// Passes over chunks of kChunk slots (8 warps x 256):
 //   1. per chunk and expert, the count (warp-private counters fed by
 //      __match_any_sync, one writer lane per expert and step);
-//   2. one block: per expert the exclusive prefix over chunks, the totals, and
-//      the exclusive prefix over experts -> offsets;
+//   2. per expert the exclusive prefix over chunks, the totals and the
+//      exclusive prefix over experts -> offsets (and, on request, the grouped
+//      FFN's tile plan) -- run by the last block of pass 1 to finish, found
+//      with one atomic ticket;
 //   3. per chunk again: each warp's base = chunk base + earlier warps'
 //      counts, and each slot's rank among equal experts earlier in its warp
 //      step -> perm_token[p] = t, inv_perm[i] = p.
+// Small batches run all three inside one block.
+#include <string.h>
+
 #include <mutex>
 
+#include "gemm_tc.cuh"
 #include "kernels.cuh"
 
 namespace moe {
@@ -53,10 +60,42 @@ __device__ __forceinline__ void warp_counts(const int32_t* idx, int64_t S, int64
   }
 }
 
+// Exclusive scan of v over the block's kPermWarps warps (256 threads);
+// *total receives the sum.  Every thread calls it.
+__device__ __forceinline__ int32_t scan256_excl(int32_t v, int32_t* warp_tot, int32_t* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int32_t incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int32_t n = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += n;
+  }
+  __syncthreads();
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  int32_t base = 0, sum = 0;
+#pragma unroll
+  for (int w = 0; w < kPermWarps; ++w) {
+    base += w < warp ? warp_tot[w] : 0;
+    sum += warp_tot[w];
+  }
+  *total = sum;
+  return incl - v + base;
+}
+
+// Pass 1: per chunk and expert, the count.  The last block to finish (a
+// ticket taken after a memory fence) then runs pass 2 -- per expert the
+// exclusive prefix over chunks plus the expert's offset, turning the counts
+// into each chunk's base positions -- and writes the offsets and, when asked,
+// the tile plan.  The ticket is zero on entry and is reset by that block.
 __global__ void __launch_bounds__(kPermWarps * 32) perm_count_kernel(const int32_t* __restrict__ idx, int64_t S,
                                                                      int E, int32_t* __restrict__ chunk_counts,
+                                                                     int32_t* __restrict__ ticket,
+                                                                     int32_t* __restrict__ offsets, PlanOut plan,
                                                                      int32_t* status) {
-  extern __shared__ int32_t cnt[];  // [kPermWarps][E]
+  extern __shared__ int32_t cnt[];  // [kPermWarps][E]; the last block reuses it as [E] totals
+  __shared__ int32_t warp_tot[kPermWarps];
+  __shared__ int is_last;
   for (int i = threadIdx.x; i < kPermWarps * E; i += blockDim.x) cnt[i] = 0;
   __syncthreads();
   const int64_t base = (int64_t)blockIdx.x * kChunk;
@@ -68,50 +107,76 @@ __global__ void __launch_bounds__(kPermWarps * 32) perm_count_kernel(const int32
     for (int w = 0; w < kPermWarps; ++w) s += cnt[w * E + e];
     chunk_counts[(int64_t)blockIdx.x * E + e] = s;
   }
-}
-
-// One block of 1024 threads.  Turns chunk_counts[c][e] into the absolute base
-// position of chunk c's first slot of expert e, and writes offsets[0..E].
-__global__ void __launch_bounds__(1024) perm_scan_kernel(int32_t* __restrict__ chunk_counts, int nchunks, int E,
-                                                         int32_t* __restrict__ offsets) {
-  __shared__ int32_t tot[1024];
-  __shared__ int32_t warp_tot[32];
-  const int e = threadIdx.x;
-  int32_t run = 0;
-  if (e < E) {
-    for (int c = 0; c < nchunks; ++c) {
-      const int32_t v = chunk_counts[(int64_t)c * E + e];
-      chunk_counts[(int64_t)c * E + e] = run;
-      run += v;
-    }
-  }
-  // exclusive scan of the totals over experts
-  const int lane = e & 31, warp = e >> 5;
-  int32_t incl = run;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) is_last = atomicAdd(ticket, 1) == (int)gridDim.x - 1;
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  const int nchunks = gridDim.x;
+  int32_t* tot = cnt;  // [E] counts, then offsets
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int32_t run = 0;
+    for (int c0 = 0; c0 < nchunks; c0 += 8) {  // eight loads in flight, then the running sum
+      int32_t v[8];
 #pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int32_t n = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += n;
-  }
-  if (lane == 31) warp_tot[warp] = incl;
-  __syncthreads();
-  if (warp == 0) {
-    int32_t v = warp_tot[lane];
-    int32_t vi = v;
+      for (int u = 0; u < 8; ++u) v[u] = c0 + u < nchunks ? __ldcg(chunk_counts + (int64_t)(c0 + u) * E + e) : 0;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int32_t n = __shfl_up_sync(0xffffffffu, vi, o);
-      if (lane >= o) vi += n;
+      for (int u = 0; u < 8; ++u) {
+        if (c0 + u < nchunks) chunk_counts[(int64_t)(c0 + u) * E + e] = run;
+        run += v[u];
+      }
     }
-    warp_tot[lane] = vi - v;
+    tot[e] = run;
   }
   __syncthreads();
-  const int32_t excl = incl - run + warp_tot[warp];
-  tot[e] = excl;
-  if (e < E) offsets[e] = excl;
-  if (e == E - 1) offsets[E] = excl + run;
+  // scans over experts: each thread owns a contiguous group of `per` experts
+  const int per = (E + (int)blockDim.x - 1) / (int)blockDim.x;
+  const int e0 = threadIdx.x * per;
+  int32_t mine = 0, pad_mine = 0, til_mine = 0;
+  for (int e = e0; e < e0 + per && e < E; ++e) {
+    mine += tot[e];
+    pad_mine += (tot[e] + 127) / 128 * 128;
+    if (plan.bn > 0) til_mine += (tot[e] + plan.bn - 1) / plan.bn;
+  }
+  int32_t total, pad_total = 0, til_total = 0;
+  int32_t off = scan256_excl(mine, warp_tot, &total);
+  int32_t pbase = 0, tbase = 0;
+  if (plan.bn > 0) {
+    pbase = scan256_excl(pad_mine, warp_tot, &pad_total);
+    tbase = scan256_excl(til_mine, warp_tot, &til_total);
+  }
   __syncthreads();
-  if (e < E)
+  for (int e = e0; e < e0 + per && e < E; ++e) {
+    const int32_t n = tot[e];
+    offsets[e] = off;
+    if (plan.bn > 0) {
+      plan.poff[e] = pbase;
+      const int til = (n + plan.bn - 1) / plan.bn;
+      for (int j = 0; j < til && tbase + j < plan.max_tiles; ++j) {
+        TileEntry te;
+        te.e = e;
+        te.row0 = pbase + j * plan.bn;
+        te.nvalid = min(plan.bn, n - j * plan.bn);
+        te.p0 = off + j * plan.bn;
+        plan.tiles[tbase + j] = te;
+      }
+      pbase += (n + 127) / 128 * 128;
+      tbase += til;
+    }
+    tot[e] = off;  // the expert's offset, for the chunk bases below
+    off += n;
+  }
+  if (threadIdx.x == 0) {
+    offsets[E] = total;
+    if (plan.bn > 0) {
+      plan.poff[E] = pad_total;
+      *plan.ntiles = min(til_total, plan.max_tiles);
+    }
+    *ticket = 0;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x)
     for (int c = 0; c < nchunks; ++c) chunk_counts[(int64_t)c * E + e] += tot[e];
 }
 
@@ -158,54 +223,25 @@ __global__ void __launch_bounds__(kPermWarps * 32) perm_scatter_kernel(const int
   }
 }
 
-// Small batches (decode): the same three passes inside one block of 32
-// warps, each warp owning a contiguous range of ceil(S/32) slots; the
-// per-warp expert counters live in shared memory.  One launch instead of three.
-constexpr int kSmallWarps = 32;
-constexpr int64_t kSmallMaxS = 8192;
+// Up to kBlockMaxS slots: the same passes inside one block of 32 warps,
+// each warp owning a contiguous range of slots, the per-warp expert counters
+// in shared memory -- one launch instead of three.  The block can also write
+// the grouped FFN's tile plan (padded offsets and tile list), which needs the
+// same per-expert counts.
+constexpr int kBlockWarps = 32;
+constexpr int64_t kBlockMaxS = 8192;   // beyond, one SM's scattered stores are the bottleneck
 
-__global__ void __launch_bounds__(kSmallWarps * 32) perm_small_kernel(const int32_t* __restrict__ idx, int64_t S,
-                                                                     int k, int E, int32_t* __restrict__ offsets,
-                                                                     int32_t* __restrict__ perm_token,
-                                                                     int32_t* __restrict__ inv_perm,
-                                                                     int32_t* status) {
-  extern __shared__ int32_t cnt[];  // [kSmallWarps][E], then [E] totals
-  int32_t* tot = cnt + kSmallWarps * E;
-  __shared__ int32_t warp_tot[32];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t per = ((S + kSmallWarps - 1) / kSmallWarps + 31) / 32 * 32;  // slots per warp, multiple of 32
-  for (int i = threadIdx.x; i < kSmallWarps * E; i += blockDim.x) cnt[i] = 0;
-  __syncthreads();
-  int32_t* my = cnt + warp * E;
-  const int64_t lo = warp * per, hi = min(S, lo + per);
-  for (int64_t base = lo; base < hi; base += 32) {
-    const int64_t i = base + lane;
-    const int e = (i < hi) ? slot_expert(idx, S, i, E, status) : -1;
-    const unsigned peers = __match_any_sync(0xffffffffu, e);
-    if (e >= 0 && lane == __ffs(peers) - 1) my[e] += __popc(peers);
-    __syncwarp();
-  }
-  __syncthreads();
-  // per expert: exclusive prefix over warps, total
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    int32_t run = 0;
-    for (int w = 0; w < kSmallWarps; ++w) {
-      const int32_t v = cnt[w * E + e];
-      cnt[w * E + e] = run;
-      run += v;
-    }
-    tot[e] = run;
-  }
-  __syncthreads();
-  // exclusive scan of the totals over experts (E <= 1024 = blockDim)
-  const int e = threadIdx.x;
-  const int32_t v = e < E ? tot[e] : 0;
+// Exclusive scan of one value per thread over a 1024-thread block; *total
+// receives the sum.  Every thread calls it.
+__device__ __forceinline__ int32_t block_scan_excl(int32_t v, int32_t* warp_tot, int32_t* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int32_t incl = v;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
     const int32_t n = __shfl_up_sync(0xffffffffu, incl, o);
     if (lane >= o) incl += n;
   }
+  __syncthreads();  // warp_tot free
   if (lane == 31) warp_tot[warp] = incl;
   __syncthreads();
   if (warp == 0) {
@@ -217,41 +253,138 @@ __global__ void __launch_bounds__(kSmallWarps * 32) perm_small_kernel(const int3
       if (lane >= o) wi += n;
     }
     warp_tot[lane] = wi - wv;
+    if (lane == 31) warp_tot[32] = wi;
   }
   __syncthreads();
-  const int32_t excl = incl - v + warp_tot[warp];
+  *total = warp_tot[32];
+  return incl - v + warp_tot[warp];
+}
+
+// The experts of a warp's next 4 x 32 slots, loaded together.
+__device__ __forceinline__ void load4(const int32_t* idx, int64_t S, int64_t base, int64_t hi, int E, int32_t* status,
+                                      int (&e)[4]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int64_t i = base + u * 32 + lane;
+    e[u] = (i < hi) ? slot_expert(idx, S, i, E, status) : -1;
+  }
+}
+
+__global__ void __launch_bounds__(kBlockWarps * 32) perm_block_kernel(const int32_t* __restrict__ idx, int64_t S,
+                                                                     int k, int E, int32_t* __restrict__ offsets,
+                                                                     int32_t* __restrict__ perm_token,
+                                                                     int32_t* __restrict__ inv_perm,
+                                                                     int32_t* status, PlanOut plan) {
+  extern __shared__ int32_t cnt[];  // [kBlockWarps][E], then [E] offsets
+  int32_t* tot = cnt + kBlockWarps * E;
+  __shared__ int32_t warp_tot[33];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t per = ((S + kBlockWarps - 1) / kBlockWarps + 127) / 128 * 128;  // slots per warp
+  for (int i = threadIdx.x; i < kBlockWarps * E; i += blockDim.x) cnt[i] = 0;
   __syncthreads();
+  int32_t* my = cnt + warp * E;
+  const int64_t lo = warp * per, hi = min(S, lo + per);
+  for (int64_t base = lo; base < hi; base += 128) {
+    int ev[4];
+    load4(idx, S, base, hi, E, status, ev);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const unsigned peers = __match_any_sync(0xffffffffu, ev[u]);
+      if (ev[u] >= 0 && lane == __ffs(peers) - 1) my[ev[u]] += __popc(peers);
+      __syncwarp();
+    }
+  }
+  __syncthreads();
+  // per expert: exclusive prefix over warps, total
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int32_t run = 0;
+    for (int w = 0; w < kBlockWarps; ++w) {
+      const int32_t v = cnt[w * E + e];
+      cnt[w * E + e] = run;
+      run += v;
+    }
+    tot[e] = run;
+  }
+  __syncthreads();
+  // exclusive scan of the totals over experts (E <= 1024 = blockDim)
+  const int e = threadIdx.x;
+  const int32_t n_e = e < E ? tot[e] : 0;
+  int32_t total;
+  const int32_t excl = block_scan_excl(n_e, warp_tot, &total);
   if (e < E) {
     tot[e] = excl;
     offsets[e] = excl;
   }
-  if (e == E - 1) offsets[E] = excl + v;
-  __syncthreads();
-  for (int i = threadIdx.x; i < kSmallWarps * E; i += blockDim.x) cnt[i] += tot[i % E];
-  __syncthreads();
-  for (int64_t base = lo; base < hi; base += 32) {
-    const int64_t i = base + lane;
-    const int ee = (i < hi) ? slot_expert(idx, S, i, E, nullptr) : -1;
-    const unsigned peers = __match_any_sync(0xffffffffu, ee);
-    if (ee >= 0) {
-      const int32_t p = my[ee] + __popc(peers & ((1u << lane) - 1u));
-      perm_token[p] = (int32_t)(i / k);
-      inv_perm[i] = p;
-    } else if (i < hi) {
-      inv_perm[i] = -1;
+  if (e == 0) offsets[E] = total;
+  if (plan.bn > 0) {
+    // padded offsets (segments start on multiples of 128 rows) and the tiles
+    const int32_t pad = (n_e + 127) / 128 * 128;
+    const int32_t til = (n_e + plan.bn - 1) / plan.bn;
+    int32_t pad_total, til_total;
+    const int32_t pbase = block_scan_excl(pad, warp_tot, &pad_total);
+    const int32_t tbase = block_scan_excl(til, warp_tot, &til_total);
+    if (e < E) {
+      plan.poff[e] = pbase;
+      for (int j = 0; j < til && tbase + j < plan.max_tiles; ++j) {
+        TileEntry te;
+        te.e = e;
+        te.row0 = pbase + j * plan.bn;
+        te.nvalid = min(plan.bn, n_e - j * plan.bn);
+        te.p0 = excl + j * plan.bn;
+        plan.tiles[tbase + j] = te;
+      }
     }
-    __syncwarp();
-    if (ee >= 0 && lane == __ffs(peers) - 1) my[ee] += __popc(peers);
-    __syncwarp();
+    if (e == 0) {
+      plan.poff[E] = pad_total;
+      *plan.ntiles = min(til_total, plan.max_tiles);
+    }
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < kBlockWarps * E; i += blockDim.x) cnt[i] += tot[i % E];
+  __syncthreads();
+  for (int64_t base = lo; base < hi; base += 128) {
+    int ev[4];
+    load4(idx, S, base, hi, E, nullptr, ev);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int64_t i = base + u * 32 + lane;
+      const int ee = ev[u];
+      const unsigned peers = __match_any_sync(0xffffffffu, ee);
+      if (ee >= 0) {
+        const int32_t p = my[ee] + __popc(peers & ((1u << lane) - 1u));
+        perm_token[p] = (int32_t)(i / k);
+        inv_perm[i] = p;
+      } else if (i < hi) {
+        inv_perm[i] = -1;
+      }
+      __syncwarp();
+      if (ee >= 0 && lane == __ffs(peers) - 1) my[ee] += __popc(peers);
+      __syncwarp();
+    }
   }
 }
 
 cudaError_t launch_permute(const int32_t* idx, int64_t S, int k, int E, int32_t* offsets, int32_t* perm_token,
-                           int32_t* inv_perm, PermuteScratch scratch, int32_t* status, cudaStream_t s) {
-  const size_t small_smem = sizeof(int32_t) * (size_t)(kSmallWarps + 1) * E;
-  if (S > 0 && S <= kSmallMaxS && small_smem <= 48 * 1024) {
-    perm_small_kernel<<<1, kSmallWarps * 32, small_smem, s>>>(idx, S, k, E, offsets, perm_token, inv_perm, status);
+                           int32_t* inv_perm, PermuteScratch scratch, int32_t* status, cudaStream_t s,
+                           const PlanOut* plan, bool* planned) {
+  if (planned) *planned = false;
+  const size_t block_smem = sizeof(int32_t) * (size_t)(kBlockWarps + 1) * E;
+  if (S > 0 && S <= kBlockMaxS) {
+    // E <= 1024 needs at most 132 KB
+    cudaError_t e = cudaFuncSetAttribute(perm_block_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)(sizeof(int32_t) * (kBlockWarps + 1) * 1024));
+    if (e != cudaSuccess) return e;
+    PlanOut p;
+    if (plan) {
+      p = *plan;
+    } else {
+      memset(&p, 0, sizeof(p));
+    }
+    perm_block_kernel<<<1, kBlockWarps * 32, block_smem, s>>>(idx, S, k, E, offsets, perm_token, inv_perm, status,
+                                                              p);
     count_launches(1);
+    if (planned && plan && plan->bn > 0) *planned = true;
     return cudaGetLastError();
   }
   const int nchunks = (int)((S + kChunk - 1) / kChunk);
@@ -260,11 +393,20 @@ cudaError_t launch_permute(const int32_t* idx, int64_t S, int k, int E, int32_t*
     return cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (E + 1), s);
   }
   const size_t smem = sizeof(int32_t) * kPermWarps * E;
-  perm_count_kernel<<<nchunks, kPermWarps * 32, smem, s>>>(idx, S, E, scratch.chunk_counts, status);
-  perm_scan_kernel<<<1, 1024, 0, s>>>(scratch.chunk_counts, nchunks, E, offsets);
+  PlanOut p;
+  if (plan) {
+    p = *plan;
+  } else {
+    memset(&p, 0, sizeof(p));
+  }
+  cudaError_t e = cudaMemsetAsync(scratch.ticket, 0, sizeof(int32_t), s);
+  if (e != cudaSuccess) return e;
+  perm_count_kernel<<<nchunks, kPermWarps * 32, smem, s>>>(idx, S, E, scratch.chunk_counts, scratch.ticket, offsets,
+                                                           p, status);
   perm_scatter_kernel<<<nchunks, kPermWarps * 32, smem, s>>>(idx, S, k, E, scratch.chunk_counts, perm_token,
                                                               inv_perm);
-  count_launches(3);
+  count_launches(2);
+  if (planned && plan && plan->bn > 0) *planned = true;
   return cudaGetLastError();
 }
 
@@ -287,13 +429,16 @@ namespace {
 
 constexpr int kFixedScratchInts = 65536;  // 256 KiB: nchunks * E <= 65536
 static __device__ __align__(256) int32_t g_fixed_perm_scratch[kFixedScratchInts];
+static __device__ int32_t g_fixed_perm_ticket;
 
 constexpr int kMaxDevices = 64;
 int32_t* g_fixed_scratch_ptr[kMaxDevices] = {nullptr};
 std::mutex g_fixed_scratch_mu;
 
-// Device address of the array on the current device, looked up once per device.
-cudaError_t fixed_scratch_ptr(int32_t** out) {
+int32_t* g_fixed_ticket_ptr[kMaxDevices] = {nullptr};
+
+// Device addresses of the arrays on the current device, looked up once per device.
+cudaError_t fixed_scratch_ptr(int32_t** out, int32_t** ticket) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -303,9 +448,14 @@ cudaError_t fixed_scratch_ptr(int32_t** out) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_fixed_perm_scratch);
     if (e != cudaSuccess) return e;
+    void* q = nullptr;
+    e = cudaGetSymbolAddress(&q, g_fixed_perm_ticket);
+    if (e != cudaSuccess) return e;
     g_fixed_scratch_ptr[dev] = static_cast<int32_t*>(p);
+    g_fixed_ticket_ptr[dev] = static_cast<int32_t*>(q);
   }
   *out = g_fixed_scratch_ptr[dev];
+  *ticket = g_fixed_ticket_ptr[dev];
   return cudaSuccess;
 }
 
@@ -322,12 +472,14 @@ extern "C" moe_status moe_permute_fixed_scratch(const int32_t* topk_idx, int64_t
   const int64_t nchunks = (S + kChunk - 1) / kChunk;
   if (nchunks * (int64_t)E > kFixedScratchInts) return MOE_ERR_WORKSPACE;  // beyond the fixed capacity
   int32_t* scratch = nullptr;
-  if (fixed_scratch_ptr(&scratch) != cudaSuccess) return MOE_ERR_CUDA;
+  int32_t* ticket = nullptr;
+  if (fixed_scratch_ptr(&scratch, &ticket) != cudaSuccess) return MOE_ERR_CUDA;
   PermuteScratch ps;
   ps.chunk_counts = scratch;
+  ps.ticket = ticket;
   ps.nchunks = (int)nchunks;
   return launch_permute(topk_idx, S, k, E, offsets, perm_token, inv_perm, ps, dev_status,
-                        reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+                        reinterpret_cast<cudaStream_t>(stream), nullptr, nullptr) == cudaSuccess
              ? MOE_OK
              : MOE_ERR_CUDA;
 }

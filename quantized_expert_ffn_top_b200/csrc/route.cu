@@ -138,8 +138,11 @@ cudaError_t launch_router_logits(const uint16_t* x, int64_t T, int H, const uint
 // warp arg-max; lane 0 writes the index and exp(L - L_0); a final pass divides
 // by the sum.  A NaN, or a row without a finite logit, raises the status word
 // and writes indices 0..k-1 with zero weights.
+// The logits may arrive as nparts partial sums (a router GEMM split along
+// H), added here in part order; logits_out (nullable) receives the sums.
 template <int J>
-__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, int64_t T, int E, int k,
+__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, int nparts, int64_t part_stride,
+                                                   float* __restrict__ logits_out, int64_t T, int E, int k,
                                                    int32_t* __restrict__ idx, float* __restrict__ w,
                                                    int32_t* status) {
   const int lane = threadIdx.x & 31;
@@ -152,7 +155,19 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
   for (int j = 0; j < J; ++j) {
     const int e = lane + 32 * j;
     v[j] = e < E ? __ldg(L + e) : -INFINITY;
+  }
+  for (int p = 1; p < nparts; ++p) {
+#pragma unroll
+    for (int j = 0; j < J; ++j) {
+      const int e = lane + 32 * j;
+      if (e < E) v[j] += __ldg(L + p * part_stride + e);
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < J; ++j) {
+    const int e = lane + 32 * j;
     if (e < E && isnan(v[j])) bad = true;
+    if (e < E && logits_out) logits_out[t * E + e] = v[j];
   }
   uint32_t taken = 0u;
 #pragma unroll
@@ -200,17 +215,19 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
   for (int r = lane; r < k; r += 32) w[t * k + r] = __fdiv_rn(w[t * k + r], sum);
 }
 
-cudaError_t launch_topk(const float* logits, int64_t T, int E, int k, int32_t* idx, float* w, int32_t* status,
-                        cudaStream_t s) {
+cudaError_t launch_topk(const float* logits, int nparts, int64_t part_stride, float* logits_out, int64_t T, int E,
+                        int k, int32_t* idx, float* w, int32_t* status, cudaStream_t s) {
   if (T == 0) return cudaSuccess;
   const unsigned grid = (unsigned)((T + 7) / 8);
   const int J = (E + 31) / 32;
-  if (J <= 1) topk_kernel<1><<<grid, 256, 0, s>>>(logits, T, E, k, idx, w, status);
-  else if (J <= 2) topk_kernel<2><<<grid, 256, 0, s>>>(logits, T, E, k, idx, w, status);
-  else if (J <= 4) topk_kernel<4><<<grid, 256, 0, s>>>(logits, T, E, k, idx, w, status);
-  else if (J <= 8) topk_kernel<8><<<grid, 256, 0, s>>>(logits, T, E, k, idx, w, status);
-  else if (J <= 16) topk_kernel<16><<<grid, 256, 0, s>>>(logits, T, E, k, idx, w, status);
-  else topk_kernel<32><<<grid, 256, 0, s>>>(logits, T, E, k, idx, w, status);
+#define MOE_TOPK(JJ) topk_kernel<JJ><<<grid, 256, 0, s>>>(logits, nparts, part_stride, logits_out, T, E, k, idx, w, status)
+  if (J <= 1) MOE_TOPK(1);
+  else if (J <= 2) MOE_TOPK(2);
+  else if (J <= 4) MOE_TOPK(4);
+  else if (J <= 8) MOE_TOPK(8);
+  else if (J <= 16) MOE_TOPK(16);
+  else MOE_TOPK(32);
+#undef MOE_TOPK
   count_launches(1);
   return cudaGetLastError();
 }
