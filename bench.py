@@ -22,6 +22,9 @@ Rank 0 prints one JSON line.  Besides the contract keys it carries:
                and the output copied back inside the timed region
   decode       the decode workload (T=4, static activation scales): step time
                and the expert-weight streaming rate of moe_grouped_ffn (GB/s)
+  configs      the FP8 W8A8 + shared-expert and the large MXFP4 workloads:
+               tokens/s (median, p10/p90), GEMM TFLOP/s against the format's
+               tensor peak, active-expert weight GB/s against HBM, routing
   cpu_baseline the CPU oracle on a bounded token sample (rank 0, N = 1)
   clocks       nvidia-smi samples taken during the timed region
 `--impl reference` times the CPU oracle instead (the only other arm).
@@ -56,6 +59,7 @@ def parse():
     ap.add_argument("--workload", default="prefill")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-configs", action="store_true", help="skip the per-config report (fp8_shared, large)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
     ap.add_argument("--profile-range", action="store_true",
                     help="bracket the timed prefill replays with cudaProfilerStart/Stop (for ncu --profile-from-start off)")
@@ -143,11 +147,22 @@ def build_layer(ops, synth, torch, w, static: bool):
     prepared = ops.moe_prepare_weights(bank)
     torch.cuda.synchronize()
     del bank
+    shared = None
+    if w.shared_I:
+        s13 = synth.cuda_normal((1, 2 * w.shared_I, w.H), w.w_std, synth.TID_SH_W13)
+        s2 = synth.cuda_normal((1, w.H, w.shared_I), w.w_std, synth.TID_SH_W2)
+        sbank = ops.quantize_bank(fmt, s13, s2, ws)
+        if static and fmt != ops.FMT_MXFP4:
+            # the shared expert reads the routed layer's x scale; its own h scale
+            sbank.a2_gs = torch.tensor([synth.static_act_scales()[1]], dtype=torch.float32, device="cuda")
+        shared = ops.moe_prepare_weights(sbank)
+        del s13, s2, sbank
+    torch.cuda.synchronize()
     torch.cuda.empty_cache()
     x = synth.cuda_normal((w.T, w.H), 1.0, synth.TID_X, dtype=torch.bfloat16)
     wr = synth.cuda_normal((w.E, w.H), w.wr_std, synth.TID_WR, dtype=torch.bfloat16)
     bias = synth.cuda_router_bias(w)
-    return prepared, x, wr, bias
+    return prepared, x, wr, bias, shared
 
 
 def algorithmic(w, bank_fmt: str, offsets: np.ndarray):
@@ -208,13 +223,13 @@ def time_forward(ops, torch, layer, w, act, steps, warmup, flush, stage=True, ho
     events around each replay); the per-stage split comes from a second graph
     that records the library's stage events.  host_io runs time the eager
     user call with the host<->device copies inside the events."""
-    prepared, x, wr, bias = layer
-    ws = ops.new_workspace(ops.workspace_size(w.T, w.k, prepared, None, act))
+    prepared, x, wr, bias, shared = layer
+    ws = ops.new_workspace(ops.workspace_size(w.T, w.k, prepared, shared, act))
     out = torch.empty_like(x)
     stream = torch.cuda.current_stream()
 
     def fwd():
-        ops.moe_forward(x, wr, bias, w.k, prepared, None, act, ws, out=out)
+        ops.moe_forward(x, wr, bias, w.k, prepared, shared, act, ws, out=out)
 
     l0 = ops.moe_kernel_launch_count()
     for _ in range(max(warmup, 1)):
@@ -285,7 +300,7 @@ def time_grouped_ffn(ops, torch, layer, w, act, steps, warmup, flush):
     """Device time of the grouped expert FFN alone (moe_grouped_ffn: tile
     plan, activation quantisation, gate|up + SwiGLU, down) on the layer's
     routed slots, one CUDA-graph replay per step, L2 flushed before each."""
-    prepared, x, wr, bias = layer
+    prepared, x, wr, bias, _ = layer
     ws = ops.new_workspace(ops.workspace_size(w.T, w.k, prepared, None, act))
     idx, _ = ops.moe_route(x, wr, bias, w.k, ws)
     off, perm, _ = ops.moe_permute(idx, w.E, ops.new_workspace(1 << 24))
@@ -313,6 +328,35 @@ def time_grouped_ffn(ops, torch, layer, w, act, steps, warmup, flush):
     if ops.moe_get_device_status(ws) != 0:
         raise RuntimeError("device status reported a fault in the grouped FFN")
     return [a.elapsed_time(b) for a, b in evs], off.cpu().numpy()
+
+
+def config_report(ops, torch, synth, name, act, steps, warmup, flush, pk):
+    """Per-config figures: tokens/s, the GEMMs' TFLOP/s against the format's
+    tensor peak, the active experts' weight GB/s against HBM, and the routing
+    histogram.  Stage times come from the library's stage events."""
+    w = synth.workload(name)
+    layer = build_layer(ops, synth, torch, w, static=(w.fmt == "nvfp4"))
+    r = time_forward(ops, torch, layer, w, act, steps, warmup, flush)
+    del layer
+    torch.cuda.empty_cache()
+    alg = algorithmic(w, w.fmt, r["offsets"])
+    st = r["stages"]
+    ms = np.array(r["ms"])
+    peak = pk["bf16_tflops"] * (FP8_PER_BF16 if w.fmt == "fp8" else FP4_PER_BF16)
+    up, down = st.get("ffn_up", 0.0), st.get("ffn_down", 0.0)
+    rep_ = {"workload": workload_name(w), "act_scales": "static" if w.fmt == "nvfp4" else "dynamic",
+            "ms_median": float(np.median(ms)), "ms_p10": float(np.percentile(ms, 10)),
+            "ms_p90": float(np.percentile(ms, 90)), "tokens_per_s": w.T / (float(np.median(ms)) * 1e-3),
+            "stages_ms": st, "routing": {"active_experts": alg["active_experts"],
+                                         "max_over_mean": alg["max_over_mean"], "zero_experts": alg["zero_experts"]}}
+    if up > 0 and down > 0:
+        tf_up = alg["flops_up"] / (up * 1e-3) / 1e12
+        tf_down = alg["flops_down"] / (down * 1e-3) / 1e12
+        gbs = (alg["wbytes_up"] + alg["wbytes_down"]) / ((up + down) * 1e-3) / 1e9
+        rep_.update({"gemm_up_tflops": tf_up, "gemm_up_frac": tf_up / peak, "gemm_down_tflops": tf_down,
+                     "gemm_down_frac": tf_down / peak, "tensor_peak_tflops": peak,
+                     "weight_gbs": gbs, "weight_hbm_frac": gbs / pk["hbm_gbs"]})
+    return rep_
 
 
 # ------------------------------------------------------------ CPU oracle ----
@@ -504,6 +548,9 @@ def main():
                               measured_traffic("ffn_up", "decode"), measured_traffic("ffn_down", "decode")),
                           "hbm_frac": gbs / pk["hbm_gbs"] if gbs else None, "stages_ms": rd["stages"]}
         del dl
+
+    if not args.no_configs:
+        line["configs"] = [config_report(ops, torch, synth, n, act, 10, 3, flush, pk) for n in ("fp8_shared", "large")]
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_oracle_sample(w, args.cpu_seconds, static=True)

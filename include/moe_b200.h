@@ -221,8 +221,12 @@ moe_status moe_combine(const uint16_t* y_perm, const int32_t* inv_perm, const fl
  * "Changes in this fork") -> combine.  x [T][H] bf16, wr [E][H] bf16,
  * bias [E] (nullable), out [T][H] bf16 (device).  routed and shared
  * (nullable, E == 1) must be PREPARED and of one format; the shared expert
- * reads the same quantised x as the routed experts.  Intermediates live in
- * `ws`. */
+ * reads the same x scale as the routed experts.  Intermediates live in `ws`.
+ * The shared expert runs on a library-owned side stream forked from `stream`
+ * after the x scale and joined before the combine (event record / wait, so a
+ * graph capture of `stream` captures both branches); it overlaps routing and
+ * the permutation.  Concurrent forwards on one device share that side stream
+ * and serialise their shared experts. */
 moe_status moe_forward(const uint16_t* x, int64_t T, const uint16_t* wr, const float* bias, int32_t k,
                        const moe_weights* routed, const moe_weights* shared, int32_t act, uint16_t* out, void* ws,
                        size_t ws_bytes, moe_stream_t stream);
@@ -246,8 +250,12 @@ moe_status moe_get_device_status(void* ws, moe_stream_t stream, int32_t* host_st
  *   MOE_OPT_GEMM_PAIR: 1 runs 256-token tiles on CTA pairs (tcgen05
  *                     cta_group::2, 256 weight rows per tile) when the weight
  *                     rows per expert divide by 256; 0 (default) keeps one
- *                     CTA per 128-row tile. */
-typedef enum { MOE_OPT_FFN_PATH = 1, MOE_OPT_GEMM_TILE_N = 2, MOE_OPT_GEMM_PAIR = 3 } moe_option;
+ *                     CTA per 128-row tile.
+ *   MOE_OPT_PDL:       1 (default) launches the layer's kernels with
+ *                     programmatic dependent launch, so each one's setup
+ *                     overlaps the previous kernel's tail; 0 launches them
+ *                     plainly. */
+typedef enum { MOE_OPT_FFN_PATH = 1, MOE_OPT_GEMM_TILE_N = 2, MOE_OPT_GEMM_PAIR = 3, MOE_OPT_PDL = 4 } moe_option;
 moe_status moe_set_option(int32_t option, int32_t value);
 
 /* moe_permute for callers that cannot allocate device memory (no workspace

@@ -216,6 +216,9 @@ ForwardWs carve_forward(Carver& c, int64_t T, int k, const moe_weights* routed, 
 
 // --------------------------------------------------------------- helpers --
 __global__ void identity_routing_kernel(int64_t T, int32_t* offsets, int32_t* perm) {
+  pdl_wait();  // inputs come from the previous kernels
+  pdl_trigger();
+
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i < T) perm[i] = (int32_t)i;
   if (i == 0) {
@@ -414,11 +417,57 @@ moe_status run_grouped_ffn(const uint16_t* x, int64_t T, int64_t S, const int32_
   return MOE_OK;
 }
 
+// A side stream per device and a fork/join pair of events per call: work
+// enqueued on `stream` after fork() depends on everything before it on the
+// caller's stream, and the caller's stream waits for it at join().  Both are
+// stream operations, so a graph capture of the caller's stream captures the
+// fork and the join.  One side stream per device: concurrent forwards on one
+// device serialise their shared experts (correctly, by their own events).
+struct SideFork {
+  cudaStream_t stream = nullptr;
+  cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
+  bool forked = false;
+  moe_status fork(cudaStream_t s) {
+    static cudaStream_t side[64];
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MOE_ERR_CUDA;
+    {
+      std::lock_guard<std::mutex> lk(mu);
+      if (!side[dev] && cudaStreamCreateWithFlags(&side[dev], cudaStreamNonBlocking) != cudaSuccess)
+        return MOE_ERR_CUDA;
+      stream = side[dev];
+    }
+    if (cudaEventCreateWithFlags(&ev_fork, cudaEventDisableTiming) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaEventCreateWithFlags(&ev_join, cudaEventDisableTiming) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaEventRecord(ev_fork, s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaStreamWaitEvent(stream, ev_fork, 0) != cudaSuccess) return MOE_ERR_CUDA;
+    forked = true;
+    return MOE_OK;
+  }
+  moe_status join(cudaStream_t s) {
+    moe_status st = MOE_OK;
+    if (forked) {
+      if (cudaEventRecord(ev_join, stream) != cudaSuccess || cudaStreamWaitEvent(s, ev_join, 0) != cudaSuccess)
+        st = MOE_ERR_CUDA;
+      forked = false;
+    }
+    return st;
+  }
+  ~SideFork() {
+    if (ev_fork) cudaEventDestroy(ev_fork);
+    if (ev_join) cudaEventDestroy(ev_join);
+  }
+};
+
 bool dynamic_x_scale(const moe_weights* w, int act) {
   return act == MOE_ACT_MATCH && w->fmt != MOE_FMT_MXFP4 && !w->a13_gs;
 }
 
 }  // namespace
+
+static int g_pdl = 1;  // MOE_OPT_PDL
+bool pdl_enabled() { return g_pdl != 0; }
 
 static uint64_t g_launches = 0;
 static std::mutex g_launch_mu;
@@ -461,6 +510,11 @@ moe_status moe_set_option(int32_t option, int32_t value) {
   if (option == MOE_OPT_GEMM_TILE_N) {
     if (value != 0 && value != 64 && value != 128 && value != 192 && value != 256) return MOE_ERR_INVALID_ARG;
     g_gemm_bn = value;
+    return MOE_OK;
+  }
+  if (option == MOE_OPT_PDL) {
+    if (value != 0 && value != 1) return MOE_ERR_INVALID_ARG;
+    g_pdl = value;
     return MOE_OK;
   }
   if (option == MOE_OPT_GEMM_PAIR) {
@@ -649,15 +703,46 @@ moe_status moe_forward(const uint16_t* x, int64_t T, const uint16_t* wr, const f
   if (T == 0) return MOE_OK;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int64_t S = T * k;
-  // 1. router
+  // 1. dynamic activation scale of x (shared by routed and shared experts)
+  if (dynamic_x_scale(routed, act)) {
+    stage_mark(MOE_STAGE_ACT_QUANT, false, s);
+    MOE_TRY(launch_amax(x, 1, T * H, f.head.x_amax, num_sms(), s));
+    stage_mark(MOE_STAGE_ACT_QUANT, true, s);
+  }
+  // 2. shared expert: every token, identity order, on a side stream forked
+  // here and joined before the combine, so it overlaps routing and the
+  // permutation; it reads the routed layer's x scale
+  SideFork side;
+  if (shared) {
+    st = side.fork(s);
+    if (st != MOE_OK) return st;
+    cudaStream_t s2 = side.stream;
+    stage_mark(MOE_STAGE_SHARED, false, s2);
+    cudaError_t le = launch_pdl(identity_routing_kernel, dim3((unsigned)((T + 255) / 256)), dim3(256), 0, s2, T,
+                                f.sh_offsets, f.sh_perm);
+    count_launches(1);
+    if (le == cudaSuccess) le = cudaGetLastError();
+    st = le != cudaSuccess ? MOE_ERR_CUDA : MOE_OK;
+    if (st == MOE_OK) {
+      moe_weights sh = *shared;
+      sh.a13_gs = routed->a13_gs;
+      st = run_grouped_ffn(x, T, T, f.sh_perm, f.sh_offsets, &sh, act, f.sh_y, f.sh_ffn, f.head.x_amax,
+                           f.head.sh_h_amax, f.head.status, s2, true);
+    }
+    stage_mark(MOE_STAGE_SHARED, true, s2);
+    if (st != MOE_OK) {
+      side.join(s);
+      return st;
+    }
+  }
+  // 3. router
   stage_mark(MOE_STAGE_ROUTE, false, s);
   int nparts = 1;
-  MOE_TRY(run_router(x, T, H, wr, bias, E, f.logits, &nparts, f.head.status, s));
-  MOE_TRY(launch_topk(f.logits, nparts, T * (int64_t)E, nullptr, T, E, k, f.idx, f.w, f.head.status, s));
+  st = cuda_status(run_router(x, T, H, wr, bias, E, f.logits, &nparts, f.head.status, s));
+  if (st == MOE_OK)
+    st = cuda_status(launch_topk(f.logits, nparts, T * (int64_t)E, nullptr, T, E, k, f.idx, f.w, f.head.status, s));
   stage_mark(MOE_STAGE_ROUTE, true, s);
-  // 2. histogram + permutation
-  stage_mark(MOE_STAGE_PERMUTE, false, s);
-  // the permutation also writes the routed FFN's tile plan when it runs in one block
+  // 4. histogram + permutation; it also writes the routed FFN's tile plan
   PlanOut plan;
   plan.bn = use_gemm_path(routed, S, act) ? gemm_tile_n(S, E) : kGemvTokens;
   plan.poff = f.ffn.poff;
@@ -665,31 +750,21 @@ moe_status moe_forward(const uint16_t* x, int64_t T, const uint16_t* wr, const f
   plan.ntiles = f.ffn.ntiles;
   plan.max_tiles = (int)max_tiles(S, E);
   bool planned = false;
-  MOE_TRY(launch_permute(f.idx, S, k, E, f.offsets, f.perm, f.inv, f.pscratch, f.head.status, s, &plan, &planned));
-  stage_mark(MOE_STAGE_PERMUTE, true, s);
-  // 3. dynamic activation scale of x (shared by routed and shared experts)
-  if (dynamic_x_scale(routed, act)) {
-    stage_mark(MOE_STAGE_ACT_QUANT, false, s);
-    MOE_TRY(launch_amax(x, 1, T * H, f.head.x_amax, num_sms(), s));
-    stage_mark(MOE_STAGE_ACT_QUANT, true, s);
+  if (st == MOE_OK) {
+    stage_mark(MOE_STAGE_PERMUTE, false, s);
+    st = cuda_status(
+        launch_permute(f.idx, S, k, E, f.offsets, f.perm, f.inv, f.pscratch, f.head.status, s, &plan, &planned));
+    stage_mark(MOE_STAGE_PERMUTE, true, s);
   }
-  // 4. routed experts
-  st = run_grouped_ffn(x, T, S, f.perm, f.offsets, routed, act, f.y_perm, f.ffn, f.head.x_amax, f.head.h_amax,
-                       f.head.status, s, false, f.inv, k, f.idx, planned);
-  if (st != MOE_OK) return st;
-  // 5. shared expert: every token, identity order; it reads routed's x scale
+  // 5. routed experts
+  if (st == MOE_OK)
+    st = run_grouped_ffn(x, T, S, f.perm, f.offsets, routed, act, f.y_perm, f.ffn, f.head.x_amax, f.head.h_amax,
+                         f.head.status, s, false, f.inv, k, f.idx, planned);
   if (shared) {
-    stage_mark(MOE_STAGE_SHARED, false, s);
-    identity_routing_kernel<<<(unsigned)((T + 255) / 256), 256, 0, s>>>(T, f.sh_offsets, f.sh_perm);
-    count_launches(1);
-    MOE_TRY(cudaGetLastError());
-    moe_weights sh = *shared;
-    sh.a13_gs = routed->a13_gs;
-    st = run_grouped_ffn(x, T, T, f.sh_perm, f.sh_offsets, &sh, act, f.sh_y, f.sh_ffn, f.head.x_amax,
-                         f.head.sh_h_amax, f.head.status, s, true);
-    if (st != MOE_OK) return st;
-    stage_mark(MOE_STAGE_SHARED, true, s);
+    const moe_status js = side.join(s);
+    if (st == MOE_OK) st = js;
   }
+  if (st != MOE_OK) return st;
   // 6. combine
   stage_mark(MOE_STAGE_COMBINE, false, s);
   st = cuda_status(launch_combine(f.y_perm, f.inv, f.w, T, k, H, f.sh_y, out, f.head.status, s));

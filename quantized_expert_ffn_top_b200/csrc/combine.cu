@@ -18,6 +18,9 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const uint16_t
                                                                   const float* __restrict__ w, int64_t T, int k,
                                                                   int H, const uint16_t* __restrict__ shared_y,
                                                                   uint16_t* __restrict__ out, int32_t* status) {
+  pdl_wait();  // inputs come from the previous kernels
+  pdl_trigger();
+
   __shared__ int32_t sp[kCombineMaxK];
   __shared__ float sw[kCombineMaxK];
   const int64_t t = blockIdx.x;
@@ -81,9 +84,10 @@ cudaError_t launch_combine(const uint16_t* y_perm, const int32_t* inv_perm, cons
   if (T == 0) return cudaSuccess;
   if (k > kCombineMaxK) return cudaErrorInvalidValue;
   const dim3 grid((unsigned)T, (unsigned)((H + kCombineCols - 1) / kCombineCols));
-  combine_kernel<<<grid, kCombineThreads, 0, s>>>(y_perm, inv_perm, w, T, k, H, shared_y, out, status);
+  cudaError_t e = launch_pdl(combine_kernel, grid, dim3(kCombineThreads), 0, s, y_perm, inv_perm, w, T, k, H, shared_y,
+                             out, status);
   count_launches(1);
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace moe

@@ -22,6 +22,16 @@ constexpr int kWarp = 32;
 
 // ----------------------------------------------------------- status word --
 // The first 4 bytes of every workspace.  0 = OK, otherwise a moe_status.
+// Programmatic dependent launch (sm_90 and later).  A kernel launched with
+// the programmatic-serialisation attribute may start while the kernel before
+// it in the stream is still running; pdl_wait() returns once that kernel (and
+// so every earlier one) has completed and its memory is visible, so it comes
+// before the first read of anything they wrote.  pdl_trigger() lets the next
+// kernel start launching.  Both are no-ops for a kernel launched without the
+// attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ void raise_status(int32_t* st, int32_t code) {
   if (st) atomicCAS(st, 0, code);
 }

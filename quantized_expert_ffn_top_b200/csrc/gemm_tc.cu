@@ -173,6 +173,9 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN, PAIR>::kThreads, 1)
   if constexpr (PAIR) tc::cluster_sync();
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
+  // the setup above overlaps the previous kernel's tail (programmatic launch)
+  pdl_wait();
+  pdl_trigger();
   const uint32_t rank = PAIR ? tc::cluster_rank() : 0u;
   // tiles: (token tile, weight-row block of 128 rows, or 256 for a pair)
   const int MT = g.R / (PAIR ? 256 : 128);
@@ -208,10 +211,13 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN, PAIR>::kThreads, 1)
     // ------------------------------------------------------------ producer
     int stage = 0;
     uint32_t phase = 0;
+    // each tile's entry is read one tile ahead, off the critical path
+    TileEntry te_next = t_first < ntiles ? tile_at((t_first / ksplit) / MT) : TileEntry{};
     for (int t = t_first; t < ntiles && !*abort; t += t_step) {
       const int tt = t / ksplit, split = t % ksplit;
       const int kb0 = split * nkb / ksplit, kb1 = (split + 1) * nkb / ksplit;
-      const TileEntry te = tile_at(tt / MT);
+      const TileEntry te = te_next;
+      if (t + t_step < ntiles) te_next = tile_at(((t + t_step) / ksplit) / MT);
       const int mt = PAIR ? (tt % MT) * 2 + (int)rank : tt % MT;   // this CTA's 128-row weight block
       const uint8_t* sfa = F::kBs ? g.w_sf + (size_t)te.e * g.R * ncols_w + (size_t)mt * (ncols_w / 4) * 512 : nullptr;
       for (int kb = kb0; kb < kb1; ++kb) {
@@ -273,10 +279,13 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN, PAIR>::kThreads, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     // a pair's MMAs are issued by its leader (rank 0) alone
+    // each tile's entry is read one tile ahead, off the critical path
+    TileEntry te_next = t_first < ntiles ? tile_at((t_first / ksplit) / MT) : TileEntry{};
     for (int t = t_first; (!PAIR || rank == 0) && t < ntiles && !*abort; t += t_step) {
       const int tt = t / ksplit, split = t % ksplit;
       const int kb0 = split * nkb / ksplit, kb1 = (split + 1) * nkb / ksplit;
-      const TileEntry te = tile_at(tt / MT);
+      const TileEntry te = te_next;
+      if (t + t_step < ntiles) te_next = tile_at(((t + t_step) / ksplit) / MT);
       if (!tc::mbar_wait(&tempty[acc], acc_phase ^ 1u, abort)) {
         if (lane == 0) raise_status(g.status, MOE_ERR_TIMEOUT);
         *abort = 1;
@@ -379,6 +388,8 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN, PAIR>::kThreads, 1)
     float hmax = 0.0f;
     int acc = 0;
     uint32_t acc_phase = 0;
+    // each tile's entry is read one tile ahead, off the critical path
+    TileEntry te_next = t_first < ntiles ? tile_at((t_first / ksplit) / MT) : TileEntry{};
     for (int t = t_first; t < ntiles; t += t_step) {
       if (!tc::mbar_wait(&tfull[acc], acc_phase, abort)) {
         if (lane == 0) raise_status(g.status, MOE_ERR_TIMEOUT);
@@ -387,7 +398,8 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN, PAIR>::kThreads, 1)
       }
       tc::fence_after_sync();
       const int tt = t / ksplit, split = t % ksplit;
-      const TileEntry te = tile_at(tt / MT);
+      const TileEntry te = te_next;
+      if (t + t_step < ntiles) te_next = tile_at(((t + t_step) / ksplit) / MT);
       const int mt = PAIR ? (tt % MT) * 2 + (int)rank : tt % MT;   // this CTA's 128 weight rows
       const int ncol = min(BN, (te.nvalid + 15) & ~15);
       const int c_lo = cw * 64;
@@ -649,11 +661,13 @@ cudaError_t launch_cfg(const GemmArgs& g, const void* a_base, int64_t a_rows, co
   if constexpr (PAIR) {
     cudaLaunchConfig_t cfg;
     memset(&cfg, 0, sizeof(cfg));
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.blockDim = dim3(C::kThreads);
     cfg.dynamicSmemBytes = C::kSmem;
     cfg.stream = s;
@@ -667,6 +681,7 @@ cudaError_t launch_cfg(const GemmArgs& g, const void* a_base, int64_t a_rows, co
     if (dev < 0 || dev >= 16) return cudaErrorInvalidDevice;
     if (max_pairs[dev] == 0) {
       cfg.gridDim = dim3((unsigned)(num_sms & ~1));
+      cfg.numAttrs = 1;  // the cluster shape alone
       int n = 0;
       e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
       if (e != cudaSuccess) return e;
@@ -675,10 +690,12 @@ cudaError_t launch_cfg(const GemmArgs& g, const void* a_base, int64_t a_rows, co
     }
     const int pairs = max_pairs[dev] < num_sms / 2 ? max_pairs[dev] : num_sms / 2;
     cfg.gridDim = dim3((unsigned)(2 * pairs));
+    cfg.numAttrs = pdl_enabled() ? 2 : 1;
     e = cudaLaunchKernelEx(&cfg, kern, ma, mb, msfa, msfb, my, g);
     if (e != cudaSuccess) return e;
   } else {
-    kern<<<num_sms, C::kThreads, C::kSmem, s>>>(ma, mb, msfa, msfb, my, g);
+    e = launch_pdl(kern, dim3(num_sms), dim3(C::kThreads), C::kSmem, s, ma, mb, msfa, msfb, my, g);
+    if (e != cudaSuccess) return e;
   }
   count_launches(1);
   return cudaGetLastError();
@@ -757,6 +774,9 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ 
                                                     int32_t* __restrict__ poff, TileEntry* __restrict__ tiles,
                                                     int32_t* __restrict__ num_tiles, int max_tiles,
                                                     int32_t* status) {
+  pdl_wait();  // inputs come from the previous kernels
+  pdl_trigger();
+
   __shared__ int32_t s_pad[1024], s_til[1024];
   __shared__ int bad;
   const int e = threadIdx.x;
@@ -806,9 +826,10 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ 
 
 cudaError_t launch_plan(const int32_t* offsets, int E, int64_t S, int bn, int32_t* poff, TileEntry* tiles,
                         int32_t* num_tiles, int max_tiles, int32_t* status, cudaStream_t s) {
-  plan_kernel<<<1, 1024, 0, s>>>(offsets, E, S, bn, poff, tiles, num_tiles, max_tiles, status);
+  cudaError_t e = launch_pdl(plan_kernel, dim3(1), dim3(1024), 0, s, offsets, E, S, bn, poff, tiles, num_tiles,
+                             max_tiles, status);
   count_launches(1);
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 // ---------------------------------------------------- padded quantisation --
@@ -818,6 +839,9 @@ cudaError_t launch_plan(const int32_t* offsets, int E, int64_t S, int bn, int32_
 // offsets[e]); lane l quantises scale blocks l, l + 32, ... of the row.
 template <int FMT, bool SRC_X>
 __global__ void __launch_bounds__(256) quant_padded_kernel(QuantPaddedArgs a) {
+  pdl_wait();  // inputs come from the previous kernels
+  pdl_trigger();
+
   constexpr int bs = FMT == MOE_FMT_MXFP4 ? 32 : 16;
   const int nb = a.K / bs;
   const int lane = threadIdx.x & 31;
@@ -908,6 +932,9 @@ __global__ void __launch_bounds__(256) quant_padded_kernel(QuantPaddedArgs a) {
 // of the slots inv_perm[t * k + j].
 template <int FMT>
 __global__ void __launch_bounds__(256) quant_tokens_kernel(QuantPaddedArgs a) {
+  pdl_wait();  // inputs come from the previous kernels
+  pdl_trigger();
+
   constexpr int bs = FMT == MOE_FMT_MXFP4 ? 32 : 16;
   constexpr int kPer = 64;
   constexpr int kWords = FMT == MOE_FMT_FP8 ? 16 : 8;  // 32-bit code words per lane
@@ -1053,23 +1080,25 @@ __global__ void __launch_bounds__(256) quant_tokens_kernel(QuantPaddedArgs a) {
 
 cudaError_t launch_quant_padded(const QuantPaddedArgs& a, bool src_x, int fmt, int num_sms, cudaStream_t s) {
   if (a.S == 0) return cudaSuccess;
+  cudaError_t e = cudaSuccess;
   if (src_x && a.inv_perm && a.K % 64 == 0) {
     const int64_t blocks = (a.T + 7) / 8;
     const int grid = (int)(blocks < (int64_t)num_sms * 8 ? blocks : (int64_t)num_sms * 8);
     switch (fmt) {
-      case MOE_FMT_NVFP4: quant_tokens_kernel<MOE_FMT_NVFP4><<<grid, 256, 0, s>>>(a); break;
-      case MOE_FMT_MXFP4: quant_tokens_kernel<MOE_FMT_MXFP4><<<grid, 256, 0, s>>>(a); break;
-      case MOE_FMT_FP8: quant_tokens_kernel<MOE_FMT_FP8><<<grid, 256, 0, s>>>(a); break;
+      case MOE_FMT_NVFP4: e = launch_pdl(quant_tokens_kernel<MOE_FMT_NVFP4>, dim3(grid), dim3(256), 0, s, a); break;
+      case MOE_FMT_MXFP4: e = launch_pdl(quant_tokens_kernel<MOE_FMT_MXFP4>, dim3(grid), dim3(256), 0, s, a); break;
+      case MOE_FMT_FP8: e = launch_pdl(quant_tokens_kernel<MOE_FMT_FP8>, dim3(grid), dim3(256), 0, s, a); break;
       default: return cudaErrorInvalidValue;
     }
+    if (e != cudaSuccess) return e;
     count_launches(1);
     return cudaGetLastError();
   }
   const int64_t blocks = (a.S + 7) / 8;
   const int grid = (int)(blocks < (int64_t)num_sms * 8 ? blocks : (int64_t)num_sms * 8);
-#define MOE_QP(F)                                                              \
-  if (src_x) quant_padded_kernel<F, true><<<grid, 256, 0, s>>>(a);           \
-  else quant_padded_kernel<F, false><<<grid, 256, 0, s>>>(a);
+#define MOE_QP(F)                                                                  \
+  e = src_x ? launch_pdl(quant_padded_kernel<F, true>, dim3(grid), dim3(256), 0, s, a) \
+            : launch_pdl(quant_padded_kernel<F, false>, dim3(grid), dim3(256), 0, s, a);
   switch (fmt) {
     case MOE_FMT_NVFP4: MOE_QP(MOE_FMT_NVFP4) break;
     case MOE_FMT_MXFP4: MOE_QP(MOE_FMT_MXFP4) break;
@@ -1077,6 +1106,7 @@ cudaError_t launch_quant_padded(const QuantPaddedArgs& a, bool src_x, int fmt, i
     default: return cudaErrorInvalidValue;
   }
 #undef MOE_QP
+  if (e != cudaSuccess) return e;
   count_launches(1);
   return cudaGetLastError();
 }

@@ -236,6 +236,8 @@ __global__ void __launch_bounds__((1 + kGemvConsumers) * 32, 1)
     tc::prefetch_tmap(&tmap_w);
   }
   __syncthreads();
+  pdl_wait();  // the setup above overlaps the previous kernel's tail
+  pdl_trigger();
 
   const int n_items = __ldg(a.num_tiles) * MT;
   const int i0 = (int)((int64_t)blockIdx.x * n_items / gridDim.x);
@@ -487,7 +489,8 @@ static cudaError_t launch_stage(const GemvArgs& a, int num_sms, cudaStream_t s) 
   cudaError_t err =
       cudaFuncSetAttribute(gemv_ffn_kernel<FMT, STAGE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
-  gemv_ffn_kernel<FMT, STAGE><<<num_sms, (1 + kGemvConsumers) * 32, smem, s>>>(m, a, stages);
+  err = launch_pdl(gemv_ffn_kernel<FMT, STAGE>, dim3(num_sms), dim3((1 + kGemvConsumers) * 32), smem, s, m, a, stages);
+  if (err != cudaSuccess) return err;
   count_launches(1);
   return cudaGetLastError();
 }

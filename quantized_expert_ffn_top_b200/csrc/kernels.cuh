@@ -1,12 +1,37 @@
 // Kernel launchers of the B200 MoE layer (internal; the C ABI is in api.cu).
 #pragma once
 
+#include <string.h>
+
+#include <utility>
+
 #include "common.cuh"
 
 namespace moe {
 
 // Host-side count of kernel launches (moe_kernel_launch_count).
 void count_launches(int n);
+
+// Launch with programmatic dependent launch allowed (MOE_OPT_PDL, on by
+// default): the kernel may begin while the previous kernel in the stream
+// finishes; it calls pdl_wait() before reading that kernel's results.
+bool pdl_enabled();
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 __device__ __forceinline__ float load_f32(const float* p) { return __ldg(p); }
 __device__ __forceinline__ float load_f32(const uint16_t* p) { return bf16_to_f32(__ldg(p)); }

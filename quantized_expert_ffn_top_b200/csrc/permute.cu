@@ -93,6 +93,9 @@ __global__ void __launch_bounds__(kPermWarps * 32) perm_count_kernel(const int32
                                                                      int32_t* __restrict__ ticket,
                                                                      int32_t* __restrict__ offsets, PlanOut plan,
                                                                      int32_t* status) {
+  pdl_wait();  // inputs come from the previous kernels
+  pdl_trigger();
+
   extern __shared__ int32_t cnt[];  // [kPermWarps][E]; the last block reuses it as [E] totals
   __shared__ int32_t warp_tot[kPermWarps];
   __shared__ int is_last;
@@ -185,6 +188,9 @@ __global__ void __launch_bounds__(kPermWarps * 32) perm_scatter_kernel(const int
                                                                        const int32_t* __restrict__ chunk_base,
                                                                        int32_t* __restrict__ perm_token,
                                                                        int32_t* __restrict__ inv_perm) {
+  pdl_wait();  // inputs come from the previous kernels
+  pdl_trigger();
+
   extern __shared__ int32_t cnt[];  // [kPermWarps][E]
   for (int i = threadIdx.x; i < kPermWarps * E; i += blockDim.x) cnt[i] = 0;
   __syncthreads();
@@ -276,6 +282,9 @@ __global__ void __launch_bounds__(kBlockWarps * 32) perm_block_kernel(const int3
                                                                      int32_t* __restrict__ perm_token,
                                                                      int32_t* __restrict__ inv_perm,
                                                                      int32_t* status, PlanOut plan) {
+  pdl_wait();  // inputs come from the previous kernels
+  pdl_trigger();
+
   extern __shared__ int32_t cnt[];  // [kBlockWarps][E], then [E] offsets
   int32_t* tot = cnt + kBlockWarps * E;
   __shared__ int32_t warp_tot[33];
@@ -381,8 +390,9 @@ cudaError_t launch_permute(const int32_t* idx, int64_t S, int k, int E, int32_t*
     } else {
       memset(&p, 0, sizeof(p));
     }
-    perm_block_kernel<<<1, kBlockWarps * 32, block_smem, s>>>(idx, S, k, E, offsets, perm_token, inv_perm, status,
-                                                              p);
+    e = launch_pdl(perm_block_kernel, dim3(1), dim3(kBlockWarps * 32), block_smem, s, idx, S, k, E, offsets, perm_token,
+                   inv_perm, status, p);
+    if (e != cudaSuccess) return e;
     count_launches(1);
     if (planned && plan && plan->bn > 0) *planned = true;
     return cudaGetLastError();
@@ -401,10 +411,12 @@ cudaError_t launch_permute(const int32_t* idx, int64_t S, int k, int E, int32_t*
   }
   cudaError_t e = cudaMemsetAsync(scratch.ticket, 0, sizeof(int32_t), s);
   if (e != cudaSuccess) return e;
-  perm_count_kernel<<<nchunks, kPermWarps * 32, smem, s>>>(idx, S, E, scratch.chunk_counts, scratch.ticket, offsets,
-                                                           p, status);
-  perm_scatter_kernel<<<nchunks, kPermWarps * 32, smem, s>>>(idx, S, k, E, scratch.chunk_counts, perm_token,
-                                                              inv_perm);
+  e = launch_pdl(perm_count_kernel, dim3(nchunks), dim3(kPermWarps * 32), smem, s, idx, S, E, scratch.chunk_counts,
+                 scratch.ticket, offsets, p, status);
+  if (e != cudaSuccess) return e;
+  e = launch_pdl(perm_scatter_kernel, dim3(nchunks), dim3(kPermWarps * 32), smem, s, idx, S, k, E,
+                 (const int32_t*)scratch.chunk_counts, perm_token, inv_perm);
+  if (e != cudaSuccess) return e;
   count_launches(2);
   if (planned && plan && plan->bn > 0) *planned = true;
   return cudaGetLastError();

@@ -14,6 +14,9 @@ namespace moe {
 // ------------------------------------------------------------------ amax --
 template <typename In>
 __global__ void __launch_bounds__(256) amax_kernel(const In* __restrict__ x, int64_t n, float* __restrict__ out) {
+  pdl_wait();  // inputs come from the previous kernels
+  pdl_trigger();
+
   float m = 0.0f;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) m = fmaxf(m, fabsf(load_f32(x + i)));
@@ -34,9 +37,10 @@ cudaError_t launch_amax(const void* x, int x_dtype, int64_t n, float* out, int n
   int64_t blocks = (n + 255) / 256;
   int grid = (int)(blocks < (int64_t)num_sms * 8 ? blocks : (int64_t)num_sms * 8);
   if (x_dtype == 0)
-    amax_kernel<float><<<grid, 256, 0, s>>>(static_cast<const float*>(x), n, out);
+    e = launch_pdl(amax_kernel<float>, dim3(grid), dim3(256), 0, s, static_cast<const float*>(x), n, out);
   else
-    amax_kernel<uint16_t><<<grid, 256, 0, s>>>(static_cast<const uint16_t*>(x), n, out);
+    e = launch_pdl(amax_kernel<uint16_t>, dim3(grid), dim3(256), 0, s, static_cast<const uint16_t*>(x), n, out);
+  if (e != cudaSuccess) return e;
   count_launches(1);
   return cudaGetLastError();
 }

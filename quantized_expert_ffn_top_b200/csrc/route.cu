@@ -25,6 +25,9 @@ __global__ void __launch_bounds__(kSmallThreads) router_logits_small_kernel(cons
                                                                            int H, const uint16_t* __restrict__ wr,
                                                                            const float* __restrict__ bias, int E,
                                                                            float* __restrict__ logits) {
+  pdl_wait();  // inputs come from the previous kernels
+  pdl_trigger();
+
   __shared__ float part[kSmallThreads / 32][kSmallTGroup];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int e = blockIdx.x;
@@ -71,6 +74,9 @@ __global__ void __launch_bounds__(256) router_logits_tiled_kernel(const uint16_t
                                                                   const uint16_t* __restrict__ wr,
                                                                   const float* __restrict__ bias, int E,
                                                                   float* __restrict__ logits) {
+  pdl_wait();  // inputs come from the previous kernels
+  pdl_trigger();
+
   __shared__ float xs[32][65];
   __shared__ float ws[32][65];
   const int tid = threadIdx.x;
@@ -123,10 +129,12 @@ cudaError_t launch_router_logits(const uint16_t* x, int64_t T, int H, const uint
   if (T == 0) return cudaSuccess;
   if (T <= 64 && H % 8 == 0) {
     dim3 grid((unsigned)E, (unsigned)((T + kSmallTGroup - 1) / kSmallTGroup));
-    router_logits_small_kernel<<<grid, kSmallThreads, 0, s>>>(x, T, H, wr, bias, E, logits);
+    cudaError_t e = launch_pdl(router_logits_small_kernel, grid, dim3(kSmallThreads), 0, s, x, T, H, wr, bias, E, logits);
+    if (e != cudaSuccess) return e;
   } else {
     dim3 grid((unsigned)((T + 63) / 64), (E + 63) / 64);
-    router_logits_tiled_kernel<<<grid, 256, 0, s>>>(x, T, H, wr, bias, E, logits);
+    cudaError_t e = launch_pdl(router_logits_tiled_kernel, grid, dim3(256), 0, s, x, T, H, wr, bias, E, logits);
+    if (e != cudaSuccess) return e;
   }
   count_launches(1);
   return cudaGetLastError();
@@ -145,6 +153,9 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
                                                    float* __restrict__ logits_out, int64_t T, int E, int k,
                                                    int32_t* __restrict__ idx, float* __restrict__ w,
                                                    int32_t* status) {
+  pdl_wait();  // inputs come from the previous kernels
+  pdl_trigger();
+
   const int lane = threadIdx.x & 31;
   const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (t >= T) return;
@@ -220,7 +231,9 @@ cudaError_t launch_topk(const float* logits, int nparts, int64_t part_stride, fl
   if (T == 0) return cudaSuccess;
   const unsigned grid = (unsigned)((T + 7) / 8);
   const int J = (E + 31) / 32;
-#define MOE_TOPK(JJ) topk_kernel<JJ><<<grid, 256, 0, s>>>(logits, nparts, part_stride, logits_out, T, E, k, idx, w, status)
+  cudaError_t e = cudaSuccess;
+#define MOE_TOPK(JJ) \
+  e = launch_pdl(topk_kernel<JJ>, dim3(grid), dim3(256), 0, s, logits, nparts, part_stride, logits_out, T, E, k, idx, w, status)
   if (J <= 1) MOE_TOPK(1);
   else if (J <= 2) MOE_TOPK(2);
   else if (J <= 4) MOE_TOPK(4);
@@ -228,6 +241,7 @@ cudaError_t launch_topk(const float* logits, int nparts, int64_t part_stride, fl
   else if (J <= 16) MOE_TOPK(16);
   else MOE_TOPK(32);
 #undef MOE_TOPK
+  if (e != cudaSuccess) return e;
   count_launches(1);
   return cudaGetLastError();
 }
