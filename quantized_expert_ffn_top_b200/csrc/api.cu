@@ -276,8 +276,7 @@ moe_status run_gemm_ffn(const uint16_t* x, int64_t T, int64_t S, const int32_t* 
   const int E = w->E, H = w->H, I = w->I, fmt = w->fmt;
   const int sms = num_sms();
   const int bn = gemm_tile_n(S, E);
-  if (!planned)
-    MOE_TRY(launch_plan(offsets, E, S, bn, f.poff, f.tiles, f.ntiles, (int)max_tiles(S, E), status, s));
+  // without a plan from the permutation, the per-slot x quantiser writes it
   if (mark) stage_mark(MOE_STAGE_ACT_QUANT, false, s);
   QuantPaddedArgs qa;
   qa.E = E;
@@ -291,6 +290,18 @@ moe_status run_gemm_ffn(const uint16_t* x, int64_t T, int64_t S, const int32_t* 
   qa.inv_perm = inv;
   qa.k = k;
   qa.slot_expert = slot_expert;
+  memset(&qa.plan, 0, sizeof(qa.plan));
+  if (!planned) {
+    if (inv) {  // the token quantiser cannot write it
+      MOE_TRY(launch_plan(offsets, E, S, bn, f.poff, f.tiles, f.ntiles, (int)max_tiles(S, E), status, s));
+    } else {
+      qa.plan.bn = bn;
+      qa.plan.poff = f.poff;
+      qa.plan.tiles = f.tiles;
+      qa.plan.ntiles = f.ntiles;
+      qa.plan.max_tiles = (int)max_tiles(S, E);
+    }
+  }
   qa.x = x;
   qa.h32 = nullptr;
   qa.scale = w->a13_gs;

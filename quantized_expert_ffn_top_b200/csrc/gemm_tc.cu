@@ -833,6 +833,83 @@ cudaError_t launch_plan(const int32_t* offsets, int E, int64_t S, int bn, int32_
 }
 
 // ---------------------------------------------------- padded quantisation --
+// The tile plan inside one block of 256 threads: padded offsets into s_poff
+// [E+1] (shared memory) and, when `write`, into plan.poff together with the
+// tile list -- what plan_kernel computes.  Every thread calls it.
+__device__ void plan_in_block(const int32_t* __restrict__ offsets, int E, int64_t S, const PlanOut& plan, bool write,
+                              int32_t* s_poff, int32_t* status) {
+  __shared__ int32_t warp_tot[8];
+  __shared__ int bad;
+  const int per = (E + 255) / 256;
+  const int e0 = threadIdx.x * per;
+  if (threadIdx.x == 0) bad = (__ldg(offsets) != 0 || __ldg(offsets + E) != S) ? 1 : 0;
+  __syncthreads();
+  int32_t pad_mine = 0, til_mine = 0;
+  for (int e = e0; e < e0 + per && e < E; ++e) {
+    int32_t n = __ldg(offsets + e + 1) - __ldg(offsets + e);
+    if (n < 0) {
+      bad = 1;
+      n = 0;
+    }
+    pad_mine += (n + 127) / 128 * 128;
+    til_mine += (n + plan.bn - 1) / plan.bn;
+  }
+  // two exclusive scans over the 256 threads
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int32_t res[2], tot[2];
+  const int32_t val[2] = {pad_mine, til_mine};
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    int32_t incl = val[q];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t n = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += n;
+    }
+    __syncthreads();
+    if (lane == 31) warp_tot[warp] = incl;
+    __syncthreads();
+    int32_t base = 0, sum = 0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      base += w < warp ? warp_tot[w] : 0;
+      sum += warp_tot[w];
+    }
+    res[q] = incl - val[q] + base;
+    tot[q] = sum;
+  }
+  int32_t pbase = res[0], tbase = res[1];
+  for (int e = e0; e < e0 + per && e < E; ++e) {
+    const int32_t o = __ldg(offsets + e);
+    const int32_t n = max(0, __ldg(offsets + e + 1) - o);
+    s_poff[e] = pbase;
+    const int til = (n + plan.bn - 1) / plan.bn;
+    if (write) {
+      plan.poff[e] = pbase;
+      for (int j = 0; j < til && tbase + j < plan.max_tiles; ++j) {
+        TileEntry te;
+        te.e = e;
+        te.row0 = pbase + j * plan.bn;
+        te.nvalid = min(plan.bn, n - j * plan.bn);
+        te.p0 = o + j * plan.bn;
+        plan.tiles[tbase + j] = te;
+      }
+    }
+    pbase += (n + 127) / 128 * 128;
+    tbase += til;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    s_poff[E] = tot[0];
+    if (write) {
+      plan.poff[E] = tot[0];
+      *plan.ntiles = bad ? 0 : min(tot[1], plan.max_tiles);
+      if (bad) raise_status(status, MOE_ERR_DEVICE_FAULT);
+    }
+  }
+  __syncthreads();
+}
+
 // Quantises activation rows into the padded, blocked layout the GEMM reads.
 // One warp per slot p: its source row is x[perm_token[p]] (bf16, SRC_X) or
 // h32[padded row] (fp32), its destination the padded row poff[e] + (p -
@@ -847,13 +924,22 @@ __global__ void __launch_bounds__(256) quant_padded_kernel(QuantPaddedArgs a) {
   const int lane = threadIdx.x & 31;
   const float scale = act_scale_of(FMT, a.scale, a.amax);
   const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  // With a.plan.bn > 0 every block derives the padded offsets from the
+  // offsets itself (and block 0 also writes them and the tile list), so the
+  // tile plan needs no launch of its own.
+  __shared__ int32_t s_poff[1025];
+  const int32_t* poff = a.poff;
+  if (SRC_X && a.plan.bn > 0) {
+    plan_in_block(a.offsets, a.E, a.S, a.plan, blockIdx.x == 0, s_poff, a.status);
+    poff = s_poff;
+  }
   for (int64_t p = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); p < a.S; p += warps) {
     int64_t row = -1;
     int t = -1;
     if (lane == 0) {
       const int e = segment_of(a.offsets, a.E, (int)p);
       const int32_t o = __ldg(a.offsets + e);
-      row = (int64_t)__ldg(a.poff + e) + (p - o);
+      row = (int64_t)poff[e] + (p - o);
       if (row < 0 || row >= a.P || p < o) row = -1;
       if (SRC_X) {
         t = __ldg(a.perm_token + p);

@@ -4,6 +4,7 @@
 #include <stdint.h>
 
 #include "common.cuh"
+#include "kernels.cuh"
 
 namespace moe {
 
@@ -55,6 +56,7 @@ struct QuantPaddedArgs {
   const int32_t* inv_perm;     // x source, optional: slot of each (token, j); then each
   int k;                       //   token is quantised once and written to its k slots
   const int32_t* slot_expert;  //   optional with it: expert of each (token, j) (top-k indices)
+  PlanOut plan;                // per-slot x quantiser: also compute (and write) the tile plan
   const uint16_t* x;           // [T][K] bf16
   const float* h32;            // or fp32 rows at padded positions
   const float* scale;          // static tensor scale or NULL
