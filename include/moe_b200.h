@@ -254,8 +254,28 @@ moe_status moe_get_device_status(void* ws, moe_stream_t stream, int32_t* host_st
  *   MOE_OPT_PDL:       1 (default) launches the layer's kernels with
  *                     programmatic dependent launch, so each one's setup
  *                     overlaps the previous kernel's tail; 0 launches them
- *                     plainly. */
-typedef enum { MOE_OPT_FFN_PATH = 1, MOE_OPT_GEMM_TILE_N = 2, MOE_OPT_GEMM_PAIR = 3, MOE_OPT_PDL = 4 } moe_option;
+ *                     plainly.
+ *   MOE_OPT_EARLY_WEIGHTS: 1 (default) lets each tensor-core GEMM of the
+ *                     expert FFN load the weight tiles of its first pipeline
+ *                     stages before it waits for the previous kernel (the
+ *                     weights are inputs of the call, so only the token
+ *                     operand waits); 2 also prefetches the next stages'
+ *                     weight tiles into L2; 0 loads every stage after the
+ *                     wait.
+ *   MOE_OPT_FUSED_FFN: 1 (default) runs the gate|up and down projections of a
+ *                     64-token-tile batch (T*k < 8E; NVFP4 with a static h
+ *                     scale, or MXFP4; E <= 256) as one persistent kernel
+ *                     in which the down tiles of a token tile start as soon
+ *                     as its gate|up tiles are stored; 0 launches the two
+ *                     projections separately. */
+typedef enum {
+  MOE_OPT_FFN_PATH = 1,
+  MOE_OPT_GEMM_TILE_N = 2,
+  MOE_OPT_GEMM_PAIR = 3,
+  MOE_OPT_PDL = 4,
+  MOE_OPT_EARLY_WEIGHTS = 5,
+  MOE_OPT_FUSED_FFN = 6
+} moe_option;
 moe_status moe_set_option(int32_t option, int32_t value);
 
 /* moe_permute for callers that cannot allocate device memory (no workspace

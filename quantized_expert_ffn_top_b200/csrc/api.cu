@@ -47,6 +47,7 @@ Scalars carve_head(Carver& c) {
 }
 
 int g_ffn_path = 0;  // MOE_OPT_FFN_PATH
+static int g_fused_ffn = 1;  // MOE_OPT_FUSED_FFN
 
 // Measurement hook (moe_set_stage_events).
 cudaEvent_t g_stage_events[2 * MOE_STAGE_COUNT];
@@ -150,6 +151,7 @@ struct FfnScratch {
   uint8_t* hq;       //       [P][I/2 | I]
   uint8_t* hsf;
   float* h32;        //       [P][I] fp32 h (dynamic h scale / FP8)
+  int32_t* tile_done;  //     [max_tiles] fused FFN: gate|up slices finished per token tile
   int64_t P;
 };
 FfnScratch carve_ffn(Carver& c, int64_t S, const moe_weights* w) {
@@ -166,6 +168,7 @@ FfnScratch carve_ffn(Carver& c, int64_t S, const moe_weights* w) {
   f.hq = c.take<uint8_t>((size_t)(f.P * rbi));
   f.hsf = bs ? c.take<uint8_t>((size_t)(f.P * (w->I / bs))) : nullptr;
   f.h32 = c.take<float>((size_t)(f.P * w->I));
+  f.tile_done = c.take<int32_t>((size_t)max_tiles(S, w->E));
   return f;
 }
 
@@ -276,6 +279,11 @@ moe_status run_gemm_ffn(const uint16_t* x, int64_t T, int64_t S, const int32_t* 
   const int E = w->E, H = w->H, I = w->I, fmt = w->fmt;
   const int sms = num_sms();
   const int bn = gemm_tile_n(S, E);
+  // gate|up projection + SwiGLU quantise h in the epilogue when its scale
+  // needs no global reduction (MXFP4, or a static NVFP4 scale); with 64-token
+  // tiles the two projections then run as one kernel
+  const bool fused_h = fmt == MOE_FMT_MXFP4 || (fmt == MOE_FMT_NVFP4 && w->a2_gs);
+  const bool one_kernel = g_fused_ffn && fused_h && bn == 64 && E <= kFusedMaxE;
   // without a plan from the permutation, the per-slot x quantiser writes it
   if (mark) stage_mark(MOE_STAGE_ACT_QUANT, false, s);
   QuantPaddedArgs qa;
@@ -309,11 +317,10 @@ moe_status run_gemm_ffn(const uint16_t* x, int64_t T, int64_t S, const int32_t* 
   qa.codes = f.xq;
   qa.sf = f.xsf;
   qa.status = status;
+  qa.zero = one_kernel ? f.tile_done : nullptr;   // the fused kernel's counters
+  qa.nzero = one_kernel ? (int)max_tiles(S, E) : 0;
   MOE_TRY(launch_quant_padded(qa, true, fmt, sms, s));
   if (mark) stage_mark(MOE_STAGE_ACT_QUANT, true, s);
-  // gate|up projection + SwiGLU: quantise h in the epilogue when its scale
-  // needs no global reduction (MXFP4, or a static NVFP4 scale)
-  const bool fused_h = fmt == MOE_FMT_MXFP4 || (fmt == MOE_FMT_NVFP4 && w->a2_gs);
   GemmArgs g;
   memset(&g, 0, sizeof(g));
   g.fmt = fmt;
@@ -334,21 +341,14 @@ moe_status run_gemm_ffn(const uint16_t* x, int64_t T, int64_t S, const int32_t* 
   g.h32 = f.h32;
   g.h_amax = fused_h ? nullptr : h_amax;
   g.status = status;
-  if (mark) stage_mark(MOE_STAGE_FFN_UP, false, s);
-  if (!fused_h) MOE_TRY(cudaMemsetAsync(h_amax, 0, sizeof(float), s));
-  MOE_TRY(launch_grouped_gemm(g, fused_h ? kEpiUpQuant : kEpiUpF32, bn, w->w13, (int64_t)E * 2 * I,
-                              f.xq, f.P, sms, s));
-  if (!fused_h) {
-    QuantPaddedArgs qh = qa;
-    qh.K = I;
-    qh.h32 = f.h32;
-    qh.scale = w->a2_gs;
-    qh.amax = h_amax;
-    qh.codes = f.hq;
-    qh.sf = f.hsf;
-    MOE_TRY(launch_quant_padded(qh, false, fmt, sms, s));
-  }
-  if (mark) stage_mark(MOE_STAGE_FFN_UP, true, s);
+  // the tile list is two kernels back when the permutation or the plan kernel
+  // wrote it; when the x quantiser just before writes it, the expert offsets
+  // (older) name the experts of the early weight loads
+  const int ew = early_weights();
+  g.w_early = ew == 0 ? 0 : ((planned || inv) ? 1 : 2);
+  g.w_early_l2 = ew == 2 ? kEarlyL2Stages : 0;
+  g.offsets = offsets;
+  g.max_tiles = (int)max_tiles(S, E);
   // down projection -> y_perm
   GemmArgs d;
   memset(&d, 0, sizeof(d));
@@ -368,6 +368,43 @@ moe_status run_gemm_ffn(const uint16_t* x, int64_t T, int64_t S, const int32_t* 
   d.ldy = H;
   d.y_rows = S;
   d.status = status;
+  d.w_early = ew == 0 ? 0 : 1;  // the tile list is at least two kernels back
+  d.w_early_l2 = g.w_early_l2;
+  d.max_tiles = g.max_tiles;
+  if (one_kernel) {
+    // the weights are older than the quantiser: the ring's first pass loads
+    // before the wait (the tile list comes from the offsets in the kernel)
+    g.w_early = ew == 0 ? 0 : 1;
+    FusedArgs fa;
+    fa.offsets = offsets;
+    fa.S = S;
+    fa.P = f.P;
+    fa.tile_done = f.tile_done;
+    fa.max_tiles = (int)max_tiles(S, E);
+    if (mark) stage_mark(MOE_STAGE_FFN_UP, false, s);
+    MOE_TRY(launch_fused_ffn(g, d, fa, w->w13, (int64_t)E * 2 * I, w->w2, (int64_t)E * H, f.xq, f.hq, sms, s));
+    if (mark) {
+      stage_mark(MOE_STAGE_FFN_UP, true, s);
+      stage_mark(MOE_STAGE_FFN_DOWN, false, s);
+      stage_mark(MOE_STAGE_FFN_DOWN, true, s);
+    }
+    return MOE_OK;
+  }
+  if (mark) stage_mark(MOE_STAGE_FFN_UP, false, s);
+  if (!fused_h) MOE_TRY(cudaMemsetAsync(h_amax, 0, sizeof(float), s));
+  MOE_TRY(launch_grouped_gemm(g, fused_h ? kEpiUpQuant : kEpiUpF32, bn, w->w13, (int64_t)E * 2 * I,
+                              f.xq, f.P, sms, s));
+  if (!fused_h) {
+    QuantPaddedArgs qh = qa;
+    qh.K = I;
+    qh.h32 = f.h32;
+    qh.scale = w->a2_gs;
+    qh.amax = h_amax;
+    qh.codes = f.hq;
+    qh.sf = f.hsf;
+    MOE_TRY(launch_quant_padded(qh, false, fmt, sms, s));
+  }
+  if (mark) stage_mark(MOE_STAGE_FFN_UP, true, s);
   if (mark) stage_mark(MOE_STAGE_FFN_DOWN, false, s);
   MOE_TRY(launch_grouped_gemm(d, kEpiDown, bn, w->w2, (int64_t)E * H, f.hq, f.P, sms, s));
   if (mark) stage_mark(MOE_STAGE_FFN_DOWN, true, s);
@@ -526,6 +563,16 @@ moe_status moe_set_option(int32_t option, int32_t value) {
   if (option == MOE_OPT_PDL) {
     if (value != 0 && value != 1) return MOE_ERR_INVALID_ARG;
     g_pdl = value;
+    return MOE_OK;
+  }
+  if (option == MOE_OPT_FUSED_FFN) {
+    if (value != 0 && value != 1) return MOE_ERR_INVALID_ARG;
+    g_fused_ffn = value;
+    return MOE_OK;
+  }
+  if (option == MOE_OPT_EARLY_WEIGHTS) {
+    if (value < 0 || value > 2) return MOE_ERR_INVALID_ARG;
+    set_early_weights(value);
     return MOE_OK;
   }
   if (option == MOE_OPT_GEMM_PAIR) {

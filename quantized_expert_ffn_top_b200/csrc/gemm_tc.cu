@@ -32,12 +32,18 @@
 //    ("padded" rows), K-major codes, scales blocked the same way.
 #include <cuda.h>
 
+#include <climits>
+#include <cstdint>
+
 #include "kernels.cuh"
 #include "gemm_tc.cuh"
 #include "tc_ptx.cuh"
 
 namespace moe {
 namespace {
+
+// one warp pair's [32 tokens][36] fp32 epilogue tile
+constexpr int kEpiTileBytes = 32 * 36 * 4;
 
 template <int FMT>
 struct FmtTraits {
@@ -69,7 +75,7 @@ struct Cfg {
   // epilogue shared memory: one [32 tokens][36] fp32 tile per warp pair (SwiGLU
   // transpose; 1 KB of it per warp stages the down projection's stores) and
   // the NVFP4 h multiplier table
-  static constexpr int kEpiTile = 32 * 36 * 4;
+  static constexpr int kEpiTile = kEpiTileBytes;
   static constexpr int kEpiBytes = (4 * (BN / 64) / 2) * kEpiTile + 512;
   static constexpr int kStages = (220 * 1024 - kEpiBytes - 2048) / kStage < 8
                                      ? (220 * 1024 - kEpiBytes - 2048) / kStage
@@ -117,6 +123,214 @@ struct TokenMaps {
 
 __device__ __forceinline__ int token_box_index(int rows) {
   return rows <= 16 ? 0 : (rows <= 32 ? 1 : (rows <= 64 ? 2 : (rows <= 128 ? 3 : 4)));
+}
+
+// The plan's tile list held in registers, derived from the compact offsets
+// by one warp (E <= 256): lane l keeps offsets[8l .. 8l+8] and the tiles and
+// padded rows of all experts before 8l.  Tile tt of the list is the same
+// entry the plan kernels write: experts in order, ceil(n_e / bn) tiles each,
+// expert segments starting on multiples of 128 padded rows.
+struct WarpPlan {
+  int lo0;          // offsets[8l]
+  int hi[8];        // offsets[8l + j + 1] (held at the last offset past E)
+  int tbase, pbase; // tiles and padded rows before expert 8l
+  int ntiles;       // tiles of all experts
+  bool ok;          // offsets[0] == 0, non-decreasing, offsets[E] == S (S >= 0), fits P and max_tiles
+
+  __device__ __forceinline__ void load(const int32_t* offsets, int E, int bn, int64_t S, int64_t P, int max_tiles) {
+    const int lane = threadIdx.x & 31, e0 = 8 * lane;
+    lo0 = e0 <= E ? __ldcg(offsets + e0) : 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) hi[j] = e0 + j < E ? __ldcg(offsets + e0 + j + 1) : 0;
+    bool good = !(lane == 0 && lo0 != 0);
+    int tsum = 0, psum = 0, prev = lo0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (e0 + j >= E) hi[j] = prev;
+      const int n = hi[j] - prev;
+      if (n < 0) good = false;
+      if (e0 + j == E - 1 && S >= 0 && (int64_t)hi[j] != S) good = false;
+      const int nn = max(n, 0);
+      tsum += (nn + bn - 1) / bn;
+      psum += (nn + 127) / 128 * 128;
+      prev = hi[j];
+    }
+    int ti = tsum, pi = psum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int a = __shfl_up_sync(0xffffffffu, ti, o), b = __shfl_up_sync(0xffffffffu, pi, o);
+      if (lane >= o) {
+        ti += a;
+        pi += b;
+      }
+    }
+    tbase = ti - tsum;
+    pbase = pi - psum;
+    ntiles = __shfl_sync(0xffffffffu, ti, 31);
+    const int prows = __shfl_sync(0xffffffffu, pi, 31);
+    ok = __all_sync(0xffffffffu, good) && ntiles <= max_tiles && (int64_t)prows <= P;
+  }
+  // Entry tt (< ntiles): whole warp.
+  __device__ __forceinline__ TileEntry at(int tt, int bn) const {
+    const int lane = threadIdx.x & 31;
+    int c = tbase, pr = pbase, prev = lo0;
+    TileEntry te{-1, 0, 0, 0};
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int n = max(hi[j] - prev, 0);
+      const int til = (n + bn - 1) / bn;
+      if (te.e < 0 && tt >= c && tt < c + til) {
+        const int jt = tt - c;
+        te.e = 8 * lane + j;
+        te.row0 = pr + jt * bn;
+        te.nvalid = min(bn, n - jt * bn);
+        te.p0 = prev + jt * bn;
+      }
+      c += til;
+      pr += (n + 127) / 128 * 128;
+      prev = hi[j];
+    }
+    const unsigned m = __ballot_sync(0xffffffffu, te.e >= 0);
+    const int src = m ? __ffs(m) - 1 : 0;
+    TileEntry r;
+    r.e = m ? __shfl_sync(0xffffffffu, te.e, src) : -1;
+    r.row0 = __shfl_sync(0xffffffffu, te.row0, src);
+    r.nvalid = __shfl_sync(0xffffffffu, te.nvalid, src);
+    r.p0 = __shfl_sync(0xffffffffu, te.p0, src);
+    return r;
+  }
+};
+
+// Converts and stores an epilogue warp's slice of one tile: nch 16-column
+// chunks of its 64 accumulator columns (from c_lo), in r0..r3.
+template <int FMT, int EPI, int BN>
+__device__ __forceinline__ void epilogue_slice(const GemmArgs& g, const CUtensorMap* tmap_y, const TileEntry& te,
+                                               int mt, int split, int nch, int c_lo, int ew, int q, int lane,
+                                               float gact, float g2, float* epi_tiles, const float* r_tab,
+                                               uint16_t* y_stage, float& hmax, const uint32_t* r0,
+                                               const uint32_t* r1, const uint32_t* r2, const uint32_t* r3) {
+#pragma unroll
+  for (int ch = 0; ch < 4; ++ch) {
+    if (ch >= nch) break;  // both warps of a pair see the same ncol
+    const uint32_t* rr = ch == 0 ? r0 : (ch == 1 ? r1 : (ch == 2 ? r2 : r3));
+    float v[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(rr[j]);
+    const int c0 = c_lo + ch * 16;
+    if (EPI == kEpiLogits) {
+      const int o = mt * 128 + q * 32 + lane;  // expert
+      const float b = (g.bias && split == 0) ? __ldg(g.bias + o) : 0.0f;   // the bias joins split 0
+      float* out = g.logits + (size_t)split * g.split_stride;
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        const int tok = c0 + c;
+        if (tok < te.nvalid) out[(size_t)(te.p0 + tok) * g.ldy + o] = v[c] + b;
+      }
+    } else if (EPI == kEpiDown) {
+      const float sc = (FMT == MOE_FMT_MXFP4) ? 1.0f : __ldg(g.w_gs + te.e) * gact;
+      if (c0 + 16 <= te.nvalid) {
+        // a full chunk: stage [16 tokens][32 outputs] as bf16 in this
+        // warp's 1 KB and write it with one tensor store
+        uint16_t* stg = y_stage + ew * 512;
+        if (lane == 0) tc::bulk_wait_read();   // the previous store has read the buffer
+        __syncwarp();
+#pragma unroll
+        for (int c = 0; c < 16; ++c) stg[c * 32 + lane] = f32_to_bf16_rn(v[c] * sc);
+        tc::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tc::tma_store_2d(tmap_y, stg, mt * 128 + q * 32, te.p0 + c0);
+          tc::bulk_commit();
+        }
+      } else {
+        // the tile's last, partial chunk: the rows past nvalid belong to
+        // the next expert's slots
+        const int o = mt * 128 + q * 32 + lane;
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const int tok = c0 + c;
+          if (tok < te.nvalid) g.y[(size_t)(te.p0 + tok) * g.ldy + o] = f32_to_bf16_rn(v[c] * sc);
+        }
+      }
+    } else {
+      // gate|up rows interleave (even lane gate, odd lane up): one shuffle
+      // pairs them and SwiGLU runs on every lane.  Two chunks (32 tokens)
+      // pass through the warp pair's shared-memory tile so that each of
+      // the pair's 64 threads then owns 16 consecutive features of one
+      // token -- one NVFP4 block, half an MXFP4 block -- for the block
+      // maximum, the scale, the codes and 8-byte stores.
+      if (ch & 1) continue;  // taken together with the even chunk
+      const int part = lane & 1;
+      const float sc = (FMT == MOE_FMT_MXFP4) ? 1.0f : __ldg(g.w_gs + te.e * 2 + part) * gact;
+      const int pp = q & 1;                                       // position in the warp pair
+      float* tile = epi_tiles + (ew >> 1) * (kEpiTileBytes / 4);    // [32 tokens][36] of the pair
+      const int fl = lane >> 1;                                   // feature within the warp's 16
+      const int f_pair = mt * 64 + (q >> 1) * 32;                 // first feature of the pair
+      const int bar = 1 + (ew >> 1);
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        if (hf == 1 && ch + 1 >= nch) break;  // tokens past the tile: their rows are never stored
+        const uint32_t* rh = hf == 0 ? rr : (ch == 0 ? r1 : r3);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float a = __uint_as_float(rh[2 * i]) * sc, b = __uint_as_float(rh[2 * i + 1]) * sc;
+          const float recv = __shfl_xor_sync(0xffffffffu, part ? a : b, 1);
+          const float gg = part ? recv : a;
+          const float uu = part ? b : recv;
+          tile[(hf * 16 + 2 * i + part) * 36 + pp * 16 + fl] = silu_fast(gg) * uu;
+        }
+      }
+      asm volatile("bar.sync %0, 64;" ::"r"(bar) : "memory");
+      const int tid = pp * 32 + lane;
+      const int tl = tid >> 1, hh = tid & 1;
+      const float4* src = reinterpret_cast<const float4*>(tile + tl * 36 + 16 * hh);
+      float hv[16];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float4 f = src[j];
+        hv[4 * j] = f.x;
+        hv[4 * j + 1] = f.y;
+        hv[4 * j + 2] = f.z;
+        hv[4 * j + 3] = f.w;
+      }
+      const int tok = c0 + tl;
+      const bool valid = tok < te.nvalid;
+      const size_t row = (size_t)(te.row0 + tok);
+      const int f0 = f_pair + 16 * hh;  // this thread's 16 features
+      if (EPI == kEpiUpF32) {
+        if (valid) {
+          float4* dst = reinterpret_cast<float4*>(g.h32 + row * g.I + f0);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) dst[j] = src[j];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) hmax = fmaxf(hmax, fabsf(hv[j]));
+        }
+      } else {
+        float bmax = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) bmax = fmaxf(bmax, fabsf(hv[j]));
+        uint2 codes;
+        uint32_t scode;
+        if (FMT == MOE_FMT_NVFP4) {
+          scode = nvfp4_scale_code(bmax, g2);
+          codes = nvfp4_encode16(hv, r_tab[scode]);
+        } else {
+          bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 1));  // the 32-feature block
+          float inv;
+          mxfp4_block_scale(bmax, scode, inv);
+          codes = make_uint2(e2m1_encode8(hv, inv), e2m1_encode8(hv + 8, inv));
+        }
+        if (valid) {
+          *reinterpret_cast<uint2*>(g.hq + row * (g.I / 2) + f0 / 2) = codes;
+          if (FMT == MOE_FMT_NVFP4)
+            g.hsf[sf_blocked_offset((int64_t)row, f0 / 16, g.I / 16)] = (uint8_t)scode;
+          if (FMT == MOE_FMT_MXFP4 && hh == 0)
+            g.hsf[sf_blocked_offset((int64_t)row, f0 / 32, g.I / 32)] = (uint8_t)scode;
+        }
+      }
+      asm volatile("bar.sync %0, 64;" ::"r"(bar) : "memory");
+    }
+  }
 }
 
 template <int FMT, int EPI, int BN, bool PAIR>
@@ -173,12 +387,74 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN, PAIR>::kThreads, 1)
   if constexpr (PAIR) tc::cluster_sync();
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
-  // the setup above overlaps the previous kernel's tail (programmatic launch)
-  pdl_wait();
-  pdl_trigger();
   const uint32_t rank = PAIR ? tc::cluster_rank() : 0u;
   // tiles: (token tile, weight-row block of 128 rows, or 256 for a pair)
   const int MT = g.R / (PAIR ? 256 : 128);
+  const int nkb = g.K / F::kBK;
+  const int ncols_w = F::kBs ? g.K / F::kBs : 0;  // scale columns per row (multiple of 4)
+  // Early weight loads: the weights (and their scales) are inputs of the
+  // layer, so while the previous kernel still runs the producer fills the
+  // first pass of the ring with its first stages' weight tiles.  Each such
+  // stage's barrier expects the weight bytes now, without an arrival; the
+  // main loop arrives with the token bytes.  pre_e records the expert of
+  // every early stage, checked against the tile list once it is readable.
+  int n_pre = 0;
+  int pre_e[C::kStages];
+  if constexpr (!PAIR && EPI != kEpiLogits) {
+    if (warp == 0 && g.w_early != 0 && (g.w_early == 1 || g.E <= 256)) {
+      // past the ring, up to w_early_l2 more stages' weights go to L2
+      const int budget = C::kStages + g.w_early_l2;
+      const int nitems = min(32, (budget + nkb - 1) / nkb);
+      // lane i: the expert of this CTA's i-th work item (-1: none), every
+      // read in one round trip
+      int e_i = -1;
+      if (g.w_early == 1) {
+        const int tt_i = (int)((blockIdx.x + (unsigned)lane * gridDim.x) / (unsigned)MT);
+        const int nt = __ldcg(g.num_tiles);
+        const int e = (lane < nitems && tt_i < g.max_tiles) ? __ldcg(&g.tiles[tt_i].e) : -1;
+        e_i = tt_i < nt ? e : -1;
+      } else {
+        // the plan's tile list from the offsets
+        WarpPlan wp;
+        wp.load(g.offsets, g.E, BN, -1, INT64_MAX, INT_MAX);
+        for (int i = 0; i < nitems; ++i) {
+          const int tt = (int)((blockIdx.x + (unsigned)i * gridDim.x) / (unsigned)MT);
+          const int e = tt < wp.ntiles ? wp.at(tt, BN).e : -1;
+          if (lane == i) e_i = e;
+        }
+      }
+      int n_l2 = 0;
+      for (int i = 0; i < nitems && n_pre + n_l2 < budget; ++i) {
+        const int e = __shfl_sync(0xffffffffu, e_i, i);
+        if (e < 0 || e >= g.E) break;
+        const int mt = (int)((blockIdx.x + (unsigned)i * gridDim.x) % (unsigned)MT);
+        const uint8_t* sfa = F::kBs ? g.w_sf + (size_t)e * g.R * ncols_w + (size_t)mt * (ncols_w / 4) * 512 : nullptr;
+        for (int kb = 0; kb < nkb && n_pre + n_l2 < budget; ++kb) {
+          if (n_pre < C::kStages) {
+            if (tc::elect_one()) {
+              uint8_t* st = smem + n_pre * C::kStage;
+              tc::mbar_expect_tx_only(&full[n_pre], C::kA + C::kSFA);
+              tc::tma_load_2d(st, &tmap_a, &full[n_pre], kb * 128, e * g.R + mt * 128);
+              if (F::kBs)
+                tc::bulk_load(st + C::kA + C::kB, sfa + (size_t)kb * F::kGroups * 512, C::kSFA, &full[n_pre]);
+            }
+            __syncwarp();
+            pre_e[n_pre++] = e;
+          } else {
+            if (tc::elect_one()) {
+              tc::tma_prefetch_2d(&tmap_a, kb * 128, e * g.R + mt * 128);
+              if (F::kBs) tc::bulk_prefetch_l2(sfa + (size_t)kb * F::kGroups * 512, C::kSFA);
+            }
+            __syncwarp();
+            ++n_l2;
+          }
+        }
+      }
+    }
+  }
+  // the work above overlaps the previous kernel's tail (programmatic launch)
+  pdl_wait();
+  pdl_trigger();
   // The router GEMM may split K over ksplit CTAs per tile (partial logits
   // that the top-k kernel adds); work item t -> tile t / ksplit, split t % ksplit.
   const int ksplit = EPI == kEpiLogits ? g.ksplit : 1;
@@ -200,8 +476,6 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN, PAIR>::kThreads, 1)
   const int ntiles = ntok * MT * ksplit;
   const int t_first = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
   const int t_step = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
-  const int nkb = g.K / F::kBK;
-  const int ncols_w = F::kBs ? g.K / F::kBs : 0;  // scale columns per row (multiple of 4)
 
   // The producer and MMA warps run their loops with the whole warp, so the
   // loop state stays warp-uniform, and one elected lane issues the copies
@@ -211,6 +485,7 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN, PAIR>::kThreads, 1)
     // ------------------------------------------------------------ producer
     int stage = 0;
     uint32_t phase = 0;
+    int issued = 0;  // stages issued by this loop; the first n_pre hold early weight loads
     // each tile's entry is read one tile ahead, off the critical path
     TileEntry te_next = t_first < ntiles ? tile_at((t_first / ksplit) / MT) : TileEntry{};
     for (int t = t_first; t < ntiles && !*abort; t += t_step) {
@@ -252,11 +527,14 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN, PAIR>::kThreads, 1)
           const int bi = token_box_index(min(te.nvalid, BN));
           const uint32_t brows = min(16u << bi, (uint32_t)BN);   // the map's box height
           const int nblk = ((te.row0 & 127) + min(te.nvalid, BN) + 127) / 128;   // 128-row scale blocks in use
-          tc::mbar_expect_tx(&full[stage], C::kA + brows * 128u + C::kSFA + nblk * F::kGroups * 512);
-          tc::tma_load_2d(st, &tmap_a, &full[stage], kb * 128, te.e * g.R + mt * 128);
+          const bool early = issued < n_pre;   // weights already in flight (stage == issued)
+          if (early && pre_e[issued] != te.e) raise_status(g.status, MOE_ERR_DEVICE_FAULT);
+          tc::mbar_expect_tx(&full[stage], (early ? 0u : (uint32_t)(C::kA + C::kSFA)) + brows * 128u +
+                                               nblk * F::kGroups * 512);
+          if (!early) tc::tma_load_2d(st, &tmap_a, &full[stage], kb * 128, te.e * g.R + mt * 128);
           tc::tma_load_2d(st + C::kA, &tmaps_b.m[bi], &full[stage], kb * 128, te.row0);
           if (F::kBs) {
-            tc::bulk_load(st + C::kA + C::kB, sfa + (size_t)kb * F::kGroups * 512, C::kSFA, &full[stage]);
+            if (!early) tc::bulk_load(st + C::kA + C::kB, sfa + (size_t)kb * F::kGroups * 512, C::kSFA, &full[stage]);
             for (int nb = 0; nb < nblk; ++nb) {
               const uint8_t* sfb =
                   g.b_sf + ((size_t)(te.row0 / 128 + nb) * (ncols_w / 4) + (size_t)kb * F::kGroups) * 512;
@@ -266,10 +544,22 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN, PAIR>::kThreads, 1)
           }
         }
         __syncwarp();
+        ++issued;
         if (++stage == C::kStages) {
           stage = 0;
           phase ^= 1u;
         }
+      }
+    }
+    // early weight loads that no tile consumed (a shorter tile list, or an
+    // abort): arrive, so the barrier completes when they land, and wait for
+    // that before the shared memory goes away
+    for (int i = issued; i < n_pre; ++i) {
+      if (tc::elect_one()) tc::mbar_arrive(&full[i]);
+      __syncwarp();
+      if (!tc::mbar_wait(&full[i], 0, abort) && !*abort) {
+        if (lane == 0) raise_status(g.status, MOE_ERR_TIMEOUT);
+        *abort = 1;
       }
     }
   } else if (warp == 1) {
@@ -428,128 +718,8 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN, PAIR>::kThreads, 1)
         acc_phase ^= 1u;
       }
       if (c_lo >= ncol) continue;  // both warps of a pair (same slice) skip together
-#pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        if (ch >= nch) break;  // both warps of a pair see the same ncol
-        const uint32_t* rr = ch == 0 ? r0 : (ch == 1 ? r1 : (ch == 2 ? r2 : r3));
-        float v[16];
-#pragma unroll
-        for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(rr[j]);
-        const int c0 = c_lo + ch * 16;
-        if (EPI == kEpiLogits) {
-          const int o = mt * 128 + q * 32 + lane;  // expert
-          const float b = (g.bias && split == 0) ? __ldg(g.bias + o) : 0.0f;   // the bias joins split 0
-          float* out = g.logits + (size_t)split * g.split_stride;
-#pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const int tok = c0 + c;
-            if (tok < te.nvalid) out[(size_t)(te.p0 + tok) * g.ldy + o] = v[c] + b;
-          }
-        } else if (EPI == kEpiDown) {
-          const float sc = (FMT == MOE_FMT_MXFP4) ? 1.0f : __ldg(g.w_gs + te.e) * gact;
-          if (c0 + 16 <= te.nvalid) {
-            // a full chunk: stage [16 tokens][32 outputs] as bf16 in this
-            // warp's 1 KB and write it with one tensor store
-            uint16_t* stg = reinterpret_cast<uint16_t*>(epi_tiles) + ew * 512;
-            if (lane == 0) tc::bulk_wait_read();   // the previous store has read the buffer
-            __syncwarp();
-#pragma unroll
-            for (int c = 0; c < 16; ++c) stg[c * 32 + lane] = f32_to_bf16_rn(v[c] * sc);
-            tc::fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-              tc::tma_store_2d(&tmap_y, stg, mt * 128 + q * 32, te.p0 + c0);
-              tc::bulk_commit();
-            }
-          } else {
-            // the tile's last, partial chunk: the rows past nvalid belong to
-            // the next expert's slots
-            const int o = mt * 128 + q * 32 + lane;
-#pragma unroll
-            for (int c = 0; c < 16; ++c) {
-              const int tok = c0 + c;
-              if (tok < te.nvalid) g.y[(size_t)(te.p0 + tok) * g.ldy + o] = f32_to_bf16_rn(v[c] * sc);
-            }
-          }
-        } else {
-          // gate|up rows interleave (even lane gate, odd lane up): one shuffle
-          // pairs them and SwiGLU runs on every lane.  Two chunks (32 tokens)
-          // pass through the warp pair's shared-memory tile so that each of
-          // the pair's 64 threads then owns 16 consecutive features of one
-          // token -- one NVFP4 block, half an MXFP4 block -- for the block
-          // maximum, the scale, the codes and 8-byte stores.
-          if (ch & 1) continue;  // taken together with the even chunk
-          const int part = lane & 1;
-          const float sc = (FMT == MOE_FMT_MXFP4) ? 1.0f : __ldg(g.w_gs + te.e * 2 + part) * gact;
-          const int pp = q & 1;                                       // position in the warp pair
-          float* tile = epi_tiles + (ew >> 1) * (C::kEpiTile / 4);    // [32 tokens][36] of the pair
-          const int fl = lane >> 1;                                   // feature within the warp's 16
-          const int f_pair = mt * 64 + (q >> 1) * 32;                 // first feature of the pair
-          const int bar = 1 + (ew >> 1);
-#pragma unroll
-          for (int hf = 0; hf < 2; ++hf) {
-            if (hf == 1 && ch + 1 >= nch) break;  // tokens past the tile: their rows are never stored
-            const uint32_t* rh = hf == 0 ? rr : (ch == 0 ? r1 : r3);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const float a = __uint_as_float(rh[2 * i]) * sc, b = __uint_as_float(rh[2 * i + 1]) * sc;
-              const float recv = __shfl_xor_sync(0xffffffffu, part ? a : b, 1);
-              const float gg = part ? recv : a;
-              const float uu = part ? b : recv;
-              tile[(hf * 16 + 2 * i + part) * 36 + pp * 16 + fl] = silu_fast(gg) * uu;
-            }
-          }
-          asm volatile("bar.sync %0, 64;" ::"r"(bar) : "memory");
-          const int tid = pp * 32 + lane;
-          const int tl = tid >> 1, hh = tid & 1;
-          const float4* src = reinterpret_cast<const float4*>(tile + tl * 36 + 16 * hh);
-          float hv[16];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const float4 f = src[j];
-            hv[4 * j] = f.x;
-            hv[4 * j + 1] = f.y;
-            hv[4 * j + 2] = f.z;
-            hv[4 * j + 3] = f.w;
-          }
-          const int tok = c0 + tl;
-          const bool valid = tok < te.nvalid;
-          const size_t row = (size_t)(te.row0 + tok);
-          const int f0 = f_pair + 16 * hh;  // this thread's 16 features
-          if (EPI == kEpiUpF32) {
-            if (valid) {
-              float4* dst = reinterpret_cast<float4*>(g.h32 + row * g.I + f0);
-#pragma unroll
-              for (int j = 0; j < 4; ++j) dst[j] = src[j];
-#pragma unroll
-              for (int j = 0; j < 16; ++j) hmax = fmaxf(hmax, fabsf(hv[j]));
-            }
-          } else {
-            float bmax = 0.0f;
-#pragma unroll
-            for (int j = 0; j < 16; ++j) bmax = fmaxf(bmax, fabsf(hv[j]));
-            uint2 codes;
-            uint32_t scode;
-            if (FMT == MOE_FMT_NVFP4) {
-              scode = nvfp4_scale_code(bmax, g2);
-              codes = nvfp4_encode16(hv, r_tab[scode]);
-            } else {
-              bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 1));  // the 32-feature block
-              float inv;
-              mxfp4_block_scale(bmax, scode, inv);
-              codes = make_uint2(e2m1_encode8(hv, inv), e2m1_encode8(hv + 8, inv));
-            }
-            if (valid) {
-              *reinterpret_cast<uint2*>(g.hq + row * (g.I / 2) + f0 / 2) = codes;
-              if (FMT == MOE_FMT_NVFP4)
-                g.hsf[sf_blocked_offset((int64_t)row, f0 / 16, g.I / 16)] = (uint8_t)scode;
-              if (FMT == MOE_FMT_MXFP4 && hh == 0)
-                g.hsf[sf_blocked_offset((int64_t)row, f0 / 32, g.I / 32)] = (uint8_t)scode;
-            }
-          }
-          asm volatile("bar.sync %0, 64;" ::"r"(bar) : "memory");
-        }
-      }
+      epilogue_slice<FMT, EPI, BN>(g, &tmap_y, te, mt, split, nch, c_lo, ew, q, lane, gact, g2, epi_tiles, r_tab,
+                                   reinterpret_cast<uint16_t*>(epi_tiles), hmax, r0, r1, r2, r3);
     }
     if (EPI == kEpiDown && lane == 0) tc::bulk_wait_all();   // stores done before the CTA exits
     if (EPI == kEpiUpF32 && g.h_amax) {
@@ -574,6 +744,359 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN, PAIR>::kThreads, 1)
     if constexpr (PAIR) tc::tmem_dealloc_pair(tmem, C::kTmemCols);
     else tc::tmem_dealloc(tmem, C::kTmemCols);
   }
+}
+
+// ------------------------------------------------------- fused expert FFN --
+// gate|up + SwiGLU + h quantisation and the down projection in one
+// persistent kernel (64-token tiles, NVFP4 / MXFP4 with an h scale that needs
+// no global reduction).  Work item i is gate|up tile i for i < n1 = tiles *
+// MT1, else down tile i - n1; CTA b runs items b, b + grid, ..., so its
+// gate|up items all come before its down items and no CTA waits for a down
+// item.  (Evening out the per-CTA stage counts by handing the down items to
+// the CTAs with fewer gate|up items measured slower: the down tiles of the
+// token tiles that end last then pile up on fewer CTAs.)  Each epilogue warp counts its gate|up slice of token tile
+// tt in tile_done[tt] after storing it; the producer issues a down item's
+// token operand (h) once all MT1 * warps slices of its tile are counted.  The
+// producer keeps two cursors over the ring: weight tiles go out as soon as a
+// stage is free (before the dependency, and before the wait on the previous
+// kernel for the ring's first pass), token tiles as their data is ready.
+template <int FMT, int BN>
+struct FusedCfg {
+  using C = Cfg<FMT, kEpiUpQuant, BN, false>;
+  static constexpr int kSmem = C::kSmem + C::kEpiWarps * 1024;   // + the down store staging
+  static_assert(kSmem <= 227 * 1024, "shared memory");
+};
+
+template <int FMT, int BN>
+__global__ void __launch_bounds__(Cfg<FMT, kEpiUpQuant, BN, false>::kThreads, 1)
+    fused_ffn_kernel(const __grid_constant__ CUtensorMap tmap_w13, const __grid_constant__ TokenMaps tmaps_x,
+                     const __grid_constant__ CUtensorMap tmap_w2, const __grid_constant__ TokenMaps tmaps_h,
+                     const __grid_constant__ CUtensorMap tmap_y, const GemmArgs g1, const GemmArgs g2,
+                     const FusedArgs f) {
+  using C = Cfg<FMT, kEpiUpQuant, BN, false>;
+  using F = FmtTraits<FMT>;
+  static_assert(F::kBs > 0, "block-scaled formats only");
+  static_assert(C::kSfbBlocks == 1, "one scale block per token tile");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* ctrl = smem + C::kStages * C::kStage;
+  uint64_t* full = reinterpret_cast<uint64_t*>(ctrl);
+  uint64_t* empty = full + C::kStages;
+  uint64_t* tfull = empty + C::kStages;
+  uint64_t* tempty = tfull + C::kAccStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + C::kAccStages);
+  volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* epi_tiles = reinterpret_cast<float*>(ctrl + 1024);
+  float* r_tab = epi_tiles + (C::kEpiWarps / 2) * (C::kEpiTile / 4);
+  // the down projection's store staging, 1 KB per warp, apart from the
+  // SwiGLU tiles (a warp may start its first down tile while its pair
+  // partner still finishes the last gate|up tile)
+  uint16_t* y_stage = reinterpret_cast<uint16_t*>(r_tab + 128);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      tc::mbar_init(&full[s], 1);
+      tc::mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < C::kAccStages; ++a) {
+      tc::mbar_init(&tfull[a], 1);
+      tc::mbar_init(&tempty[a], C::kEpiWarps);
+    }
+    *abort = 0;
+    tc::fence_mbar_init();
+    tc::prefetch_tmap(&tmap_w13);
+    tc::prefetch_tmap(&tmap_w2);
+#pragma unroll
+    for (int i = 0; i < 5; ++i) {
+      tc::prefetch_tmap(&tmaps_x.m[i]);
+      tc::prefetch_tmap(&tmaps_h.m[i]);
+    }
+    tc::prefetch_tmap(&tmap_y);
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(tmem_slot, C::kTmemCols);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+
+  // Every warp derives the tile list itself; the offsets are older than the
+  // previous kernel (they are read before waiting for it).
+  WarpPlan plan;
+  plan.load(f.offsets, g1.E, BN, f.S, f.P, f.max_tiles);
+  const int ntok = plan.ok ? plan.ntiles : 0;
+  if (!plan.ok && blockIdx.x == 0 && threadIdx.x == 0) raise_status(g1.status, MOE_ERR_DEVICE_FAULT);
+  const int MT1 = g1.R / 128, MT2 = g2.R / 128;
+  const int nkb1 = g1.K / F::kBK, nkb2 = g2.K / F::kBK;
+  const int ncols1 = g1.K / F::kBs, ncols2 = g2.K / F::kBs;
+  const int n1 = ntok * MT1, total = n1 + ntok * MT2;
+  const int done_target = MT1 * C::kEpiWarps;
+  // item k of this CTA: up (gate|up or down), token tile, weight-row block
+  auto item = [&](int k, bool& up, int& tt, int& mt) -> bool {
+    const int i = (int)blockIdx.x + k * (int)gridDim.x;
+    if (i >= total) return false;
+    up = i < n1;
+    const int r = up ? i : i - n1, m = up ? MT1 : MT2;
+    tt = r / m;
+    mt = r % m;
+    return true;
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    // A cursor (weights) and B cursor (tokens): item ordinal, stage within
+    // the item, and the stage sequence number (ring slot = seq % kStages).
+    bool a_up = false, b_up = false;
+    int a_tt = 0, a_mt = 0, b_tt = 0, b_mt = 0;
+    bool a_valid = item(0, a_up, a_tt, a_mt), b_valid = a_valid;
+    b_up = a_up;
+    b_tt = a_tt;
+    b_mt = a_mt;
+    int a_e = a_valid ? plan.at(a_tt, BN).e : -1;
+    TileEntry b_te = a_valid ? plan.at(b_tt, BN) : TileEntry{};
+    int ka = 0, kba = 0, seq_a = 0, kb_b = 0, kbb = 0, seq_b = 0;
+    bool b_ready = b_up;
+    uint32_t rdy = 0;  // bit i: the token operand of B item kb_b + i is ready
+    auto issue_a = [&]() {
+      const int st = seq_a % C::kStages;
+      if (tc::elect_one()) {
+        uint8_t* sp = smem + st * C::kStage;
+        const int R = a_up ? g1.R : g2.R, nc = a_up ? ncols1 : ncols2;
+        const uint8_t* sfa = (a_up ? g1.w_sf : g2.w_sf) + (size_t)a_e * R * nc + (size_t)a_mt * (nc / 4) * 512;
+        tc::mbar_expect_tx_only(&full[st], C::kA + C::kSFA);
+        tc::tma_load_2d(sp, a_up ? &tmap_w13 : &tmap_w2, &full[st], kba * 128, a_e * R + a_mt * 128);
+        tc::bulk_load(sp + C::kA + C::kB, sfa + (size_t)kba * F::kGroups * 512, C::kSFA, &full[st]);
+      }
+      __syncwarp();
+      ++seq_a;
+      if (++kba == (a_up ? nkb1 : nkb2)) {
+        kba = 0;
+        a_valid = item(++ka, a_up, a_tt, a_mt);
+        if (a_valid) a_e = plan.at(a_tt, BN).e;
+      }
+    };
+    // the ring's first pass needs no free slot: weights before the wait
+    if (g1.w_early != 0) {
+      while (a_valid && seq_a < C::kStages) issue_a();
+    }
+    pdl_wait();
+    pdl_trigger();
+    long long t_prog = clock64();
+    while (a_valid || b_valid) {
+      bool prog = false;
+      // token tiles: every stage whose weights are out and whose data is
+      // ready (a dependency poll at most once per pass)
+      while (b_valid && seq_b < seq_a) {
+        if (!b_ready) {
+          // one round trip polls this item's and the next 31 items' token tiles
+          bool up_i = true;
+          int tt_i = 0, mt_i = 0;
+          const bool has = item(kb_b + lane, up_i, tt_i, mt_i);
+          const int v = (has && !up_i) ? tc::ld_acquire_gpu(f.tile_done + tt_i) : done_target;
+          rdy |= __ballot_sync(0xffffffffu, v >= done_target);
+          if (!(rdy & 1u)) break;
+          tc::fence_proxy_async_global();   // for every token tile seen ready here
+          b_ready = true;
+        }
+        const int st = seq_b % C::kStages;
+        if (tc::elect_one()) {
+          uint8_t* sp = smem + st * C::kStage;
+          const int bi = token_box_index(min(b_te.nvalid, BN));
+          const uint32_t brows = min(16u << bi, (uint32_t)BN);
+          const int nc = b_up ? ncols1 : ncols2;
+          tc::mbar_expect_tx(&full[st], brows * 128u + F::kGroups * 512);
+          tc::tma_load_2d(sp + C::kA, b_up ? &tmaps_x.m[bi] : &tmaps_h.m[bi], &full[st], kbb * 128, b_te.row0);
+          const uint8_t* sfb =
+              (b_up ? g1.b_sf : g2.b_sf) + ((size_t)(b_te.row0 / 128) * (nc / 4) + (size_t)kbb * F::kGroups) * 512;
+          tc::bulk_load(sp + C::kA + C::kB + C::kSFA, sfb, F::kGroups * 512, &full[st]);
+        }
+        __syncwarp();
+        ++seq_b;
+        if (++kbb == (b_up ? nkb1 : nkb2)) {
+          kbb = 0;
+          b_valid = item(++kb_b, b_up, b_tt, b_mt);
+          if (b_valid) b_te = plan.at(b_tt, BN);
+          rdy >>= 1;
+          b_ready = b_up || (rdy & 1u);
+        }
+        prog = true;
+      }
+      // weight tiles: every free ring slot, at most a ring ahead of the tokens
+      while (a_valid && seq_a < seq_b + C::kStages) {
+        const int st = seq_a % C::kStages;
+        const uint32_t par = (((uint32_t)(seq_a / C::kStages)) & 1u) ^ 1u;
+        if (__shfl_sync(0xffffffffu, (int)tc::mbar_test_wait(&empty[st], par), 0) == 0) break;
+        issue_a();
+        prog = true;
+      }
+      if (prog) {
+        t_prog = clock64();
+      } else if (*abort || clock64() - t_prog > tc::kWaitCycles) {
+        // neither cursor could move for the wait bound (all polls above are non-blocking)
+        if (!*abort) {
+          if (lane == 0) raise_status(g1.status, MOE_ERR_TIMEOUT);
+          *abort = 1;
+        }
+        break;
+      }
+    }
+    // weight tiles issued for stages whose token tiles were not (an abort):
+    // arrive, so the barrier completes when they land, and wait for that
+    for (int q = seq_b; q < seq_a; ++q) {
+      const int st = q % C::kStages;
+      if (tc::elect_one()) tc::mbar_arrive(&full[st]);
+      __syncwarp();
+      tc::mbar_wait(&full[st], ((uint32_t)(q / C::kStages)) & 1u, abort);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    pdl_wait();
+    pdl_trigger();
+    int stage = 0;
+    uint32_t phase = 0;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    bool up = false;
+    int tt = 0, mt = 0;
+    for (int k = 0; item(k, up, tt, mt) && !*abort; ++k) {
+      const TileEntry te = plan.at(tt, BN);
+      if (!tc::mbar_wait(&tempty[acc], acc_phase ^ 1u, abort)) {
+        if (lane == 0) raise_status(g1.status, MOE_ERR_TIMEOUT);
+        *abort = 1;
+        break;
+      }
+      tc::fence_after_sync();
+      const uint32_t n_mma = (uint32_t)min(BN, (te.nvalid + 15) & ~15);
+      const uint32_t d = tmem + acc * BN;
+      const uint32_t sfb0 = tmem + C::kSfbCol + sfb_col_offset<BN>(te.row0);
+      const uint32_t idesc_nv = tc::idesc_mxf4(n_mma, false, 0, 0);
+      const int nkb = up ? nkb1 : nkb2;
+      bool ok = true;
+      for (int kb = 0; kb < nkb; ++kb) {
+        if (!tc::mbar_wait(&full[stage], phase, abort)) {
+          if (lane == 0) raise_status(g1.status, MOE_ERR_TIMEOUT);
+          *abort = 1;
+          ok = false;
+          break;
+        }
+        tc::fence_after_sync();
+        if (tc::elect_one()) {
+          uint8_t* st = smem + stage * C::kStage;
+          const uint64_t dsfa = tc::desc_sf(tc::smem_u32(st + C::kA + C::kB));
+          const uint64_t dsfb = dsfa + (uint64_t)(C::kSFA >> 4);
+#pragma unroll
+          for (int grp = 0; grp < F::kGroups; ++grp) {
+            tc::sf_copy(tmem + C::kSfaCol + 4 * grp, dsfa + (uint64_t)(grp * 32));
+            tc::sf_copy(tmem + C::kSfbCol + grp * 4, dsfb + (uint64_t)(grp * 32));
+          }
+          const uint64_t da0 = tc::desc_sw128(tc::smem_u32(st)), db0 = tc::desc_sw128(tc::smem_u32(st + C::kA));
+#pragma unroll
+          for (int kk = 0; kk < F::kSteps; ++kk) {
+            const uint64_t da = da0 + (uint64_t)(kk * 2), db = db0 + (uint64_t)(kk * 2);
+            const uint32_t accum = (kb > 0 || kk > 0) ? 1u : 0u;
+            if (FMT == MOE_FMT_NVFP4) {
+              tc::mma_nvf4(d, da, db, idesc_nv, tmem + C::kSfaCol + 4 * kk, sfb0 + kk * 4, accum);
+            } else {
+              const uint32_t id = (uint32_t)(kk & 1) * 2;
+              tc::mma_mxf4(d, da, db, tc::idesc_mxf4(n_mma, true, id, id), tmem + C::kSfaCol + 4 * (kk >> 1),
+                           sfb0 + (kk >> 1) * 4, accum);
+            }
+          }
+          tc::mma_commit(&empty[stage]);
+        }
+        __syncwarp();
+        if (++stage == C::kStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (!ok) break;
+      if (tc::elect_one()) tc::mma_commit(&tfull[acc]);
+      __syncwarp();
+      if (++acc == C::kAccStages) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    pdl_wait();
+    pdl_trigger();
+    const int ew = warp - 2;
+    const int q = warp & 3;
+    const int cw = ew / 4;
+    const float gact1 = act_scale_of(FMT, g1.act_scale, g1.act_amax);
+    const float gh = FMT == MOE_FMT_NVFP4 ? act_scale_of(FMT, g1.h_scale, nullptr) : 1.0f;
+    const float gact2 = act_scale_of(FMT, g2.act_scale, g2.act_amax);
+    if constexpr (FMT == MOE_FMT_NVFP4) {
+      for (int c = ew * 32 + lane; c < 128; c += C::kEpiWarps * 32) r_tab[c] = nvfp4_multiplier((uint32_t)c, gh);
+      asm volatile("bar.sync 15, %0;" ::"r"(C::kEpiWarps * 32) : "memory");
+    }
+    float hmax = 0.0f;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    bool up = false;
+    int tt = 0, mt = 0;
+    for (int k = 0; item(k, up, tt, mt); ++k) {
+      const TileEntry te = plan.at(tt, BN);
+      if (!tc::mbar_wait(&tfull[acc], acc_phase, abort)) {
+        if (lane == 0) raise_status(g1.status, MOE_ERR_TIMEOUT);
+        *abort = 1;
+        break;
+      }
+      tc::fence_after_sync();
+      const int ncol = min(BN, (te.nvalid + 15) & ~15);
+      const int c_lo = cw * 64;
+      const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN) + (uint32_t)c_lo;
+      uint32_t r0[16], r1[16], r2[16], r3[16];
+      const int nch = c_lo < ncol ? min(4, (ncol - c_lo + 15) >> 4) : 0;
+      if (nch > 0) {
+        tc::tmem_ld16_async(tbase, r0);
+        if (nch > 1) tc::tmem_ld16_async(tbase + 16, r1);
+        if (nch > 2) tc::tmem_ld16_async(tbase + 32, r2);
+        if (nch > 3) tc::tmem_ld16_async(tbase + 48, r3);
+        tc::tmem_wait16(r0);
+        if (nch > 1) tc::tmem_wait16(r1);
+        if (nch > 2) tc::tmem_wait16(r2);
+        if (nch > 3) tc::tmem_wait16(r3);
+      }
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&tempty[acc]);
+      if (++acc == C::kAccStages) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+      if (up) {
+        if (c_lo < ncol)
+          epilogue_slice<FMT, kEpiUpQuant, BN>(g1, &tmap_y, te, mt, 0, nch, c_lo, ew, q, lane, gact1, gh, epi_tiles,
+                                               r_tab, y_stage, hmax, r0, r1, r2, r3);
+        // this warp's slice of h is stored: count it for the down tiles
+        tc::fence_proxy_async_global();
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) atomicAdd(f.tile_done + tt, 1);
+      } else if (c_lo < ncol) {
+        epilogue_slice<FMT, kEpiDown, BN>(g2, &tmap_y, te, mt, 0, nch, c_lo, ew, q, lane, gact2, 1.0f, epi_tiles,
+                                          r_tab, y_stage, hmax, r0, r1, r2, r3);
+      }
+    }
+    if (lane == 0) tc::bulk_wait_all();   // tensor stores done before the CTA exits
+  }
+
+  __syncwarp();
+  __syncthreads();
+  if (*abort) {
+    // let copies and MMAs already in flight land before the memory goes away
+    const long long t0 = clock64();
+    while (clock64() - t0 < 2000000LL) {
+    }
+  }
+  tc::fence_after_sync();
+  if (warp == 1) tc::tmem_dealloc(tmem, C::kTmemCols);
 }
 
 // ------------------------------------------------------------- tensor maps --
@@ -721,6 +1244,30 @@ cudaError_t launch_epi(const GemmArgs& g, int epi, int bn, const void* a, int64_
   return launch_bn<FMT, kEpiUpQuant>(g, bn, a, ar, b, br, sms, s);
 }
 
+template <int FMT, int BN>
+cudaError_t launch_fused_cfg(const GemmArgs& g1, const GemmArgs& g2, const FusedArgs& f, const void* w13,
+                             int64_t w13_rows, const void* w2, int64_t w2_rows, const void* xq, const void* hq,
+                             int num_sms, cudaStream_t s) {
+  using C = Cfg<FMT, kEpiUpQuant, BN, false>;
+  CUtensorMap m13, m2, my;
+  TokenMaps mx, mh;
+  if (g2.y_rows < 1 || !make_y_map(&my, g2.y, g2.y_rows, g2.ldy)) return cudaErrorInvalidValue;
+  if (!make_map(&m13, w13, w13_rows, g1.K / 2, 128)) return cudaErrorInvalidValue;
+  if (!make_map(&m2, w2, w2_rows, g2.K / 2, 128)) return cudaErrorInvalidValue;
+  for (int i = 0; i < 5; ++i) {
+    const int rows = (16 << i) < BN ? (16 << i) : BN;
+    if (!make_map(&mx.m[i], xq, f.P, g1.K / 2, rows)) return cudaErrorInvalidValue;
+    if (!make_map(&mh.m[i], hq, f.P, g2.K / 2, rows)) return cudaErrorInvalidValue;
+  }
+  auto kern = fused_ffn_kernel<FMT, BN>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, FusedCfg<FMT, BN>::kSmem);
+  if (e != cudaSuccess) return e;
+  e = launch_pdl(kern, dim3(num_sms), dim3(C::kThreads), FusedCfg<FMT, BN>::kSmem, s, m13, mx, m2, mh, my, g1, g2, f);
+  if (e != cudaSuccess) return e;
+  count_launches(1);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_grouped_gemm(const GemmArgs& g, int epi, int bn, const void* a_base, int64_t a_rows,
@@ -733,9 +1280,26 @@ cudaError_t launch_grouped_gemm(const GemmArgs& g, int epi, int bn, const void* 
   }
 }
 
+cudaError_t launch_fused_ffn(const GemmArgs& g1, const GemmArgs& g2, const FusedArgs& f, const void* w13,
+                             int64_t w13_rows, const void* w2, int64_t w2_rows, const void* xq, const void* hq,
+                             int num_sms, cudaStream_t s) {
+  if (g1.E > kFusedMaxE || g1.fmt != g2.fmt) return cudaErrorInvalidValue;
+  switch (g1.fmt) {
+    case MOE_FMT_NVFP4:
+      return launch_fused_cfg<MOE_FMT_NVFP4, 64>(g1, g2, f, w13, w13_rows, w2, w2_rows, xq, hq, num_sms, s);
+    case MOE_FMT_MXFP4:
+      return launch_fused_cfg<MOE_FMT_MXFP4, 64>(g1, g2, f, w13, w13_rows, w2, w2_rows, xq, hq, num_sms, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
 bool tensor_maps_available() { return encode_fn() != nullptr; }
 
 void set_gemm_pairs(bool on) { g_gemm_pairs = on; }
+
+static int g_early_weights = 1;  // MOE_OPT_EARLY_WEIGHTS
+void set_early_weights(int mode) { g_early_weights = mode; }
+int early_weights() { return g_early_weights; }
 
 
 int router_ksplit(int64_t T, int E, int H, int num_sms) {
@@ -839,25 +1403,34 @@ cudaError_t launch_plan(const int32_t* offsets, int E, int64_t S, int bn, int32_
 __device__ void plan_in_block(const int32_t* __restrict__ offsets, int E, int64_t S, const PlanOut& plan, bool write,
                               int32_t* s_poff, int32_t* status) {
   __shared__ int32_t warp_tot[8];
-  __shared__ int bad;
   const int per = (E + 255) / 256;
   const int e0 = threadIdx.x * per;
-  if (threadIdx.x == 0) bad = (__ldg(offsets) != 0 || __ldg(offsets + E) != S) ? 1 : 0;
-  __syncthreads();
+  // every offset is read once, all reads in flight together; the checks
+  // (offsets[0] == 0, non-decreasing, offsets[E] == S) are or-reduced at the
+  // first barrier of the scans
+  int mybad = 0;
   int32_t pad_mine = 0, til_mine = 0;
-  for (int e = e0; e < e0 + per && e < E; ++e) {
-    int32_t n = __ldg(offsets + e + 1) - __ldg(offsets + e);
-    if (n < 0) {
-      bad = 1;
-      n = 0;
+  if (e0 < E) {
+    int32_t prev = __ldg(offsets + e0);
+    if (e0 == 0 && prev != 0) mybad = 1;
+    for (int e = e0; e < e0 + per && e < E; ++e) {
+      const int32_t hi = __ldg(offsets + e + 1);
+      int32_t n = hi - prev;
+      prev = hi;
+      if (n < 0) {
+        mybad = 1;
+        n = 0;
+      }
+      if (e + 1 == E && hi != S) mybad = 1;
+      pad_mine += (n + 127) / 128 * 128;
+      til_mine += (n + plan.bn - 1) / plan.bn;
     }
-    pad_mine += (n + 127) / 128 * 128;
-    til_mine += (n + plan.bn - 1) / plan.bn;
   }
   // two exclusive scans over the 256 threads
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int32_t res[2], tot[2];
   const int32_t val[2] = {pad_mine, til_mine};
+  int bad = 0;
 #pragma unroll
   for (int q = 0; q < 2; ++q) {
     int32_t incl = val[q];
@@ -866,7 +1439,8 @@ __device__ void plan_in_block(const int32_t* __restrict__ offsets, int E, int64_
       const int32_t n = __shfl_up_sync(0xffffffffu, incl, o);
       if (lane >= o) incl += n;
     }
-    __syncthreads();
+    if (q == 0) bad = __syncthreads_or(mybad);
+    else __syncthreads();
     if (lane == 31) warp_tot[warp] = incl;
     __syncthreads();
     int32_t base = 0, sum = 0;
@@ -918,6 +1492,8 @@ template <int FMT, bool SRC_X>
 __global__ void __launch_bounds__(256) quant_padded_kernel(QuantPaddedArgs a) {
   pdl_wait();  // inputs come from the previous kernels
   pdl_trigger();
+  if (a.zero && blockIdx.x == 0)
+    for (int i = threadIdx.x; i < a.nzero; i += blockDim.x) a.zero[i] = 0;
 
   constexpr int bs = FMT == MOE_FMT_MXFP4 ? 32 : 16;
   const int nb = a.K / bs;
@@ -929,11 +1505,15 @@ __global__ void __launch_bounds__(256) quant_padded_kernel(QuantPaddedArgs a) {
   // tile plan needs no launch of its own.
   __shared__ int32_t s_poff[1025];
   const int32_t* poff = a.poff;
+  const int64_t p_first = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  // the first slot's token is read before the plan, in flight with its offsets
+  int t_first = -1;
+  if (SRC_X && lane == 0 && p_first < a.S) t_first = __ldg(a.perm_token + p_first);
   if (SRC_X && a.plan.bn > 0) {
     plan_in_block(a.offsets, a.E, a.S, a.plan, blockIdx.x == 0, s_poff, a.status);
     poff = s_poff;
   }
-  for (int64_t p = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); p < a.S; p += warps) {
+  for (int64_t p = p_first; p < a.S; p += warps) {
     int64_t row = -1;
     int t = -1;
     if (lane == 0) {
@@ -942,7 +1522,7 @@ __global__ void __launch_bounds__(256) quant_padded_kernel(QuantPaddedArgs a) {
       row = (int64_t)poff[e] + (p - o);
       if (row < 0 || row >= a.P || p < o) row = -1;
       if (SRC_X) {
-        t = __ldg(a.perm_token + p);
+        t = p == p_first ? t_first : __ldg(a.perm_token + p);
         if (t < 0 || t >= a.T) row = -1;
       }
     }
@@ -1020,6 +1600,8 @@ template <int FMT>
 __global__ void __launch_bounds__(256) quant_tokens_kernel(QuantPaddedArgs a) {
   pdl_wait();  // inputs come from the previous kernels
   pdl_trigger();
+  if (a.zero && blockIdx.x == 0)
+    for (int i = threadIdx.x; i < a.nzero; i += blockDim.x) a.zero[i] = 0;
 
   constexpr int bs = FMT == MOE_FMT_MXFP4 ? 32 : 16;
   constexpr int kPer = 64;

@@ -43,6 +43,16 @@ struct GemmArgs {
   int ksplit;                  // router: K split over this many partial outputs,
   int64_t split_stride;        //         split s at logits + s * split_stride
   int64_t dense_rows;          // > 0: token tiles are plain row blocks (no tile list)
+  // Early weight loads (programmatic launch): before waiting for the previous
+  // kernel, the producer issues the weight tiles of its first stages.  Their
+  // experts come from the tile list (1: written at least two kernels back,
+  // so complete once this kernel runs) or from `offsets` (2: the tile list
+  // is the previous kernel's output; offsets are older; E <= 256, else no
+  // early loads).  0: off.
+  int w_early;
+  int w_early_l2;              // and this many further stages' weights prefetched to L2
+  const int32_t* offsets;      // [E+1] compact expert offsets (w_early == 2; E <= 256)
+  int max_tiles;               // entries allocated in `tiles`
   int32_t* status;
 };
 
@@ -57,6 +67,8 @@ struct QuantPaddedArgs {
   int k;                       //   token is quantised once and written to its k slots
   const int32_t* slot_expert;  //   optional with it: expert of each (token, j) (top-k indices)
   PlanOut plan;                // per-slot x quantiser: also compute (and write) the tile plan
+  int32_t* zero;               // optional: nzero counters set to 0 (by block 0, after the wait)
+  int nzero;
   const uint16_t* x;           // [T][K] bf16
   const float* h32;            // or fp32 rows at padded positions
   const float* scale;          // static tensor scale or NULL
@@ -66,12 +78,33 @@ struct QuantPaddedArgs {
   int32_t* status;
 };
 
+// The expert FFN as one persistent kernel (gate|up + SwiGLU + h quantisation,
+// then down), for 64-token tiles: each CTA runs its gate|up tiles, then its
+// down tiles; a down tile's token operand waits for the gate|up slices of its
+// token tile, counted in tile_done.  The tile list comes from the offsets.
+struct FusedArgs {
+  const int32_t* offsets;      // [E+1] compact (E <= 256)
+  int64_t S;                   // slots: offsets[E]
+  int64_t P;                   // padded rows allocated for x and h
+  int32_t* tile_done;          // [max_tiles], zero on entry
+  int max_tiles;
+};
+constexpr int kFusedMaxE = 256;
+cudaError_t launch_fused_ffn(const GemmArgs& g1, const GemmArgs& g2, const FusedArgs& f, const void* w13,
+                             int64_t w13_rows, const void* w2, int64_t w2_rows, const void* xq, const void* hq,
+                             int num_sms, cudaStream_t s);
+
 cudaError_t launch_plan(const int32_t* offsets, int E, int64_t S, int bn, int32_t* poff, TileEntry* tiles,
                         int32_t* num_tiles, int max_tiles, int32_t* status, cudaStream_t s);
 cudaError_t launch_quant_padded(const QuantPaddedArgs& a, bool src_x, int fmt, int num_sms, cudaStream_t s);
 cudaError_t launch_grouped_gemm(const GemmArgs& g, int epi, int bn, const void* a_base, int64_t a_rows,
                                 const void* b_base, int64_t b_rows, int num_sms, cudaStream_t s);
 bool tensor_maps_available();
+// Early weight loads (MOE_OPT_EARLY_WEIGHTS): 0 off, 1 the ring's first pass,
+// 2 also prefetch the next stages' weights to L2.
+void set_early_weights(int mode);
+int early_weights();
+constexpr int kEarlyL2Stages = 16;
 // CTA pairs (cta_group::2) for 256-token tiles whose weight rows divide by 256.
 void set_gemm_pairs(bool on);
 // Router logits on the tensor cores, K split over ksplit partial outputs

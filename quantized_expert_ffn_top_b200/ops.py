@@ -24,6 +24,8 @@ OPT_FFN_PATH = 1
 OPT_GEMM_TILE_N = 2
 OPT_GEMM_PAIR = 3
 OPT_PDL = 4
+OPT_EARLY_WEIGHTS = 5
+OPT_FUSED_FFN = 6
 FMT_BY_NAME = {"nvfp4": FMT_NVFP4, "mxfp4": FMT_MXFP4, "fp8": FMT_FP8}
 
 EXPORTED = (

@@ -89,5 +89,12 @@ def test_host_side_argument_errors(L):
     # CTA pairs on or off
     assert L.moe_set_option(3, 2) == 1
     assert L.moe_set_option(3, 0) == 0 and L.moe_set_option(3, 1) == 0
+    # early weight loads: 0, 1 or 2
+    assert L.moe_set_option(5, 3) == 1 and L.moe_set_option(5, -1) == 1
+    for v in (0, 2, 1):
+        assert L.moe_set_option(5, v) == 0
+    # fused FFN on or off
+    assert L.moe_set_option(6, 2) == 1
+    assert L.moe_set_option(6, 0) == 0 and L.moe_set_option(6, 1) == 0
     # combine: k beyond the 1024 the kernel stages
     assert L.moe_combine(one, one, one, 1, 1025, 8, None, one, one, 1 << 20, None) == 1

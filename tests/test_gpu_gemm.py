@@ -73,6 +73,46 @@ def test_gemm_path_matches_oracle(name, over, static, skew, tile_n, pair):
             assert max_abs_rel(y[a:b], ry[a:b]) < 5 * TOL, e
 
 
+@pytest.mark.parametrize("tile_n", [64, 192])
+@pytest.mark.parametrize("name,over,static,skew", [GEMM_CASES[0], GEMM_CASES[3], GEMM_CASES[5]])
+def test_early_weight_loads_change_nothing(name, over, static, skew, tile_n):
+    """Weight tiles loaded before the wait on the previous kernel (the expert
+    named by the offsets, or by the tile list) or prefetched to L2 give the
+    same bits as loading every stage after it."""
+    ops.moe_set_option(ops.OPT_GEMM_TILE_N, tile_n)
+    ys = []
+    try:
+        for mode in (0, 1, 2):
+            ops.moe_set_option(ops.OPT_EARLY_WEIGHTS, mode)
+            *_, y, st = _run(over, static, skew, 2)
+            assert st == 0, mode
+            ys.append(y)
+    finally:
+        ops.moe_set_option(ops.OPT_EARLY_WEIGHTS, 1)
+        ops.moe_set_option(ops.OPT_GEMM_TILE_N, 0)
+    assert np.array_equal(ys[0], ys[1]) and np.array_equal(ys[0], ys[2])
+
+
+@pytest.mark.parametrize("name,over,static,skew", [GEMM_CASES[0], GEMM_CASES[2], GEMM_CASES[4], GEMM_CASES[5]])
+def test_fused_ffn_kernel_matches_two_kernels(name, over, static, skew):
+    """64-token tiles: the one-kernel FFN (down tiles waiting on their token
+    tile's gate|up slices) gives the bits of the two separate projections."""
+    ops.moe_set_option(ops.OPT_GEMM_TILE_N, 64)
+    ys = []
+    try:
+        for fused in (0, 1):
+            ops.moe_set_option(ops.OPT_FUSED_FFN, fused)
+            w, W, x, perm, off, a13, a2, y, st = _run(over, static, skew, 2)
+            assert st == 0, fused
+            ys.append(y)
+    finally:
+        ops.moe_set_option(ops.OPT_FUSED_FFN, 1)
+        ops.moe_set_option(ops.OPT_GEMM_TILE_N, 0)
+    assert np.array_equal(ys[0], ys[1])
+    ry, _ = oracle.grouped_ffn(x, perm, off, W, 1, a13 or 0.0, a2 or 0.0)
+    assert max_abs_rel(ys[1], ry) < TOL
+
+
 @pytest.mark.parametrize("name,over,static,skew", GEMM_CASES[:4])
 def test_gemm_and_gemv_paths_agree(name, over, static, skew):
     *_, yg, st1 = _run(over, static, skew, 2)
