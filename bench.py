@@ -544,7 +544,9 @@ def main():
                           "expert_weight_bytes": ad["wbytes_up"] + ad["wbytes_down"],
                           "active_experts": ad["active_experts"], "ffn_ms": ffn_ms,
                           "ffn_timing": "moe_grouped_ffn alone, graph replay, L2 flushed", "weight_gbs": gbs,
-                          "traffic": (lambda u, d: u + d if u is not None and d is not None else None)(
+                          # one fused kernel at this batch size; two launches otherwise
+                          "traffic": measured_traffic("ffn", "decode") or (
+                              lambda u, d: u + d if u is not None and d is not None else None)(
                               measured_traffic("ffn_up", "decode"), measured_traffic("ffn_down", "decode")),
                           "hbm_frac": gbs / pk["hbm_gbs"] if gbs else None, "stages_ms": rd["stages"]}
         del dl
