@@ -317,7 +317,7 @@ moe_status run_gemm_ffn(const uint16_t* x, int64_t T, int64_t S, const int32_t* 
   qa.codes = f.xq;
   qa.sf = f.xsf;
   qa.status = status;
-  qa.zero = one_kernel ? f.tile_done : nullptr;   // the fused kernel's counters
+  qa.zero = one_kernel ? f.tile_done : nullptr;   // the one-kernel FFN's counters
   qa.nzero = one_kernel ? (int)max_tiles(S, E) : 0;
   MOE_TRY(launch_quant_padded(qa, true, fmt, sms, s));
   if (mark) stage_mark(MOE_STAGE_ACT_QUANT, true, s);
@@ -372,8 +372,8 @@ moe_status run_gemm_ffn(const uint16_t* x, int64_t T, int64_t S, const int32_t* 
   d.w_early_l2 = g.w_early_l2;
   d.max_tiles = g.max_tiles;
   if (one_kernel) {
-    // the weights are older than the quantiser: the ring's first pass loads
-    // before the wait (the tile list comes from the offsets in the kernel)
+    // the weights are older than the quantiser: the first stages load before
+    // the wait (the tile list comes from the offsets in the kernel)
     g.w_early = ew == 0 ? 0 : 1;
     FusedArgs fa;
     fa.offsets = offsets;

@@ -170,6 +170,19 @@ struct WarpPlan {
     const int prows = __shfl_sync(0xffffffffu, pi, 31);
     ok = __all_sync(0xffffffffu, good) && ntiles <= max_tiles && (int64_t)prows <= P;
   }
+  // Padded row of slot p (0 <= p < offsets[E]), -1 if no expert holds it: whole warp.
+  __device__ __forceinline__ int64_t row_of_slot(int p) const {
+    int pr = pbase, prev = lo0, row = -1;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int n = max(hi[j] - prev, 0);
+      if (row < 0 && p >= prev && p < prev + n) row = pr + (p - prev);
+      pr += (n + 127) / 128 * 128;
+      prev = hi[j];
+    }
+    const unsigned m = __ballot_sync(0xffffffffu, row >= 0);
+    return m ? (int64_t)__shfl_sync(0xffffffffu, row, __ffs(m) - 1) : -1;
+  }
   // Entry tt (< ntiles): whole warp.
   __device__ __forceinline__ TileEntry at(int tt, int bn) const {
     const int lane = threadIdx.x & 31;
@@ -200,6 +213,59 @@ struct WarpPlan {
     return r;
   }
 };
+
+// Quantises scale block b (bs values v) of padded row `row` and stores its
+// codes and its scale (blocked layout, nb blocks per row of K values).
+template <int FMT>
+__device__ __forceinline__ void quant_block_store(const float* v, float scale, uint8_t* codes, uint8_t* sf,
+                                                  int64_t row, int b, int nb, int K) {
+  constexpr int bs = FMT == MOE_FMT_MXFP4 ? 32 : 16;
+  float bmax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < bs; ++i) bmax = fmaxf(bmax, fabsf(v[i]));
+  if constexpr (FMT == MOE_FMT_NVFP4) {
+    uint32_t sc;
+    float r;
+    nvfp4_block_scale(bmax, scale, sc, r);
+    *reinterpret_cast<uint2*>(codes + row * (K / 2) + b * 8) = nvfp4_encode16(v, r);
+    sf[sf_blocked_offset(row, b, nb)] = (uint8_t)sc;
+  } else if constexpr (FMT == MOE_FMT_MXFP4) {
+    uint32_t c;
+    float inv;
+    mxfp4_block_scale(bmax, c, inv);
+    uint4 w;
+    w.x = e2m1_encode8(v, inv);
+    w.y = e2m1_encode8(v + 8, inv);
+    w.z = e2m1_encode8(v + 16, inv);
+    w.w = e2m1_encode8(v + 24, inv);
+    *reinterpret_cast<uint4*>(codes + row * (K / 2) + b * 16) = w;
+    sf[sf_blocked_offset(row, b, nb)] = (uint8_t)c;
+  } else {
+    const float inv = __frcp_rn(scale);
+    uint4 w;
+    uint32_t* pw = &w.x;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      pw[i] = e4m3x2_encode(__fmul_rn(v[4 * i], inv), __fmul_rn(v[4 * i + 1], inv)) |
+              (e4m3x2_encode(__fmul_rn(v[4 * i + 2], inv), __fmul_rn(v[4 * i + 3], inv)) << 16);
+    *reinterpret_cast<uint4*>(codes + row * K + b * 16) = w;
+  }
+}
+
+// bs bf16 values at src as floats
+template <int bs>
+__device__ __forceinline__ void load_bf16_block(const uint16_t* src, float* v) {
+#pragma unroll
+  for (int i = 0; i < bs; i += 8) {
+    const uint4 w = __ldg(reinterpret_cast<const uint4*>(src + i));
+    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      v[i + 2 * j] = __uint_as_float(ww[j] << 16);
+      v[i + 2 * j + 1] = __uint_as_float(ww[j] & 0xFFFF0000u);
+    }
+  }
+}
 
 // Converts and stores an epilogue warp's slice of one tile: nch 16-column
 // chunks of its 64 accumulator columns (from c_lo), in r0..r3.
@@ -858,7 +924,7 @@ __global__ void __launch_bounds__(Cfg<FMT, kEpiUpQuant, BN, false>::kThreads, 1)
     int a_e = a_valid ? plan.at(a_tt, BN).e : -1;
     TileEntry b_te = a_valid ? plan.at(b_tt, BN) : TileEntry{};
     int ka = 0, kba = 0, seq_a = 0, kb_b = 0, kbb = 0, seq_b = 0;
-    bool b_ready = b_up;
+    bool b_ready = b_up;   // gate|up token tiles come from the x quantiser before this kernel
     uint32_t rdy = 0;  // bit i: the token operand of B item kb_b + i is ready
     auto issue_a = [&]() {
       const int st = seq_a % C::kStages;
@@ -878,9 +944,13 @@ __global__ void __launch_bounds__(Cfg<FMT, kEpiUpQuant, BN, false>::kThreads, 1)
         if (a_valid) a_e = plan.at(a_tt, BN).e;
       }
     };
-    // the ring's first pass needs no free slot: weights before the wait
+    // Before the wait on the previous kernel (the x quantiser), at most
+    // kPreStages weight stages per CTA are put in flight (the ring's first
+    // pass needs no free slot): a deeper burst queues that kernel's own reads
+    // behind it.
+    constexpr int kPreStages = 3 < C::kStages ? 3 : C::kStages;
     if (g1.w_early != 0) {
-      while (a_valid && seq_a < C::kStages) issue_a();
+      while (a_valid && seq_a < kPreStages) issue_a();
     }
     pdl_wait();
     pdl_trigger();
@@ -920,7 +990,7 @@ __global__ void __launch_bounds__(Cfg<FMT, kEpiUpQuant, BN, false>::kThreads, 1)
           b_valid = item(++kb_b, b_up, b_tt, b_mt);
           if (b_valid) b_te = plan.at(b_tt, BN);
           rdy >>= 1;
-          b_ready = b_up || (rdy & 1u);
+          b_ready = b_up || (rdy & 1u) != 0;
         }
         prog = true;
       }
@@ -1535,17 +1605,7 @@ __global__ void __launch_bounds__(256) quant_padded_kernel(QuantPaddedArgs a) {
     for (int b = lane; b < nb; b += 32) {
       float v[bs];
       if (SRC_X) {
-        const uint16_t* src = a.x + (int64_t)t * a.K + b * bs;
-#pragma unroll
-        for (int i = 0; i < bs; i += 8) {
-          const uint4 w = __ldg(reinterpret_cast<const uint4*>(src + i));
-          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            v[i + 2 * j] = __uint_as_float(ww[j] << 16);
-            v[i + 2 * j + 1] = __uint_as_float(ww[j] & 0xFFFF0000u);
-          }
-        }
+        load_bf16_block<bs>(a.x + (int64_t)t * a.K + b * bs, v);
       } else {
         const float* src = a.h32 + row * a.K + b * bs;
 #pragma unroll
@@ -1557,36 +1617,7 @@ __global__ void __launch_bounds__(256) quant_padded_kernel(QuantPaddedArgs a) {
           v[i + 3] = w.w;
         }
       }
-      float bmax = 0.0f;
-#pragma unroll
-      for (int i = 0; i < bs; ++i) bmax = fmaxf(bmax, fabsf(v[i]));
-      if constexpr (FMT == MOE_FMT_NVFP4) {
-        uint32_t sc;
-        float r;
-        nvfp4_block_scale(bmax, scale, sc, r);
-        *reinterpret_cast<uint2*>(a.codes + row * (a.K / 2) + b * 8) = nvfp4_encode16(v, r);
-        a.sf[sf_blocked_offset(row, b, nb)] = (uint8_t)sc;
-      } else if constexpr (FMT == MOE_FMT_MXFP4) {
-        uint32_t c;
-        float inv;
-        mxfp4_block_scale(bmax, c, inv);
-        uint4 w;
-        w.x = e2m1_encode8(v, inv);
-        w.y = e2m1_encode8(v + 8, inv);
-        w.z = e2m1_encode8(v + 16, inv);
-        w.w = e2m1_encode8(v + 24, inv);
-        *reinterpret_cast<uint4*>(a.codes + row * (a.K / 2) + b * 16) = w;
-        a.sf[sf_blocked_offset(row, b, nb)] = (uint8_t)c;
-      } else {
-        const float inv = __frcp_rn(scale);
-        uint4 w;
-        uint32_t* pw = &w.x;
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          pw[i] = e4m3x2_encode(__fmul_rn(v[4 * i], inv), __fmul_rn(v[4 * i + 1], inv)) |
-                  (e4m3x2_encode(__fmul_rn(v[4 * i + 2], inv), __fmul_rn(v[4 * i + 3], inv)) << 16);
-        *reinterpret_cast<uint4*>(a.codes + row * a.K + b * 16) = w;
-      }
+      quant_block_store<FMT>(v, scale, a.codes, a.sf, row, b, nb, a.K);
     }
   }
 }
