@@ -244,13 +244,14 @@ moe_status moe_get_device_status(void* ws, moe_stream_t stream, int32_t* host_st
  *                     MOE_ERR_UNSUPPORTED where the shapes do not allow it).
  * Not thread-safe; set before enqueuing. */
 /*   MOE_OPT_GEMM_TILE_N: token-tile width of the tensor-core path: 0 (default:
- *                     64 while T*k < 8E, 192 while T*k <= 384E, else 256),
- *                     64 (four accumulators), 128 or 192 (two) or 256 (one,
- *                     drained to registers).
- *   MOE_OPT_GEMM_PAIR: 1 runs 256-token tiles on CTA pairs (tcgen05
- *                     cta_group::2, 256 weight rows per tile) when the weight
- *                     rows per expert divide by 256; 0 (default) keeps one
- *                     CTA per 128-row tile.
+ *                     64 while T*k < 8E, else 192), 64 (four accumulators),
+ *                     128 or 192 (two) or 256 (one, drained to registers).
+ *   MOE_OPT_GEMM_PAIR: CTA pairs (tcgen05 cta_group::2, 256 weight rows per
+ *                     tile, each CTA staging half of the token tile) for 192-
+ *                     and 256-token tiles when the weight rows per expert
+ *                     divide by 256: 0 never, 1 always, 2 (default) only for a
+ *                     projection whose K loop has at least 12 stages (K >=
+ *                     3072 for NVFP4 / MXFP4, 1536 for FP8).
  *   MOE_OPT_PDL:       1 (default) launches the layer's kernels with
  *                     programmatic dependent launch, so each one's setup
  *                     overlaps the previous kernel's tail; 0 launches them

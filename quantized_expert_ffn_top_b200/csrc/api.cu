@@ -268,8 +268,7 @@ bool use_gemm_path(const moe_weights* w, int64_t S, int act) {
 // dominate.  Arguments only, no device read-back.
 int gemm_tile_n(int64_t S, int E) {
   if (g_gemm_bn) return g_gemm_bn;
-  if (S < 8 * (int64_t)E) return 64;
-  return S <= 384 * (int64_t)E ? 192 : 256;
+  return S < 8 * (int64_t)E ? 64 : 192;
 }
 
 moe_status run_gemm_ffn(const uint16_t* x, int64_t T, int64_t S, const int32_t* perm, const int32_t* offsets,
@@ -576,8 +575,8 @@ moe_status moe_set_option(int32_t option, int32_t value) {
     return MOE_OK;
   }
   if (option == MOE_OPT_GEMM_PAIR) {
-    if (value != 0 && value != 1) return MOE_ERR_INVALID_ARG;
-    set_gemm_pairs(value != 0);
+    if (value < 0 || value > 2) return MOE_ERR_INVALID_ARG;
+    set_gemm_pairs(value);
     return MOE_OK;
   }
   return MOE_ERR_INVALID_ARG;

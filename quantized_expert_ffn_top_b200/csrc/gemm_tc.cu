@@ -55,13 +55,13 @@ struct FmtTraits {
   static constexpr int kGroups = kBs ? kBK / (4 * kBs) : 0;         // 4-column scale groups per stage
 };
 
-// PAIR: a tile is 256 weight rows x BN tokens computed by a cluster of two
+// PAIR: a tile is 256 weight rows x BN (192 or 256) tokens computed by a cluster of two
 // CTAs (cta_group::2): each CTA stages its 128 weight rows, half of the token
 // rows and all BN tokens' scales, and owns its 128 rows of the accumulator.
 template <int FMT, int EPI, int BN, bool PAIR = false>
 struct Cfg {
   static_assert(BN == 64 || BN == 128 || BN == 192 || BN == 256, "token tile width");
-  static_assert(!PAIR || BN == 256, "CTA pairs run 256-token tiles");
+  static_assert(!PAIR || BN == 256 || BN == 192, "CTA pairs run 192- or 256-token tiles");
   using F = FmtTraits<FMT>;
   // Scale blocks cover 128 token rows; a tile starts on a multiple of 64
   // rows, so a 192-wide tile may start half way into its first block and
@@ -573,8 +573,8 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN, PAIR>::kThreads, 1)
           uint8_t* st = smem + stage * C::kStage;
           const int nh = min(BN, (te.nvalid + 31) & ~31) >> 1;      // token rows per CTA
           const int bi = token_box_index(nh);
-          const uint32_t brows = min(16u << bi, (uint32_t)BN);   // the map's box height
-          const int nblk = (min(te.nvalid, BN) + 127) / 128;
+          const uint32_t brows = min(16u << bi, (uint32_t)(BN / 2));   // the map's box height
+          const int nblk = ((te.row0 & 127) + min(te.nvalid, BN) + 127) / 128;   // 128-row scale blocks in use
           const uint32_t cbar = tc::cluster_addr(&full[stage], 0);
           if (rank == 0)
             tc::mbar_expect_tx(&full[stage], 2u * (C::kA + brows * 128u + C::kSFA + nblk * F::kGroups * 512));
@@ -1226,7 +1226,12 @@ bool make_y_map(CUtensorMap* m, void* base, int64_t rows, int64_t ld) {
          CUDA_SUCCESS;
 }
 
-bool g_gemm_pairs = false;  // CTA pairs for 256-token tiles (MOE_OPT_GEMM_PAIR)
+// CTA pairs (MOE_OPT_GEMM_PAIR): 0 never, 1 wherever the tile allows, 2 where
+// a tile's K loop has at least kPairMinStages stages -- shorter loops lose
+// more to the pair's cross-CTA hand-offs than they gain from staging half of
+// the token tile per CTA.
+int g_gemm_pairs = 2;
+constexpr int kPairMinStages = 12;
 
 template <int FMT, int EPI, int BN, bool PAIR>
 cudaError_t launch_cfg(const GemmArgs& g, const void* a_base, int64_t a_rows, const void* b_base, int64_t b_rows,
@@ -1241,8 +1246,10 @@ cudaError_t launch_cfg(const GemmArgs& g, const void* a_base, int64_t a_rows, co
   if (EPI == kEpiDown && (g.y_rows < 1 || !make_y_map(&my, g.y, g.y_rows, g.ldy))) return cudaErrorInvalidValue;
   const int64_t rb = FMT == kFmtBF16 ? 2 * (int64_t)g.K : (FMT == MOE_FMT_FP8 ? g.K : g.K / 2);
   if (!make_map(&ma, a_base, a_rows, rb, 128)) return cudaErrorInvalidValue;
+  // token boxes of 16, 32, 64, 128 and 256 rows, capped at the rows one CTA stages
+  constexpr int kBRows = PAIR ? BN / 2 : BN;
   for (int i = 0; i < 5; ++i)
-    if (!make_map(&mb.m[i], b_base, b_rows, rb, (16 << i) < BN ? (16 << i) : BN)) return cudaErrorInvalidValue;
+    if (!make_map(&mb.m[i], b_base, b_rows, rb, (16 << i) < kBRows ? (16 << i) : kBRows)) return cudaErrorInvalidValue;
   if (PAIR && F::kBs) {
     const int64_t groups = g.K / F::kBs / 4;  // 512-byte blocks per 128 rows
     if (!make_sf_map(&msfa, g.w_sf, a_rows / 128 * groups, F::kGroups)) return cudaErrorInvalidValue;
@@ -1297,8 +1304,10 @@ cudaError_t launch_cfg(const GemmArgs& g, const void* a_base, int64_t a_rows, co
 template <int FMT, int EPI>
 cudaError_t launch_bn(const GemmArgs& g, int bn, const void* a, int64_t ar, const void* b, int64_t br, int sms,
                       cudaStream_t s) {
-  if (bn == 256 && g_gemm_pairs && g.R % 256 == 0 && sms >= 2)
-    return launch_cfg<FMT, EPI, 256, true>(g, a, ar, b, br, sms, s);
+  const bool pairs = EPI != kEpiLogits && g.R % 256 == 0 && sms >= 2 &&
+                     (g_gemm_pairs == 1 || (g_gemm_pairs == 2 && g.K / FmtTraits<FMT>::kBK >= kPairMinStages));
+  if (bn == 256 && pairs) return launch_cfg<FMT, EPI, 256, true>(g, a, ar, b, br, sms, s);
+  if (bn == 192 && pairs) return launch_cfg<FMT, EPI, 192, true>(g, a, ar, b, br, sms, s);
   if (bn == 256) return launch_cfg<FMT, EPI, 256, false>(g, a, ar, b, br, sms, s);
   if (bn == 192) return launch_cfg<FMT, EPI, 192, false>(g, a, ar, b, br, sms, s);
   if (bn == 64) return launch_cfg<FMT, EPI, 64, false>(g, a, ar, b, br, sms, s);
@@ -1365,7 +1374,7 @@ cudaError_t launch_fused_ffn(const GemmArgs& g1, const GemmArgs& g2, const Fused
 
 bool tensor_maps_available() { return encode_fn() != nullptr; }
 
-void set_gemm_pairs(bool on) { g_gemm_pairs = on; }
+void set_gemm_pairs(int mode) { g_gemm_pairs = mode; }
 
 static int g_early_weights = 1;  // MOE_OPT_EARLY_WEIGHTS
 void set_early_weights(int mode) { g_early_weights = mode; }

@@ -105,8 +105,9 @@ bool tensor_maps_available();
 void set_early_weights(int mode);
 int early_weights();
 constexpr int kEarlyL2Stages = 16;
-// CTA pairs (cta_group::2) for 256-token tiles whose weight rows divide by 256.
-void set_gemm_pairs(bool on);
+// CTA pairs (cta_group::2) for 192- and 256-token tiles whose weight rows
+// divide by 256: 0 off, 1 on, 2 for long K loops only (the default).
+void set_gemm_pairs(int mode);
 // Router logits on the tensor cores, K split over ksplit partial outputs
 // (logits_parts + s * part_stride, the bias in part 0; the top-k kernel adds
 // them): E % 128 == 0, H % 64 == 0.  64-token tiles.

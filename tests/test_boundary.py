@@ -82,13 +82,14 @@ def test_host_side_argument_errors(L):
     assert L.moe_permute(one, 4, 2, 2000, one, one, one, one, 1 << 20, None) == 1
     assert L.moe_set_option(1, 5) == 1 and L.moe_set_option(99, 0) == 1
     assert L.moe_set_option(1, 0) == 0
-    # token tile: 0 (by batch size), 64, 128 or 256
+    # token tile: 0 (by batch size), 64, 128, 192 or 256
     assert L.moe_set_option(2, 32) == 1 and L.moe_set_option(2, 96) == 1
     for v in (64, 128, 256, 0):
         assert L.moe_set_option(2, v) == 0
-    # CTA pairs on or off
-    assert L.moe_set_option(3, 2) == 1
-    assert L.moe_set_option(3, 0) == 0 and L.moe_set_option(3, 1) == 0
+    # CTA pairs: off, on, for long K loops
+    assert L.moe_set_option(3, 3) == 1 and L.moe_set_option(3, -1) == 1
+    for v in (0, 1, 2):
+        assert L.moe_set_option(3, v) == 0
     # early weight loads: 0, 1 or 2
     assert L.moe_set_option(5, 3) == 1 and L.moe_set_option(5, -1) == 1
     for v in (0, 2, 1):

@@ -50,18 +50,18 @@ def _run(over, static, skew, path):
     return w, W, x, perm, off, a13, a2, dev_to_f64(y), st
 
 
-@pytest.mark.parametrize("tile_n,pair", [(64, 1), (128, 1), (192, 1), (256, 0), (256, 1)])
+@pytest.mark.parametrize("tile_n,pair", [(64, 1), (128, 1), (192, 0), (192, 1), (256, 0), (256, 1)])
 @pytest.mark.parametrize("name,over,static,skew", GEMM_CASES)
 def test_gemm_path_matches_oracle(name, over, static, skew, tile_n, pair):
-    """Every token-tile width; 256-token tiles on one CTA and on CTA pairs
-    (cta_group::2, 256 weight rows per tile)."""
+    """Every token-tile width; 192- and 256-token tiles on one CTA and on CTA
+    pairs (cta_group::2, 256 weight rows per tile; 64 and 128 ignore pairs)."""
     ops.moe_set_option(ops.OPT_GEMM_TILE_N, tile_n)
     ops.moe_set_option(ops.OPT_GEMM_PAIR, pair)
     try:
         w, W, x, perm, off, a13, a2, y, st = _run(over, static, skew, 2)
     finally:
         ops.moe_set_option(ops.OPT_GEMM_TILE_N, 0)
-        ops.moe_set_option(ops.OPT_GEMM_PAIR, 0)
+        ops.moe_set_option(ops.OPT_GEMM_PAIR, 2)
     assert st == 0
     ry, _ = oracle.grouped_ffn(x, perm, off, W, 1, a13 or 0.0, a2 or 0.0)
     err = max_abs_rel(y, ry)
