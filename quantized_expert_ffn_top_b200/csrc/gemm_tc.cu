@@ -96,6 +96,8 @@ struct Cfg {
   // barriers (full, empty, tfull, tempty), the tensor-memory address and the
   // abort flag share the 1 KB control block
   static_assert((2 * kStages + 2 * kAccStages) * 8 + 8 <= 1024, "control block overflow");
+  // the down projection double-buffers its store staging there: 2 KB per warp
+  static_assert(kEpiWarps * 2048 <= kEpiBytes, "store staging");
 };
 
 // Tensor-memory column offset of a tile's first token inside its 128-row
@@ -273,8 +275,9 @@ template <int FMT, int EPI, int BN>
 __device__ __forceinline__ void epilogue_slice(const GemmArgs& g, const CUtensorMap* tmap_y, const TileEntry& te,
                                                int mt, int split, int nch, int c_lo, int ew, int q, int lane,
                                                float gact, float g2, float* epi_tiles, const float* r_tab,
-                                               uint16_t* y_stage, float& hmax, const uint32_t* r0,
-                                               const uint32_t* r1, const uint32_t* r2, const uint32_t* r3) {
+                                               uint16_t* y_stage, int ybufs, int& ypar, float& hmax,
+                                               const uint32_t* r0, const uint32_t* r1, const uint32_t* r2,
+                                               const uint32_t* r3) {
 #pragma unroll
   for (int ch = 0; ch < 4; ++ch) {
     if (ch >= nch) break;  // both warps of a pair see the same ncol
@@ -295,10 +298,15 @@ __device__ __forceinline__ void epilogue_slice(const GemmArgs& g, const CUtensor
     } else if (EPI == kEpiDown) {
       const float sc = (FMT == MOE_FMT_MXFP4) ? 1.0f : __ldg(g.w_gs + te.e) * gact;
       if (c0 + 16 <= te.nvalid) {
-        // a full chunk: stage [16 tokens][32 outputs] as bf16 in this
-        // warp's 1 KB and write it with one tensor store
-        uint16_t* stg = y_stage + ew * 512;
-        if (lane == 0) tc::bulk_wait_read();   // the previous store has read the buffer
+        // a full chunk: stage [16 tokens][32 outputs] as bf16 in one of this
+        // warp's ybufs 1 KB buffers and write it with one tensor store; with
+        // two buffers the store of the previous chunk may still be reading
+        uint16_t* stg = y_stage + (ew * ybufs + (ybufs == 2 ? ypar : 0)) * 512;
+        if (lane == 0) {
+          if (ybufs == 2) tc::bulk_wait_read_but1();   // the store from this buffer has read it
+          else tc::bulk_wait_read();
+        }
+        ypar ^= 1;
         __syncwarp();
 #pragma unroll
         for (int c = 0; c < 16; ++c) stg[c * 32 + lane] = f32_to_bf16_rn(v[c] * sc);
@@ -742,6 +750,7 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN, PAIR>::kThreads, 1)
       asm volatile("bar.sync 15, %0;" ::"r"(C::kEpiWarps * 32) : "memory");
     }
     float hmax = 0.0f;
+    int ypar = 0;   // down projection: the store-staging buffer in turn
     int acc = 0;
     uint32_t acc_phase = 0;
     // each tile's entry is read one tile ahead, off the critical path
@@ -785,7 +794,7 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN, PAIR>::kThreads, 1)
       }
       if (c_lo >= ncol) continue;  // both warps of a pair (same slice) skip together
       epilogue_slice<FMT, EPI, BN>(g, &tmap_y, te, mt, split, nch, c_lo, ew, q, lane, gact, g2, epi_tiles, r_tab,
-                                   reinterpret_cast<uint16_t*>(epi_tiles), hmax, r0, r1, r2, r3);
+                                   reinterpret_cast<uint16_t*>(epi_tiles), 2, ypar, hmax, r0, r1, r2, r3);
     }
     if (EPI == kEpiDown && lane == 0) tc::bulk_wait_all();   // stores done before the CTA exits
     if (EPI == kEpiUpF32 && g.h_amax) {
@@ -1106,6 +1115,7 @@ __global__ void __launch_bounds__(Cfg<FMT, kEpiUpQuant, BN, false>::kThreads, 1)
       asm volatile("bar.sync 15, %0;" ::"r"(C::kEpiWarps * 32) : "memory");
     }
     float hmax = 0.0f;
+    int ypar = 0;   // down projection: the store-staging buffer in turn
     int acc = 0;
     uint32_t acc_phase = 0;
     bool up = false;
@@ -1143,7 +1153,7 @@ __global__ void __launch_bounds__(Cfg<FMT, kEpiUpQuant, BN, false>::kThreads, 1)
       if (up) {
         if (c_lo < ncol)
           epilogue_slice<FMT, kEpiUpQuant, BN>(g1, &tmap_y, te, mt, 0, nch, c_lo, ew, q, lane, gact1, gh, epi_tiles,
-                                               r_tab, y_stage, hmax, r0, r1, r2, r3);
+                                               r_tab, y_stage, 1, ypar, hmax, r0, r1, r2, r3);
         // this warp's slice of h is stored: count it for the down tiles
         tc::fence_proxy_async_global();
         __threadfence();
@@ -1151,7 +1161,7 @@ __global__ void __launch_bounds__(Cfg<FMT, kEpiUpQuant, BN, false>::kThreads, 1)
         if (lane == 0) atomicAdd(f.tile_done + tt, 1);
       } else if (c_lo < ncol) {
         epilogue_slice<FMT, kEpiDown, BN>(g2, &tmap_y, te, mt, 0, nch, c_lo, ew, q, lane, gact2, 1.0f, epi_tiles,
-                                          r_tab, y_stage, hmax, r0, r1, r2, r3);
+                                          r_tab, y_stage, 1, ypar, hmax, r0, r1, r2, r3);
       }
     }
     if (lane == 0) tc::bulk_wait_all();   // tensor stores done before the CTA exits
