@@ -2,18 +2,19 @@
 // (+ shared_y[t]), accumulated in fp32 in the order j = 0..k-1 and rounded
 // once to bf16.  The always-on shared expert enters with weight 1.0 (the
 // shared expert of the Domir6/FreeToken fork README, "Changes in this fork").
-// Grid: token x 512-column stretch, 64 threads of 8 columns (16-byte loads)
-// each.  The token's k slot indices and weights are staged in shared memory
-// first, so every thread then issues its k row loads four at a time.
+// Grid: token x stretch of 8 * blockDim.x columns; each thread owns 8
+// columns (16-byte loads).  Every warp reads the token's slot indices and
+// weights itself, 32 at a time into lane registers, and broadcasts them with
+// shuffles, so no shared memory or block barrier is involved; a thread then
+// issues up to eight row loads at once.
 #include "kernels.cuh"
 
 namespace moe {
 
-constexpr int kCombineThreads = 64;
-constexpr int kCombineCols = kCombineThreads * 8;
+constexpr int kCombineThreads = 256;
 constexpr int kCombineMaxK = 1024;  // k <= E <= 1024
 
-__global__ void __launch_bounds__(kCombineThreads) combine_kernel(const uint16_t* __restrict__ y_perm,
+__global__ void __launch_bounds__(kCombineThreads, 4) combine_kernel(const uint16_t* __restrict__ y_perm,
                                                                   const int32_t* __restrict__ inv_perm,
                                                                   const float* __restrict__ w, int64_t T, int k,
                                                                   int H, const uint16_t* __restrict__ shared_y,
@@ -21,22 +22,11 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const uint16_t
   pdl_wait();  // inputs come from the previous kernels
   pdl_trigger();
 
-  __shared__ int32_t sp[kCombineMaxK];
-  __shared__ float sw[kCombineMaxK];
   const int64_t t = blockIdx.x;
   const int64_t S = T * k;
-  for (int j = threadIdx.x; j < k; j += kCombineThreads) {
-    int32_t p = __ldg(inv_perm + t * k + j);
-    if (p >= S) {
-      if (blockIdx.y == 0) raise_status(status, MOE_ERR_DEVICE_FAULT);
-      p = -1;
-    }
-    sp[j] = p;
-    sw[j] = __ldg(w + t * k + j);
-  }
-  __syncthreads();
-  const int c = blockIdx.y * kCombineCols + threadIdx.x * 8;
-  if (c >= H) return;
+  const int lane = threadIdx.x & 31;
+  const int c = blockIdx.y * (blockDim.x * 8) + threadIdx.x * 8;
+  const bool active = c < H;  // every lane takes part in the shuffles
   float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
   auto add = [&](const uint4& v, float wj) {
     const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
@@ -46,22 +36,37 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const uint16_t
       acc[2 * i + 1] = fmaf(wj, __uint_as_float(vv[i] & 0xFFFF0000u), acc[2 * i + 1]);
     }
   };
-  int j = 0;
-  for (; j + 4 <= k; j += 4) {
-    uint4 v[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int32_t p = sp[j + u];
-      v[u] = p >= 0 ? __ldg(reinterpret_cast<const uint4*>(y_perm + (int64_t)p * H + c)) : make_uint4(0, 0, 0, 0);
+  for (int j0 = 0; j0 < k; j0 += 32) {
+    const int nj = min(32, k - j0);
+    int32_t pl = -1;
+    float wl = 0.0f;
+    if (lane < nj) {
+      pl = __ldg(inv_perm + t * k + j0 + lane);
+      wl = __ldg(w + t * k + j0 + lane);
+      if (pl >= S) {
+        if (blockIdx.y == 0 && threadIdx.x < 32) raise_status(status, MOE_ERR_DEVICE_FAULT);
+        pl = -1;
+      }
     }
+    // slots j0 .. j0 + nj - 1, eight loads in flight, summed in slot order
+    for (int jb = 0; jb < nj; jb += 8) {
+      uint4 v[8];
+      int32_t pj[8];
 #pragma unroll
-    for (int u = 0; u < 4; ++u)
-      if (sp[j + u] >= 0) add(v[u], sw[j + u]);
+      for (int u = 0; u < 8; ++u) {
+        pj[u] = __shfl_sync(0xffffffffu, pl, (jb + u) & 31);
+        if (jb + u >= nj) pj[u] = -1;
+        v[u] = (active && pj[u] >= 0) ? __ldg(reinterpret_cast<const uint4*>(y_perm + (int64_t)pj[u] * H + c))
+                                      : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const float wj = __shfl_sync(0xffffffffu, wl, (jb + u) & 31);
+        if (pj[u] >= 0) add(v[u], wj);
+      }
+    }
   }
-  for (; j < k; ++j) {
-    const int32_t p = sp[j];
-    if (p >= 0) add(__ldg(reinterpret_cast<const uint4*>(y_perm + (int64_t)p * H + c)), sw[j]);
-  }
+  if (!active) return;
   if (shared_y) {
     const uint4 v = __ldg(reinterpret_cast<const uint4*>(shared_y + t * H + c));
     const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
@@ -83,9 +88,11 @@ cudaError_t launch_combine(const uint16_t* y_perm, const int32_t* inv_perm, cons
                            const uint16_t* shared_y, uint16_t* out, int32_t* status, cudaStream_t s) {
   if (T == 0) return cudaSuccess;
   if (k > kCombineMaxK) return cudaErrorInvalidValue;
-  const dim3 grid((unsigned)T, (unsigned)((H + kCombineCols - 1) / kCombineCols));
-  cudaError_t e = launch_pdl(combine_kernel, grid, dim3(kCombineThreads), 0, s, y_perm, inv_perm, w, T, k, H, shared_y,
-                             out, status);
+  // narrower blocks for small H, so no warp is idle
+  const int threads = min(kCombineThreads, ((H / 8) + 31) / 32 * 32);
+  const dim3 grid((unsigned)T, (unsigned)((H + threads * 8 - 1) / (threads * 8)));
+  cudaError_t e = launch_pdl(combine_kernel, grid, dim3(threads), 0, s, y_perm, inv_perm, w, T, k, H, shared_y, out,
+                             status);
   count_launches(1);
   return e != cudaSuccess ? e : cudaGetLastError();
 }
