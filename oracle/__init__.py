@@ -20,7 +20,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "moe_oracle.cpp")
 _LIB = os.path.join(_HERE, "libmoe_oracle.so")
 
-FMT_NVFP4, FMT_MXFP4, FMT_FP8 = 1, 2, 3
+FMT_NVFP4, FMT_MXFP4, FMT_FP8, FMT_BF16 = 1, 2, 3, 4
 ACT_BF16, ACT_MATCH = 0, 1
 
 
@@ -65,6 +65,8 @@ def _declare(L):
     L.orc_quant_nvfp4.argtypes = [P, i64, i64, f32, P, P]; L.orc_quant_nvfp4.restype = None
     L.orc_quant_mxfp4.argtypes = [P, i64, i64, P, P]; L.orc_quant_mxfp4.restype = None
     L.orc_quant_fp8.argtypes = [P, i64, f32, P]; L.orc_quant_fp8.restype = None
+    L.orc_bf16_encode.argtypes = [f32]; L.orc_bf16_encode.restype = ctypes.c_int
+    L.orc_quant_bf16.argtypes = [P, i64, P]; L.orc_quant_bf16.restype = None
     L.orc_dequant.argtypes = [ctypes.c_int, P, P, ctypes.c_double, i64, i64, P]; L.orc_dequant.restype = None
     L.orc_router_logits.argtypes = [P, i64, i32, P, i32, P, P]; L.orc_router_logits.restype = None
     L.orc_topk.argtypes = [P, i64, i32, i32, P, P]; L.orc_topk.restype = ctypes.c_int
@@ -148,6 +150,18 @@ def quant_fp8(x: np.ndarray, s: float):
     return codes
 
 
+def bf16_encode(v: float) -> int:
+    return int(lib().orc_bf16_encode(float(np.float32(v))))
+
+
+def quant_bf16(x: np.ndarray) -> np.ndarray:
+    """fp32 -> bf16 codes (little-endian uint16 bytes), the oracle's own rounding."""
+    x = _c(x, np.float32)
+    codes = np.zeros(x.shape[:-1] + (2 * x.shape[-1],), np.uint8)
+    lib().orc_quant_bf16(_p(x), x.size, _p(codes))
+    return codes
+
+
 def dequant(fmt: int, codes: np.ndarray, sf, gs: float, rows: int, K: int) -> np.ndarray:
     codes = _c(codes, np.uint8)
     sf = None if sf is None else _c(sf, np.uint8)
@@ -214,6 +228,8 @@ def quantize_expert_weights(fmt: int, w13: np.ndarray, w2: np.ndarray) -> Weight
     MXFP4 has block scales only."""
     E, twoI, H = w13.shape
     I = twoI // 2
+    if fmt == FMT_BF16:
+        return Weights(fmt, E, H, I, quant_bf16(w13), None, None, quant_bf16(w2), None, None)
     if fmt == FMT_FP8:
         c13 = np.zeros((E, twoI, H), np.uint8)
         c2 = np.zeros((E, H, I), np.uint8)

@@ -23,7 +23,9 @@
 //  * Code formats (not on the pages, which only name them): e2m1 and e8m0 from
 //    the OCP Microscaling Formats (MX) v1.0 specification, e4m3 ("E4M3FN")
 //    from the OCP 8-bit Floating Point specification; NVFP4 = e2m1 elements,
-//    one e4m3 scale per 16 elements, one fp32 global scale per tensor.
+//    one e4m3 scale per 16 elements, one fp32 global scale per tensor; bf16
+//    (the BF16 checkpoints of the upstream README, "About") = the upper half
+//    of the fp32 encoding: 1 sign, 8 exponent, 7 mantissa bits, no scales.
 //
 // Precision: every sum, product and transcendental is evaluated in double.
 // Where floating point decides an integer (a quantised code), the decision is
@@ -42,7 +44,7 @@
 
 namespace {
 
-enum { FMT_NVFP4 = 1, FMT_MXFP4 = 2, FMT_FP8 = 3 };
+enum { FMT_NVFP4 = 1, FMT_MXFP4 = 2, FMT_FP8 = 3, FMT_BF16 = 4 };
 enum { ACT_BF16 = 0, ACT_MATCH = 1 };
 
 inline double bf16_to_double(uint16_t b) {
@@ -234,6 +236,27 @@ void orc_quant_fp8(const float* x, int64_t n, float s, uint8_t* codes) {
   for (int64_t i = 0; i < n; ++i) codes[i] = (uint8_t)orc_e4m3_encode(x[i] * inv);
 }
 
+// fp32 -> bf16: keep the upper 16 bits of the fp32 encoding after rounding
+// the lower 16 to nearest, ties to even (a carry may run into the exponent,
+// up to infinity).  NaN stays a quiet NaN.
+int orc_bf16_encode(float v) {
+  uint32_t u;
+  std::memcpy(&u, &v, 4);
+  if ((u & 0x7F800000u) == 0x7F800000u && (u & 0x007FFFFFu)) return (int)((u >> 16) | 0x40u);
+  const uint32_t low = u & 0xFFFFu, high = u >> 16;
+  if (low > 0x8000u || (low == 0x8000u && (high & 1u))) return (int)((high + 1u) & 0xFFFFu);
+  return (int)high;
+}
+
+// BF16 codes: one bf16 per element, little-endian uint16 in the code bytes.
+void orc_quant_bf16(const float* x, int64_t n, uint8_t* codes) {
+  for (int64_t i = 0; i < n; ++i) {
+    const int b = orc_bf16_encode(x[i]);
+    codes[2 * i] = (uint8_t)(b & 0xFF);
+    codes[2 * i + 1] = (uint8_t)(b >> 8);
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Dequantisation (exact in double)
 // ---------------------------------------------------------------------------
@@ -256,13 +279,14 @@ static const DecodeTables& tables() {
 static inline double dq_elem(int fmt, const uint8_t* crow, const uint8_t* sfrow, double gs, int64_t k) {
   const DecodeTables& tb = tables();
   if (fmt == FMT_FP8) return tb.e4m3[crow[k]] * gs;
+  if (fmt == FMT_BF16) return bf16_to_double((uint16_t)(crow[2 * k] | (crow[2 * k + 1] << 8)));
   int nib = (crow[k >> 1] >> ((k & 1) * 4)) & 15;
   double v = tb.e2m1[nib];
   if (fmt == FMT_NVFP4) return v * tb.e4m3[sfrow[k / 16]] * gs;
   return v * tb.e8m0[sfrow[k / 32]];
 }
 
-static inline int64_t row_bytes(int fmt, int64_t K) { return fmt == FMT_FP8 ? K : K / 2; }
+static inline int64_t row_bytes(int fmt, int64_t K) { return fmt == FMT_FP8 ? K : (fmt == FMT_BF16 ? 2 * K : K / 2); }
 static inline int64_t sf_per_row(int fmt, int64_t K) {
   return fmt == FMT_NVFP4 ? K / 16 : (fmt == FMT_MXFP4 ? K / 32 : 0);
 }
@@ -372,14 +396,14 @@ typedef struct {
 static double w13_elem(const orc_weights* W, int32_t e, int32_t row, int32_t h) {
   const int64_t rb = row_bytes(W->fmt, W->H), nsf = sf_per_row(W->fmt, W->H);
   const int64_t r = (int64_t)e * 2 * W->I + row;
-  double gs = (W->fmt == FMT_MXFP4) ? 1.0 : (double)W->w13_gs[e * 2 + (row >= W->I ? 1 : 0)];
+  double gs = (W->fmt == FMT_MXFP4 || W->fmt == FMT_BF16) ? 1.0 : (double)W->w13_gs[e * 2 + (row >= W->I ? 1 : 0)];
   return dq_elem(W->fmt, W->w13 + r * rb, W->w13_sf ? W->w13_sf + r * nsf : nullptr, gs, h);
 }
 
 static double w2_elem(const orc_weights* W, int32_t e, int32_t o, int32_t i) {
   const int64_t rb = row_bytes(W->fmt, W->I), nsf = sf_per_row(W->fmt, W->I);
   const int64_t r = (int64_t)e * W->H + o;
-  double gs = (W->fmt == FMT_MXFP4) ? 1.0 : (double)W->w2_gs[e];
+  double gs = (W->fmt == FMT_MXFP4 || W->fmt == FMT_BF16) ? 1.0 : (double)W->w2_gs[e];
   return dq_elem(W->fmt, W->w2 + r * rb, W->w2_sf ? W->w2_sf + r * nsf : nullptr, gs, i);
 }
 
@@ -403,12 +427,16 @@ static void activation_rows(int fmt, int act, const std::vector<float>& xf, int6
     orc_quant_nvfp4(xf.data(), rows, K, s, codes.data(), sf.data());
   } else if (fmt == FMT_MXFP4) {
     orc_quant_mxfp4(xf.data(), rows, K, codes.data(), sf.data());
+  } else if (fmt == FMT_BF16) {
+    // MATCH with bf16 weights: the activations are rounded to bf16
+    orc_quant_bf16(xf.data(), rows * K, codes.data());
   } else {
     s = static_scale > 0 ? static_scale : orc_fp8_scale(orc_amax(xf.data(), rows * K));
     orc_quant_fp8(xf.data(), rows * K, s, codes.data());
   }
   if (scale_used) *scale_used = s;
-  orc_dequant(fmt, codes.data(), fmt == FMT_FP8 ? nullptr : sf.data(), (double)s, rows, K, out.data());
+  orc_dequant(fmt, codes.data(), (fmt == FMT_FP8 || fmt == FMT_BF16) ? nullptr : sf.data(), (double)s, rows, K,
+              out.data());
 }
 
 // y for a list of slots (token row, expert): the SwiGLU expert FFN.
@@ -526,8 +554,10 @@ int orc_moe_forward(const uint16_t* x, int64_t T, int32_t H, const uint16_t* wr,
     tokens = all.data();
     n_tokens = T;
   }
-  const bool dyn_h = (act == ACT_MATCH && routed->fmt != FMT_MXFP4 && !(a2_static > 0));
-  const bool dyn_sh = (shared && act == ACT_MATCH && routed->fmt != FMT_MXFP4 && !(sh_a2_static > 0));
+  // MXFP4 and bf16 activations have no per-tensor scale
+  const bool scaled = routed->fmt == FMT_NVFP4 || routed->fmt == FMT_FP8;
+  const bool dyn_h = (act == ACT_MATCH && scaled && !(a2_static > 0));
+  const bool dyn_sh = (shared && act == ACT_MATCH && scaled && !(sh_a2_static > 0));
   // Tokens whose FFN is evaluated: the subset, or all of them when a dynamic
   // h scale couples every slot.
   std::vector<int32_t> eval_tok;

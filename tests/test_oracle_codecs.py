@@ -126,3 +126,25 @@ def test_format_maxima(orc):
     finite = [orc.e4m3_decode(c) for c in range(256) if not math.isnan(orc.e4m3_decode(c))]
     assert max(finite) == 448.0 and min(finite) == -448.0
     assert orc.e8m0_decode(254) == 2.0 ** 127
+
+
+def test_bf16_rounding_matches_torch(orc):
+    """fp32 -> bf16 round-to-nearest-even against torch's conversion: random
+    values over the whole range, exact ties both ways, subnormals, overflow to
+    infinity; NaN stays NaN."""
+    rng = np.random.default_rng(11)
+    bits = rng.integers(0, 2 ** 32, 20000, dtype=np.uint64).astype(np.uint32)
+    ties = (rng.integers(0, 2 ** 16, 2000, dtype=np.uint32) << 16) | 0x8000
+    edge = np.array([0x7F7FFFFF, 0x7F7F8000, 0x00000001, 0x80008000, 0x3F808000, 0x3F818000, 0xFF7FFFFF],
+                    np.uint32)
+    u = np.concatenate([bits, ties, edge])
+    f = u.view(np.float32)
+    ours = np.ascontiguousarray(orc.quant_bf16(f.reshape(1, -1))).view(np.uint16).reshape(-1)
+    ref = torch.from_numpy(f.copy()).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    nan = np.isnan(f)
+    assert np.array_equal(ours[~nan], ref[~nan])
+    ob = (ours[nan].astype(np.uint32) << 16).view(np.float32)
+    assert np.all(np.isnan(ob))
+    # decoding the codes gives the bf16 values exactly
+    d = orc.dequant(4, orc.quant_bf16(f[~nan].reshape(1, -1)), None, 1.0, 1, int((~nan).sum()))
+    assert np.array_equal(d.reshape(-1), (ref[~nan].astype(np.uint32) << 16).view(np.float32).astype(np.float64))

@@ -27,6 +27,9 @@ def _bf(bits):
 def _indep_dequant(fmt, codes, sf, gs, K):
     """Decode without the oracle: golden e2m1 table, torch's e4m3, 2^(c-127)."""
     rows = codes.shape[0]
+    if fmt == 4:  # bf16 bit patterns, decoded by torch
+        b = np.ascontiguousarray(codes).view(np.uint16).copy()
+        return torch.from_numpy(b.view(np.int16)).view(torch.bfloat16).double().numpy().reshape(rows, K)
     if fmt == 3:
         v = torch.from_numpy(codes.copy()).view(torch.float8_e4m3fn).double().numpy()
         return v * gs
@@ -71,7 +74,7 @@ def _layer(orc, fmt, E, H, I, seed=0, identical=False):
     return orc.quantize_expert_weights(fmt, w13, w2)
 
 
-@pytest.mark.parametrize("fmt", [1, 2, 3])
+@pytest.mark.parametrize("fmt", [1, 2, 3, 4])
 def test_single_expert_is_dense_swiglu(orc, fmt):
     T, H, I = 6, 64, 64
     W = _layer(orc, fmt, 1, H, I)
@@ -84,7 +87,7 @@ def test_single_expert_is_dense_swiglu(orc, fmt):
     assert np.all(r["w"] == 1.0) and np.all(r["idx"] == 0)
 
 
-@pytest.mark.parametrize("fmt", [1, 2, 3])
+@pytest.mark.parametrize("fmt", [1, 2, 3, 4])
 def test_identical_experts_reduce_to_dense(orc, fmt):
     T, H, I, E, k = 9, 64, 64, 6, 3
     W = _layer(orc, fmt, E, H, I, identical=True)
@@ -210,3 +213,49 @@ def test_static_scales_make_tokens_independent(orc):
     full = orc.moe_forward(x, wr, None, wk.k, W, act=1, a13_static=a13, a2_static=a2)
     one = orc.moe_forward(x[3:4], wr, None, wk.k, W, act=1, a13_static=a13, a2_static=a2)
     assert np.array_equal(one["out"][0], full["out"][3])
+
+
+def test_bf16_weights_match_mode_rounds_h_to_bf16(orc):
+    """BF16 expert weights in MATCH mode: x is bf16 already and h is rounded to
+    bf16 (torch's rounding here) before the down projection."""
+    T, H, I = 5, 64, 128
+    W = _layer(orc, 4, 1, H, I)
+    x = synth.x_bits(synth.workload("tiny", H=H), T=T)
+    wr = synth.router_bits(synth.workload("tiny", E=1, H=H))
+    r = orc.moe_forward(x, wr, None, 1, W, act=orc.ACT_MATCH)
+    W13, W2 = _expert_dense(orc, W, 0)
+    h, _ = _dense_swiglu(_bf(x), W13, W2)
+    hb = torch.from_numpy(h.astype(np.float32)).to(torch.bfloat16).double().numpy()
+    assert np.allclose(r["out"], hb @ W2.T, rtol=1e-12, atol=1e-12)
+    # and it differs from A16 (h kept in double) by at most bf16's rounding of h
+    a16 = orc.moe_forward(x, wr, None, 1, W, act=orc.ACT_BF16)["out"]
+    bound = (np.abs(h) * 2.0 ** -8) @ np.abs(W2).T + 1e-12
+    assert np.all(np.abs(r["out"] - a16) <= bound)
+
+
+def test_bf16_weights_equal_nvfp4_weights_when_exact(orc):
+    """NVFP4 weights with g = 1 and 2-significant-bit scales decode to values
+    bf16 holds exactly; stored as BF16 weights they give the same layer."""
+    rng = np.random.default_rng(5)
+    E, H, I, T, k = 3, 64, 64, 7, 2
+    c13 = rng.integers(0, 256, (E, 2 * I, H // 2), dtype=np.uint8)
+    c2 = rng.integers(0, 256, (E, H, I // 2), dtype=np.uint8)
+    # e4m3 codes with mantissa 0 or 4 (1.0 or 1.5 times a power of two)
+    def scales(shape):
+        ex = rng.integers(4, 10, shape)
+        return ((ex << 3) | (rng.integers(0, 2, shape) * 4)).astype(np.uint8)
+    s13, s2 = scales((E, 2 * I, H // 16)), scales((E, H, I // 16))
+    g13, g2 = np.ones((E, 2), np.float32), np.ones(E, np.float32)
+    Wn = orc.Weights(1, E, H, I, c13, s13, g13, c2, s2, g2)
+    d13 = np.stack([orc.dequant(1, c13[e], s13[e], 1.0, 2 * I, H) for e in range(E)])
+    d2 = np.stack([orc.dequant(1, c2[e], s2[e], 1.0, H, I) for e in range(E)])
+    # exact in bf16: the low 16 bits of the fp32 encoding are zero
+    f13, f2 = d13.astype(np.float32), d2.astype(np.float32)
+    assert np.all(f13.view(np.uint32) & 0xFFFF == 0) and np.all(f2.view(np.uint32) & 0xFFFF == 0)
+    Wb = orc.quantize_expert_weights(4, f13, f2)
+    wk = synth.workload("tiny", E=E, H=H, k=k)
+    x = synth.x_bits(wk, T=T)
+    wr = synth.router_bits(wk)
+    a = orc.moe_forward(x, wr, None, k, Wn, act=orc.ACT_BF16)["out"]
+    b = orc.moe_forward(x, wr, None, k, Wb, act=orc.ACT_BF16)["out"]
+    assert np.array_equal(a, b)
