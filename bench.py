@@ -140,7 +140,7 @@ def build_layer(ops, synth, torch, w, static: bool):
     del chunks13, chunks2
     bank = ops.quantize_bank(fmt, w13, w2, ws)
     del w13, w2
-    if static and fmt != ops.FMT_MXFP4:
+    if static and fmt in (ops.FMT_NVFP4, ops.FMT_FP8):
         a13, a2 = synth.static_act_scales()
         bank.a13_gs = torch.tensor([a13], dtype=torch.float32, device="cuda")
         bank.a2_gs = torch.tensor([a2], dtype=torch.float32, device="cuda")
@@ -152,7 +152,7 @@ def build_layer(ops, synth, torch, w, static: bool):
         s13 = synth.cuda_normal((1, 2 * w.shared_I, w.H), w.w_std, synth.TID_SH_W13)
         s2 = synth.cuda_normal((1, w.H, w.shared_I), w.w_std, synth.TID_SH_W2)
         sbank = ops.quantize_bank(fmt, s13, s2, ws)
-        if static and fmt != ops.FMT_MXFP4:
+        if static and fmt in (ops.FMT_NVFP4, ops.FMT_FP8):
             # the shared expert reads the routed layer's x scale; its own h scale
             sbank.a2_gs = torch.tensor([synth.static_act_scales()[1]], dtype=torch.float32, device="cuda")
         shared = ops.moe_prepare_weights(sbank)
@@ -176,6 +176,8 @@ def algorithmic(w, bank_fmt: str, offsets: np.ndarray):
     active = int((counts > 0).sum())
     if bank_fmt == "fp8":
         per13, per2 = 2 * I * H, H * I
+    elif bank_fmt == "bf16":
+        per13, per2 = 2 * I * H * 2, H * I * 2
     else:
         bs = 16 if bank_fmt == "nvfp4" else 32
         per13 = 2 * I * H // 2 + 2 * I * H // bs
@@ -342,9 +344,9 @@ def config_report(ops, torch, synth, name, act, steps, warmup, flush, pk):
     alg = algorithmic(w, w.fmt, r["offsets"])
     st = r["stages"]
     ms = np.array(r["ms"])
-    peak = pk["bf16_tflops"] * (FP8_PER_BF16 if w.fmt == "fp8" else FP4_PER_BF16)
+    peak = pk["bf16_tflops"] * {"fp8": FP8_PER_BF16, "bf16": 1.0}.get(w.fmt, FP4_PER_BF16)
     up, down = st.get("ffn_up", 0.0), st.get("ffn_down", 0.0)
-    rep_ = {"workload": workload_name(w), "act_scales": "static" if w.fmt == "nvfp4" else "dynamic",
+    rep_ = {"workload": workload_name(w), "act_scales": {"nvfp4": "static", "bf16": "none"}.get(w.fmt, "dynamic"),
             "ms_median": float(np.median(ms)), "ms_p10": float(np.percentile(ms, 10)),
             "ms_p90": float(np.percentile(ms, 90)), "tokens_per_s": w.T / (float(np.median(ms)) * 1e-3),
             "stages_ms": st, "routing": {"active_experts": alg["active_experts"],
@@ -432,8 +434,9 @@ def run_reference(args):
 
 
 def workload_name(w) -> str:
+    acts = {"fp8": "W8A8", "bf16": "bf16"}.get(w.fmt, "W4A4")
     s = (f"{w.name}: T={w.T} H={w.H} E={w.E} top-{w.k} I={w.I} {w.fmt.upper()} weights, "
-         f"{'W4A4' if w.fmt != 'fp8' else 'W8A8'} activations, {w.router} router")
+         f"{acts} activations, {w.router} router")
     if w.shared_I:
         s += f", shared expert I={w.shared_I}"
     return s
@@ -552,7 +555,8 @@ def main():
         del dl
 
     if not args.no_configs:
-        line["configs"] = [config_report(ops, torch, synth, n, act, 10, 3, flush, pk) for n in ("fp8_shared", "large")]
+        line["configs"] = [config_report(ops, torch, synth, n, act, 10, 3, flush, pk)
+                           for n in ("fp8_shared", "large", "bf16_prefill")]
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_oracle_sample(w, args.cpu_seconds, static=True)

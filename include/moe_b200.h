@@ -67,8 +67,12 @@ typedef enum {
  *  FP8:   e4m3 elements, one fp32 per-tensor scale per part: the per-tensor
  *         W8A8 scheme of FreeToken commit 58f4b9ec0e, where a fused
  *         projection keeps one scale per part and the parts' row ranges come
- *         from the load-time weight_scale run-lengths. */
-typedef enum { MOE_FMT_NVFP4 = 1, MOE_FMT_MXFP4 = 2, MOE_FMT_FP8 = 3 } moe_fmt;
+ *         from the load-time weight_scale run-lengths.
+ *  BF16:  bf16 elements (bit patterns, 2 bytes), no scales: the BF16
+ *         checkpoints of the upstream README ("About").  Activations are bf16
+ *         in both activation modes (MATCH rounds h to bf16); always on the
+ *         tensor cores (tcgen05 kind::f16). */
+typedef enum { MOE_FMT_NVFP4 = 1, MOE_FMT_MXFP4 = 2, MOE_FMT_FP8 = 3, MOE_FMT_BF16 = 4 } moe_fmt;
 
 /* Activation precision.
  *  BF16:  activations stay in bf16/fp32 (weight-only quantisation).
@@ -91,12 +95,13 @@ typedef enum { MOE_LAYOUT_CANONICAL = 0, MOE_LAYOUT_PREPARED = 1 } moe_layout;
  * Merged gate|up projection ("merged projections", atomicmilkshake fork
  * README, "What else changed") followed by the down projection
  * ("ffn_down_exps", same README, "Known limits").  CANONICAL layout:
- *   w13    [E][2I][H/2]  (FP8: [E][2I][H])   rows 0..I-1 gate, I..2I-1 up
- *   w13_sf [E][2I][H/16] e4m3 (NVFP4) | [E][2I][H/32] e8m0 (MXFP4) | NULL (FP8)
- *   w13_gs [E][2] fp32   gate and up part scales (NVFP4, FP8); NULL for MXFP4
- *   w2     [E][H][I/2]   (FP8: [E][H][I])
+ *   w13    [E][2I][H/2]  (FP8: [E][2I][H] bytes, BF16: [E][2I][H] bf16)
+ *          rows 0..I-1 gate, I..2I-1 up
+ *   w13_sf [E][2I][H/16] e4m3 (NVFP4) | [E][2I][H/32] e8m0 (MXFP4) | NULL (FP8, BF16)
+ *   w13_gs [E][2] fp32   gate and up part scales (NVFP4, FP8); NULL for MXFP4, BF16
+ *   w2     [E][H][I/2]   (FP8: [E][H][I] bytes, BF16: [E][H][I] bf16)
  *   w2_sf  [E][H][I/16] | [E][H][I/32] | NULL
- *   w2_gs  [E] fp32      (NVFP4, FP8); NULL for MXFP4
+ *   w2_gs  [E] fp32      (NVFP4, FP8); NULL for MXFP4, BF16
  *   a13_gs, a2_gs: one fp32 each, the static activation scale of x and of h
  *          in MATCH mode (NVFP4 global scale / FP8 per-tensor scale); NULL
  *          selects the dynamic amax-derived scale.  Unused for MXFP4.
@@ -145,13 +150,15 @@ moe_status moe_prepare_weights(const moe_weights* canonical, void* dst, size_t d
  *   NVFP4: sc = e4m3(bmax/(6 g)), r = 1/(dec(sc) g), q = e2m1(x r)  (16-blocks)
  *   MXFP4: c = clamp(floor(log2 bmax) - 2 + 127, 0, 254), q = e2m1(x 2^(127-c))
  *   FP8:   q = e4m3(x * (1/s))
- * in fp32, round-to-nearest-even, saturating.  x (device) is fp32
+ *   BF16:  q = bf16(x)  (no scale; scale_out receives 1)
+ * in fp32, round-to-nearest-even, saturating (BF16: overflowing to inf).  x (device) is fp32
  * (x_dtype 0) or bf16 bits (x_dtype 1).  scale_in (device, one fp32) is the
  * NVFP4 global scale g / FP8 scale s; NULL derives it from the amax of all
  * rows*K values (NVFP4 amax/2688, FP8 amax/448, 1 when the amax is 0).
  * scale_out (device, nullable) receives the scale used.  codes (device):
- * [rows][K/2] (FP8: [rows][K]); sf (device): [rows][K/16 | K/32], NULL for
- * FP8.  K % 16 (NVFP4) / 32 (MXFP4) == 0.  Used to quantise checkpoints on the
+ * [rows][K/2] (FP8: [rows][K] bytes, BF16: [rows][K] bf16); sf (device):
+ * [rows][K/16 | K/32], NULL for FP8 and BF16.  K % 16 (NVFP4, BF16) / 32
+ * (MXFP4) == 0.  Used to quantise checkpoints on the
  * device, and the same device code quantises activations inside the layer. */
 moe_status moe_quantize(int32_t fmt, const void* x, int32_t x_dtype, int64_t rows, int64_t K,
                         const float* scale_in, uint8_t* codes, uint8_t* sf, float* scale_out, void* ws,

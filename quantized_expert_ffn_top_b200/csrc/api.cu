@@ -82,11 +82,16 @@ moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_E
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int block_size(int fmt) { return fmt == MOE_FMT_NVFP4 ? 16 : (fmt == MOE_FMT_MXFP4 ? 32 : 0); }
+// bytes of one row of K weight or activation elements in a format
+int64_t fmt_row_bytes(int fmt, int64_t K) {
+  return fmt == MOE_FMT_FP8 ? K : (fmt == MOE_FMT_BF16 ? 2 * K : K / 2);
+}
 
 // Shape and pointer checks of a weight bank.
 moe_status check_weights(const moe_weights* w, bool need_prepared) {
   if (!w) return MOE_ERR_INVALID_ARG;
-  if (w->fmt != MOE_FMT_NVFP4 && w->fmt != MOE_FMT_MXFP4 && w->fmt != MOE_FMT_FP8) return MOE_ERR_UNSUPPORTED;
+  if (w->fmt != MOE_FMT_NVFP4 && w->fmt != MOE_FMT_MXFP4 && w->fmt != MOE_FMT_FP8 && w->fmt != MOE_FMT_BF16)
+    return MOE_ERR_UNSUPPORTED;
   if (w->E < 1 || w->E > 1024 || w->H <= 0 || w->I <= 0) return MOE_ERR_INVALID_ARG;
   if (w->H % 128 != 0 || w->I % 128 != 0) return MOE_ERR_UNSUPPORTED;
   if (w->layout != MOE_LAYOUT_CANONICAL && w->layout != MOE_LAYOUT_PREPARED) return MOE_ERR_INVALID_ARG;
@@ -94,8 +99,8 @@ moe_status check_weights(const moe_weights* w, bool need_prepared) {
   if (!w->w13 || !w->w2) return MOE_ERR_INVALID_ARG;
   if (!aligned16(w->w13) || !aligned16(w->w2) || !aligned16(w->w13_sf) || !aligned16(w->w2_sf))
     return MOE_ERR_INVALID_ARG;
-  if (w->fmt != MOE_FMT_FP8 && (!w->w13_sf || !w->w2_sf)) return MOE_ERR_INVALID_ARG;
-  if (w->fmt != MOE_FMT_MXFP4 && (!w->w13_gs || !w->w2_gs)) return MOE_ERR_INVALID_ARG;
+  if (block_size(w->fmt) && (!w->w13_sf || !w->w2_sf)) return MOE_ERR_INVALID_ARG;
+  if ((w->fmt == MOE_FMT_NVFP4 || w->fmt == MOE_FMT_FP8) && (!w->w13_gs || !w->w2_gs)) return MOE_ERR_INVALID_ARG;
   return MOE_OK;
 }
 
@@ -157,7 +162,7 @@ struct FfnScratch {
 FfnScratch carve_ffn(Carver& c, int64_t S, const moe_weights* w) {
   FfnScratch f;
   const int bs = w->fmt == MOE_FMT_NVFP4 ? 16 : (w->fmt == MOE_FMT_MXFP4 ? 32 : 0);
-  const int64_t rbh = w->fmt == MOE_FMT_FP8 ? w->H : w->H / 2, rbi = w->fmt == MOE_FMT_FP8 ? w->I : w->I / 2;
+  const int64_t rbh = fmt_row_bytes(w->fmt, w->H), rbi = fmt_row_bytes(w->fmt, w->I);
   f.P = padded_rows(S, w->E);
   f.h = c.take<float>((size_t)S * w->I);
   f.poff = c.take<int32_t>((size_t)w->E + 1);
@@ -248,8 +253,9 @@ cudaError_t run_router(const uint16_t* x, int64_t T, int H, const uint16_t* wr, 
 }
 
 bool gemm_shapes_ok(const moe_weights* w, int act) {
-  if (act != MOE_ACT_MATCH || !tensor_maps_available()) return false;
-  const int kb = w->fmt == MOE_FMT_FP8 ? 128 : 256;
+  // BF16 weights: bf16 activations in either mode
+  if ((act != MOE_ACT_MATCH && w->fmt != MOE_FMT_BF16) || !tensor_maps_available()) return false;
+  const int kb = w->fmt == MOE_FMT_FP8 ? 128 : (w->fmt == MOE_FMT_BF16 ? 64 : 256);
   return w->H % kb == 0 && w->I % kb == 0 && w->I % 64 == 0;
 }
 
@@ -257,7 +263,7 @@ bool gemm_shapes_ok(const moe_weights* w, int act) {
 // it; the weight-streaming GEMV for BF16 activations and other shapes.
 bool use_gemm_path(const moe_weights* w, int64_t S, int act) {
   (void)S;
-  if (g_ffn_path == 1) return false;
+  if (g_ffn_path == 1 && w->fmt != MOE_FMT_BF16) return false;   // (no GEMV for BF16 weights)
   return gemm_shapes_ok(w, act);
 }
 
@@ -281,8 +287,8 @@ moe_status run_gemm_ffn(const uint16_t* x, int64_t T, int64_t S, const int32_t* 
   // gate|up projection + SwiGLU quantise h in the epilogue when its scale
   // needs no global reduction (MXFP4, or a static NVFP4 scale); with 64-token
   // tiles the two projections then run as one kernel
-  const bool fused_h = fmt == MOE_FMT_MXFP4 || (fmt == MOE_FMT_NVFP4 && w->a2_gs);
-  const bool one_kernel = g_fused_ffn && fused_h && bn == 64 && E <= kFusedMaxE;
+  const bool fused_h = fmt == MOE_FMT_MXFP4 || fmt == MOE_FMT_BF16 || (fmt == MOE_FMT_NVFP4 && w->a2_gs);
+  const bool one_kernel = g_fused_ffn && fused_h && fmt != MOE_FMT_BF16 && bn == 64 && E <= kFusedMaxE;
   // without a plan from the permutation, the per-slot x quantiser writes it
   if (mark) stage_mark(MOE_STAGE_ACT_QUANT, false, s);
   QuantPaddedArgs qa;
@@ -424,7 +430,7 @@ moe_status run_grouped_ffn(const uint16_t* x, int64_t T, int64_t S, const int32_
   if (use_gemm_path(w, S, act))
     return run_gemm_ffn(x, T, S, perm, offsets, inv, k, slot_expert, w, y_perm, scratch, x_amax, h_amax, status, s,
                         mark, planned);
-  if (g_ffn_path == 2) return MOE_ERR_UNSUPPORTED;
+  if (g_ffn_path == 2 || w->fmt == MOE_FMT_BF16) return MOE_ERR_UNSUPPORTED;   // the GEMV has no BF16 weights
   GemvArgs a;
   a.fmt = w->fmt;
   a.act = act;
@@ -508,7 +514,7 @@ struct SideFork {
 };
 
 bool dynamic_x_scale(const moe_weights* w, int act) {
-  return act == MOE_ACT_MATCH && w->fmt != MOE_FMT_MXFP4 && !w->a13_gs;
+  return act == MOE_ACT_MATCH && (w->fmt == MOE_FMT_NVFP4 || w->fmt == MOE_FMT_FP8) && !w->a13_gs;
 }
 
 }  // namespace
@@ -600,7 +606,7 @@ size_t moe_prepared_weights_size(const moe_weights* w) {
   if (check_weights(w, false) != MOE_OK) return 0;
   const int64_t E = w->E, H = w->H, I = w->I;
   const int bs = block_size(w->fmt);
-  const int64_t rb13 = w->fmt == MOE_FMT_FP8 ? H : H / 2, rb2 = w->fmt == MOE_FMT_FP8 ? I : I / 2;
+  const int64_t rb13 = fmt_row_bytes(w->fmt, H), rb2 = fmt_row_bytes(w->fmt, I);
   Carver c(nullptr);
   c.take<uint8_t>((size_t)(E * 2 * I * rb13));
   c.take<uint8_t>((size_t)(E * H * rb2));
@@ -620,7 +626,7 @@ moe_status moe_prepare_weights(const moe_weights* w, void* dst, size_t dst_bytes
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int64_t E = w->E, H = w->H, I = w->I;
   const int bs = block_size(w->fmt);
-  const int64_t rb13 = w->fmt == MOE_FMT_FP8 ? H : H / 2, rb2 = w->fmt == MOE_FMT_FP8 ? I : I / 2;
+  const int64_t rb13 = fmt_row_bytes(w->fmt, H), rb2 = fmt_row_bytes(w->fmt, I);
   Carver c(dst);
   uint8_t* w13 = c.take<uint8_t>((size_t)(E * 2 * I * rb13));
   uint8_t* w2 = c.take<uint8_t>((size_t)(E * H * rb2));
@@ -648,18 +654,20 @@ moe_status moe_prepare_weights(const moe_weights* w, void* dst, size_t dst_bytes
 moe_status moe_quantize(int32_t fmt, const void* x, int32_t x_dtype, int64_t rows, int64_t K, const float* scale_in,
                         uint8_t* codes, uint8_t* sf, float* scale_out, void* ws, size_t ws_bytes,
                         moe_stream_t stream) {
-  if (fmt != MOE_FMT_NVFP4 && fmt != MOE_FMT_MXFP4 && fmt != MOE_FMT_FP8) return MOE_ERR_UNSUPPORTED;
+  if (fmt != MOE_FMT_NVFP4 && fmt != MOE_FMT_MXFP4 && fmt != MOE_FMT_FP8 && fmt != MOE_FMT_BF16)
+    return MOE_ERR_UNSUPPORTED;
   if (rows < 0 || K <= 0 || (x_dtype != 0 && x_dtype != 1)) return MOE_ERR_INVALID_ARG;
   const int bs = fmt == MOE_FMT_MXFP4 ? 32 : 16;
   if (K % bs != 0) return MOE_ERR_UNSUPPORTED;
-  if (rows > 0 && (!x || !codes || (fmt != MOE_FMT_FP8 && !sf))) return MOE_ERR_INVALID_ARG;
+  if (rows > 0 && (!x || !codes || (block_size(fmt) && !sf))) return MOE_ERR_INVALID_ARG;
   if (!aligned16(codes)) return MOE_ERR_INVALID_ARG;
   Carver c(ws);
   Scalars head = carve_head(c);
   if (!ws || ws_bytes < c.off) return MOE_ERR_WORKSPACE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (rows == 0) return MOE_OK;
-  if (fmt != MOE_FMT_MXFP4 && !scale_in) MOE_TRY(launch_amax(x, x_dtype, rows * K, head.x_amax, num_sms(), s));
+  if ((fmt == MOE_FMT_NVFP4 || fmt == MOE_FMT_FP8) && !scale_in)
+    MOE_TRY(launch_amax(x, x_dtype, rows * K, head.x_amax, num_sms(), s));
   return cuda_status(launch_quantize(fmt, x, x_dtype, rows, K, scale_in, head.x_amax, codes, sf, scale_out,
                                      num_sms(), s));
 }

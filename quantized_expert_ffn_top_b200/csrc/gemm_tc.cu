@@ -222,6 +222,20 @@ template <int FMT>
 __device__ __forceinline__ void quant_block_store(const float* v, float scale, uint8_t* codes, uint8_t* sf,
                                                   int64_t row, int b, int nb, int K) {
   constexpr int bs = FMT == MOE_FMT_MXFP4 ? 32 : 16;
+  if constexpr (FMT == kFmtBF16) {
+    // bf16 activations: the 16 values (bf16 already) are stored as they are
+    uint32_t p[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      p[i] = (uint32_t)f32_to_bf16_rn(v[2 * i]) | ((uint32_t)f32_to_bf16_rn(v[2 * i + 1]) << 16);
+    uint4* dst = reinterpret_cast<uint4*>(codes + row * (int64_t)K * 2 + b * 32);
+    dst[0] = make_uint4(p[0], p[1], p[2], p[3]);
+    dst[1] = make_uint4(p[4], p[5], p[6], p[7]);
+    (void)scale;
+    (void)sf;
+    (void)nb;
+    return;
+  }
   float bmax = 0.0f;
 #pragma unroll
   for (int i = 0; i < bs; ++i) bmax = fmaxf(bmax, fabsf(v[i]));
@@ -296,7 +310,7 @@ __device__ __forceinline__ void epilogue_slice(const GemmArgs& g, const CUtensor
         if (tok < te.nvalid) out[(size_t)(te.p0 + tok) * g.ldy + o] = v[c] + b;
       }
     } else if (EPI == kEpiDown) {
-      const float sc = (FMT == MOE_FMT_MXFP4) ? 1.0f : __ldg(g.w_gs + te.e) * gact;
+      const float sc = (FMT == MOE_FMT_MXFP4 || FMT == kFmtBF16) ? 1.0f : __ldg(g.w_gs + te.e) * gact;
       if (c0 + 16 <= te.nvalid) {
         // a full chunk: stage [16 tokens][32 outputs] as bf16 in one of this
         // warp's ybufs 1 KB buffers and write it with one tensor store; with
@@ -335,7 +349,7 @@ __device__ __forceinline__ void epilogue_slice(const GemmArgs& g, const CUtensor
       // maximum, the scale, the codes and 8-byte stores.
       if (ch & 1) continue;  // taken together with the even chunk
       const int part = lane & 1;
-      const float sc = (FMT == MOE_FMT_MXFP4) ? 1.0f : __ldg(g.w_gs + te.e * 2 + part) * gact;
+      const float sc = (FMT == MOE_FMT_MXFP4 || FMT == kFmtBF16) ? 1.0f : __ldg(g.w_gs + te.e * 2 + part) * gact;
       const int pp = q & 1;                                       // position in the warp pair
       float* tile = epi_tiles + (ew >> 1) * (kEpiTileBytes / 4);    // [32 tokens][36] of the pair
       const int fl = lane >> 1;                                   // feature within the warp's 16
@@ -378,6 +392,17 @@ __device__ __forceinline__ void epilogue_slice(const GemmArgs& g, const CUtensor
           for (int j = 0; j < 4; ++j) dst[j] = src[j];
 #pragma unroll
           for (int j = 0; j < 16; ++j) hmax = fmaxf(hmax, fabsf(hv[j]));
+        }
+      } else if constexpr (FMT == kFmtBF16) {
+        // bf16 weights: h in bf16, 16 features (32 bytes) per thread
+        if (valid) {
+          uint32_t p[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            p[j] = (uint32_t)f32_to_bf16_rn(hv[2 * j]) | ((uint32_t)f32_to_bf16_rn(hv[2 * j + 1]) << 16);
+          uint4* dst = reinterpret_cast<uint4*>(g.hq + row * (int64_t)g.I * 2 + f0 * 2);
+          dst[0] = make_uint4(p[0], p[1], p[2], p[3]);
+          dst[1] = make_uint4(p[4], p[5], p[6], p[7]);
         }
       } else {
         float bmax = 0.0f;
@@ -1314,10 +1339,12 @@ cudaError_t launch_cfg(const GemmArgs& g, const void* a_base, int64_t a_rows, co
 template <int FMT, int EPI>
 cudaError_t launch_bn(const GemmArgs& g, int bn, const void* a, int64_t ar, const void* b, int64_t br, int sms,
                       cudaStream_t s) {
-  const bool pairs = EPI != kEpiLogits && g.R % 256 == 0 && sms >= 2 &&
-                     (g_gemm_pairs == 1 || (g_gemm_pairs == 2 && g.K / FmtTraits<FMT>::kBK >= kPairMinStages));
-  if (bn == 256 && pairs) return launch_cfg<FMT, EPI, 256, true>(g, a, ar, b, br, sms, s);
-  if (bn == 192 && pairs) return launch_cfg<FMT, EPI, 192, true>(g, a, ar, b, br, sms, s);
+  if constexpr (FMT != kFmtBF16) {   // (no pair form of the bf16 MMA here)
+    const bool pairs = EPI != kEpiLogits && g.R % 256 == 0 && sms >= 2 &&
+                       (g_gemm_pairs == 1 || (g_gemm_pairs == 2 && g.K / FmtTraits<FMT>::kBK >= kPairMinStages));
+    if (bn == 256 && pairs) return launch_cfg<FMT, EPI, 256, true>(g, a, ar, b, br, sms, s);
+    if (bn == 192 && pairs) return launch_cfg<FMT, EPI, 192, true>(g, a, ar, b, br, sms, s);
+  }
   if (bn == 256) return launch_cfg<FMT, EPI, 256, false>(g, a, ar, b, br, sms, s);
   if (bn == 192) return launch_cfg<FMT, EPI, 192, false>(g, a, ar, b, br, sms, s);
   if (bn == 64) return launch_cfg<FMT, EPI, 64, false>(g, a, ar, b, br, sms, s);
@@ -1365,6 +1392,7 @@ cudaError_t launch_grouped_gemm(const GemmArgs& g, int epi, int bn, const void* 
     case MOE_FMT_NVFP4: return launch_epi<MOE_FMT_NVFP4>(g, epi, bn, a_base, a_rows, b_base, b_rows, num_sms, s);
     case MOE_FMT_MXFP4: return launch_epi<MOE_FMT_MXFP4>(g, epi, bn, a_base, a_rows, b_base, b_rows, num_sms, s);
     case MOE_FMT_FP8: return launch_epi<MOE_FMT_FP8>(g, epi, bn, a_base, a_rows, b_base, b_rows, num_sms, s);
+    case kFmtBF16: return launch_epi<kFmtBF16>(g, epi, bn, a_base, a_rows, b_base, b_rows, num_sms, s);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -1799,7 +1827,7 @@ __global__ void __launch_bounds__(256) quant_tokens_kernel(QuantPaddedArgs a) {
 cudaError_t launch_quant_padded(const QuantPaddedArgs& a, bool src_x, int fmt, int num_sms, cudaStream_t s) {
   if (a.S == 0) return cudaSuccess;
   cudaError_t e = cudaSuccess;
-  if (src_x && a.inv_perm && a.K % 64 == 0) {
+  if (src_x && a.inv_perm && a.K % 64 == 0 && fmt != kFmtBF16) {
     const int64_t blocks = (a.T + 7) / 8;
     const int grid = (int)(blocks < (int64_t)num_sms * 8 ? blocks : (int64_t)num_sms * 8);
     switch (fmt) {
@@ -1821,6 +1849,7 @@ cudaError_t launch_quant_padded(const QuantPaddedArgs& a, bool src_x, int fmt, i
     case MOE_FMT_NVFP4: MOE_QP(MOE_FMT_NVFP4) break;
     case MOE_FMT_MXFP4: MOE_QP(MOE_FMT_MXFP4) break;
     case MOE_FMT_FP8: MOE_QP(MOE_FMT_FP8) break;
+    case kFmtBF16: MOE_QP(kFmtBF16) break;
     default: return cudaErrorInvalidValue;
   }
 #undef MOE_QP

@@ -2,7 +2,7 @@
 // the fused quantise-and-dequantise of activation rows used by the GEMV path.
 //
 // The quantisation rules are those of the expert-weight formats the FreeToken
-// upstream README names ("About": MXFP4, NVFP4, FP8) applied to activations
+// upstream README names ("About": MXFP4, NVFP4, FP8, BF16) applied to activations
 // for the W4A4 / W8A8 schemes (FreeToken commit 58f4b9ec0e: per-tensor FP8
 // with a dynamic activation scale).  One thread owns one scale block, so the
 // block maximum is a private loop and the codes of a block leave as one
@@ -60,7 +60,7 @@ __global__ void __launch_bounds__(256) quantize_kernel(int fmt, const In* __rest
                                                        float* __restrict__ scale_out) {
   const int bs = fmt == MOE_FMT_MXFP4 ? 32 : 16;
   const int64_t nblk = rows * (K / bs);
-  const float scale = fmt == MOE_FMT_MXFP4 ? 1.0f : resolve_scale(fmt, scale_in, amax);
+  const float scale = (fmt == MOE_FMT_MXFP4 || fmt == MOE_FMT_BF16) ? 1.0f : resolve_scale(fmt, scale_in, amax);
   if (scale_out && blockIdx.x == 0 && threadIdx.x == 0) *scale_out = scale;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < nblk; b += stride) {
@@ -91,6 +91,15 @@ __global__ void __launch_bounds__(256) quantize_kernel(int fmt, const In* __rest
       w.w = e2m1_encode8(v + 24, inv);
       *reinterpret_cast<uint4*>(codes + b * 16) = w;
       sf[b] = (uint8_t)c;
+    } else if (fmt == MOE_FMT_BF16) {
+      // bf16: round to nearest even, 16 values = 32 bytes
+      uint32_t p[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        p[i] = (uint32_t)f32_to_bf16_rn(v[2 * i]) | ((uint32_t)f32_to_bf16_rn(v[2 * i + 1]) << 16);
+      uint4* dst = reinterpret_cast<uint4*>(codes + b * 32);
+      dst[0] = make_uint4(p[0], p[1], p[2], p[3]);
+      dst[1] = make_uint4(p[4], p[5], p[6], p[7]);
     } else {
       const float inv = __frcp_rn(scale);
       uint4 w;

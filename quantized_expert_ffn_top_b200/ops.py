@@ -17,7 +17,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libmoe_b200.so")
 
 MOE_OK = 0
-FMT_NVFP4, FMT_MXFP4, FMT_FP8 = 1, 2, 3
+FMT_NVFP4, FMT_MXFP4, FMT_FP8, FMT_BF16 = 1, 2, 3, 4
 ACT_BF16, ACT_MATCH = 0, 1
 LAYOUT_CANONICAL, LAYOUT_PREPARED = 0, 1
 OPT_FFN_PATH = 1
@@ -26,7 +26,12 @@ OPT_GEMM_PAIR = 3
 OPT_PDL = 4
 OPT_EARLY_WEIGHTS = 5
 OPT_FUSED_FFN = 6
-FMT_BY_NAME = {"nvfp4": FMT_NVFP4, "mxfp4": FMT_MXFP4, "fp8": FMT_FP8}
+FMT_BY_NAME = {"nvfp4": FMT_NVFP4, "mxfp4": FMT_MXFP4, "fp8": FMT_FP8, "bf16": FMT_BF16}
+
+
+def row_bytes(fmt: int, K: int) -> int:
+    """Bytes of one row of K weight elements in a format."""
+    return K if fmt == FMT_FP8 else (2 * K if fmt == FMT_BF16 else K // 2)
 
 EXPORTED = (
     "moe_status_string", "moe_version", "moe_set_option", "moe_workspace_size", "moe_prepared_weights_size",
@@ -182,8 +187,8 @@ def moe_prepare_weights(bank: WeightBank, stream=None) -> WeightBank:
         off = ptr - dst.data_ptr()
         return dst[off:off + numel]
 
-    rb13 = bank.H if bank.fmt == FMT_FP8 else bank.H // 2
-    rb2 = bank.I if bank.fmt == FMT_FP8 else bank.I // 2
+    rb13 = row_bytes(bank.fmt, bank.H)
+    rb2 = row_bytes(bank.fmt, bank.I)
     bs = {FMT_NVFP4: 16, FMT_MXFP4: 32}.get(bank.fmt, 0)
     return replace(bank, layout=LAYOUT_PREPARED,
                    w13=view(out.w13, bank.E * 2 * bank.I * rb13),
@@ -199,8 +204,7 @@ def moe_quantize(fmt: int, x: torch.Tensor, scale_in: torch.Tensor | None = None
     """x: [rows][K] fp32 or bf16 (device).  Returns (codes, sf, scale_used)."""
     rows, K = x.shape
     dt = {torch.float32: 0, torch.bfloat16: 1}[x.dtype]
-    cb = K if fmt == FMT_FP8 else K // 2
-    codes = torch.empty((rows, cb), dtype=torch.uint8, device=x.device)
+    codes = torch.empty((rows, row_bytes(fmt, K)), dtype=torch.uint8, device=x.device)
     bs = {FMT_NVFP4: 16, FMT_MXFP4: 32}.get(fmt, 0)
     sf = torch.empty((rows, K // bs), dtype=torch.uint8, device=x.device) if bs else None
     scale_out = torch.ones(1, dtype=torch.float32, device=x.device)
@@ -294,14 +298,15 @@ def quantize_bank(fmt: int, w13: torch.Tensor, w2: torch.Tensor, ws: torch.Tenso
     I = twoI // 2
     dev = w13.device
     bs = {FMT_NVFP4: 16, FMT_MXFP4: 32}.get(fmt, 0)
-    cb13 = H if fmt == FMT_FP8 else H // 2
-    cb2 = I if fmt == FMT_FP8 else I // 2
+    cb13 = row_bytes(fmt, H)
+    cb2 = row_bytes(fmt, I)
     c13 = torch.empty((E, twoI, cb13), dtype=torch.uint8, device=dev)
     c2 = torch.empty((E, H, cb2), dtype=torch.uint8, device=dev)
     s13 = torch.empty((E, twoI, H // bs), dtype=torch.uint8, device=dev) if bs else None
     s2 = torch.empty((E, H, I // bs), dtype=torch.uint8, device=dev) if bs else None
-    g13 = torch.ones((E, 2), dtype=torch.float32, device=dev) if fmt != FMT_MXFP4 else None
-    g2 = torch.ones(E, dtype=torch.float32, device=dev) if fmt != FMT_MXFP4 else None
+    scaled = fmt in (FMT_NVFP4, FMT_FP8)
+    g13 = torch.ones((E, 2), dtype=torch.float32, device=dev) if scaled else None
+    g2 = torch.ones(E, dtype=torch.float32, device=dev) if scaled else None
     ws = ws if ws is not None else new_workspace(4096, dev)
     L = lib()
     st = _stream()

@@ -65,6 +65,8 @@ WORKLOADS = {
     "prefill": Workload("prefill", 4096, 2048, 128, 8, 768, "nvfp4", "zipf"),
     "fp8_shared": Workload("fp8_shared", 512, 2048, 256, 8, 512, "fp8", "uniform", shared_I=512),
     "large": Workload("large", 16384, 4096, 256, 8, 2048, "mxfp4", "zipf"),
+    # the prefill layer with BF16 expert weights (bf16 activations throughout)
+    "bf16_prefill": Workload("bf16_prefill", 4096, 2048, 128, 8, 768, "bf16", "zipf"),
 }
 
 

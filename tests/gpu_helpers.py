@@ -9,7 +9,7 @@ import torch
 import oracle
 from quantized_expert_ffn_top_b200 import ops, synth
 
-FMT = {"nvfp4": oracle.FMT_NVFP4, "mxfp4": oracle.FMT_MXFP4, "fp8": oracle.FMT_FP8}
+FMT = {"nvfp4": oracle.FMT_NVFP4, "mxfp4": oracle.FMT_MXFP4, "fp8": oracle.FMT_FP8, "bf16": oracle.FMT_BF16}
 
 # max-abs-relative error bound of the layer's outputs against the fp64 oracle
 TOL = 2e-2

@@ -57,6 +57,12 @@ def test_workspace_and_prepared_sizes(L):
     p = L.moe_prepared_weights_size(ctypes.byref(b))
     # w13 8*512*64 + w2 8*128*128 + sf13 8*512*8 + sf2 8*128*16 bytes, 256-aligned pieces
     assert p >= 8 * 512 * 64 + 8 * 128 * 128 + 8 * 512 * 8 + 8 * 128 * 16
+    # BF16 weights: no scales, two bytes an element
+    bb = ops.MoeWeightsC(4, 8, 128, 256, 0, 256, None, None, 256, None, None, None, None)
+    assert L.moe_workspace_size(8, 2, ctypes.byref(bb), None, 0) > 0
+    assert L.moe_workspace_size(8, 2, ctypes.byref(bb), None, 1) > 0
+    pb = L.moe_prepared_weights_size(ctypes.byref(bb))
+    assert 8 * 512 * 256 + 8 * 128 * 512 <= pb < 8 * 512 * 256 + 8 * 128 * 512 + 4096
 
 
 def test_host_side_argument_errors(L):
@@ -77,7 +83,8 @@ def test_host_side_argument_errors(L):
     assert L.moe_forward(one, 4, one, None, 2, ctypes.byref(d), None, 1, one, one, 1 << 30, None) == 2
     # quantize: K not a multiple of the block, unknown format
     assert L.moe_quantize(1, one, 0, 2, 24, None, one, one, None, one, 1 << 20, None) == 2
-    assert L.moe_quantize(4, one, 0, 2, 32, None, one, one, None, one, 1 << 20, None) == 2
+    assert L.moe_quantize(5, one, 0, 2, 32, None, one, one, None, one, 1 << 20, None) == 2
+    assert L.moe_quantize(4, one, 0, 2, 24, None, one, None, None, one, 1 << 20, None) == 2  # BF16, K % 16
     # permute: E out of range
     assert L.moe_permute(one, 4, 2, 2000, one, one, one, one, 1 << 20, None) == 1
     assert L.moe_set_option(1, 5) == 1 and L.moe_set_option(99, 0) == 1

@@ -113,6 +113,40 @@ def test_fused_ffn_kernel_matches_two_kernels(name, over, static, skew):
     assert max_abs_rel(ys[1], ry) < TOL
 
 
+BF16_CASES = [
+    ("bf16-ragged", dict(fmt="bf16", T=200, H=512, E=8, k=2, I=256), 1.2),
+    ("bf16-small-batch", dict(fmt="bf16", T=4, H=256, E=16, k=4, I=256), 0.0),
+    ("bf16-some-empty", dict(fmt="bf16", T=64, H=256, E=32, k=2, I=256), 2.5),
+    ("bf16-long-k", dict(fmt="bf16", T=96, H=1024, E=4, k=2, I=384), 1.0),
+]
+
+
+@pytest.mark.parametrize("tile_n", [0, 64, 192, 256])
+@pytest.mark.parametrize("act", [0, 1])
+@pytest.mark.parametrize("name,over,skew", BF16_CASES)
+def test_bf16_weights_match_oracle(name, over, skew, act, tile_n):
+    """BF16 expert weights on the tensor cores (kind::f16): x gathered into
+    padded bf16 rows, h stored in bf16 by the gate|up epilogue."""
+    ops.moe_set_option(ops.OPT_GEMM_TILE_N, tile_n)
+    try:
+        w = synth.workload("tiny", **over)
+        W, _ = oracle_bank(w)
+        bank = device_bank(W)
+        idx = synth.random_topk_idx(w.T, w.k, w.E, skew=skew)
+        off, perm, inv, _ = oracle.permute(idx, w.E)
+        x = synth.x_bits(w)
+        ws = ops.new_workspace(ops.workspace_size(w.T, w.k, bank, None, act))
+        y = ops.moe_grouped_ffn(bits_to_dev_bf16(x), w.k, torch.from_numpy(perm).cuda(),
+                                torch.from_numpy(off).cuda(), bank, act, ws)
+        torch.cuda.synchronize()
+        st = ops.moe_get_device_status(ws)
+    finally:
+        ops.moe_set_option(ops.OPT_GEMM_TILE_N, 0)
+    assert st == 0
+    ry, _ = oracle.grouped_ffn(x, perm, off, W, act)
+    assert max_abs_rel(dev_to_f64(y), ry) < TOL
+
+
 @pytest.mark.parametrize("name,over,static,skew", GEMM_CASES[:4])
 def test_gemm_and_gemv_paths_agree(name, over, static, skew):
     *_, yg, st1 = _run(over, static, skew, 2)

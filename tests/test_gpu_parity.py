@@ -71,7 +71,7 @@ def test_e2m1_conversion_matches_oracle_on_every_bf16_below_8():
     assert bad[0].size == 0, f"{bad[0].size} mismatches: {blocks[:, 1:][bad][:5]} got {nib[:, 1:][bad][:5]}"
 
 
-@pytest.mark.parametrize("fmt", ["nvfp4", "mxfp4", "fp8"])
+@pytest.mark.parametrize("fmt", ["nvfp4", "mxfp4", "fp8", "bf16"])
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("static", [False, True])
 def test_quantize_matches_oracle(fmt, dtype, static):
@@ -86,7 +86,7 @@ def test_quantize_matches_oracle(fmt, dtype, static):
         xd = bits_to_dev_bf16(bits)
     else:
         xd = torch.from_numpy(xf).cuda()
-    f = {"nvfp4": 1, "mxfp4": 2, "fp8": 3}[fmt]
+    f = {"nvfp4": 1, "mxfp4": 2, "fp8": 3, "bf16": 4}[fmt]
     scale = 0.0123 if static else None
     sd = torch.tensor([scale], dtype=torch.float32, device="cuda") if static else None
     codes, sf, s_used = ops.moe_quantize(f, xd, scale_in=sd)
@@ -96,6 +96,9 @@ def test_quantize_matches_oracle(fmt, dtype, static):
     elif f == 2:
         g = 1.0
         rc, rs = oracle.quant_mxfp4(xf)
+    elif f == 4:
+        g = 1.0
+        rc, rs = oracle.quant_bf16(xf), None
     else:
         g = scale if static else oracle.fp8_scale(oracle.amax(xf))
         rc, rs = oracle.quant_fp8(xf, g), None
@@ -104,6 +107,8 @@ def test_quantize_matches_oracle(fmt, dtype, static):
         assert np.array_equal(sf.cpu().numpy(), rs)
     if f != 2:
         assert float(s_used.item()) == np.float32(g)
+    if f == 4:
+        assert sf is None
 
 
 # --------------------------------------------------------------- routing ----
@@ -247,6 +252,11 @@ FWD_CASES = [
     # H = 2048 + 256: the per-token x quantiser's second stretch is ragged
     ("tiny", dict(T=40, H=2304, E=8, k=3, I=256), 1, False),
     ("tiny", dict(fmt="fp8", T=40, H=2176, E=8, k=3, I=256), 1, False),
+    # BF16 expert weights (tensor cores, kind::f16) in both activation modes,
+    # a shared expert, and a prefill-sized batch with Zipf routing
+    ("tiny", dict(fmt="bf16"), 1, False), ("tiny", dict(fmt="bf16"), 0, False),
+    ("tiny", dict(fmt="bf16", T=24, H=256, E=16, k=4, I=128, shared_I=128), 1, False),
+    ("prefill", dict(fmt="bf16", T=512, H=512, E=32, k=4, I=256), 1, False),
 ]
 
 
