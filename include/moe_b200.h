@@ -145,6 +145,25 @@ size_t moe_prepared_weights_size(const moe_weights* canonical);
 moe_status moe_prepare_weights(const moe_weights* canonical, void* dst, size_t dst_bytes,
                                moe_weights* prepared, moe_stream_t stream);
 
+/* Bytes moe_dequantize_weights() writes for a CANONICAL NVFP4 / MXFP4 / FP8
+ * bank: E*2I*H + E*H*I bf16 values (0 for a BF16 or invalid bank). */
+size_t moe_dequantized_weights_size(const moe_weights* canonical);
+
+/* Load-time expansion of a CANONICAL NVFP4 / MXFP4 / FP8 bank into a
+ * CANONICAL BF16 bank, for bf16-activation (W4A16 / W8A16) prefill on the
+ * bf16 tensor cores: each weight is decoded by its format's definition
+ * (NVFP4 e2m1 * e4m3 * g, MXFP4 e2m1 * 2^(c-127), FP8 e4m3 * s) in fp32 and
+ * rounded once to bf16 (nearest even).  The bank then runs like any BF16
+ * bank (moe_prepare_weights, then the layer): it takes 4x the bytes of the
+ * FP4 bank (2x FP8) in HBM and streams them at that size, so it pays at
+ * prefill, where the layer is compute-bound, not at decode.  Writes into dst
+ * (device, dst_bytes >= moe_dequantized_weights_size()), fills *bf16 (host)
+ * with pointers into dst; static activation scales are dropped (BF16 has
+ * none).  MOE_ERR_UNSUPPORTED for a BF16 bank, MOE_ERR_INVALID_ARG for a
+ * PREPARED one.  Enqueued on `stream`. */
+moe_status moe_dequantize_weights(const moe_weights* canonical, void* dst, size_t dst_bytes, moe_weights* bf16,
+                                  moe_stream_t stream);
+
 /* Quantise `rows` x `K` values into a CANONICAL-layout tensor of format
  * `fmt`, with the same rules the layer applies to activations:
  *   NVFP4: sc = e4m3(bmax/(6 g)), r = 1/(dec(sc) g), q = e2m1(x r)  (16-blocks)

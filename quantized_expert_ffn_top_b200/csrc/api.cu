@@ -617,6 +617,39 @@ size_t moe_prepared_weights_size(const moe_weights* w) {
   return align_up(c.off, kAlign);
 }
 
+size_t moe_dequantized_weights_size(const moe_weights* w) {
+  if (check_weights(w, false) != MOE_OK || w->fmt == MOE_FMT_BF16) return 0;
+  Carver c(nullptr);
+  c.take<uint16_t>((size_t)w->E * 2 * w->I * w->H);
+  c.take<uint16_t>((size_t)w->E * w->H * w->I);
+  return align_up(c.off, kAlign);
+}
+
+moe_status moe_dequantize_weights(const moe_weights* w, void* dst, size_t dst_bytes, moe_weights* out,
+                                  moe_stream_t stream) {
+  moe_status st = check_weights(w, false);
+  if (st != MOE_OK) return st;
+  if (w->fmt == MOE_FMT_BF16) return MOE_ERR_UNSUPPORTED;
+  if (w->layout != MOE_LAYOUT_CANONICAL || !dst || !out) return MOE_ERR_INVALID_ARG;
+  if (dst_bytes < moe_dequantized_weights_size(w)) return MOE_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t E = w->E, H = w->H, I = w->I;
+  Carver c(dst);
+  uint16_t* w13 = c.take<uint16_t>((size_t)(E * 2 * I * H));
+  uint16_t* w2 = c.take<uint16_t>((size_t)(E * H * I));
+  MOE_TRY(launch_dequant_bf16(w->fmt, w->w13, w->w13_sf, w->w13_gs, 2, I, E, 2 * I, H, w13, s));
+  MOE_TRY(launch_dequant_bf16(w->fmt, w->w2, w->w2_sf, w->w2_gs, 1, H, E, H, I, w2, s));
+  *out = *w;
+  out->fmt = MOE_FMT_BF16;
+  out->layout = MOE_LAYOUT_CANONICAL;
+  out->w13 = reinterpret_cast<const uint8_t*>(w13);
+  out->w2 = reinterpret_cast<const uint8_t*>(w2);
+  out->w13_sf = out->w2_sf = nullptr;
+  out->w13_gs = out->w2_gs = nullptr;
+  out->a13_gs = out->a2_gs = nullptr;
+  return MOE_OK;
+}
+
 moe_status moe_prepare_weights(const moe_weights* w, void* dst, size_t dst_bytes, moe_weights* prepared,
                                moe_stream_t stream) {
   moe_status st = check_weights(w, false);

@@ -117,6 +117,8 @@ cudaError_t launch_combine(const uint16_t* y_perm, const int32_t* inv_perm, cons
 // prepare.cu
 cudaError_t launch_prepare_rows(int fmt, const uint8_t* src, uint8_t* dst, int64_t E, int64_t R, int64_t row_bytes,
                                 bool interleave, cudaStream_t s);
+cudaError_t launch_dequant_bf16(int fmt, const uint8_t* codes, const uint8_t* sf, const float* gs, int gstride,
+                                int64_t part_rows, int64_t E, int64_t R, int64_t K, uint16_t* out, cudaStream_t s);
 cudaError_t launch_prepare_sf(const uint8_t* src, uint8_t* dst, int64_t E, int64_t R, int64_t ncols,
                               int64_t ncols_padded, bool interleave, cudaStream_t s);
 

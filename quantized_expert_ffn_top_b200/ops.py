@@ -35,7 +35,7 @@ def row_bytes(fmt: int, K: int) -> int:
 
 EXPORTED = (
     "moe_status_string", "moe_version", "moe_set_option", "moe_workspace_size", "moe_prepared_weights_size",
-    "moe_prepare_weights", "moe_quantize", "moe_route", "moe_route_logits", "moe_permute", "moe_grouped_ffn",
+    "moe_prepare_weights", "moe_dequantize_weights", "moe_dequantized_weights_size", "moe_quantize", "moe_route", "moe_route_logits", "moe_permute", "moe_grouped_ffn",
     "moe_combine", "moe_forward", "moe_get_device_status", "moe_set_stage_events", "moe_kernel_launch_count",
     "moe_permute_fixed_scratch",
 )
@@ -84,6 +84,8 @@ def _declare(L):
         "moe_workspace_size": ([i64, i32, W, W, i32], sz),
         "moe_prepared_weights_size": ([W], sz),
         "moe_prepare_weights": ([W, P, sz, W, P], ctypes.c_int),
+        "moe_dequantized_weights_size": ([W], sz),
+        "moe_dequantize_weights": ([W, P, sz, W, P], ctypes.c_int),
         "moe_quantize": ([i32, P, i32, i64, i64, P, P, P, P, P, sz, P], ctypes.c_int),
         "moe_route": ([P, i64, i32, P, P, i32, i32, P, P, P, P, sz, P], ctypes.c_int),
         "moe_route_logits": ([P, i64, i32, i32, P, P, P, sz, P], ctypes.c_int),
@@ -196,6 +198,23 @@ def moe_prepare_weights(bank: WeightBank, stream=None) -> WeightBank:
                    w13_sf=view(out.w13_sf, bank.E * 2 * bank.I * bank.H // bs) if bs else None,
                    w2_sf=view(out.w2_sf, bank.E * bank.H * bank.I // bs) if bs else None,
                    keep=[dst])
+
+
+def moe_dequantize_weights(bank: WeightBank, stream=None) -> WeightBank:
+    """CANONICAL NVFP4 / MXFP4 / FP8 bank -> CANONICAL BF16 bank (device), for
+    bf16-activation prefill on the bf16 tensor cores."""
+    c = bank.struct()
+    n = lib().moe_dequantized_weights_size(ctypes.byref(c))
+    if n == 0:
+        raise MoeError(2, "moe_dequantized_weights_size")
+    dst = torch.empty(int(n), dtype=torch.uint8, device=bank.w13.device)
+    out = MoeWeightsC()
+    _check(lib().moe_dequantize_weights(ctypes.byref(c), _p(dst), n, ctypes.byref(out), _stream(stream)),
+           "moe_dequantize_weights")
+    E, H, I = bank.E, bank.H, bank.I
+    return WeightBank(FMT_BF16, E, H, I, dst[:E * 2 * I * H * 2], None, None,
+                      dst[out.w2 - dst.data_ptr():out.w2 - dst.data_ptr() + E * H * I * 2], None, None,
+                      keep=[dst])
 
 
 # ------------------------------------------------------------ entry points --

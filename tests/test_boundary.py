@@ -63,6 +63,10 @@ def test_workspace_and_prepared_sizes(L):
     assert L.moe_workspace_size(8, 2, ctypes.byref(bb), None, 1) > 0
     pb = L.moe_prepared_weights_size(ctypes.byref(bb))
     assert 8 * 512 * 256 + 8 * 128 * 512 <= pb < 8 * 512 * 256 + 8 * 128 * 512 + 4096
+    # FP4 -> BF16 expansion: two bytes per weight; none for a BF16 bank
+    d = L.moe_dequantized_weights_size(ctypes.byref(b))
+    assert 2 * (8 * 512 * 128 + 8 * 128 * 256) <= d < 2 * (8 * 512 * 128 + 8 * 128 * 256) + 4096
+    assert L.moe_dequantized_weights_size(ctypes.byref(bb)) == 0
 
 
 def test_host_side_argument_errors(L):

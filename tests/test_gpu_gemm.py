@@ -147,6 +147,44 @@ def test_bf16_weights_match_oracle(name, over, skew, act, tile_n):
     assert max_abs_rel(dev_to_f64(y), ry) < TOL
 
 
+@pytest.mark.parametrize("fmt", ["nvfp4", "mxfp4", "fp8"])
+def test_dequantized_bank_and_a16_layer(fmt):
+    """moe_dequantize_weights: every bf16 weight equals the oracle's decode
+    rounded to bf16 (torch); the bf16-activation layer on the expanded bank
+    (bf16 tensor cores) matches the oracle's A16 layer on the quantised bank."""
+    from tests.gpu_helpers import routed_inputs
+    w = synth.workload("tiny", fmt=fmt, T=96, H=256, E=8, k=2, I=256)
+    W, _ = oracle_bank(w)
+    bf = ops.moe_dequantize_weights(device_bank(W, prepare=False))
+    torch.cuda.synchronize()
+    E, H, I = W.E, W.H, W.I
+
+    def ref_bits(codes, sf, gs, rows, K):
+        d = oracle.dequant(W.fmt, codes, sf, gs, rows, K).astype(np.float32)
+        return torch.from_numpy(d).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+    got13 = bf.w13.cpu().numpy().view(np.uint16).reshape(E, 2 * I, H)
+    got2 = bf.w2.cpu().numpy().view(np.uint16).reshape(E, H, I)
+    for e in range(E):
+        for part in range(2):
+            rows = slice(part * I, (part + 1) * I)
+            sf = None if W.w13_sf is None else W.w13_sf[e, rows]
+            gs = 1.0 if W.w13_gs is None else float(W.w13_gs[e, part])
+            assert np.array_equal(got13[e, rows], ref_bits(W.w13[e, rows], sf, gs, I, H)), (e, part)
+        sf = None if W.w2_sf is None else W.w2_sf[e]
+        gs = 1.0 if W.w2_gs is None else float(W.w2_gs[e])
+        assert np.array_equal(got2[e], ref_bits(W.w2[e], sf, gs, H, I)), e
+    bank = ops.moe_prepare_weights(bf)
+    x, wr, b = routed_inputs(w)
+    ws = ops.new_workspace(ops.workspace_size(w.T, w.k, bank, None, 0))
+    out = ops.moe_forward(bits_to_dev_bf16(x), bits_to_dev_bf16(wr), None if b is None else torch.from_numpy(b).cuda(),
+                          w.k, bank, None, 0, ws)
+    assert ops.moe_get_device_status(ws) == 0
+    r = oracle.moe_forward(x, wr, b, w.k, W, act=oracle.ACT_BF16)
+    keep = ~ambiguous_tokens(r["logits"], w.k, 1e-4, boundary_only=True)
+    assert max_abs_rel(dev_to_f64(out)[keep], r["out"][keep]) < TOL
+
+
 @pytest.mark.parametrize("name,over,static,skew", GEMM_CASES[:4])
 def test_gemm_and_gemv_paths_agree(name, over, static, skew):
     *_, yg, st1 = _run(over, static, skew, 2)
