@@ -268,10 +268,10 @@ bool use_gemm_path(const moe_weights* w, int64_t S, int act) {
 }
 
 // Token tile: 64 wide while the average expert holds fewer than 8 slots
-// (decode: deep weight streaming, small B stages); 192 wide up to 384 slots
-// per expert on average (two accumulator buffers, so one tile's epilogue
-// overlaps the next tile's MMAs); 256 wide beyond, where full tiles
-// dominate.  Arguments only, no device read-back.
+// (decode: deep weight streaming, small B stages), 192 wide beyond (two
+// accumulator buffers, so one tile's epilogue overlaps the next tile's MMAs;
+// measured as fast as or faster than 256 up to the large prefill, with or
+// without CTA pairs).  Arguments only, no device read-back.
 int gemm_tile_n(int64_t S, int E) {
   if (g_gemm_bn) return g_gemm_bn;
   return S < 8 * (int64_t)E ? 64 : 192;

@@ -50,9 +50,14 @@ __device__ __forceinline__ void warp_counts(const int32_t* idx, int64_t S, int64
                                             int32_t* status) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int32_t* my = cnt + warp * E;
+  // the lane's eight slot experts are read up front, in one round trip
+  int ev[kSlotsPerWarp / 32];
+#pragma unroll
+  for (int st = 0; st < kSlotsPerWarp / 32; ++st)
+    ev[st] = slot_expert(idx, S, base + (int64_t)warp * kSlotsPerWarp + st * 32 + lane, E, status);
+#pragma unroll
   for (int st = 0; st < kSlotsPerWarp / 32; ++st) {
-    const int64_t i = base + (int64_t)warp * kSlotsPerWarp + st * 32 + lane;
-    const int e = slot_expert(idx, S, i, E, status);
+    const int e = ev[st];
     const unsigned peers = __match_any_sync(0xffffffffu, e);
     const int leader = __ffs(peers) - 1;
     if (e >= 0 && lane == leader) my[e] += __popc(peers);
@@ -179,8 +184,18 @@ __global__ void __launch_bounds__(kPermWarps * 32) perm_count_kernel(const int32
     *ticket = 0;
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < E; e += blockDim.x)
-    for (int c = 0; c < nchunks; ++c) chunk_counts[(int64_t)c * E + e] += tot[e];
+  // chunk bases: the expert's offset added to the prefixes, eight in flight
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    const int32_t o = tot[e];
+    for (int c0 = 0; c0 < nchunks; c0 += 8) {
+      int32_t v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = c0 + u < nchunks ? __ldcg(chunk_counts + (int64_t)(c0 + u) * E + e) : 0;
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (c0 + u < nchunks) chunk_counts[(int64_t)(c0 + u) * E + e] = v[u] + o;
+    }
+  }
 }
 
 __global__ void __launch_bounds__(kPermWarps * 32) perm_scatter_kernel(const int32_t* __restrict__ idx, int64_t S,
@@ -210,9 +225,14 @@ __global__ void __launch_bounds__(kPermWarps * 32) perm_scatter_kernel(const int
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int32_t* my = cnt + warp * E;
+  int ev[kSlotsPerWarp / 32];
+#pragma unroll
+  for (int st = 0; st < kSlotsPerWarp / 32; ++st)
+    ev[st] = slot_expert(idx, S, base + (int64_t)warp * kSlotsPerWarp + st * 32 + lane, E, nullptr);
+#pragma unroll
   for (int st = 0; st < kSlotsPerWarp / 32; ++st) {
     const int64_t i = base + (int64_t)warp * kSlotsPerWarp + st * 32 + lane;
-    const int e = slot_expert(idx, S, i, E, nullptr);
+    const int e = ev[st];
     const unsigned peers = __match_any_sync(0xffffffffu, e);
     const int leader = __ffs(peers) - 1;
     if (e >= 0) {
