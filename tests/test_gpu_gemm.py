@@ -193,6 +193,27 @@ def test_gemm_and_gemv_paths_agree(name, over, static, skew):
     assert max_abs_rel(yg, yv) < TOL
 
 
+@pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4"])
+def test_long_k_loop_default_options_match_oracle(fmt):
+    """The large prefill's K (H = 4096: 16 stages a tile) with the default
+    options, so the gate|up projection runs on CTA pairs and the down
+    projection on single CTAs, Zipf-like skew, ragged tiles."""
+    w = synth.workload("tiny", fmt=fmt, T=300, H=4096, E=8, k=2, I=512)
+    W, _ = oracle_bank(w)
+    a13, a2 = (None, None) if fmt == "mxfp4" else synth.static_act_scales()
+    bank = device_bank(W, a13, a2)
+    idx = synth.random_topk_idx(w.T, w.k, w.E, skew=1.5)
+    off, perm, inv, _ = oracle.permute(idx, w.E)
+    x = synth.x_bits(w)
+    ws = ops.new_workspace(ops.workspace_size(w.T, w.k, bank, None, 1))
+    y = ops.moe_grouped_ffn(bits_to_dev_bf16(x), w.k, torch.from_numpy(perm).cuda(), torch.from_numpy(off).cuda(),
+                            bank, 1, ws)
+    torch.cuda.synchronize()
+    assert ops.moe_get_device_status(ws) == 0
+    ry, _ = oracle.grouped_ffn(x, perm, off, W, 1, a13 or 0.0, a2 or 0.0)
+    assert max_abs_rel(dev_to_f64(y), ry) < TOL
+
+
 @pytest.fixture(scope="module")
 def prefill_layer():
     w = synth.workload("prefill")

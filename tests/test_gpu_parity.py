@@ -257,6 +257,9 @@ FWD_CASES = [
     ("tiny", dict(fmt="bf16"), 1, False), ("tiny", dict(fmt="bf16"), 0, False),
     ("tiny", dict(fmt="bf16", T=24, H=256, E=16, k=4, I=128, shared_I=128), 1, False),
     ("prefill", dict(fmt="bf16", T=512, H=512, E=32, k=4, I=256), 1, False),
+    # degenerate layers: one expert (k = 1), every expert picked (k = E), one token
+    ("tiny", dict(E=1, k=1, T=16), 1, False), ("tiny", dict(E=4, k=4, T=33), 1, False),
+    ("tiny", dict(T=1), 1, False),
 ]
 
 
@@ -277,3 +280,21 @@ def test_forward_matches_oracle(name, over, act, static):
     keep = ~ambiguous_tokens(r["logits"], w.k, 1e-4, boundary_only=True)
     err = max_abs_rel(dev_to_f64(out)[keep], r["out"][keep])
     assert err < TOL, err
+
+
+def test_forward_and_ffn_with_no_tokens():
+    """T = 0: every entry point returns success and writes nothing."""
+    w = synth.workload("tiny")
+    W, _ = oracle_bank(w)
+    bank = device_bank(W)
+    x = torch.zeros((0, w.H), dtype=torch.bfloat16, device="cuda")
+    wr = bits_to_dev_bf16(synth.router_bits(w))
+    W_ = ws(ops.workspace_size(0, w.k, bank, None, 1))
+    out = ops.moe_forward(x, wr, None, w.k, bank, None, 1, W_)
+    assert out.shape == (0, w.H)
+    off = torch.zeros(w.E + 1, dtype=torch.int32, device="cuda")
+    perm = torch.zeros(0, dtype=torch.int32, device="cuda")
+    y = ops.moe_grouped_ffn(x, w.k, perm, off, bank, 1, W_)
+    assert y.shape == (0, w.H)
+    torch.cuda.synchronize()
+    assert ops.moe_get_device_status(W_) == 0
