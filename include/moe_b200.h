@@ -219,16 +219,21 @@ moe_status moe_permute(const int32_t* topk_idx, int64_t T, int32_t k, int32_t E,
  *   [g | u] = act(x_t) W13_e^T,  h = g / (1 + exp(-g)) * u,
  *   y_perm[p] = act(h) W2_e^T                      (bf16 [S][H], device out)
  * act() is the identity (BF16) or the quantiser of the weights' format
- * (MATCH, see moe_act; the tensor amax of h is taken over all S slots).
- * x [T][H] bf16, perm_token [S], offsets [E+1] (device); w must be
- * PREPARED.  With quantised activations (MATCH) and H, I multiples of 256
- * (FP4) or 128 (FP8) the FFN runs as a tcgen05 block-scaled grouped GEMM at
- * every batch size -- 64-token tiles while T*k < 8E (decode: each active
- * expert's weights stream once), 192- or 256-token tiles beyond (prefill).  BF16
- * activations and other shapes take a TMA-fed mma.sync GEMV that streams
- * each active expert's weights once (the decode split of the atomicmilkshake
- * fork README, "Quant types": MMVQ for decode, MMQ for prefill).  The choice
- * is a host decision on the arguments, never a device read-back. */
+ * (MATCH, see moe_act; the tensor amax of h is taken over all S slots; bf16
+ * rounding for BF16 weights).  x [T][H] bf16, perm_token [S], offsets [E+1]
+ * (device); w must be PREPARED.  With quantised activations (MATCH) and H, I
+ * multiples of 256 (FP4) or 128 (FP8) the FFN runs as a tcgen05 block-scaled
+ * grouped GEMM at every batch size -- 64-token tiles while T*k < 8E (decode:
+ * each active expert's weights stream once; with NVFP4 and a static h scale
+ * or MXFP4 both projections in one kernel, MOE_OPT_FUSED_FFN), 192-token
+ * tiles beyond (prefill; CTA pairs for long K loops, MOE_OPT_GEMM_PAIR).  BF16
+ * weights (H, I multiples of 64) always run the bf16 tcgen05 GEMM.  bf16
+ * activations with FP4/FP8 weights and other shapes take a TMA-fed mma.sync
+ * GEMV that streams each active expert's weights once (the decode split of
+ * the atomicmilkshake fork README, "Quant types": MMVQ for decode, MMQ for
+ * prefill); moe_dequantize_weights gives such layers the tensor cores at
+ * prefill.  The choice is a host decision on the arguments, never a device
+ * read-back. */
 moe_status moe_grouped_ffn(const uint16_t* x, int64_t T, int32_t k, const int32_t* perm_token,
                            const int32_t* offsets, const moe_weights* w, int32_t act, uint16_t* y_perm, void* ws,
                            size_t ws_bytes, moe_stream_t stream);
@@ -265,9 +270,10 @@ moe_status moe_get_device_status(void* ws, moe_stream_t stream, int32_t* host_st
 
 /* Process-wide switches for A/B measurement (the pattern of the
  * FREETOKEN_FP8_ROWWISE_MM variable in FreeToken commit 58f4b9ec0e).
- *   MOE_OPT_FFN_PATH: 0 = heuristic (default), 1 = force the GEMV path,
- *                     2 = force the tensor-core GEMM path (returns
- *                     MOE_ERR_UNSUPPORTED where the shapes do not allow it).
+ *   MOE_OPT_FFN_PATH: 0 = heuristic (default), 1 = force the GEMV path
+ *                     (BF16 weights keep the GEMM), 2 = force the tensor-core
+ *                     GEMM path (returns MOE_ERR_UNSUPPORTED where the shapes
+ *                     do not allow it).
  * Not thread-safe; set before enqueuing. */
 /*   MOE_OPT_GEMM_TILE_N: token-tile width of the tensor-core path: 0 (default:
  *                     64 while T*k < 8E, else 192), 64 (four accumulators),
