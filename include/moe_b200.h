@@ -300,14 +300,22 @@ moe_status moe_get_device_status(void* ws, moe_stream_t stream, int32_t* host_st
  *                     scale, or MXFP4; E <= 256) as one persistent kernel
  *                     in which the down tiles of a token tile start as soon
  *                     as its gate|up tiles are stored; 0 launches the two
- *                     projections separately. */
+ *                     projections separately.
+ *   MOE_OPT_PERMUTE_QUANT: 1 (default) lets moe_forward, when that one-kernel
+ *                     FFN runs on quantised activations and T <= 8, E <= 256
+ *                     and H % 64 == 0, quantise x inside the one-block
+ *                     permutation kernel, and the FFN kernel then derives its
+ *                     tile list from the top-k ids, so its first weight loads
+ *                     overlap the permutation; 0 runs the x quantiser as a
+ *                     kernel of its own.  Results are identical either way. */
 typedef enum {
   MOE_OPT_FFN_PATH = 1,
   MOE_OPT_GEMM_TILE_N = 2,
   MOE_OPT_GEMM_PAIR = 3,
   MOE_OPT_PDL = 4,
   MOE_OPT_EARLY_WEIGHTS = 5,
-  MOE_OPT_FUSED_FFN = 6
+  MOE_OPT_FUSED_FFN = 6,
+  MOE_OPT_PERMUTE_QUANT = 7
 } moe_option;
 moe_status moe_set_option(int32_t option, int32_t value);
 

@@ -48,6 +48,7 @@ Scalars carve_head(Carver& c) {
 
 int g_ffn_path = 0;  // MOE_OPT_FFN_PATH
 static int g_fused_ffn = 1;  // MOE_OPT_FUSED_FFN
+static int g_perm_quant = 1;  // MOE_OPT_PERMUTE_QUANT
 
 // Measurement hook (moe_set_stage_events).
 cudaEvent_t g_stage_events[2 * MOE_STAGE_COUNT];
@@ -277,18 +278,36 @@ int gemm_tile_n(int64_t S, int E) {
   return S < 8 * (int64_t)E ? 64 : 192;
 }
 
+// The gate|up GEMM quantises h in its epilogue when h's scale needs no
+// global reduction (MXFP4, or a static NVFP4 scale; BF16 h is not quantised).
+bool h_in_epilogue(const moe_weights* w) {
+  return w->fmt == MOE_FMT_MXFP4 || w->fmt == MOE_FMT_BF16 || (w->fmt == MOE_FMT_NVFP4 && w->a2_gs);
+}
+
+// Both projections as one kernel: block-scaled FP4 weights, h quantised in
+// the epilogue, 64-token tiles, E <= 256.
+bool ffn_one_kernel(const moe_weights* w, int64_t S) {
+  return g_fused_ffn && h_in_epilogue(w) && (w->fmt == MOE_FMT_NVFP4 || w->fmt == MOE_FMT_MXFP4) &&
+         gemm_tile_n(S, w->E) == 64 && w->E <= kFusedMaxE;
+}
+
+// x_ready: the permutation kernel has already quantised x into the padded
+// rows and zeroed the one-kernel FFN's counters (one_kernel only); the FFN
+// then takes its tile list from the top-k ids (slot_expert).
 moe_status run_gemm_ffn(const uint16_t* x, int64_t T, int64_t S, const int32_t* perm, const int32_t* offsets,
                         const int32_t* inv, int k, const int32_t* slot_expert, const moe_weights* w,
                         uint16_t* y_perm, const FfnScratch& f,
-                        float* x_amax, float* h_amax, int32_t* status, cudaStream_t s, bool mark, bool planned) {
+                        float* x_amax, float* h_amax, int32_t* status, cudaStream_t s, bool mark, bool planned,
+                        bool x_ready) {
   const int E = w->E, H = w->H, I = w->I, fmt = w->fmt;
   const int sms = num_sms();
   const int bn = gemm_tile_n(S, E);
   // gate|up projection + SwiGLU quantise h in the epilogue when its scale
-  // needs no global reduction (MXFP4, or a static NVFP4 scale); with 64-token
-  // tiles the two projections then run as one kernel
-  const bool fused_h = fmt == MOE_FMT_MXFP4 || fmt == MOE_FMT_BF16 || (fmt == MOE_FMT_NVFP4 && w->a2_gs);
-  const bool one_kernel = g_fused_ffn && fused_h && fmt != MOE_FMT_BF16 && bn == 64 && E <= kFusedMaxE;
+  // needs no global reduction; with 64-token tiles the two projections then
+  // run as one kernel
+  const bool fused_h = h_in_epilogue(w);
+  const bool one_kernel = ffn_one_kernel(w, S);
+  if (x_ready && (!one_kernel || !slot_expert || !planned)) return MOE_ERR_INVALID_ARG;
   // without a plan from the permutation, the per-slot x quantiser writes it
   if (mark) stage_mark(MOE_STAGE_ACT_QUANT, false, s);
   QuantPaddedArgs qa;
@@ -324,7 +343,7 @@ moe_status run_gemm_ffn(const uint16_t* x, int64_t T, int64_t S, const int32_t* 
   qa.status = status;
   qa.zero = one_kernel ? f.tile_done : nullptr;   // the one-kernel FFN's counters
   qa.nzero = one_kernel ? (int)max_tiles(S, E) : 0;
-  MOE_TRY(launch_quant_padded(qa, true, fmt, sms, s));
+  if (!x_ready) MOE_TRY(launch_quant_padded(qa, true, fmt, sms, s));
   if (mark) stage_mark(MOE_STAGE_ACT_QUANT, true, s);
   GemmArgs g;
   memset(&g, 0, sizeof(g));
@@ -382,6 +401,7 @@ moe_status run_gemm_ffn(const uint16_t* x, int64_t T, int64_t S, const int32_t* 
     g.w_early = ew == 0 ? 0 : 1;
     FusedArgs fa;
     fa.offsets = offsets;
+    fa.slot_expert = x_ready ? slot_expert : nullptr;   // the offsets are one kernel back then
     fa.S = S;
     fa.P = f.P;
     fa.tile_done = f.tile_done;
@@ -424,12 +444,13 @@ moe_status run_grouped_ffn(const uint16_t* x, int64_t T, int64_t S, const int32_
                            const moe_weights* w, int act, uint16_t* y_perm, const FfnScratch& scratch,
                            float* x_amax, float* h_amax, int32_t* status, cudaStream_t s,
                            bool shared_stage = false, const int32_t* inv = nullptr, int k = 0,
-                           const int32_t* slot_expert = nullptr, bool planned = false) {
+                           const int32_t* slot_expert = nullptr, bool planned = false, bool x_ready = false) {
   if (S == 0) return MOE_OK;
   const bool mark = !shared_stage;
   if (use_gemm_path(w, S, act))
     return run_gemm_ffn(x, T, S, perm, offsets, inv, k, slot_expert, w, y_perm, scratch, x_amax, h_amax, status, s,
-                        mark, planned);
+                        mark, planned, x_ready);
+  if (x_ready) return MOE_ERR_INVALID_ARG;
   if (g_ffn_path == 2 || w->fmt == MOE_FMT_BF16) return MOE_ERR_UNSUPPORTED;   // the GEMV has no BF16 weights
   GemvArgs a;
   a.fmt = w->fmt;
@@ -573,6 +594,11 @@ moe_status moe_set_option(int32_t option, int32_t value) {
   if (option == MOE_OPT_FUSED_FFN) {
     if (value != 0 && value != 1) return MOE_ERR_INVALID_ARG;
     g_fused_ffn = value;
+    return MOE_OK;
+  }
+  if (option == MOE_OPT_PERMUTE_QUANT) {
+    if (value != 0 && value != 1) return MOE_ERR_INVALID_ARG;
+    g_perm_quant = value;
     return MOE_OK;
   }
   if (option == MOE_OPT_EARLY_WEIGHTS) {
@@ -847,17 +873,37 @@ moe_status moe_forward(const uint16_t* x, int64_t T, const uint16_t* wr, const f
   plan.tiles = f.ffn.tiles;
   plan.ntiles = f.ffn.ntiles;
   plan.max_tiles = (int)max_tiles(S, E);
-  bool planned = false;
+  // Small batches on the one-kernel FFN: the one-block permutation also
+  // quantises x, and the FFN takes its tile list from the top-k ids (two
+  // kernels back), so its first weight loads go out while the permutation
+  // runs.
+  SlotQuantOut q;
+  memset(&q, 0, sizeof(q));
+  const bool want_q = g_perm_quant && act == MOE_ACT_MATCH && use_gemm_path(routed, S, act) &&
+                      ffn_one_kernel(routed, S) && H % 64 == 0 && permute_can_quantize(S, T, E);
+  if (want_q) {
+    q.fmt = routed->fmt;
+    q.x = x;
+    q.K = H;
+    q.P = f.ffn.P;
+    q.scale = routed->a13_gs;
+    q.amax = f.head.x_amax;
+    q.codes = f.ffn.xq;
+    q.sf = f.ffn.xsf;
+    q.zero = f.ffn.tile_done;
+    q.nzero = (int)max_tiles(S, E);
+  }
+  bool planned = false, x_ready = false;
   if (st == MOE_OK) {
     stage_mark(MOE_STAGE_PERMUTE, false, s);
-    st = cuda_status(
-        launch_permute(f.idx, S, k, E, f.offsets, f.perm, f.inv, f.pscratch, f.head.status, s, &plan, &planned));
+    st = cuda_status(launch_permute(f.idx, S, k, E, f.offsets, f.perm, f.inv, f.pscratch, f.head.status, s, &plan,
+                                    &planned, want_q ? &q : nullptr, &x_ready));
     stage_mark(MOE_STAGE_PERMUTE, true, s);
   }
   // 5. routed experts
   if (st == MOE_OK)
     st = run_grouped_ffn(x, T, S, f.perm, f.offsets, routed, act, f.y_perm, f.ffn, f.head.x_amax, f.head.h_amax,
-                         f.head.status, s, false, f.inv, k, f.idx, planned);
+                         f.head.status, s, false, f.inv, k, f.idx, planned, x_ready);
   if (shared) {
     const moe_status js = side.join(s);
     if (st == MOE_OK) st = js;

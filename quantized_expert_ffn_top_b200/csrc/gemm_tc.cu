@@ -38,6 +38,7 @@
 #include "kernels.cuh"
 #include "gemm_tc.cuh"
 #include "tc_ptx.cuh"
+#include "token_quant.cuh"
 
 namespace moe {
 namespace {
@@ -110,13 +111,6 @@ __device__ __forceinline__ uint32_t sfb_col_offset(int row0) {
   return (BN == 64 || BN == 192) ? (uint32_t)((row0 & 127) >> 5) : 0u;
 }
 
-__device__ __forceinline__ float act_scale_of(int fmt, const float* st, const float* amax) {
-  if (fmt == MOE_FMT_MXFP4) return 1.0f;
-  if (st) return __ldg(st);
-  if (!amax) return 1.0f;
-  return fmt == MOE_FMT_NVFP4 ? nvfp4_tensor_scale(*amax) : fp8_tensor_scale(*amax);
-}
-
 // Token-operand maps with box heights 16, 32, 64, 128, 256 rows: a tile
 // loads only the rows it covers, rounded up to one of these.
 struct TokenMaps {
@@ -128,7 +122,8 @@ __device__ __forceinline__ int token_box_index(int rows) {
 }
 
 // The plan's tile list held in registers, derived from the compact offsets
-// by one warp (E <= 256): lane l keeps offsets[8l .. 8l+8] and the tiles and
+// (or the per-expert counts) by one warp (E <= 256): lane l keeps
+// offsets[8l .. 8l+8] and the tiles and
 // padded rows of all experts before 8l.  Tile tt of the list is the same
 // entry the plan kernels write: experts in order, ceil(n_e / bn) tiles each,
 // expert segments starting on multiples of 128 padded rows.
@@ -145,14 +140,50 @@ struct WarpPlan {
 #pragma unroll
     for (int j = 0; j < 8; ++j) hi[j] = e0 + j < E ? __ldcg(offsets + e0 + j + 1) : 0;
     bool good = !(lane == 0 && lo0 != 0);
-    int tsum = 0, psum = 0, prev = lo0;
+    int prev = lo0;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       if (e0 + j >= E) hi[j] = prev;
-      const int n = hi[j] - prev;
-      if (n < 0) good = false;
+      if (hi[j] < prev) good = false;
       if (e0 + j == E - 1 && S >= 0 && (int64_t)hi[j] != S) good = false;
-      const int nn = max(n, 0);
+      prev = hi[j];
+    }
+    finish(bn, P, max_tiles, good);
+  }
+  // The same list from the per-expert slot counts cnt[0..E) (shared memory);
+  // bad: a slot named no expert in [0, E).
+  __device__ __forceinline__ void load_counts(const int32_t* cnt, bool bad, int E, int bn, int64_t S, int64_t P,
+                                              int max_tiles) {
+    const int lane = threadIdx.x & 31, e0 = 8 * lane;
+    int sum = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      hi[j] = e0 + j < E ? cnt[e0 + j] : 0;
+      sum += hi[j];
+    }
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int a = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += a;
+    }
+    lo0 = incl - sum;
+    int run = lo0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      run += hi[j];
+      hi[j] = run;
+    }
+    const int total = __shfl_sync(0xffffffffu, incl, 31);
+    finish(bn, P, max_tiles, !bad && (S < 0 || (int64_t)total == S));
+  }
+  // tiles and padded rows before expert 8l, the totals, and the checks
+  __device__ __forceinline__ void finish(int bn, int64_t P, int max_tiles, bool good) {
+    const int lane = threadIdx.x & 31;
+    int tsum = 0, psum = 0, prev = lo0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int nn = max(hi[j] - prev, 0);
       tsum += (nn + bn - 1) / bn;
       psum += (nn + 127) / 128 * 128;
       prev = hi[j];
@@ -863,7 +894,8 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN, PAIR>::kThreads, 1)
 template <int FMT, int BN>
 struct FusedCfg {
   using C = Cfg<FMT, kEpiUpQuant, BN, false>;
-  static constexpr int kSmem = C::kSmem + C::kEpiWarps * 1024;   // + the down store staging
+  // + the down store staging and the expert counts (+ a flag)
+  static constexpr int kSmem = C::kSmem + C::kEpiWarps * 1024 + (kFusedMaxE + 1) * 4;
   static_assert(kSmem <= 227 * 1024, "shared memory");
 };
 
@@ -892,6 +924,7 @@ __global__ void __launch_bounds__(Cfg<FMT, kEpiUpQuant, BN, false>::kThreads, 1)
   // SwiGLU tiles (a warp may start its first down tile while its pair
   // partner still finishes the last gate|up tile)
   uint16_t* y_stage = reinterpret_cast<uint16_t*>(r_tab + 128);
+  int32_t* hist = reinterpret_cast<int32_t*>(y_stage + C::kEpiWarps * 512);  // [kFusedMaxE] counts, bad flag
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -914,6 +947,32 @@ __global__ void __launch_bounds__(Cfg<FMT, kEpiUpQuant, BN, false>::kThreads, 1)
     }
     tc::prefetch_tmap(&tmap_y);
   }
+  if (warp == 0 && f.slot_expert) {
+    // Slot counts per expert from the slots' expert ids: 32 slots per step,
+    // the first lane of each group of equal ids adds the group's size.
+    for (int e = lane; e <= kFusedMaxE; e += 32) hist[e] = 0;
+    __syncwarp();
+    bool bad = false;
+    for (int64_t base = 0; base < f.S; base += 32 * 8) {
+      int ev[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int64_t i = base + 32 * u + lane;
+        ev[u] = i < f.S ? __ldcg(f.slot_expert + i) : -1;
+        if (i < f.S && (ev[u] < 0 || ev[u] >= g1.E)) {
+          bad = true;
+          ev[u] = -1;
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const unsigned peers = __match_any_sync(0xffffffffu, ev[u]);
+        if (ev[u] >= 0 && lane == __ffs(peers) - 1) hist[ev[u]] += __popc(peers);
+        __syncwarp();
+      }
+    }
+    if (__any_sync(0xffffffffu, bad) && lane == 0) hist[kFusedMaxE] = 1;
+  }
   if (warp == 1) {
     tc::tmem_alloc(tmem_slot, C::kTmemCols);
     tc::tmem_relinquish();
@@ -923,10 +982,14 @@ __global__ void __launch_bounds__(Cfg<FMT, kEpiUpQuant, BN, false>::kThreads, 1)
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
 
-  // Every warp derives the tile list itself; the offsets are older than the
-  // previous kernel (they are read before waiting for it).
+  // Every warp derives the tile list itself, from the offsets or from the
+  // slots' expert ids; either is older than the previous kernel (read before
+  // waiting for it).
   WarpPlan plan;
-  plan.load(f.offsets, g1.E, BN, f.S, f.P, f.max_tiles);
+  if (f.slot_expert)
+    plan.load_counts(hist, hist[kFusedMaxE] != 0, g1.E, BN, f.S, f.P, f.max_tiles);
+  else
+    plan.load(f.offsets, g1.E, BN, f.S, f.P, f.max_tiles);
   const int ntok = plan.ok ? plan.ntiles : 0;
   if (!plan.ok && blockIdx.x == 0 && threadIdx.x == 0) raise_status(g1.status, MOE_ERR_DEVICE_FAULT);
   const int MT1 = g1.R / 128, MT2 = g2.R / 128;
@@ -1681,14 +1744,7 @@ __global__ void __launch_bounds__(256) quant_tokens_kernel(QuantPaddedArgs a) {
   if (a.zero && blockIdx.x == 0)
     for (int i = threadIdx.x; i < a.nzero; i += blockDim.x) a.zero[i] = 0;
 
-  constexpr int bs = FMT == MOE_FMT_MXFP4 ? 32 : 16;
-  constexpr int kPer = 64;
-  constexpr int kWords = FMT == MOE_FMT_FP8 ? 16 : 8;  // 32-bit code words per lane
-  constexpr int kLaneBytes = kWords * 4;
-  constexpr int kVec = kLaneBytes / 16;
-  __shared__ uint4 tbuf[8][32 * kVec];  // per warp: the stretch's codes, for the reorder
-  const int nb = a.K / bs;
-  const int lane = threadIdx.x & 31;
+  __shared__ uint4 tbuf[8][TokenQuant<FMT>::kWarpBuf];  // per warp: the stretch's codes, for the reorder
   const float scale = act_scale_of(FMT, a.scale, a.amax);
   const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
   // NVFP4: the multiplier r = 1 / (dec(sc) g) of every non-negative scale code
@@ -1700,7 +1756,6 @@ __global__ void __launch_bounds__(256) quant_tokens_kernel(QuantPaddedArgs a) {
   // padded row of the slot of (token t, pick j): -1 for a dropped slot, -2 if
   // the permutation is inconsistent
   auto resolve = [&](int64_t t, int j) -> int64_t {
-    if (j >= a.k) return -1;
     const int32_t p = __ldg(a.inv_perm + t * a.k + j);
     if (p >= a.S) return -2;
     if (p < 0) return -1;
@@ -1715,113 +1770,9 @@ __global__ void __launch_bounds__(256) quant_tokens_kernel(QuantPaddedArgs a) {
     const int64_t row = (int64_t)__ldg(a.poff + e) + (p - o);
     return (row >= 0 && row < a.P && p >= o && p < o1) ? row : -2;
   };
-  for (int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < a.T; t += warps) {
-    const int64_t row_first = resolve(t, lane);  // issued before the x loads
-    for (int c0 = 0; c0 < a.K; c0 += 32 * kPer) {
-      const int c = c0 + lane * kPer;
-      const bool active = c < a.K;
-      uint32_t w[kWords];
-      uint32_t sfw = 0;
-      if (active) {
-        // the lane's 64 bf16 values stay packed (32 registers); each scale
-        // block is unpacked when it is quantised
-        uint32_t raw[kPer / 2];
-        const uint4* src = reinterpret_cast<const uint4*>(a.x + t * a.K + c);
-#pragma unroll
-        for (int i = 0; i < kPer / 8; ++i) {
-          const uint4 u = __ldg(src + i);
-          raw[4 * i] = u.x;
-          raw[4 * i + 1] = u.y;
-          raw[4 * i + 2] = u.z;
-          raw[4 * i + 3] = u.w;
-        }
-        auto unpack = [&](float* v, int first, int n) {
-#pragma unroll
-          for (int i = 0; i < n / 2; ++i) {
-            v[2 * i] = __uint_as_float(raw[first / 2 + i] << 16);
-            v[2 * i + 1] = __uint_as_float(raw[first / 2 + i] & 0xFFFF0000u);
-          }
-        };
-        if constexpr (FMT == MOE_FMT_NVFP4) {
-#pragma unroll
-          for (int b = 0; b < 4; ++b) {
-            float v[16];
-            unpack(v, 16 * b, 16);
-            float bmax = 0.0f;
-#pragma unroll
-            for (int i = 0; i < 16; ++i) bmax = fmaxf(bmax, fabsf(v[i]));
-            const uint32_t sc = nvfp4_scale_code(bmax, scale);
-            const uint2 cw = nvfp4_encode16(v, r_tab[sc]);
-            w[2 * b] = cw.x;
-            w[2 * b + 1] = cw.y;
-            sfw |= sc << (8 * b);
-          }
-        } else if constexpr (FMT == MOE_FMT_MXFP4) {
-#pragma unroll
-          for (int b = 0; b < 2; ++b) {
-            float v[32];
-            unpack(v, 32 * b, 32);
-            float bmax = 0.0f;
-#pragma unroll
-            for (int i = 0; i < 32; ++i) bmax = fmaxf(bmax, fabsf(v[i]));
-            uint32_t sc;
-            float inv;
-            mxfp4_block_scale(bmax, sc, inv);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) w[4 * b + q] = e2m1_encode8(v + 8 * q, inv);
-            sfw |= sc << (8 * b);
-          }
-        } else {
-          const float inv = __frcp_rn(scale);
-#pragma unroll
-          for (int i = 0; i < kWords; ++i) {
-            float v[4];
-            unpack(v, 4 * i, 4);
-            w[i] = e4m3x2_encode(__fmul_rn(v[0], inv), __fmul_rn(v[1], inv)) |
-                   (e4m3x2_encode(__fmul_rn(v[2], inv), __fmul_rn(v[3], inv)) << 16);
-          }
-        }
-      }
-      // Codes in store order: lane l's 16-byte pieces v are bytes 512 v + 16 l
-      // of the stretch, so every store instruction covers 512 contiguous bytes.
-      uint4* tb = tbuf[threadIdx.x >> 5];
-      if (active) {
-#pragma unroll
-        for (int v = 0; v < kVec; ++v) tb[lane * kVec + v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
-      }
-      __syncwarp();
-      const int seg = min(a.K - c0, 32 * kPer) * kLaneBytes / kPer;  // code bytes in this stretch
-      uint4 wc[kVec];
-#pragma unroll
-      for (int v = 0; v < kVec; ++v) {
-        const int off = 512 * v + 16 * lane;
-        wc[v] = off < seg ? tb[off / 16] : make_uint4(0, 0, 0, 0);
-      }
-      __syncwarp();
-      for (int j0 = 0; j0 < a.k; j0 += 32) {
-        // lane j resolves the padded row of slot j0 + j (-1: dropped slot, -2: bad)
-        const int64_t myrow = (j0 == 0) ? row_first : resolve(t, j0 + lane);
-        const int nj = min(32, a.k - j0);
-        for (int jj = 0; jj < nj; ++jj) {
-          const int64_t row = __shfl_sync(0xffffffffu, myrow, jj);
-          if (row < 0) {
-            if (row == -2 && lane == 0 && c0 == 0) raise_status(a.status, MOE_ERR_DEVICE_FAULT);
-            continue;
-          }
-          uint4* dst = reinterpret_cast<uint4*>(a.codes + row * ((int64_t)a.K * kLaneBytes / kPer) +
-                                                (int64_t)c0 * kLaneBytes / kPer);
-#pragma unroll
-          for (int v = 0; v < kVec; ++v)
-            if (512 * v + 16 * lane < seg) dst[(512 * v) / 16 + lane] = wc[v];
-          if (!active) continue;
-          if constexpr (FMT == MOE_FMT_NVFP4)
-            *reinterpret_cast<uint32_t*>(a.sf + sf_blocked_offset(row, c / bs, nb)) = sfw;
-          else if constexpr (FMT == MOE_FMT_MXFP4)
-            *reinterpret_cast<uint16_t*>(a.sf + sf_blocked_offset(row, c / bs, nb)) = (uint16_t)sfw;
-        }
-      }
-    }
-  }
+  for (int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < a.T; t += warps)
+    quant_token_slots<FMT>(a.x + t * a.K, a.K, a.k, scale, r_tab, tbuf[threadIdx.x >> 5],
+                           [&](int j) { return resolve(t, j); }, a.codes, a.sf, a.status);
 }
 
 cudaError_t launch_quant_padded(const QuantPaddedArgs& a, bool src_x, int fmt, int num_sms, cudaStream_t s) {

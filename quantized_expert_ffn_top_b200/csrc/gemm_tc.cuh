@@ -81,9 +81,13 @@ struct QuantPaddedArgs {
 // The expert FFN as one persistent kernel (gate|up + SwiGLU + h quantisation,
 // then down), for 64-token tiles: each CTA runs its gate|up tiles, then its
 // down tiles; a down tile's token operand waits for the gate|up slices of its
-// token tile, counted in tile_done.  The tile list comes from the offsets.
+// token tile, counted in tile_done.  The tile list comes from the offsets,
+// or, when slot_expert is given, from the slots' expert ids: the top-k ids
+// are then read before the wait on the previous kernel, so that kernel may
+// be the one that writes the offsets.
 struct FusedArgs {
   const int32_t* offsets;      // [E+1] compact (E <= 256)
+  const int32_t* slot_expert;  // optional: [S] expert of each slot (flat top-k ids), all in [0, E)
   int64_t S;                   // slots: offsets[E]
   int64_t P;                   // padded rows allocated for x and h
   int32_t* tile_done;          // [max_tiles], zero on entry

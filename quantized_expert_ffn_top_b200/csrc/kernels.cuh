@@ -76,11 +76,30 @@ struct PlanOut {
   int32_t* ntiles;
   int max_tiles;
 };
+// x quantisation (MATCH mode) the one-block permutation can run once it has
+// placed the slots: every token row is quantised once into the padded rows
+// of its slots (the plan's padded offsets, so it needs plan.bn > 0).
+struct SlotQuantOut {
+  int fmt;                 // MOE_FMT_NVFP4, MOE_FMT_MXFP4 or MOE_FMT_FP8
+  const uint16_t* x;       // [T][K] bf16, T = S / k
+  int K;                   // a multiple of 64
+  int64_t P;               // padded rows allocated for the codes
+  const float* scale;      // static per-tensor scale, or NULL
+  const float* amax;       // dynamic: amax(x)
+  uint8_t* codes;          // [P][K/2 | K]
+  uint8_t* sf;             // blocked block scales
+  int32_t* zero;           // optional: nzero counters set to 0
+  int nzero;
+};
 // *planned (nullable) tells whether `plan` was written; if not, the caller
-// runs the plan kernel itself.
+// runs the plan kernel itself.  *quantized (nullable) tells whether the x
+// quantisation `quant` asked for was done.
 cudaError_t launch_permute(const int32_t* idx, int64_t S, int k, int E, int32_t* offsets, int32_t* perm_token,
                            int32_t* inv_perm, PermuteScratch scratch, int32_t* status, cudaStream_t s,
-                           const PlanOut* plan, bool* planned);
+                           const PlanOut* plan, bool* planned, const SlotQuantOut* quant = nullptr,
+                           bool* quantized = nullptr);
+// Whether launch_permute can quantise x in its one-block pass for S slots.
+bool permute_can_quantize(int64_t S, int64_t T, int E);
 
 // gemv.cu -- small-batch expert FFN (one pass over each active expert).
 struct GemvArgs {

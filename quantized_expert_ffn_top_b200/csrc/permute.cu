@@ -25,6 +25,7 @@
 
 #include "gemm_tc.cuh"
 #include "kernels.cuh"
+#include "token_quant.cuh"
 
 namespace moe {
 
@@ -256,6 +257,12 @@ __global__ void __launch_bounds__(kPermWarps * 32) perm_scatter_kernel(const int
 // same per-expert counts.
 constexpr int kBlockWarps = 32;
 constexpr int64_t kBlockMaxS = 8192;   // beyond, one SM's scattered stores are the bottleneck
+// x quantisation inside the block: a warp per token.  One SM then moves
+// every token's bytes (about 12 KB a token at H = 2048, k = 8), so it pays
+// only for the smallest batches: measured 2 us faster than the separate
+// quantiser at T = 4 and 6 us slower at T = 32.
+constexpr int64_t kBlockQuantMaxT = 8;
+constexpr int kBlockQuantMaxE = 256;
 
 // Exclusive scan of one value per thread over a 1024-thread block; *total
 // receives the sum.  Every thread calls it.
@@ -297,16 +304,32 @@ __device__ __forceinline__ void load4(const int32_t* idx, int64_t S, int64_t bas
   }
 }
 
+// Dynamic shared memory of the one-block kernel: the per-warp counters and
+// the offsets ([kBlockWarps + 1][E] ints); with the x quantisation also the
+// padded offsets ([E]), then, from the next 16-byte boundary, the warps'
+// reorder buffers and the NVFP4 multiplier table.
+constexpr size_t block_quant_buf_offset(int E) { return ((size_t)(kBlockWarps + 2) * E * 4 + 15) / 16 * 16; }
+template <int QFMT>
+constexpr size_t block_smem_bytes(int E) {
+  return QFMT == 0 ? (size_t)(kBlockWarps + 1) * E * 4
+                   : block_quant_buf_offset(E) + (size_t)kBlockWarps * TokenQuant<QFMT>::kWarpBuf * 16 + 128 * 4;
+}
+
+// QFMT != 0: after placing the slots, the block also quantises x (format
+// QFMT) into the padded rows of the slots, as the per-token x quantiser does.
+template <int QFMT>
 __global__ void __launch_bounds__(kBlockWarps * 32) perm_block_kernel(const int32_t* __restrict__ idx, int64_t S,
                                                                      int k, int E, int32_t* __restrict__ offsets,
                                                                      int32_t* __restrict__ perm_token,
                                                                      int32_t* __restrict__ inv_perm,
-                                                                     int32_t* status, PlanOut plan) {
+                                                                     int32_t* status, PlanOut plan, SlotQuantOut q) {
   pdl_wait();  // inputs come from the previous kernels
   pdl_trigger();
 
-  extern __shared__ int32_t cnt[];  // [kBlockWarps][E], then [E] offsets
+  extern __shared__ __align__(16) int32_t blk_smem[];
+  int32_t* cnt = blk_smem;  // [kBlockWarps][E], then [E] offsets (then the quantisation's part)
   int32_t* tot = cnt + kBlockWarps * E;
+  int32_t* pofs = tot + E;  // QFMT: [E] padded offsets
   __shared__ int32_t warp_tot[33];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t per = ((S + kBlockWarps - 1) / kBlockWarps + 127) / 128 * 128;  // slots per warp
@@ -355,6 +378,7 @@ __global__ void __launch_bounds__(kBlockWarps * 32) perm_block_kernel(const int3
     const int32_t tbase = block_scan_excl(til, warp_tot, &til_total);
     if (e < E) {
       plan.poff[e] = pbase;
+      if (QFMT != 0) pofs[e] = pbase;
       for (int j = 0; j < til && tbase + j < plan.max_tiles; ++j) {
         TileEntry te;
         te.e = e;
@@ -392,30 +416,91 @@ __global__ void __launch_bounds__(kBlockWarps * 32) perm_block_kernel(const int3
       __syncwarp();
     }
   }
+  if constexpr (QFMT != 0) {
+    using Q = TokenQuant<QFMT>;
+    uint4* tbuf = reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(cnt) + block_quant_buf_offset(E));
+    float* r_tab = reinterpret_cast<float*>(tbuf + kBlockWarps * Q::kWarpBuf);
+    const float scale = act_scale_of(QFMT, q.scale, q.amax);
+    if (QFMT == MOE_FMT_NVFP4 && threadIdx.x < 128) r_tab[threadIdx.x] = nvfp4_multiplier(threadIdx.x, scale);
+    for (int i = threadIdx.x; i < q.nzero; i += blockDim.x) q.zero[i] = 0;
+    __syncthreads();  // inv_perm (global, this block's stores), padded offsets, table
+    const int64_t T = S / k;
+    for (int64_t t = warp; t < T; t += kBlockWarps) {
+      // padded row of slot (t, j): the slot's rank in its expert past the
+      // expert's first padded row
+      auto row_of = [&](int j) -> int64_t {
+        const int64_t i = t * k + j;
+        const int32_t p = __ldcg(inv_perm + i);
+        if (p < 0) return -1;
+        const int e = __ldg(idx + i);
+        if (e < 0 || e >= E) return -2;
+        const int64_t row = (int64_t)pofs[e] + (p - tot[e]);
+        return (row >= 0 && row < q.P) ? row : -2;
+      };
+      quant_token_slots<QFMT>(q.x + t * q.K, q.K, k, scale, r_tab, tbuf + warp * Q::kWarpBuf, row_of, q.codes,
+                              q.sf, status);
+    }
+  }
+}
+
+bool permute_can_quantize(int64_t S, int64_t T, int E) {
+  return S > 0 && S <= kBlockMaxS && T <= kBlockQuantMaxT && E <= kBlockQuantMaxE;
+}
+
+template <int QFMT>
+cudaError_t launch_perm_block(const int32_t* idx, int64_t S, int k, int E, int32_t* offsets, int32_t* perm_token,
+                              int32_t* inv_perm, int32_t* status, cudaStream_t s, const PlanOut& p,
+                              const SlotQuantOut& q) {
+  const size_t smem = block_smem_bytes<QFMT>(E);
+  // E <= 1024 needs at most 132 KB without the quantisation, E <= 256 at
+  // most 99 KB with it
+  const size_t smem_max = block_smem_bytes<QFMT>(QFMT == 0 ? 1024 : kBlockQuantMaxE);
+  cudaError_t e = cudaFuncSetAttribute(perm_block_kernel<QFMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem_max);
+  if (e != cudaSuccess) return e;
+  e = launch_pdl(perm_block_kernel<QFMT>, dim3(1), dim3(kBlockWarps * 32), smem, s, idx, S, k, E, offsets,
+                 perm_token, inv_perm, status, p, q);
+  if (e != cudaSuccess) return e;
+  count_launches(1);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_permute(const int32_t* idx, int64_t S, int k, int E, int32_t* offsets, int32_t* perm_token,
                            int32_t* inv_perm, PermuteScratch scratch, int32_t* status, cudaStream_t s,
-                           const PlanOut* plan, bool* planned) {
+                           const PlanOut* plan, bool* planned, const SlotQuantOut* quant, bool* quantized) {
   if (planned) *planned = false;
-  const size_t block_smem = sizeof(int32_t) * (size_t)(kBlockWarps + 1) * E;
+  if (quantized) *quantized = false;
   if (S > 0 && S <= kBlockMaxS) {
-    // E <= 1024 needs at most 132 KB
-    cudaError_t e = cudaFuncSetAttribute(perm_block_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)(sizeof(int32_t) * (kBlockWarps + 1) * 1024));
-    if (e != cudaSuccess) return e;
     PlanOut p;
     if (plan) {
       p = *plan;
     } else {
       memset(&p, 0, sizeof(p));
     }
-    e = launch_pdl(perm_block_kernel, dim3(1), dim3(kBlockWarps * 32), block_smem, s, idx, S, k, E, offsets, perm_token,
-                   inv_perm, status, p);
+    SlotQuantOut q;
+    memset(&q, 0, sizeof(q));
+    const bool with_q = quant && p.bn > 0 && quant->K % 64 == 0 && permute_can_quantize(S, S / k, E);
+    if (with_q) q = *quant;
+    cudaError_t e;
+    switch (with_q ? q.fmt : 0) {
+      case MOE_FMT_NVFP4:
+        e = launch_perm_block<MOE_FMT_NVFP4>(idx, S, k, E, offsets, perm_token, inv_perm, status, s, p, q);
+        break;
+      case MOE_FMT_MXFP4:
+        e = launch_perm_block<MOE_FMT_MXFP4>(idx, S, k, E, offsets, perm_token, inv_perm, status, s, p, q);
+        break;
+      case MOE_FMT_FP8:
+        e = launch_perm_block<MOE_FMT_FP8>(idx, S, k, E, offsets, perm_token, inv_perm, status, s, p, q);
+        break;
+      default:
+        e = launch_perm_block<0>(idx, S, k, E, offsets, perm_token, inv_perm, status, s, p, q);
+        q.fmt = 0;
+        break;
+    }
     if (e != cudaSuccess) return e;
-    count_launches(1);
     if (planned && plan && plan->bn > 0) *planned = true;
-    return cudaGetLastError();
+    if (quantized) *quantized = with_q && q.fmt != 0;
+    return cudaSuccess;
   }
   const int nchunks = (int)((S + kChunk - 1) / kChunk);
   if (nchunks == 0) {

@@ -26,6 +26,7 @@ OPT_GEMM_PAIR = 3
 OPT_PDL = 4
 OPT_EARLY_WEIGHTS = 5
 OPT_FUSED_FFN = 6
+OPT_PERMUTE_QUANT = 7
 FMT_BY_NAME = {"nvfp4": FMT_NVFP4, "mxfp4": FMT_MXFP4, "fp8": FMT_FP8, "bf16": FMT_BF16}
 
 

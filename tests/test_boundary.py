@@ -108,5 +108,7 @@ def test_host_side_argument_errors(L):
     # fused FFN on or off
     assert L.moe_set_option(6, 2) == 1
     assert L.moe_set_option(6, 0) == 0 and L.moe_set_option(6, 1) == 0
+    assert L.moe_set_option(7, 2) == 1 and L.moe_set_option(7, -1) == 1
+    assert L.moe_set_option(7, 0) == 0 and L.moe_set_option(7, 1) == 0
     # combine: k beyond the 1024 the kernel stages
     assert L.moe_combine(one, one, one, 1, 1025, 8, None, one, one, 1 << 20, None) == 1

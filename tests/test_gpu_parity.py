@@ -282,6 +282,57 @@ def test_forward_matches_oracle(name, over, act, static):
     assert err < TOL, err
 
 
+# small batches (T <= 8) on the one-kernel FFN (tensor-core shapes: H and I
+# multiples of 256): x quantised inside the permutation kernel (NVFP4 static
+# and dynamic x scales; MXFP4 with a ragged second 2048-value stretch and at
+# E = 256; a single slot)
+PERM_QUANT_CASES = [
+    ("decode", {}, "static"),
+    ("tiny", dict(H=256), "h-static"),
+    ("tiny", dict(fmt="mxfp4", T=7, H=256, E=8, k=2, I=256), "none"),
+    ("tiny", dict(fmt="mxfp4", T=8, H=2304, E=32, k=2, I=256), "none"),
+    ("tiny", dict(fmt="mxfp4", T=8, H=256, E=256, k=8, I=256), "none"),
+    ("tiny", dict(T=1, k=1, E=8, H=256), "static"),
+]
+
+
+@pytest.mark.parametrize("name,over,scales", PERM_QUANT_CASES)
+def test_permutation_with_x_quantisation_changes_nothing(name, over, scales):
+    """The permutation kernel that also quantises x (and the FFN kernel that
+    then takes its tile list from the top-k ids) gives the bits of the
+    separate x quantiser, with one kernel launch fewer."""
+    w = synth.workload(name, **over)
+    W, _ = oracle_bank(w)
+    a13, a2 = synth.static_act_scales()
+    if scales == "h-static":
+        a13 = None
+    elif scales == "none":
+        a13 = a2 = None
+    bank = device_bank(W, a13, a2)
+    x, wr, b = routed_inputs(w)
+    xd, wrd = bits_to_dev_bf16(x), bits_to_dev_bf16(wr)
+    bd = None if b is None else torch.from_numpy(b).cuda()
+    W_ = ws(ops.workspace_size(w.T, w.k, bank, None, 1))
+    outs, launches = [], []
+    try:
+        for opt in (0, 1):
+            ops.moe_set_option(ops.OPT_PERMUTE_QUANT, opt)
+            n0 = ops.moe_kernel_launch_count()
+            out = ops.moe_forward(xd, wrd, bd, w.k, bank, None, 1, W_)
+            launches.append(ops.moe_kernel_launch_count() - n0)
+            assert ops.moe_get_device_status(W_) == 0, opt
+            outs.append(out.view(torch.int16).cpu().numpy())
+    finally:
+        ops.moe_set_option(ops.OPT_PERMUTE_QUANT, 1)
+    assert np.array_equal(outs[0], outs[1])
+    assert launches[1] == launches[0] - 1, launches
+    r = oracle.moe_forward(x, wr, b, w.k, W, None, act=1, a13_static=a13 or 0.0, a2_static=a2 or 0.0)
+    keep = ~ambiguous_tokens(r["logits"], w.k, 1e-4, boundary_only=True)
+    got = outs[1].view(np.uint16).astype(np.uint32) << 16
+    err = max_abs_rel(got.view(np.float32).astype(np.float64)[keep], r["out"][keep])
+    assert err < TOL, err
+
+
 def test_forward_and_ffn_with_no_tokens():
     """T = 0: every entry point returns success and writes nothing."""
     w = synth.workload("tiny")
