@@ -19,7 +19,9 @@ Rank 0 prints one JSON line.  Besides the contract keys it carries:
   stages       per-stage device time (ms) from the library's stage events
   roofline     the dominant stage against the measured peak
   e2e          the same metric with the input copied from pinned host memory
-               and the output copied back inside the timed region
+               and the output copied back inside the timed region, through
+               moe_forward_host (token slices whose copies overlap the other
+               slices' forwards; checked against the device-resident output)
   decode       the decode workload (T=4, static activation scales): step time
                and the expert-weight streaming rate of moe_grouped_ffn (GB/s)
   configs      the FP8 W8A8 + shared-expert and the large MXFP4 workloads:
@@ -61,6 +63,7 @@ def parse():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-configs", action="store_true", help="skip the per-config report (fp8_shared, large)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
+    ap.add_argument("--e2e-slices", type=int, default=4, help="token slices of the end-to-end leg")
     ap.add_argument("--profile-range", action="store_true",
                     help="bracket the timed prefill replays with cudaProfilerStart/Stop (for ncu --profile-from-start off)")
     return ap.parse_args()
@@ -298,6 +301,45 @@ def time_forward(ops, torch, layer, w, act, steps, warmup, flush, stage=True, ho
                 status=ops.moe_get_device_status(ws))
 
 
+def time_forward_host(ops, torch, layer, w, act, steps, warmup, flush, n_slices):
+    """Times `steps` calls of moe_forward_host (pinned host x in, host out
+    back, n_slices token slices) with CUDA events on the caller's stream,
+    which the call joins after its last copy-out.  Returns the step times
+    and the number of tokens whose output differs from the device-resident
+    forward's by more than the layer tolerance (a slice may route a token
+    whose top-k logits tie within rounding differently)."""
+    prepared, x, wr, bias, shared = layer
+    Ts = -(-w.T // n_slices)
+    ws = ops.new_workspace(ops.workspace_size(Ts, w.k, prepared, shared, act))
+    ref = ops.moe_forward(x, wr, bias, w.k, prepared, shared, act,
+                          ops.new_workspace(ops.workspace_size(w.T, w.k, prepared, shared, act)))
+    x_host = x.cpu().pin_memory()
+    out_host = torch.empty(x.shape, dtype=x.dtype).pin_memory()
+    x_dev, out_dev = torch.empty_like(x), torch.empty_like(x)
+    stream = torch.cuda.current_stream()
+
+    def fwd():
+        ops.moe_forward_host(x_host, wr, bias, w.k, prepared, shared, act, ws, x_dev, out_dev, out_host,
+                             n_slices=n_slices)
+
+    for _ in range(max(warmup, 1)):
+        fwd()
+    torch.cuda.synchronize()
+    if ops.moe_get_device_status(ws) != 0:
+        raise RuntimeError("device status reported a fault in moe_forward_host")
+    r = ref.float().cpu()
+    err = ((out_host.float() - r).abs().amax(dim=1) / r.abs().max().clamp_min(1e-30)).numpy()
+    bad = int((err > 2e-2).sum())
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for i in range(steps):
+        flush.zero_()
+        evs[i][0].record(stream)
+        fwd()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    return dict(ms=[a.elapsed_time(b) for a, b in evs], bad_tokens=bad)
+
+
 def time_grouped_ffn(ops, torch, layer, w, act, steps, warmup, flush):
     """Device time of the grouped expert FFN alone (moe_grouped_ffn: tile
     plan, activation quantisation, gate|up + SwiGLU, down) on the layer's
@@ -502,12 +544,25 @@ def main():
     ms = total_s * 1e3 / args.steps
     value = job_throughput(w.T, args.steps, world, total_s)
 
-    # end to end: pinned host input -> device -> forward -> host output
+    # end to end: pinned host input -> device -> forward -> host output, in
+    # token slices whose copies overlap the other slices' forwards; the
+    # whole batch after one copy when that path fails its check
     barrier()
-    res_e2e = time_forward(ops, torch, layer, w, act, args.steps, 2, flush, stage=False, host_io=True)
+    method = f"moe_forward_host, {args.e2e_slices} token slices"
+    try:
+        res_e2e = time_forward_host(ops, torch, layer, w, act, args.steps, 2, flush, args.e2e_slices)
+        if res_e2e["bad_tokens"] > max(1, w.T // 1000):
+            raise RuntimeError(f"{res_e2e['bad_tokens']} tokens differ from the device-resident forward")
+    except (RuntimeError, ops.MoeError) as exc:
+        method = f"copy in, moe_forward, copy out (sliced path not used: {exc})"
+        res_e2e = time_forward(ops, torch, layer, w, act, args.steps, 2, flush, stage=False, host_io=True)
+    # whether any rank fell back (every rank runs this collective once)
+    fell_back = max_over_ranks(0.0 if method.startswith("moe_forward_host") else 1.0) > 0
     e2e_s = max_over_ranks(float(np.sum(res_e2e["ms"])) / 1e3)
     e2e = {"value": job_throughput(w.T, args.steps, world, e2e_s), "unit": "tokens/s",
-           "h2d_bytes_per_step": w.T * w.H * 2, "d2h_bytes_per_step": w.T * w.H * 2}
+           "h2d_bytes_per_step": w.T * w.H * 2, "d2h_bytes_per_step": w.T * w.H * 2, "method": method}
+    if not fell_back:
+        e2e["tokens_off_by_routing_ties"] = res_e2e["bad_tokens"]
 
     alg = algorithmic(w, w.fmt, res["offsets"])
     stages = res["stages"]

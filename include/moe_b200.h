@@ -12,6 +12,7 @@
  *            quantised weights of the slot's expert          moe_grouped_ffn
  *   out_t  = sum_j w[t,j] y_{inv_perm[t*k+j]} (+ shared_t)    moe_combine
  *   all of the above, enqueued as one call                   moe_forward
+ *   the same from host buffers, copies overlapped            moe_forward_host
  *
  * Conventions shared by every entry point
  *  - Pointers marked (device) are CUDA device pointers; (host) are host
@@ -261,6 +262,36 @@ moe_status moe_combine(const uint16_t* y_perm, const int32_t* inv_perm, const fl
 moe_status moe_forward(const uint16_t* x, int64_t T, const uint16_t* wr, const float* bias, int32_t k,
                        const moe_weights* routed, const moe_weights* shared, int32_t act, uint16_t* out, void* ws,
                        size_t ws_bytes, moe_stream_t stream);
+
+/* moe_forward on host buffers, with the copies overlapped.  This entry point
+ * is an engineering addition: the pages run the layer on activations already
+ * on the device.  x_host and out_host ([T][H] bf16, host) are copied through
+ * the caller's device staging buffers x_dev and out_dev ([T][H] bf16 each,
+ * 16-byte aligned).  The batch is cut into n_slices (1 ..
+ * MOE_MAX_HOST_SLICES) slices of ceil(T / n_slices) consecutive tokens.
+ * Slice i is copied in on a library-owned copy stream, run through
+ * moe_forward on `stream` once it has landed, and copied out on a second
+ * copy stream once its forward is done.  The copies of one slice therefore
+ * overlap the forward of another, provided the host buffers are page-locked
+ * (pageable ones work but do not overlap).  `stream` waits for the last
+ * copy-out, so synchronise `stream` before reading out_host.  The call
+ * itself only enqueues.  Each token's result is that of a forward of its
+ * slice:
+ *  - When an activation's tensor scale is derived from the batch (MATCH with
+ *    NVFP4 or FP8 weights and no a13_gs or no a2_gs), tokens are not
+ *    independent, and the batch is run as one slice.
+ *  - Otherwise a token's result equals its whole-batch result up to the
+ *    router's summation order: the router may split its K loop differently
+ *    at another batch size, which can flip a top-k choice whose logits tie
+ *    to within rounding.
+ * ws: at least moe_workspace_size(ceil(T / n_slices), k, routed, shared,
+ * act) bytes; the slices' forwards reuse it one after the other.  Argument
+ * errors return before anything is enqueued. */
+#define MOE_MAX_HOST_SLICES 64
+moe_status moe_forward_host(const uint16_t* x_host, int64_t T, const uint16_t* wr, const float* bias, int32_t k,
+                            const moe_weights* routed, const moe_weights* shared, int32_t act, uint16_t* out_host,
+                            uint16_t* x_dev, uint16_t* out_dev, int32_t n_slices, void* ws, size_t ws_bytes,
+                            moe_stream_t stream);
 
 /* Synchronises `stream`, copies the device status word of `ws` into
  * *host_status (a moe_status value: MOE_OK, MOE_ERR_DEVICE_FAULT or

@@ -538,6 +538,42 @@ bool dynamic_x_scale(const moe_weights* w, int act) {
   return act == MOE_ACT_MATCH && (w->fmt == MOE_FMT_NVFP4 || w->fmt == MOE_FMT_FP8) && !w->a13_gs;
 }
 
+// Whether an activation's tensor scale is derived from the whole batch (x's
+// with x scale a13, or h's), so that a token's result depends on the others.
+bool batch_scaled(const moe_weights* w, const float* a13, int act) {
+  return act == MOE_ACT_MATCH && (w->fmt == MOE_FMT_NVFP4 || w->fmt == MOE_FMT_FP8) && (!a13 || !w->a2_gs);
+}
+
+// The copy-in and copy-out streams of moe_forward_host, one pair per device.
+moe_status copy_streams(cudaStream_t* in, cudaStream_t* out) {
+  static cudaStream_t s_in[64], s_out[64];
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MOE_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!s_in[dev] && cudaStreamCreateWithFlags(&s_in[dev], cudaStreamNonBlocking) != cudaSuccess) return MOE_ERR_CUDA;
+  if (!s_out[dev] && cudaStreamCreateWithFlags(&s_out[dev], cudaStreamNonBlocking) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  *in = s_in[dev];
+  *out = s_out[dev];
+  return MOE_OK;
+}
+
+// Events of one moe_forward_host call, released when it returns (the driver
+// frees a pending event's resources once it completes).
+struct EventSet {
+  cudaEvent_t ev[2 * MOE_MAX_HOST_SLICES + 2] = {};
+  int n = 0;
+  moe_status create(int count) {
+    for (; n < count; ++n)
+      if (cudaEventCreateWithFlags(&ev[n], cudaEventDisableTiming) != cudaSuccess) return MOE_ERR_CUDA;
+    return MOE_OK;
+  }
+  ~EventSet() {
+    for (int i = 0; i < n; ++i) cudaEventDestroy(ev[i]);
+  }
+};
+
 }  // namespace
 
 static int g_pdl = 1;  // MOE_OPT_PDL
@@ -913,6 +949,76 @@ moe_status moe_forward(const uint16_t* x, int64_t T, const uint16_t* wr, const f
   stage_mark(MOE_STAGE_COMBINE, false, s);
   st = cuda_status(launch_combine(f.y_perm, f.inv, f.w, T, k, H, f.sh_y, out, f.head.status, s));
   stage_mark(MOE_STAGE_COMBINE, true, s);
+  return st;
+}
+
+moe_status moe_forward_host(const uint16_t* x_host, int64_t T, const uint16_t* wr, const float* bias, int32_t k,
+                            const moe_weights* routed, const moe_weights* shared, int32_t act, uint16_t* out_host,
+                            uint16_t* x_dev, uint16_t* out_dev, int32_t n_slices, void* ws, size_t ws_bytes,
+                            moe_stream_t stream) {
+  moe_status st = check_weights(routed, true);
+  if (st != MOE_OK) return st;
+  if (shared) {
+    st = check_weights(shared, true);
+    if (st != MOE_OK) return st;
+    if (shared->E != 1 || shared->H != routed->H || shared->fmt != routed->fmt) return MOE_ERR_INVALID_ARG;
+  }
+  const int64_t H = routed->H;
+  if (T < 0 || k < 1 || k > routed->E || (act != MOE_ACT_BF16 && act != MOE_ACT_MATCH)) return MOE_ERR_INVALID_ARG;
+  if (T * (int64_t)k > INT32_MAX || n_slices < 1 || n_slices > MOE_MAX_HOST_SLICES) return MOE_ERR_INVALID_ARG;
+  if (T > 0 && (!x_host || !out_host || !x_dev || !out_dev || !wr)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x_dev) || !aligned16(out_dev) || !aligned16(wr) || (H * 2) % 16 != 0) return MOE_ERR_INVALID_ARG;
+  // one slice when a tensor scale depends on the whole batch
+  int64_t n = n_slices;
+  if (batch_scaled(routed, routed->a13_gs, act) || (shared && batch_scaled(shared, routed->a13_gs, act))) n = 1;
+  if (n > T) n = T > 0 ? T : 1;
+  const int64_t Ts = T > 0 ? (T + n - 1) / n : 0;  // tokens per slice (the last may have fewer)
+  n = T > 0 ? (T + Ts - 1) / Ts : 0;
+  Carver c(nullptr);
+  carve_forward(c, Ts, k, routed, shared);
+  if (!ws || ws_bytes < c.off) return MOE_ERR_WORKSPACE;
+  if (T == 0) return MOE_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream), s_in = nullptr, s_out = nullptr;
+  st = copy_streams(&s_in, &s_out);
+  if (st != MOE_OK) return st;
+  EventSet es;
+  st = es.create((int)(2 * n + 2));
+  if (st != MOE_OK) return st;
+  cudaEvent_t ev_start = es.ev[0], ev_end = es.ev[1];
+  cudaEvent_t* in_done = es.ev + 2;
+  cudaEvent_t* fwd_done = es.ev + 2 + n;
+  const size_t row = (size_t)H * sizeof(uint16_t);
+  // the copy streams start after the work already on the caller's stream
+  if (cudaEventRecord(ev_start, s) != cudaSuccess || cudaStreamWaitEvent(s_in, ev_start, 0) != cudaSuccess ||
+      cudaStreamWaitEvent(s_out, ev_start, 0) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  // every slice's copy-in, back to back on the copy-in stream
+  for (int64_t i = 0; i < n && st == MOE_OK; ++i) {
+    const int64_t t0 = i * Ts, Ti = (T - t0) < Ts ? (T - t0) : Ts;
+    if (cudaMemcpyAsync(x_dev + t0 * H, x_host + t0 * H, (size_t)Ti * row, cudaMemcpyHostToDevice, s_in) !=
+            cudaSuccess ||
+        cudaEventRecord(in_done[i], s_in) != cudaSuccess)
+      st = MOE_ERR_CUDA;
+  }
+  // forwards on the caller's stream, each after its slice arrived; each
+  // slice's copy-out after its forward
+  for (int64_t i = 0; i < n && st == MOE_OK; ++i) {
+    const int64_t t0 = i * Ts, Ti = (T - t0) < Ts ? (T - t0) : Ts;
+    if (cudaStreamWaitEvent(s, in_done[i], 0) != cudaSuccess) {
+      st = MOE_ERR_CUDA;
+      break;
+    }
+    st = moe_forward(x_dev + t0 * H, Ti, wr, bias, k, routed, shared, act, out_dev + t0 * H, ws, ws_bytes, stream);
+    if (st != MOE_OK) break;
+    if (cudaEventRecord(fwd_done[i], s) != cudaSuccess || cudaStreamWaitEvent(s_out, fwd_done[i], 0) != cudaSuccess ||
+        cudaMemcpyAsync(out_host + t0 * H, out_dev + t0 * H, (size_t)Ti * row, cudaMemcpyDeviceToHost, s_out) !=
+            cudaSuccess)
+      st = MOE_ERR_CUDA;
+  }
+  // the caller's stream waits for the last copy-out (also after an error,
+  // so that no copy of this call is left unordered against later work)
+  const bool joined = cudaEventRecord(ev_end, s_out) == cudaSuccess && cudaStreamWaitEvent(s, ev_end, 0) == cudaSuccess;
+  if (st == MOE_OK && !joined) st = MOE_ERR_CUDA;
   return st;
 }
 

@@ -38,8 +38,9 @@ EXPORTED = (
     "moe_status_string", "moe_version", "moe_set_option", "moe_workspace_size", "moe_prepared_weights_size",
     "moe_prepare_weights", "moe_dequantize_weights", "moe_dequantized_weights_size", "moe_quantize", "moe_route", "moe_route_logits", "moe_permute", "moe_grouped_ffn",
     "moe_combine", "moe_forward", "moe_get_device_status", "moe_set_stage_events", "moe_kernel_launch_count",
-    "moe_permute_fixed_scratch",
+    "moe_permute_fixed_scratch", "moe_forward_host",
 )
+MAX_HOST_SLICES = 64
 STAGES = ("route", "permute", "act_quant", "ffn_up", "ffn_down", "shared", "combine")
 
 
@@ -98,6 +99,7 @@ def _declare(L):
         "moe_set_stage_events": ([ctypes.POINTER(ctypes.c_void_p), i32], ctypes.c_int),
         "moe_kernel_launch_count": ([], ctypes.c_uint64),
         "moe_permute_fixed_scratch": ([P, i64, i32, i32, P, P, P, P, P], ctypes.c_int),
+        "moe_forward_host": ([P, i64, P, P, i32, W, W, i32, P, P, P, i32, P, sz, P], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -296,6 +298,31 @@ def moe_forward(x: torch.Tensor, wr: torch.Tensor, bias: torch.Tensor | None, k:
     _check(lib().moe_forward(_p(x), T, _p(wr), _p(bias), k, ctypes.byref(r),
                              ctypes.byref(s) if s is not None else None, act, _p(o), _p(ws), ws.numel(),
                              _stream(stream)), "moe_forward")
+    return o
+
+
+def _hp(t):
+    if t.is_cuda or not t.is_contiguous():
+        raise ValueError("contiguous host tensor expected")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def moe_forward_host(x_host: torch.Tensor, wr: torch.Tensor, bias: torch.Tensor | None, k: int,
+                     routed: WeightBank, shared: WeightBank | None, act: int, ws: torch.Tensor,
+                     x_dev: torch.Tensor, out_dev: torch.Tensor, out_host: torch.Tensor | None = None,
+                     n_slices: int = 4, stream=None) -> torch.Tensor:
+    """The layer on host buffers: x_host [T][H] bf16 (host; pinned for the
+    copies to overlap) -> out_host [T][H] bf16 (host), through the device
+    staging buffers x_dev and out_dev, in n_slices token slices whose copies
+    overlap each other's forwards.  Only enqueues: synchronise the stream
+    before reading out_host."""
+    T, H = x_host.shape
+    o = out_host if out_host is not None else torch.empty((T, H), dtype=torch.bfloat16, pin_memory=True)
+    r = routed.struct()
+    s = shared.struct() if shared is not None else None
+    _check(lib().moe_forward_host(_hp(x_host), T, _p(wr), _p(bias), k, ctypes.byref(r),
+                                  ctypes.byref(s) if s is not None else None, act, _hp(o), _p(x_dev), _p(out_dev),
+                                  int(n_slices), _p(ws), ws.numel(), _stream(stream)), "moe_forward_host")
     return o
 
 

@@ -112,3 +112,17 @@ def test_host_side_argument_errors(L):
     assert L.moe_set_option(7, 0) == 0 and L.moe_set_option(7, 1) == 0
     # combine: k beyond the 1024 the kernel stages
     assert L.moe_combine(one, one, one, 1, 1025, 8, None, one, one, 1 << 20, None) == 1
+    # forward on host buffers: slice count, staging alignment, workspace for
+    # one slice -- all rejected before anything is enqueued
+    g = _bank(layout=1)
+    host = ctypes.create_string_buffer(64 * 128 * 2)
+    hp = ctypes.cast(host, P)
+
+    def fh(T=64, n=4, xd=one, ws_bytes=1 << 30):
+        return L.moe_forward_host(hp, T, one, None, 2, ctypes.byref(g), None, 1, hp, xd, one, n, one, ws_bytes,
+                                  None)
+    assert fh(n=0) == 1 and fh(n=ops.MAX_HOST_SLICES + 1) == 1 and fh(T=-1) == 1
+    assert fh(xd=P(258)) == 1
+    one_slice = L.moe_workspace_size(16, 2, ctypes.byref(g), None, 1)
+    assert fh(ws_bytes=one_slice - 1) == 3
+    assert fh(T=0, ws_bytes=one_slice) == 0

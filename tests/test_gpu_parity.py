@@ -333,6 +333,42 @@ def test_permutation_with_x_quantisation_changes_nothing(name, over, scales):
     assert err < TOL, err
 
 
+# the layer on host buffers: token slices (static scales; a ragged last
+# slice), and one slice when the x scale depends on the batch
+HOST_CASES = [
+    ("tiny", dict(T=40, H=256, E=8, k=2, I=256), "static", 4),
+    ("tiny", dict(T=37, H=256, E=16, k=4, I=256), "static", 5),
+    ("tiny", dict(T=24, H=256, E=8, k=2, I=256), "none", 3),
+]
+
+
+@pytest.mark.parametrize("name,over,scales,n_slices", HOST_CASES)
+def test_forward_on_host_buffers_matches_oracle(name, over, scales, n_slices):
+    """moe_forward_host: slices copied in, run and copied out on three
+    streams give the oracle's layer output, with a workspace sized for one
+    slice."""
+    w = synth.workload(name, **over)
+    W, _ = oracle_bank(w)
+    a13, a2 = synth.static_act_scales() if scales == "static" else (None, None)
+    bank = device_bank(W, a13, a2)
+    x, wr, b = routed_inputs(w)
+    Ts = -(-w.T // n_slices) if scales == "static" else w.T
+    W_ = ws(ops.workspace_size(Ts, w.k, bank, None, 1))
+    x_host = torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16).pin_memory()
+    x_dev = torch.empty((w.T, w.H), dtype=torch.bfloat16, device="cuda")
+    out_dev = torch.empty_like(x_dev)
+    bd = None if b is None else torch.from_numpy(b).cuda()
+    out = ops.moe_forward_host(x_host, bits_to_dev_bf16(wr), bd, w.k, bank, None, 1, W_, x_dev, out_dev,
+                               n_slices=n_slices)
+    torch.cuda.synchronize()
+    assert ops.moe_get_device_status(W_) == 0
+    assert torch.equal(out_dev.cpu(), out)
+    r = oracle.moe_forward(x, wr, b, w.k, W, None, act=1, a13_static=a13 or 0.0, a2_static=a2 or 0.0)
+    keep = ~ambiguous_tokens(r["logits"], w.k, 1e-4, boundary_only=True)
+    err = max_abs_rel(out.float().numpy().astype(np.float64)[keep], r["out"][keep])
+    assert err < TOL, err
+
+
 def test_forward_and_ffn_with_no_tokens():
     """T = 0: every entry point returns success and writes nothing."""
     w = synth.workload("tiny")
