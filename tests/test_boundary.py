@@ -121,6 +121,8 @@ def test_host_side_argument_errors(L):
     def fh(T=64, n=4, xd=one, ws_bytes=1 << 30):
         return L.moe_forward_host(hp, T, one, None, 2, ctypes.byref(g), None, 1, hp, xd, one, n, one, ws_bytes,
                                   None)
+    hdr = open(os.path.join(ROOT, "include", "moe_b200.h")).read()
+    assert int(re.search(r"#define MOE_MAX_HOST_SLICES (\d+)", hdr).group(1)) == ops.MAX_HOST_SLICES
     assert fh(n=0) == 1 and fh(n=ops.MAX_HOST_SLICES + 1) == 1 and fh(T=-1) == 1
     assert fh(xd=P(258)) == 1
     one_slice = L.moe_workspace_size(16, 2, ctypes.byref(g), None, 1)
