@@ -18,7 +18,8 @@
 //   3. per chunk again: each warp's base = chunk base + earlier warps'
 //      counts, and each slot's rank among equal experts earlier in its warp
 //      step -> perm_token[p] = t, inv_perm[i] = p.
-// Small batches run all three inside one block.
+// Small batches run all three inside one block, which in the forward at up
+// to 8 tokens also quantises x into the FFN's padded rows.
 #include <string.h>
 
 #include <mutex>
