@@ -74,8 +74,10 @@ def _declare(L):
     L.orc_grouped_ffn.argtypes = [P, i64, P, P, ctypes.POINTER(OrcWeights), i32, f32, f32, P, i32, P]
     L.orc_grouped_ffn.restype = ctypes.c_int
     L.orc_combine.argtypes = [P, P, P, i64, i32, i32, P, P]; L.orc_combine.restype = None
+    L.orc_router_logits_ordered.argtypes = [P, i64, i32, P, i32, P, i32, P]
+    L.orc_router_logits_ordered.restype = ctypes.c_int
     L.orc_moe_forward.argtypes = [P, i64, i32, P, P, i32, i32, ctypes.POINTER(OrcWeights),
-                                  ctypes.POINTER(OrcWeights), i32, f32, f32, f32, P, i64, P, P, P, P, i32]
+                                  ctypes.POINTER(OrcWeights), i32, f32, f32, f32, P, i64, P, P, P, P, i32, i32]
     L.orc_moe_forward.restype = ctypes.c_int
     L.orc_num_threads_available.argtypes = []; L.orc_num_threads_available.restype = ctypes.c_int
 
@@ -182,6 +184,24 @@ def router_logits(x_bf16_bits: np.ndarray, wr_bf16_bits: np.ndarray, bias=None) 
     return out
 
 
+ROUTER_ORDER_SMALL_BATCH = 1   # 256 partial sums, exchange within groups of 32, groups in order
+ROUTER_ORDER_SEQUENTIAL = 2
+
+
+def router_logits_ordered(x_bf16_bits: np.ndarray, wr_bf16_bits: np.ndarray, bias=None,
+                          order: int = ROUTER_ORDER_SMALL_BATCH) -> np.ndarray:
+    """fp32 logits [T][E] in one of the fixed summation orders (see moe_oracle.cpp)."""
+    x = _c(x_bf16_bits, np.uint16)
+    wr = _c(wr_bf16_bits, np.uint16)
+    T, H = x.shape
+    E = wr.shape[0]
+    b = None if bias is None else _c(bias, np.float32)
+    out = np.zeros((T, E), np.float32)
+    if lib().orc_router_logits_ordered(_p(x), T, H, _p(wr), E, _p(b), int(order), _p(out)) != 0:
+        raise ValueError("oracle router_logits_ordered rejected its arguments")
+    return out
+
+
 def topk(logits: np.ndarray, k: int):
     """-> (idx int32 [T,k], w float64 [T,k], status)."""
     L = _c(logits, np.float64)
@@ -219,6 +239,30 @@ class Weights:
     def struct(self) -> OrcWeights:
         return OrcWeights(self.fmt, self.E, self.H, self.I, _p(self.w13), _p(self.w13_sf), _p(self.w13_gs),
                           _p(self.w2), _p(self.w2_sf), _p(self.w2_gs))
+
+
+def quantize_expert_weights_by_expert(fmt: int, E: int, w13_of, w2_of, threads: int = 1) -> Weights:
+    """quantize_expert_weights for banks too large to hold in fp32 at once:
+    w13_of(e) and w2_of(e) return expert e's fp32 [2I][H] and [H][I]; experts
+    are drawn and quantised `threads` at a time (the quantisers release the
+    interpreter lock)."""
+    from concurrent.futures import ThreadPoolExecutor
+    first = quantize_expert_weights(fmt, w13_of(0)[None], w2_of(0)[None])
+    H, I = first.H, first.I
+    parts = [None] * E
+    parts[0] = first
+
+    def one(e):
+        parts[e] = quantize_expert_weights(fmt, w13_of(e)[None], w2_of(e)[None])
+
+    with ThreadPoolExecutor(max(1, threads)) as ex:
+        list(ex.map(one, range(1, E)))
+
+    def cat(name):
+        a = [getattr(p, name) for p in parts]
+        return None if a[0] is None else np.concatenate(a)
+
+    return Weights(fmt, E, H, I, cat("w13"), cat("w13_sf"), cat("w13_gs"), cat("w2"), cat("w2_sf"), cat("w2_gs"))
 
 
 def quantize_expert_weights(fmt: int, w13: np.ndarray, w2: np.ndarray) -> Weights:
@@ -305,8 +349,9 @@ def combine(y_perm, inv_perm, w, k: int, shared_y=None) -> np.ndarray:
 
 def moe_forward(x_bf16_bits, wr_bf16_bits, bias, k: int, routed: Weights, shared: Weights | None = None,
                 act: int = ACT_MATCH, a13_static=0.0, a2_static=0.0, sh_a2_static=0.0, tokens=None,
-                nthreads: int = 0):
-    """The whole layer.  Returns dict(out [n][H], logits [n][E], idx [n][k], w [n][k], status)."""
+                nthreads: int = 0, router_order: int = 0):
+    """The whole layer.  Returns dict(out [n][H], logits [n][E], idx [n][k], w [n][k], status).
+    router_order 0 routes on fp64 logits; 1 or 2 on fp32 logits in that fixed order."""
     x = _c(x_bf16_bits, np.uint16)
     wr = _c(wr_bf16_bits, np.uint16)
     T, H = x.shape
@@ -323,7 +368,7 @@ def moe_forward(x_bf16_bits, wr_bf16_bits, bias, k: int, routed: Weights, shared
     st = lib().orc_moe_forward(_p(x), T, H, _p(wr), _p(b), E, k, ctypes.byref(rs),
                                ctypes.byref(ss) if ss is not None else None, act, float(a13_static),
                                float(a2_static), float(sh_a2_static), _p(tok), n, _p(out), _p(logits), _p(idx),
-                               _p(w), nthreads or default_threads())
+                               _p(w), nthreads or default_threads(), int(router_order))
     return dict(out=out, logits=logits, idx=idx, w=w, status=st)
 
 

@@ -307,6 +307,7 @@ void orc_dequant(int fmt, const uint8_t* codes, const uint8_t* sf, double gs, in
 // L[t,e] = sum_h x[t,h] * Wr[e,h] (+ b[e]); bf16 inputs, double arithmetic.
 void orc_router_logits(const uint16_t* x, int64_t T, int32_t H, const uint16_t* wr, int32_t E,
                        const float* bias, double* logits) {
+#pragma omp parallel for schedule(static)
   for (int64_t t = 0; t < T; ++t)
     for (int32_t e = 0; e < E; ++e) {
       double acc = 0.0;
@@ -314,6 +315,58 @@ void orc_router_logits(const uint16_t* x, int64_t T, int32_t H, const uint16_t* 
       if (bias) acc += (double)bias[e];
       logits[t * E + e] = acc;
     }
+}
+
+// The same logits in fp32, in the fixed summation orders of the library's
+// CUDA-core router kernels, so that a routing decision taken on them can be
+// compared bit for bit.  Near ties at the k-th pick are real: the
+// atomicmilkshake/FreeToken fork README ("Known limits") reports a
+// first-token argmax that flips between two plausible experts.  A product of
+// two bf16 values is exact in fp32, so every step below is one fp32 rounding
+// of a sum (std::fma on floats).
+//  order 1 (small batches): 256 partial sums.  Partial p takes the 8
+//    consecutive columns from 8p, then the 8 from 8p + 2048, from 8p + 4096,
+//    and so on, adding one column at a time.  Each group of 32 partials
+//    (p = 32g .. 32g + 31) is combined by exchange: for d = 16, 8, 4, 2, 1 in
+//    turn, every partial q becomes its value plus the value of partial q xor d
+//    (both from before the step); the group's sum is then partial 32g.  The
+//    8 group sums are added in order g = 0 .. 7 onto 0, and the bias (or 0)
+//    last.  Needs H % 8 == 0.
+//  order 2 (sequential): one sum over h = 0 .. H-1 in turn, then the bias (or 0).
+// Returns -1 for an unknown order or H % 8 != 0 with order 1.
+int orc_router_logits_ordered(const uint16_t* x, int64_t T, int32_t H, const uint16_t* wr, int32_t E,
+                              const float* bias, int32_t order, float* logits) {
+  if (order != 1 && order != 2) return -1;
+  if (order == 1 && H % 8 != 0) return -1;
+  auto f32 = [](uint16_t b) { return (float)bf16_to_double(b); };
+  for (int64_t t = 0; t < T; ++t)
+    for (int32_t e = 0; e < E; ++e) {
+      const uint16_t* xr = x + t * H;
+      const uint16_t* wrow = wr + (int64_t)e * H;
+      float sum = 0.0f;
+      if (order == 2) {
+        for (int32_t h = 0; h < H; ++h) sum = std::fma(f32(xr[h]), f32(wrow[h]), sum);
+      } else {
+        float part[256];
+        for (int p = 0; p < 256; ++p) {
+          float acc = 0.0f;
+          for (int32_t h0 = 8 * p; h0 < H; h0 += 2048)
+            for (int c = 0; c < 8; ++c) acc = std::fma(f32(xr[h0 + c]), f32(wrow[h0 + c]), acc);
+          part[p] = acc;
+        }
+        for (int g = 0; g < 8; ++g) {
+          float* v = part + 32 * g;
+          for (int d = 16; d >= 1; d /= 2) {
+            float nv[32];
+            for (int q = 0; q < 32; ++q) nv[q] = v[q] + v[q ^ d];
+            for (int q = 0; q < 32; ++q) v[q] = nv[q];
+          }
+        }
+        for (int g = 0; g < 8; ++g) sum = sum + part[32 * g];
+      }
+      logits[t * E + e] = sum + (bias ? bias[e] : 0.0f);
+    }
+  return 0;
 }
 
 // Top-k: the k largest logits in descending order, ties to the lower expert
@@ -538,13 +591,16 @@ void orc_combine(const double* y_perm, const int32_t* inv_perm, const double* w,
 //   dynamic (<= 0).  In MATCH mode the shared expert reads the same quantised
 //   x as the routed experts and quantises its own h.
 // Dynamic h scales need every slot's h, so with a subset and a dynamic h scale
-// all tokens are evaluated.  Returns 0, or -1 on invalid input (NaN logits,
+// all tokens are evaluated.  router_order 0 takes the logits in double (the
+// definition); 1 or 2 takes them in fp32 in one of the fixed orders of
+// orc_router_logits_ordered, so that the routing decisions are the ones a
+// router summing in that order takes.  Returns 0, or -1 on invalid input (NaN logits,
 // out-of-range sizes).
 int orc_moe_forward(const uint16_t* x, int64_t T, int32_t H, const uint16_t* wr, const float* bias, int32_t E,
                     int32_t k, const orc_weights* routed, const orc_weights* shared, int32_t act,
                     float a13_static, float a2_static, float sh_a2_static, const int32_t* tokens,
                     int64_t n_tokens, double* out, double* logits_out, int32_t* idx_out, double* w_out,
-                    int32_t nthreads) {
+                    int32_t nthreads, int32_t router_order) {
   if (k < 1 || k > E || routed->E != E || routed->H != H) return -1;
   if (shared && (shared->H != H || shared->fmt != routed->fmt)) return -1;
   std::vector<int32_t> all;
@@ -573,7 +629,13 @@ int orc_moe_forward(const uint16_t* x, int64_t T, int32_t H, const uint16_t* wr,
   for (int64_t r = 0; r < NE; ++r) std::memcpy(&xe[(size_t)r * H], x + (size_t)eval_tok[r] * H, 2 * (size_t)H);
   std::vector<double> logits((size_t)NE * E), w((size_t)NE * k);
   std::vector<int32_t> idx((size_t)NE * k);
-  orc_router_logits(xe.data(), NE, H, wr, E, bias, logits.data());
+  if (router_order == 0) {
+    orc_router_logits(xe.data(), NE, H, wr, E, bias, logits.data());
+  } else {
+    std::vector<float> lf((size_t)NE * E);
+    if (orc_router_logits_ordered(xe.data(), NE, H, wr, E, bias, router_order, lf.data()) != 0) return -1;
+    for (size_t i = 0; i < lf.size(); ++i) logits[i] = (double)lf[i];
+  }
   int st = orc_topk(logits.data(), NE, E, k, idx.data(), w.data());
   // Activation of x: quantised over the whole tensor (all T tokens).
   std::vector<float> xf;

@@ -62,3 +62,56 @@ def routed_inputs(w: synth.Workload, seed: int = synth.SEED):
     wr = synth.router_bits(w, seed)
     b = synth.router_bias(w, seed)
     return x, wr, b
+
+
+def router_order(T: int, E: int, H: int) -> int:
+    """Which fixed fp32 summation order moe_route's logits follow (the header
+    documents it): 1 = the small-batch order (T <= 64, H % 8 == 0), 2 = one
+    sequential sum, 0 = the tensor cores' own order (T >= 128, E % 128 == 0,
+    H % 64 == 0), which the oracle cannot replay."""
+    if T >= 128 and E % 128 == 0 and H % 64 == 0:
+        return 0
+    if T <= 64 and H % 8 == 0:
+        return 1
+    return 2
+
+
+def routing_tol(L_ref: np.ndarray, L_gpu: np.ndarray, floor: float = 1e-6) -> float:
+    """Half-width of the band in which a top-k choice taken on the GPU's fp32
+    logits may differ from one taken on the oracle's: twice the largest
+    logit difference actually seen (a gap wider than that cannot flip)."""
+    return max(2.0 * float(np.max(np.abs(np.asarray(L_gpu, np.float64) - L_ref))), floor)
+
+
+def report_ambiguous(amb: np.ndarray, what: str, limit: float = 0.01) -> float:
+    """Prints and bounds the fraction of tokens left out as ambiguous."""
+    frac = float(np.mean(amb)) if amb.size else 0.0
+    print(f"{what}: {int(np.sum(amb))} of {amb.size} tokens ambiguous ({100 * frac:.3f} %)")
+    assert frac < limit, f"{what}: {100 * frac:.3f} % of tokens ambiguous"
+    return frac
+
+
+def forward_reference(w: synth.Workload, x, wr, b, W, Ws=None, act: int = 1, a13=None, a2=None, sh_a2=None,
+                      tokens=None, route_T: int | None = None, what: str = ""):
+    """The oracle's layer output for moe_forward's inputs, and the tokens whose
+    routing both sides decide alike.  Where the library's router sums in a
+    fixed order (router_order) the oracle routes on the same fp32 logits and
+    every token is kept; behind the tensor-core router, tokens whose k/k+1
+    logit gap lies within routing_tol of the GPU's own logits (moe_route on
+    the same batch) are left out, counted and bounded.  route_T: the batch
+    size the router sees (a slice of moe_forward_host)."""
+    order = router_order(route_T or w.T, w.E, w.H)
+    r = oracle.moe_forward(x, wr, b, w.k, W, Ws, act=act, a13_static=a13 or 0.0, a2_static=a2 or 0.0,
+                           sh_a2_static=sh_a2 or 0.0, tokens=tokens, router_order=order)
+    if order:
+        return r, np.ones(r["out"].shape[0], bool)
+    logits = torch.empty((w.T, w.E), dtype=torch.float32, device="cuda")
+    ws = ops.new_workspace(w.T * w.E * 16 + (1 << 20))
+    ops.moe_route(bits_to_dev_bf16(x), bits_to_dev_bf16(wr), None if b is None else torch.from_numpy(b).cuda(),
+                  w.k, ws, logits=logits)
+    gl = logits.cpu().numpy()
+    if tokens is not None:
+        gl = gl[np.asarray(tokens)]
+    amb = ambiguous_tokens(r["logits"], w.k, routing_tol(r["logits"], gl), boundary_only=True)
+    report_ambiguous(amb, what or f"forward {w.name}")
+    return r, ~amb

@@ -259,3 +259,16 @@ def test_bf16_weights_equal_nvfp4_weights_when_exact(orc):
     a = orc.moe_forward(x, wr, None, k, Wn, act=orc.ACT_BF16)["out"]
     b = orc.moe_forward(x, wr, None, k, Wb, act=orc.ACT_BF16)["out"]
     assert np.array_equal(a, b)
+
+
+def test_bank_by_expert_equals_whole_bank(orc):
+    """The per-expert, threaded bank builder gives the bytes of the
+    whole-array one (NVFP4 with its per-part scales, MXFP4)."""
+    for fmt, name in ((orc.FMT_NVFP4, "nvfp4"), (orc.FMT_MXFP4, "mxfp4"), (orc.FMT_FP8, "fp8")):
+        w = synth.workload("tiny", fmt=name, E=5, H=256, I=256)
+        A = orc.quantize_expert_weights(fmt, synth.all_w13(w), synth.all_w2(w))
+        B = orc.quantize_expert_weights_by_expert(fmt, w.E, lambda e: synth.expert_w13(w, e),
+                                                  lambda e: synth.expert_w2(w, e), threads=3)
+        for f in ("w13", "w13_sf", "w13_gs", "w2", "w2_sf", "w2_gs"):
+            a, b = getattr(A, f), getattr(B, f)
+            assert (a is None and b is None) or np.array_equal(a, b), (name, f)

@@ -122,3 +122,106 @@ def test_permute_then_unpermute_is_identity(orc):
     y_perm = x[perm]
     out = orc.combine(y_perm, inv, np.full((T, k), 1.0 / k), k)
     assert np.array_equal(out, x)
+
+
+# ------------------------------------------------ fixed-order fp32 logits ----
+def _f32_to_bits(a):
+    a = np.asarray(a, np.float32)
+    assert np.array_equal(_bits_to_f64(synth.to_bf16_bits(a)), a.astype(np.float64)), "values must be bf16-exact"
+    return synth.to_bf16_bits(a)
+
+
+@pytest.mark.parametrize("order", [1, 2])
+@pytest.mark.parametrize("H", [8, 2048, 2304, 4096])
+def test_ordered_logits_exact_on_small_integers(orc, order, H):
+    """Small-integer products: every partial sum is an integer below 2^24, so
+    any summation order gives the exact dot product (integer arithmetic)."""
+    rng = np.random.default_rng(H + order)
+    xi = rng.integers(-4, 5, (5, H))
+    wi = rng.integers(-4, 5, (7, H))
+    bias = rng.integers(-8, 9, 7).astype(np.float32)
+    L = orc.router_logits_ordered(_f32_to_bits(xi), _f32_to_bits(wi), bias, order=order)
+    assert np.array_equal(L.astype(np.int64), xi @ wi.T + bias.astype(np.int64))
+
+
+def _one_hot_products(H, cols_vals):
+    """x = 1 everywhere on the given columns, w = the wanted product there."""
+    x = np.zeros((1, H), np.float32)
+    w = np.zeros((1, H), np.float32)
+    for c, v in cols_vals:
+        x[0, c] = 1.0
+        w[0, c] = v
+    return _f32_to_bits(x), _f32_to_bits(w)
+
+
+def test_ordered_logits_follow_the_stated_order(orc):
+    """Hand-derived sums where fp32 rounding reveals the order.  2^24 + 1 is a
+    tie that rounds to the even 2^24; 2^24 + 2 is exact."""
+    big = float(2 ** 24)
+    # products 2^24 at column 0, 1 at columns 8 and 9 (partial 1 of the small
+    # batch order): sequentially 2^24 + 1 + 1 = 2^24; partial 0 = 2^24, partial
+    # 1 = 2, joined by the exchange step d = 1: 2^24 + 2
+    x, w = _one_hot_products(2048, [(0, big), (8, 1.0), (9, 1.0)])
+    assert orc.router_logits_ordered(x, w, order=2)[0, 0] == big
+    assert orc.router_logits_ordered(x, w, order=1)[0, 0] == big + 2
+    # partials 1 and 3 (columns 8 and 24) each hold 1: the exchange adds them
+    # at d = 2 before partial 0 joins at d = 1 -> 2^24 + 2; sequentially 2^24
+    x, w = _one_hot_products(2048, [(0, big), (8, 1.0), (24, 1.0)])
+    assert orc.router_logits_ordered(x, w, order=1)[0, 0] == big + 2
+    assert orc.router_logits_ordered(x, w, order=2)[0, 0] == big
+    # partials 1 and 2 (columns 8 and 16): partial 2 meets partial 0 at d = 2
+    # (2^24 + 1 -> 2^24), partial 1 meets partial 3 (0) there, and at d = 1
+    # 2^24 + 1 -> 2^24 again
+    x, w = _one_hot_products(2048, [(0, big), (8, 1.0), (16, 1.0)])
+    assert orc.router_logits_ordered(x, w, order=1)[0, 0] == big
+    # group sums in order g = 0..7 onto 0: group 0 = 1, group 1 = 2^24
+    # (partial 32, column 256), group 2 = 1 (partial 64, column 512):
+    # 1 + 2^24 -> 2^24 (tie to even), + 1 -> 2^24
+    x, w = _one_hot_products(2048, [(0, 1.0), (256, big), (512, 1.0)])
+    assert orc.router_logits_ordered(x, w, order=1)[0, 0] == big
+    # a partial's second stretch starts 2048 columns on: columns 2048 and 2049
+    # belong to partial 0, which already holds 2^24 (each + 1 rounds away) ...
+    x, w = _one_hot_products(4096, [(0, big), (2048, 1.0), (2049, 1.0)])
+    assert orc.router_logits_ordered(x, w, order=1)[0, 0] == big
+    # ... while columns 2056 and 2057 belong to partial 1, which sums them to 2
+    x, w = _one_hot_products(4096, [(0, big), (2056, 1.0), (2057, 1.0)])
+    assert orc.router_logits_ordered(x, w, order=1)[0, 0] == big + 2
+    assert orc.router_logits_ordered(x, w, order=2)[0, 0] == big
+
+
+@pytest.mark.parametrize("order", [1, 2])
+def test_ordered_logits_within_the_fp32_summation_bound(orc, order):
+    """Any summation order of n terms in fp32 is within (n - 1) u sum|terms|
+    (u = 2^-24, first order) of the exact sum, here the fp64 definition."""
+    w = synth.workload("decode")
+    x = synth.x_bits(w)
+    wr = synth.router_bits(w)
+    b = np.linspace(-1, 1, w.E).astype(np.float32)
+    L = orc.router_logits_ordered(x, wr, b, order=order).astype(np.float64)
+    ref = orc.router_logits(x, wr, b)
+    absum = np.abs(_bits_to_f64(x)) @ np.abs(_bits_to_f64(wr)).T + np.abs(b.astype(np.float64))
+    bound = (w.H + 1) * 2.0 ** -24 * absum * 1.01
+    assert np.all(np.abs(L - ref) <= bound)
+    assert np.any(L != ref.astype(np.float32))   # fp32 rounding really happened
+
+
+def test_ordered_logits_reject_ragged_small_batch_order(orc):
+    x = synth.to_bf16_bits(np.ones((1, 12), np.float32))
+    with pytest.raises(ValueError):
+        orc.router_logits_ordered(x, x, order=1)
+    assert orc.router_logits_ordered(x, x, order=2)[0, 0] == 12.0
+
+
+def test_forward_routes_on_the_ordered_logits(orc):
+    """orc_moe_forward with a fixed router order selects on exactly the fp32
+    logits of router_logits_ordered (converted to double)."""
+    w = synth.workload("tiny")
+    x = synth.x_bits(w)
+    wr = synth.router_bits(w)
+    W = orc.quantize_expert_weights(orc.FMT_NVFP4, synth.all_w13(w), synth.all_w2(w))
+    r = orc.moe_forward(x, wr, None, w.k, W, act=orc.ACT_MATCH, router_order=1)
+    L = orc.router_logits_ordered(x, wr, None, order=1).astype(np.float64)
+    assert np.array_equal(r["logits"], L)
+    idx, wt, _ = orc.topk(L, w.k)
+    assert np.array_equal(r["idx"], idx)
+    assert np.array_equal(r["w"], wt)
