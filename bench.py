@@ -281,16 +281,17 @@ def time_forward(ops, torch, layer, w, act, steps, warmup, flush, stage=True, ho
                     fwd()
             finally:
                 ops.moe_set_stage_events(None)
-            acc = {n: [] for n in ops.STAGES}
+            # only the stages this forward records (the others' events hold
+            # nothing but the binding's set-up records)
+            mask = ops.moe_stage_mask()
+            ran = [(si, n) for si, n in enumerate(ops.STAGES) if mask >> si & 1]
+            acc = {n: [] for _, n in ran}
             for i in range(steps):
                 flush.zero_()
                 g2.replay()
                 torch.cuda.synchronize()
-                for si, name in enumerate(ops.STAGES):
-                    try:
-                        acc[name].append(evs[2 * si].elapsed_time(evs[2 * si + 1]))
-                    except RuntimeError:
-                        pass
+                for si, name in ran:
+                    acc[name].append(evs[2 * si].elapsed_time(evs[2 * si + 1]))
             stages = {n: float(np.mean(v)) for n, v in acc.items() if v}
             del g2
         del graph
@@ -329,7 +330,13 @@ def time_forward_host(ops, torch, layer, w, act, steps, warmup, flush, n_slices)
         raise RuntimeError("device status reported a fault in moe_forward_host")
     r = ref.float().cpu()
     err = ((out_host.float() - r).abs().amax(dim=1) / r.abs().max().clamp_min(1e-30)).numpy()
-    bad = int((err > 2e-2).sum())
+    off = np.nonzero(err > 2e-2)[0]
+    if off.size:
+        ties = routing_near_ties(ops, torch, x, wr, bias, w.k, n_slices, off)
+        if not ties.all():
+            raise RuntimeError(f"{int((~ties).sum())} tokens differ from the device-resident forward "
+                               "without a routing near-tie")
+    bad = int(off.size)
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     for i in range(steps):
         flush.zero_()
@@ -338,6 +345,27 @@ def time_forward_host(ops, torch, layer, w, act, steps, warmup, flush, n_slices)
         evs[i][1].record(stream)
     torch.cuda.synchronize()
     return dict(ms=[a.elapsed_time(b) for a, b in evs], bad_tokens=bad)
+
+
+def routing_near_ties(ops, torch, x, wr, bias, k, n_slices, tokens):
+    """For each token listed: whether its top-k choice may legitimately differ
+    between a forward of its slice and of the whole batch -- the gap between
+    its k-th and (k+1)-th whole-batch logits is within twice the largest
+    difference between the two routers' logits (the router splits its sums
+    differently at another batch size)."""
+    T, E = x.shape[0], wr.shape[0]
+    ws = ops.new_workspace(T * E * 16 + (1 << 20))
+    Lw = torch.empty((T, E), dtype=torch.float32, device=x.device)
+    ops.moe_route(x, wr, bias, k, ws, logits=Lw)
+    Ls = torch.empty_like(Lw)
+    Ts = -(-T // n_slices)
+    for t0 in range(0, T, Ts):
+        ops.moe_route(x[t0:t0 + Ts], wr, bias, k, ws, logits=Ls[t0:t0 + Ts])
+    torch.cuda.synchronize()
+    band = 2.0 * float((Ls - Lw).abs().max().item())
+    srt = torch.sort(Lw[torch.as_tensor(tokens, device=x.device)], dim=1, descending=True).values
+    gap = (srt[:, k - 1] - srt[:, k]) if k < E else torch.full((len(tokens),), float("inf"), device=x.device)
+    return (gap <= band).cpu().numpy()
 
 
 def time_grouped_ffn(ops, torch, layer, w, act, steps, warmup, flush):
@@ -374,12 +402,14 @@ def time_grouped_ffn(ops, torch, layer, w, act, steps, warmup, flush):
     return [a.elapsed_time(b) for a, b in evs], off.cpu().numpy()
 
 
-def config_report(ops, torch, synth, name, act, steps, warmup, flush, pk):
+def config_report(ops, torch, synth, name, act, steps, warmup, flush, pk, static=None):
     """Per-config figures: tokens/s, the GEMMs' TFLOP/s against the format's
     tensor peak, the active experts' weight GB/s against HBM, and the routing
-    histogram.  Stage times come from the library's stage events."""
+    histogram.  Stage times come from the library's stage events.  static:
+    static activation scales (default: for NVFP4 layers)."""
     w = synth.workload(name)
-    layer = build_layer(ops, synth, torch, w, static=(w.fmt == "nvfp4"))
+    static = (w.fmt == "nvfp4") if static is None else static
+    layer = build_layer(ops, synth, torch, w, static=static)
     r = time_forward(ops, torch, layer, w, act, steps, warmup, flush)
     del layer
     torch.cuda.empty_cache()
@@ -388,7 +418,9 @@ def config_report(ops, torch, synth, name, act, steps, warmup, flush, pk):
     ms = np.array(r["ms"])
     peak = pk["bf16_tflops"] * {"fp8": FP8_PER_BF16, "bf16": 1.0}.get(w.fmt, FP4_PER_BF16)
     up, down = st.get("ffn_up", 0.0), st.get("ffn_down", 0.0)
-    rep_ = {"workload": workload_name(w), "act_scales": {"nvfp4": "static", "bf16": "none"}.get(w.fmt, "dynamic"),
+    scales = "none" if w.fmt == "bf16" else ("static" if static and w.fmt in ("nvfp4", "fp8") else
+                                               ("dynamic" if w.fmt in ("nvfp4", "fp8") else "none (block scales only)"))
+    rep_ = {"workload": workload_name(w), "act_scales": scales,
             "ms_median": float(np.median(ms)), "ms_p10": float(np.percentile(ms, 10)),
             "ms_p90": float(np.percentile(ms, 90)), "tokens_per_s": w.T / (float(np.median(ms)) * 1e-3),
             "stages_ms": st, "routing": {"active_experts": alg["active_experts"],
@@ -551,8 +583,6 @@ def main():
     method = f"moe_forward_host, {args.e2e_slices} token slices"
     try:
         res_e2e = time_forward_host(ops, torch, layer, w, act, args.steps, 2, flush, args.e2e_slices)
-        if res_e2e["bad_tokens"] > max(1, w.T // 1000):
-            raise RuntimeError(f"{res_e2e['bad_tokens']} tokens differ from the device-resident forward")
     except (RuntimeError, ops.MoeError) as exc:
         method = f"copy in, moe_forward, copy out (sliced path not used: {exc})"
         res_e2e = time_forward(ops, torch, layer, w, act, args.steps, 2, flush, stage=False, host_io=True)
@@ -607,11 +637,17 @@ def main():
                               lambda u, d: u + d if u is not None and d is not None else None)(
                               measured_traffic("ffn_up", "decode"), measured_traffic("ffn_down", "decode")),
                           "hbm_frac": gbs / pk["hbm_gbs"] if gbs else None, "stages_ms": rd["stages"]}
+        # the metric's second half, where the driver's record keeps it
+        line["roofline"]["decode"] = {"kernel": "moe_grouped_ffn (decode workload)", "bound": "hbm",
+                                      "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                                      "frac": line["decode"]["hbm_frac"], "traffic": line["decode"]["traffic"],
+                                      "bytes": ad["wbytes_up"] + ad["wbytes_down"], "ms": ffn_ms,
+                                      "peak_source": pk_kind}
         del dl
 
     if not args.no_configs:
-        line["configs"] = [config_report(ops, torch, synth, n, act, 10, 3, flush, pk)
-                           for n in ("fp8_shared", "large", "bf16_prefill")]
+        line["configs"] = [config_report(ops, torch, synth, "prefill", act, 10, 3, flush, pk, static=False)] + [
+            config_report(ops, torch, synth, n, act, 10, 3, flush, pk) for n in ("fp8_shared", "large", "bf16_prefill")]
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_oracle_sample(w, args.cpu_seconds, static=True)

@@ -32,9 +32,14 @@
  *    atomicmilkshake/FreeToken fork README describes under "What else
  *    changed" for a kernel switch without a default).
  *  - Faults found on the device (an expert index out of range, a NaN or
- *    all -inf logit row, a bounded wait that ran out) set a status word inside
- *    `ws`; the affected outputs are written with zeros, never left
- *    uninitialised.  moe_get_device_status() reads and clears the word.
+ *    all -inf logit row) set a status word inside `ws`; the affected outputs
+ *    are written with zeros (or the slot is dropped), never left
+ *    uninitialised.  A bounded device wait that ran out (MOE_OPT_WAIT_CYCLES)
+ *    sets the word to MOE_ERR_TIMEOUT: the kernel that gave up lets its
+ *    copies in flight land, frees its tensor memory and returns, and the
+ *    later kernels of the call still run, but the outputs of that call are
+ *    then unspecified.  moe_get_device_status() reads and clears the word;
+ *    the next call on the same workspace starts clean.
  *  - A launch failure returns MOE_ERR_CUDA.
  */
 #ifndef MOE_B200_H
@@ -192,7 +197,20 @@ moe_status moe_quantize(int32_t fmt, const void* x, int32_t x_dtype, int64_t row
  *  nullable), logits [T][E] fp32 (device, nullable output), topk_idx [T][k]
  *  int32 (device out), topk_w [T][k] fp32 (device out).
  * 1 <= k <= E <= 1024; T >= 0 (T == 0 enqueues nothing).  A row with a NaN
- * logit or no finite logit sets the device status word. */
+ * logit or no finite logit sets the device status word.
+ * Summation order of the logits (all fp32; each product of two bf16 values
+ * is exact, so only the sums round), the same on every launch:
+ *  - T <= 64 and H % 8 == 0: 256 partial sums per logit; partial p adds the
+ *    8 columns from 8p, then the 8 from 8p + 2048, 8p + 4096, ..., one
+ *    column at a time; each group of 32 partials is combined by exchange
+ *    (for d = 16, 8, 4, 2, 1 every partial q becomes q + (q xor d)), the
+ *    group's sum being partial 32g; the 8 group sums are added in order onto
+ *    0, then the bias (or 0).  A CPU replay of this order reproduces the
+ *    logits, and so the routing, bit for bit.
+ *  - T >= 128, E % 128 == 0, H % 64 == 0: the bf16 tensor cores (tcgen05),
+ *    with fp32 accumulation in their own order, H split in up to 4 parts
+ *    added in order.
+ *  - otherwise: one sequential sum over h = 0 .. H-1, then the bias (or 0). */
 moe_status moe_route(const uint16_t* x, int64_t T, int32_t H, const uint16_t* wr, const float* bias, int32_t E,
                      int32_t k, float* logits, int32_t* topk_idx, float* topk_w, void* ws, size_t ws_bytes,
                      moe_stream_t stream);
@@ -285,13 +303,68 @@ moe_status moe_forward(const uint16_t* x, int64_t T, const uint16_t* wr, const f
  *    at another batch size, which can flip a top-k choice whose logits tie
  *    to within rounding.
  * ws: at least moe_workspace_size(ceil(T / n_slices), k, routed, shared,
- * act) bytes; the slices' forwards reuse it one after the other.  Argument
- * errors return before anything is enqueued. */
+ * act) bytes (moe_workspace_size never decreases with T, so that size also
+ * serves a shorter last slice); the slices' forwards reuse it one after the
+ * other.  Argument errors return before anything is enqueued.  `stream`
+ * waits for the last copy-in and the last copy-out, also after an error. */
 #define MOE_MAX_HOST_SLICES 64
 moe_status moe_forward_host(const uint16_t* x_host, int64_t T, const uint16_t* wr, const float* bias, int32_t k,
                             const moe_weights* routed, const moe_weights* shared, int32_t act, uint16_t* out_host,
                             uint16_t* x_dev, uint16_t* out_dev, int32_t n_slices, void* ws, size_t ws_bytes,
                             moe_stream_t stream);
+
+/* Host -> HBM expert streaming: an LRU pool of `n_slots` expert slots in
+ * HBM in front of an expert bank kept in page-locked host memory, for layers
+ * whose experts do not all fit in HBM.  This is the expert slot pool of the
+ * atomicmilkshake/FreeToken fork README ("Known limits") and the host-memory
+ * expert offload with a global LRU expert cache of the FreeToken upstream
+ * README ("About"), decided and copied on the device: a forward through the
+ * cache performs no host synchronisation and can be captured in a CUDA
+ * graph.  Per call, an admit kernel marks the experts the batch routes to,
+ * keeps those already resident (hits), gives every other one the least
+ * recently used slot that no expert of this batch holds (empty slots first)
+ * and rewrites the top-k ids into slot ids; a fetch kernel copies the
+ * admitted experts from host memory into their slots over PCIe; the layer
+ * then runs on the pool as a bank of n_slots experts.  The result is the
+ * layer's result on the whole bank.
+ * Filled by moe_expert_cache_init; treat the fields as read-only. */
+typedef struct {
+  moe_weights bank;          /* the bank as given: PREPARED, page-locked host memory (a13_gs, a2_gs device) */
+  moe_weights pool;          /* the slots: PREPARED, E = n_slots, device memory */
+  const void* bank_dev[6];   /* device addresses of bank.w13, w13_sf, w13_gs, w2, w2_sf, w2_gs (or NULL) */
+  int32_t* state;            /* device: clock, counters, slot and expert maps */
+  int32_t n_slots;
+} moe_expert_cache;
+
+/* Device bytes moe_expert_cache_init needs for a pool of n_slots experts of
+ * `bank` (0 on invalid arguments). */
+size_t moe_expert_cache_bytes(const moe_weights* bank, int32_t n_slots);
+
+/* Sets up a cache: `bank` is a PREPARED bank (moe_prepare_weights, then
+ * copied to host memory) whose w13, w13_sf, w13_gs, w2, w2_sf and w2_gs live
+ * in page-locked, device-mapped host memory (cudaHostAlloc / pinned torch
+ * tensors) and whose a13_gs / a2_gs, if any, are device pointers.
+ * 1 <= n_slots <= min(E, 1024).  `dev` (device, dev_bytes >=
+ * moe_expert_cache_bytes) holds the pool and the state; the pool starts
+ * empty.  Enqueued on `stream`.  MOE_ERR_INVALID_ARG when a host array is not
+ * mapped into the device's address space. */
+moe_status moe_expert_cache_init(const moe_weights* bank, int32_t n_slots, void* dev, size_t dev_bytes,
+                                 moe_expert_cache* cache, moe_stream_t stream);
+
+/* moe_forward with the routed experts streamed through `cache` (no shared
+ * expert): route, admit, fetch, permute, grouped FFN on the pool, combine.
+ * The pool must hold every expert one batch can route to: n_slots >=
+ * min(E, T*k), else MOE_ERR_INVALID_ARG.  ws: moe_workspace_size(T, k,
+ * &cache->bank, NULL, act) bytes.  Calls through one cache must not overlap
+ * on the GPU (they share its slots). */
+moe_status moe_forward_cached(const uint16_t* x, int64_t T, const uint16_t* wr, const float* bias, int32_t k,
+                              const moe_expert_cache* cache, int32_t act, uint16_t* out, void* ws, size_t ws_bytes,
+                              moe_stream_t stream);
+
+/* Synchronises `stream` and reads the cache's counters: stats[0] calls so
+ * far, [1] experts fetched by the last call, [2] experts fetched in all, [3]
+ * hits in all (host, 4 values). */
+moe_status moe_expert_cache_stats(const moe_expert_cache* cache, moe_stream_t stream, int64_t* stats);
 
 /* Synchronises `stream`, copies the device status word of `ws` into
  * *host_status (a moe_status value: MOE_OK, MOE_ERR_DEVICE_FAULT or
@@ -338,7 +411,36 @@ moe_status moe_get_device_status(void* ws, moe_stream_t stream, int32_t* host_st
  *                     permutation kernel, and the FFN kernel then derives its
  *                     tile list from the top-k ids, so its first weight loads
  *                     overlap the permutation; 0 runs the x quantiser as a
- *                     kernel of its own.  Results are identical either way. */
+ *                     kernel of its own.  Results are identical either way.
+ *   MOE_OPT_WAIT_CYCLES: bound of every device wait, in SM clock cycles
+ *                     (1 .. 2^31 - 1; 0 restores the default of 2e9, about
+ *                     a second at 1.965 GHz).  A wait that runs past it gives
+ *                     up with MOE_ERR_TIMEOUT (see the conventions above);
+ *                     a small bound makes ordinary waits for memory run out,
+ *                     which is how the timeout path is tested.
+ *   MOE_OPT_FUSED_COMBINE: 1 (default) lets moe_forward, when its routed (and
+ *                     shared) experts run on the grouped tensor-core GEMM
+ *                     (not the one-kernel FFN) and the weights are not BF16,
+ *                     do the weighted combine in the down projection's
+ *                     epilogue: each output row gets w * y added in fp32
+ *                     (reductions in L2) and one pass rounds the rows to
+ *                     bf16, so y_perm is neither written nor read back.  The
+ *                     order of the k additions then varies from run to run
+ *                     (results within fp32 rounding of each other); 0 keeps
+ *                     bf16 y_perm and the ordered combine of moe_combine,
+ *                     which is bit-reproducible.
+ *   MOE_OPT_SMALL_BATCH_FORWARD: 1 (default) runs moe_forward at T <= 32 on
+ *                     the one-kernel FFN (NVFP4 with a static h scale, or
+ *                     MXFP4; H % 256 == 0; E <= 256) with no shared expert as
+ *                     two kernels: the router (logits, x quantised into a
+ *                     layout the FFN copies token rows from, top-k in its
+ *                     last block), then the FFN, which needs no permutation
+ *                     (a tile's rows are its expert's slots in flat order),
+ *                     adds w * y into fp32 output rows in its down epilogue
+ *                     and rounds them to bf16 in the CTA that finishes last.
+ *                     The logits and routing are those of moe_route; the
+ *                     order of the k additions varies from run to run.  0
+ *                     keeps the permutation and the ordered combine. */
 typedef enum {
   MOE_OPT_FFN_PATH = 1,
   MOE_OPT_GEMM_TILE_N = 2,
@@ -346,7 +448,10 @@ typedef enum {
   MOE_OPT_PDL = 4,
   MOE_OPT_EARLY_WEIGHTS = 5,
   MOE_OPT_FUSED_FFN = 6,
-  MOE_OPT_PERMUTE_QUANT = 7
+  MOE_OPT_PERMUTE_QUANT = 7,
+  MOE_OPT_WAIT_CYCLES = 8,
+  MOE_OPT_FUSED_COMBINE = 9,
+  MOE_OPT_SMALL_BATCH_FORWARD = 10
 } moe_option;
 moe_status moe_set_option(int32_t option, int32_t value);
 
@@ -380,6 +485,9 @@ moe_status moe_permute_fixed_scratch(const int32_t* topk_idx, int64_t T, int32_t
  * stream, so a caller can time each stage with cudaEventElapsedTime.  Stages
  * a call does not run are not recorded.  NULL turns the hook off.  Not
  * thread-safe; the handles must outlive the calls that record them.
+ * moe_stage_mask: bit s is set when stage s has been recorded since events
+ * were last installed (stages a call does not run stay clear; turning the
+ * hook off keeps the mask).
  * moe_kernel_launch_count: number of kernels this library has launched in
  * the process so far (host-side count of kernel launches). */
 typedef enum {
@@ -393,6 +501,7 @@ typedef enum {
   MOE_STAGE_COUNT = 7
 } moe_stage;
 moe_status moe_set_stage_events(void* const* events, int32_t n_events);
+uint32_t moe_stage_mask(void);
 uint64_t moe_kernel_launch_count(void);
 
 #ifdef __cplusplus

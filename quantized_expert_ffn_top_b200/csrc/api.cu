@@ -48,16 +48,21 @@ Scalars carve_head(Carver& c) {
 
 int g_ffn_path = 0;  // MOE_OPT_FFN_PATH
 static int g_fused_ffn = 1;  // MOE_OPT_FUSED_FFN
+static int g_fused_combine = 1;  // MOE_OPT_FUSED_COMBINE
+static int g_small_forward = 1;  // MOE_OPT_SMALL_BATCH_FORWARD
 static int g_perm_quant = 1;  // MOE_OPT_PERMUTE_QUANT
 
 // Measurement hook (moe_set_stage_events).
 cudaEvent_t g_stage_events[2 * MOE_STAGE_COUNT];
 bool g_stage_on = false;
+uint32_t g_stage_mask = 0;   // stages recorded since the hook was set
 
 // External records, so that events captured into a CUDA graph stay readable
 // by the caller after each replay.
 void stage_mark(int stage, bool end, cudaStream_t s) {
-  if (g_stage_on) cudaEventRecordWithFlags(g_stage_events[2 * stage + (end ? 1 : 0)], s, cudaEventRecordExternal);
+  if (!g_stage_on) return;
+  cudaEventRecordWithFlags(g_stage_events[2 * stage + (end ? 1 : 0)], s, cudaEventRecordExternal);
+  g_stage_mask |= 1u << stage;
 }
 
 int num_sms() {
@@ -106,13 +111,10 @@ moe_status check_weights(const moe_weights* w, bool need_prepared) {
 }
 
 // ---------------------------------------------------------------- layouts --
-// Partial logits of the tensor-core router GEMM split along H: at most as
-// many as 256 SMs can take (the split used at run time is never larger).
-int router_parts_max(int64_t T, int E) {
-  const int64_t items = (T + kRouterBN - 1) / kRouterBN * (E >= 128 ? E / 128 : 1);
-  int64_t ks = items > 0 ? 256 / items : 1;
-  return (int)(ks < 1 ? 1 : (ks > kRouterMaxSplit ? kRouterMaxSplit : ks));
-}
+// Partial logits of the tensor-core router GEMM split along H: room for the
+// largest split at every batch size, so that every scratch size below grows
+// with T (a workspace sized for T serves every smaller batch).
+constexpr int kRouterParts = kRouterMaxSplit;
 
 // Router scratch: the (partial) logits.
 struct RouteWs {
@@ -122,7 +124,7 @@ struct RouteWs {
 RouteWs carve_route(Carver& c, int64_t T, int E) {
   RouteWs r;
   r.head = carve_head(c);
-  r.parts = c.take<float>((size_t)T * E * router_parts_max(T, E));
+  r.parts = c.take<float>((size_t)T * E * kRouterParts);
   return r;
 }
 
@@ -144,6 +146,8 @@ int g_gemm_bn = 0;  // token tile of the tensor-core path (MOE_OPT_GEMM_TILE_N);
 int64_t padded_rows(int64_t S, int E) { return (int64_t)align_up((size_t)(S + (int64_t)E * 127), 128) + 256; }
 // Tile list bound for the smallest token group (8 slots, the GEMV's MMA n).
 int64_t max_tiles(int64_t S, int E) { return S / 8 + E + 1; }
+// Bytes of the one-kernel FFN's counters (FfnScratch::counters).
+size_t counters_bytes(int64_t S, int E) { return sizeof(int32_t) * (size_t)(4 + max_tiles(S, E)); }
 
 // Scratch of the grouped FFN: GEMV path (h fp32 per compact slot) and tensor
 // core path (padded, blocked quantised activations and the tile plan).
@@ -157,7 +161,17 @@ struct FfnScratch {
   uint8_t* hq;       //       [P][I/2 | I]
   uint8_t* hsf;
   float* h32;        //       [P][I] fp32 h (dynamic h scale / FP8)
-  int32_t* tile_done;  //     [max_tiles] fused FFN: gate|up slices finished per token tile
+  // one-kernel FFN counters, cleared together: [0] the item counter, [1] CTAs
+  // finished, [2] the decode router's ticket, [4 ..] gate|up slices finished
+  // per token tile
+  int32_t* counters;
+  int32_t* work;
+  int32_t* done;
+  int32_t* ticket;
+  int32_t* tile_done;  //     [max_tiles]
+  float* w_perm;       //     [S] routing weight of each slot position (combine in the down epilogue)
+  uint8_t* xg;         //     small batches: x in the gather layout, [min(S, 32)][8][H/2]
+  uint8_t* xsl;        //     and its scale lines, [min(S, 32)][H / (4 bs)][16]
   int64_t P;
 };
 FfnScratch carve_ffn(Carver& c, int64_t S, const moe_weights* w) {
@@ -174,7 +188,16 @@ FfnScratch carve_ffn(Carver& c, int64_t S, const moe_weights* w) {
   f.hq = c.take<uint8_t>((size_t)(f.P * rbi));
   f.hsf = bs ? c.take<uint8_t>((size_t)(f.P * (w->I / bs))) : nullptr;
   f.h32 = c.take<float>((size_t)(f.P * w->I));
-  f.tile_done = c.take<int32_t>((size_t)max_tiles(S, w->E));
+  f.counters = c.take<int32_t>((size_t)(4 + max_tiles(S, w->E)));
+  f.work = f.counters ? f.counters : nullptr;
+  f.done = f.counters ? f.counters + 1 : nullptr;
+  f.ticket = f.counters ? f.counters + 2 : nullptr;
+  f.tile_done = f.counters ? f.counters + 4 : nullptr;
+  f.w_perm = c.take<float>((size_t)S);
+  // (T <= S: min(S, kGatherMaxT) rows cover every batch that gathers)
+  const int64_t tg = S < kGatherMaxT ? S : kGatherMaxT;
+  f.xg = bs ? c.take<uint8_t>((size_t)(tg * 8 * (w->H / 2))) : nullptr;
+  f.xsl = bs ? c.take<uint8_t>((size_t)(tg * (w->H / (4 * bs)) * 16)) : nullptr;
   return f;
 }
 
@@ -182,12 +205,14 @@ struct ForwardWs {
   Scalars head;
   float* logits;
   int32_t* idx;
+  int32_t* idx_slot;   // forward through an expert cache: the top-k ids as slot ids
   float* w;
   int32_t* offsets;
   int32_t* perm;
   int32_t* inv;
   PermuteScratch pscratch;
   uint16_t* y_perm;
+  float* out32;        // [T][H] fp32 output rows (combine in the down epilogue)
   FfnScratch ffn;
   int32_t* sh_offsets;
   int32_t* sh_perm;
@@ -199,8 +224,9 @@ ForwardWs carve_forward(Carver& c, int64_t T, int k, const moe_weights* routed, 
   const int E = routed->E;
   const int64_t S = T * k;
   f.head = carve_head(c);
-  f.logits = c.take<float>((size_t)T * E * router_parts_max(T, E));
+  f.logits = c.take<float>((size_t)T * E * kRouterParts);
   f.idx = c.take<int32_t>((size_t)S);
+  f.idx_slot = c.take<int32_t>((size_t)S);
   f.w = c.take<float>((size_t)S);
   f.offsets = c.take<int32_t>((size_t)E + 1);
   f.perm = c.take<int32_t>((size_t)S);
@@ -209,6 +235,7 @@ ForwardWs carve_forward(Carver& c, int64_t T, int k, const moe_weights* routed, 
   f.pscratch.chunk_counts = c.take<int32_t>((size_t)(f.pscratch.nchunks > 0 ? f.pscratch.nchunks : 1) * E);
   f.pscratch.ticket = c.take<int32_t>(1);
   f.y_perm = c.take<uint16_t>((size_t)S * routed->H);
+  f.out32 = c.take<float>((size_t)T * routed->H);
   f.ffn = carve_ffn(c, S, routed);
   if (shared) {
     f.sh_offsets = c.take<int32_t>(2);
@@ -243,9 +270,7 @@ __global__ void identity_routing_kernel(int64_t T, int32_t* offsets, int32_t* pe
 cudaError_t run_router(const uint16_t* x, int64_t T, int H, const uint16_t* wr, const float* bias, int E,
                        float* parts, int* nparts, int32_t* status, cudaStream_t s) {
   if (T >= 128 && E % 128 == 0 && H % 64 == 0 && tensor_maps_available()) {
-    int ks = router_ksplit(T, E, H, num_sms());
-    const int cap = router_parts_max(T, E);
-    ks = ks > cap ? cap : ks;
+    const int ks = router_ksplit(T, E, H, num_sms());   // at most kRouterParts
     *nparts = ks;
     return launch_router_gemm(x, T, H, wr, bias, E, parts, T * (int64_t)E, ks, status, num_sms(), s);
   }
@@ -291,63 +316,26 @@ bool ffn_one_kernel(const moe_weights* w, int64_t S) {
          gemm_tile_n(S, w->E) == 64 && w->E <= kFusedMaxE;
 }
 
-// x_ready: the permutation kernel has already quantised x into the padded
-// rows and zeroed the one-kernel FFN's counters (one_kernel only); the FFN
-// then takes its tile list from the top-k ids (slot_expert).
-moe_status run_gemm_ffn(const uint16_t* x, int64_t T, int64_t S, const int32_t* perm, const int32_t* offsets,
-                        const int32_t* inv, int k, const int32_t* slot_expert, const moe_weights* w,
-                        uint16_t* y_perm, const FfnScratch& f,
-                        float* x_amax, float* h_amax, int32_t* status, cudaStream_t s, bool mark, bool planned,
-                        bool x_ready) {
-  const int E = w->E, H = w->H, I = w->I, fmt = w->fmt;
-  const int sms = num_sms();
-  const int bn = gemm_tile_n(S, E);
-  // gate|up projection + SwiGLU quantise h in the epilogue when its scale
-  // needs no global reduction; with 64-token tiles the two projections then
-  // run as one kernel
-  const bool fused_h = h_in_epilogue(w);
-  const bool one_kernel = ffn_one_kernel(w, S);
-  if (x_ready && (!one_kernel || !slot_expert || !planned)) return MOE_ERR_INVALID_ARG;
-  // without a plan from the permutation, the per-slot x quantiser writes it
-  if (mark) stage_mark(MOE_STAGE_ACT_QUANT, false, s);
-  QuantPaddedArgs qa;
-  qa.E = E;
-  qa.K = H;
-  qa.S = S;
-  qa.T = T;
-  qa.P = f.P;
-  qa.offsets = offsets;
-  qa.poff = f.poff;
-  qa.perm_token = perm;
-  qa.inv_perm = inv;
-  qa.k = k;
-  qa.slot_expert = slot_expert;
-  memset(&qa.plan, 0, sizeof(qa.plan));
-  if (!planned) {
-    if (inv) {  // the token quantiser cannot write it
-      MOE_TRY(launch_plan(offsets, E, S, bn, f.poff, f.tiles, f.ntiles, (int)max_tiles(S, E), status, s));
-    } else {
-      qa.plan.bn = bn;
-      qa.plan.poff = f.poff;
-      qa.plan.tiles = f.tiles;
-      qa.plan.ntiles = f.ntiles;
-      qa.plan.max_tiles = (int)max_tiles(S, E);
-    }
-  }
-  qa.x = x;
-  qa.h32 = nullptr;
-  qa.scale = w->a13_gs;
-  qa.amax = x_amax;
-  qa.codes = f.xq;
-  qa.sf = f.xsf;
-  qa.status = status;
-  qa.zero = one_kernel ? f.tile_done : nullptr;   // the one-kernel FFN's counters
-  qa.nzero = one_kernel ? (int)max_tiles(S, E) : 0;
-  if (!x_ready) MOE_TRY(launch_quant_padded(qa, true, fmt, sms, s));
-  if (mark) stage_mark(MOE_STAGE_ACT_QUANT, true, s);
-  GemmArgs g;
+// The weighted combine in the down projection's epilogue
+// (MOE_OPT_FUSED_COMBINE): the routed experts on the grouped GEMM (not the
+// one-kernel FFN) behind the per-token x quantiser, which writes each slot's
+// routing weight by position, and the shared expert, if any, on the grouped
+// GEMM too.  Arguments only.
+bool combine_in_down(const moe_weights* routed, const moe_weights* shared, int64_t T, int k, int act) {
+  const int64_t S = T * k;
+  if (!g_fused_combine || !use_gemm_path(routed, S, act) || ffn_one_kernel(routed, S)) return false;
+  if (routed->fmt == MOE_FMT_BF16 || routed->H % 64 != 0) return false;
+  if (shared && (!use_gemm_path(shared, T, act) || ffn_one_kernel(shared, T))) return false;
+  return true;
+}
+
+// The GEMM arguments of the two projections: gate|up (+ SwiGLU, h in the
+// epilogue when fused_h) over the quantised x rows, down over h.
+void ffn_gemm_args(const moe_weights* w, const FfnScratch& f, int64_t S, float* x_amax, float* h_amax,
+                   int32_t* status, bool fused_h, uint16_t* y_perm, GemmArgs& g, GemmArgs& d) {
+  const int E = w->E, H = w->H, I = w->I;
   memset(&g, 0, sizeof(g));
-  g.fmt = fmt;
+  g.fmt = w->fmt;
   g.E = E;
   g.K = H;
   g.R = 2 * I;
@@ -365,18 +353,10 @@ moe_status run_gemm_ffn(const uint16_t* x, int64_t T, int64_t S, const int32_t* 
   g.h32 = f.h32;
   g.h_amax = fused_h ? nullptr : h_amax;
   g.status = status;
-  // the tile list is two kernels back when the permutation or the plan kernel
-  // wrote it; when the x quantiser just before writes it, the expert offsets
-  // (older) name the experts of the early weight loads
-  const int ew = early_weights();
-  g.w_early = ew == 0 ? 0 : ((planned || inv) ? 1 : 2);
-  g.w_early_l2 = ew == 2 ? kEarlyL2Stages : 0;
-  g.offsets = offsets;
   g.max_tiles = (int)max_tiles(S, E);
-  // down projection -> y_perm
-  GemmArgs d;
+  g.wait_cycles = wait_cycles();
   memset(&d, 0, sizeof(d));
-  d.fmt = fmt;
+  d.fmt = w->fmt;
   d.E = E;
   d.K = I;
   d.R = H;
@@ -392,22 +372,120 @@ moe_status run_gemm_ffn(const uint16_t* x, int64_t T, int64_t S, const int32_t* 
   d.ldy = H;
   d.y_rows = S;
   d.status = status;
+  d.max_tiles = g.max_tiles;
+  d.wait_cycles = g.wait_cycles;
+}
+
+// Small batches whose x goes to the gather layout (the one-kernel FFN copies
+// its token rows from there, so no permutation is waited for).
+bool gather_x(const moe_weights* w, int64_t T) {
+  return T <= kGatherMaxT && (w->fmt == MOE_FMT_NVFP4 || w->fmt == MOE_FMT_MXFP4) && w->H % 256 == 0;
+}
+
+// x_ready: the permutation kernel has already quantised x into the padded
+// rows (one_kernel only); the FFN then takes its tile list from the top-k ids
+// (slot_expert).
+moe_status run_gemm_ffn(const uint16_t* x, int64_t T, int64_t S, const int32_t* perm, const int32_t* offsets,
+                        const int32_t* inv, int k, const int32_t* slot_expert, const moe_weights* w,
+                        uint16_t* y_perm, const FfnScratch& f,
+                        float* x_amax, float* h_amax, int32_t* status, cudaStream_t s, bool mark, bool planned,
+                        bool x_ready, const float* topk_w, float* out32) {
+  const int E = w->E, H = w->H, fmt = w->fmt;
+  const int sms = num_sms();
+  const int bn = gemm_tile_n(S, E);
+  // gate|up projection + SwiGLU quantise h in the epilogue when its scale
+  // needs no global reduction; with 64-token tiles the two projections then
+  // run as one kernel
+  const bool fused_h = h_in_epilogue(w);
+  const bool one_kernel = ffn_one_kernel(w, S);
+  // small batches on the one-kernel FFN: x in the gather layout
+  const bool gather = one_kernel && !x_ready && gather_x(w, T);
+  if (x_ready && (!one_kernel || !slot_expert || !planned)) return MOE_ERR_INVALID_ARG;
+  if (out32 && one_kernel) return MOE_ERR_INVALID_ARG;
+  if (out32 && topk_w && (!inv || fmt == MOE_FMT_BF16 || H % 64 != 0)) return MOE_ERR_INVALID_ARG;
+  if (mark) stage_mark(MOE_STAGE_ACT_QUANT, false, s);
+  // the one-kernel FFN's counters are read before that kernel waits for the
+  // one before it, so they are cleared a step earlier (with x_ready, the
+  // forward cleared them before the router)
+  if (one_kernel && !x_ready) MOE_TRY(cudaMemsetAsync(f.counters, 0, counters_bytes(S, E), s));
+  if (gather) {
+    GatherQuant gq{w->a13_gs, x_amax, f.xg, f.xsl};
+    MOE_TRY(launch_quant_gather(fmt, x, T, H, gq, s));
+  } else {
+    QuantPaddedArgs qa;
+    memset(&qa, 0, sizeof(qa));
+    qa.E = E;
+    qa.K = H;
+    qa.S = S;
+    qa.T = T;
+    qa.P = f.P;
+    qa.offsets = offsets;
+    qa.poff = f.poff;
+    qa.perm_token = perm;
+    qa.inv_perm = inv;
+    qa.k = k;
+    qa.slot_expert = slot_expert;
+    // the combine in the down epilogue reads each slot's routing weight by
+    // position; the token quantiser writes it on the way
+    qa.topk_w = out32 ? topk_w : nullptr;
+    qa.w_perm = out32 && topk_w ? f.w_perm : nullptr;
+    if (!planned) {
+      if (inv) {  // the token quantiser cannot write it
+        MOE_TRY(launch_plan(offsets, E, S, bn, f.poff, f.tiles, f.ntiles, (int)max_tiles(S, E), status, s));
+      } else {
+        qa.plan.bn = bn;
+        qa.plan.poff = f.poff;
+        qa.plan.tiles = f.tiles;
+        qa.plan.ntiles = f.ntiles;
+        qa.plan.max_tiles = (int)max_tiles(S, E);
+      }
+    }
+    qa.x = x;
+    qa.scale = w->a13_gs;
+    qa.amax = x_amax;
+    qa.codes = f.xq;
+    qa.sf = f.xsf;
+    qa.status = status;
+    if (!x_ready) MOE_TRY(launch_quant_padded(qa, true, fmt, sms, s));
+  }
+  if (mark) stage_mark(MOE_STAGE_ACT_QUANT, true, s);
+  GemmArgs g, d;
+  ffn_gemm_args(w, f, S, x_amax, h_amax, status, fused_h, y_perm, g, d);
+  // the tile list is two kernels back when the permutation or the plan kernel
+  // wrote it; when the x quantiser just before writes it, the expert offsets
+  // (older) name the experts of the early weight loads
+  const int ew = early_weights();
+  g.w_early = ew == 0 ? 0 : ((planned || inv) ? 1 : 2);
+  g.w_early_l2 = ew == 2 ? kEarlyL2Stages : 0;
+  g.offsets = offsets;
   d.w_early = ew == 0 ? 0 : 1;  // the tile list is at least two kernels back
   d.w_early_l2 = g.w_early_l2;
-  d.max_tiles = g.max_tiles;
+  d.out32 = out32;
+  d.perm_token = perm;
+  d.w_perm = out32 && topk_w ? f.w_perm : nullptr;
+  d.out_rows = T;
   if (one_kernel) {
     // the weights are older than the quantiser: the first stages load before
     // the wait (the tile list comes from the offsets in the kernel)
     g.w_early = ew == 0 ? 0 : 1;
     FusedArgs fa;
+    memset(&fa, 0, sizeof(fa));
     fa.offsets = offsets;
     fa.slot_expert = x_ready ? slot_expert : nullptr;   // the offsets are one kernel back then
     fa.S = S;
     fa.P = f.P;
     fa.tile_done = f.tile_done;
+    fa.work = f.work;
     fa.max_tiles = (int)max_tiles(S, E);
+    if (gather) {
+      fa.xg = f.xg;
+      fa.xsl = f.xsl;
+      fa.perm_token = perm;
+      fa.k = k > 0 ? k : 1;
+      fa.T = T;
+    }
     if (mark) stage_mark(MOE_STAGE_FFN_UP, false, s);
-    MOE_TRY(launch_fused_ffn(g, d, fa, w->w13, (int64_t)E * 2 * I, w->w2, (int64_t)E * H, f.xq, f.hq, sms, s));
+    MOE_TRY(launch_fused_ffn(g, d, fa, w->w13, (int64_t)E * 2 * w->I, w->w2, (int64_t)E * H, f.xq, f.hq, sms, s));
     if (mark) {
       stage_mark(MOE_STAGE_FFN_UP, true, s);
       stage_mark(MOE_STAGE_FFN_DOWN, false, s);
@@ -417,16 +495,24 @@ moe_status run_gemm_ffn(const uint16_t* x, int64_t T, int64_t S, const int32_t* 
   }
   if (mark) stage_mark(MOE_STAGE_FFN_UP, false, s);
   if (!fused_h) MOE_TRY(cudaMemsetAsync(h_amax, 0, sizeof(float), s));
-  MOE_TRY(launch_grouped_gemm(g, fused_h ? kEpiUpQuant : kEpiUpF32, bn, w->w13, (int64_t)E * 2 * I,
+  MOE_TRY(launch_grouped_gemm(g, fused_h ? kEpiUpQuant : kEpiUpF32, bn, w->w13, (int64_t)E * 2 * w->I,
                               f.xq, f.P, sms, s));
   if (!fused_h) {
-    QuantPaddedArgs qh = qa;
-    qh.K = I;
+    QuantPaddedArgs qh;
+    memset(&qh, 0, sizeof(qh));
+    qh.E = E;
+    qh.K = w->I;
+    qh.S = S;
+    qh.T = T;
+    qh.P = f.P;
+    qh.offsets = offsets;
+    qh.poff = f.poff;
     qh.h32 = f.h32;
     qh.scale = w->a2_gs;
     qh.amax = h_amax;
     qh.codes = f.hq;
     qh.sf = f.hsf;
+    qh.status = status;
     MOE_TRY(launch_quant_padded(qh, false, fmt, sms, s));
   }
   if (mark) stage_mark(MOE_STAGE_FFN_UP, true, s);
@@ -444,13 +530,14 @@ moe_status run_grouped_ffn(const uint16_t* x, int64_t T, int64_t S, const int32_
                            const moe_weights* w, int act, uint16_t* y_perm, const FfnScratch& scratch,
                            float* x_amax, float* h_amax, int32_t* status, cudaStream_t s,
                            bool shared_stage = false, const int32_t* inv = nullptr, int k = 0,
-                           const int32_t* slot_expert = nullptr, bool planned = false, bool x_ready = false) {
+                           const int32_t* slot_expert = nullptr, bool planned = false, bool x_ready = false,
+                           const float* topk_w = nullptr, float* out32 = nullptr) {
   if (S == 0) return MOE_OK;
   const bool mark = !shared_stage;
   if (use_gemm_path(w, S, act))
     return run_gemm_ffn(x, T, S, perm, offsets, inv, k, slot_expert, w, y_perm, scratch, x_amax, h_amax, status, s,
-                        mark, planned, x_ready);
-  if (x_ready) return MOE_ERR_INVALID_ARG;
+                        mark, planned, x_ready, topk_w, out32);
+  if (x_ready || out32) return MOE_ERR_INVALID_ARG;
   if (g_ffn_path == 2 || w->fmt == MOE_FMT_BF16) return MOE_ERR_UNSUPPORTED;   // the GEMV has no BF16 weights
   GemvArgs a;
   a.fmt = w->fmt;
@@ -478,6 +565,7 @@ moe_status run_grouped_ffn(const uint16_t* x, int64_t T, int64_t S, const int32_
   a.tiles = scratch.tiles;
   a.num_tiles = scratch.ntiles;
   a.status = status;
+  a.wait_cycles = wait_cycles();
   const int sms = num_sms();
   if (!planned)
     MOE_TRY(launch_plan(offsets, w->E, S, kGemvTokens, scratch.poff, scratch.tiles, scratch.ntiles,
@@ -562,7 +650,7 @@ moe_status copy_streams(cudaStream_t* in, cudaStream_t* out) {
 // Events of one moe_forward_host call, released when it returns (the driver
 // frees a pending event's resources once it completes).
 struct EventSet {
-  cudaEvent_t ev[2 * MOE_MAX_HOST_SLICES + 2] = {};
+  cudaEvent_t ev[2 * MOE_MAX_HOST_SLICES + 3] = {};
   int n = 0;
   moe_status create(int count) {
     for (; n < count; ++n)
@@ -578,6 +666,9 @@ struct EventSet {
 
 static int g_pdl = 1;  // MOE_OPT_PDL
 bool pdl_enabled() { return g_pdl != 0; }
+
+static long long g_wait_cycles = tc_default_wait_cycles();  // MOE_OPT_WAIT_CYCLES
+long long wait_cycles() { return g_wait_cycles; }
 
 static uint64_t g_launches = 0;
 static std::mutex g_launch_mu;
@@ -640,6 +731,21 @@ moe_status moe_set_option(int32_t option, int32_t value) {
   if (option == MOE_OPT_EARLY_WEIGHTS) {
     if (value < 0 || value > 2) return MOE_ERR_INVALID_ARG;
     set_early_weights(value);
+    return MOE_OK;
+  }
+  if (option == MOE_OPT_SMALL_BATCH_FORWARD) {
+    if (value != 0 && value != 1) return MOE_ERR_INVALID_ARG;
+    g_small_forward = value;
+    return MOE_OK;
+  }
+  if (option == MOE_OPT_FUSED_COMBINE) {
+    if (value != 0 && value != 1) return MOE_ERR_INVALID_ARG;
+    g_fused_combine = value;
+    return MOE_OK;
+  }
+  if (option == MOE_OPT_WAIT_CYCLES) {
+    if (value < 0) return MOE_ERR_INVALID_ARG;
+    g_wait_cycles = value == 0 ? tc_default_wait_cycles() : (long long)value;
     return MOE_OK;
   }
   if (option == MOE_OPT_GEMM_PAIR) {
@@ -863,6 +969,67 @@ moe_status moe_forward(const uint16_t* x, int64_t T, const uint16_t* wr, const f
   if (T == 0) return MOE_OK;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int64_t S = T * k;
+  // Small batches on the one-kernel FFN with no shared expert: two kernels.
+  // The router computes the logits, quantises x into the gather layout and
+  // picks every token's top k in its last block; the FFN takes its tiles from
+  // the top-k ids (a tile's rows are its expert's slots in flat order, so no
+  // permutation is needed), copies the token rows from the gather layout,
+  // adds w * y into fp32 output rows in its down epilogue, and its last CTA
+  // rounds them into `out`.
+  const bool small2 = g_small_forward && !shared && act == MOE_ACT_MATCH && use_gemm_path(routed, S, act) &&
+                      ffn_one_kernel(routed, S) && gather_x(routed, T) && H % 8 == 0;
+  if (small2) {
+    MOE_TRY(cudaMemsetAsync(f.ffn.counters, 0, counters_bytes(S, E), s));
+    MOE_TRY(cudaMemsetAsync(f.out32, 0, sizeof(float) * (size_t)T * H, s));
+    if (dynamic_x_scale(routed, act)) {
+      stage_mark(MOE_STAGE_ACT_QUANT, false, s);
+      MOE_TRY(launch_amax(x, 1, T * H, f.head.x_amax, num_sms(), s));
+      stage_mark(MOE_STAGE_ACT_QUANT, true, s);
+    }
+    stage_mark(MOE_STAGE_ROUTE, false, s);
+    const GatherQuant gq{routed->a13_gs, f.head.x_amax, f.ffn.xg, f.ffn.xsl};
+    MOE_TRY(launch_router_decode(routed->fmt, x, T, H, wr, bias, E, k, f.logits, f.idx, f.w, f.ffn.ticket, gq,
+                                 f.head.status, s));
+    stage_mark(MOE_STAGE_ROUTE, true, s);
+    GemmArgs g, d;
+    ffn_gemm_args(routed, f.ffn, S, f.head.x_amax, f.head.h_amax, f.head.status, true, f.y_perm, g, d);
+    g.w_early = early_weights() == 0 ? 0 : 1;
+    d.w_early = g.w_early;
+    d.out32 = f.out32;
+    d.out_rows = T;
+    FusedArgs fa;
+    memset(&fa, 0, sizeof(fa));
+    fa.offsets = f.offsets;
+    fa.slot_expert = f.idx;
+    fa.S = S;
+    fa.P = f.ffn.P;
+    fa.tile_done = f.ffn.tile_done;
+    fa.work = f.ffn.work;
+    fa.max_tiles = (int)max_tiles(S, E);
+    fa.xg = f.ffn.xg;
+    fa.xsl = f.ffn.xsl;
+    fa.k = k;
+    fa.topk_w = f.w;
+    fa.out = out;
+    fa.done = f.ffn.done;
+    fa.T = T;
+    stage_mark(MOE_STAGE_FFN_UP, false, s);
+    MOE_TRY(launch_fused_ffn(g, d, fa, routed->w13, (int64_t)E * 2 * routed->I, routed->w2, (int64_t)E * H,
+                             f.ffn.xq, f.ffn.hq, num_sms(), s));
+    stage_mark(MOE_STAGE_FFN_UP, true, s);
+    return MOE_OK;
+  }
+  // Small batches on the one-kernel FFN: the one-block permutation also
+  // quantises x, and the FFN takes its tile list from the top-k ids (two
+  // kernels back), so its first weight loads go out while the permutation
+  // runs.  The FFN's item counter is cleared here, before the router.
+  const bool want_q = g_perm_quant && act == MOE_ACT_MATCH && use_gemm_path(routed, S, act) &&
+                      ffn_one_kernel(routed, S) && H % 64 == 0 && permute_can_quantize(S, T, E);
+  if (want_q) MOE_TRY(cudaMemsetAsync(f.ffn.counters, 0, counters_bytes(S, E), s));
+  // The weighted combine in the down epilogues (routed and shared experts
+  // add into fp32 rows, cleared here, before the fork), then one rounding pass.
+  const bool fused_combine = combine_in_down(routed, shared, T, k, act);
+  if (fused_combine) MOE_TRY(cudaMemsetAsync(f.out32, 0, sizeof(float) * (size_t)T * H, s));
   // 1. dynamic activation scale of x (shared by routed and shared experts)
   if (dynamic_x_scale(routed, act)) {
     stage_mark(MOE_STAGE_ACT_QUANT, false, s);
@@ -887,7 +1054,8 @@ moe_status moe_forward(const uint16_t* x, int64_t T, const uint16_t* wr, const f
       moe_weights sh = *shared;
       sh.a13_gs = routed->a13_gs;
       st = run_grouped_ffn(x, T, T, f.sh_perm, f.sh_offsets, &sh, act, f.sh_y, f.sh_ffn, f.head.x_amax,
-                           f.head.sh_h_amax, f.head.status, s2, true);
+                           f.head.sh_h_amax, f.head.status, s2, true, nullptr, 0, nullptr, false, false, nullptr,
+                           fused_combine ? f.out32 : nullptr);
     }
     stage_mark(MOE_STAGE_SHARED, true, s2);
     if (st != MOE_OK) {
@@ -909,14 +1077,8 @@ moe_status moe_forward(const uint16_t* x, int64_t T, const uint16_t* wr, const f
   plan.tiles = f.ffn.tiles;
   plan.ntiles = f.ffn.ntiles;
   plan.max_tiles = (int)max_tiles(S, E);
-  // Small batches on the one-kernel FFN: the one-block permutation also
-  // quantises x, and the FFN takes its tile list from the top-k ids (two
-  // kernels back), so its first weight loads go out while the permutation
-  // runs.
   SlotQuantOut q;
   memset(&q, 0, sizeof(q));
-  const bool want_q = g_perm_quant && act == MOE_ACT_MATCH && use_gemm_path(routed, S, act) &&
-                      ffn_one_kernel(routed, S) && H % 64 == 0 && permute_can_quantize(S, T, E);
   if (want_q) {
     q.fmt = routed->fmt;
     q.x = x;
@@ -926,8 +1088,6 @@ moe_status moe_forward(const uint16_t* x, int64_t T, const uint16_t* wr, const f
     q.amax = f.head.x_amax;
     q.codes = f.ffn.xq;
     q.sf = f.ffn.xsf;
-    q.zero = f.ffn.tile_done;
-    q.nzero = (int)max_tiles(S, E);
   }
   bool planned = false, x_ready = false;
   if (st == MOE_OK) {
@@ -939,15 +1099,19 @@ moe_status moe_forward(const uint16_t* x, int64_t T, const uint16_t* wr, const f
   // 5. routed experts
   if (st == MOE_OK)
     st = run_grouped_ffn(x, T, S, f.perm, f.offsets, routed, act, f.y_perm, f.ffn, f.head.x_amax, f.head.h_amax,
-                         f.head.status, s, false, f.inv, k, f.idx, planned, x_ready);
+                         f.head.status, s, false, f.inv, k, f.idx, planned, x_ready, f.w,
+                         fused_combine ? f.out32 : nullptr);
   if (shared) {
     const moe_status js = side.join(s);
     if (st == MOE_OK) st = js;
   }
   if (st != MOE_OK) return st;
-  // 6. combine
+  // 6. combine (or, when the down epilogues did it, the rounding to bf16)
   stage_mark(MOE_STAGE_COMBINE, false, s);
-  st = cuda_status(launch_combine(f.y_perm, f.inv, f.w, T, k, H, f.sh_y, out, f.head.status, s));
+  if (fused_combine)
+    st = cuda_status(launch_round_rows(f.out32, T * (int64_t)H, out, num_sms(), s));
+  else
+    st = cuda_status(launch_combine(f.y_perm, f.inv, f.w, T, k, H, f.sh_y, out, f.head.status, s));
   stage_mark(MOE_STAGE_COMBINE, true, s);
   return st;
 }
@@ -982,11 +1146,11 @@ moe_status moe_forward_host(const uint16_t* x_host, int64_t T, const uint16_t* w
   st = copy_streams(&s_in, &s_out);
   if (st != MOE_OK) return st;
   EventSet es;
-  st = es.create((int)(2 * n + 2));
+  st = es.create((int)(2 * n + 3));
   if (st != MOE_OK) return st;
-  cudaEvent_t ev_start = es.ev[0], ev_end = es.ev[1];
-  cudaEvent_t* in_done = es.ev + 2;
-  cudaEvent_t* fwd_done = es.ev + 2 + n;
+  cudaEvent_t ev_start = es.ev[0], ev_end = es.ev[1], ev_in_end = es.ev[2];
+  cudaEvent_t* in_done = es.ev + 3;
+  cudaEvent_t* fwd_done = es.ev + 3 + n;
   const size_t row = (size_t)H * sizeof(uint16_t);
   // the copy streams start after the work already on the caller's stream
   if (cudaEventRecord(ev_start, s) != cudaSuccess || cudaStreamWaitEvent(s_in, ev_start, 0) != cudaSuccess ||
@@ -1015,18 +1179,182 @@ moe_status moe_forward_host(const uint16_t* x_host, int64_t T, const uint16_t* w
             cudaSuccess)
       st = MOE_ERR_CUDA;
   }
-  // the caller's stream waits for the last copy-out (also after an error,
-  // so that no copy of this call is left unordered against later work)
-  const bool joined = cudaEventRecord(ev_end, s_out) == cudaSuccess && cudaStreamWaitEvent(s, ev_end, 0) == cudaSuccess;
+  // the caller's stream waits for the last copy-in and the last copy-out
+  // (also after an error, so that no copy of this call is left unordered
+  // against later work on `stream`, and a capture of `stream` joins both
+  // copy streams)
+  const bool joined = cudaEventRecord(ev_in_end, s_in) == cudaSuccess &&
+                      cudaEventRecord(ev_end, s_out) == cudaSuccess &&
+                      cudaStreamWaitEvent(s, ev_in_end, 0) == cudaSuccess &&
+                      cudaStreamWaitEvent(s, ev_end, 0) == cudaSuccess;
   if (st == MOE_OK && !joined) st = MOE_ERR_CUDA;
   return st;
 }
 
+size_t moe_expert_cache_bytes(const moe_weights* bank, int32_t n_slots) {
+  if (check_weights(bank, true) != MOE_OK || n_slots < 1 || n_slots > bank->E || n_slots > 1024) return 0;
+  moe_weights one = *bank;
+  one.E = n_slots;
+  one.layout = MOE_LAYOUT_CANONICAL;
+  const size_t pool = moe_prepared_weights_size(&one);
+  Carver c(nullptr);
+  c.take<uint8_t>(pool);
+  c.take<float>((size_t)n_slots * 2);
+  c.take<float>((size_t)n_slots);
+  c.take<int32_t>(cache_state_words(bank->E, n_slots));
+  return align_up(c.off, kAlign);
+}
+
+moe_status moe_expert_cache_init(const moe_weights* bank, int32_t n_slots, void* dev, size_t dev_bytes,
+                                 moe_expert_cache* cache, moe_stream_t stream) {
+  moe_status st = check_weights(bank, true);
+  if (st != MOE_OK) return st;
+  if (!cache || !dev || n_slots < 1 || n_slots > bank->E || n_slots > 1024) return MOE_ERR_INVALID_ARG;
+  if (dev_bytes < moe_expert_cache_bytes(bank, n_slots)) return MOE_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  moe_expert_cache cc;
+  memset(&cc, 0, sizeof(cc));
+  cc.bank = *bank;
+  cc.n_slots = n_slots;
+  // device addresses of the host arrays (they must be mapped)
+  const void* host[6] = {bank->w13, bank->w13_sf, bank->w13_gs, bank->w2, bank->w2_sf, bank->w2_gs};
+  for (int i = 0; i < 6; ++i) {
+    if (!host[i]) continue;
+    void* d = nullptr;
+    if (cudaHostGetDevicePointer(&d, const_cast<void*>(host[i]), 0) != cudaSuccess || !d) {
+      cudaGetLastError();   // clear the error this query leaves behind
+      return MOE_ERR_INVALID_ARG;
+    }
+    cc.bank_dev[i] = d;
+  }
+  // the pool: a PREPARED bank of n_slots experts, then its part scales and the state
+  const int64_t n = n_slots, H = bank->H, I = bank->I;
+  const int bs = block_size(bank->fmt);
+  const int64_t rb13 = fmt_row_bytes(bank->fmt, H), rb2 = fmt_row_bytes(bank->fmt, I);
+  Carver c(dev);
+  uint8_t* w13 = c.take<uint8_t>((size_t)(n * 2 * I * rb13));
+  uint8_t* w2 = c.take<uint8_t>((size_t)(n * H * rb2));
+  uint8_t* sf13 = bs ? c.take<uint8_t>((size_t)(n * 2 * I * (H / bs))) : nullptr;
+  uint8_t* sf2 = bs ? c.take<uint8_t>((size_t)(n * H * (I / bs))) : nullptr;
+  float* gs13 = c.take<float>((size_t)n * 2);
+  float* gs2 = c.take<float>((size_t)n);
+  int32_t* state = c.take<int32_t>(cache_state_words(bank->E, n_slots));
+  cc.pool = *bank;
+  cc.pool.E = n_slots;
+  cc.pool.w13 = w13;
+  cc.pool.w2 = w2;
+  cc.pool.w13_sf = sf13;
+  cc.pool.w2_sf = sf2;
+  cc.pool.w13_gs = bank->w13_gs ? gs13 : nullptr;
+  cc.pool.w2_gs = bank->w2_gs ? gs2 : nullptr;
+  cc.state = state;
+  // empty pool: clock and counters 0, slot_of / expert_of -1, stamps 0
+  const size_t words = cache_state_words(bank->E, n_slots);
+  MOE_TRY(cudaMemsetAsync(state, 0, words * sizeof(int32_t), s));
+  MOE_TRY(cudaMemsetAsync(state + 4, 0xFF, ((size_t)bank->E + n_slots) * sizeof(int32_t), s));
+  *cache = cc;
+  return MOE_OK;
+}
+
+moe_status moe_forward_cached(const uint16_t* x, int64_t T, const uint16_t* wr, const float* bias, int32_t k,
+                              const moe_expert_cache* cache, int32_t act, uint16_t* out, void* ws, size_t ws_bytes,
+                              moe_stream_t stream) {
+  if (!cache) return MOE_ERR_INVALID_ARG;
+  moe_status st = check_weights(&cache->bank, true);
+  if (st != MOE_OK) return st;
+  st = check_weights(&cache->pool, true);
+  if (st != MOE_OK) return st;
+  const moe_weights* bank = &cache->bank;
+  const moe_weights* pool = &cache->pool;
+  const int E = bank->E, H = bank->H, n = cache->n_slots;
+  if (T < 0 || k < 1 || k > E || (act != MOE_ACT_BF16 && act != MOE_ACT_MATCH)) return MOE_ERR_INVALID_ARG;
+  if (T * (int64_t)k > INT32_MAX) return MOE_ERR_INVALID_ARG;
+  if (T > 0 && (!x || !wr || !out)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(wr) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+  const int64_t S = T * k;
+  if ((int64_t)n < (S < E ? S : E)) return MOE_ERR_INVALID_ARG;   // a batch must fit in the pool
+  Carver c(ws);
+  ForwardWs f = carve_forward(c, T, k, bank, nullptr);
+  if (!ws || ws_bytes < c.off) return MOE_ERR_WORKSPACE;
+  if (T == 0) return MOE_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (dynamic_x_scale(pool, act)) MOE_TRY(launch_amax(x, 1, T * H, f.head.x_amax, num_sms(), s));
+  // route on the whole bank's router
+  stage_mark(MOE_STAGE_ROUTE, false, s);
+  int nparts = 1;
+  MOE_TRY(run_router(x, T, H, wr, bias, E, f.logits, &nparts, f.head.status, s));
+  MOE_TRY(launch_topk(f.logits, nparts, T * (int64_t)E, nullptr, T, E, k, f.idx, f.w, f.head.status, s));
+  stage_mark(MOE_STAGE_ROUTE, true, s);
+  // admit the batch's experts into slots and fetch the missing ones
+  MOE_TRY(launch_cache_admit(f.idx, S, E, n, cache->state, f.idx_slot, f.head.status, s));
+  CacheCopy cc;
+  memset(&cc, 0, sizeof(cc));
+  const int64_t I = bank->I;
+  const int bs = block_size(bank->fmt);
+  const int64_t rb13 = fmt_row_bytes(bank->fmt, H), rb2 = fmt_row_bytes(bank->fmt, I);
+  cc.src[0] = static_cast<const uint8_t*>(cache->bank_dev[0]);
+  cc.dst[0] = const_cast<uint8_t*>(pool->w13);
+  cc.bytes[0] = 2 * I * rb13;
+  cc.src[1] = static_cast<const uint8_t*>(cache->bank_dev[3]);
+  cc.dst[1] = const_cast<uint8_t*>(pool->w2);
+  cc.bytes[1] = H * rb2;
+  cc.nregions = 2;
+  if (bs) {
+    cc.src[2] = static_cast<const uint8_t*>(cache->bank_dev[1]);
+    cc.dst[2] = const_cast<uint8_t*>(pool->w13_sf);
+    cc.bytes[2] = 2 * I * (H / bs);
+    cc.src[3] = static_cast<const uint8_t*>(cache->bank_dev[4]);
+    cc.dst[3] = const_cast<uint8_t*>(pool->w2_sf);
+    cc.bytes[3] = H * (I / bs);
+    cc.nregions = 4;
+  }
+  if (bank->w13_gs) {
+    cc.gs_src[0] = static_cast<const float*>(cache->bank_dev[2]);
+    cc.gs_dst[0] = const_cast<float*>(pool->w13_gs);
+    cc.gs_per[0] = 2;
+    cc.gs_src[1] = static_cast<const float*>(cache->bank_dev[5]);
+    cc.gs_dst[1] = const_cast<float*>(pool->w2_gs);
+    cc.gs_per[1] = 1;
+    cc.ngs = 2;
+  }
+  MOE_TRY(launch_cache_fetch(cache->state, E, n, cc, num_sms(), s));
+  // the layer on the pool: slot ids are the experts now
+  stage_mark(MOE_STAGE_PERMUTE, false, s);
+  PlanOut plan;
+  plan.bn = use_gemm_path(pool, S, act) ? gemm_tile_n(S, n) : kGemvTokens;
+  plan.poff = f.ffn.poff;
+  plan.tiles = f.ffn.tiles;
+  plan.ntiles = f.ffn.ntiles;
+  plan.max_tiles = (int)max_tiles(S, n);
+  bool planned = false;
+  MOE_TRY(launch_permute(f.idx_slot, S, k, n, f.offsets, f.perm, f.inv, f.pscratch, f.head.status, s, &plan,
+                         &planned));
+  stage_mark(MOE_STAGE_PERMUTE, true, s);
+  st = run_grouped_ffn(x, T, S, f.perm, f.offsets, pool, act, f.y_perm, f.ffn, f.head.x_amax, f.head.h_amax,
+                       f.head.status, s, false, f.inv, k, f.idx_slot, planned, false);
+  if (st != MOE_OK) return st;
+  stage_mark(MOE_STAGE_COMBINE, false, s);
+  st = cuda_status(launch_combine(f.y_perm, f.inv, f.w, T, k, H, nullptr, out, f.head.status, s));
+  stage_mark(MOE_STAGE_COMBINE, true, s);
+  return st;
+}
+
+moe_status moe_expert_cache_stats(const moe_expert_cache* cache, moe_stream_t stream, int64_t* stats) {
+  if (!cache || !cache->state || !stats) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int32_t h[4] = {0, 0, 0, 0};
+  if (cudaMemcpyAsync(h, cache->state, sizeof(h), cudaMemcpyDeviceToHost, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+  for (int i = 0; i < 4; ++i) stats[i] = h[i];
+  return MOE_OK;
+}
+
 moe_status moe_set_stage_events(void* const* events, int32_t n_events) {
   if (!events) {
-    g_stage_on = false;
+    g_stage_on = false;   // the mask keeps what the hook recorded
     return MOE_OK;
   }
+  g_stage_mask = 0;
   if (n_events < 2 * MOE_STAGE_COUNT) return MOE_ERR_INVALID_ARG;
   for (int i = 0; i < 2 * MOE_STAGE_COUNT; ++i) {
     if (!events[i]) return MOE_ERR_INVALID_ARG;
@@ -1035,6 +1363,8 @@ moe_status moe_set_stage_events(void* const* events, int32_t n_events) {
   g_stage_on = true;
   return MOE_OK;
 }
+
+uint32_t moe_stage_mask(void) { return g_stage_mask; }
 
 uint64_t moe_kernel_launch_count(void) { return launches_so_far(); }
 

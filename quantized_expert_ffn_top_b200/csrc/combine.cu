@@ -97,4 +97,34 @@ cudaError_t launch_combine(const uint16_t* y_perm, const int32_t* inv_perm, cons
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 
+// The last step of a forward whose down projection added w * y into fp32
+// rows (the combine in the down epilogue): out = bf16(out32), round to
+// nearest even, eight values a thread.
+__global__ void __launch_bounds__(256) round_rows_kernel(const float* __restrict__ out32, int64_t n8,
+                                                         uint16_t* __restrict__ out) {
+  pdl_wait();  // inputs come from the previous kernels
+  pdl_trigger();
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += (int64_t)gridDim.x * blockDim.x) {
+    const float4 a = __ldcs(reinterpret_cast<const float4*>(out32) + 2 * i);
+    const float4 b = __ldcs(reinterpret_cast<const float4*>(out32) + 2 * i + 1);
+    uint4 o;
+    o.x = (uint32_t)f32_to_bf16_rn(a.x) | ((uint32_t)f32_to_bf16_rn(a.y) << 16);
+    o.y = (uint32_t)f32_to_bf16_rn(a.z) | ((uint32_t)f32_to_bf16_rn(a.w) << 16);
+    o.z = (uint32_t)f32_to_bf16_rn(b.x) | ((uint32_t)f32_to_bf16_rn(b.y) << 16);
+    o.w = (uint32_t)f32_to_bf16_rn(b.z) | ((uint32_t)f32_to_bf16_rn(b.w) << 16);
+    reinterpret_cast<uint4*>(out)[i] = o;
+  }
+}
+
+cudaError_t launch_round_rows(const float* out32, int64_t n, uint16_t* out, int num_sms, cudaStream_t s) {
+  if (n == 0) return cudaSuccess;
+  if (n % 8 != 0) return cudaErrorInvalidValue;
+  const int64_t n8 = n / 8;
+  const int64_t blocks = (n8 + 255) / 256;
+  const int grid = (int)(blocks < (int64_t)num_sms * 8 ? blocks : (int64_t)num_sms * 8);
+  cudaError_t e = launch_pdl(round_rows_kernel, dim3(grid), dim3(256), 0, s, out32, n8, out);
+  count_launches(1);
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
+
 }  // namespace moe

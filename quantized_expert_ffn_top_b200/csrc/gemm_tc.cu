@@ -322,7 +322,7 @@ __device__ __forceinline__ void epilogue_slice(const GemmArgs& g, const CUtensor
                                                float gact, float g2, float* epi_tiles, const float* r_tab,
                                                uint16_t* y_stage, int ybufs, int& ypar, float& hmax,
                                                const uint32_t* r0, const uint32_t* r1, const uint32_t* r2,
-                                               const uint32_t* r3) {
+                                               const uint32_t* r3, int ltok = -1, float lw = 0.0f) {
 #pragma unroll
   for (int ch = 0; ch < 4; ++ch) {
     if (ch >= nch) break;  // both warps of a pair see the same ncol
@@ -342,6 +342,39 @@ __device__ __forceinline__ void epilogue_slice(const GemmArgs& g, const CUtensor
       }
     } else if (EPI == kEpiDown) {
       const float sc = (FMT == MOE_FMT_MXFP4 || FMT == kFmtBF16) ? 1.0f : __ldg(g.w_gs + te.e) * gact;
+      if (g.out32) {
+        // the weighted un-permute in the epilogue: lanes 0..15 fetch the
+        // chunk's tokens and routing weights, every lane adds w * y for its
+        // output row (32 consecutive floats per warp and token: one L2
+        // reduction transaction)
+        const int o = mt * 128 + q * 32 + lane;
+        int tk = -1;
+        float wt = 0.0f;
+        if (!g.perm_token) {
+          // rows below 32 (gather mode): lane r already holds row r's token and weight
+          const int st = __shfl_sync(0xffffffffu, ltok, (c0 + lane) & 31);
+          const float sw = __shfl_sync(0xffffffffu, lw, (c0 + lane) & 31);
+          if (lane < 16 && c0 + lane < te.nvalid && c0 + lane < 32) {
+            tk = st;
+            wt = sw;
+          }
+        } else if (lane < 16 && c0 + lane < te.nvalid) {
+          const int p = te.p0 + c0 + lane;
+          tk = __ldg(g.perm_token + p);
+          wt = g.w_perm ? __ldg(g.w_perm + p) : 1.0f;
+        }
+        if (tk >= g.out_rows || (lane < 16 && c0 + lane < te.nvalid && tk < 0)) {
+          raise_status(g.status, MOE_ERR_DEVICE_FAULT);
+          tk = -1;
+        }
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const int t = __shfl_sync(0xffffffffu, tk, c);
+          const float ww = __shfl_sync(0xffffffffu, wt, c);
+          if (t >= 0) atomicAdd(g.out32 + (size_t)t * g.ldy + o, ww * (v[c] * sc));
+        }
+        continue;
+      }
       if (c0 + 16 <= te.nvalid) {
         // a full chunk: stage [16 tokens][32 outputs] as bf16 in one of this
         // warp's ybufs 1 KB buffers and write it with one tensor store; with
@@ -618,7 +651,7 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN, PAIR>::kThreads, 1)
     int issued = 0;  // stages issued by this loop; the first n_pre hold early weight loads
     // each tile's entry is read one tile ahead, off the critical path
     TileEntry te_next = t_first < ntiles ? tile_at((t_first / ksplit) / MT) : TileEntry{};
-    for (int t = t_first; t < ntiles && !*abort; t += t_step) {
+    for (int t = t_first; t < ntiles && !tc::aborted(abort); t += t_step) {
       const int tt = t / ksplit, split = t % ksplit;
       const int kb0 = split * nkb / ksplit, kb1 = (split + 1) * nkb / ksplit;
       const TileEntry te = te_next;
@@ -626,7 +659,7 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN, PAIR>::kThreads, 1)
       const int mt = PAIR ? (tt % MT) * 2 + (int)rank : tt % MT;   // this CTA's 128-row weight block
       const uint8_t* sfa = F::kBs ? g.w_sf + (size_t)te.e * g.R * ncols_w + (size_t)mt * (ncols_w / 4) * 512 : nullptr;
       for (int kb = kb0; kb < kb1; ++kb) {
-        if (!tc::mbar_wait(&empty[stage], phase ^ 1u, abort)) {
+        if (!tc::mbar_wait(&empty[stage], phase ^ 1u, abort, g.wait_cycles)) {
           if (lane == 0) raise_status(g.status, MOE_ERR_TIMEOUT);
           *abort = 1;
           break;
@@ -687,7 +720,7 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN, PAIR>::kThreads, 1)
     for (int i = issued; i < n_pre; ++i) {
       if (tc::elect_one()) tc::mbar_arrive(&full[i]);
       __syncwarp();
-      if (!tc::mbar_wait(&full[i], 0, abort) && !*abort) {
+      if (!tc::mbar_wait(&full[i], 0, abort, g.wait_cycles) && !tc::aborted(abort)) {
         if (lane == 0) raise_status(g.status, MOE_ERR_TIMEOUT);
         *abort = 1;
       }
@@ -701,12 +734,12 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN, PAIR>::kThreads, 1)
     // a pair's MMAs are issued by its leader (rank 0) alone
     // each tile's entry is read one tile ahead, off the critical path
     TileEntry te_next = t_first < ntiles ? tile_at((t_first / ksplit) / MT) : TileEntry{};
-    for (int t = t_first; (!PAIR || rank == 0) && t < ntiles && !*abort; t += t_step) {
+    for (int t = t_first; (!PAIR || rank == 0) && t < ntiles && !tc::aborted(abort); t += t_step) {
       const int tt = t / ksplit, split = t % ksplit;
       const int kb0 = split * nkb / ksplit, kb1 = (split + 1) * nkb / ksplit;
       const TileEntry te = te_next;
       if (t + t_step < ntiles) te_next = tile_at(((t + t_step) / ksplit) / MT);
-      if (!tc::mbar_wait(&tempty[acc], acc_phase ^ 1u, abort)) {
+      if (!tc::mbar_wait(&tempty[acc], acc_phase ^ 1u, abort, g.wait_cycles)) {
         if (lane == 0) raise_status(g.status, MOE_ERR_TIMEOUT);
         *abort = 1;
         break;
@@ -721,7 +754,7 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN, PAIR>::kThreads, 1)
                idesc_bf = tc::idesc_bf16(n_mma);
       bool ok = true;
       for (int kb = kb0; kb < kb1; ++kb) {
-        if (!tc::mbar_wait(&full[stage], phase, abort)) {
+        if (!tc::mbar_wait(&full[stage], phase, abort, g.wait_cycles)) {
           if (lane == 0) raise_status(g.status, MOE_ERR_TIMEOUT);
           *abort = 1;
           ok = false;
@@ -812,7 +845,11 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN, PAIR>::kThreads, 1)
     // each tile's entry is read one tile ahead, off the critical path
     TileEntry te_next = t_first < ntiles ? tile_at((t_first / ksplit) / MT) : TileEntry{};
     for (int t = t_first; t < ntiles; t += t_step) {
-      if (!tc::mbar_wait(&tfull[acc], acc_phase, abort)) {
+      bool ok = tc::mbar_wait(&tfull[acc], acc_phase, abort, g.wait_cycles);
+      // the two warps of a pair meet at named barriers in the SwiGLU
+      // epilogue, so they go on, or give up, together
+      if constexpr (EPI == kEpiUpQuant || EPI == kEpiUpF32) ok = tc::pair_all(ok, 1 + (ew >> 1));
+      if (!ok) {
         if (lane == 0) raise_status(g.status, MOE_ERR_TIMEOUT);
         *abort = 1;
         break;
@@ -881,25 +918,57 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN, PAIR>::kThreads, 1)
 // gate|up + SwiGLU + h quantisation and the down projection in one
 // persistent kernel (64-token tiles, NVFP4 / MXFP4 with an h scale that needs
 // no global reduction).  Work item i is gate|up tile i for i < n1 = tiles *
-// MT1, else down tile i - n1; CTA b runs items b, b + grid, ..., so its
-// gate|up items all come before its down items and no CTA waits for a down
-// item.  (Evening out the per-CTA stage counts by handing the down items to
-// the CTAs with fewer gate|up items measured slower: the down tiles of the
-// token tiles that end last then pile up on fewer CTAs.)  Each epilogue warp counts its gate|up slice of token tile
-// tt in tile_done[tt] after storing it; the producer issues a down item's
-// token operand (h) once all MT1 * warps slices of its tile are counted.  The
-// producer keeps two cursors over the ring: weight tiles go out as soon as a
-// stage is free (before the dependency, and before the wait on the previous
-// kernel for the ring's first pass), token tiles as their data is ready.
+// MT1, else down tile i - n1.  The CTAs take items from a counter in global
+// memory, in increasing order, so every gate|up item is taken -- by a CTA
+// that is running -- before any down item, and a CTA runs its items in the
+// order it took them: a down item's wait for the gate|up items of its token
+// tile always ends, whether or not all CTAs are resident at once (a kernel on
+// another stream, MPS), and the work evens out across CTAs by itself.  Each
+// epilogue warp counts its gate|up slice of token tile tt in tile_done[tt]
+// after storing it; the producer issues a down item's token operand (h) once
+// all MT1 * warps slices of its tile are counted.  The producer keeps two
+// cursors: weight tiles go out as soon as a ring stage is free (the first
+// item's first stages before the wait on the previous kernel), token tiles as
+// their data is ready; the items it takes reach the MMA and epilogue warps
+// through a queue in shared memory.
 template <int FMT, int BN>
 struct FusedCfg {
   using C = Cfg<FMT, kEpiUpQuant, BN, false>;
-  // + the down store staging and the expert counts (+ a flag)
-  static constexpr int kSmem = C::kSmem + C::kEpiWarps * 1024 + (kFusedMaxE + 1) * 4;
+  // queue entries: the items between the epilogue and the weight cursor
+  // (at most two rings of stages and the accumulators) fit with room to spare
+  static constexpr int kQ = 32;
+  static_assert(kQ >= 2 * C::kStages + C::kAccStages + 2, "item queue");
+  // + the down store staging, the item queue, the expert counts (+ a flag),
+  // 32 ints per warp for gathering a tile's slots
+  static constexpr int kSmem =
+      C::kSmem + C::kEpiWarps * 1024 + kQ * (8 + 8 + 4) + (kFusedMaxE + 1) * 4 + (2 + C::kEpiWarps) * 32 * 4;
   static_assert(kSmem <= 227 * 1024, "shared memory");
 };
 
-template <int FMT, int BN>
+// Lane r (< n <= 32) receives the flat index of the (first + r)-th slot
+// routed to expert e (slots in increasing order), -1 in the other lanes; a
+// whole warp calls it, `stash` is 32 ints of the warp's own shared memory.
+__device__ __forceinline__ int tile_slot_of_lane(const int32_t* __restrict__ slot_expert, int64_t S, int e,
+                                                 int first, int n, int* stash) {
+  const int lane = threadIdx.x & 31;
+  int seen = 0;
+  for (int64_t base = 0; base < S && seen < first + n; base += 32) {
+    const int64_t i = base + lane;
+    const bool hit = i < S && __ldcg(slot_expert + i) == e;
+    const unsigned m = __ballot_sync(0xffffffffu, hit);
+    if (hit) {
+      const int r = seen + __popc(m & ((1u << lane) - 1u)) - first;
+      if (r >= 0 && r < n) stash[r] = (int)i;
+    }
+    seen += __popc(m);
+  }
+  __syncwarp();
+  const int sl = lane < n ? stash[lane] : -1;
+  __syncwarp();
+  return sl;
+}
+
+template <int FMT, int BN, bool GATHER>
 __global__ void __launch_bounds__(Cfg<FMT, kEpiUpQuant, BN, false>::kThreads, 1)
     fused_ffn_kernel(const __grid_constant__ CUtensorMap tmap_w13, const __grid_constant__ TokenMaps tmaps_x,
                      const __grid_constant__ CUtensorMap tmap_w2, const __grid_constant__ TokenMaps tmaps_h,
@@ -907,6 +976,8 @@ __global__ void __launch_bounds__(Cfg<FMT, kEpiUpQuant, BN, false>::kThreads, 1)
                      const FusedArgs f) {
   using C = Cfg<FMT, kEpiUpQuant, BN, false>;
   using F = FmtTraits<FMT>;
+  using FC = FusedCfg<FMT, BN>;
+  constexpr int kQ = FC::kQ;
   static_assert(F::kBs > 0, "block-scaled formats only");
   static_assert(C::kSfbBlocks == 1, "one scale block per token tile");
   extern __shared__ uint8_t smem_raw[];
@@ -924,7 +995,18 @@ __global__ void __launch_bounds__(Cfg<FMT, kEpiUpQuant, BN, false>::kThreads, 1)
   // SwiGLU tiles (a warp may start its first down tile while its pair
   // partner still finishes the last gate|up tile)
   uint16_t* y_stage = reinterpret_cast<uint16_t*>(r_tab + 128);
-  int32_t* hist = reinterpret_cast<int32_t*>(y_stage + C::kEpiWarps * 512);  // [kFusedMaxE] counts, bad flag
+  // item queue: entry j holds an item id (-1: no more items); q_full[j]
+  // completes when the producer has written it, q_free[j] when the MMA warp
+  // and every epilogue warp have read it
+  uint64_t* q_full = reinterpret_cast<uint64_t*>(y_stage + C::kEpiWarps * 512);
+  uint64_t* q_free = q_full + kQ;
+  volatile int32_t* q_id = reinterpret_cast<volatile int32_t*>(q_free + kQ);
+  int32_t* hist = const_cast<int32_t*>(q_id) + kQ;  // [kFusedMaxE] counts, bad flag
+  int* stash = hist + kFusedMaxE + 1 + (threadIdx.x >> 5) * 32;   // this warp's 32 ints
+  // gather mode on the forward: the slots' experts come from the previous
+  // kernel (the router), so everything waits for it
+  const bool ids_from_prev = GATHER && f.slot_expert != nullptr;
+  if (ids_from_prev) pdl_wait();
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -935,6 +1017,10 @@ __global__ void __launch_bounds__(Cfg<FMT, kEpiUpQuant, BN, false>::kThreads, 1)
     for (int a = 0; a < C::kAccStages; ++a) {
       tc::mbar_init(&tfull[a], 1);
       tc::mbar_init(&tempty[a], C::kEpiWarps);
+    }
+    for (int j = 0; j < kQ; ++j) {
+      tc::mbar_init(&q_full[j], 1);
+      tc::mbar_init(&q_free[j], 1 + C::kEpiWarps);
     }
     *abort = 0;
     tc::fence_mbar_init();
@@ -997,32 +1083,61 @@ __global__ void __launch_bounds__(Cfg<FMT, kEpiUpQuant, BN, false>::kThreads, 1)
   const int ncols1 = g1.K / F::kBs, ncols2 = g2.K / F::kBs;
   const int n1 = ntok * MT1, total = n1 + ntok * MT2;
   const int done_target = MT1 * C::kEpiWarps;
-  // item k of this CTA: up (gate|up or down), token tile, weight-row block
-  auto item = [&](int k, bool& up, int& tt, int& mt) -> bool {
-    const int i = (int)blockIdx.x + k * (int)gridDim.x;
-    if (i >= total) return false;
+  const long long wait_lim = g1.wait_cycles;
+  // item i: up (gate|up or down), token tile, weight-row block
+  auto decode = [&](int i, bool& up, int& tt, int& mt) {
     up = i < n1;
     const int r = up ? i : i - n1, m = up ? MT1 : MT2;
     tt = r / m;
     mt = r % m;
-    return true;
   };
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    // A cursor (weights) and B cursor (tokens): item ordinal, stage within
-    // the item, and the stage sequence number (ring slot = seq % kStages).
-    bool a_up = false, b_up = false;
-    int a_tt = 0, a_mt = 0, b_tt = 0, b_mt = 0;
-    bool a_valid = item(0, a_up, a_tt, a_mt), b_valid = a_valid;
-    b_up = a_up;
-    b_tt = a_tt;
-    b_mt = a_mt;
-    int a_e = a_valid ? plan.at(a_tt, BN).e : -1;
-    TileEntry b_te = a_valid ? plan.at(b_tt, BN) : TileEntry{};
-    int ka = 0, kba = 0, seq_a = 0, kb_b = 0, kbb = 0, seq_b = 0;
-    bool b_ready = b_up;   // gate|up token tiles come from the x quantiser before this kernel
-    uint32_t rdy = 0;  // bit i: the token operand of B item kb_b + i is ready
+    // Items are taken one ahead: lane 0 holds the counter's answer for the
+    // next item while the current one's weights go out.
+    int pending = 0;
+    if (lane == 0) pending = atomicAdd(f.work, 1);
+    int pushed = 0;          // queue entries written (items, then the end mark)
+    bool ended = false;      // the end mark is in the queue
+    // weight cursor: item, stage within it, stage sequence number (ring slot
+    // = seq % kStages)
+    bool a_valid = false, a_up = false;
+    int a_tt = 0, a_mt = 0, a_e = 0, kba = 0, seq_a = 0;
+    // token cursor: queue position, stage within the item, sequence number
+    int b_pos = 0, kbb = 0, seq_b = 0;
+    bool b_have = false, b_up = false, b_ready = false;
+    int b_tt = 0, b_mt = 0;
+    TileEntry b_te{};
+    int b_tok = -1;    // gather mode: lane r (< nvalid) holds the token of tile row r
+    uint32_t rdy = 0;  // bit i: the token operand of the item at queue position b_pos + i is ready
+    // Moves the weight cursor to a newly taken item and queues it; false
+    // when the queue has no room right now.
+    auto take_next = [&]() -> bool {
+      if (pushed - b_pos >= kQ) return false;   // the token cursor still reads that entry
+      const int j = pushed % kQ;
+      const uint32_t par = ((uint32_t)(pushed / kQ) & 1u) ^ 1u;
+      if (__shfl_sync(0xffffffffu, (int)tc::mbar_test_wait(&q_free[j], par), 0) == 0) return false;
+      int id = __shfl_sync(0xffffffffu, pending, 0);
+      id = id < total ? id : -1;
+      if (lane == 0) {
+        if (id >= 0) pending = atomicAdd(f.work, 1);
+        q_id[j] = id;
+        tc::mbar_arrive(&q_full[j]);
+      }
+      __syncwarp();
+      ++pushed;
+      if (id < 0) {
+        ended = true;
+        a_valid = false;
+        return true;
+      }
+      decode(id, a_up, a_tt, a_mt);
+      a_e = plan.at(a_tt, BN).e;
+      kba = 0;
+      a_valid = true;
+      return true;
+    };
     auto issue_a = [&]() {
       const int st = seq_a % C::kStages;
       if (tc::elect_one()) {
@@ -1035,41 +1150,80 @@ __global__ void __launch_bounds__(Cfg<FMT, kEpiUpQuant, BN, false>::kThreads, 1)
       }
       __syncwarp();
       ++seq_a;
-      if (++kba == (a_up ? nkb1 : nkb2)) {
-        kba = 0;
-        a_valid = item(++ka, a_up, a_tt, a_mt);
-        if (a_valid) a_e = plan.at(a_tt, BN).e;
-      }
+      if (++kba == (a_up ? nkb1 : nkb2)) a_valid = false;
     };
     // Before the wait on the previous kernel (the x quantiser), at most
-    // kPreStages weight stages per CTA are put in flight (the ring's first
-    // pass needs no free slot): a deeper burst queues that kernel's own reads
-    // behind it.
+    // kPreStages weight stages of the first item are put in flight (the
+    // ring's first pass needs no free slot): a deeper burst queues that
+    // kernel's own reads behind it.
     constexpr int kPreStages = 3 < C::kStages ? 3 : C::kStages;
-    if (g1.w_early != 0) {
+    take_next();
+    if (g1.w_early != 0)
       while (a_valid && seq_a < kPreStages) issue_a();
-    }
     pdl_wait();
     pdl_trigger();
     long long t_prog = clock64();
-    while (a_valid || b_valid) {
+    while (true) {
       bool prog = false;
       // token tiles: every stage whose weights are out and whose data is
       // ready (a dependency poll at most once per pass)
-      while (b_valid && seq_b < seq_a) {
+      while (seq_b < seq_a) {
+        if (!b_have) {
+          const int id = q_id[b_pos % kQ];   // written by this warp, always an item here
+          decode(id, b_up, b_tt, b_mt);
+          b_te = plan.at(b_tt, BN);
+          b_have = true;
+          b_ready = b_up || (rdy & 1u) != 0;   // gate|up token tiles come from the x quantiser before this kernel
+          if (GATHER && b_up) {
+            // the tile's rows are its expert's slots in flat order (one tile
+            // per expert: at most kGatherMaxT slots; more means slots that
+            // repeat a token, which the rows past 32 do not get)
+            const int n = min(b_te.nvalid, kGatherMaxT);
+            if (b_te.nvalid > kGatherMaxT && lane == 0) raise_status(g1.status, MOE_ERR_DEVICE_FAULT);
+            if (f.perm_token) {
+              b_tok = lane < n ? __ldg(f.perm_token + b_te.p0 + lane) : -1;
+            } else {
+              const int sl = tile_slot_of_lane(f.slot_expert, f.S, b_te.e, 0, n, stash);
+              b_tok = sl >= 0 ? sl / f.k : -1;
+            }
+            if (b_tok >= f.T) b_tok = -1;
+          }
+        }
         if (!b_ready) {
-          // one round trip polls this item's and the next 31 items' token tiles
-          bool up_i = true;
-          int tt_i = 0, mt_i = 0;
-          const bool has = item(kb_b + lane, up_i, tt_i, mt_i);
-          const int v = (has && !up_i) ? tc::ld_acquire_gpu(f.tile_done + tt_i) : done_target;
+          // one round trip polls the token tiles of this and the next 31 queued items
+          int v = 0;
+          if (b_pos + lane < pushed) {
+            const int id = q_id[(b_pos + lane) % kQ];
+            bool up_i = true;
+            int tt_i = 0, mt_i = 0;
+            if (id >= 0) decode(id, up_i, tt_i, mt_i);
+            v = (id >= 0 && !up_i) ? tc::ld_acquire_gpu(f.tile_done + tt_i) : done_target;
+          }
           rdy |= __ballot_sync(0xffffffffu, v >= done_target);
           if (!(rdy & 1u)) break;
           tc::fence_proxy_async_global();   // for every token tile seen ready here
           b_ready = true;
         }
         const int st = seq_b % C::kStages;
-        if (tc::elect_one()) {
+        if (GATHER && b_up) {
+          // x rows by bulk copies from the gather layout: lane r copies tile
+          // row r's 128 code bytes (the variant swizzled for r % 8) and its
+          // scale lines, one per 4-scale group of the stage
+          uint8_t* sp = smem + st * C::kStage;
+          const int n = min(b_te.nvalid, kGatherMaxT);
+          if (tc::elect_one()) tc::mbar_expect_tx(&full[st], (uint32_t)n * (128u + F::kGroups * 16u));
+          __syncwarp();
+          const int t = b_tok >= 0 ? b_tok : 0;   // a bad slot still completes its bytes
+          if (lane < n) {
+            const uint8_t* src = f.xg + ((int64_t)t * 8 + (lane & 7)) * (g1.K / 2) + (int64_t)kbb * 128;
+            tc::bulk_load(sp + C::kA + lane * 128, src, 128u, &full[st]);
+            const uint8_t* lines = f.xsl + ((int64_t)t * (ncols1 / 4) + (int64_t)kbb * F::kGroups) * 16;
+#pragma unroll
+            for (int gi = 0; gi < F::kGroups; ++gi)
+              tc::bulk_load(sp + C::kA + C::kB + C::kSFA + gi * 512 + lane * 16, lines + gi * 16, 16u, &full[st]);
+          }
+          __syncwarp();
+        } else if (tc::elect_one()) {
           uint8_t* sp = smem + st * C::kStage;
           const int bi = token_box_index(min(b_te.nvalid, BN));
           const uint32_t brows = min(16u << bi, (uint32_t)BN);
@@ -1084,29 +1238,33 @@ __global__ void __launch_bounds__(Cfg<FMT, kEpiUpQuant, BN, false>::kThreads, 1)
         ++seq_b;
         if (++kbb == (b_up ? nkb1 : nkb2)) {
           kbb = 0;
-          b_valid = item(++kb_b, b_up, b_tt, b_mt);
-          if (b_valid) b_te = plan.at(b_tt, BN);
+          ++b_pos;
+          b_have = false;
           rdy >>= 1;
-          b_ready = b_up || (rdy & 1u) != 0;
         }
         prog = true;
       }
       // weight tiles: every free ring slot, at most a ring ahead of the tokens
-      while (a_valid && seq_a < seq_b + C::kStages) {
+      while (seq_a < seq_b + C::kStages) {
+        if (!a_valid) {
+          if (ended || !take_next()) break;
+          prog = true;
+          if (!a_valid) break;   // the end mark
+        }
         const int st = seq_a % C::kStages;
         const uint32_t par = (((uint32_t)(seq_a / C::kStages)) & 1u) ^ 1u;
         if (__shfl_sync(0xffffffffu, (int)tc::mbar_test_wait(&empty[st], par), 0) == 0) break;
         issue_a();
         prog = true;
       }
+      if (ended && !a_valid && seq_b == seq_a) break;   // every item's stages are out
       if (prog) {
         t_prog = clock64();
-      } else if (*abort || clock64() - t_prog > tc::kWaitCycles) {
-        // neither cursor could move for the wait bound (all polls above are non-blocking)
-        if (!*abort) {
-          if (lane == 0) raise_status(g1.status, MOE_ERR_TIMEOUT);
-          *abort = 1;
-        }
+      } else if (__any_sync(0xffffffffu, *abort != 0 || clock64() - t_prog > wait_lim)) {
+        // neither cursor could move for the wait bound (all polls above are
+        // non-blocking), or another warp gave up: the warp leaves as one
+        if (lane == 0 && !*abort) raise_status(g1.status, MOE_ERR_TIMEOUT);
+        *abort = 1;
         break;
       }
     }
@@ -1116,7 +1274,7 @@ __global__ void __launch_bounds__(Cfg<FMT, kEpiUpQuant, BN, false>::kThreads, 1)
       const int st = q % C::kStages;
       if (tc::elect_one()) tc::mbar_arrive(&full[st]);
       __syncwarp();
-      tc::mbar_wait(&full[st], ((uint32_t)(q / C::kStages)) & 1u, abort);
+      tc::mbar_wait(&full[st], ((uint32_t)(q / C::kStages)) & 1u, abort, wait_lim);
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
@@ -1126,11 +1284,22 @@ __global__ void __launch_bounds__(Cfg<FMT, kEpiUpQuant, BN, false>::kThreads, 1)
     uint32_t phase = 0;
     int acc = 0;
     uint32_t acc_phase = 0;
-    bool up = false;
-    int tt = 0, mt = 0;
-    for (int k = 0; item(k, up, tt, mt) && !*abort; ++k) {
+    for (int k = 0; !tc::aborted(abort); ++k) {
+      const int j = k % kQ;
+      if (!tc::mbar_wait(&q_full[j], (uint32_t)(k / kQ) & 1u, abort, wait_lim)) {
+        if (lane == 0) raise_status(g1.status, MOE_ERR_TIMEOUT);
+        *abort = 1;
+        break;
+      }
+      const int id = q_id[j];
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&q_free[j]);
+      if (id < 0) break;
+      bool up = false;
+      int tt = 0, mt = 0;
+      decode(id, up, tt, mt);
       const TileEntry te = plan.at(tt, BN);
-      if (!tc::mbar_wait(&tempty[acc], acc_phase ^ 1u, abort)) {
+      if (!tc::mbar_wait(&tempty[acc], acc_phase ^ 1u, abort, wait_lim)) {
         if (lane == 0) raise_status(g1.status, MOE_ERR_TIMEOUT);
         *abort = 1;
         break;
@@ -1138,12 +1307,14 @@ __global__ void __launch_bounds__(Cfg<FMT, kEpiUpQuant, BN, false>::kThreads, 1)
       tc::fence_after_sync();
       const uint32_t n_mma = (uint32_t)min(BN, (te.nvalid + 15) & ~15);
       const uint32_t d = tmem + acc * BN;
-      const uint32_t sfb0 = tmem + C::kSfbCol + sfb_col_offset<BN>(te.row0);
+      // gathered rows start at tile row 0 of the stage; loaded ones at the
+      // tile's padded row
+      const uint32_t sfb0 = tmem + C::kSfbCol + ((GATHER && up) ? 0u : sfb_col_offset<BN>(te.row0));
       const uint32_t idesc_nv = tc::idesc_mxf4(n_mma, false, 0, 0);
       const int nkb = up ? nkb1 : nkb2;
       bool ok = true;
       for (int kb = 0; kb < nkb; ++kb) {
-        if (!tc::mbar_wait(&full[stage], phase, abort)) {
+        if (!tc::mbar_wait(&full[stage], phase, abort, wait_lim)) {
           if (lane == 0) raise_status(g1.status, MOE_ERR_TIMEOUT);
           *abort = 1;
           ok = false;
@@ -1167,8 +1338,8 @@ __global__ void __launch_bounds__(Cfg<FMT, kEpiUpQuant, BN, false>::kThreads, 1)
             if (FMT == MOE_FMT_NVFP4) {
               tc::mma_nvf4(d, da, db, idesc_nv, tmem + C::kSfaCol + 4 * kk, sfb0 + kk * 4, accum);
             } else {
-              const uint32_t id = (uint32_t)(kk & 1) * 2;
-              tc::mma_mxf4(d, da, db, tc::idesc_mxf4(n_mma, true, id, id), tmem + C::kSfaCol + 4 * (kk >> 1),
+              const uint32_t id2 = (uint32_t)(kk & 1) * 2;
+              tc::mma_mxf4(d, da, db, tc::idesc_mxf4(n_mma, true, id2, id2), tmem + C::kSfaCol + 4 * (kk >> 1),
                            sfb0 + (kk >> 1) * 4, accum);
             }
           }
@@ -1206,11 +1377,25 @@ __global__ void __launch_bounds__(Cfg<FMT, kEpiUpQuant, BN, false>::kThreads, 1)
     int ypar = 0;   // down projection: the store-staging buffer in turn
     int acc = 0;
     uint32_t acc_phase = 0;
-    bool up = false;
-    int tt = 0, mt = 0;
-    for (int k = 0; item(k, up, tt, mt); ++k) {
+    const int pbar = 1 + (ew >> 1);   // this warp pair's named barrier
+    for (int k = 0;; ++k) {
+      const int j = k % kQ;
+      // the two warps of a pair meet at named barriers in the SwiGLU
+      // epilogue, so they go on, or give up, together
+      if (!tc::pair_all(tc::mbar_wait(&q_full[j], (uint32_t)(k / kQ) & 1u, abort, wait_lim), pbar)) {
+        if (lane == 0) raise_status(g1.status, MOE_ERR_TIMEOUT);
+        *abort = 1;
+        break;
+      }
+      const int id = q_id[j];
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&q_free[j]);
+      if (id < 0) break;
+      bool up = false;
+      int tt = 0, mt = 0;
+      decode(id, up, tt, mt);
       const TileEntry te = plan.at(tt, BN);
-      if (!tc::mbar_wait(&tfull[acc], acc_phase, abort)) {
+      if (!tc::pair_all(tc::mbar_wait(&tfull[acc], acc_phase, abort, wait_lim), pbar)) {
         if (lane == 0) raise_status(g1.status, MOE_ERR_TIMEOUT);
         *abort = 1;
         break;
@@ -1238,6 +1423,15 @@ __global__ void __launch_bounds__(Cfg<FMT, kEpiUpQuant, BN, false>::kThreads, 1)
         acc = 0;
         acc_phase ^= 1u;
       }
+      // the forward's combine in the down epilogue: lane r gets tile row r's
+      // token and routing weight
+      int ltok = -1;
+      float lw = 0.0f;
+      if (GATHER && !up && g2.out32 && f.slot_expert) {
+        const int sl = tile_slot_of_lane(f.slot_expert, f.S, te.e, 0, min(te.nvalid, kGatherMaxT), stash);
+        ltok = sl >= 0 ? sl / f.k : -1;
+        lw = sl >= 0 ? __ldg(f.topk_w + sl) : 0.0f;
+      }
       if (up) {
         if (c_lo < ncol)
           epilogue_slice<FMT, kEpiUpQuant, BN>(g1, &tmap_y, te, mt, 0, nch, c_lo, ew, q, lane, gact1, gh, epi_tiles,
@@ -1249,13 +1443,14 @@ __global__ void __launch_bounds__(Cfg<FMT, kEpiUpQuant, BN, false>::kThreads, 1)
         if (lane == 0) atomicAdd(f.tile_done + tt, 1);
       } else if (c_lo < ncol) {
         epilogue_slice<FMT, kEpiDown, BN>(g2, &tmap_y, te, mt, 0, nch, c_lo, ew, q, lane, gact2, 1.0f, epi_tiles,
-                                          r_tab, y_stage, 1, ypar, hmax, r0, r1, r2, r3);
+                                          r_tab, y_stage, 1, ypar, hmax, r0, r1, r2, r3, ltok, lw);
       }
     }
     if (lane == 0) tc::bulk_wait_all();   // tensor stores done before the CTA exits
   }
 
   __syncwarp();
+  __threadfence();   // this CTA's output reductions before the count below
   __syncthreads();
   if (*abort) {
     // let copies and MMAs already in flight land before the memory goes away
@@ -1265,6 +1460,28 @@ __global__ void __launch_bounds__(Cfg<FMT, kEpiUpQuant, BN, false>::kThreads, 1)
   }
   tc::fence_after_sync();
   if (warp == 1) tc::tmem_dealloc(tmem, C::kTmemCols);
+  if constexpr (GATHER) {
+    if (f.out) {
+      // the CTA that finishes last rounds the fp32 output rows to bf16
+      __shared__ int last;
+      if (threadIdx.x == 0) last = atomicAdd(f.done, 1) == (int)gridDim.x - 1;
+      __syncthreads();
+      if (last) {
+        __threadfence();
+        const int64_t n8 = f.T * (g2.R / 8);
+        for (int64_t i = threadIdx.x; i < n8; i += blockDim.x) {
+          const float4 a = __ldcg(reinterpret_cast<const float4*>(g2.out32) + 2 * i);
+          const float4 b = __ldcg(reinterpret_cast<const float4*>(g2.out32) + 2 * i + 1);
+          uint4 o;
+          o.x = (uint32_t)f32_to_bf16_rn(a.x) | ((uint32_t)f32_to_bf16_rn(a.y) << 16);
+          o.y = (uint32_t)f32_to_bf16_rn(a.z) | ((uint32_t)f32_to_bf16_rn(a.w) << 16);
+          o.z = (uint32_t)f32_to_bf16_rn(b.x) | ((uint32_t)f32_to_bf16_rn(b.y) << 16);
+          o.w = (uint32_t)f32_to_bf16_rn(b.z) | ((uint32_t)f32_to_bf16_rn(b.w) << 16);
+          reinterpret_cast<uint4*>(f.out)[i] = o;
+        }
+      }
+    }
+  }
 }
 
 // ------------------------------------------------------------- tensor maps --
@@ -1423,7 +1640,7 @@ cudaError_t launch_epi(const GemmArgs& g, int epi, int bn, const void* a, int64_
   return launch_bn<FMT, kEpiUpQuant>(g, bn, a, ar, b, br, sms, s);
 }
 
-template <int FMT, int BN>
+template <int FMT, int BN, bool GATHER>
 cudaError_t launch_fused_cfg(const GemmArgs& g1, const GemmArgs& g2, const FusedArgs& f, const void* w13,
                              int64_t w13_rows, const void* w2, int64_t w2_rows, const void* xq, const void* hq,
                              int num_sms, cudaStream_t s) {
@@ -1438,7 +1655,7 @@ cudaError_t launch_fused_cfg(const GemmArgs& g1, const GemmArgs& g2, const Fused
     if (!make_map(&mx.m[i], xq, f.P, g1.K / 2, rows)) return cudaErrorInvalidValue;
     if (!make_map(&mh.m[i], hq, f.P, g2.K / 2, rows)) return cudaErrorInvalidValue;
   }
-  auto kern = fused_ffn_kernel<FMT, BN>;
+  auto kern = fused_ffn_kernel<FMT, BN, GATHER>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, FusedCfg<FMT, BN>::kSmem);
   if (e != cudaSuccess) return e;
   e = launch_pdl(kern, dim3(num_sms), dim3(C::kThreads), FusedCfg<FMT, BN>::kSmem, s, m13, mx, m2, mh, my, g1, g2, f);
@@ -1464,16 +1681,27 @@ cudaError_t launch_fused_ffn(const GemmArgs& g1, const GemmArgs& g2, const Fused
                              int64_t w13_rows, const void* w2, int64_t w2_rows, const void* xq, const void* hq,
                              int num_sms, cudaStream_t s) {
   if (g1.E > kFusedMaxE || g1.fmt != g2.fmt) return cudaErrorInvalidValue;
+  // gather mode: a tile holds at most kGatherMaxT rows (T <= kGatherMaxT),
+  // and its tokens come from perm_token or from the slots' experts
+  if (f.xg && (f.T > kGatherMaxT || !f.xsl || (!f.perm_token && !f.slot_expert) || f.k < 1))
+    return cudaErrorInvalidValue;
+  if (f.out && (!f.xg || !f.slot_expert || !g2.out32 || !f.done || !f.topk_w)) return cudaErrorInvalidValue;
   switch (g1.fmt) {
     case MOE_FMT_NVFP4:
-      return launch_fused_cfg<MOE_FMT_NVFP4, 64>(g1, g2, f, w13, w13_rows, w2, w2_rows, xq, hq, num_sms, s);
+      return f.xg ? launch_fused_cfg<MOE_FMT_NVFP4, 64, true>(g1, g2, f, w13, w13_rows, w2, w2_rows, xq, hq, num_sms, s)
+                  : launch_fused_cfg<MOE_FMT_NVFP4, 64, false>(g1, g2, f, w13, w13_rows, w2, w2_rows, xq, hq, num_sms,
+                                                               s);
     case MOE_FMT_MXFP4:
-      return launch_fused_cfg<MOE_FMT_MXFP4, 64>(g1, g2, f, w13, w13_rows, w2, w2_rows, xq, hq, num_sms, s);
+      return f.xg ? launch_fused_cfg<MOE_FMT_MXFP4, 64, true>(g1, g2, f, w13, w13_rows, w2, w2_rows, xq, hq, num_sms, s)
+                  : launch_fused_cfg<MOE_FMT_MXFP4, 64, false>(g1, g2, f, w13, w13_rows, w2, w2_rows, xq, hq, num_sms,
+                                                               s);
     default: return cudaErrorInvalidValue;
   }
 }
 
 bool tensor_maps_available() { return encode_fn() != nullptr; }
+
+long long tc_default_wait_cycles() { return tc::kDefaultWaitCycles; }
 
 void set_gemm_pairs(int mode) { g_gemm_pairs = mode; }
 
@@ -1506,6 +1734,7 @@ cudaError_t launch_router_gemm(const uint16_t* x, int64_t T, int H, const uint16
   g.split_stride = part_stride;
   g.ldy = E;
   g.status = status;
+  g.wait_cycles = wait_cycles();
   const int64_t items = (T + kRouterBN - 1) / kRouterBN * (E / 128) * ksplit;
   const int grid = (int)(items < num_sms ? items : num_sms);
   return launch_cfg<kFmtBF16, kEpiLogits, kRouterBN, false>(g, wr, E, x, T, grid, s);
@@ -1768,11 +1997,46 @@ __global__ void __launch_bounds__(256) quant_tokens_kernel(QuantPaddedArgs a) {
     }
     const int32_t o = __ldg(a.offsets + e), o1 = __ldg(a.offsets + e + 1);
     const int64_t row = (int64_t)__ldg(a.poff + e) + (p - o);
-    return (row >= 0 && row < a.P && p >= o && p < o1) ? row : -2;
+    const bool ok = row >= 0 && row < a.P && p >= o && p < o1;
+    if (ok && a.w_perm) a.w_perm[p] = __ldg(a.topk_w + t * a.k + j);   // the slot's routing weight
+    return ok ? row : -2;
   };
   for (int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < a.T; t += warps)
     quant_token_slots<FMT>(a.x + t * a.K, a.K, a.k, scale, r_tab, tbuf[threadIdx.x >> 5],
                            [&](int j) { return resolve(t, j); }, a.codes, a.sf, a.status);
+}
+
+// x of a small batch into the gather layout (quant_token_gather): a warp per
+// token, whatever the routing.
+template <int FMT>
+__global__ void __launch_bounds__(256) quant_gather_kernel(const uint16_t* __restrict__ x, int64_t T, int K,
+                                                           GatherQuant q) {
+  pdl_wait();  // inputs come from the previous kernels
+  pdl_trigger();
+  constexpr int bs = FMT == MOE_FMT_MXFP4 ? 32 : 16;
+  __shared__ float r_tab[128];
+  const float scale = act_scale_of(FMT, q.scale, q.amax);
+  if (FMT == MOE_FMT_NVFP4 && threadIdx.x < 128) r_tab[threadIdx.x] = nvfp4_multiplier(threadIdx.x, scale);
+  __syncthreads();
+  const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t < T)
+    quant_token_gather<FMT>(x + t * K, K, scale, r_tab, q.xg + t * 8 * (K / 2), q.xsl + t * (K / (4 * bs)) * 16);
+}
+
+cudaError_t launch_quant_gather(int fmt, const uint16_t* x, int64_t T, int K, const GatherQuant& q, cudaStream_t s) {
+  if (T == 0) return cudaSuccess;
+  if (T > kGatherMaxT || K % 256 != 0) return cudaErrorInvalidValue;
+  const dim3 grid((unsigned)((T + 7) / 8));
+  cudaError_t e;
+  if (fmt == MOE_FMT_NVFP4)
+    e = launch_pdl(quant_gather_kernel<MOE_FMT_NVFP4>, grid, dim3(256), 0, s, x, T, K, q);
+  else if (fmt == MOE_FMT_MXFP4)
+    e = launch_pdl(quant_gather_kernel<MOE_FMT_MXFP4>, grid, dim3(256), 0, s, x, T, K, q);
+  else
+    return cudaErrorInvalidValue;
+  if (e != cudaSuccess) return e;
+  count_launches(1);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_quant_padded(const QuantPaddedArgs& a, bool src_x, int fmt, int num_sms, cudaStream_t s) {

@@ -38,6 +38,13 @@ struct GemmArgs {
   uint16_t* y;                 // down: y_perm [y_rows][ldy] bf16
   int ldy;
   int64_t y_rows;
+  // down, with the combine in the epilogue (out32 != NULL): out32[t][o] +=
+  // w_perm[p] * y[p][o] for slot p of token t = perm_token[p] (w_perm NULL:
+  // weight 1), fp32 reductions; t outside [0, out_rows) is a device fault
+  float* out32;
+  const int32_t* perm_token;
+  const float* w_perm;
+  int64_t out_rows;
   float* logits;               // router: logits [T][ldy] fp32 (+ bias)
   const float* bias;
   int ksplit;                  // router: K split over this many partial outputs,
@@ -54,6 +61,7 @@ struct GemmArgs {
   const int32_t* offsets;      // [E+1] compact expert offsets (w_early == 2; E <= 256)
   int max_tiles;               // entries allocated in `tiles`
   int32_t* status;
+  long long wait_cycles;       // bound of every device wait (SM clocks)
 };
 
 struct QuantPaddedArgs {
@@ -66,6 +74,8 @@ struct QuantPaddedArgs {
   const int32_t* inv_perm;     // x source, optional: slot of each (token, j); then each
   int k;                       //   token is quantised once and written to its k slots
   const int32_t* slot_expert;  //   optional with it: expert of each (token, j) (top-k indices)
+  const float* topk_w;         //   optional with it: weight of each (token, j); then
+  float* w_perm;               //   w_perm[slot position] receives it
   PlanOut plan;                // per-slot x quantiser: also compute (and write) the tile plan
   int32_t* zero;               // optional: nzero counters set to 0 (by block 0, after the wait)
   int nzero;
@@ -79,31 +89,57 @@ struct QuantPaddedArgs {
 };
 
 // The expert FFN as one persistent kernel (gate|up + SwiGLU + h quantisation,
-// then down), for 64-token tiles: each CTA runs its gate|up tiles, then its
-// down tiles; a down tile's token operand waits for the gate|up slices of its
-// token tile, counted in tile_done.  The tile list comes from the offsets,
-// or, when slot_expert is given, from the slots' expert ids: the top-k ids
-// are then read before the wait on the previous kernel, so that kernel may
-// be the one that writes the offsets.
+// then down), for 64-token tiles: the CTAs take work items (every gate|up
+// tile, then every down tile) from the counter `work` in increasing order; a
+// down tile's token operand waits for the gate|up slices of its token tile,
+// counted in tile_done.  The tile list comes from the offsets, or, when
+// slot_expert is given, from the slots' expert ids: the top-k ids are then
+// read before the wait on the previous kernel, so that kernel may be the one
+// that writes the offsets.
 struct FusedArgs {
   const int32_t* offsets;      // [E+1] compact (E <= 256)
   const int32_t* slot_expert;  // optional: [S] expert of each slot (flat top-k ids), all in [0, E)
   int64_t S;                   // slots: offsets[E]
   int64_t P;                   // padded rows allocated for x and h
   int32_t* tile_done;          // [max_tiles], zero on entry
+  int32_t* work;               // item counter, zero on entry and set at least two launches before
+                               // this kernel (it is read before the wait on the previous one)
   int max_tiles;
+  // Gather mode (small batches, at most kGatherMaxT slots per expert): the
+  // gate|up token operand is copied row by row from the gather layout of x
+  // (quant_token_gather), so nothing waits for a permutation.  The rows of
+  // a tile are the slots of its expert in flat order; their tokens come from
+  // perm_token (the grouped FFN) or, with slot_expert, from the slots
+  // themselves (token = slot / k; the forward, which reads slot_expert only
+  // after the wait on the previous kernel, the router).
+  const uint8_t* xg;           // [T][8][K/2] codes, swizzled per row % 8
+  const uint8_t* xsl;          // [T][K/(4 bs)][16] scale lines
+  const int32_t* perm_token;   // [S] token of each slot position, or NULL
+  int k;                       // slots per token (slot_expert mode)
+  // the forward's combine in the down epilogue (slot_expert mode): out32
+  // rows get topk_w[slot] * y (g2.out32 is set too); the CTA that finishes
+  // last rounds them to bf16 into out
+  const float* topk_w;
+  uint16_t* out;
+  int32_t* done;               // CTAs finished, zero on entry
+  int64_t T;
 };
 constexpr int kFusedMaxE = 256;
 cudaError_t launch_fused_ffn(const GemmArgs& g1, const GemmArgs& g2, const FusedArgs& f, const void* w13,
                              int64_t w13_rows, const void* w2, int64_t w2_rows, const void* xq, const void* hq,
                              int num_sms, cudaStream_t s);
 
+// x of a small batch (T <= kGatherMaxT) into the gather layout the
+// one-kernel FFN copies its token rows from (NVFP4 or MXFP4, K % 256 == 0).
+cudaError_t launch_quant_gather(int fmt, const uint16_t* x, int64_t T, int K, const GatherQuant& q, cudaStream_t s);
 cudaError_t launch_plan(const int32_t* offsets, int E, int64_t S, int bn, int32_t* poff, TileEntry* tiles,
                         int32_t* num_tiles, int max_tiles, int32_t* status, cudaStream_t s);
 cudaError_t launch_quant_padded(const QuantPaddedArgs& a, bool src_x, int fmt, int num_sms, cudaStream_t s);
 cudaError_t launch_grouped_gemm(const GemmArgs& g, int epi, int bn, const void* a_base, int64_t a_rows,
                                 const void* b_base, int64_t b_rows, int num_sms, cudaStream_t s);
 bool tensor_maps_available();
+// The default bound of every device wait (about a second of SM clocks).
+long long tc_default_wait_cycles();
 // Early weight loads (MOE_OPT_EARLY_WEIGHTS): 0 off, 1 the ring's first pass,
 // 2 also prefetch the next stages' weights to L2.
 void set_early_weights(int mode);

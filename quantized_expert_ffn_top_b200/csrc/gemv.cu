@@ -247,12 +247,12 @@ __global__ void __launch_bounds__((1 + kGemvConsumers) * 32, 1)
     // ---------------------------------------------------------- producer
     int stage = 0;
     uint32_t phase = 0;
-    for (int it = i0; it < i1 && !*abort; ++it) {
+    for (int it = i0; it < i1 && !tc::aborted(abort); ++it) {
       const TileEntry te = a.tiles[it / MT];
       const int rb = it % MT;
       const uint8_t* sf_blk = SF ? SF + (size_t)te.e * R * ncols + (size_t)(rb >> 1) * (ncols / 4) * 512 : nullptr;
       for (int kc = 0; kc < nkc; ++kc) {
-        if (!tc::mbar_wait(&empty[stage], phase ^ 1u, abort)) {
+        if (!tc::mbar_wait(&empty[stage], phase ^ 1u, abort, a.wait_cycles)) {
           if (lane == 0) raise_status(a.status, MOE_ERR_TIMEOUT);
           *abort = 1;
           break;
@@ -292,7 +292,7 @@ __global__ void __launch_bounds__((1 + kGemvConsumers) * 32, 1)
     // Bounded barrier of the consumer warps (the producer keeps streaming).
     auto consumer_sync = [&]() -> bool {
       tc::mbar_arrive(bbar);
-      const bool ok = tc::mbar_wait(bbar, bphase, abort);
+      const bool ok = tc::mbar_wait(bbar, bphase, abort, a.wait_cycles);
       bphase ^= 1u;
       if (!ok) {
         if (lane == 0) raise_status(a.status, MOE_ERR_TIMEOUT);
@@ -300,7 +300,7 @@ __global__ void __launch_bounds__((1 + kGemvConsumers) * 32, 1)
       }
       return ok;
     };
-    for (int it = i0; it < i1 && !*abort; ++it) {
+    for (int it = i0; it < i1 && !tc::aborted(abort); ++it) {
       const int entry = it / MT;
       const TileEntry te = a.tiles[entry];
       const int rb = it % MT;
@@ -340,7 +340,7 @@ __global__ void __launch_bounds__((1 + kGemvConsumers) * 32, 1)
       const int64_t r0 = (int64_t)rb * kItemRows + rl;
       float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
       for (int kc = 0; kc < nkc; ++kc) {
-        if (!tc::mbar_wait(&full[stage], phase, abort)) {
+        if (!tc::mbar_wait(&full[stage], phase, abort, a.wait_cycles)) {
           if (lane == 0) raise_status(a.status, MOE_ERR_TIMEOUT);
           *abort = 1;
           break;

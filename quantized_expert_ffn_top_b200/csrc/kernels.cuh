@@ -12,6 +12,9 @@ namespace moe {
 // Host-side count of kernel launches (moe_kernel_launch_count).
 void count_launches(int n);
 
+// Bound of every device wait in SM clocks (MOE_OPT_WAIT_CYCLES).
+long long wait_cycles();
+
 // Launch with programmatic dependent launch allowed (MOE_OPT_PDL, on by
 // default): the kernel may begin while the previous kernel in the stream
 // finishes; it calls pdl_wait() before reading that kernel's results.
@@ -53,6 +56,19 @@ cudaError_t launch_quantize(int fmt, const void* x, int x_dtype, int64_t rows, i
                             const float* amax, uint8_t* codes, uint8_t* sf, float* scale_out, int num_sms,
                             cudaStream_t s);
 
+// Small batches: where and how x is quantised into the gather layout
+// (quant_token_gather in token_quant.cuh): the static tensor scale or the
+// amax it comes from (NVFP4), the codes [T][8][K/2] and the scale lines.
+// Tokens a gathering batch may hold: a tile's scale lines serve rows below 32,
+// and a token picks an expert at most once.
+constexpr int kGatherMaxT = 32;
+struct GatherQuant {
+  const float* scale;
+  const float* amax;
+  uint8_t* xg;
+  uint8_t* xsl;
+};
+
 // route.cu
 cudaError_t launch_router_logits(const uint16_t* x, int64_t T, int H, const uint16_t* wr, const float* bias, int E,
                                  float* logits, cudaStream_t s);
@@ -60,6 +76,13 @@ cudaError_t launch_router_logits(const uint16_t* x, int64_t T, int H, const uint
 // (nullable) receives their sum.
 cudaError_t launch_topk(const float* logits, int nparts, int64_t part_stride, float* logits_out, int64_t T, int E,
                         int k, int32_t* idx, float* w, int32_t* status, cudaStream_t s);
+// The one-kernel forward's router at T <= 32 (fmt NVFP4 or MXFP4, H % 256 ==
+// 0, E <= 256): logits (the small-batch order), x into the gather layout, and
+// the top k by the block that finishes last (`ticket`: zero on entry, left
+// zero).
+cudaError_t launch_router_decode(int fmt, const uint16_t* x, int64_t T, int H, const uint16_t* wr, const float* bias,
+                                 int E, int k, float* logits, int32_t* idx, float* w, int32_t* ticket,
+                                 const GatherQuant& q, int32_t* status, cudaStream_t s);
 
 // permute.cu
 struct PermuteScratch {
@@ -124,6 +147,7 @@ struct GemvArgs {
   const struct TileEntry* tiles;  // token groups of at most 8 slots per expert
   const int32_t* num_tiles;
   int32_t* status;
+  long long wait_cycles;   // bound of every device wait (SM clocks)
 };
 constexpr int kGemvTokens = 8;  // token columns of one GEMV work item (the MMA n)
 cudaError_t launch_gemv_up(const GemvArgs& a, int num_sms, cudaStream_t s);
@@ -132,6 +156,29 @@ cudaError_t launch_gemv_down(const GemvArgs& a, int num_sms, cudaStream_t s);
 // combine.cu
 cudaError_t launch_combine(const uint16_t* y_perm, const int32_t* inv_perm, const float* w, int64_t T, int k, int H,
                            const uint16_t* shared_y, uint16_t* out, int32_t* status, cudaStream_t s);
+// out[i] = bf16(out32[i]) for n values (n % 8 == 0, 16-byte aligned).
+cudaError_t launch_round_rows(const float* out32, int64_t n, uint16_t* out, int num_sms, cudaStream_t s);
+
+// cache.cu -- the HBM slot pool in front of a host-memory expert bank.
+// An expert's regions (W13, its scales, W2, its scales) are contiguous in
+// the PREPARED layout; src[r] + e * bytes[r] (device addresses of mapped
+// host memory) goes to dst[r] + slot * bytes[r], and gs_per[g] fp32 part
+// scales of gs_src[g] + e * gs_per[g] go to gs_dst[g] + slot * gs_per[g].
+struct CacheCopy {
+  const uint8_t* src[4];
+  uint8_t* dst[4];
+  int64_t bytes[4];
+  int nregions;
+  const float* gs_src[2];
+  float* gs_dst[2];
+  int gs_per[2];
+  int ngs;
+};
+size_t cache_state_words(int E, int n_slots);
+cudaError_t launch_cache_admit(const int32_t* idx, int64_t S, int E, int n_slots, int32_t* state, int32_t* idx_slot,
+                               int32_t* status, cudaStream_t s);
+cudaError_t launch_cache_fetch(const int32_t* state, int E, int n_slots, const CacheCopy& cc, int num_sms,
+                               cudaStream_t s);
 
 // prepare.cu
 cudaError_t launch_prepare_rows(int fmt, const uint8_t* src, uint8_t* dst, int64_t E, int64_t R, int64_t row_bytes,

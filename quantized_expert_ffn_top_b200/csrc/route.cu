@@ -9,6 +9,7 @@
 #include <math.h>
 
 #include "kernels.cuh"
+#include "token_quant.cuh"
 
 namespace moe {
 
@@ -21,18 +22,16 @@ namespace moe {
 constexpr int kSmallTGroup = 8;
 constexpr int kSmallThreads = 256;
 
-__global__ void __launch_bounds__(kSmallThreads) router_logits_small_kernel(const uint16_t* __restrict__ x, int64_t T,
-                                                                           int H, const uint16_t* __restrict__ wr,
-                                                                           const float* __restrict__ bias, int E,
-                                                                           float* __restrict__ logits) {
-  pdl_wait();  // inputs come from the previous kernels
-  pdl_trigger();
-
-  __shared__ float part[kSmallThreads / 32][kSmallTGroup];
+// The logits of expert `e` for tokens t0 .. t0 + nt - 1 (nt <= 8), by one
+// block of kSmallThreads threads, in the fixed order the header documents:
+// thread p adds the 8 columns from 8p, then those 2048 further on, ...; the
+// 32 threads of a warp are combined by an xor exchange; the 8 warp sums are
+// added in order; then the bias.
+__device__ __forceinline__ void small_logits_block(const uint16_t* __restrict__ x, int H,
+                                                   const uint16_t* __restrict__ wr, const float* __restrict__ bias,
+                                                   int E, int e, int64_t t0, int nt, float* __restrict__ logits,
+                                                   float (*part)[kSmallTGroup]) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int e = blockIdx.x;
-  const int64_t t0 = (int64_t)blockIdx.y * kSmallTGroup;
-  const int nt = (int)((T - t0) < kSmallTGroup ? (T - t0) : kSmallTGroup);
   float acc[kSmallTGroup];
 #pragma unroll
   for (int i = 0; i < kSmallTGroup; ++i) acc[i] = 0.0f;
@@ -66,6 +65,19 @@ __global__ void __launch_bounds__(kSmallThreads) router_logits_small_kernel(cons
     for (int w = 0; w < kSmallThreads / 32; ++w) v += part[w][threadIdx.x];
     logits[(t0 + threadIdx.x) * E + e] = v + (bias ? __ldg(bias + e) : 0.0f);
   }
+}
+
+__global__ void __launch_bounds__(kSmallThreads) router_logits_small_kernel(const uint16_t* __restrict__ x, int64_t T,
+                                                                           int H, const uint16_t* __restrict__ wr,
+                                                                           const float* __restrict__ bias, int E,
+                                                                           float* __restrict__ logits) {
+  pdl_wait();  // inputs come from the previous kernels
+  pdl_trigger();
+
+  __shared__ float part[kSmallThreads / 32][kSmallTGroup];
+  const int64_t t0 = (int64_t)blockIdx.y * kSmallTGroup;
+  const int nt = (int)((T - t0) < kSmallTGroup ? (T - t0) : kSmallTGroup);
+  small_logits_block(x, H, wr, bias, E, blockIdx.x, t0, nt, logits, part);
 }
 
 // Larger T: 64 tokens x 64 experts per block, K in chunks of 32 staged in
@@ -148,37 +160,35 @@ cudaError_t launch_router_logits(const uint16_t* x, int64_t T, int H, const uint
 // and writes indices 0..k-1 with zero weights.
 // The logits may arrive as nparts partial sums (a router GEMM split along
 // H), added here in part order; logits_out (nullable) receives the sums.
-template <int J>
-__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, int nparts, int64_t part_stride,
-                                                   float* __restrict__ logits_out, int64_t T, int E, int k,
-                                                   int32_t* __restrict__ idx, float* __restrict__ w,
-                                                   int32_t* status) {
-  pdl_wait();  // inputs come from the previous kernels
-  pdl_trigger();
-
+// Top-k of one token's logits row by one warp (J = ceil(E / 32) logits per
+// lane).  COHERENT: the row was written by other blocks of this kernel, so it
+// is read through L2 (ld.cg) rather than the read-only path.
+template <int J, bool COHERENT>
+__device__ __forceinline__ void topk_token(const float* __restrict__ L, int nparts, int64_t part_stride,
+                                           float* __restrict__ logits_out_row, int E, int k,
+                                           int32_t* __restrict__ idx_row, float* __restrict__ w_row,
+                                           int32_t* status) {
   const int lane = threadIdx.x & 31;
-  const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (t >= T) return;
-  const float* L = logits + t * E;
+  auto ld = [&](const float* p) { return COHERENT ? __ldcg(p) : __ldg(p); };
   float v[J];
   bool bad = false;
 #pragma unroll
   for (int j = 0; j < J; ++j) {
     const int e = lane + 32 * j;
-    v[j] = e < E ? __ldg(L + e) : -INFINITY;
+    v[j] = e < E ? ld(L + e) : -INFINITY;
   }
   for (int p = 1; p < nparts; ++p) {
 #pragma unroll
     for (int j = 0; j < J; ++j) {
       const int e = lane + 32 * j;
-      if (e < E) v[j] += __ldg(L + p * part_stride + e);
+      if (e < E) v[j] += ld(L + p * part_stride + e);
     }
   }
 #pragma unroll
   for (int j = 0; j < J; ++j) {
     const int e = lane + 32 * j;
     if (e < E && isnan(v[j])) bad = true;
-    if (e < E && logits_out) logits_out[t * E + e] = v[j];
+    if (e < E && logits_out_row) logits_out_row[e] = v[j];
   }
   uint32_t taken = 0u;
 #pragma unroll
@@ -214,8 +224,8 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
     const float ex = expf(bv - top);
     sum += ex;
     if (lane == 0) {
-      idx[t * k + r] = bad ? r : be;
-      w[t * k + r] = bad ? 0.0f : ex;
+      idx_row[r] = bad ? r : be;
+      w_row[r] = bad ? 0.0f : ex;
     }
   }
   __syncwarp();
@@ -223,7 +233,100 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
     if (lane == 0) raise_status(status, MOE_ERR_DEVICE_FAULT);
     return;
   }
-  for (int r = lane; r < k; r += 32) w[t * k + r] = __fdiv_rn(w[t * k + r], sum);
+  for (int r = lane; r < k; r += 32) w_row[r] = __fdiv_rn(w_row[r], sum);
+}
+
+// One warp per token; lane l holds logits l, l+32, ... in registers.  Each
+// round picks the largest not-yet-taken logit (ties -> lower index) with a
+// warp arg-max; lane 0 writes the index and exp(L - L_0); a final pass divides
+// by the sum.  A NaN, or a row without a finite logit, raises the status word
+// and writes indices 0..k-1 with zero weights.
+// The logits may arrive as nparts partial sums (a router GEMM split along
+// H), added here in part order; logits_out (nullable) receives the sums.
+template <int J>
+__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, int nparts, int64_t part_stride,
+                                                   float* __restrict__ logits_out, int64_t T, int E, int k,
+                                                   int32_t* __restrict__ idx, float* __restrict__ w,
+                                                   int32_t* status) {
+  pdl_wait();  // inputs come from the previous kernels
+  pdl_trigger();
+
+  const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= T) return;
+  topk_token<J, false>(logits + t * E, nparts, part_stride, logits_out ? logits_out + t * E : nullptr, E, k,
+                       idx + t * k, w + t * k, status);
+}
+
+// The first kernel of the one-kernel forward at small batches (T <= 32):
+// the logits exactly as router_logits_small_kernel computes them (the same
+// fixed summation order), block (0, g) also quantises its token group into
+// the gather layout (quant_token_gather), and the block that finishes last
+// -- one ticket, reset by that block -- picks every token's top k.
+template <int QFMT, int J>
+__global__ void __launch_bounds__(kSmallThreads) router_decode_kernel(const uint16_t* __restrict__ x, int64_t T,
+                                                                     int H, const uint16_t* __restrict__ wr,
+                                                                     const float* __restrict__ bias, int E, int k,
+                                                                     float* __restrict__ logits,
+                                                                     int32_t* __restrict__ idx, float* __restrict__ w,
+                                                                     int32_t* ticket, GatherQuant q,
+                                                                     int32_t* status) {
+  pdl_wait();  // inputs come from the previous kernels
+  pdl_trigger();
+
+  __shared__ float part[kSmallThreads / 32][kSmallTGroup];
+  __shared__ float r_tab[128];
+  __shared__ int is_last;
+  const int warp = threadIdx.x >> 5;
+  const int64_t t0 = (int64_t)blockIdx.y * kSmallTGroup;
+  const int nt = (int)((T - t0) < kSmallTGroup ? (T - t0) : kSmallTGroup);
+  small_logits_block(x, H, wr, bias, E, blockIdx.x, t0, nt, logits, part);
+  if (blockIdx.x == 0) {
+    constexpr int bs = QFMT == MOE_FMT_MXFP4 ? 32 : 16;
+    const float scale = act_scale_of(QFMT, q.scale, q.amax);
+    if (QFMT == MOE_FMT_NVFP4 && threadIdx.x < 128) r_tab[threadIdx.x] = nvfp4_multiplier(threadIdx.x, scale);
+    __syncthreads();
+    if (warp < nt) {
+      const int64_t t = t0 + warp;
+      quant_token_gather<QFMT>(x + t * H, H, scale, r_tab, q.xg + t * 8 * (H / 2), q.xsl + t * (H / (4 * bs)) * 16);
+    }
+  }
+  // the block that finishes last picks the top k of every token
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) is_last = atomicAdd(ticket, 1) == (int)(gridDim.x * gridDim.y) - 1;
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  for (int64_t t = warp; t < T; t += kSmallThreads / 32)
+    topk_token<J, true>(logits + t * E, 1, 0, nullptr, E, k, idx + t * k, w + t * k, status);
+  if (threadIdx.x == 0) *ticket = 0;
+}
+
+cudaError_t launch_router_decode(int fmt, const uint16_t* x, int64_t T, int H, const uint16_t* wr, const float* bias,
+                                 int E, int k, float* logits, int32_t* idx, float* w, int32_t* ticket,
+                                 const GatherQuant& q, int32_t* status, cudaStream_t s) {
+  if (T == 0) return cudaSuccess;
+  if (T > kGatherMaxT || H % 256 != 0 || E > 256) return cudaErrorInvalidValue;
+  const dim3 grid((unsigned)E, (unsigned)((T + kSmallTGroup - 1) / kSmallTGroup));
+  const int J = (E + 31) / 32;
+  cudaError_t e = cudaErrorInvalidValue;
+#define MOE_RD(F, JJ) \
+  e = launch_pdl(router_decode_kernel<F, JJ>, grid, dim3(kSmallThreads), 0, s, x, T, H, wr, bias, E, k, logits, idx, w, \
+                 ticket, q, status)
+#define MOE_RD_J(F) \
+  if (J <= 1) MOE_RD(F, 1); else if (J <= 2) MOE_RD(F, 2); else if (J <= 4) MOE_RD(F, 4); else MOE_RD(F, 8);
+  if (fmt == MOE_FMT_NVFP4) {
+    MOE_RD_J(MOE_FMT_NVFP4)
+  } else if (fmt == MOE_FMT_MXFP4) {
+    MOE_RD_J(MOE_FMT_MXFP4)
+  } else {
+    return cudaErrorInvalidValue;
+  }
+#undef MOE_RD_J
+#undef MOE_RD
+  if (e != cudaSuccess) return e;
+  count_launches(1);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_topk(const float* logits, int nparts, int64_t part_stride, float* logits_out, int64_t T, int E,

@@ -10,9 +10,11 @@
 namespace moe {
 namespace tc {
 
-// A wait that has not completed after this many SM clocks (about a second)
-// gives up: the kernel raises MOE_ERR_TIMEOUT instead of hanging.
-constexpr long long kWaitCycles = 2000000000LL;
+// Default bound of every device wait, in SM clocks (about a second at
+// 1.965 GHz): a wait that has not completed by then gives up and the kernel
+// raises MOE_ERR_TIMEOUT instead of hanging.  The kernels take the bound as
+// an argument (MOE_OPT_WAIT_CYCLES).
+constexpr long long kDefaultWaitCycles = 2000000000LL;
 
 // One lane of a converged warp (the same lane on every call).
 __device__ __forceinline__ bool elect_one() {
@@ -61,15 +63,52 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* b, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Bounded wait on phase `parity`; false when it timed out or `abort` was set.
-__device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, volatile int* abort) {
-  if (mbar_try_wait(b, parity)) return true;
+// Below this many cycles a bound is checked between non-blocking tests
+// (try_wait may suspend the thread until the phase completes, past a short
+// bound): the bound, not the hardware's suspend limit, decides when a wait
+// gives up.  Such bounds serve to test the timeout path.
+constexpr long long kShortWaitCycles = 1000000LL;
+// Bounded wait of one thread on phase `parity`; false when it ran past
+// `limit` cycles or `abort` was set.
+__device__ __forceinline__ bool mbar_wait_thread(uint64_t* b, uint32_t parity, volatile int* abort, long long limit) {
+  if (limit >= kShortWaitCycles) {
+    if (mbar_try_wait(b, parity)) return true;
+    const long long t0 = clock64();
+    while (!mbar_try_wait(b, parity)) {
+      if (*abort) return false;
+      if (clock64() - t0 > limit) return false;
+    }
+    return true;
+  }
   const long long t0 = clock64();
-  while (!mbar_try_wait(b, parity)) {
+  while (!mbar_test_wait(b, parity)) {
     if (*abort) return false;
-    if (clock64() - t0 > kWaitCycles) return false;
+    if (clock64() - t0 > limit) return false;
   }
   return true;
+}
+// The same wait for a whole converged warp.  Every lane gets the same answer
+// (false if any lane gave up), so the warp leaves its loop as one: the
+// .sync.aligned instructions after it (elect, shuffles, tensor-memory loads)
+// never see a split warp.
+__device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, volatile int* abort, long long limit) {
+  return __all_sync(0xffffffffu, mbar_wait_thread(b, parity, abort, limit));
+}
+// Whether the CTA's abort flag is set, as one answer for the whole warp (the
+// flag may change between two lanes' reads).
+__device__ __forceinline__ bool aborted(volatile int* abort) { return __any_sync(0xffffffffu, *abort != 0); }
+// AND of `p` over the 64 threads of two warps that meet at named barrier
+// `bar` (both warps must call it, converged): the two decide together.
+__device__ __forceinline__ bool pair_all(bool p, int bar) {
+  uint32_t r;
+  __syncwarp();
+  asm volatile(
+      "{\n\t.reg .pred a, b;\n\tsetp.ne.u32 a, %1, 0;\n\tbar.red.and.pred b, %2, 64, a;\n\t"
+      "selp.u32 %0, 1, 0, b;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)p), "r"(bar)
+      : "memory");
+  return r != 0;
 }
 
 // ----------------------------------------------------- CTA pairs (clusters) --

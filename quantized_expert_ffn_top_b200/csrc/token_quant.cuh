@@ -157,3 +157,105 @@ __device__ __forceinline__ void quant_token_slots(const uint16_t* __restrict__ x
 }
 
 }  // namespace moe
+
+namespace moe {
+
+// Small batches: the quantised x rows in a layout the expert FFN can gather
+// from with plain bulk copies, whatever the routing.  For token t and
+// variant v (0..7) the codes of K-stage kb (256 values, 128 bytes) sit at
+// xg[((t * 8 + v) * K / 2) + kb * 128] with their 16-byte pieces in the
+// order of the tensor cores' 128-byte swizzle for a row r with r % 8 == v
+// (piece p at position p ^ v): a row copied into tile row r of a stage is
+// then already where the MMA reads it.  The block scales go to 16-byte
+// lines, one per group of 4 scales (xsl[(t * K / (4 bs) + g) * 16]: the
+// group's 4 scale bytes, then 12 zero bytes): copied to line r of the
+// group's 512-byte block they are tile row r's scales for rows below 32.
+
+template <int FMT>
+__device__ __forceinline__ void quant_token_gather(const uint16_t* __restrict__ xt, int K, float scale,
+                                                   const float* r_tab, uint8_t* __restrict__ xg_t,
+                                                   uint8_t* __restrict__ xsl_t) {
+  static_assert(FMT == MOE_FMT_NVFP4 || FMT == MOE_FMT_MXFP4, "block-scaled FP4 formats");
+  using Q = TokenQuant<FMT>;
+  constexpr int bs = Q::kBs, kPer = Q::kPer;
+  const int lane = threadIdx.x & 31;
+  for (int c0 = 0; c0 < K; c0 += 32 * kPer) {
+    const int c = c0 + lane * kPer;
+    const bool active = c < K;
+    uint32_t w[8];
+    uint32_t sfw = 0;
+    if (active) {
+      uint32_t raw[kPer / 2];
+      const uint4* src = reinterpret_cast<const uint4*>(xt + c);
+#pragma unroll
+      for (int i = 0; i < kPer / 8; ++i) {
+        const uint4 u = __ldg(src + i);
+        raw[4 * i] = u.x;
+        raw[4 * i + 1] = u.y;
+        raw[4 * i + 2] = u.z;
+        raw[4 * i + 3] = u.w;
+      }
+      auto unpack = [&](float* v, int first, int n) {
+#pragma unroll
+        for (int i = 0; i < n / 2; ++i) {
+          v[2 * i] = __uint_as_float(raw[first / 2 + i] << 16);
+          v[2 * i + 1] = __uint_as_float(raw[first / 2 + i] & 0xFFFF0000u);
+        }
+      };
+      if constexpr (FMT == MOE_FMT_NVFP4) {
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          float v[16];
+          unpack(v, 16 * b, 16);
+          float bmax = 0.0f;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) bmax = fmaxf(bmax, fabsf(v[i]));
+          const uint32_t sc = nvfp4_scale_code(bmax, scale);
+          const uint2 cw = nvfp4_encode16(v, r_tab[sc]);
+          w[2 * b] = cw.x;
+          w[2 * b + 1] = cw.y;
+          sfw |= sc << (8 * b);
+        }
+      } else {
+#pragma unroll
+        for (int b = 0; b < 2; ++b) {
+          float v[32];
+          unpack(v, 32 * b, 32);
+          float bmax = 0.0f;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) bmax = fmaxf(bmax, fabsf(v[i]));
+          uint32_t sc;
+          float inv;
+          mxfp4_block_scale(bmax, sc, inv);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) w[4 * b + q] = e2m1_encode8(v + 8 * q, inv);
+          sfw |= sc << (8 * b);
+        }
+      }
+    }
+    // the lane's 32 code bytes are pieces 2 (lane % 4) and 2 (lane % 4) + 1
+    // of K-stage (c / 256); one copy per variant
+    if (active) {
+      const int64_t kb_off = (int64_t)(c / 256) * 128;
+      const int p0 = 2 * (lane & 3);
+      const uint4 a = make_uint4(w[0], w[1], w[2], w[3]), b = make_uint4(w[4], w[5], w[6], w[7]);
+#pragma unroll
+      for (int v = 0; v < 8; ++v) {
+        uint8_t* row = xg_t + (int64_t)v * (K / 2) + kb_off;
+        *reinterpret_cast<uint4*>(row + ((p0 ^ v) << 4)) = a;
+        *reinterpret_cast<uint4*>(row + (((p0 + 1) ^ v) << 4)) = b;
+      }
+    }
+    // scale lines: NVFP4 holds one group of 4 scales per lane, MXFP4 two
+    // scales (half a group): the even lane of a pair writes the line
+    if constexpr (FMT == MOE_FMT_NVFP4) {
+      if (active) *reinterpret_cast<uint4*>(xsl_t + (int64_t)(c / 64) * 16) = make_uint4(sfw, 0u, 0u, 0u);
+    } else {
+      const uint32_t hi = __shfl_down_sync(0xffffffffu, sfw, 1);
+      if (active && (lane & 1) == 0)
+        *reinterpret_cast<uint4*>(xsl_t + (int64_t)(c / 128) * 16) = make_uint4(sfw | (hi << 16), 0u, 0u, 0u);
+    }
+  }
+}
+
+}  // namespace moe

@@ -27,6 +27,9 @@ OPT_PDL = 4
 OPT_EARLY_WEIGHTS = 5
 OPT_FUSED_FFN = 6
 OPT_PERMUTE_QUANT = 7
+OPT_WAIT_CYCLES = 8
+OPT_FUSED_COMBINE = 9
+OPT_SMALL_BATCH_FORWARD = 10
 FMT_BY_NAME = {"nvfp4": FMT_NVFP4, "mxfp4": FMT_MXFP4, "fp8": FMT_FP8, "bf16": FMT_BF16}
 
 
@@ -38,7 +41,8 @@ EXPORTED = (
     "moe_status_string", "moe_version", "moe_set_option", "moe_workspace_size", "moe_prepared_weights_size",
     "moe_prepare_weights", "moe_dequantize_weights", "moe_dequantized_weights_size", "moe_quantize", "moe_route", "moe_route_logits", "moe_permute", "moe_grouped_ffn",
     "moe_combine", "moe_forward", "moe_get_device_status", "moe_set_stage_events", "moe_kernel_launch_count",
-    "moe_permute_fixed_scratch", "moe_forward_host",
+    "moe_permute_fixed_scratch", "moe_forward_host", "moe_stage_mask", "moe_expert_cache_bytes",
+    "moe_expert_cache_init", "moe_forward_cached", "moe_expert_cache_stats",
 )
 MAX_HOST_SLICES = 64
 STAGES = ("route", "permute", "act_quant", "ffn_up", "ffn_down", "shared", "combine")
@@ -57,6 +61,13 @@ class MoeWeightsC(ctypes.Structure):
         ("w13", ctypes.c_void_p), ("w13_sf", ctypes.c_void_p), ("w13_gs", ctypes.c_void_p),
         ("w2", ctypes.c_void_p), ("w2_sf", ctypes.c_void_p), ("w2_gs", ctypes.c_void_p),
         ("a13_gs", ctypes.c_void_p), ("a2_gs", ctypes.c_void_p),
+    ]
+
+
+class MoeExpertCacheC(ctypes.Structure):
+    _fields_ = [
+        ("bank", MoeWeightsC), ("pool", MoeWeightsC), ("bank_dev", ctypes.c_void_p * 6),
+        ("state", ctypes.c_void_p), ("n_slots", ctypes.c_int32),
     ]
 
 
@@ -98,6 +109,12 @@ def _declare(L):
         "moe_get_device_status": ([P, P, ctypes.POINTER(ctypes.c_int32)], ctypes.c_int),
         "moe_set_stage_events": ([ctypes.POINTER(ctypes.c_void_p), i32], ctypes.c_int),
         "moe_kernel_launch_count": ([], ctypes.c_uint64),
+        "moe_stage_mask": ([], ctypes.c_uint32),
+        "moe_expert_cache_bytes": ([W, i32], sz),
+        "moe_expert_cache_init": ([W, i32, P, sz, ctypes.POINTER(MoeExpertCacheC), P], ctypes.c_int),
+        "moe_forward_cached": ([P, i64, P, P, i32, ctypes.POINTER(MoeExpertCacheC), i32, P, P, sz, P], ctypes.c_int),
+        "moe_expert_cache_stats": ([ctypes.POINTER(MoeExpertCacheC), P, ctypes.POINTER(ctypes.c_int64)],
+                                   ctypes.c_int),
         "moe_permute_fixed_scratch": ([P, i64, i32, i32, P, P, P, P, P], ctypes.c_int),
         "moe_forward_host": ([P, i64, P, P, i32, W, W, i32, P, P, P, i32, P, sz, P], ctypes.c_int),
     }
@@ -326,6 +343,52 @@ def moe_forward_host(x_host: torch.Tensor, wr: torch.Tensor, bias: torch.Tensor 
     return o
 
 
+# ------------------------------------------------------------ expert cache --
+@dataclass
+class ExpertCache:
+    """An HBM pool of n_slots expert slots in front of a host-memory bank."""
+    c: MoeExpertCacheC
+    dev: torch.Tensor
+    host: WeightBank
+
+
+def bank_to_host(bank: WeightBank) -> WeightBank:
+    """A PREPARED device bank copied to page-locked host memory (the activation
+    scales stay on the device)."""
+    if bank.layout != LAYOUT_PREPARED:
+        raise ValueError("a PREPARED bank is expected")
+    h = lambda t: None if t is None else t.cpu().pin_memory()
+    return replace(bank, w13=h(bank.w13), w13_sf=h(bank.w13_sf), w13_gs=h(bank.w13_gs), w2=h(bank.w2),
+                   w2_sf=h(bank.w2_sf), w2_gs=h(bank.w2_gs), keep=[])
+
+
+def moe_expert_cache_init(host_bank: WeightBank, n_slots: int, stream=None) -> ExpertCache:
+    b = host_bank.struct()
+    n = lib().moe_expert_cache_bytes(ctypes.byref(b), int(n_slots))
+    if n == 0:
+        raise MoeError(1, "moe_expert_cache_bytes")
+    dev = torch.empty(int(n), dtype=torch.uint8, device="cuda")
+    c = MoeExpertCacheC()
+    _check(lib().moe_expert_cache_init(ctypes.byref(b), int(n_slots), _p(dev), n, ctypes.byref(c), _stream(stream)),
+           "moe_expert_cache_init")
+    return ExpertCache(c, dev, host_bank)
+
+
+def moe_forward_cached(x: torch.Tensor, wr: torch.Tensor, bias: torch.Tensor | None, k: int, cache: ExpertCache,
+                       act: int, ws: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    T, H = x.shape
+    o = out if out is not None else torch.empty((T, H), dtype=torch.bfloat16, device=x.device)
+    _check(lib().moe_forward_cached(_p(x), T, _p(wr), _p(bias), k, ctypes.byref(cache.c), act, _p(o), _p(ws),
+                                    ws.numel(), _stream(stream)), "moe_forward_cached")
+    return o
+
+
+def moe_expert_cache_stats(cache: ExpertCache, stream=None) -> dict:
+    v = (ctypes.c_int64 * 4)()
+    _check(lib().moe_expert_cache_stats(ctypes.byref(cache.c), _stream(stream), v), "moe_expert_cache_stats")
+    return {"calls": int(v[0]), "fetched_last": int(v[1]), "fetched": int(v[2]), "hits": int(v[3])}
+
+
 def moe_get_device_status(ws: torch.Tensor, stream=None) -> int:
     v = ctypes.c_int32(0)
     _check(lib().moe_get_device_status(_p(ws), _stream(stream), ctypes.byref(v)), "moe_get_device_status")
@@ -395,6 +458,11 @@ def moe_set_stage_events(events):
             e.record()
     arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
     _check(lib().moe_set_stage_events(arr, len(events)), "moe_set_stage_events")
+
+
+def moe_stage_mask() -> int:
+    """Bit s: stage STAGES[s] was recorded since events were last installed."""
+    return int(lib().moe_stage_mask())
 
 
 def moe_kernel_launch_count() -> int:

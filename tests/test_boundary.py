@@ -128,3 +128,45 @@ def test_host_side_argument_errors(L):
     one_slice = L.moe_workspace_size(16, 2, ctypes.byref(g), None, 1)
     assert fh(ws_bytes=one_slice - 1) == 3
     assert fh(T=0, ws_bytes=one_slice) == 0
+
+
+def test_wait_bound_option(L):
+    """MOE_OPT_WAIT_CYCLES: any positive cycle count, 0 restores the default,
+    a negative count is rejected."""
+    assert L.moe_set_option(ops.OPT_WAIT_CYCLES, -1) == 1
+    assert L.moe_set_option(ops.OPT_WAIT_CYCLES, 1) == 0
+    assert L.moe_set_option(ops.OPT_WAIT_CYCLES, 2 ** 31 - 1) == 0
+    assert L.moe_set_option(ops.OPT_WAIT_CYCLES, 0) == 0
+    hdr = open(os.path.join(ROOT, "include", "moe_b200.h")).read()
+    assert re.search(r"MOE_OPT_WAIT_CYCLES = (\d+)", hdr).group(1) == str(ops.OPT_WAIT_CYCLES)
+
+
+@pytest.mark.parametrize("E,H,I,k", [(128, 128, 256, 2), (256, 4096, 2048, 8), (8, 256, 256, 2)])
+def test_workspace_size_never_decreases_with_T(L, E, H, I, k):
+    """A workspace sized for T serves every smaller batch: moe_forward_host
+    sizes one for its first slice and runs a shorter last slice in it.  The
+    sweep crosses the batch sizes where the router's split of H changes."""
+    b = _bank(E=E, H=H, I=I, layout=1)
+    prev = 0
+    for T in sorted(set(range(0, 300)) | set(range(300, 9000, 37)) | {4036, 4037, 4096, 4100, 16384, 16385}):
+        n = L.moe_workspace_size(T, k, ctypes.byref(b), None, 1)
+        assert n >= prev, (T, n, prev)
+        prev = n
+
+
+def test_host_slices_with_a_shorter_last_slice(L):
+    """An uneven last slice that falls where the router's split is deeper than
+    at the first slice's size: the workspace for ceil(T / n) tokens is
+    accepted, and no slice needs more (checked by the host-side sizing
+    before anything is enqueued)."""
+    g = _bank(E=128, H=128, I=256, layout=1)
+    T, n = 63 * 4100 + 4037, 64
+    Ts = -(-T // n)
+    ws_bytes = L.moe_workspace_size(Ts, 2, ctypes.byref(g), None, 1)
+    assert ws_bytes >= L.moe_workspace_size(T - (n - 1) * Ts, 2, ctypes.byref(g), None, 1)
+    P = ctypes.c_void_p
+    one = P(256)
+    host = P(4096)
+    # one byte short is rejected on the host, before any CUDA call
+    assert L.moe_forward_host(host, T, one, None, 2, ctypes.byref(g), None, 1, host, one, one, n, one,
+                              ws_bytes - 1, None) == 3

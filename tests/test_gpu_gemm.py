@@ -285,3 +285,30 @@ def test_fp8_shared_forward_full_size():
     r, keep = forward_reference(w, x, wr, b, W, Ws, act=1, what="fp8_shared")
     err = max_abs_rel(dev_to_f64(out)[keep], r["out"][keep])
     assert err < TOL, err
+
+
+GATHER_CASES = [
+    ("nvfp4-decode", dict(fmt="nvfp4", T=4, H=2048, E=128, k=8, I=768), True, 0.0),
+    ("nvfp4-32", dict(fmt="nvfp4", T=32, H=512, E=32, k=4, I=256), True, 1.2),
+    ("mxfp4-7", dict(fmt="mxfp4", T=7, H=512, E=6, k=2, I=256), False, 0.8),
+]
+
+
+@pytest.mark.parametrize("name,over,static,skew", GATHER_CASES)
+def test_gathered_token_rows_change_nothing(name, over, static, skew):
+    """Small batches (T <= 32): the one-kernel FFN copies each tile's token
+    rows from the gather layout of x instead of loading quantised padded rows;
+    y_perm is bit-identical to the two separate projections' and within the
+    tolerance of the oracle."""
+    ys = []
+    try:
+        for fused in (0, 1):
+            ops.moe_set_option(ops.OPT_FUSED_FFN, fused)
+            w, W, x, perm, off, a13, a2, y, st = _run(over, static, skew, 2)
+            assert st == 0, fused
+            ys.append(y)
+    finally:
+        ops.moe_set_option(ops.OPT_FUSED_FFN, 1)
+    assert np.array_equal(ys[0], ys[1])
+    ry, _ = oracle.grouped_ffn(x, perm, off, W, 1, a13 or 0.0, a2 or 0.0)
+    assert max_abs_rel(ys[1], ry) < TOL

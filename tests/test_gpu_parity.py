@@ -10,8 +10,9 @@ import torch
 
 import oracle
 from quantized_expert_ffn_top_b200 import ops, synth
-from tests.gpu_helpers import (TOL, ambiguous_tokens, bits_to_dev_bf16, dev_to_f64, device_bank, max_abs_rel,
-                               oracle_bank, routed_inputs)
+from tests.gpu_helpers import (TOL, ambiguous_tokens, bits_to_dev_bf16, dev_to_f64, device_bank,
+                               forward_reference, max_abs_rel, oracle_bank, report_ambiguous, routed_inputs,
+                               router_order, routing_tol)
 
 pytestmark = pytest.mark.gpu
 
@@ -137,28 +138,50 @@ def test_route_logits_flags_invalid_rows():
     assert np.allclose(wn[3], 0.25)
 
 
-@pytest.mark.parametrize("name,over", [("tiny", {}), ("decode", {}), ("prefill", {}), ("large", dict(T=300)),
-                                       ("fp8_shared", dict(T=130))])
+ROUTE_CASES = [("tiny", {}), ("decode", {}), ("prefill", {}), ("large", dict(T=300)), ("fp8_shared", dict(T=130)),
+               # small batches: the fixed small-batch order, Zipf bias, H = 4096 (two stretches),
+               # H = 2304 (a ragged second stretch), one token
+               ("prefill", dict(T=64)), ("large", dict(T=37)), ("decode", dict(T=9, H=2304, E=60, k=4)),
+               ("large", dict(T=1)),
+               # the sequential order: 64 < T < 128, or E not a multiple of 128
+               ("decode", dict(T=100)), ("prefill", dict(T=300, E=60, k=4)), ("tiny", dict(T=200))]
+
+
+@pytest.mark.parametrize("name,over", ROUTE_CASES)
 def test_route_matches_oracle(name, over):
-    """Small batches use the CUDA-core router, larger ones the tcgen05 bf16 GEMM."""
+    """Small batches and shapes off the tensor-core grid sum the logits in a
+    fixed fp32 order that the oracle replays: logits, indices and the
+    selection are then bit-exact on every token.  Larger batches use the
+    tcgen05 bf16 GEMM: its logits are within rounding of the fp64 ones, and
+    the indices match on every token whose k/k+1 gap exceeds twice the
+    largest logit difference seen (those left out are counted and bounded)."""
     w = synth.workload(name, **over)
     x, wr, b = routed_inputs(w)
     logits = torch.empty((w.T, w.E), dtype=torch.float32, device="cuda")
     idx, wt = ops.moe_route(bits_to_dev_bf16(x), bits_to_dev_bf16(wr),
                             None if b is None else torch.from_numpy(b).cuda(), w.k, ws(), logits=logits)
-    RL = oracle.router_logits(x, wr, b)
-    gl = logits.cpu().numpy().astype(np.float64)
-    assert max_abs_rel(gl, RL) < 1e-5
-    ridx, rw, _ = oracle.topk(RL, w.k)
-    amb = ambiguous_tokens(RL, w.k, 1e-4)
-    assert amb.mean() < 0.05
+    gl = logits.cpu().numpy()
     gi = idx.cpu().numpy()
+    order = router_order(w.T, w.E, w.H)
+    RL = oracle.router_logits(x, wr, b)
+    assert max_abs_rel(gl.astype(np.float64), RL) < 1e-5
+    if order:
+        OL = oracle.router_logits_ordered(x, wr, b, order=order)
+        assert np.array_equal(gl, OL), f"order {order}: {np.sum(gl != OL)} logits differ"
+        ridx, rw, st = oracle.topk(OL.astype(np.float64), w.k)
+        assert st == 0
+        assert np.array_equal(gi, ridx)
+        assert np.allclose(wt.cpu().numpy(), rw, rtol=2e-6, atol=1e-7)
+        return
+    ridx, rw, _ = oracle.topk(RL, w.k)
+    amb = ambiguous_tokens(RL, w.k, routing_tol(RL, gl))
+    report_ambiguous(amb, f"route {name} {over}")
     assert np.array_equal(gi[~amb], ridx[~amb])
     assert np.allclose(wt.cpu().numpy()[~amb], rw[~amb], rtol=1e-4, atol=1e-6)
     # ambiguous tokens: still k distinct experts, ordered by the GPU's logits
     for t in np.nonzero(amb)[0]:
         assert len(set(gi[t])) == w.k
-        assert np.all(np.diff(gl[t, gi[t]]) <= 0)
+        assert np.all(np.diff(gl[t, gi[t]].astype(np.float64)) <= 0)
 
 
 # ----------------------------------------------------------- permutation ----
@@ -260,6 +283,11 @@ FWD_CASES = [
     # degenerate layers: one expert (k = 1), every expert picked (k = E), one token
     ("tiny", dict(E=1, k=1, T=16), 1, False), ("tiny", dict(E=4, k=4, T=33), 1, False),
     ("tiny", dict(T=1), 1, False),
+    # a shared expert beside the one-kernel FFN at small batches: two
+    # persistent FFN kernels (routed, shared) run at once on two streams, so
+    # neither has every SM to itself
+    ("decode", dict(shared_I=768), 1, True),
+    ("tiny", dict(fmt="mxfp4", T=6, H=256, E=8, k=2, I=256, shared_I=256), 1, False),
 ]
 
 
@@ -275,9 +303,7 @@ def test_forward_matches_oracle(name, over, act, static):
     out = ops.moe_forward(bits_to_dev_bf16(x), bits_to_dev_bf16(wr), None if b is None else torch.from_numpy(b).cuda(),
                           w.k, bank, sbank, act, W_)
     assert ops.moe_get_device_status(W_) == 0
-    r = oracle.moe_forward(x, wr, b, w.k, W, Ws, act=act, a13_static=a13 or 0.0, a2_static=a2 or 0.0,
-                           sh_a2_static=a2 or 0.0)
-    keep = ~ambiguous_tokens(r["logits"], w.k, 1e-4, boundary_only=True)
+    r, keep = forward_reference(w, x, wr, b, W, Ws, act=act, a13=a13, a2=a2, sh_a2=a2, what=f"{name} {over}")
     err = max_abs_rel(dev_to_f64(out)[keep], r["out"][keep])
     assert err < TOL, err
 
@@ -315,6 +341,7 @@ def test_permutation_with_x_quantisation_changes_nothing(name, over, scales):
     W_ = ws(ops.workspace_size(w.T, w.k, bank, None, 1))
     outs, launches = [], []
     try:
+        ops.moe_set_option(ops.OPT_SMALL_BATCH_FORWARD, 0)   # the permutation path
         for opt in (0, 1):
             ops.moe_set_option(ops.OPT_PERMUTE_QUANT, opt)
             n0 = ops.moe_kernel_launch_count()
@@ -324,10 +351,11 @@ def test_permutation_with_x_quantisation_changes_nothing(name, over, scales):
             outs.append(out.view(torch.int16).cpu().numpy())
     finally:
         ops.moe_set_option(ops.OPT_PERMUTE_QUANT, 1)
+        ops.moe_set_option(ops.OPT_SMALL_BATCH_FORWARD, 1)
     assert np.array_equal(outs[0], outs[1])
     assert launches[1] == launches[0] - 1, launches
-    r = oracle.moe_forward(x, wr, b, w.k, W, None, act=1, a13_static=a13 or 0.0, a2_static=a2 or 0.0)
-    keep = ~ambiguous_tokens(r["logits"], w.k, 1e-4, boundary_only=True)
+    r, keep = forward_reference(w, x, wr, b, W, act=1, a13=a13, a2=a2)
+    assert keep.all()
     got = outs[1].view(np.uint16).astype(np.uint32) << 16
     err = max_abs_rel(got.view(np.float32).astype(np.float64)[keep], r["out"][keep])
     assert err < TOL, err
@@ -363,8 +391,7 @@ def test_forward_on_host_buffers_matches_oracle(name, over, scales, n_slices):
     torch.cuda.synchronize()
     assert ops.moe_get_device_status(W_) == 0
     assert torch.equal(out_dev.cpu(), out)
-    r = oracle.moe_forward(x, wr, b, w.k, W, None, act=1, a13_static=a13 or 0.0, a2_static=a2 or 0.0)
-    keep = ~ambiguous_tokens(r["logits"], w.k, 1e-4, boundary_only=True)
+    r, keep = forward_reference(w, x, wr, b, W, act=1, a13=a13, a2=a2, route_T=Ts)
     err = max_abs_rel(out.float().numpy().astype(np.float64)[keep], r["out"][keep])
     assert err < TOL, err
 
@@ -385,3 +412,89 @@ def test_forward_and_ffn_with_no_tokens():
     assert y.shape == (0, w.H)
     torch.cuda.synchronize()
     assert ops.moe_get_device_status(W_) == 0
+
+
+# the weighted combine in the down projection's epilogue (fp32 reductions)
+# against the ordered combine of bf16 y_perm, and both against the oracle:
+# NVFP4 prefill-shaped batches (192-token tiles, single CTAs and CTA pairs),
+# MXFP4, and FP8 with a shared expert adding into the same rows
+FUSED_COMBINE_CASES = [
+    ("prefill", dict(T=600, E=32), True),
+    ("tiny", dict(T=300, H=4096, E=8, k=2, I=512), True),
+    ("tiny", dict(fmt="mxfp4", T=200, H=512, E=8, k=2, I=256), False),
+    ("fp8_shared", dict(T=160, H=256, E=16, k=4, I=128, shared_I=128), False),
+]
+
+
+@pytest.mark.parametrize("name,over,static", FUSED_COMBINE_CASES)
+def test_combine_in_down_epilogue_matches_ordered_combine(name, over, static):
+    w = synth.workload(name, **over)
+    W, Ws = oracle_bank(w)
+    a13, a2 = synth.static_act_scales() if static else (None, None)
+    bank = device_bank(W, a13, a2)
+    sbank = device_bank(Ws, None, a2) if Ws is not None else None
+    x, wr, b = routed_inputs(w)
+    xd, wrd = bits_to_dev_bf16(x), bits_to_dev_bf16(wr)
+    bd = None if b is None else torch.from_numpy(b).cuda()
+    W_ = ws(ops.workspace_size(w.T, w.k, bank, sbank, 1))
+    outs = []
+    try:
+        for fused in (0, 1):
+            ops.moe_set_option(ops.OPT_FUSED_COMBINE, fused)
+            n0 = ops.moe_kernel_launch_count()
+            o = ops.moe_forward(xd, wrd, bd, w.k, bank, sbank, 1, W_)
+            assert ops.moe_get_device_status(W_) == 0, fused
+            outs.append(dev_to_f64(o))
+    finally:
+        ops.moe_set_option(ops.OPT_FUSED_COMBINE, 1)
+    # apart by the bf16 rounding of y_perm and of each output (a few bf16
+    # ulps of the largest output), half the layer tolerance at most
+    assert max_abs_rel(outs[1], outs[0]) < 1e-2
+    r, keep = forward_reference(w, x, wr, b, W, Ws, act=1, a13=a13, a2=a2, sh_a2=a2, what=f"{name} {over}")
+    for o in outs:
+        assert max_abs_rel(o[keep], r["out"][keep]) < TOL
+
+
+# small batches in two kernels (router with x quantisation and top-k; the
+# FFN gathering token rows, combining in its down epilogue and rounding in
+# its last CTA) against the permutation path, and both against the oracle on
+# every token (the small-batch router's order is replayed exactly)
+SMALL_FORWARD_CASES = [
+    ("decode", {}, "static"), ("decode", dict(T=1), "static"), ("decode", dict(T=32), "static"),
+    ("decode", dict(T=9, E=256), "h-static"),
+    ("tiny", dict(fmt="mxfp4", T=16, H=512, E=8, k=2, I=256), "none"),
+    ("tiny", dict(fmt="mxfp4", T=5, H=2304, E=64, k=4, I=512), "none"),
+]
+
+
+@pytest.mark.parametrize("name,over,scales", SMALL_FORWARD_CASES)
+def test_small_batch_forward_in_two_kernels(name, over, scales):
+    w = synth.workload(name, **over)
+    W, _ = oracle_bank(w)
+    a13, a2 = synth.static_act_scales()
+    if scales == "h-static":
+        a13 = None
+    elif scales == "none":
+        a13 = a2 = None
+    bank = device_bank(W, a13, a2)
+    x, wr, b = routed_inputs(w)
+    xd, wrd = bits_to_dev_bf16(x), bits_to_dev_bf16(wr)
+    bd = None if b is None else torch.from_numpy(b).cuda()
+    W_ = ws(ops.workspace_size(w.T, w.k, bank, None, 1))
+    outs, launches = [], []
+    try:
+        for opt in (0, 1):
+            ops.moe_set_option(ops.OPT_SMALL_BATCH_FORWARD, opt)
+            n0 = ops.moe_kernel_launch_count()
+            o = ops.moe_forward(xd, wrd, bd, w.k, bank, None, 1, W_)
+            launches.append(ops.moe_kernel_launch_count() - n0)
+            assert ops.moe_get_device_status(W_) == 0, opt
+            outs.append(dev_to_f64(o))
+    finally:
+        ops.moe_set_option(ops.OPT_SMALL_BATCH_FORWARD, 1)
+    assert launches[1] == (3 if a13 is None and w.fmt == "nvfp4" else 2), launches
+    assert max_abs_rel(outs[1], outs[0]) < 1e-2
+    r, keep = forward_reference(w, x, wr, b, W, act=1, a13=a13, a2=a2)
+    assert keep.all()
+    for o in outs:
+        assert max_abs_rel(o, r["out"]) < TOL
