@@ -418,7 +418,7 @@ moe_status moe_get_device_status(void* ws, moe_stream_t stream, int32_t* host_st
  *                     up with MOE_ERR_TIMEOUT (see the conventions above);
  *                     a small bound makes ordinary waits for memory run out,
  *                     which is how the timeout path is tested.
- *   MOE_OPT_FUSED_COMBINE: 1 (default) lets moe_forward, when its routed (and
+ *   MOE_OPT_FUSED_COMBINE: 1 lets moe_forward, when its routed (and
  *                     shared) experts run on the grouped tensor-core GEMM
  *                     (not the one-kernel FFN) and the weights are not BF16,
  *                     do the weighted combine in the down projection's
@@ -428,7 +428,8 @@ moe_status moe_get_device_status(void* ws, moe_stream_t stream, int32_t* host_st
  *                     order of the k additions then varies from run to run
  *                     (results within fp32 rounding of each other); 0 keeps
  *                     bf16 y_perm and the ordered combine of moe_combine,
- *                     which is bit-reproducible.
+ *                     which is bit-reproducible (the default: the reductions
+ *                     measured slower than the bf16 round trip).
  *   MOE_OPT_SMALL_BATCH_FORWARD: 1 (default) runs moe_forward at T <= 32 on
  *                     the one-kernel FFN (NVFP4 with a static h scale, or
  *                     MXFP4; H % 256 == 0; E <= 256) with no shared expert as
@@ -440,7 +441,17 @@ moe_status moe_get_device_status(void* ws, moe_stream_t stream, int32_t* host_st
  *                     and rounds them to bf16 in the CTA that finishes last.
  *                     The logits and routing are those of moe_route; the
  *                     order of the k additions varies from run to run.  0
- *                     keeps the permutation and the ordered combine. */
+ *                     keeps the permutation and the ordered combine.
+ *   MOE_OPT_GATHER_X:  1 (default) lets the one-kernel FFN of a batch of at
+ *                     most 32 tokens copy its token rows from a
+ *                     routing-independent layout of the quantised x; 0 keeps
+ *                     the quantised padded rows (and turns the two-kernel
+ *                     small-batch forward off).
+ *   MOE_OPT_FFN_SCHEDULE: 0 (default) the one-kernel FFN's CTAs take work
+ *                     items from a counter; 1 CTA b runs items b, b + grid,
+ *                     ... -- for measurement only: a down item may then wait
+ *                     on a CTA that is not resident (a concurrent kernel, MPS)
+ *                     until the wait bound runs out. */
 typedef enum {
   MOE_OPT_FFN_PATH = 1,
   MOE_OPT_GEMM_TILE_N = 2,
@@ -451,7 +462,9 @@ typedef enum {
   MOE_OPT_PERMUTE_QUANT = 7,
   MOE_OPT_WAIT_CYCLES = 8,
   MOE_OPT_FUSED_COMBINE = 9,
-  MOE_OPT_SMALL_BATCH_FORWARD = 10
+  MOE_OPT_SMALL_BATCH_FORWARD = 10,
+  MOE_OPT_GATHER_X = 11,
+  MOE_OPT_FFN_SCHEDULE = 12
 } moe_option;
 moe_status moe_set_option(int32_t option, int32_t value);
 

@@ -48,8 +48,10 @@ Scalars carve_head(Carver& c) {
 
 int g_ffn_path = 0;  // MOE_OPT_FFN_PATH
 static int g_fused_ffn = 1;  // MOE_OPT_FUSED_FFN
-static int g_fused_combine = 1;  // MOE_OPT_FUSED_COMBINE
+static int g_fused_combine = 0;  // MOE_OPT_FUSED_COMBINE
 static int g_small_forward = 1;  // MOE_OPT_SMALL_BATCH_FORWARD
+static int g_gather_x = 1;       // MOE_OPT_GATHER_X
+static int g_ffn_schedule = 0;   // MOE_OPT_FFN_SCHEDULE
 static int g_perm_quant = 1;  // MOE_OPT_PERMUTE_QUANT
 
 // Measurement hook (moe_set_stage_events).
@@ -378,8 +380,9 @@ void ffn_gemm_args(const moe_weights* w, const FfnScratch& f, int64_t S, float* 
 
 // Small batches whose x goes to the gather layout (the one-kernel FFN copies
 // its token rows from there, so no permutation is waited for).
-bool gather_x(const moe_weights* w, int64_t T) {
-  return T <= kGatherMaxT && (w->fmt == MOE_FMT_NVFP4 || w->fmt == MOE_FMT_MXFP4) && w->H % 256 == 0;
+bool gather_x(const moe_weights* w, int64_t T, int64_t S) {
+  return g_gather_x && T <= kGatherMaxT && S <= kGatherMaxS && (w->fmt == MOE_FMT_NVFP4 || w->fmt == MOE_FMT_MXFP4) &&
+         w->H % 256 == 0;
 }
 
 // x_ready: the permutation kernel has already quantised x into the padded
@@ -399,17 +402,16 @@ moe_status run_gemm_ffn(const uint16_t* x, int64_t T, int64_t S, const int32_t* 
   const bool fused_h = h_in_epilogue(w);
   const bool one_kernel = ffn_one_kernel(w, S);
   // small batches on the one-kernel FFN: x in the gather layout
-  const bool gather = one_kernel && !x_ready && gather_x(w, T);
+  const bool gather = one_kernel && !x_ready && gather_x(w, T, S);
   if (x_ready && (!one_kernel || !slot_expert || !planned)) return MOE_ERR_INVALID_ARG;
   if (out32 && one_kernel) return MOE_ERR_INVALID_ARG;
   if (out32 && topk_w && (!inv || fmt == MOE_FMT_BF16 || H % 64 != 0)) return MOE_ERR_INVALID_ARG;
   if (mark) stage_mark(MOE_STAGE_ACT_QUANT, false, s);
-  // the one-kernel FFN's counters are read before that kernel waits for the
-  // one before it, so they are cleared a step earlier (with x_ready, the
-  // forward cleared them before the router)
-  if (one_kernel && !x_ready) MOE_TRY(cudaMemsetAsync(f.counters, 0, counters_bytes(S, E), s));
+  // the x quantiser clears the one-kernel FFN's counters (with x_ready, the
+  // permutation kernel did)
+  const int ncounters = (int)(counters_bytes(S, E) / sizeof(int32_t));
   if (gather) {
-    GatherQuant gq{w->a13_gs, x_amax, f.xg, f.xsl};
+    GatherQuant gq{w->a13_gs, x_amax, f.xg, f.xsl, one_kernel ? f.counters : nullptr, one_kernel ? ncounters : 0};
     MOE_TRY(launch_quant_gather(fmt, x, T, H, gq, s));
   } else {
     QuantPaddedArgs qa;
@@ -446,6 +448,8 @@ moe_status run_gemm_ffn(const uint16_t* x, int64_t T, int64_t S, const int32_t* 
     qa.codes = f.xq;
     qa.sf = f.xsf;
     qa.status = status;
+    qa.zero = one_kernel ? f.counters : nullptr;
+    qa.nzero = one_kernel ? ncounters : 0;
     if (!x_ready) MOE_TRY(launch_quant_padded(qa, true, fmt, sms, s));
   }
   if (mark) stage_mark(MOE_STAGE_ACT_QUANT, true, s);
@@ -476,6 +480,7 @@ moe_status run_gemm_ffn(const uint16_t* x, int64_t T, int64_t S, const int32_t* 
     fa.P = f.P;
     fa.tile_done = f.tile_done;
     fa.work = f.work;
+    fa.static_items = g_ffn_schedule;
     fa.max_tiles = (int)max_tiles(S, E);
     if (gather) {
       fa.xg = f.xg;
@@ -733,6 +738,16 @@ moe_status moe_set_option(int32_t option, int32_t value) {
     set_early_weights(value);
     return MOE_OK;
   }
+  if (option == MOE_OPT_GATHER_X) {
+    if (value != 0 && value != 1) return MOE_ERR_INVALID_ARG;
+    g_gather_x = value;
+    return MOE_OK;
+  }
+  if (option == MOE_OPT_FFN_SCHEDULE) {
+    if (value != 0 && value != 1) return MOE_ERR_INVALID_ARG;
+    g_ffn_schedule = value;
+    return MOE_OK;
+  }
   if (option == MOE_OPT_SMALL_BATCH_FORWARD) {
     if (value != 0 && value != 1) return MOE_ERR_INVALID_ARG;
     g_small_forward = value;
@@ -977,7 +992,7 @@ moe_status moe_forward(const uint16_t* x, int64_t T, const uint16_t* wr, const f
   // adds w * y into fp32 output rows in its down epilogue, and its last CTA
   // rounds them into `out`.
   const bool small2 = g_small_forward && !shared && act == MOE_ACT_MATCH && use_gemm_path(routed, S, act) &&
-                      ffn_one_kernel(routed, S) && gather_x(routed, T) && H % 8 == 0;
+                      ffn_one_kernel(routed, S) && gather_x(routed, T, S) && H % 8 == 0;
   if (small2) {
     MOE_TRY(cudaMemsetAsync(f.ffn.counters, 0, counters_bytes(S, E), s));
     MOE_TRY(cudaMemsetAsync(f.out32, 0, sizeof(float) * (size_t)T * H, s));
@@ -1005,6 +1020,7 @@ moe_status moe_forward(const uint16_t* x, int64_t T, const uint16_t* wr, const f
     fa.P = f.ffn.P;
     fa.tile_done = f.ffn.tile_done;
     fa.work = f.ffn.work;
+    fa.static_items = g_ffn_schedule;
     fa.max_tiles = (int)max_tiles(S, E);
     fa.xg = f.ffn.xg;
     fa.xsl = f.ffn.xsl;
@@ -1025,7 +1041,6 @@ moe_status moe_forward(const uint16_t* x, int64_t T, const uint16_t* wr, const f
   // runs.  The FFN's item counter is cleared here, before the router.
   const bool want_q = g_perm_quant && act == MOE_ACT_MATCH && use_gemm_path(routed, S, act) &&
                       ffn_one_kernel(routed, S) && H % 64 == 0 && permute_can_quantize(S, T, E);
-  if (want_q) MOE_TRY(cudaMemsetAsync(f.ffn.counters, 0, counters_bytes(S, E), s));
   // The weighted combine in the down epilogues (routed and shared experts
   // add into fp32 rows, cleared here, before the fork), then one rounding pass.
   const bool fused_combine = combine_in_down(routed, shared, T, k, act);
@@ -1088,6 +1103,8 @@ moe_status moe_forward(const uint16_t* x, int64_t T, const uint16_t* wr, const f
     q.amax = f.head.x_amax;
     q.codes = f.ffn.xq;
     q.sf = f.ffn.xsf;
+    q.zero = f.ffn.counters;   // the one-kernel FFN's counters, cleared on the way
+    q.nzero = (int)(counters_bytes(S, E) / sizeof(int32_t));
   }
   bool planned = false, x_ready = false;
   if (st == MOE_OK) {

@@ -939,34 +939,11 @@ struct FusedCfg {
   static constexpr int kQ = 32;
   static_assert(kQ >= 2 * C::kStages + C::kAccStages + 2, "item queue");
   // + the down store staging, the item queue, the expert counts (+ a flag),
-  // 32 ints per warp for gathering a tile's slots
+  // the slot or token of every slot position of a gathering batch
   static constexpr int kSmem =
-      C::kSmem + C::kEpiWarps * 1024 + kQ * (8 + 8 + 4) + (kFusedMaxE + 1) * 4 + (2 + C::kEpiWarps) * 32 * 4;
+      C::kSmem + C::kEpiWarps * 1024 + kQ * (8 + 8 + 4) + (kFusedMaxE + 1) * 4 + kGatherMaxS * 2;
   static_assert(kSmem <= 227 * 1024, "shared memory");
 };
-
-// Lane r (< n <= 32) receives the flat index of the (first + r)-th slot
-// routed to expert e (slots in increasing order), -1 in the other lanes; a
-// whole warp calls it, `stash` is 32 ints of the warp's own shared memory.
-__device__ __forceinline__ int tile_slot_of_lane(const int32_t* __restrict__ slot_expert, int64_t S, int e,
-                                                 int first, int n, int* stash) {
-  const int lane = threadIdx.x & 31;
-  int seen = 0;
-  for (int64_t base = 0; base < S && seen < first + n; base += 32) {
-    const int64_t i = base + lane;
-    const bool hit = i < S && __ldcg(slot_expert + i) == e;
-    const unsigned m = __ballot_sync(0xffffffffu, hit);
-    if (hit) {
-      const int r = seen + __popc(m & ((1u << lane) - 1u)) - first;
-      if (r >= 0 && r < n) stash[r] = (int)i;
-    }
-    seen += __popc(m);
-  }
-  __syncwarp();
-  const int sl = lane < n ? stash[lane] : -1;
-  __syncwarp();
-  return sl;
-}
 
 template <int FMT, int BN, bool GATHER>
 __global__ void __launch_bounds__(Cfg<FMT, kEpiUpQuant, BN, false>::kThreads, 1)
@@ -1002,7 +979,9 @@ __global__ void __launch_bounds__(Cfg<FMT, kEpiUpQuant, BN, false>::kThreads, 1)
   uint64_t* q_free = q_full + kQ;
   volatile int32_t* q_id = reinterpret_cast<volatile int32_t*>(q_free + kQ);
   int32_t* hist = const_cast<int32_t*>(q_id) + kQ;  // [kFusedMaxE] counts, bad flag
-  int* stash = hist + kFusedMaxE + 1 + (threadIdx.x >> 5) * 32;   // this warp's 32 ints
+  // gather mode: the slot (forward) or token (grouped FFN) of every slot
+  // position, experts in order, slots in flat order within an expert
+  uint16_t* s_slot = reinterpret_cast<uint16_t*>(hist + kFusedMaxE + 1);
   // gather mode on the forward: the slots' experts come from the previous
   // kernel (the router), so everything waits for it
   const bool ids_from_prev = GATHER && f.slot_expert != nullptr;
@@ -1058,6 +1037,50 @@ __global__ void __launch_bounds__(Cfg<FMT, kEpiUpQuant, BN, false>::kThreads, 1)
       }
     }
     if (__any_sync(0xffffffffu, bad) && lane == 0) hist[kFusedMaxE] = 1;
+    if (GATHER) {
+      // the slots in expert-major order (a counting sort, stable in the flat
+      // index): lane l holds the counts of experts 8l .. 8l + 7, turns them
+      // into the exclusive prefix as cursors, places every slot, and puts
+      // the counts back for the tile list
+      __syncwarp();
+      int cnt[8], run = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        cnt[j] = 8 * lane + j < kFusedMaxE ? hist[8 * lane + j] : 0;
+        run += cnt[j];
+      }
+      int incl = run;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int a = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += a;
+      }
+      int cur = incl - run;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (8 * lane + j < kFusedMaxE) hist[8 * lane + j] = cur;
+        cur += cnt[j];
+      }
+      __syncwarp();
+      for (int64_t base = 0; base < f.S && f.S <= kGatherMaxS; base += 32) {
+        const int64_t i = base + lane;
+        int e = i < f.S ? __ldcg(f.slot_expert + i) : -1;
+        if (e >= g1.E) e = -1;
+        const unsigned peers = __match_any_sync(0xffffffffu, e);
+        const int pos = e >= 0 ? hist[e] + __popc(peers & ((1u << lane) - 1u)) : -1;
+        __syncwarp();
+        if (e >= 0) s_slot[pos] = (uint16_t)i;
+        if (e >= 0 && lane == __ffs(peers) - 1) hist[e] += __popc(peers);
+        __syncwarp();
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (8 * lane + j < kFusedMaxE) hist[8 * lane + j] = cnt[j];
+    }
+  }
+  if (GATHER && warp == 0 && f.perm_token) {
+    // the grouped FFN gives the token of every position (an input of the call)
+    for (int64_t p = lane; p < f.S && f.S <= kGatherMaxS; p += 32) s_slot[p] = (uint16_t)__ldg(f.perm_token + p);
   }
   if (warp == 1) {
     tc::tmem_alloc(tmem_slot, C::kTmemCols);
@@ -1096,8 +1119,9 @@ __global__ void __launch_bounds__(Cfg<FMT, kEpiUpQuant, BN, false>::kThreads, 1)
     // ------------------------------------------------------------ producer
     // Items are taken one ahead: lane 0 holds the counter's answer for the
     // next item while the current one's weights go out.
-    int pending = 0;
-    if (lane == 0) pending = atomicAdd(f.work, 1);
+    int pending = 0, n_taken = 0;
+    const bool dyn = !f.static_items;
+    if (lane == 0 && !dyn) pending = (int)blockIdx.x;
     int pushed = 0;          // queue entries written (items, then the end mark)
     bool ended = false;      // the end mark is in the queue
     // weight cursor: item, stage within it, stage sequence number (ring slot
@@ -1120,8 +1144,9 @@ __global__ void __launch_bounds__(Cfg<FMT, kEpiUpQuant, BN, false>::kThreads, 1)
       if (__shfl_sync(0xffffffffu, (int)tc::mbar_test_wait(&q_free[j], par), 0) == 0) return false;
       int id = __shfl_sync(0xffffffffu, pending, 0);
       id = id < total ? id : -1;
+      ++n_taken;
       if (lane == 0) {
-        if (id >= 0) pending = atomicAdd(f.work, 1);
+        if (id >= 0) pending = f.static_items ? (int)blockIdx.x + n_taken * (int)gridDim.x : atomicAdd(f.work, 1);
         q_id[j] = id;
         tc::mbar_arrive(&q_full[j]);
       }
@@ -1157,11 +1182,32 @@ __global__ void __launch_bounds__(Cfg<FMT, kEpiUpQuant, BN, false>::kThreads, 1)
     // ring's first pass needs no free slot): a deeper burst queues that
     // kernel's own reads behind it.
     constexpr int kPreStages = 3 < C::kStages ? 3 : C::kStages;
-    take_next();
-    if (g1.w_early != 0)
-      while (a_valid && seq_a < kPreStages) issue_a();
+    if (!dyn) {
+      take_next();
+      if (g1.w_early != 0)
+        while (a_valid && seq_a < kPreStages) issue_a();
+    } else if (g1.w_early != 0 && (int)blockIdx.x < total) {
+      // The counter is cleared by the kernel before this one, so items are
+      // taken after the wait.  The first items go to the first CTAs to get
+      // there, one each: CTA b prefetches item b's first stages into L2 for
+      // whichever CTA takes it.
+      bool up = false;
+      int tt = 0, mt = 0;
+      decode((int)blockIdx.x, up, tt, mt);
+      const int e = plan.at(tt, BN).e;
+      const int R = up ? g1.R : g2.R, nc = up ? ncols1 : ncols2, nkb = up ? nkb1 : nkb2;
+      const uint8_t* sfa = (up ? g1.w_sf : g2.w_sf) + (size_t)e * R * nc + (size_t)mt * (nc / 4) * 512;
+      if (tc::elect_one()) {
+        for (int kb = 0; kb < kPreStages && kb < nkb; ++kb) {
+          tc::tma_prefetch_2d(up ? &tmap_w13 : &tmap_w2, kb * 128, e * R + mt * 128);
+          tc::bulk_prefetch_l2(sfa + (size_t)kb * F::kGroups * 512, C::kSFA);
+        }
+      }
+      __syncwarp();
+    }
     pdl_wait();
     pdl_trigger();
+    if (dyn && lane == 0) pending = atomicAdd(f.work, 1);
     long long t_prog = clock64();
     while (true) {
       bool prog = false;
@@ -1180,12 +1226,8 @@ __global__ void __launch_bounds__(Cfg<FMT, kEpiUpQuant, BN, false>::kThreads, 1)
             // repeat a token, which the rows past 32 do not get)
             const int n = min(b_te.nvalid, kGatherMaxT);
             if (b_te.nvalid > kGatherMaxT && lane == 0) raise_status(g1.status, MOE_ERR_DEVICE_FAULT);
-            if (f.perm_token) {
-              b_tok = lane < n ? __ldg(f.perm_token + b_te.p0 + lane) : -1;
-            } else {
-              const int sl = tile_slot_of_lane(f.slot_expert, f.S, b_te.e, 0, n, stash);
-              b_tok = sl >= 0 ? sl / f.k : -1;
-            }
+            const int v = lane < n && b_te.p0 + lane < f.S ? (int)s_slot[b_te.p0 + lane] : -1;
+            b_tok = v < 0 ? -1 : (f.perm_token ? v : v / f.k);
             if (b_tok >= f.T) b_tok = -1;
           }
         }
@@ -1428,7 +1470,8 @@ __global__ void __launch_bounds__(Cfg<FMT, kEpiUpQuant, BN, false>::kThreads, 1)
       int ltok = -1;
       float lw = 0.0f;
       if (GATHER && !up && g2.out32 && f.slot_expert) {
-        const int sl = tile_slot_of_lane(f.slot_expert, f.S, te.e, 0, min(te.nvalid, kGatherMaxT), stash);
+        const int n = min(te.nvalid, kGatherMaxT);
+        const int sl = lane < n && te.p0 + lane < f.S ? (int)s_slot[te.p0 + lane] : -1;
         ltok = sl >= 0 ? sl / f.k : -1;
         lw = sl >= 0 ? __ldg(f.topk_w + sl) : 0.0f;
       }
@@ -1683,7 +1726,7 @@ cudaError_t launch_fused_ffn(const GemmArgs& g1, const GemmArgs& g2, const Fused
   if (g1.E > kFusedMaxE || g1.fmt != g2.fmt) return cudaErrorInvalidValue;
   // gather mode: a tile holds at most kGatherMaxT rows (T <= kGatherMaxT),
   // and its tokens come from perm_token or from the slots' experts
-  if (f.xg && (f.T > kGatherMaxT || !f.xsl || (!f.perm_token && !f.slot_expert) || f.k < 1))
+  if (f.xg && (f.T > kGatherMaxT || f.S > kGatherMaxS || !f.xsl || (!f.perm_token && !f.slot_expert) || f.k < 1))
     return cudaErrorInvalidValue;
   if (f.out && (!f.xg || !f.slot_expert || !g2.out32 || !f.done || !f.topk_w)) return cudaErrorInvalidValue;
   switch (g1.fmt) {
@@ -2018,6 +2061,8 @@ __global__ void __launch_bounds__(256) quant_gather_kernel(const uint16_t* __res
   const float scale = act_scale_of(FMT, q.scale, q.amax);
   if (FMT == MOE_FMT_NVFP4 && threadIdx.x < 128) r_tab[threadIdx.x] = nvfp4_multiplier(threadIdx.x, scale);
   __syncthreads();
+  if (q.zero && blockIdx.x == 0)
+    for (int i = threadIdx.x; i < q.nzero; i += blockDim.x) q.zero[i] = 0;
   const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (t < T)
     quant_token_gather<FMT>(x + t * K, K, scale, r_tab, q.xg + t * 8 * (K / 2), q.xsl + t * (K / (4 * bs)) * 16);

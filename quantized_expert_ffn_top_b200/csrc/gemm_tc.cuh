@@ -104,6 +104,8 @@ struct FusedArgs {
   int32_t* tile_done;          // [max_tiles], zero on entry
   int32_t* work;               // item counter, zero on entry and set at least two launches before
                                // this kernel (it is read before the wait on the previous one)
+  int static_items;            // 1: CTA b runs items b, b + grid, ... instead (for A/B measurement:
+                               // it assumes every CTA is resident at once)
   int max_tiles;
   // Gather mode (small batches, at most kGatherMaxT slots per expert): the
   // gate|up token operand is copied row by row from the gather layout of x

@@ -62,11 +62,16 @@ cudaError_t launch_quantize(int fmt, const void* x, int x_dtype, int64_t rows, i
 // Tokens a gathering batch may hold: a tile's scale lines serve rows below 32,
 // and a token picks an expert at most once.
 constexpr int kGatherMaxT = 32;
+// Slots a gathering batch may hold: the one-kernel FFN keeps the token of
+// every slot position in shared memory.
+constexpr int kGatherMaxS = 256;
 struct GatherQuant {
   const float* scale;
   const float* amax;
   uint8_t* xg;
   uint8_t* xsl;
+  int32_t* zero;   // optional: nzero counters set to 0 (by block 0, after the wait)
+  int nzero;
 };
 
 // route.cu

@@ -30,6 +30,8 @@ OPT_PERMUTE_QUANT = 7
 OPT_WAIT_CYCLES = 8
 OPT_FUSED_COMBINE = 9
 OPT_SMALL_BATCH_FORWARD = 10
+OPT_GATHER_X = 11
+OPT_FFN_SCHEDULE = 12
 FMT_BY_NAME = {"nvfp4": FMT_NVFP4, "mxfp4": FMT_MXFP4, "fp8": FMT_FP8, "bf16": FMT_BF16}
 
 

@@ -446,7 +446,7 @@ def test_combine_in_down_epilogue_matches_ordered_combine(name, over, static):
             assert ops.moe_get_device_status(W_) == 0, fused
             outs.append(dev_to_f64(o))
     finally:
-        ops.moe_set_option(ops.OPT_FUSED_COMBINE, 1)
+        ops.moe_set_option(ops.OPT_FUSED_COMBINE, 0)   # the default
     # apart by the bf16 rounding of y_perm and of each output (a few bf16
     # ulps of the largest output), half the layer tolerance at most
     assert max_abs_rel(outs[1], outs[0]) < 1e-2

@@ -44,7 +44,7 @@ def test_wait_that_runs_out_sets_timeout_and_the_next_call_is_clean(name, base, 
     bd = None if b is None else torch.from_numpy(b).cuda()
     ws = ops.new_workspace(ops.workspace_size(w.T, w.k, bank, None, ops.ACT_MATCH))
     try:
-        ops.moe_set_option(ops.OPT_FUSED_COMBINE, 0)   # the ordered combine: bit-reproducible runs
+        ops.moe_set_option(ops.OPT_FUSED_COMBINE, 0)   # the ordered combine (the default): bit-reproducible
         ref = ops.moe_forward(xd, wrd, bd, w.k, bank, None, ops.ACT_MATCH, ws)
         assert ops.moe_get_device_status(ws) == 0
         try:
@@ -59,5 +59,5 @@ def test_wait_that_runs_out_sets_timeout_and_the_next_call_is_clean(name, base, 
         out = ops.moe_forward(xd, wrd, bd, w.k, bank, None, ops.ACT_MATCH, ws)
         assert ops.moe_get_device_status(ws) == 0
     finally:
-        ops.moe_set_option(ops.OPT_FUSED_COMBINE, 1)
+        ops.moe_set_option(ops.OPT_FUSED_COMBINE, 0)   # the default
     assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
