@@ -207,9 +207,12 @@ moe_status moe_quantize(int32_t fmt, const void* x, int32_t x_dtype, int64_t row
  *    group's sum being partial 32g; the 8 group sums are added in order onto
  *    0, then the bias (or 0).  A CPU replay of this order reproduces the
  *    logits, and so the routing, bit for bit.
- *  - T >= 128, E % 128 == 0, H % 64 == 0: the bf16 tensor cores (tcgen05),
- *    with fp32 accumulation in their own order, H split in up to 4 parts
- *    added in order.
+ *  - T >= 128, H % 64 == 0 and either (a) ceil(T / 128) >= SMs / 2,
+ *    E % 16 == 0, 16 <= E <= 256, k <= 16 (one kernel: all of H accumulated
+ *    in one tensor-memory accumulator, the top k picked in its epilogue;
+ *    MOE_OPT_ROUTER_TOPK) or (b) E % 128 == 0 (H split in up to 4 parts
+ *    added in order, then the top-k kernel): the bf16 tensor cores
+ *    (tcgen05), fp32 accumulation in their own order.
  *  - otherwise: one sequential sum over h = 0 .. H-1, then the bias (or 0). */
 moe_status moe_route(const uint16_t* x, int64_t T, int32_t H, const uint16_t* wr, const float* bias, int32_t E,
                      int32_t k, float* logits, int32_t* topk_idx, float* topk_w, void* ws, size_t ws_bytes,
@@ -430,7 +433,7 @@ moe_status moe_get_device_status(void* ws, moe_stream_t stream, int32_t* host_st
  *                     bf16 y_perm and the ordered combine of moe_combine,
  *                     which is bit-reproducible (the default: the reductions
  *                     measured slower than the bf16 round trip).
- *   MOE_OPT_SMALL_BATCH_FORWARD: 1 (default) runs moe_forward at T <= 32 on
+ *   MOE_OPT_SMALL_BATCH_FORWARD: 1 runs moe_forward at T <= 32 on
  *                     the one-kernel FFN (NVFP4 with a static h scale, or
  *                     MXFP4; H % 256 == 0; E <= 256) with no shared expert as
  *                     two kernels: the router (logits, x quantised into a
@@ -441,12 +444,18 @@ moe_status moe_get_device_status(void* ws, moe_stream_t stream, int32_t* host_st
  *                     and rounds them to bf16 in the CTA that finishes last.
  *                     The logits and routing are those of moe_route; the
  *                     order of the k additions varies from run to run.  0
- *                     keeps the permutation and the ordered combine.
- *   MOE_OPT_GATHER_X:  1 (default) lets the one-kernel FFN of a batch of at
- *                     most 32 tokens copy its token rows from a
- *                     routing-independent layout of the quantised x; 0 keeps
- *                     the quantised padded rows (and turns the two-kernel
- *                     small-batch forward off).
+ *                     (default: measured slower than the permutation and
+ *                     the ordered combine) keeps those.
+ *   MOE_OPT_GATHER_X:  1 lets the one-kernel FFN of a batch of at most 32
+ *                     tokens copy its token rows from a routing-independent
+ *                     layout of the quantised x; 0 (default: measured
+ *                     faster) keeps the quantised padded rows (and turns the
+ *                     two-kernel small-batch forward off).
+ *   MOE_OPT_ROUTER_TOPK: 1 (default) computes the logits and the top k in
+ *                     one tensor-core kernel when the batch's 128-token tiles
+ *                     number at least half the SMs, E % 16 == 0,
+ *                     16 <= E <= 256, H % 64 == 0 and k <= 16; 0 keeps the
+ *                     logits kernel and the separate top-k kernel.
  *   MOE_OPT_FFN_SCHEDULE: 0 (default) the one-kernel FFN's CTAs take work
  *                     items from a counter; 1 CTA b runs items b, b + grid,
  *                     ... -- for measurement only: a down item may then wait
@@ -464,7 +473,8 @@ typedef enum {
   MOE_OPT_FUSED_COMBINE = 9,
   MOE_OPT_SMALL_BATCH_FORWARD = 10,
   MOE_OPT_GATHER_X = 11,
-  MOE_OPT_FFN_SCHEDULE = 12
+  MOE_OPT_FFN_SCHEDULE = 12,
+  MOE_OPT_ROUTER_TOPK = 13
 } moe_option;
 moe_status moe_set_option(int32_t option, int32_t value);
 

@@ -49,8 +49,9 @@ Scalars carve_head(Carver& c) {
 int g_ffn_path = 0;  // MOE_OPT_FFN_PATH
 static int g_fused_ffn = 1;  // MOE_OPT_FUSED_FFN
 static int g_fused_combine = 0;  // MOE_OPT_FUSED_COMBINE
-static int g_small_forward = 1;  // MOE_OPT_SMALL_BATCH_FORWARD
-static int g_gather_x = 1;       // MOE_OPT_GATHER_X
+static int g_small_forward = 0;  // MOE_OPT_SMALL_BATCH_FORWARD
+static int g_gather_x = 0;       // MOE_OPT_GATHER_X
+static int g_router_topk = 1;    // MOE_OPT_ROUTER_TOPK
 static int g_ffn_schedule = 0;   // MOE_OPT_FFN_SCHEDULE
 static int g_perm_quant = 1;  // MOE_OPT_PERMUTE_QUANT
 
@@ -278,6 +279,22 @@ cudaError_t run_router(const uint16_t* x, int64_t T, int H, const uint16_t* wr, 
   }
   *nparts = 1;
   return launch_router_logits(x, T, H, wr, bias, E, parts, s);
+}
+
+// Logits and every token's top k.  Batches whose 128-token tiles fill at
+// least half the SMs and whose E fits one MMA (E a multiple of 16 up to 256,
+// k <= 16) take one kernel: the tensor cores with the top-k in their
+// epilogue.  Otherwise the logits go to `parts` (the
+// router GEMM's partial sums, or the CUDA-core sums) and topk_kernel picks.
+// logits_out (nullable) receives the summed logits either way.
+cudaError_t route_tokens(const uint16_t* x, int64_t T, int H, const uint16_t* wr, const float* bias, int E, int k,
+                         float* parts, float* logits_out, int32_t* idx, float* w, int32_t* status, cudaStream_t s) {
+  if (g_router_topk && router_topk_fits(T, E, H, k, num_sms()))
+    return launch_router_topk(x, T, H, wr, bias, E, k, logits_out, idx, w, status, num_sms(), s);
+  int nparts = 1;
+  const cudaError_t e = run_router(x, T, H, wr, bias, E, parts, &nparts, status, s);
+  if (e != cudaSuccess) return e;
+  return launch_topk(parts, nparts, T * (int64_t)E, logits_out, T, E, k, idx, w, status, s);
 }
 
 bool gemm_shapes_ok(const moe_weights* w, int act) {
@@ -743,6 +760,11 @@ moe_status moe_set_option(int32_t option, int32_t value) {
     g_gather_x = value;
     return MOE_OK;
   }
+  if (option == MOE_OPT_ROUTER_TOPK) {
+    if (value != 0 && value != 1) return MOE_ERR_INVALID_ARG;
+    g_router_topk = value;
+    return MOE_OK;
+  }
   if (option == MOE_OPT_FFN_SCHEDULE) {
     if (value != 0 && value != 1) return MOE_ERR_INVALID_ARG;
     g_ffn_schedule = value;
@@ -899,10 +921,7 @@ moe_status moe_route(const uint16_t* x, int64_t T, int32_t H, const uint16_t* wr
   if (!ws || ws_bytes < c.off) return MOE_ERR_WORKSPACE;
   if (T == 0) return MOE_OK;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  int nparts = 1;
-  MOE_TRY(run_router(x, T, H, wr, bias, E, r.parts, &nparts, r.head.status, s));
-  return cuda_status(
-      launch_topk(r.parts, nparts, T * (int64_t)E, logits, T, E, k, topk_idx, topk_w, r.head.status, s));
+  return cuda_status(route_tokens(x, T, H, wr, bias, E, k, r.parts, logits, topk_idx, topk_w, r.head.status, s));
 }
 
 moe_status moe_route_logits(const float* logits, int64_t T, int32_t E, int32_t k, int32_t* topk_idx, float* topk_w,
@@ -1080,10 +1099,7 @@ moe_status moe_forward(const uint16_t* x, int64_t T, const uint16_t* wr, const f
   }
   // 3. router
   stage_mark(MOE_STAGE_ROUTE, false, s);
-  int nparts = 1;
-  st = cuda_status(run_router(x, T, H, wr, bias, E, f.logits, &nparts, f.head.status, s));
-  if (st == MOE_OK)
-    st = cuda_status(launch_topk(f.logits, nparts, T * (int64_t)E, nullptr, T, E, k, f.idx, f.w, f.head.status, s));
+  st = cuda_status(route_tokens(x, T, H, wr, bias, E, k, f.logits, nullptr, f.idx, f.w, f.head.status, s));
   stage_mark(MOE_STAGE_ROUTE, true, s);
   // 4. histogram + permutation; it also writes the routed FFN's tile plan
   PlanOut plan;
@@ -1298,9 +1314,7 @@ moe_status moe_forward_cached(const uint16_t* x, int64_t T, const uint16_t* wr, 
   if (dynamic_x_scale(pool, act)) MOE_TRY(launch_amax(x, 1, T * H, f.head.x_amax, num_sms(), s));
   // route on the whole bank's router
   stage_mark(MOE_STAGE_ROUTE, false, s);
-  int nparts = 1;
-  MOE_TRY(run_router(x, T, H, wr, bias, E, f.logits, &nparts, f.head.status, s));
-  MOE_TRY(launch_topk(f.logits, nparts, T * (int64_t)E, nullptr, T, E, k, f.idx, f.w, f.head.status, s));
+  MOE_TRY(route_tokens(x, T, H, wr, bias, E, k, f.logits, nullptr, f.idx, f.w, f.head.status, s));
   stage_mark(MOE_STAGE_ROUTE, true, s);
   // admit the batch's experts into slots and fetch the missing ones
   MOE_TRY(launch_cache_admit(f.idx, S, E, n, cache->state, f.idx_slot, f.head.status, s));

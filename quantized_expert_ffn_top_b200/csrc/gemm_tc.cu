@@ -39,6 +39,7 @@
 #include "gemm_tc.cuh"
 #include "tc_ptx.cuh"
 #include "token_quant.cuh"
+#include "topk_warp.cuh"
 
 namespace moe {
 namespace {
@@ -344,10 +345,10 @@ __device__ __forceinline__ void epilogue_slice(const GemmArgs& g, const CUtensor
       const float sc = (FMT == MOE_FMT_MXFP4 || FMT == kFmtBF16) ? 1.0f : __ldg(g.w_gs + te.e) * gact;
       if (g.out32) {
         // the weighted un-permute in the epilogue: lanes 0..15 fetch the
-        // chunk's tokens and routing weights, every lane adds w * y for its
-        // output row (32 consecutive floats per warp and token: one L2
-        // reduction transaction)
-        const int o = mt * 128 + q * 32 + lane;
+        // chunk's tokens and routing weights; the warp's [tokens][32
+        // outputs] block passes through its staging buffer (ybufs KB, 8
+        // tokens per KB) so that each lane then adds 4 consecutive outputs
+        // of one token with one vector reduction
         int tk = -1;
         float wt = 0.0f;
         if (!g.perm_token) {
@@ -367,11 +368,26 @@ __device__ __forceinline__ void epilogue_slice(const GemmArgs& g, const CUtensor
           raise_status(g.status, MOE_ERR_DEVICE_FAULT);
           tk = -1;
         }
+        float* sb = reinterpret_cast<float*>(y_stage) + ew * ybufs * 256;
+        float* orow = g.out32 + mt * 128 + q * 32 + 4 * (lane & 7);
+        const int nb = ybufs >= 2 ? 16 : 8;   // tokens per pass
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const int t = __shfl_sync(0xffffffffu, tk, c);
-          const float ww = __shfl_sync(0xffffffffu, wt, c);
-          if (t >= 0) atomicAdd(g.out32 + (size_t)t * g.ldy + o, ww * (v[c] * sc));
+        for (int h = 0; h < 16; h += 8) {
+          if (h > 0 && nb == 16) break;     // one pass took all 16
+          __syncwarp();                     // the previous pass has read the buffer
+#pragma unroll
+          for (int c = 0; c < 16; ++c)
+            if (c >= h && c < h + nb) sb[(c - h) * 32 + lane] = v[c] * sc;
+          __syncwarp();
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            if (4 * i >= nb) break;                // uniform: lanes read tokens lane / 8 + 4i
+            const int cc = (lane >> 3) + 4 * i;   // token of this read, within the pass
+            const int t = __shfl_sync(0xffffffffu, tk, h + cc);
+            const float ww = __shfl_sync(0xffffffffu, wt, h + cc);
+            const float4 y4 = *reinterpret_cast<const float4*>(sb + cc * 32 + 4 * (lane & 7));
+            if (t >= 0) tc::red_add_v4(orow + (size_t)t * g.ldy, ww * y4.x, ww * y4.y, ww * y4.z, ww * y4.w);
+          }
         }
         continue;
       }
@@ -1134,7 +1150,11 @@ __global__ void __launch_bounds__(Cfg<FMT, kEpiUpQuant, BN, false>::kThreads, 1)
     int b_tt = 0, b_mt = 0;
     TileEntry b_te{};
     int b_tok = -1;    // gather mode: lane r (< nvalid) holds the token of tile row r
-    uint32_t rdy = 0;  // bit i: the token operand of the item at queue position b_pos + i is ready
+    // token tiles whose gate|up slices are all stored: bit i of rdy is token
+    // tile rdy_base + i (down items are taken in increasing token-tile order,
+    // so one poll of 32 tiles ahead covers the next down items)
+    uint32_t rdy = 0;
+    int rdy_base = 0;
     // Moves the weight cursor to a newly taken item and queues it; false
     // when the queue has no room right now.
     auto take_next = [&]() -> bool {
@@ -1219,7 +1239,8 @@ __global__ void __launch_bounds__(Cfg<FMT, kEpiUpQuant, BN, false>::kThreads, 1)
           decode(id, b_up, b_tt, b_mt);
           b_te = plan.at(b_tt, BN);
           b_have = true;
-          b_ready = b_up || (rdy & 1u) != 0;   // gate|up token tiles come from the x quantiser before this kernel
+          // gate|up token tiles come from the x quantiser before this kernel
+          b_ready = b_up || (b_tt >= rdy_base && b_tt < rdy_base + 32 && ((rdy >> (b_tt - rdy_base)) & 1u));
           if (GATHER && b_up) {
             // the tile's rows are its expert's slots in flat order (one tile
             // per expert: at most kGatherMaxT slots; more means slots that
@@ -1232,17 +1253,15 @@ __global__ void __launch_bounds__(Cfg<FMT, kEpiUpQuant, BN, false>::kThreads, 1)
           }
         }
         if (!b_ready) {
-          // one round trip polls the token tiles of this and the next 31 queued items
-          int v = 0;
-          if (b_pos + lane < pushed) {
-            const int id = q_id[(b_pos + lane) % kQ];
-            bool up_i = true;
-            int tt_i = 0, mt_i = 0;
-            if (id >= 0) decode(id, up_i, tt_i, mt_i);
-            v = (id >= 0 && !up_i) ? tc::ld_acquire_gpu(f.tile_done + tt_i) : done_target;
+          // one round trip polls this token tile and the next 31
+          if (b_tt < rdy_base || b_tt >= rdy_base + 32) {
+            rdy = 0;
+            rdy_base = b_tt;
           }
+          const int tt_i = rdy_base + lane;
+          const int v = tt_i < ntok ? tc::ld_acquire_gpu(f.tile_done + tt_i) : 0;
           rdy |= __ballot_sync(0xffffffffu, v >= done_target);
-          if (!(rdy & 1u)) break;
+          if (!((rdy >> (b_tt - rdy_base)) & 1u)) break;
           tc::fence_proxy_async_global();   // for every token tile seen ready here
           b_ready = true;
         }
@@ -1282,7 +1301,6 @@ __global__ void __launch_bounds__(Cfg<FMT, kEpiUpQuant, BN, false>::kThreads, 1)
           kbb = 0;
           ++b_pos;
           b_have = false;
-          rdy >>= 1;
         }
         prog = true;
       }
@@ -1707,6 +1725,251 @@ cudaError_t launch_fused_cfg(const GemmArgs& g1, const GemmArgs& g2, const Fused
   return cudaGetLastError();
 }
 
+// ------------------------------------------------------ router with top-k --
+// Router logits and the top-k of every token in one kernel for batches large
+// enough that the 128-token tiles fill the SMs: 128 tokens of x on the MMA's
+// M side, all E experts of Wr on its N side (bf16 kind::f16, fp32
+// accumulation over all of H, E a multiple of 16 up to 256), so each
+// accumulator lane holds one token's E logits.  The epilogue thread of lane
+// t reads its row from tensor memory 16 columns at a time, adds the bias and
+// keeps the k largest (descending, ties to the lower expert) in registers,
+// while the other accumulator buffer takes the next tile's MMAs; the weights
+// are exp(L_j - L_0) / sum over the k picks.  Smaller batches take the
+// router GEMM split along H and the top-k kernel: with fewer tiles than SMs
+// one CTA per tile streams its operands too slowly, and a cluster sharing
+// each tile (partials exchanged through distributed shared memory) measured
+// slower than the two kernels.
+constexpr int kRouteTopkMaxK = 16;   // k beyond this takes the router GEMM and topk_kernel
+constexpr int kRouteStages = 4;
+
+template <int NE>
+struct RouteTopkCfg {
+  static constexpr int kA = 128 * 128;   // 128 token rows x 64 bf16
+  static constexpr int kB = NE * 128;    // NE expert rows x 64 bf16
+  static constexpr int kStage = (kA + kB + 1023) / 1024 * 1024;
+  static constexpr int kSmem = kRouteStages * kStage + 1024 /*align*/ + 1024 /*barriers*/;
+  static constexpr int kThreads = 6 * 32;   // producer, MMA, 4 epilogue warps
+  static_assert(kSmem <= 227 * 1024, "shared memory");
+  static_assert(2 * NE <= 512, "two accumulators in tensor memory");
+};
+
+// Keeps tv/te (descending, an empty slot holding index -1) as the KMAX
+// largest of the logits seen, offered in increasing expert order: only a
+// strictly larger logit moves ahead, so an equal one stays behind the lower
+// expert index; an empty slot takes anything.
+template <int KMAX>
+__device__ __forceinline__ void topk_insert(float (&tv)[KMAX], int (&te)[KMAX], float l, int e) {
+  if (l > tv[KMAX - 1] || te[KMAX - 1] < 0) {
+    float cv = l;
+    int ce = e;
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      if (cv > tv[j] || te[j] < 0) {
+        const float sv = tv[j];
+        const int se = te[j];
+        tv[j] = cv;
+        te[j] = ce;
+        cv = sv;
+        ce = se;
+      }
+    }
+  }
+}
+
+// KMAX: k rounded up to a power of two; the epilogue thread keeps the KMAX
+// largest logits sorted and reports the first k.
+template <int NE, int KMAX>
+__global__ void __launch_bounds__(RouteTopkCfg<NE>::kThreads, 1)
+    router_topk_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_wr,
+                       const float* __restrict__ bias, int64_t T, int H, int E, int k,
+                       float* __restrict__ logits_out, int32_t* __restrict__ idx, float* __restrict__ wout,
+                       int32_t* status, long long wait_lim) {
+  using C = RouteTopkCfg<NE>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* ctrl = smem + kRouteStages * C::kStage;
+  uint64_t* full = reinterpret_cast<uint64_t*>(ctrl);
+  uint64_t* empty = full + kRouteStages;
+  uint64_t* tfull = empty + kRouteStages;
+  uint64_t* tempty = tfull + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kRouteStages; ++s) {
+      tc::mbar_init(&full[s], 1);
+      tc::mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      tc::mbar_init(&tfull[a], 1);
+      tc::mbar_init(&tempty[a], 4);
+    }
+    *abort = 0;
+    tc::fence_mbar_init();
+    tc::prefetch_tmap(&tmap_x);
+    tc::prefetch_tmap(&tmap_wr);
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(tmem_slot, 2 * NE);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  pdl_wait();  // x comes from the caller's earlier work
+  pdl_trigger();
+  const int ntiles = (int)((T + 127) / 128);
+  const int nkb = H / 64;
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int t = blockIdx.x; t < ntiles && !tc::aborted(abort); t += gridDim.x) {
+      for (int kb = 0; kb < nkb; ++kb) {
+        if (!tc::mbar_wait(&empty[stage], phase ^ 1u, abort, wait_lim)) {
+          if (lane == 0) raise_status(status, MOE_ERR_TIMEOUT);
+          *abort = 1;
+          break;
+        }
+        if (tc::elect_one()) {
+          uint8_t* st = smem + stage * C::kStage;
+          tc::mbar_expect_tx(&full[stage], (uint32_t)(C::kA + E * 128));
+          tc::tma_load_2d(st, &tmap_x, &full[stage], kb * 128, t * 128);
+          tc::tma_load_2d(st + C::kA, &tmap_wr, &full[stage], kb * 128, 0);
+        }
+        __syncwarp();
+        if (++stage == kRouteStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    int stage = 0;
+    uint32_t phase = 0;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    const uint32_t idesc = tc::idesc_bf16((uint32_t)E);
+    for (int t = blockIdx.x; t < ntiles && !tc::aborted(abort); t += gridDim.x) {
+      if (!tc::mbar_wait(&tempty[acc], acc_phase ^ 1u, abort, wait_lim)) {
+        if (lane == 0) raise_status(status, MOE_ERR_TIMEOUT);
+        *abort = 1;
+        break;
+      }
+      tc::fence_after_sync();
+      const uint32_t d = tmem + (uint32_t)(acc * NE);
+      bool ok = true;
+      for (int kb = 0; kb < nkb; ++kb) {
+        if (!tc::mbar_wait(&full[stage], phase, abort, wait_lim)) {
+          if (lane == 0) raise_status(status, MOE_ERR_TIMEOUT);
+          *abort = 1;
+          ok = false;
+          break;
+        }
+        tc::fence_after_sync();
+        if (tc::elect_one()) {
+          uint8_t* st = smem + stage * C::kStage;
+          const uint64_t da0 = tc::desc_sw128(tc::smem_u32(st)), db0 = tc::desc_sw128(tc::smem_u32(st + C::kA));
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            tc::mma_bf16(d, da0 + (uint64_t)(kk * 2), db0 + (uint64_t)(kk * 2), idesc,
+                         (kb > 0 || kk > 0) ? 1u : 0u);
+          tc::mma_commit(&empty[stage]);
+        }
+        __syncwarp();
+        if (++stage == kRouteStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (!ok) break;
+      if (tc::elect_one()) tc::mma_commit(&tfull[acc]);
+      __syncwarp();
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;   // tensor-memory lane quarter: tokens 32q .. 32q + 31 of the tile
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+      if (!tc::mbar_wait(&tfull[acc], acc_phase, abort, wait_lim)) {
+        if (lane == 0) raise_status(status, MOE_ERR_TIMEOUT);
+        *abort = 1;
+        break;
+      }
+      tc::fence_after_sync();
+      const int64_t tok = (int64_t)t * 128 + q * 32 + lane;
+      const uint32_t base = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * NE);
+      // the KMAX largest so far, descending; an empty slot holds index -1
+      float tv[KMAX];
+      int te[KMAX];
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j) {
+        tv[j] = -INFINITY;
+        te[j] = -1;
+      }
+      bool bad = false;
+      for (int c0 = 0; c0 < E; c0 += 16) {
+        float v[16];
+        tc::tmem_ld16(base + (uint32_t)c0, v);
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const int e = c0 + c;
+          const float l = v[c] + (bias ? __ldg(bias + e) : 0.0f);
+          if (logits_out && tok < T) logits_out[tok * E + e] = l;
+          if (isnan(l)) bad = true;
+          topk_insert<KMAX>(tv, te, l, e);
+        }
+      }
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&tempty[acc]);
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+      if (tok >= T) continue;
+      if (!(tv[0] > -INFINITY)) bad = true;
+      if (bad) {
+        raise_status(status, MOE_ERR_DEVICE_FAULT);
+        for (int j = 0; j < k; ++j) {
+          idx[tok * k + j] = j;
+          wout[tok * k + j] = 0.0f;
+        }
+        continue;
+      }
+      float ex[KMAX], sum = 0.0f;
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j)
+        if (j < k) {
+          ex[j] = expf(tv[j] - tv[0]);
+          sum += ex[j];
+        }
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j)
+        if (j < k) {
+          idx[tok * k + j] = te[j];
+          wout[tok * k + j] = __fdiv_rn(ex[j], sum);
+        }
+    }
+  }
+  __syncwarp();
+  __syncthreads();
+  if (*abort) {
+    const long long w0 = clock64();
+    while (clock64() - w0 < 2000000LL) {
+    }
+  }
+  tc::fence_after_sync();
+  if (warp == 1) tc::tmem_dealloc(tmem, 2 * NE);
+}
+
 }  // namespace
 
 cudaError_t launch_grouped_gemm(const GemmArgs& g, int epi, int bn, const void* a_base, int64_t a_rows,
@@ -1729,15 +1992,16 @@ cudaError_t launch_fused_ffn(const GemmArgs& g1, const GemmArgs& g2, const Fused
   if (f.xg && (f.T > kGatherMaxT || f.S > kGatherMaxS || !f.xsl || (!f.perm_token && !f.slot_expert) || f.k < 1))
     return cudaErrorInvalidValue;
   if (f.out && (!f.xg || !f.slot_expert || !g2.out32 || !f.done || !f.topk_w)) return cudaErrorInvalidValue;
+  const FusedArgs& fa = f;
   switch (g1.fmt) {
     case MOE_FMT_NVFP4:
-      return f.xg ? launch_fused_cfg<MOE_FMT_NVFP4, 64, true>(g1, g2, f, w13, w13_rows, w2, w2_rows, xq, hq, num_sms, s)
-                  : launch_fused_cfg<MOE_FMT_NVFP4, 64, false>(g1, g2, f, w13, w13_rows, w2, w2_rows, xq, hq, num_sms,
-                                                               s);
+      return fa.xg ? launch_fused_cfg<MOE_FMT_NVFP4, 64, true>(g1, g2, fa, w13, w13_rows, w2, w2_rows, xq, hq, num_sms, s)
+                   : launch_fused_cfg<MOE_FMT_NVFP4, 64, false>(g1, g2, fa, w13, w13_rows, w2, w2_rows, xq, hq,
+                                                                num_sms, s);
     case MOE_FMT_MXFP4:
-      return f.xg ? launch_fused_cfg<MOE_FMT_MXFP4, 64, true>(g1, g2, f, w13, w13_rows, w2, w2_rows, xq, hq, num_sms, s)
-                  : launch_fused_cfg<MOE_FMT_MXFP4, 64, false>(g1, g2, f, w13, w13_rows, w2, w2_rows, xq, hq, num_sms,
-                                                               s);
+      return fa.xg ? launch_fused_cfg<MOE_FMT_MXFP4, 64, true>(g1, g2, fa, w13, w13_rows, w2, w2_rows, xq, hq, num_sms, s)
+                   : launch_fused_cfg<MOE_FMT_MXFP4, 64, false>(g1, g2, fa, w13, w13_rows, w2, w2_rows, xq, hq,
+                                                                num_sms, s);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -1781,6 +2045,49 @@ cudaError_t launch_router_gemm(const uint16_t* x, int64_t T, int H, const uint16
   const int64_t items = (T + kRouterBN - 1) / kRouterBN * (E / 128) * ksplit;
   const int grid = (int)(items < num_sms ? items : num_sms);
   return launch_cfg<kFmtBF16, kEpiLogits, kRouterBN, false>(g, wr, E, x, T, grid, s);
+}
+
+bool router_topk_fits(int64_t T, int E, int H, int k, int num_sms) {
+  return T >= 128 && (T + 127) / 128 >= num_sms / 2 && E >= 16 && E <= 256 && E % 16 == 0 && H % 64 == 0 && k >= 1 &&
+         k <= kRouteTopkMaxK && tensor_maps_available();
+}
+
+cudaError_t launch_router_topk(const uint16_t* x, int64_t T, int H, const uint16_t* wr, const float* bias, int E,
+                               int k, float* logits_out, int32_t* idx, float* w, int32_t* status, int num_sms,
+                               cudaStream_t s) {
+  if (T == 0) return cudaSuccess;
+  if (!router_topk_fits(T, E, H, k, num_sms)) return cudaErrorInvalidValue;
+  CUtensorMap mx, mw;
+  if (!make_map(&mx, x, T, 2 * (int64_t)H, 128)) return cudaErrorInvalidValue;
+  if (!make_map(&mw, wr, E, 2 * (int64_t)H, E)) return cudaErrorInvalidValue;
+  const int64_t ntiles = (T + 127) / 128;
+  const int grid = (int)(ntiles < num_sms ? ntiles : num_sms);
+  const long long lim = wait_cycles();
+  cudaError_t e = cudaErrorInvalidValue;
+#define MOE_RT(NE, KM)                                                                                      \
+  {                                                                                                         \
+    auto kern = router_topk_kernel<NE, KM>;                                                                 \
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, RouteTopkCfg<NE>::kSmem);    \
+    if (e == cudaSuccess)                                                                                   \
+      e = launch_pdl(kern, dim3(grid), dim3(RouteTopkCfg<NE>::kThreads), RouteTopkCfg<NE>::kSmem, s, mx, mw, \
+                     bias, T, H, E, k, logits_out, idx, w, status, lim);                                    \
+  }
+#define MOE_RT_K(NE)                 \
+  if (k <= 1) MOE_RT(NE, 1)          \
+  else if (k <= 2) MOE_RT(NE, 2)     \
+  else if (k <= 4) MOE_RT(NE, 4)     \
+  else if (k <= 8) MOE_RT(NE, 8)     \
+  else MOE_RT(NE, 16)
+  if (E <= 128) {
+    MOE_RT_K(128)
+  } else {
+    MOE_RT_K(256)
+  }
+#undef MOE_RT_K
+#undef MOE_RT
+  if (e != cudaSuccess) return e;
+  count_launches(1);
+  return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------- planning --

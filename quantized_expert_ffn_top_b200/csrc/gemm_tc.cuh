@@ -156,6 +156,16 @@ void set_gemm_pairs(int mode);
 constexpr int kRouterBN = 64;
 constexpr int kRouterMaxSplit = 4;
 int router_ksplit(int64_t T, int E, int H, int num_sms);
+// Router logits and top-k in one tcgen05 kernel (T >= 128; E a multiple of
+// 16 up to 256; H % 64 == 0; k <= 16): 128 tokens per tile on the MMA's M
+// side, every expert on its N side, the top-k kept per token in registers by
+// the epilogue.  logits_out (nullable) receives the logits.
+bool router_topk_fits(int64_t T, int E, int H, int k, int num_sms);
+// Logits and top-k in one kernel, for batches whose 128-token tiles fill at
+// least half the SMs (router_topk_fits).
+cudaError_t launch_router_topk(const uint16_t* x, int64_t T, int H, const uint16_t* wr, const float* bias, int E,
+                               int k, float* logits_out, int32_t* idx, float* w, int32_t* status, int num_sms,
+                               cudaStream_t s);
 cudaError_t launch_router_gemm(const uint16_t* x, int64_t T, int H, const uint16_t* wr, const float* bias, int E,
                                float* logits_parts, int64_t part_stride, int ksplit, int32_t* status, int num_sms,
                                cudaStream_t s);

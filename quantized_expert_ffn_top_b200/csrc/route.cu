@@ -10,6 +10,7 @@
 
 #include "kernels.cuh"
 #include "token_quant.cuh"
+#include "topk_warp.cuh"
 
 namespace moe {
 
@@ -153,89 +154,6 @@ cudaError_t launch_router_logits(const uint16_t* x, int64_t T, int H, const uint
 }
 
 // -------------------------------------------------------------- top-k -----
-// One warp per token; lane l holds logits l, l+32, ... in registers.  Each
-// round picks the largest not-yet-taken logit (ties -> lower index) with a
-// warp arg-max; lane 0 writes the index and exp(L - L_0); a final pass divides
-// by the sum.  A NaN, or a row without a finite logit, raises the status word
-// and writes indices 0..k-1 with zero weights.
-// The logits may arrive as nparts partial sums (a router GEMM split along
-// H), added here in part order; logits_out (nullable) receives the sums.
-// Top-k of one token's logits row by one warp (J = ceil(E / 32) logits per
-// lane).  COHERENT: the row was written by other blocks of this kernel, so it
-// is read through L2 (ld.cg) rather than the read-only path.
-template <int J, bool COHERENT>
-__device__ __forceinline__ void topk_token(const float* __restrict__ L, int nparts, int64_t part_stride,
-                                           float* __restrict__ logits_out_row, int E, int k,
-                                           int32_t* __restrict__ idx_row, float* __restrict__ w_row,
-                                           int32_t* status) {
-  const int lane = threadIdx.x & 31;
-  auto ld = [&](const float* p) { return COHERENT ? __ldcg(p) : __ldg(p); };
-  float v[J];
-  bool bad = false;
-#pragma unroll
-  for (int j = 0; j < J; ++j) {
-    const int e = lane + 32 * j;
-    v[j] = e < E ? ld(L + e) : -INFINITY;
-  }
-  for (int p = 1; p < nparts; ++p) {
-#pragma unroll
-    for (int j = 0; j < J; ++j) {
-      const int e = lane + 32 * j;
-      if (e < E) v[j] += ld(L + p * part_stride + e);
-    }
-  }
-#pragma unroll
-  for (int j = 0; j < J; ++j) {
-    const int e = lane + 32 * j;
-    if (e < E && isnan(v[j])) bad = true;
-    if (e < E && logits_out_row) logits_out_row[e] = v[j];
-  }
-  uint32_t taken = 0u;
-#pragma unroll
-  for (int j = 0; j < J; ++j)
-    if (lane + 32 * j >= E) taken |= 1u << j;
-  float top = 0.0f, sum = 0.0f;
-  bad = __any_sync(0xffffffffu, bad);
-  for (int r = 0; r < k; ++r) {
-    float bv = -INFINITY;
-    int be = 0x7fffffff;
-#pragma unroll
-    for (int j = 0; j < J; ++j) {
-      const int e = lane + 32 * j;
-      if (!(taken & (1u << j)) && (v[j] > bv || (v[j] == bv && e < be))) {
-        bv = v[j];
-        be = e;
-      }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-      if (ov > bv || (ov == bv && oe < be)) {
-        bv = ov;
-        be = oe;
-      }
-    }
-    if (be != 0x7fffffff && (be & 31) == lane) taken |= 1u << (be >> 5);
-    if (r == 0) {
-      top = bv;
-      if (!(top > -INFINITY)) bad = true;
-    }
-    const float ex = expf(bv - top);
-    sum += ex;
-    if (lane == 0) {
-      idx_row[r] = bad ? r : be;
-      w_row[r] = bad ? 0.0f : ex;
-    }
-  }
-  __syncwarp();
-  if (bad) {
-    if (lane == 0) raise_status(status, MOE_ERR_DEVICE_FAULT);
-    return;
-  }
-  for (int r = lane; r < k; r += 32) w_row[r] = __fdiv_rn(w_row[r], sum);
-}
-
 // One warp per token; lane l holds logits l, l+32, ... in registers.  Each
 // round picks the largest not-yet-taken logit (ties -> lower index) with a
 // warp arg-max; lane 0 writes the index and exp(L - L_0); a final pass divides

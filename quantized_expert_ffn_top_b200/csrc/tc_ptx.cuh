@@ -174,6 +174,11 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 }
 // Contiguous copy (16-byte aligned addresses, size a multiple of 16).
 // Acquire load of a flag at GPU scope.
+// Adds four consecutive floats at p (16-byte aligned) in L2, one reduction
+// request for all four.
+__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
+}
 __device__ __forceinline__ int ld_acquire_gpu(const int* p) {
   int v;
   asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");

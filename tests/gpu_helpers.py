@@ -64,12 +64,16 @@ def routed_inputs(w: synth.Workload, seed: int = synth.SEED):
     return x, wr, b
 
 
-def router_order(T: int, E: int, H: int) -> int:
+def router_order(T: int, E: int, H: int, k: int) -> int:
     """Which fixed fp32 summation order moe_route's logits follow (the header
     documents it): 1 = the small-batch order (T <= 64, H % 8 == 0), 2 = one
-    sequential sum, 0 = the tensor cores' own order (T >= 128, E % 128 == 0,
-    H % 64 == 0), which the oracle cannot replay."""
-    if T >= 128 and E % 128 == 0 and H % 64 == 0:
+    sequential sum, 0 = the tensor cores' own order (T >= 128, H % 64 == 0
+    and either E % 128 == 0, or the one-kernel router: 128-token tiles for at
+    least half the SMs, 16 <= E <= 256 with E % 16 == 0, k <= 16), which the
+    oracle cannot replay."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    one_kernel = (T + 127) // 128 >= sms // 2 and 16 <= E <= 256 and E % 16 == 0 and k <= 16
+    if T >= 128 and H % 64 == 0 and (one_kernel or E % 128 == 0):
         return 0
     if T <= 64 and H % 8 == 0:
         return 1
@@ -100,7 +104,7 @@ def forward_reference(w: synth.Workload, x, wr, b, W, Ws=None, act: int = 1, a13
     logit gap lies within routing_tol of the GPU's own logits (moe_route on
     the same batch) are left out, counted and bounded.  route_T: the batch
     size the router sees (a slice of moe_forward_host)."""
-    order = router_order(route_T or w.T, w.E, w.H)
+    order = router_order(route_T or w.T, w.E, w.H, w.k)
     r = oracle.moe_forward(x, wr, b, w.k, W, Ws, act=act, a13_static=a13 or 0.0, a2_static=a2 or 0.0,
                            sh_a2_static=sh_a2 or 0.0, tokens=tokens, router_order=order)
     if order:

@@ -302,6 +302,7 @@ def test_gathered_token_rows_change_nothing(name, over, static, skew):
     tolerance of the oracle."""
     ys = []
     try:
+        ops.moe_set_option(ops.OPT_GATHER_X, 1)
         for fused in (0, 1):
             ops.moe_set_option(ops.OPT_FUSED_FFN, fused)
             w, W, x, perm, off, a13, a2, y, st = _run(over, static, skew, 2)
@@ -309,6 +310,7 @@ def test_gathered_token_rows_change_nothing(name, over, static, skew):
             ys.append(y)
     finally:
         ops.moe_set_option(ops.OPT_FUSED_FFN, 1)
+        ops.moe_set_option(ops.OPT_GATHER_X, 0)
     assert np.array_equal(ys[0], ys[1])
     ry, _ = oracle.grouped_ffn(x, perm, off, W, 1, a13 or 0.0, a2 or 0.0)
     assert max_abs_rel(ys[1], ry) < TOL

@@ -30,6 +30,11 @@ def ws(nbytes=1 << 24):
     return ops.new_workspace(nbytes)
 
 
+def route_ws_bytes(w) -> int:
+    # moe_route's partial logits (up to 4 parts of T x E fp32) and the status words
+    return max(1 << 24, 16 * w.T * w.E + (1 << 20))
+
+
 # ----------------------------------------------------------- quantisers ----
 def _all_finite_bf16_as_f32(limit=None):
     bits = np.arange(1 << 16, dtype=np.uint32)
@@ -143,8 +148,17 @@ ROUTE_CASES = [("tiny", {}), ("decode", {}), ("prefill", {}), ("large", dict(T=3
                # H = 2304 (a ragged second stretch), one token
                ("prefill", dict(T=64)), ("large", dict(T=37)), ("decode", dict(T=9, H=2304, E=60, k=4)),
                ("large", dict(T=1)),
-               # the sequential order: 64 < T < 128, or E not a multiple of 128
-               ("decode", dict(T=100)), ("prefill", dict(T=300, E=60, k=4)), ("tiny", dict(T=200))]
+               # the sequential order: 64 < T < 128, or E off the tensor-core grid
+               ("decode", dict(T=100)), ("prefill", dict(T=300, E=60, k=4)), ("tiny", dict(T=200)),
+               ("prefill", dict(T=129, E=48, k=6)), ("prefill", dict(T=1000, E=32, k=16)),
+               ("prefill", dict(T=257, E=16, k=1)),
+               # the router GEMM: E = 256 with a ragged tile; k = 17
+               ("large", dict(T=700)), ("prefill", dict(T=300, E=128, k=17)),
+               # the one-kernel router with top-k (128-token tiles for half the
+               # SMs and more): ragged last tile with small E, k = 16 (the most
+               # it takes)
+               ("prefill", dict(T=9600, k=4)), ("prefill", dict(T=9601, E=48, k=6)),
+               ("prefill", dict(T=9500, E=32, k=16))]
 
 
 @pytest.mark.parametrize("name,over", ROUTE_CASES)
@@ -159,10 +173,11 @@ def test_route_matches_oracle(name, over):
     x, wr, b = routed_inputs(w)
     logits = torch.empty((w.T, w.E), dtype=torch.float32, device="cuda")
     idx, wt = ops.moe_route(bits_to_dev_bf16(x), bits_to_dev_bf16(wr),
-                            None if b is None else torch.from_numpy(b).cuda(), w.k, ws(), logits=logits)
+                            None if b is None else torch.from_numpy(b).cuda(), w.k, ws(route_ws_bytes(w)),
+                            logits=logits)
     gl = logits.cpu().numpy()
     gi = idx.cpu().numpy()
-    order = router_order(w.T, w.E, w.H)
+    order = router_order(w.T, w.E, w.H, w.k)
     RL = oracle.router_logits(x, wr, b)
     assert max_abs_rel(gl.astype(np.float64), RL) < 1e-5
     if order:
@@ -182,6 +197,46 @@ def test_route_matches_oracle(name, over):
     for t in np.nonzero(amb)[0]:
         assert len(set(gi[t])) == w.k
         assert np.all(np.diff(gl[t, gi[t]].astype(np.float64)) <= 0)
+
+
+ROUTER_TOPK_CASES = [("prefill", dict(T=9600)), ("large", dict(T=10240)), ("prefill", dict(T=9601, E=48, k=6)),
+                     ("prefill", dict(T=9500, E=32, k=16))]
+
+
+@pytest.mark.parametrize("name,over", ROUTER_TOPK_CASES)
+def test_router_topk_kernel_agrees_with_router_gemm(name, over):
+    """The one-kernel router (all of H in one accumulator, top-k in the
+    epilogue) against the two-kernel router (logits, then the top-k kernel):
+    logits within fp32 rounding of each other; indices and weights equal on
+    every token whose top-k order the difference cannot flip."""
+    w = synth.workload(name, **over)
+    x, wr, b = routed_inputs(w)
+    xd, wrd = bits_to_dev_bf16(x), bits_to_dev_bf16(wr)
+    bd = None if b is None else torch.from_numpy(b).cuda()
+    res = []
+    try:
+        for opt in (0, 1):
+            ops.moe_set_option(ops.OPT_ROUTER_TOPK, opt)
+            logits = torch.empty((w.T, w.E), dtype=torch.float32, device="cuda")
+            W = ws(route_ws_bytes(w))
+            n0 = ops.moe_kernel_launch_count()
+            idx, wt = ops.moe_route(xd, wrd, bd, w.k, W, logits=logits)
+            n = ops.moe_kernel_launch_count() - n0
+            assert ops.moe_get_device_status(W) == 0
+            res.append((logits.cpu().numpy().astype(np.float64), idx.cpu().numpy(), wt.cpu().numpy(), n))
+    finally:
+        ops.moe_set_option(ops.OPT_ROUTER_TOPK, 1)
+    (l0, i0, w0, n0_), (l1, i1, w1, n1_) = res
+    assert n1_ == 1 and n0_ == 2, (n0_, n1_)
+    RL = oracle.router_logits(x, wr, b)
+    assert max_abs_rel(l1, RL) < 1e-5 and max_abs_rel(l0, RL) < 1e-5
+    amb = ambiguous_tokens(l0, w.k, 2.0 * float(np.max(np.abs(l1 - l0))) + 1e-7)
+    report_ambiguous(amb, f"router_topk {name} {over}")
+    assert np.array_equal(i1[~amb], i0[~amb])
+    assert np.allclose(w1[~amb], w0[~amb], rtol=1e-4, atol=1e-6)
+    # every token: k distinct experts, descending in the kernel's own logits
+    assert all(len(set(r)) == w.k for r in i1)
+    assert np.all(np.diff(np.take_along_axis(l1, i1.astype(np.int64), 1), axis=1) <= 0)
 
 
 # ----------------------------------------------------------- permutation ----
@@ -351,7 +406,6 @@ def test_permutation_with_x_quantisation_changes_nothing(name, over, scales):
             outs.append(out.view(torch.int16).cpu().numpy())
     finally:
         ops.moe_set_option(ops.OPT_PERMUTE_QUANT, 1)
-        ops.moe_set_option(ops.OPT_SMALL_BATCH_FORWARD, 1)
     assert np.array_equal(outs[0], outs[1])
     assert launches[1] == launches[0] - 1, launches
     r, keep = forward_reference(w, x, wr, b, W, act=1, a13=a13, a2=a2)
@@ -483,6 +537,7 @@ def test_small_batch_forward_in_two_kernels(name, over, scales):
     W_ = ws(ops.workspace_size(w.T, w.k, bank, None, 1))
     outs, launches = [], []
     try:
+        ops.moe_set_option(ops.OPT_GATHER_X, 1)
         for opt in (0, 1):
             ops.moe_set_option(ops.OPT_SMALL_BATCH_FORWARD, opt)
             n0 = ops.moe_kernel_launch_count()
@@ -491,7 +546,8 @@ def test_small_batch_forward_in_two_kernels(name, over, scales):
             assert ops.moe_get_device_status(W_) == 0, opt
             outs.append(dev_to_f64(o))
     finally:
-        ops.moe_set_option(ops.OPT_SMALL_BATCH_FORWARD, 1)
+        ops.moe_set_option(ops.OPT_SMALL_BATCH_FORWARD, 0)
+        ops.moe_set_option(ops.OPT_GATHER_X, 0)
     assert launches[1] == (3 if a13 is None and w.fmt == "nvfp4" else 2), launches
     assert max_abs_rel(outs[1], outs[0]) < 1e-2
     r, keep = forward_reference(w, x, wr, b, W, act=1, a13=a13, a2=a2)
