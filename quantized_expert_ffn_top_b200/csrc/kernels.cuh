@@ -92,7 +92,6 @@ cudaError_t launch_router_decode(int fmt, const uint16_t* x, int64_t T, int H, c
 // permute.cu
 struct PermuteScratch {
   int32_t* chunk_counts;   // [nchunks][E]
-  int32_t* ticket;         // one int: blocks done counting
   int nchunks;
 };
 int permute_chunk_slots();

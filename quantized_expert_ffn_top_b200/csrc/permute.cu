@@ -8,16 +8,17 @@
 // for a dense block of rows.  Slots keep their flat order i = t*k + j inside a
 // segment (stable), which makes the permutation unique and bit-comparable.
 //
-// Passes over chunks of kChunk slots (8 warps x 256):
+// Two passes over chunks of kChunk slots (8 warps x 256):
 //   1. per chunk and expert, the count (warp-private counters fed by
 //      __match_any_sync, one writer lane per expert and step);
-//   2. per expert the exclusive prefix over chunks, the totals and the
-//      exclusive prefix over experts -> offsets (and, on request, the grouped
-//      FFN's tile plan) -- run by the last block of pass 1 to finish, found
-//      with one atomic ticket;
-//   3. per chunk again: each warp's base = chunk base + earlier warps'
-//      counts, and each slot's rank among equal experts earlier in its warp
-//      step -> perm_token[p] = t, inv_perm[i] = p.
+//   2. per chunk again: every block reads all chunks' counts, so it knows
+//      for each expert the slots in earlier chunks and the total; a scan of
+//      the totals over experts gives the offsets (block 0 writes them and,
+//      on request, the grouped FFN's tile plan); each warp's base = expert
+//      offset + earlier chunks + earlier warps, and each slot's rank among
+//      equal experts earlier in its warp step -> perm_token[p] = t,
+//      inv_perm[i] = p.
+// No block waits for another inside a kernel, and nothing is cleared first.
 // Small batches run all three inside one block, which in the forward at up
 // to 8 tokens also quantises x into the FFN's padded rows.
 #include <string.h>
@@ -90,22 +91,14 @@ __device__ __forceinline__ int32_t scan256_excl(int32_t v, int32_t* warp_tot, in
   return incl - v + base;
 }
 
-// Pass 1: per chunk and expert, the count.  The last block to finish (a
-// ticket taken after a memory fence) then runs pass 2 -- per expert the
-// exclusive prefix over chunks plus the expert's offset, turning the counts
-// into each chunk's base positions -- and writes the offsets and, when asked,
-// the tile plan.  The ticket is zero on entry and is reset by that block.
+// Pass 1: per chunk and expert, the count.
 __global__ void __launch_bounds__(kPermWarps * 32) perm_count_kernel(const int32_t* __restrict__ idx, int64_t S,
                                                                      int E, int32_t* __restrict__ chunk_counts,
-                                                                     int32_t* __restrict__ ticket,
-                                                                     int32_t* __restrict__ offsets, PlanOut plan,
                                                                      int32_t* status) {
   pdl_wait();  // inputs come from the previous kernels
   pdl_trigger();
 
-  extern __shared__ int32_t cnt[];  // [kPermWarps][E]; the last block reuses it as [E] totals
-  __shared__ int32_t warp_tot[kPermWarps];
-  __shared__ int is_last;
+  extern __shared__ int32_t cnt[];  // [kPermWarps][E]
   for (int i = threadIdx.x; i < kPermWarps * E; i += blockDim.x) cnt[i] = 0;
   __syncthreads();
   const int64_t base = (int64_t)blockIdx.x * kChunk;
@@ -117,50 +110,66 @@ __global__ void __launch_bounds__(kPermWarps * 32) perm_count_kernel(const int32
     for (int w = 0; w < kPermWarps; ++w) s += cnt[w * E + e];
     chunk_counts[(int64_t)blockIdx.x * E + e] = s;
   }
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) is_last = atomicAdd(ticket, 1) == (int)gridDim.x - 1;
-  __syncthreads();
-  if (!is_last) return;
-  __threadfence();
-  const int nchunks = gridDim.x;
-  int32_t* tot = cnt;  // [E] counts, then offsets
+}
+
+// Pass 2 (see the file's head).  Dynamic shared memory: [kPermWarps][E]
+// counters, then [E] totals and [E] earlier-chunk counts.
+__global__ void __launch_bounds__(kPermWarps * 32) perm_scatter_kernel(const int32_t* __restrict__ idx, int64_t S,
+                                                                       int k, int E,
+                                                                       const int32_t* __restrict__ chunk_counts,
+                                                                       int32_t* __restrict__ offsets, PlanOut plan,
+                                                                       int32_t* __restrict__ perm_token,
+                                                                       int32_t* __restrict__ inv_perm) {
+  pdl_wait();  // inputs come from the previous kernels
+  pdl_trigger();
+
+  extern __shared__ int32_t cnt[];
+  int32_t* tot = cnt + kPermWarps * E;   // [E] slots of the expert in all chunks, then its offset
+  int32_t* before = tot + E;             // [E] slots of the expert in earlier chunks
+  __shared__ int32_t warp_tot[kPermWarps];
+  for (int i = threadIdx.x; i < kPermWarps * E; i += blockDim.x) cnt[i] = 0;
+  const int nchunks = gridDim.x, c = blockIdx.x;
+  // every chunk's count of expert e, eight loads in flight
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    int32_t run = 0;
-    for (int c0 = 0; c0 < nchunks; c0 += 8) {  // eight loads in flight, then the running sum
+    int32_t run = 0, pre = 0;
+    for (int c0 = 0; c0 < nchunks; c0 += 8) {
       int32_t v[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) v[u] = c0 + u < nchunks ? __ldcg(chunk_counts + (int64_t)(c0 + u) * E + e) : 0;
+      for (int u = 0; u < 8; ++u) v[u] = c0 + u < nchunks ? __ldg(chunk_counts + (int64_t)(c0 + u) * E + e) : 0;
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
-        if (c0 + u < nchunks) chunk_counts[(int64_t)(c0 + u) * E + e] = run;
+        if (c0 + u == c) pre = run;
         run += v[u];
       }
     }
     tot[e] = run;
+    before[e] = pre;
   }
   __syncthreads();
+  const int64_t base = (int64_t)c * kChunk;
+  warp_counts(idx, S, base, E, cnt, nullptr);
   // scans over experts: each thread owns a contiguous group of `per` experts
   const int per = (E + (int)blockDim.x - 1) / (int)blockDim.x;
   const int e0 = threadIdx.x * per;
   int32_t mine = 0, pad_mine = 0, til_mine = 0;
+  const bool with_plan = c == 0 && plan.bn > 0;
   for (int e = e0; e < e0 + per && e < E; ++e) {
     mine += tot[e];
     pad_mine += (tot[e] + 127) / 128 * 128;
-    if (plan.bn > 0) til_mine += (tot[e] + plan.bn - 1) / plan.bn;
+    if (with_plan) til_mine += (tot[e] + plan.bn - 1) / plan.bn;
   }
   int32_t total, pad_total = 0, til_total = 0;
   int32_t off = scan256_excl(mine, warp_tot, &total);
   int32_t pbase = 0, tbase = 0;
-  if (plan.bn > 0) {
+  if (with_plan) {
     pbase = scan256_excl(pad_mine, warp_tot, &pad_total);
     tbase = scan256_excl(til_mine, warp_tot, &til_total);
   }
   __syncthreads();
   for (int e = e0; e < e0 + per && e < E; ++e) {
     const int32_t n = tot[e];
-    offsets[e] = off;
-    if (plan.bn > 0) {
+    if (c == 0) offsets[e] = off;
+    if (with_plan) {
       plan.poff[e] = pbase;
       const int til = (n + plan.bn - 1) / plan.bn;
       for (int j = 0; j < til && tbase + j < plan.max_tiles; ++j) {
@@ -174,49 +183,20 @@ __global__ void __launch_bounds__(kPermWarps * 32) perm_count_kernel(const int32
       pbase += (n + 127) / 128 * 128;
       tbase += til;
     }
-    tot[e] = off;  // the expert's offset, for the chunk bases below
+    tot[e] = off;  // the expert's offset
     off += n;
   }
-  if (threadIdx.x == 0) {
+  if (c == 0 && threadIdx.x == 0) {
     offsets[E] = total;
-    if (plan.bn > 0) {
+    if (with_plan) {
       plan.poff[E] = pad_total;
       *plan.ntiles = min(til_total, plan.max_tiles);
     }
-    *ticket = 0;
   }
   __syncthreads();
-  // chunk bases: the expert's offset added to the prefixes, eight in flight
+  // exclusive prefix over warps per expert, from the chunk's base
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    const int32_t o = tot[e];
-    for (int c0 = 0; c0 < nchunks; c0 += 8) {
-      int32_t v[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) v[u] = c0 + u < nchunks ? __ldcg(chunk_counts + (int64_t)(c0 + u) * E + e) : 0;
-#pragma unroll
-      for (int u = 0; u < 8; ++u)
-        if (c0 + u < nchunks) chunk_counts[(int64_t)(c0 + u) * E + e] = v[u] + o;
-    }
-  }
-}
-
-__global__ void __launch_bounds__(kPermWarps * 32) perm_scatter_kernel(const int32_t* __restrict__ idx, int64_t S,
-                                                                       int k, int E,
-                                                                       const int32_t* __restrict__ chunk_base,
-                                                                       int32_t* __restrict__ perm_token,
-                                                                       int32_t* __restrict__ inv_perm) {
-  pdl_wait();  // inputs come from the previous kernels
-  pdl_trigger();
-
-  extern __shared__ int32_t cnt[];  // [kPermWarps][E]
-  for (int i = threadIdx.x; i < kPermWarps * E; i += blockDim.x) cnt[i] = 0;
-  __syncthreads();
-  const int64_t base = (int64_t)blockIdx.x * kChunk;
-  warp_counts(idx, S, base, E, cnt, nullptr);
-  __syncthreads();
-  // exclusive prefix over warps per expert, offset by the chunk's base
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    int32_t run = chunk_base[(int64_t)blockIdx.x * E + e];
+    int32_t run = tot[e] + before[e];
 #pragma unroll
     for (int w = 0; w < kPermWarps; ++w) {
       const int32_t v = cnt[w * E + e];
@@ -508,20 +488,17 @@ cudaError_t launch_permute(const int32_t* idx, int64_t S, int k, int E, int32_t*
     // no slots: offsets are all zero
     return cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (E + 1), s);
   }
-  const size_t smem = sizeof(int32_t) * kPermWarps * E;
   PlanOut p;
   if (plan) {
     p = *plan;
   } else {
     memset(&p, 0, sizeof(p));
   }
-  cudaError_t e = cudaMemsetAsync(scratch.ticket, 0, sizeof(int32_t), s);
+  cudaError_t e = launch_pdl(perm_count_kernel, dim3(nchunks), dim3(kPermWarps * 32),
+                             sizeof(int32_t) * kPermWarps * E, s, idx, S, E, scratch.chunk_counts, status);
   if (e != cudaSuccess) return e;
-  e = launch_pdl(perm_count_kernel, dim3(nchunks), dim3(kPermWarps * 32), smem, s, idx, S, E, scratch.chunk_counts,
-                 scratch.ticket, offsets, p, status);
-  if (e != cudaSuccess) return e;
-  e = launch_pdl(perm_scatter_kernel, dim3(nchunks), dim3(kPermWarps * 32), smem, s, idx, S, k, E,
-                 (const int32_t*)scratch.chunk_counts, perm_token, inv_perm);
+  e = launch_pdl(perm_scatter_kernel, dim3(nchunks), dim3(kPermWarps * 32), sizeof(int32_t) * (kPermWarps + 2) * E,
+                 s, idx, S, k, E, (const int32_t*)scratch.chunk_counts, offsets, p, perm_token, inv_perm);
   if (e != cudaSuccess) return e;
   count_launches(2);
   if (planned && plan && plan->bn > 0) *planned = true;
@@ -547,16 +524,13 @@ namespace {
 
 constexpr int kFixedScratchInts = 65536;  // 256 KiB: nchunks * E <= 65536
 static __device__ __align__(256) int32_t g_fixed_perm_scratch[kFixedScratchInts];
-static __device__ int32_t g_fixed_perm_ticket;
 
 constexpr int kMaxDevices = 64;
 int32_t* g_fixed_scratch_ptr[kMaxDevices] = {nullptr};
 std::mutex g_fixed_scratch_mu;
 
-int32_t* g_fixed_ticket_ptr[kMaxDevices] = {nullptr};
-
-// Device addresses of the arrays on the current device, looked up once per device.
-cudaError_t fixed_scratch_ptr(int32_t** out, int32_t** ticket) {
+// Device address of the array on the current device, looked up once per device.
+cudaError_t fixed_scratch_ptr(int32_t** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -566,14 +540,9 @@ cudaError_t fixed_scratch_ptr(int32_t** out, int32_t** ticket) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_fixed_perm_scratch);
     if (e != cudaSuccess) return e;
-    void* q = nullptr;
-    e = cudaGetSymbolAddress(&q, g_fixed_perm_ticket);
-    if (e != cudaSuccess) return e;
     g_fixed_scratch_ptr[dev] = static_cast<int32_t*>(p);
-    g_fixed_ticket_ptr[dev] = static_cast<int32_t*>(q);
   }
   *out = g_fixed_scratch_ptr[dev];
-  *ticket = g_fixed_ticket_ptr[dev];
   return cudaSuccess;
 }
 
@@ -590,11 +559,9 @@ extern "C" moe_status moe_permute_fixed_scratch(const int32_t* topk_idx, int64_t
   const int64_t nchunks = (S + kChunk - 1) / kChunk;
   if (nchunks * (int64_t)E > kFixedScratchInts) return MOE_ERR_WORKSPACE;  // beyond the fixed capacity
   int32_t* scratch = nullptr;
-  int32_t* ticket = nullptr;
-  if (fixed_scratch_ptr(&scratch, &ticket) != cudaSuccess) return MOE_ERR_CUDA;
+  if (fixed_scratch_ptr(&scratch) != cudaSuccess) return MOE_ERR_CUDA;
   PermuteScratch ps;
   ps.chunk_counts = scratch;
-  ps.ticket = ticket;
   ps.nchunks = (int)nchunks;
   return launch_permute(topk_idx, S, k, E, offsets, perm_token, inv_perm, ps, dev_status,
                         reinterpret_cast<cudaStream_t>(stream), nullptr, nullptr) == cudaSuccess
