@@ -197,7 +197,8 @@ PROFILE_RANGE = False
 
 # Sources the grouped GEMM is built from; a stored ncu traffic figure counts
 # only while they are unchanged.
-GEMM_SOURCES = ("gemm_tc.cu", "gemm_tc.cuh", "tc_ptx.cuh", "common.cuh", "kernels.cuh", "token_quant.cuh")
+GEMM_SOURCES = ("gemm_tc.cu", "gemm_tc.cuh", "tc_ptx.cuh", "common.cuh", "kernels.cuh", "token_quant.cuh",
+                "topk_warp.cuh")
 
 
 def gemm_sources_sha256() -> str:

@@ -456,14 +456,6 @@ moe_status moe_get_device_status(void* ws, moe_stream_t stream, int32_t* host_st
  *                     number at least half the SMs, E % 16 == 0,
  *                     16 <= E <= 256, H % 64 == 0 and k <= 16; 0 keeps the
  *                     logits kernel and the separate top-k kernel.
- *   MOE_OPT_GATHER_ROWS: 1 (default) lets moe_forward, when the gate|up
- *                     projection runs on the grouped tensor-core GEMM with
- *                     single-CTA tiles (not the one-kernel FFN, not CTA
- *                     pairs), NVFP4 / MXFP4 / FP8 weights and H % 64 == 0,
- *                     quantise each token's x once and have the GEMM gather
- *                     its token rows (four rows per tensor copy) instead of
- *                     writing the codes to all k slot rows; the results are
- *                     the same bits.  0 keeps the k copies.
  *   MOE_OPT_FFN_SCHEDULE: 0 (default) the one-kernel FFN's CTAs take work
  *                     items from a counter; 1 CTA b runs items b, b + grid,
  *                     ... -- for measurement only: a down item may then wait
@@ -482,8 +474,7 @@ typedef enum {
   MOE_OPT_SMALL_BATCH_FORWARD = 10,
   MOE_OPT_GATHER_X = 11,
   MOE_OPT_FFN_SCHEDULE = 12,
-  MOE_OPT_ROUTER_TOPK = 13,
-  MOE_OPT_GATHER_ROWS = 14
+  MOE_OPT_ROUTER_TOPK = 13
 } moe_option;
 moe_status moe_set_option(int32_t option, int32_t value);
 

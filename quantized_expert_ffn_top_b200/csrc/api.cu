@@ -52,7 +52,6 @@ static int g_fused_combine = 0;  // MOE_OPT_FUSED_COMBINE
 static int g_small_forward = 0;  // MOE_OPT_SMALL_BATCH_FORWARD
 static int g_gather_x = 0;       // MOE_OPT_GATHER_X
 static int g_router_topk = 1;    // MOE_OPT_ROUTER_TOPK
-static int g_gather_rows = 0;    // MOE_OPT_GATHER_ROWS
 static int g_ffn_schedule = 0;   // MOE_OPT_FFN_SCHEDULE
 static int g_perm_quant = 1;  // MOE_OPT_PERMUTE_QUANT
 
@@ -419,11 +418,6 @@ moe_status run_gemm_ffn(const uint16_t* x, int64_t T, int64_t S, const int32_t* 
   const bool one_kernel = ffn_one_kernel(w, S);
   // small batches on the one-kernel FFN: x in the gather layout
   const bool gather = one_kernel && !x_ready && gather_x(w, T, S);
-  // larger batches with the token quantiser: each token's codes once, the
-  // gate|up GEMM gathering its token rows (single-CTA tiles; the quantiser
-  // takes H % 64 == 0)
-  const bool gather_rows = g_gather_rows && !one_kernel && inv && fmt != MOE_FMT_BF16 && H % 64 == 0 &&
-                           !gemm_pairs_for(fmt, 2 * w->I, H, sms);
   if (x_ready && (!one_kernel || !slot_expert || !planned)) return MOE_ERR_INVALID_ARG;
   if (out32 && one_kernel) return MOE_ERR_INVALID_ARG;
   if (out32 && topk_w && (!inv || fmt == MOE_FMT_BF16 || H % 64 != 0)) return MOE_ERR_INVALID_ARG;
@@ -468,7 +462,6 @@ moe_status run_gemm_ffn(const uint16_t* x, int64_t T, int64_t S, const int32_t* 
     qa.amax = x_amax;
     qa.codes = f.xq;
     qa.sf = f.xsf;
-    qa.codes_tok = gather_rows ? f.xq : nullptr;   // [T][row bytes]: T <= P rows fit
     qa.status = status;
     qa.zero = one_kernel ? f.counters : nullptr;
     qa.nzero = one_kernel ? ncounters : 0;
@@ -484,11 +477,6 @@ moe_status run_gemm_ffn(const uint16_t* x, int64_t T, int64_t S, const int32_t* 
   g.w_early = ew == 0 ? 0 : ((planned || inv) ? 1 : 2);
   g.w_early_l2 = ew == 2 ? kEarlyL2Stages : 0;
   g.offsets = offsets;
-  if (gather_rows) {
-    g.gather_tok = perm;
-    g.b_tok = f.xq;
-    g.b_tok_rows = T;
-  }
   d.w_early = ew == 0 ? 0 : 1;  // the tile list is at least two kernels back
   d.w_early_l2 = g.w_early_l2;
   d.out32 = out32;
@@ -768,11 +756,6 @@ moe_status moe_set_option(int32_t option, int32_t value) {
   if (option == MOE_OPT_GATHER_X) {
     if (value != 0 && value != 1) return MOE_ERR_INVALID_ARG;
     g_gather_x = value;
-    return MOE_OK;
-  }
-  if (option == MOE_OPT_GATHER_ROWS) {
-    if (value != 0 && value != 1) return MOE_ERR_INVALID_ARG;
-    g_gather_rows = value;
     return MOE_OK;
   }
   if (option == MOE_OPT_ROUTER_TOPK) {

@@ -665,37 +665,13 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN, PAIR>::kThreads, 1)
     int stage = 0;
     uint32_t phase = 0;
     int issued = 0;  // stages issued by this loop; the first n_pre hold early weight loads
-    // Gathered token rows: lane l issues the tensor copies of row quads l and
-    // l + 32 (rows 4q .. 4q + 3) and holds their tokens, read one tile ahead;
-    // rows past the tile's valid ones repeat its last token.
-    constexpr bool kGatherForm = (EPI == kEpiUpQuant || EPI == kEpiUpF32) && !PAIR && FMT != kFmtBF16;
-    constexpr int kQuads = (BN / 4 + 31) / 32;
-    const bool gath = kGatherForm && g.gather_tok != nullptr;
-    int gt[kQuads][4], gt_next[kQuads][4];
-    auto gather_tokens = [&](const TileEntry& e, int (&out)[kQuads][4]) {
-#pragma unroll
-      for (int h = 0; h < kQuads; ++h)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int r = 4 * (lane + 32 * h) + j, n = min(e.nvalid, BN);
-          out[h][j] = (gath && n > 0 && 4 * (lane + 32 * h) < n) ? __ldg(g.gather_tok + e.p0 + min(r, n - 1)) : 0;
-        }
-    };
     // each tile's entry is read one tile ahead, off the critical path
     TileEntry te_next = t_first < ntiles ? tile_at((t_first / ksplit) / MT) : TileEntry{};
-    if (gath && t_first < ntiles) gather_tokens(te_next, gt_next);
     for (int t = t_first; t < ntiles && !tc::aborted(abort); t += t_step) {
       const int tt = t / ksplit, split = t % ksplit;
       const int kb0 = split * nkb / ksplit, kb1 = (split + 1) * nkb / ksplit;
       const TileEntry te = te_next;
-#pragma unroll
-      for (int h = 0; h < kQuads; ++h)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) gt[h][j] = gt_next[h][j];
-      if (t + t_step < ntiles) {
-        te_next = tile_at(((t + t_step) / ksplit) / MT);
-        if (gath) gather_tokens(te_next, gt_next);
-      }
+      if (t + t_step < ntiles) te_next = tile_at(((t + t_step) / ksplit) / MT);
       const int mt = PAIR ? (tt % MT) * 2 + (int)rank : tt % MT;   // this CTA's 128-row weight block
       const uint8_t* sfa = F::kBs ? g.w_sf + (size_t)te.e * g.R * ncols_w + (size_t)mt * (ncols_w / 4) * 512 : nullptr;
       for (int kb = kb0; kb < kb1; ++kb) {
@@ -725,40 +701,24 @@ __global__ void __launch_bounds__(Cfg<FMT, EPI, BN, PAIR>::kThreads, 1)
               tc::tma_load_2d_pair(st + C::kA + C::kB + C::kSFA + nb * F::kGroups * 512, &tmap_sfb, cbar, 0,
                                    (te.row0 / 128 + nb) * (ncols_w / 4) + kb * F::kGroups);
           }
-        } else if (!PAIR) {
+        } else if (!PAIR && tc::elect_one()) {
           uint8_t* st = smem + stage * C::kStage;
-          const int nquads = (min(te.nvalid, BN) + 3) >> 2;   // gathered row quads
-          if (tc::elect_one()) {
-            const int bi = token_box_index(min(te.nvalid, BN));
-            const uint32_t brows = min(16u << bi, (uint32_t)BN);   // the map's box height
-            const uint32_t bbytes = gath ? (uint32_t)nquads * 512u : brows * 128u;
-            const int nblk = ((te.row0 & 127) + min(te.nvalid, BN) + 127) / 128;   // 128-row scale blocks in use
-            const bool early = issued < n_pre;   // weights already in flight (stage == issued)
-            if (early && pre_e[issued] != te.e) raise_status(g.status, MOE_ERR_DEVICE_FAULT);
-            tc::mbar_expect_tx(&full[stage], (early ? 0u : (uint32_t)(C::kA + C::kSFA)) + bbytes +
-                                                 nblk * F::kGroups * 512);
-            if (!early) tc::tma_load_2d(st, &tmap_a, &full[stage], kb * 128, te.e * g.R + mt * 128);
-            if (!gath) tc::tma_load_2d(st + C::kA, &tmaps_b.m[bi], &full[stage], kb * 128, te.row0);
-            if (F::kBs) {
-              if (!early)
-                tc::bulk_load(st + C::kA + C::kB, sfa + (size_t)kb * F::kGroups * 512, C::kSFA, &full[stage]);
-              for (int nb = 0; nb < nblk; ++nb) {
-                const uint8_t* sfb =
-                    g.b_sf + ((size_t)(te.row0 / 128 + nb) * (ncols_w / 4) + (size_t)kb * F::kGroups) * 512;
-                tc::bulk_load(st + C::kA + C::kB + C::kSFA + nb * F::kGroups * 512, sfb, F::kGroups * 512,
-                              &full[stage]);
-              }
-            }
-          }
-          __syncwarp();
-          if (kGatherForm && gath) {
-            // the stage's bytes are expected above; each lane copies its quads
-#pragma unroll
-            for (int h = 0; h < kQuads; ++h) {
-              const int q4 = lane + 32 * h;
-              if (q4 < nquads)
-                tc::tma_gather4(st + C::kA + q4 * 512, &tmaps_b.m[0], &full[stage], kb * 128, gt[h][0], gt[h][1],
-                                gt[h][2], gt[h][3]);
+          const int bi = token_box_index(min(te.nvalid, BN));
+          const uint32_t brows = min(16u << bi, (uint32_t)BN);   // the map's box height
+          const int nblk = ((te.row0 & 127) + min(te.nvalid, BN) + 127) / 128;   // 128-row scale blocks in use
+          const bool early = issued < n_pre;   // weights already in flight (stage == issued)
+          if (early && pre_e[issued] != te.e) raise_status(g.status, MOE_ERR_DEVICE_FAULT);
+          tc::mbar_expect_tx(&full[stage], (early ? 0u : (uint32_t)(C::kA + C::kSFA)) + brows * 128u +
+                                               nblk * F::kGroups * 512);
+          if (!early) tc::tma_load_2d(st, &tmap_a, &full[stage], kb * 128, te.e * g.R + mt * 128);
+          tc::tma_load_2d(st + C::kA, &tmaps_b.m[bi], &full[stage], kb * 128, te.row0);
+          if (F::kBs) {
+            if (!early) tc::bulk_load(st + C::kA + C::kB, sfa + (size_t)kb * F::kGroups * 512, C::kSFA, &full[stage]);
+            for (int nb = 0; nb < nblk; ++nb) {
+              const uint8_t* sfb =
+                  g.b_sf + ((size_t)(te.row0 / 128 + nb) * (ncols_w / 4) + (size_t)kb * F::kGroups) * 512;
+              tc::bulk_load(st + C::kA + C::kB + C::kSFA + nb * F::kGroups * 512, sfb, F::kGroups * 512,
+                            &full[stage]);
             }
           }
         }
@@ -1666,12 +1626,6 @@ cudaError_t launch_cfg(const GemmArgs& g, const void* a_base, int64_t a_rows, co
   constexpr int kBRows = PAIR ? BN / 2 : BN;
   for (int i = 0; i < 5; ++i)
     if (!make_map(&mb.m[i], b_base, b_rows, rb, (16 << i) < kBRows ? (16 << i) : kBRows)) return cudaErrorInvalidValue;
-  if (g.gather_tok) {
-    // gathered token rows: one row per token, box one row high
-    if (PAIR || FMT == kFmtBF16 || (EPI != kEpiUpQuant && EPI != kEpiUpF32) || !g.b_tok || g.b_tok_rows < 1)
-      return cudaErrorInvalidValue;
-    if (!make_map(&mb.m[0], g.b_tok, g.b_tok_rows, rb, 1)) return cudaErrorInvalidValue;
-  }
   if (PAIR && F::kBs) {
     const int64_t groups = g.K / F::kBs / 4;  // 512-byte blocks per 128 rows
     if (!make_sf_map(&msfa, g.w_sf, a_rows / 128 * groups, F::kGroups)) return cudaErrorInvalidValue;
@@ -1723,17 +1677,12 @@ cudaError_t launch_cfg(const GemmArgs& g, const void* a_base, int64_t a_rows, co
   return cudaGetLastError();
 }
 
-bool pairs_for(int fmt, int R, int K, int num_sms) {
-  if (fmt == kFmtBF16 || R % 256 != 0 || num_sms < 2) return false;   // (no pair form of the bf16 MMA here)
-  const int bk = fmt == MOE_FMT_FP8 ? FmtTraits<MOE_FMT_FP8>::kBK : FmtTraits<MOE_FMT_NVFP4>::kBK;
-  return g_gemm_pairs == 1 || (g_gemm_pairs == 2 && K / bk >= kPairMinStages);
-}
-
 template <int FMT, int EPI>
 cudaError_t launch_bn(const GemmArgs& g, int bn, const void* a, int64_t ar, const void* b, int64_t br, int sms,
                       cudaStream_t s) {
-  if constexpr (FMT != kFmtBF16) {
-    const bool pairs = EPI != kEpiLogits && !g.gather_tok && pairs_for(FMT, g.R, g.K, sms);
+  if constexpr (FMT != kFmtBF16) {   // (no pair form of the bf16 MMA here)
+    const bool pairs = EPI != kEpiLogits && g.R % 256 == 0 && sms >= 2 &&
+                       (g_gemm_pairs == 1 || (g_gemm_pairs == 2 && g.K / FmtTraits<FMT>::kBK >= kPairMinStages));
     if (bn == 256 && pairs) return launch_cfg<FMT, EPI, 256, true>(g, a, ar, b, br, sms, s);
     if (bn == 192 && pairs) return launch_cfg<FMT, EPI, 192, true>(g, a, ar, b, br, sms, s);
   }
@@ -2062,8 +2011,6 @@ bool tensor_maps_available() { return encode_fn() != nullptr; }
 long long tc_default_wait_cycles() { return tc::kDefaultWaitCycles; }
 
 void set_gemm_pairs(int mode) { g_gemm_pairs = mode; }
-
-bool gemm_pairs_for(int fmt, int R, int K, int num_sms) { return pairs_for(fmt, R, K, num_sms); }
 
 static int g_early_weights = 1;  // MOE_OPT_EARLY_WEIGHTS
 void set_early_weights(int mode) { g_early_weights = mode; }
@@ -2406,10 +2353,7 @@ __global__ void __launch_bounds__(256) quant_tokens_kernel(QuantPaddedArgs a) {
   };
   for (int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < a.T; t += warps)
     quant_token_slots<FMT>(a.x + t * a.K, a.K, a.k, scale, r_tab, tbuf[threadIdx.x >> 5],
-                           [&](int j) { return resolve(t, j); }, a.codes, a.sf, a.status,
-                           a.codes_tok ? a.codes_tok + t * ((int64_t)a.K * TokenQuant<FMT>::kLaneBytes /
-                                                             TokenQuant<FMT>::kPer)
-                                       : nullptr);
+                           [&](int j) { return resolve(t, j); }, a.codes, a.sf, a.status);
 }
 
 // x of a small batch into the gather layout (quant_token_gather): a warp per

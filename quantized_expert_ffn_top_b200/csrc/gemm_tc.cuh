@@ -57,13 +57,6 @@ struct GemmArgs {
   // is the previous kernel's output; offsets are older; E <= 256, else no
   // early loads).  0: off.
   int w_early;
-  // up projection, gathered token rows (single-CTA tiles): tile row r's codes
-  // are row gather_tok[p0 + r] of b_tok ([b_tok_rows][row bytes], one row
-  // per token), loaded four rows per tensor copy; its scales still come from
-  // b_sf over padded rows
-  const int32_t* gather_tok;
-  const void* b_tok;
-  int64_t b_tok_rows;
   int w_early_l2;              // and this many further stages' weights prefetched to L2
   const int32_t* offsets;      // [E+1] compact expert offsets (w_early == 2; E <= 256)
   int max_tiles;               // entries allocated in `tiles`
@@ -84,8 +77,6 @@ struct QuantPaddedArgs {
   const float* topk_w;         //   optional with it: weight of each (token, j); then
   float* w_perm;               //   w_perm[slot position] receives it
   PlanOut plan;                // per-slot x quantiser: also compute (and write) the tile plan
-  uint8_t* codes_tok;          // optional with inv_perm: each token's codes once, row t (the slots'
-                               //   scales still go to their padded rows)
   int32_t* zero;               // optional: nzero counters set to 0 (by block 0, after the wait)
   int nzero;
   const uint16_t* x;           // [T][K] bf16
@@ -170,9 +161,6 @@ int router_ksplit(int64_t T, int E, int H, int num_sms);
 // side, every expert on its N side, the top-k kept per token in registers by
 // the epilogue.  logits_out (nullable) receives the logits.
 bool router_topk_fits(int64_t T, int E, int H, int k, int num_sms);
-// Whether the grouped GEMM runs R weight rows with reduction length K on CTA
-// pairs (MOE_OPT_GEMM_PAIR); gathered token rows need single-CTA tiles.
-bool gemm_pairs_for(int fmt, int R, int K, int num_sms);
 // Logits and top-k in one kernel, for batches whose 128-token tiles fill at
 // least half the SMs (router_topk_fits).
 cudaError_t launch_router_topk(const uint16_t* x, int64_t T, int H, const uint16_t* wr, const float* bias, int E,

@@ -146,17 +146,6 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* m, uin
       "l"(m), "r"(x), "r"(y), "r"(smem_u32(bar))
       : "memory");
 }
-// Four rows y0..y3 of a 2D map whose box is one row high, columns from x,
-// into four consecutive box rows at dst (the map's swizzle applies as for a
-// four-row box there).
-__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* m, uint64_t* bar, int x, int y0, int y1,
-                                            int y2, int y3) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes [%0], "
-      "[%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_u32(dst)),
-      "l"(m), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3), "r"(smem_u32(bar))
-      : "memory");
-}
 // The same load into this CTA's shared memory, completing on an mbarrier
 // given by its cluster address, which may be the pair leader's (cta_group::2).
 __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* m, uint32_t cbar, int x, int y) {

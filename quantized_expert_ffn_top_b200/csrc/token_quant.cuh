@@ -41,14 +41,11 @@ struct TokenQuant {
 // (the slot is skipped and the status word raised).  tb: the warp's reorder
 // buffer (TokenQuant<FMT>::kWarpBuf uint4 of shared memory); r_tab: the NVFP4
 // multipliers of the 128 non-negative scale codes for this scale.
-// tok_codes (nullable): the token's codes go there once, in the same row
-// layout, instead of to every slot row (the slots' block scales still go to
-// their padded rows) -- for a GEMM that gathers its token rows.
 template <int FMT, class RowOf>
 __device__ __forceinline__ void quant_token_slots(const uint16_t* __restrict__ xt, int K, int k, float scale,
                                                   const float* r_tab, uint4* tb, RowOf&& row_of,
                                                   uint8_t* __restrict__ codes, uint8_t* __restrict__ sf,
-                                                  int32_t* status, uint8_t* __restrict__ tok_codes = nullptr) {
+                                                  int32_t* status) {
   using Q = TokenQuant<FMT>;
   constexpr int bs = Q::kBs, kPer = Q::kPer, kWords = Q::kWords, kLaneBytes = Q::kLaneBytes, kVec = Q::kVec;
   const int nb = K / bs;
@@ -134,12 +131,6 @@ __device__ __forceinline__ void quant_token_slots(const uint16_t* __restrict__ x
       wc[v] = off < seg ? tb[off / 16] : make_uint4(0, 0, 0, 0);
     }
     __syncwarp();
-    if (tok_codes) {
-      uint4* dst = reinterpret_cast<uint4*>(tok_codes + (int64_t)c0 * kLaneBytes / kPer);
-#pragma unroll
-      for (int v = 0; v < kVec; ++v)
-        if (512 * v + 16 * lane < seg) dst[(512 * v) / 16 + lane] = wc[v];
-    }
     for (int j0 = 0; j0 < k; j0 += 32) {
       // lane j holds the padded row of slot j0 + j
       const int64_t myrow = (j0 == 0) ? row_first : (j0 + lane < k ? row_of(j0 + lane) : -1);
@@ -150,13 +141,11 @@ __device__ __forceinline__ void quant_token_slots(const uint16_t* __restrict__ x
           if (row == -2 && lane == 0 && c0 == 0) raise_status(status, MOE_ERR_DEVICE_FAULT);
           continue;
         }
-        if (!tok_codes) {
-          uint4* dst = reinterpret_cast<uint4*>(codes + row * ((int64_t)K * kLaneBytes / kPer) +
-                                                (int64_t)c0 * kLaneBytes / kPer);
+        uint4* dst = reinterpret_cast<uint4*>(codes + row * ((int64_t)K * kLaneBytes / kPer) +
+                                              (int64_t)c0 * kLaneBytes / kPer);
 #pragma unroll
-          for (int v = 0; v < kVec; ++v)
-            if (512 * v + 16 * lane < seg) dst[(512 * v) / 16 + lane] = wc[v];
-        }
+        for (int v = 0; v < kVec; ++v)
+          if (512 * v + 16 * lane < seg) dst[(512 * v) / 16 + lane] = wc[v];
         if (!active) continue;
         if constexpr (FMT == MOE_FMT_NVFP4)
           *reinterpret_cast<uint32_t*>(sf + sf_blocked_offset(row, c / bs, nb)) = sfw;

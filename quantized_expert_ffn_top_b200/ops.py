@@ -33,7 +33,6 @@ OPT_SMALL_BATCH_FORWARD = 10
 OPT_GATHER_X = 11
 OPT_FFN_SCHEDULE = 12
 OPT_ROUTER_TOPK = 13
-OPT_GATHER_ROWS = 14
 FMT_BY_NAME = {"nvfp4": FMT_NVFP4, "mxfp4": FMT_MXFP4, "fp8": FMT_FP8, "bf16": FMT_BF16}
 
 

@@ -363,51 +363,6 @@ def test_forward_matches_oracle(name, over, act, static):
     assert err < TOL, err
 
 
-# larger batches on the grouped GEMM: each token's x quantised once and its
-# rows gathered by the gate|up GEMM (four per tensor copy) against the codes
-# written to all k slot rows -- the same codes and scales, so the same bits;
-# and the gathered form against the oracle.  NVFP4 with static scales (the
-# prefill layer), dynamic scales (fp32 h, the gate|up GEMM's other epilogue),
-# MXFP4, FP8 (K below the CTA-pair length), ragged tiles with few experts.
-GATHER_ROWS_CASES = [
-    ("prefill", {}, "static"),
-    ("prefill", dict(T=1000), "none"),
-    ("tiny", dict(fmt="mxfp4", T=700, H=2048, E=16, k=4, I=512), "none"),
-    ("tiny", dict(fmt="fp8", T=600, H=1024, E=8, k=2, I=512), "none"),
-    ("tiny", dict(T=333, H=512, E=4, k=2, I=256), "static"),
-]
-
-
-@pytest.mark.parametrize("name,over,scales", GATHER_ROWS_CASES)
-def test_gathered_token_rows_give_the_same_bits(name, over, scales):
-    w = synth.workload(name, **over)
-    W, _ = oracle_bank(w)
-    a13, a2 = synth.static_act_scales()
-    if scales == "none" or w.fmt == "mxfp4":
-        a13 = a2 = None
-    bank = device_bank(W, a13, a2)
-    x, wr, b = routed_inputs(w)
-    xd, wrd = bits_to_dev_bf16(x), bits_to_dev_bf16(wr)
-    bd = None if b is None else torch.from_numpy(b).cuda()
-    W_ = ws(ops.workspace_size(w.T, w.k, bank, None, 1))
-    outs = []
-    try:
-        for opt in (0, 1):
-            ops.moe_set_option(ops.OPT_GATHER_ROWS, opt)
-            out = ops.moe_forward(xd, wrd, bd, w.k, bank, None, 1, W_)
-            assert ops.moe_get_device_status(W_) == 0, opt
-            outs.append(out.view(torch.int16).cpu().numpy())
-    finally:
-        ops.moe_set_option(ops.OPT_GATHER_ROWS, 1)
-    assert np.array_equal(outs[0], outs[1])
-    tokens = np.linspace(0, w.T - 1, min(w.T, 256)).astype(np.int64) if (a13 is not None or w.fmt == "mxfp4") else None
-    r, keep = forward_reference(w, x, wr, b, W, act=1, a13=a13, a2=a2, tokens=tokens, what=f"gather rows {name}")
-    got = (outs[1].view(np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
-    if tokens is not None:
-        got = got[tokens]
-    assert max_abs_rel(got[keep], r["out"][keep]) < TOL
-
-
 # small batches (T <= 8) on the one-kernel FFN (tensor-core shapes: H and I
 # multiples of 256): x quantised inside the permutation kernel (NVFP4 static
 # and dynamic x scales; MXFP4 with a ragged second 2048-value stretch and at

@@ -37,8 +37,8 @@ def test_fixed_scratch_permute_matches_workspace_permute_twice():
     assert torch.cuda.is_available()
     ws = ops.new_workspace(1 << 22)
     # both calls take the multi-block path (more than 8192 slots), which is the
-    # one that uses the fixed array and its ticket: 16 chunks x 128 experts,
-    # then 6 chunks x 60 experts in the same array
+    # one that uses the fixed array: 16 chunks x 128 experts, then 6 chunks x
+    # 60 experts in the same array
     cases = [(4096, 8, 128, 1.1, 0), (3000, 4, 60, 0.3, 1)]
     for T, k, E, skew, seed in cases:
         idx = torch.from_numpy(synth.random_topk_idx(T, k, E, seed=seed, skew=skew)).cuda()
