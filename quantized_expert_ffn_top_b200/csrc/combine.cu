@@ -56,7 +56,7 @@ __global__ void __launch_bounds__(kCombineThreads, 4) combine_kernel(const uint1
       for (int u = 0; u < 8; ++u) {
         pj[u] = __shfl_sync(0xffffffffu, pl, (jb + u) & 31);
         if (jb + u >= nj) pj[u] = -1;
-        v[u] = (active && pj[u] >= 0) ? __ldg(reinterpret_cast<const uint4*>(y_perm + (int64_t)pj[u] * H + c))
+        v[u] = (active && pj[u] >= 0) ? __ldcs(reinterpret_cast<const uint4*>(y_perm + (int64_t)pj[u] * H + c))
                                       : make_uint4(0, 0, 0, 0);
       }
 #pragma unroll

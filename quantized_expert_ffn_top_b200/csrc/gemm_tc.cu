@@ -407,7 +407,7 @@ __device__ __forceinline__ void epilogue_slice(const GemmArgs& g, const CUtensor
         tc::fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          tc::tma_store_2d(tmap_y, stg, mt * 128 + q * 32, te.p0 + c0);
+          tc::tma_store_2d_keep(tmap_y, stg, mt * 128 + q * 32, te.p0 + c0, tc::l2_policy_evict_last());
           tc::bulk_commit();
         }
       } else {
