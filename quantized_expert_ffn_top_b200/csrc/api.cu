@@ -421,7 +421,8 @@ moe_status run_gemm_ffn(const uint16_t* x, int64_t T, int64_t S, const int32_t* 
   if (x_ready && (!one_kernel || !slot_expert || !planned)) return MOE_ERR_INVALID_ARG;
   if (out32 && one_kernel) return MOE_ERR_INVALID_ARG;
   if (out32 && topk_w && (!inv || fmt == MOE_FMT_BF16 || H % 64 != 0)) return MOE_ERR_INVALID_ARG;
-  if (mark) stage_mark(MOE_STAGE_ACT_QUANT, false, s);
+  // (with x_ready the permutation kernel quantised x: no stage of its own)
+  if (mark && !x_ready) stage_mark(MOE_STAGE_ACT_QUANT, false, s);
   // the x quantiser clears the one-kernel FFN's counters (with x_ready, the
   // permutation kernel did)
   const int ncounters = (int)(counters_bytes(S, E) / sizeof(int32_t));
@@ -467,7 +468,7 @@ moe_status run_gemm_ffn(const uint16_t* x, int64_t T, int64_t S, const int32_t* 
     qa.nzero = one_kernel ? ncounters : 0;
     if (!x_ready) MOE_TRY(launch_quant_padded(qa, true, fmt, sms, s));
   }
-  if (mark) stage_mark(MOE_STAGE_ACT_QUANT, true, s);
+  if (mark && !x_ready) stage_mark(MOE_STAGE_ACT_QUANT, true, s);
   GemmArgs g, d;
   ffn_gemm_args(w, f, S, x_amax, h_amax, status, fused_h, y_perm, g, d);
   // the tile list is two kernels back when the permutation or the plan kernel
@@ -506,11 +507,7 @@ moe_status run_gemm_ffn(const uint16_t* x, int64_t T, int64_t S, const int32_t* 
     }
     if (mark) stage_mark(MOE_STAGE_FFN_UP, false, s);
     MOE_TRY(launch_fused_ffn(g, d, fa, w->w13, (int64_t)E * 2 * w->I, w->w2, (int64_t)E * H, f.xq, f.hq, sms, s));
-    if (mark) {
-      stage_mark(MOE_STAGE_FFN_UP, true, s);
-      stage_mark(MOE_STAGE_FFN_DOWN, false, s);
-      stage_mark(MOE_STAGE_FFN_DOWN, true, s);
-    }
+    if (mark) stage_mark(MOE_STAGE_FFN_UP, true, s);   // both projections: no separate down stage
     return MOE_OK;
   }
   if (mark) stage_mark(MOE_STAGE_FFN_UP, false, s);
