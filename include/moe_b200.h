@@ -433,8 +433,9 @@ moe_status moe_get_device_status(void* ws, moe_stream_t stream, int32_t* host_st
  *                     bf16 y_perm and the ordered combine of moe_combine,
  *                     which is bit-reproducible (the default: the reductions
  *                     measured slower than the bf16 round trip).
- *   MOE_OPT_SMALL_BATCH_FORWARD: 1 runs moe_forward at T <= 32 on
- *                     the one-kernel FFN (NVFP4 with a static h scale, or
+ *   MOE_OPT_SMALL_BATCH_FORWARD: 1 (with MOE_OPT_GATHER_X = 1) runs
+ *                     moe_forward at T <= 32 on the one-kernel FFN (NVFP4
+ *                     with a static h scale, or
  *                     MXFP4; H % 256 == 0; E <= 256) with no shared expert as
  *                     two kernels: the router (logits, x quantised into a
  *                     layout the FFN copies token rows from, top-k in its

@@ -141,6 +141,20 @@ def test_wait_bound_option(L):
     assert re.search(r"MOE_OPT_WAIT_CYCLES = (\d+)", hdr).group(1) == str(ops.OPT_WAIT_CYCLES)
 
 
+def test_switch_options_take_0_or_1_and_match_the_header(L):
+    """The on/off switches added with the routing and small-batch paths
+    accept 0 and 1, reject anything else, and carry the header's numbers;
+    each is put back to its default."""
+    hdr = open(os.path.join(ROOT, "include", "moe_b200.h")).read()
+    defaults = {"FUSED_COMBINE": 0, "SMALL_BATCH_FORWARD": 0, "GATHER_X": 0, "FFN_SCHEDULE": 0, "ROUTER_TOPK": 1}
+    for name, default in defaults.items():
+        opt = getattr(ops, "OPT_" + name)
+        assert re.search(r"^\s+MOE_OPT_%s = (\d+),?\s*$" % name, hdr, re.M).group(1) == str(opt), name
+        assert L.moe_set_option(opt, 2) == 1 and L.moe_set_option(opt, -1) == 1, name
+        assert L.moe_set_option(opt, 1 - default) == 0, name
+        assert L.moe_set_option(opt, default) == 0, name
+
+
 @pytest.mark.parametrize("E,H,I,k", [(128, 128, 256, 2), (256, 4096, 2048, 8), (8, 256, 256, 2)])
 def test_workspace_size_never_decreases_with_T(L, E, H, I, k):
     """A workspace sized for T serves every smaller batch: moe_forward_host
