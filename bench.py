@@ -529,6 +529,16 @@ def max_over_ranks(value: float, device="cuda") -> float:
     return float(t.item())
 
 
+def _round_floats(v, digits: int = 4):
+    if isinstance(v, float):
+        return float(f"{v:.{digits}g}")
+    if isinstance(v, dict):
+        return {k: _round_floats(x, digits) for k, x in v.items()}
+    if isinstance(v, list):
+        return [_round_floats(x, digits) for x in v]
+    return v
+
+
 def job_throughput(tokens_per_rank: int, steps: int, world: int, slowest_s: float) -> float:
     """Whole-job tokens/s: every replica's tokens over the slowest replica's time."""
     return world * tokens_per_rank * steps / slowest_s
@@ -652,6 +662,11 @@ def main():
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_oracle_sample(w, args.cpu_seconds, static=True)
+    # the per-config and decode blocks at four significant digits, so the
+    # line stays short
+    for key in ("configs", "decode"):
+        if key in line:
+            line[key] = _round_floats(line[key])
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
