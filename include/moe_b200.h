@@ -37,8 +37,13 @@
  *    uninitialised.  A bounded device wait that ran out (MOE_OPT_WAIT_CYCLES)
  *    sets the word to MOE_ERR_TIMEOUT: the kernel that gave up lets its
  *    copies in flight land, frees its tensor memory and returns, and the
- *    later kernels of the call still run, but the outputs of that call are
- *    then unspecified.  moe_get_device_status() reads and clears the word;
+ *    later kernels of the call still run.  The layer's output (moe_forward,
+ *    moe_forward_host, moe_forward_cached, moe_combine) is then written as
+ *    zeros -- the combine reads the word -- except after the two-kernel
+ *    small-batch forward (MOE_OPT_SMALL_BATCH_FORWARD), whose output is then
+ *    unspecified, like the other calls' intermediate outputs.  A word left
+ *    at MOE_ERR_TIMEOUT by an earlier call zeroes the next combine on the
+ *    same workspace too.  moe_get_device_status() reads and clears the word;
  *    the next call on the same workspace starts clean.
  *  - A launch failure returns MOE_ERR_CUDA.
  */

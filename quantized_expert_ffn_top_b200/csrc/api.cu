@@ -1137,7 +1137,7 @@ moe_status moe_forward(const uint16_t* x, int64_t T, const uint16_t* wr, const f
   // 6. combine (or, when the down epilogues did it, the rounding to bf16)
   stage_mark(MOE_STAGE_COMBINE, false, s);
   if (fused_combine)
-    st = cuda_status(launch_round_rows(f.out32, T * (int64_t)H, out, num_sms(), s));
+    st = cuda_status(launch_round_rows(f.out32, T * (int64_t)H, out, f.head.status, num_sms(), s));
   else
     st = cuda_status(launch_combine(f.y_perm, f.inv, f.w, T, k, H, f.sh_y, out, f.head.status, s));
   stage_mark(MOE_STAGE_COMBINE, true, s);

@@ -27,6 +27,12 @@ __global__ void __launch_bounds__(kCombineThreads, 4) combine_kernel(const uint1
   const int lane = threadIdx.x & 31;
   const int c = blockIdx.y * (blockDim.x * 8) + threadIdx.x * 8;
   const bool active = c < H;  // every lane takes part in the shuffles
+  // an earlier kernel of the call gave up on a bounded wait: its outputs
+  // are unspecified, so the layer's output is written as zeros
+  if (status && __ldcg(status) == MOE_ERR_TIMEOUT) {
+    if (active) *reinterpret_cast<uint4*>(out + t * H + c) = make_uint4(0u, 0u, 0u, 0u);
+    return;
+  }
   float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
   auto add = [&](const uint4& v, float wj) {
     const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
@@ -101,9 +107,14 @@ cudaError_t launch_combine(const uint16_t* y_perm, const int32_t* inv_perm, cons
 // rows (the combine in the down epilogue): out = bf16(out32), round to
 // nearest even, eight values a thread.
 __global__ void __launch_bounds__(256) round_rows_kernel(const float* __restrict__ out32, int64_t n8,
-                                                         uint16_t* __restrict__ out) {
+                                                         uint16_t* __restrict__ out, const int32_t* status) {
   pdl_wait();  // inputs come from the previous kernels
   pdl_trigger();
+  if (status && __ldcg(status) == MOE_ERR_TIMEOUT) {   // as in combine_kernel: zeros after a timeout
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += (int64_t)gridDim.x * blockDim.x)
+      reinterpret_cast<uint4*>(out)[i] = make_uint4(0u, 0u, 0u, 0u);
+    return;
+  }
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += (int64_t)gridDim.x * blockDim.x) {
     const float4 a = __ldcs(reinterpret_cast<const float4*>(out32) + 2 * i);
     const float4 b = __ldcs(reinterpret_cast<const float4*>(out32) + 2 * i + 1);
@@ -116,13 +127,14 @@ __global__ void __launch_bounds__(256) round_rows_kernel(const float* __restrict
   }
 }
 
-cudaError_t launch_round_rows(const float* out32, int64_t n, uint16_t* out, int num_sms, cudaStream_t s) {
+cudaError_t launch_round_rows(const float* out32, int64_t n, uint16_t* out, const int32_t* status, int num_sms,
+                              cudaStream_t s) {
   if (n == 0) return cudaSuccess;
   if (n % 8 != 0) return cudaErrorInvalidValue;
   const int64_t n8 = n / 8;
   const int64_t blocks = (n8 + 255) / 256;
   const int grid = (int)(blocks < (int64_t)num_sms * 8 ? blocks : (int64_t)num_sms * 8);
-  cudaError_t e = launch_pdl(round_rows_kernel, dim3(grid), dim3(256), 0, s, out32, n8, out);
+  cudaError_t e = launch_pdl(round_rows_kernel, dim3(grid), dim3(256), 0, s, out32, n8, out, status);
   count_launches(1);
   return e != cudaSuccess ? e : cudaGetLastError();
 }

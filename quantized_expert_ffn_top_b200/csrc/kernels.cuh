@@ -161,7 +161,8 @@ cudaError_t launch_gemv_down(const GemvArgs& a, int num_sms, cudaStream_t s);
 cudaError_t launch_combine(const uint16_t* y_perm, const int32_t* inv_perm, const float* w, int64_t T, int k, int H,
                            const uint16_t* shared_y, uint16_t* out, int32_t* status, cudaStream_t s);
 // out[i] = bf16(out32[i]) for n values (n % 8 == 0, 16-byte aligned).
-cudaError_t launch_round_rows(const float* out32, int64_t n, uint16_t* out, int num_sms, cudaStream_t s);
+cudaError_t launch_round_rows(const float* out32, int64_t n, uint16_t* out, const int32_t* status, int num_sms,
+                              cudaStream_t s);
 
 // cache.cu -- the HBM slot pool in front of a host-memory expert bank.
 // An expert's regions (W13, its scales, W2, its scales) are contiguous in

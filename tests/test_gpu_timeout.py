@@ -4,13 +4,14 @@ Every wait in the tensor-core kernels (the TMA ring, the accumulator
 hand-offs, the one-kernel FFN's wait for a token tile's gate|up slices) gives
 up after MOE_OPT_WAIT_CYCLES SM clocks.  With the bound set to one cycle,
 ordinary waits for memory run out: the call must still return, the device
-status word must read MOE_ERR_TIMEOUT, and the next call on the same
-workspace, with the default bound, must be clean and give the same bits as
-before.  Covered: the one-kernel decode FFN, the 192-token grouped GEMMs on
-single CTAs, and the CTA-pair (cta_group::2) gate|up GEMM of a long K loop.
-Nothing here faults or hangs the GPU: a wait that runs out sets a flag that
-the kernel's other warps see, they leave their loops, the copies in flight
-land and the tensor memory is freed before the kernel returns."""
+status word must read MOE_ERR_TIMEOUT, the timed-out call's output must be
+all zeros, and the next call on the same workspace, with the default bound,
+must be clean and give the same bits as before.  Covered: the one-kernel
+decode FFN, the 192-token grouped GEMMs on single CTAs, and the CTA-pair
+(cta_group::2) gate|up GEMM of a long K loop.  Nothing here faults or hangs
+the GPU: a wait that runs out sets a flag that the kernel's other warps see,
+they leave their loops, the copies in flight land and the tensor memory is
+freed before the kernel returns."""
 import numpy as np
 import pytest
 import torch
@@ -49,12 +50,15 @@ def test_wait_that_runs_out_sets_timeout_and_the_next_call_is_clean(name, base, 
         assert ops.moe_get_device_status(ws) == 0
         try:
             ops.moe_set_option(ops.OPT_WAIT_CYCLES, 1)
-            ops.moe_forward(xd, wrd, bd, w.k, bank, None, ops.ACT_MATCH, ws)
+            bad = ops.moe_forward(xd, wrd, bd, w.k, bank, None, ops.ACT_MATCH, ws)
             torch.cuda.synchronize()            # the call returned and the kernels ended
             st = ops.moe_get_device_status(ws)
         finally:
             ops.moe_set_option(ops.OPT_WAIT_CYCLES, 0)
         assert st == MOE_ERR_TIMEOUT, st
+        # the layer's output after a timeout: zeros, not whatever the
+        # kernels that gave up left behind
+        assert not bad.view(torch.int16).any()
         assert ops.moe_get_device_status(ws) == 0       # read and cleared
         out = ops.moe_forward(xd, wrd, bd, w.k, bank, None, ops.ACT_MATCH, ws)
         assert ops.moe_get_device_status(ws) == 0
