@@ -7,11 +7,11 @@ ordinary waits for memory run out: the call must still return, the device
 status word must read MOE_ERR_TIMEOUT, the timed-out call's output must be
 all zeros, and the next call on the same workspace, with the default bound,
 must be clean and give the same bits as before.  Covered: the one-kernel
-decode FFN, the 192-token grouped GEMMs on single CTAs, and the CTA-pair
-(cta_group::2) gate|up GEMM of a long K loop.  Nothing here faults or hangs
-the GPU: a wait that runs out sets a flag that the kernel's other warps see,
-they leave their loops, the copies in flight land and the tensor memory is
-freed before the kernel returns."""
+decode FFN, the 192-token grouped GEMMs on single CTAs, the CTA-pair
+(cta_group::2) gate|up GEMM of a long K loop and the one-kernel router.
+Nothing here faults or hangs the GPU: a wait that runs out sets a flag that
+the kernel's other warps see, they leave their loops, the copies in flight
+land and the tensor memory is freed before the kernel returns."""
 import numpy as np
 import pytest
 import torch
@@ -30,6 +30,8 @@ CASES = [
     ("prefill-single-cta", "prefill", dict(T=512, E=16)),
     # K = 4096 (16 stages): the gate|up projection on CTA pairs
     ("prefill-cta-pairs", "tiny", dict(T=300, H=4096, E=8, k=2, I=512)),
+    # 128-token tiles for half the SMs and more: the one-kernel router with top-k
+    ("router-topk", "prefill", dict(T=9600)),
 ]
 
 
