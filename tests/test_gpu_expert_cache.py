@@ -4,7 +4,8 @@ in HBM smaller than the bank, whose experts live in page-locked host memory.
 * every batch's output equals the whole-bank forward's (within rounding of
   the combine) and the oracle's (routing replayed exactly at small batches);
 * the counters (experts fetched per call, hits) equal those of the pool's
-  stated policy replayed on the host: the batch's resident experts are hits,
+  stated policy replayed on the host by the oracle's model
+  (oracle/slot_pool.py): the batch's resident experts are hits,
   every other one takes, in expert order, the next slot of the ordering
   "empty slots, then least recently used, ties to the lower slot", among the
   slots no expert of this batch holds;
@@ -15,46 +16,12 @@ import pytest
 import torch
 
 import oracle
+from oracle.slot_pool import SlotPool
 from quantized_expert_ffn_top_b200 import ops, synth
 from tests.gpu_helpers import (TOL, bits_to_dev_bf16, dev_to_f64, device_bank, forward_reference, max_abs_rel,
                                oracle_bank)
 
 pytestmark = pytest.mark.gpu
-
-
-class PoolMirror:
-    """The admit policy on the host: which expert each slot holds."""
-
-    def __init__(self, E, n):
-        self.slot_of = [-1] * E
-        self.expert_of = [-1] * n
-        self.stamp = [0] * n
-        self.clock = 0
-
-    def admit(self, experts):
-        self.clock += 1
-        active = set(int(e) for e in experts)
-        hits = 0
-        for s, e in enumerate(self.expert_of):
-            if e in active:
-                self.stamp[s] = self.clock
-                hits += 1
-        keys = []
-        for s, e in enumerate(self.expert_of):
-            if e in active:
-                continue
-            keys.append((0 if e < 0 else self.stamp[s] + 1, s))
-        keys.sort()
-        misses = sorted(e for e in active if self.slot_of[e] < 0)
-        for r, e in enumerate(misses):
-            v = keys[r][1]
-            old = self.expert_of[v]
-            if old >= 0:
-                self.slot_of[old] = -1
-            self.expert_of[v] = e
-            self.slot_of[e] = v
-            self.stamp[v] = self.clock
-        return len(misses), hits
 
 
 CASES = [
@@ -79,7 +46,7 @@ def test_forward_through_the_slot_pool(name, over, n_slots, static, batches):
     wrd = bits_to_dev_bf16(wr)
     ws_c = ops.new_workspace(ops.workspace_size(w.T, w.k, hbank, None, 1))
     ws_d = ops.new_workspace(ops.workspace_size(w.T, w.k, dbank, None, 1))
-    mirror = PoolMirror(w.E, n_slots)
+    mirror = SlotPool(w.E, n_slots)
     fetched_total = 0
     seen = set()
     for b in range(batches):
