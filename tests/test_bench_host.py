@@ -74,3 +74,17 @@ def test_workload_label_names_the_sizes():
     assert s.startswith("fp8_shared: T=512 H=2048 E=256 top-8 I=512 FP8 weights, W8A8 activations")
     assert s.endswith("shared expert I=512")
     assert "W4A4" in bench.workload_name(synth.workload("decode"))
+
+
+def test_per_config_figures_are_rounded_but_keep_their_structure():
+    d = {"ms": 0.123456789, "stages_ms": {"route": 0.0247123, "ffn_up": 0.0954}, "n": 7, "name": "x",
+         "list": [1234567.89, 0.000123456]}
+    r = bench._round_floats(d)
+    assert r == {"ms": 0.1235, "stages_ms": {"route": 0.02471, "ffn_up": 0.0954}, "n": 7, "name": "x",
+                 "list": [1235000.0, 0.0001235]}
+    assert isinstance(r["n"], int)
+
+
+def test_job_throughput_counts_every_rank():
+    # value = tokens of all ranks / the slowest rank's time
+    assert bench.job_throughput(4096, 20, 8, 0.02) == 4096 * 20 * 8 / 0.02
