@@ -99,7 +99,7 @@ __global__ void __launch_bounds__(kAdmitThreads) cache_admit_kernel(const int32_
   for (int e0 = 0; e0 < E; e0 += blockDim.x) {
     const int e = e0 + tid;
     const bool miss = e < E && active[e] && c.slot_of[e] < 0;
-    // rank among this round's misses: a block-wide count through shared memory
+    // rank among this pass's misses (experts e0 .. e0 + blockDim.x - 1): a block-wide count through shared memory
     __shared__ int wcount[32];
     const unsigned m = __ballot_sync(0xffffffffu, miss);
     if ((tid & 31) == 0) wcount[tid >> 5] = __popc(m);
