@@ -184,3 +184,18 @@ def test_host_slices_with_a_shorter_last_slice(L):
     # one byte short is rejected on the host, before any CUDA call
     assert L.moe_forward_host(host, T, one, None, 2, ctypes.byref(g), None, 1, host, one, one, n, one,
                               ws_bytes - 1, None) == 3
+
+
+def test_expert_cache_sizing(L):
+    """moe_expert_cache_bytes: 0 for a canonical bank or a slot count outside
+    1 .. min(E, 1024); otherwise at least the PREPARED bytes of n_slots
+    experts, growing with n_slots."""
+    prep = _bank(E=64, H=256, I=256, layout=1)
+    assert L.moe_expert_cache_bytes(ctypes.byref(_bank(E=64, H=256, I=256, layout=0)), 8) == 0
+    assert L.moe_expert_cache_bytes(ctypes.byref(prep), 0) == 0
+    assert L.moe_expert_cache_bytes(ctypes.byref(prep), 65) == 0
+    sizes = [L.moe_expert_cache_bytes(ctypes.byref(prep), n) for n in (1, 8, 32, 64)]
+    assert all(s > 0 for s in sizes) and sizes == sorted(sizes) and len(set(sizes)) == 4
+    for n, s in zip((1, 8, 32, 64), sizes):
+        one = _bank(E=n, H=256, I=256, layout=1)
+        assert s >= L.moe_prepared_weights_size(ctypes.byref(one))
