@@ -52,12 +52,14 @@ STAGES = ("route", "permute", "act_quant", "ffn_up", "ffn_down", "shared", "comb
 
 
 class MoeError(RuntimeError):
+    """A moe_status other than MOE_OK, with the call that returned it."""
     def __init__(self, status: int, where: str):
         super().__init__(f"{where}: {status_string(status)}")
         self.status = status
 
 
 class MoeWeightsC(ctypes.Structure):
+    """The C struct moe_weights: format, sizes, layout and device (or host) pointers."""
     _fields_ = [
         ("fmt", ctypes.c_int32), ("E", ctypes.c_int32), ("H", ctypes.c_int32), ("I", ctypes.c_int32),
         ("layout", ctypes.c_int32),
@@ -68,6 +70,7 @@ class MoeWeightsC(ctypes.Structure):
 
 
 class MoeExpertCacheC(ctypes.Structure):
+    """The C struct moe_expert_cache, filled by moe_expert_cache_init."""
     _fields_ = [
         ("bank", MoeWeightsC), ("pool", MoeWeightsC), ("bank_dev", ctypes.c_void_p * 6),
         ("state", ctypes.c_void_p), ("n_slots", ctypes.c_int32),
@@ -128,6 +131,7 @@ def _declare(L):
 
 
 def status_string(st: int) -> str:
+    """moe_status_string: the name and meaning of a status code."""
     return lib().moe_status_string(int(st)).decode()
 
 
@@ -182,6 +186,7 @@ def _ref(b: WeightBank | None):
 
 
 def workspace_size(T: int, k: int, routed: WeightBank, shared: WeightBank | None = None, act: int = ACT_MATCH) -> int:
+    """moe_workspace_size: bytes of workspace moe_forward (and the stages) need for T tokens."""
     r = routed.struct()
     s = shared.struct() if shared is not None else None
     n = lib().moe_workspace_size(int(T), int(k), ctypes.byref(r), ctypes.byref(s) if s is not None else None,
@@ -197,6 +202,7 @@ def new_workspace(nbytes: int, device=None) -> torch.Tensor:
 
 
 def moe_prepare_weights(bank: WeightBank, stream=None) -> WeightBank:
+    """moe_prepare_weights: a bank in the PREPARED layout (interleaved W13 rows, blocked scales), new device memory."""
     c = bank.struct()
     n = lib().moe_prepared_weights_size(ctypes.byref(c))
     if n == 0:
@@ -269,6 +275,7 @@ def moe_route(x: torch.Tensor, wr: torch.Tensor, bias: torch.Tensor | None, k: i
 
 
 def moe_route_logits(logits: torch.Tensor, k: int, ws: torch.Tensor, stream=None):
+    """moe_route_logits: top-k indices and renormalised weights from fp32 logits [T][E]."""
     T, E = logits.shape
     idx = torch.empty((T, k), dtype=torch.int32, device=logits.device)
     w = torch.empty((T, k), dtype=torch.float32, device=logits.device)
@@ -278,6 +285,7 @@ def moe_route_logits(logits: torch.Tensor, k: int, ws: torch.Tensor, stream=None
 
 
 def moe_permute(topk_idx: torch.Tensor, E: int, ws: torch.Tensor, stream=None):
+    """moe_permute: offsets [E+1], perm_token [S] and inv_perm [S] of the top-k ids [T][k]."""
     T, k = topk_idx.shape
     S = T * k
     offsets = torch.empty(E + 1, dtype=torch.int32, device=topk_idx.device)
@@ -290,6 +298,7 @@ def moe_permute(topk_idx: torch.Tensor, E: int, ws: torch.Tensor, stream=None):
 
 def moe_grouped_ffn(x: torch.Tensor, k: int, perm_token: torch.Tensor, offsets: torch.Tensor, w: WeightBank,
                     act: int, ws: torch.Tensor, y_perm: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """moe_grouped_ffn: the experts' SwiGLU FFN over the permuted slots, y_perm [T*k][H] bf16."""
     T, H = x.shape
     y = y_perm if y_perm is not None else torch.empty((T * k, H), dtype=torch.bfloat16, device=x.device)
     ws_ = w.struct()
@@ -300,6 +309,7 @@ def moe_grouped_ffn(x: torch.Tensor, k: int, perm_token: torch.Tensor, offsets: 
 
 def moe_combine(y_perm: torch.Tensor, inv_perm: torch.Tensor, topk_w: torch.Tensor, ws: torch.Tensor,
                 shared_y: torch.Tensor | None = None, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """moe_combine: out[t] = sum_j w[t,j] y_perm[inv_perm[t*k+j]] (+ shared_y[t]), bf16."""
     T, k = topk_w.shape
     H = y_perm.shape[1]
     o = out if out is not None else torch.empty((T, H), dtype=torch.bfloat16, device=y_perm.device)
@@ -311,6 +321,7 @@ def moe_combine(y_perm: torch.Tensor, inv_perm: torch.Tensor, topk_w: torch.Tens
 def moe_forward(x: torch.Tensor, wr: torch.Tensor, bias: torch.Tensor | None, k: int, routed: WeightBank,
                 shared: WeightBank | None, act: int, ws: torch.Tensor, out: torch.Tensor | None = None,
                 stream=None) -> torch.Tensor:
+    """moe_forward: the whole layer, x [T][H] bf16 -> out [T][H] bf16, on the current stream."""
     T, H = x.shape
     o = out if out is not None else torch.empty((T, H), dtype=torch.bfloat16, device=x.device)
     r = routed.struct()
@@ -366,6 +377,7 @@ def bank_to_host(bank: WeightBank) -> WeightBank:
 
 
 def moe_expert_cache_init(host_bank: WeightBank, n_slots: int, stream=None) -> ExpertCache:
+    """moe_expert_cache_init: an HBM pool of n_slots experts in front of a PREPARED bank in pinned host memory."""
     b = host_bank.struct()
     n = lib().moe_expert_cache_bytes(ctypes.byref(b), int(n_slots))
     if n == 0:
@@ -379,6 +391,7 @@ def moe_expert_cache_init(host_bank: WeightBank, n_slots: int, stream=None) -> E
 
 def moe_forward_cached(x: torch.Tensor, wr: torch.Tensor, bias: torch.Tensor | None, k: int, cache: ExpertCache,
                        act: int, ws: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """moe_forward_cached: the layer through the slot pool (misses fetched from host memory)."""
     T, H = x.shape
     o = out if out is not None else torch.empty((T, H), dtype=torch.bfloat16, device=x.device)
     _check(lib().moe_forward_cached(_p(x), T, _p(wr), _p(bias), k, ctypes.byref(cache.c), act, _p(o), _p(ws),
@@ -387,18 +400,21 @@ def moe_forward_cached(x: torch.Tensor, wr: torch.Tensor, bias: torch.Tensor | N
 
 
 def moe_expert_cache_stats(cache: ExpertCache, stream=None) -> dict:
+    """moe_expert_cache_stats: calls, experts fetched (last call and in total) and hits."""
     v = (ctypes.c_int64 * 4)()
     _check(lib().moe_expert_cache_stats(ctypes.byref(cache.c), _stream(stream), v), "moe_expert_cache_stats")
     return {"calls": int(v[0]), "fetched_last": int(v[1]), "fetched": int(v[2]), "hits": int(v[3])}
 
 
 def moe_get_device_status(ws: torch.Tensor, stream=None) -> int:
+    """moe_get_device_status: the workspace's device status word (synchronises; clears it)."""
     v = ctypes.c_int32(0)
     _check(lib().moe_get_device_status(_p(ws), _stream(stream), ctypes.byref(v)), "moe_get_device_status")
     return int(v.value)
 
 
 def moe_set_option(option: int, value: int):
+    """moe_set_option: a process-wide switch (OPT_*; the header documents values and defaults)."""
     _check(lib().moe_set_option(int(option), int(value)), "moe_set_option")
 
 
@@ -469,4 +485,5 @@ def moe_stage_mask() -> int:
 
 
 def moe_kernel_launch_count() -> int:
+    """Kernels this process has launched through the library so far."""
     return int(lib().moe_kernel_launch_count())
